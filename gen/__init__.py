@@ -1,0 +1,270 @@
+"""Seeded synthetic inputs for the routed-MoE block: shapes, layouts and generators.
+
+Both the CPU oracle (through the host library) and the GPU path (through the
+device library) consume the bytes drawn here; this module holds none of the
+block's own arithmetic.  Workload shapes follow the Flash-MoE pages' model
+description (Qwen3.5-397B-A17B: hidden 4096, 512 routed experts, top-4 plus
+one shared expert, 4-bit or 2-bit group-64 affine experts).
+
+Input recipe (all synthetic, no dataset and no trained weights):
+  * expert weights N(0, 0.02), quantised per group of 64 along the input dim
+    (min/max affine, bf16 scale and bias, codes packed LSB-first);
+  * router N(0, 0.02) bf16 (tiny layer: N(0, 1/H) so that logits are ~N(0,1));
+  * shared-expert gate vector N(0, 0.02) bf16;
+  * RMSNorm weight gamma = 1 (tests also draw gamma = 1 + 0.1 N(0,1));
+  * token hidden states N(0, 1) fp32, a fresh seeded draw per token;
+  * Zipf-routed variant: per-expert logit bias ln p_pi(e), p_r ~ r^-1.1.
+"""
+import ctypes
+import dataclasses
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+GROUP = 64
+KIND_GATE, KIND_UP, KIND_DOWN, KIND_ROUTER, KIND_SHARED_GATE, KIND_GAMMA, KIND_PERM = range(7)
+EXPERT_SHARED = 0xFFFFFFF
+EXPERT_LAYER = 0xFFFFFFE
+WEIGHT_SEED = 0
+TOKEN_SEED = 1
+
+_host = None
+_cuda = None
+
+
+def host_lib():
+    global _host
+    if _host is None:
+        _build.build()
+        lib = ctypes.CDLL(_build.HOST_SO)
+        u64, i64, f32 = ctypes.c_uint64, ctypes.c_int64, ctypes.c_float
+        vp = ctypes.c_void_p
+        lib.fg_host_key.restype = u64
+        lib.fg_host_key.argtypes = [u64, u64]
+        lib.fg_host_stream_id.restype = u64
+        lib.fg_host_stream_id.argtypes = [u64, u64, u64]
+        lib.fg_host_normal_f32.argtypes = [u64, f32, i64, vp]
+        lib.fg_host_normal_bf16.argtypes = [u64, f32, i64, vp]
+        lib.fg_host_uniform_u32.argtypes = [u64, ctypes.c_uint32, i64, vp]
+        lib.fg_host_packed.argtypes = [u64, f32, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+        _host = lib
+    return _host
+
+
+def cuda_lib():
+    global _cuda
+    if _cuda is None:
+        _build.build()
+        lib = ctypes.CDLL(_build.CUDA_SO)
+        u64, i64, f32, i32, vp = ctypes.c_uint64, ctypes.c_longlong, ctypes.c_float, ctypes.c_int, ctypes.c_void_p
+        lib.fg_cuda_packed_bank.restype = i32
+        lib.fg_cuda_packed_bank.argtypes = [u64, u64, u64, i32, i32, f32, i32, i32, i32, i32, vp, i64, i64, i64, i64,
+                                            vp]
+        lib.fg_cuda_normal_f32.restype = i32
+        lib.fg_cuda_normal_f32.argtypes = [u64, f32, i64, vp, vp]
+        lib.fg_cuda_normal_bf16.restype = i32
+        lib.fg_cuda_normal_bf16.argtypes = [u64, f32, i64, vp, vp]
+        _cuda = lib
+    return _cuda
+
+
+def key(seed, layer, expert, kind):
+    lib = host_lib()
+    return int(lib.fg_host_key(seed, lib.fg_host_stream_id(layer, expert, kind)))
+
+
+def token_key(t):
+    """Key of token t's hidden state (seed 1, stream t)."""
+    return int(host_lib().fg_host_key(TOKEN_SEED, t))
+
+
+# ----------------------------------------------------------------------------------------------- shapes
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerSpec:
+    """One routed-MoE layer: hidden H, E routed experts of intermediate I, top-K, code width."""
+    hidden: int
+    experts: int
+    inter: int
+    top_k: int
+    bits: int
+    group: int = GROUP
+    eps: float = 1e-6
+    weight_std: float = 0.02
+    router_std: float = 0.02
+    shared_gate_std: float = 0.02
+    zipf: float = 0.0          # > 0: per-expert logit bias ln p_pi(e), p_r ~ r^-zipf
+    random_gamma: bool = False  # False: gamma = 1
+
+
+def tiny_layer(bits=4):
+    """Tiny layer: hidden 256, 8 experts of intermediate 128, top-2; router N(0, 1/H)."""
+    return LayerSpec(hidden=256, experts=8, inter=128, top_k=2, bits=bits, router_std=1.0 / math.sqrt(256))
+
+
+def qwen397_layer(bits=4, zipf=0.0):
+    """Qwen3.5-397B-A17B-shaped MoE layer: hidden 4096, 512 experts of intermediate 1024, top-4 + shared."""
+    return LayerSpec(hidden=4096, experts=512, inter=1024, top_k=4, bits=bits, zipf=zipf)
+
+
+def _align16(n):
+    return (n + 15) // 16 * 16
+
+
+def record_layout(bits, hidden, inter, group=GROUP):
+    """Byte layout of one expert record: gate{qw,scale,bias} | up{...} | down{...}.
+
+    A packed [out][in] matrix is qw uint32[out][in*bits/32] (code j of a word at
+    bits [bits*j, bits*j+bits)) followed by scale and bias bf16[out][in/group];
+    every sub-array starts on a 16-byte boundary.  Returns (record_bytes, off[9]).
+    """
+    off = []
+    pos = 0
+    for out_dim, in_dim in ((inter, hidden), (inter, hidden), (hidden, inter)):
+        for nbytes in (out_dim * in_dim * bits // 8, out_dim * (in_dim // group) * 2, out_dim * (in_dim // group) * 2):
+            off.append(pos)
+            pos = _align16(pos + nbytes)
+    return pos, off
+
+
+def record_bytes(spec):
+    return record_layout(spec.bits, spec.hidden, spec.inter, spec.group)[0]
+
+
+def matrix_shapes(spec):
+    """(rows, cols) of gate, up, down."""
+    return ((spec.inter, spec.hidden), (spec.inter, spec.hidden), (spec.hidden, spec.inter))
+
+
+def algorithmic_bytes_per_token(spec):
+    """Bytes one token must read: K routed + 1 shared expert records (packed codes + scales + biases) + router."""
+    return (spec.top_k + 1) * _payload_bytes(spec) + spec.experts * spec.hidden * 2
+
+
+def _payload_bytes(spec):
+    total = 0
+    for rows, cols in matrix_shapes(spec):
+        total += rows * cols * spec.bits // 8 + 2 * rows * (cols // spec.group) * 2
+    return total
+
+
+# ----------------------------------------------------------------------------------------------- host generation
+
+
+def host_record(spec, seed, layer, expert_id):
+    """One expert record (numpy uint8) drawn on the host."""
+    lib = host_lib()
+    nbytes, off = record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    rec = np.zeros(nbytes, dtype=np.uint8)
+    base = rec.ctypes.data
+    for m, (rows, cols) in enumerate(matrix_shapes(spec)):
+        k = key(seed, layer, expert_id, m)
+        lib.fg_host_packed(k, spec.weight_std, spec.bits, spec.group, rows, cols, base + off[3 * m],
+                           base + off[3 * m + 1], base + off[3 * m + 2])
+    return rec
+
+
+def host_normal_f32(k, std, n):
+    out = np.empty(n, dtype=np.float32)
+    host_lib().fg_host_normal_f32(k, std, n, out.ctypes.data)
+    return out
+
+
+def host_normal_bf16(k, std, n):
+    out = np.empty(n, dtype=np.uint16)
+    host_lib().fg_host_normal_bf16(k, std, n, out.ctypes.data)
+    return out
+
+
+def zipf_logit_bias(spec, seed, layer):
+    """Per-expert logit bias ln p_pi(e) with p_r ~ r^-zipf over ranks 1..E and pi a seeded permutation."""
+    E = spec.experts
+    draws = np.empty(E, dtype=np.uint32)
+    lib = host_lib()
+    k = key(seed, layer, EXPERT_LAYER, KIND_PERM)
+    # Fisher-Yates with draw i choosing among E - i remaining positions.
+    perm = np.arange(E)
+    for i in range(E - 1, 0, -1):
+        lib.fg_host_uniform_u32(lib.fg_host_key(k, i), i + 1, 1, draws.ctypes.data)
+        j = int(draws[0])
+        perm[i], perm[j] = perm[j], perm[i]
+    ranks = np.arange(1, E + 1, dtype=np.float64)
+    p = ranks ** (-spec.zipf)
+    p /= p.sum()
+    return np.log(p[perm]).astype(np.float32)
+
+
+@dataclasses.dataclass
+class HostLayer:
+    spec: LayerSpec
+    routed: dict            # expert id -> uint8 record
+    shared: np.ndarray      # uint8 record
+    w_router: np.ndarray    # uint16 (bf16 bits) [E][H]
+    w_shared_gate: np.ndarray  # uint16 [H]
+    gamma: np.ndarray       # float32 [H]
+    logit_bias: object      # float32 [E] or None
+
+
+def host_gamma(spec, seed, layer):
+    if spec.random_gamma:
+        return (1.0 + host_normal_f32(key(seed, layer, EXPERT_LAYER, KIND_GAMMA), 0.1, spec.hidden)).astype(np.float32)
+    return np.ones(spec.hidden, dtype=np.float32)
+
+
+def host_layer(spec, seed=WEIGHT_SEED, layer=0, experts=None):
+    """Draws a layer on the host; `experts` limits which routed records are drawn (default: all)."""
+    ids = range(spec.experts) if experts is None else sorted(set(int(e) for e in experts))
+    routed = {e: host_record(spec, seed, layer, e) for e in ids}
+    shared = host_record(spec, seed, layer, EXPERT_SHARED)
+    wr = host_normal_bf16(key(seed, layer, EXPERT_LAYER, KIND_ROUTER), spec.router_std,
+                          spec.experts * spec.hidden).reshape(spec.experts, spec.hidden)
+    wsg = host_normal_bf16(key(seed, layer, EXPERT_LAYER, KIND_SHARED_GATE), spec.shared_gate_std, spec.hidden)
+    bias = zipf_logit_bias(spec, seed, layer) if spec.zipf > 0 else None
+    return HostLayer(spec, routed, shared, wr, wsg, host_gamma(spec, seed, layer), bias)
+
+
+def host_tokens(t0, T, hidden):
+    """Hidden states of tokens t0..t0+T-1: fresh N(0,1) fp32 draws, shape [T][H]."""
+    out = np.empty((T, hidden), dtype=np.float32)
+    for i in range(T):
+        out[i] = host_normal_f32(token_key(t0 + i), 1.0, hidden)
+    return out
+
+
+def bank_array(hl):
+    """All routed records of a fully drawn host layer as one [E][record] uint8 array."""
+    E = hl.spec.experts
+    if len(hl.routed) != E:
+        raise ValueError("layer was drawn with a subset of experts")
+    return np.stack([hl.routed[e] for e in range(E)])
+
+
+# ----------------------------------------------------------------------------------------------- device generation
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RuntimeError(f"{what}: CUDA error {rc}")
+
+
+def device_fill_bank(spec, seed, layer, expert_id0, n, dst, stream_ptr):
+    """Draws records expert_id0 .. expert_id0+n-1 into device buffer `dst` (torch uint8 [n*record])."""
+    lib = cuda_lib()
+    nbytes, off = record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    assert dst.numel() >= n * nbytes
+    for m, (rows, cols) in enumerate(matrix_shapes(spec)):
+        _check(lib.fg_cuda_packed_bank(seed, layer, expert_id0, n, m, spec.weight_std, spec.bits, spec.group, rows,
+                                       cols, dst.data_ptr(), nbytes, off[3 * m], off[3 * m + 1], off[3 * m + 2],
+                                       stream_ptr), "fg_cuda_packed_bank")
+
+
+def device_normal_f32(k, std, dst, stream_ptr):
+    _check(cuda_lib().fg_cuda_normal_f32(k, std, dst.numel(), dst.data_ptr(), stream_ptr), "fg_cuda_normal_f32")
+
+
+def device_normal_bf16(k, std, dst, stream_ptr):
+    _check(cuda_lib().fg_cuda_normal_bf16(k, std, dst.numel(), dst.data_ptr(), stream_ptr), "fg_cuda_normal_bf16")

@@ -1,0 +1,85 @@
+"""Test-side helpers: an independent numpy packer/dequantiser, the error metric and layer marshalling."""
+import numpy as np
+
+import gen
+
+
+def f32_to_bf16_exact(v):
+    """bf16 bit pattern of values that are exactly representable in bf16 (asserts it)."""
+    a = np.asarray(v, dtype=np.float32)
+    u = a.view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0), "value not exactly representable in bf16"
+    return (u >> 16).astype(np.uint16)
+
+
+def bf16_to_f64(b):
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def np_pack(codes, bits):
+    """Packs unsigned codes [rows][cols] into uint32 words, field j of a word at bits [bits*j, bits*j+bits)."""
+    per = 32 // bits
+    rows, cols = codes.shape
+    w = codes.astype(np.uint64).reshape(rows, cols // per, per)
+    shifts = (np.arange(per, dtype=np.uint64) * np.uint64(bits))
+    return np.bitwise_or.reduce(w << shifts, axis=-1).astype(np.uint32)
+
+
+def np_unpack(words, bits, cols):
+    """Inverse of np_pack, vectorised over whole words."""
+    per = 32 // bits
+    w = np.asarray(words, dtype=np.uint32).astype(np.uint64)
+    rows = w.shape[0]
+    shifts = (np.arange(per, dtype=np.uint64) * np.uint64(bits))
+    c = (w[..., None] >> shifts) & np.uint64((1 << bits) - 1)
+    return c.reshape(rows, -1)[:, :cols].astype(np.int64)
+
+
+def dense_from_record(rec, spec_bits, hidden, inter, group=64):
+    """Dense fp64 gate, up, down of one record, via whole-array unpacking (independent of the oracle's decoder)."""
+    nbytes, off = gen.record_layout(spec_bits, hidden, inter, group)
+    rec = np.asarray(rec, dtype=np.uint8)
+    out = []
+    for m, (rows, cols) in enumerate(((inter, hidden), (inter, hidden), (hidden, inter))):
+        nw = rows * cols * spec_bits // 32
+        ng = rows * cols // group
+        qw = rec[off[3 * m]:off[3 * m] + 4 * nw].view(np.uint32).reshape(rows, -1)
+        s = bf16_to_f64(rec[off[3 * m + 1]:off[3 * m + 1] + 2 * ng].view(np.uint16)).reshape(rows, -1)
+        b = bf16_to_f64(rec[off[3 * m + 2]:off[3 * m + 2] + 2 * ng].view(np.uint16)).reshape(rows, -1)
+        codes = np_unpack(qw, spec_bits, cols).astype(np.float64)
+        out.append(codes * np.repeat(s, group, axis=1) + np.repeat(b, group, axis=1))
+    return out
+
+
+def max_rel_err(got, ref, floor=1e-2):
+    """max_i |g_i - r_i| / max(|r_i|, floor * rms(r)) over the last axis, maximised over rows."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+    den = np.maximum(np.abs(ref), floor * rms)
+    den = np.where(den > 0, den, 1.0)
+    return float(np.max(np.abs(got - ref) / den)) if got.size else 0.0
+
+
+def oracle_layer(hl, top_k=None, gamma=True):
+    """Marshals a gen.HostLayer (all routed experts drawn) into an oracle.Layer."""
+    import oracle
+    spec = hl.spec
+    nbytes, off = gen.record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    return oracle.Layer(gen.bank_array(hl), hl.shared, hl.w_router, hl.w_shared_gate,
+                        hl.gamma if gamma else None, hl.logit_bias, spec.bits, spec.hidden, spec.inter,
+                        top_k if top_k is not None else spec.top_k, nbytes, off, eps=spec.eps, group=spec.group)
+
+
+def oracle_layer_sparse(hl, top_k=None):
+    """Oracle layer over a host layer drawn with a subset of experts (only those may be selected)."""
+    import oracle
+    spec = hl.spec
+    nbytes, off = gen.record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    return oracle.Layer(dict(hl.routed), hl.shared, hl.w_router, hl.w_shared_gate, hl.gamma, hl.logit_bias,
+                        spec.bits, spec.hidden, spec.inter, top_k if top_k is not None else spec.top_k, nbytes, off,
+                        eps=spec.eps, group=spec.group)
+
+
+def silu(z):
+    return z / (1.0 + np.exp(-z))
