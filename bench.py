@@ -1,0 +1,328 @@
+"""Benchmark of the routed-MoE decode block on B200: MoE-layer decode tokens/s and effective weight GB/s.
+
+One step = one decode token through one MoE layer (RMSNorm -> router GEMV ->
+softmax/top-K -> gate/up dequant GEMV + SwiGLU for K routed + 1 shared expert ->
+down dequant GEMV + weighted combine + sigmoid-gated shared expert + residual).
+Tokens run strictly one after another, each with a fresh seeded input.  Layer
+copies are rotated per token so that the router and shared expert do not stay
+resident in L2 (the working set exceeds the 126 MB L2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl fmoe|reference]
+
+Under torchrun each rank runs its own replica on its own tokens (weak scaling,
+no collective on the data path); the reported time is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "MoE-layer decode tokens/s and effective weight GB/s (fraction of HBM peak), 1×B200"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {
+    # name: (spec factory, description)
+    "qwen397-4bit": (lambda: __import__("gen").qwen397_layer(4),
+                     "Qwen3.5-397B-A17B-shaped MoE layer, 4-bit group-64 experts, batch-1 decode"),
+    "qwen397-2bit-zipf": (lambda: __import__("gen").qwen397_layer(2, zipf=1.1),
+                          "Qwen3.5-397B-A17B-shaped MoE layer, 2-bit group-64 experts, Zipf(1.1) routing, batch-1 decode"),
+    "tiny-4bit": (lambda: __import__("gen").tiny_layer(4), "tiny MoE layer (H256, E8, I128, top-2), 4-bit"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="fmoe", choices=["fmoe", "reference"])
+    ap.add_argument("--workload", default="qwen397-4bit", choices=sorted(WORKLOADS))
+    ap.add_argument("--copies", type=int, default=16, help="resident layer copies rotated per token")
+    ap.add_argument("--graph-tokens", type=int, default=1000, help="tokens per captured CUDA graph")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, index, period=0.01):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: no clock record
+            self.nv = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self.nv
+        names = {getattr(nv, k): k for k in dir(nv) if k.startswith("nvmlClocksEventReason") or
+                 k.startswith("nvmlClocksThrottleReason")}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in names.items():
+                    if isinstance(bit, int) and bit and (mask & bit) == bit and bit != 0xFFFFFFFFFFFFFFFF:
+                        self.reasons.add(name.replace("nvmlClocksEventReason", "").replace(
+                            "nvmlClocksThrottleReason", ""))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def record(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = sorted(r for r in self.reasons if r not in ("GpuIdle", "None", "All", "Unknown"))
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_oracle_rate(spec, budget_s, t0=1_000_000):
+    """Times the CPU oracle (all host cores) on a bounded sample of the workload: tokens/s.
+
+    Drawing the inputs (router, shared expert, the experts a token selects) is
+    not timed; the oracle's whole forward pass (norm, router, softmax, top-K,
+    K+1 expert FFNs, combine) is."""
+    import gen
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    base = gen.host_layer(spec, 0, 0, experts=[])
+    nbytes, off = gen.record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    records = {}
+    n, spent, t = 0, 0.0, t0
+    while spent < budget_s and n < 256:
+        h = gen.host_tokens(t, 1, spec.hidden)
+        x = oracle.rmsnorm(h[0], base.gamma, spec.eps)
+        sel = oracle.topk(oracle.softmax(oracle.router_logits(base.w_router, base.logit_bias, x)), spec.top_k)
+        for e in sel.tolist():
+            if e not in records:
+                records[e] = gen.host_record(spec, 0, 0, e)
+        L = oracle.Layer(dict(records), base.shared, base.w_router, base.w_shared_gate, base.gamma, base.logit_bias,
+                         spec.bits, spec.hidden, spec.inter, spec.top_k, nbytes, off, eps=spec.eps, group=spec.group)
+        s = time.perf_counter()
+        L.forward(h)
+        spent += time.perf_counter() - s
+        n += 1
+        t += 1
+    return n / spent, cores, n, spent
+
+
+def run_reference(args, spec, desc, world, rank):
+    if rank != 0:
+        return
+    rate, cores, n, spent = cpu_oracle_rate(spec, max(args.cpu_seconds, 5.0))
+    line = {"metric": METRIC, "impl": "reference", "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": n, "warmup": 0, "ms_per_step": 1e3 / rate, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": desc},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n} tokens of the workload ({spent:.1f} s of oracle time; the requested "
+                                       f"{args.steps} steps would not fit a few minutes)"},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    import gen
+    spec = WORKLOADS[args.workload][0]()
+    desc = WORKLOADS[args.workload][1]
+    if args.impl == "reference":
+        return run_reference(args, spec, desc, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    import bit_dequant_expert_router_b200 as fmoe
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    fmoe.lib()
+
+    # ---- resident inputs: layer copies and token states
+    ncopy = max(1, args.copies)
+    layers = [gen.binding_layer(gen.device_layer(spec, seed=0, layer=c, device=dev)) for c in range(ncopy)]
+    G = min(args.graph_tokens, args.steps)
+    steps = (args.steps + G - 1) // G * G
+    h = gen.device_tokens(rank * 10_000_000, G, spec.hidden, device=dev)
+    out = torch.empty_like(h)
+    ws = fmoe.workspace(max(fmoe.moe_layer_workspace_size(l, 1) for l in layers), dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step(i, s):
+        fmoe.moe_layer(layers[i % ncopy], h[i % G], out=out[i % G], ws=ws, stream=s)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i, stream)
+    stream.synchronize()
+    fmoe.workspace_check(ws, stream)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            step(i, stream)
+    graph.replay()
+    stream.synchronize()
+
+    # ---- timed region: `steps` tokens, as steps / G graph replays
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(steps // G):
+            graph.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    fmoe.workspace_check(ws, stream)
+    tokens = steps * world
+    value = tokens / (ms / 1e3)
+    ms_per_step = ms / steps
+
+    # ---- per-kernel durations: a separate replay with trace events around each kernel
+    tr = min(G, 500)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(tr)]
+    tgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(tgraph, stream=stream):
+        for i in range(tr):
+            fmoe.trace_next_layer(evs[i])
+            step(i, stream)
+    tgraph.replay()
+    stream.synchronize()
+    dur = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs]) * 1e3
+    router_us, gateup_us, down_us = (float(np.mean(dur[:, k])) for k in range(3))
+    del tgraph
+
+    # ---- end to end through the C ABI with host buffers: H2D of h, the layer, D2H of out, every step
+    e2e = None
+    if not args.no_e2e:
+        hh = torch.empty((G, spec.hidden), dtype=torch.float32, pin_memory=True)
+        hh.copy_(h.cpu())
+        oh = torch.empty_like(hh, pin_memory=True)
+        hd = torch.empty((spec.hidden,), dtype=torch.float32, device=dev)
+        od = torch.empty_like(hd)
+        egraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(egraph, stream=stream):
+            for i in range(G):
+                hd.copy_(hh[i], non_blocking=True)
+                fmoe.moe_layer(layers[i % ncopy], hd, out=od, ws=ws, stream=stream)
+                oh[i].copy_(od, non_blocking=True)
+        egraph.replay()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps // G):
+            egraph.replay()
+        e1.record(stream)
+        e1.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        bpt = spec.hidden * 4
+        e2e = {"value": steps * world / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bpt,
+               "d2h_bytes_per_step": bpt}
+        del egraph
+
+    # ---- roofline of the dominant kernel (gate/up + SwiGLU over K routed + 1 shared expert)
+    peak, peak_kind = peak_hbm()
+    rec_mat = spec.inter * spec.hidden * spec.bits // 8 + 2 * spec.inter * (spec.hidden // spec.group) * 2
+    gateup_bytes = (spec.top_k + 1) * 2 * rec_mat
+    achieved = gateup_bytes / (gateup_us * 1e-6) / 1e9
+    bytes_tok = gen.algorithmic_bytes_per_token(spec)
+    eff = bytes_tok * (value / world) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, n, spent = cpu_oracle_rate(spec, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} tokens of this workload, layer copy 0 ({spent:.1f} s of oracle time)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32", "data": "synthetic",
+            "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
+                       "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": 1,
+                       "layer_copies": ncopy, "graph_tokens": G,
+                       "l2": f"inputs larger than L2: {ncopy} resident layer copies "
+                             f"({ncopy * gen.record_bytes(spec) * (spec.experts + 1) / 1e9:.1f} GB) rotated per token",
+                       "parallelism": f"replicas x{world}"},
+            "effective_gbs": eff, "frac_of_peak": eff / peak, "bytes_per_token": bytes_tok,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "kernel": "gateup_kernel", "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": gateup_bytes},
+            "kernels_us": {"router": router_us, "gateup": gateup_us, "down": down_us},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * steps,
+            "clocks": clk.record(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

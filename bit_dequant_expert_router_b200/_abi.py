@@ -1,0 +1,226 @@
+"""ctypes binding of libfmoe.so (include/fmoe.h): argument marshalling only.
+
+Every function takes torch tensors that already live on the GPU, passes their
+device pointers and the current torch stream to the C ABI, and raises
+FmoeError on a non-OK status.  No step of the block runs in Python; if the
+shared library is missing the import of a function fails loudly.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(_HERE, "libfmoe.so")
+
+FMOE_OK = 0
+STATUS_NAMES = {0: "FMOE_OK", 1: "FMOE_ERR_INVALID_ARG", 2: "FMOE_ERR_ALIGNMENT", 3: "FMOE_ERR_UNSUPPORTED",
+                4: "FMOE_ERR_WORKSPACE", 5: "FMOE_ERR_CUDA", 6: "FMOE_ERR_DEVICE_TIMEOUT"}
+
+
+class FmoeError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class FmoeBank(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("num_experts", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("base", ctypes.c_void_p), ("stride", ctypes.c_int64), ("off", ctypes.c_int64 * 9)]
+
+
+class FmoeLayer(ctypes.Structure):
+    _fields_ = [("routed", FmoeBank), ("shared", FmoeBank), ("w_router", ctypes.c_void_p),
+                ("router_bias", ctypes.c_void_p), ("w_shared_gate", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("eps", ctypes.c_float), ("top_k", ctypes.c_int32)]
+
+
+_lib = None
+
+# (name, restype, argtypes) of every entry point declared in include/fmoe.h
+_vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+SIGNATURES = [
+    ("fmoe_bank_layout", _i, [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
+    ("fmoe_rmsnorm", _i, [_vp, _vp, _f, _i, _i, _vp, _vp]),
+    ("fmoe_router_topk", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    ("fmoe_router_topk_workspace_size", _sz, [_i, _i]),
+    ("fmoe_expert_ffn", _i, [ctypes.POINTER(FmoeBank), _i, _vp, _vp, _vp, _sz, _vp]),
+    ("fmoe_expert_ffn_workspace_size", _sz, [ctypes.POINTER(FmoeBank)]),
+    ("fmoe_moe_layer", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    ("fmoe_moe_layer_workspace_size", _sz, [ctypes.POINTER(FmoeLayer), _i]),
+    ("fmoe_moe_stack", _i, [ctypes.POINTER(FmoeLayer), _i, _vp, _i, _vp, _vp, _sz, _vp]),
+    ("fmoe_trace_next_layer", _i, [ctypes.POINTER(ctypes.c_void_p), _i]),
+    ("fmoe_workspace_init", _i, [_vp, _sz, _vp]),
+    ("fmoe_workspace_check", _i, [_vp, _vp]),
+    ("fmoe_last_error", ctypes.c_char_p, []),
+    ("fmoe_status_string", ctypes.c_char_p, [_i]),
+    ("fmoe_version", _i, []),
+]
+
+
+def lib():
+    """Loads libfmoe.so (built in-tree by build.py); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(SO_PATH):
+            raise RuntimeError(f"{SO_PATH} is missing: build it with `python -m bit_dequant_expert_router_b200.build` "
+                               "(there is no fallback implementation)")
+        L = ctypes.CDLL(SO_PATH)
+        for name, res, args in SIGNATURES:
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != FMOE_OK:
+        raise FmoeError(status, lib().fmoe_last_error().decode())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t, dtype=None, what="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def bank_layout(bits, hidden, inter, group_size=64):
+    """Canonical record layout: (record_bytes, [9 offsets])."""
+    nb = ctypes.c_int64()
+    off = (ctypes.c_int64 * 9)()
+    _check(lib().fmoe_bank_layout(bits, group_size, hidden, inter, ctypes.byref(nb), off))
+    return nb.value, list(off)
+
+
+class Bank:
+    """A bank of expert records held in one device tensor (uint8)."""
+
+    def __init__(self, storage, bits, hidden, inter, num_experts, stride, off, group_size=64):
+        self.storage = storage
+        self.s = FmoeBank(bits, group_size, hidden, inter, num_experts, 0,
+                          _ptr(storage, torch.uint8, "bank storage").value, stride, (ctypes.c_int64 * 9)(*off))
+
+
+class Layer:
+    """One MoE layer: routed and shared banks, router (bf16 bits as int16/uint16), shared gate, gamma, bias."""
+
+    def __init__(self, routed, shared, w_router, w_shared_gate, gamma=None, router_bias=None, eps=1e-6, top_k=4):
+        self.routed, self.shared = routed, shared
+        self.tensors = (w_router, w_shared_gate, gamma, router_bias)
+        self.s = FmoeLayer(routed.s, shared.s, _ptr(w_router, None, "w_router"), _ptr(router_bias, torch.float32,
+                           "router_bias"), _ptr(w_shared_gate, None, "w_shared_gate"), _ptr(gamma, torch.float32, "gamma"),
+                           eps, top_k)
+
+    @property
+    def hidden(self):
+        return self.s.routed.hidden
+
+    @property
+    def top_k(self):
+        return self.s.top_k
+
+
+def trace_next_layer(events):
+    """Makes the next moe_layer call record 4 torch.cuda.Events around its kernels (None cancels)."""
+    if events is None:
+        _check(lib().fmoe_trace_next_layer(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().fmoe_trace_next_layer(arr, len(events)))
+
+
+def workspace(nbytes, device=None, stream=None):
+    """Allocates a zero-initialised workspace tensor of `nbytes` (torch allocations are 512-byte aligned)."""
+    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
+    workspace_init(ws, stream)
+    return ws
+
+
+def workspace_init(ws, stream=None):
+    _check(lib().fmoe_workspace_init(_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def workspace_check(ws, stream=None):
+    _check(lib().fmoe_workspace_check(_ptr(ws, torch.uint8, "ws"), _stream(stream)))
+
+
+def rmsnorm(h, gamma, eps, out=None, stream=None):
+    T, H = h.shape
+    out = torch.empty_like(h) if out is None else out
+    _check(lib().fmoe_rmsnorm(_ptr(h, torch.float32, "h"), _ptr(gamma, torch.float32, "gamma"), eps, T, H,
+                              _ptr(out, torch.float32, "out"), _stream(stream)))
+    return out
+
+
+def router_topk_workspace_size(T, E):
+    return lib().fmoe_router_topk_workspace_size(T, E)
+
+
+def router_topk(x, w_router, top_k, logit_bias=None, idx=None, w=None, probs=None, ws=None, stream=None):
+    T, H = x.shape
+    E = w_router.shape[0]
+    idx = torch.empty((T, top_k), dtype=torch.int32, device=x.device) if idx is None else idx
+    w = torch.empty((T, top_k), dtype=torch.float32, device=x.device) if w is None else w
+    if ws is None:
+        ws = workspace(router_topk_workspace_size(T, E), x.device, stream)
+    _check(lib().fmoe_router_topk(_ptr(x, torch.float32, "x"), _ptr(w_router, None, "w_router"),
+                                  _ptr(logit_bias, torch.float32, "logit_bias"), T, H, E, top_k,
+                                  _ptr(idx, torch.int32, "idx"), _ptr(w, torch.float32, "w"),
+                                  _ptr(probs, torch.float32, "probs"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                  _stream(stream)))
+    return idx, w
+
+
+def expert_ffn_workspace_size(bank):
+    return lib().fmoe_expert_ffn_workspace_size(ctypes.byref(bank.s))
+
+
+def expert_ffn(bank, expert, x, y=None, ws=None, stream=None):
+    y = torch.empty_like(x) if y is None else y
+    if ws is None:
+        ws = workspace(expert_ffn_workspace_size(bank), x.device, stream)
+    _check(lib().fmoe_expert_ffn(ctypes.byref(bank.s), expert, _ptr(x, torch.float32, "x"),
+                                 _ptr(y, torch.float32, "y"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                 _stream(stream)))
+    return y
+
+
+def moe_layer_workspace_size(layer, T=1):
+    return lib().fmoe_moe_layer_workspace_size(ctypes.byref(layer.s), T)
+
+
+def moe_layer(layer, h, out=None, topk_idx=None, topk_w=None, ws=None, stream=None):
+    T = h.shape[0] if h.dim() == 2 else 1
+    out = torch.empty_like(h) if out is None else out
+    if ws is None:
+        ws = workspace(moe_layer_workspace_size(layer, T), h.device, stream)
+    _check(lib().fmoe_moe_layer(ctypes.byref(layer.s), _ptr(h, torch.float32, "h"), T,
+                                _ptr(out, torch.float32, "out"), _ptr(topk_idx, torch.int32, "topk_idx"),
+                                _ptr(topk_w, torch.float32, "topk_w"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                _stream(stream)))
+    return out
+
+
+def moe_stack(layers, h, out=None, ws=None, stream=None):
+    T = h.shape[0] if h.dim() == 2 else 1
+    out = torch.empty_like(h) if out is None else out
+    arr = (FmoeLayer * len(layers))(*[l.s for l in layers])
+    if ws is None:
+        ws = workspace(max(moe_layer_workspace_size(l, T) for l in layers), h.device, stream)
+    _check(lib().fmoe_moe_stack(arr, len(layers), _ptr(h, torch.float32, "h"), T, _ptr(out, torch.float32, "out"),
+                                _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+    return out

@@ -1,0 +1,412 @@
+// fmoe_api.cu -- the C ABI of libfmoe.so: argument validation, workspace
+// layout and kernel dispatch.  Every entry point validates on the host before
+// enqueuing anything and reports through fmoe_status (never aborts).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fmoe.h"
+#include "fmoe_internal.h"
+
+namespace fmoe {
+
+cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, cudaStream_t s);
+
+namespace {
+
+thread_local char g_msg[512] = "";
+thread_local cudaEvent_t g_trace[4] = {nullptr, nullptr, nullptr, nullptr};
+thread_local bool g_trace_on = false;
+
+fmoe_status fail(fmoe_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+fmoe_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// Workspace regions (byte offsets), in this order.
+struct WsLayout {
+  size_t ctrl, xq_limbs, xq_cs, logits, idx, wts, act, total;
+};
+
+WsLayout layout(int H, int E, int K, int I, int T) {
+  WsLayout L;
+  L.ctrl = 0;
+  L.xq_limbs = up(sizeof(WsControl));
+  L.xq_cs = L.xq_limbs + up((size_t)T * 3 * H);       // 3 bytes of digits per element
+  L.logits = L.xq_cs + up((size_t)T * (H / 32) * 8);  // one float2 per chunk (at most H/32 chunks)
+  L.idx = L.logits + up((size_t)T * (E + 1) * 4);
+  L.wts = L.idx + up((size_t)T * (K > 0 ? K : 1) * 4);
+  L.act = L.wts + up((size_t)T * (K + 1) * 4);
+  L.total = L.act + up((size_t)(K + 1) * (I > 0 ? I : 1) * 4);
+  return L;
+}
+
+fmoe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(FMOE_ERR_WORKSPACE, "workspace is NULL");
+  if (((uintptr_t)ws & (kAlign - 1)) != 0) return fail(FMOE_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(FMOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return FMOE_OK;
+}
+
+fmoe_status check_bank(const fmoe_bank* b, const char* name) {
+  if (!b) return fail(FMOE_ERR_INVALID_ARG, "%s bank is NULL", name);
+  if (!b->base) return fail(FMOE_ERR_INVALID_ARG, "%s bank base is NULL", name);
+  if (b->bits != 2 && b->bits != 4) return fail(FMOE_ERR_UNSUPPORTED, "%s bank: bits %d (2 or 4)", name, b->bits);
+  if (b->group_size != kGroup) return fail(FMOE_ERR_UNSUPPORTED, "%s bank: group_size %d (64)", name, b->group_size);
+  if (b->num_experts < 1) return fail(FMOE_ERR_INVALID_ARG, "%s bank: num_experts %d", name, b->num_experts);
+  const int H = b->hidden, I = b->inter;
+  if (H < 128 || I < 128 || H % 128 || I % 128)
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden %d and inter %d must be positive multiples of 128", name, H, I);
+  const int nch = H * b->bits / 128, ncd = I * b->bits / 128;
+  if (!pow2(nch) || nch > 512 || !pow2(ncd) || ncd > 512)
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden*bits/128 (%d) and inter*bits/128 (%d) must be powers of two <= 512",
+                name, nch, ncd);
+  if (!aligned16(b->base) || (b->stride & 15)) return fail(FMOE_ERR_ALIGNMENT, "%s bank: base/stride not 16-byte aligned", name);
+  if (b->num_experts > 1 && b->stride <= 0) return fail(FMOE_ERR_INVALID_ARG, "%s bank: stride %lld", name, (long long)b->stride);
+  for (int i = 0; i < 9; ++i)
+    if (b->off[i] < 0 || (b->off[i] & 15)) return fail(FMOE_ERR_ALIGNMENT, "%s bank: off[%d] not 16-byte aligned", name, i);
+  return FMOE_OK;
+}
+
+BankRef ref(const fmoe_bank& b) {
+  BankRef r;
+  r.base = static_cast<const uint8_t*>(b.base);
+  r.stride = b.stride;
+  for (int i = 0; i < 9; ++i) r.off[i] = b.off[i];
+  r.num_experts = b.num_experts;
+  return r;
+}
+
+cudaStream_t cs(fmoe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace fmoe
+
+using namespace fmoe;
+
+extern "C" {
+
+int fmoe_version(void) { return 100; }
+
+const char* fmoe_last_error(void) { return g_msg; }
+
+const char* fmoe_status_string(fmoe_status s) {
+  switch (s) {
+    case FMOE_OK: return "FMOE_OK";
+    case FMOE_ERR_INVALID_ARG: return "FMOE_ERR_INVALID_ARG";
+    case FMOE_ERR_ALIGNMENT: return "FMOE_ERR_ALIGNMENT";
+    case FMOE_ERR_UNSUPPORTED: return "FMOE_ERR_UNSUPPORTED";
+    case FMOE_ERR_WORKSPACE: return "FMOE_ERR_WORKSPACE";
+    case FMOE_ERR_CUDA: return "FMOE_ERR_CUDA";
+    case FMOE_ERR_DEVICE_TIMEOUT: return "FMOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "unknown fmoe_status";
+}
+
+fmoe_status fmoe_bank_layout(int bits, int group_size, int hidden, int inter, int64_t* record_bytes, int64_t off[9]) {
+  if (!record_bytes || !off) return fail(FMOE_ERR_INVALID_ARG, "NULL output");
+  if (bits != 2 && bits != 4) return fail(FMOE_ERR_UNSUPPORTED, "bits %d", bits);
+  if (group_size != kGroup) return fail(FMOE_ERR_UNSUPPORTED, "group_size %d", group_size);
+  if (hidden <= 0 || inter <= 0 || hidden % group_size || inter % group_size)
+    return fail(FMOE_ERR_INVALID_ARG, "hidden %d / inter %d", hidden, inter);
+  const int64_t dims[3][2] = {{inter, hidden}, {inter, hidden}, {hidden, inter}};
+  int64_t pos = 0;
+  for (int m = 0; m < 3; ++m) {
+    const int64_t rows = dims[m][0], cols = dims[m][1];
+    const int64_t sizes[3] = {rows * cols * bits / 8, rows * (cols / group_size) * 2, rows * (cols / group_size) * 2};
+    for (int k = 0; k < 3; ++k) {
+      off[3 * m + k] = pos;
+      pos = (pos + sizes[k] + 15) / 16 * 16;
+    }
+  }
+  *record_bytes = pos;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_rmsnorm(const float* h, const float* gamma, float eps, int T, int H, float* y, fmoe_stream_t stream) {
+  if (T < 0 || H < 1) return fail(FMOE_ERR_INVALID_ARG, "T %d, H %d", T, H);
+  if (T == 0) return FMOE_OK;
+  if (!h || !y) return fail(FMOE_ERR_INVALID_ARG, "h or y is NULL");
+  if (!(eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)eps);
+  cudaError_t e = launch_rmsnorm(h, gamma, eps, T, H, y, cs(stream));
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "rmsnorm launch");
+}
+
+size_t fmoe_router_topk_workspace_size(int T, int E) {
+  if (T < 1) T = 1;
+  if (T > 1024) T = 1024;
+  return layout(0, E, 32, 0, T).total;
+}
+
+fmoe_status fmoe_router_topk(const float* x, const uint16_t* w_router, const float* logit_bias, int T, int H, int E,
+                             int K, int32_t* idx, float* w, float* probs, void* ws, size_t ws_bytes,
+                             fmoe_stream_t stream) {
+  if (T < 0) return fail(FMOE_ERR_INVALID_ARG, "T %d", T);
+  if (H < 128 || H % 128 || H > 12288) return fail(FMOE_ERR_UNSUPPORTED, "H %d: a multiple of 128 in [128, 12288]", H);
+  if (E < 1 || E > 4096) return fail(FMOE_ERR_UNSUPPORTED, "E %d (1..4096)", E);
+  if (K < 1 || K > E || K > 32) return fail(FMOE_ERR_INVALID_ARG, "K %d (1..min(E, 32))", K);
+  if (T == 0) return FMOE_OK;
+  if (!x || !w_router || !idx || !w) return fail(FMOE_ERR_INVALID_ARG, "x, w_router, idx or w is NULL");
+  if (!aligned16(x) || !aligned16(w_router)) return fail(FMOE_ERR_ALIGNMENT, "x and w_router must be 16-byte aligned");
+  const int Tc = T > 1024 ? 1024 : T;
+  const WsLayout L = layout(0, E, 32, 0, Tc);
+  fmoe_status st = check_ws(ws, ws_bytes, L.total);
+  if (st != FMOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
+  for (int t0 = 0; t0 < T; t0 += 1024) {
+    const int n = T - t0 < 1024 ? T - t0 : 1024;
+    RouterParams p{};
+    p.h = x + (size_t)t0 * H;
+    p.norm = 0;
+    p.w_router = w_router;
+    p.bias = logit_bias;
+    p.w_sgate = nullptr;
+    p.T = n;
+    p.H = H;
+    p.E = E;
+    p.K = K;
+    p.logits = reinterpret_cast<float*>(base + L.logits);
+    p.idx = reinterpret_cast<int32_t*>(base + L.idx);
+    p.wts = reinterpret_cast<float*>(base + L.wts);
+    p.idx_out = idx + (size_t)t0 * K;
+    p.w_out = w + (size_t)t0 * K;
+    p.probs_out = probs ? probs + (size_t)t0 * E : nullptr;
+    p.tickets = ctrl->tickets;
+    p.err = &ctrl->err;
+    cudaError_t e = launch_router(p, 0, cs(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  }
+  return FMOE_OK;
+}
+
+size_t fmoe_expert_ffn_workspace_size(const fmoe_bank* bank) {
+  if (!bank) return 0;
+  return layout(bank->hidden, 0, 1, bank->inter, 1).total;
+}
+
+fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, float* y, void* ws, size_t ws_bytes,
+                            fmoe_stream_t stream) {
+  fmoe_status st = check_bank(bank, "expert");
+  if (st != FMOE_OK) return st;
+  if (expert < 0 || expert >= bank->num_experts)
+    return fail(FMOE_ERR_INVALID_ARG, "expert %d outside [0, %d)", expert, bank->num_experts);
+  if (!x || !y) return fail(FMOE_ERR_INVALID_ARG, "x or y is NULL");
+  if (!aligned16(x)) return fail(FMOE_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  const WsLayout L = layout(bank->hidden, 0, 1, bank->inter, 1);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != FMOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
+  const int bits = bank->bits;
+  cudaError_t e = launch_xq(x, bank->hidden, bits, base + L.xq_limbs, reinterpret_cast<float2*>(base + L.xq_cs),
+                            cs(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "digits launch");
+  ExpertParams p{};
+  p.routed = ref(*bank);
+  p.shared = ref(*bank);
+  p.idx = nullptr;
+  p.fixed_expert = expert;
+  p.K = 1;
+  p.has_shared = 0;
+  p.H = bank->hidden;
+  p.I = bank->inter;
+  p.xq_limbs = reinterpret_cast<const uint32_t*>(base + L.xq_limbs);
+  p.xq_cs = reinterpret_cast<const float2*>(base + L.xq_cs);
+  p.act = reinterpret_cast<float*>(base + L.act);
+  p.wts = nullptr;
+  p.resid = nullptr;
+  p.out = y;
+  p.err = &ctrl->err;
+  if ((e = launch_gateup(p, bits, cs(stream))) != cudaSuccess) return cuda_fail(e, "gate/up launch");
+  if ((e = launch_down(p, bits, cs(stream))) != cudaSuccess) return cuda_fail(e, "down launch");
+  return FMOE_OK;
+}
+
+static fmoe_status check_layer(const fmoe_layer* layer) {
+  if (!layer) return fail(FMOE_ERR_INVALID_ARG, "layer is NULL");
+  fmoe_status st = check_bank(&layer->routed, "routed");
+  if (st != FMOE_OK) return st;
+  if ((st = check_bank(&layer->shared, "shared")) != FMOE_OK) return st;
+  const fmoe_bank &r = layer->routed, &s = layer->shared;
+  if (r.bits != s.bits || r.hidden != s.hidden || r.inter != s.inter)
+    return fail(FMOE_ERR_UNSUPPORTED, "routed and shared banks must share bits, hidden and inter");
+  if (!layer->w_router || !layer->w_shared_gate) return fail(FMOE_ERR_INVALID_ARG, "w_router or w_shared_gate is NULL");
+  if (!aligned16(layer->w_router) || !aligned16(layer->w_shared_gate))
+    return fail(FMOE_ERR_ALIGNMENT, "w_router and w_shared_gate must be 16-byte aligned");
+  const int E = r.num_experts, K = layer->top_k;
+  if (E > 4096) return fail(FMOE_ERR_UNSUPPORTED, "E %d > 4096", E);
+  if (r.hidden > 12288) return fail(FMOE_ERR_UNSUPPORTED, "hidden %d > 12288", r.hidden);
+  if (K < 1 || K > E || K > 32) return fail(FMOE_ERR_INVALID_ARG, "top_k %d (1..min(E, 32))", K);
+  if ((K + 1) * (r.inter * r.bits / 128) > 512)
+    return fail(FMOE_ERR_UNSUPPORTED, "(top_k+1) * inter*bits/128 = %d > 512", (K + 1) * (r.inter * r.bits / 128));
+  if (!(layer->eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)layer->eps);
+  return FMOE_OK;
+}
+
+size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
+  (void)T;
+  if (!layer) return 0;
+  return layout(layer->routed.hidden, layer->routed.num_experts, layer->top_k, layer->routed.inter, 1).total;
+}
+
+// One token through the block: router (+RMSNorm, digits, top-K) -> gate/up -> down + combine.
+static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
+                               uint8_t* base, const WsLayout& L, cudaStream_t s) {
+  const fmoe_bank& r = layer->routed;
+  const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
+  WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
+  RouterParams rp{};
+  rp.h = h;
+  rp.gamma = layer->gamma;
+  rp.eps = layer->eps;
+  rp.norm = layer->gamma != nullptr;
+  rp.w_router = layer->w_router;
+  rp.bias = layer->router_bias;
+  rp.w_sgate = layer->w_shared_gate;
+  rp.T = 1;
+  rp.H = H;
+  rp.E = E;
+  rp.K = K;
+  rp.xq_limbs = base + L.xq_limbs;
+  rp.xq_cs = reinterpret_cast<float2*>(base + L.xq_cs);
+  rp.xq_limb_stride = 3LL * H;
+  rp.xq_cs_stride = H / 32;
+  rp.logits = reinterpret_cast<float*>(base + L.logits);
+  rp.idx = reinterpret_cast<int32_t*>(base + L.idx);
+  rp.wts = reinterpret_cast<float*>(base + L.wts);
+  rp.idx_out = idx_out;
+  rp.w_out = w_out;
+  rp.probs_out = nullptr;
+  rp.tickets = ctrl->tickets;
+  rp.err = &ctrl->err;
+  const bool trace = g_trace_on;
+  g_trace_on = false;
+  cudaError_t e;
+  if (trace && (e = cudaEventRecord(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  e = launch_router(rp, bits, s);
+  if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  if (trace && (e = cudaEventRecord(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  ExpertParams p{};
+  p.routed = ref(r);
+  p.shared = ref(layer->shared);
+  p.idx = rp.idx;
+  p.fixed_expert = 0;
+  p.K = K;
+  p.has_shared = 1;
+  p.H = H;
+  p.I = I;
+  p.xq_limbs = reinterpret_cast<const uint32_t*>(base + L.xq_limbs);
+  p.xq_cs = reinterpret_cast<const float2*>(base + L.xq_cs);
+  p.act = reinterpret_cast<float*>(base + L.act);
+  p.wts = rp.wts;
+  p.resid = h;
+  p.out = out;
+  p.err = &ctrl->err;
+  if ((e = launch_gateup(p, bits, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
+  if (trace && (e = cudaEventRecord(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if ((e = launch_down(p, bits, s)) != cudaSuccess) return cuda_fail(e, "down launch");
+  if (trace && (e = cudaEventRecord(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
+                           float* topk_w, void* ws, size_t ws_bytes, fmoe_stream_t stream) {
+  fmoe_status st = check_layer(layer);
+  if (st != FMOE_OK) return st;
+  if (T < 0) return fail(FMOE_ERR_INVALID_ARG, "T %d", T);
+  if (T == 0) return FMOE_OK;
+  if (!h || !out) return fail(FMOE_ERR_INVALID_ARG, "h or out is NULL");
+  if (!aligned16(h) || !aligned16(out)) return fail(FMOE_ERR_ALIGNMENT, "h and out must be 16-byte aligned");
+  const int H = layer->routed.hidden, K = layer->top_k;
+  const WsLayout L = layout(H, layer->routed.num_experts, K, layer->routed.inter, 1);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != FMOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  for (int t = 0; t < T; ++t) {
+    st = layer_token(layer, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
+                     topk_w ? topk_w + (size_t)t * K : nullptr, base, L, cs(stream));
+    if (st != FMOE_OK) return st;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int nl, const float* h, int T, float* out, void* ws,
+                           size_t ws_bytes, fmoe_stream_t stream) {
+  if (!layers || nl < 1) return fail(FMOE_ERR_INVALID_ARG, "layers NULL or count %d", nl);
+  for (int l = 0; l < nl; ++l) {
+    fmoe_status st = check_layer(&layers[l]);
+    if (st != FMOE_OK) return fail(st, "layer %d: %s", l, g_msg);
+    if (layers[l].routed.hidden != layers[0].routed.hidden)
+      return fail(FMOE_ERR_INVALID_ARG, "layer %d: hidden differs from layer 0", l);
+  }
+  for (int l = 0; l < nl; ++l) {
+    fmoe_status st = fmoe_moe_layer(&layers[l], l == 0 ? h : out, T, out, nullptr, nullptr, ws, ws_bytes, stream);
+    if (st != FMOE_OK) return st;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_trace_next_layer(void* const* events, int n) {
+  if (!events) {
+    g_trace_on = false;
+    return FMOE_OK;
+  }
+  if (n != 4) return fail(FMOE_ERR_INVALID_ARG, "trace needs 4 events, got %d", n);
+  for (int i = 0; i < 4; ++i) {
+    if (!events[i]) return fail(FMOE_ERR_INVALID_ARG, "trace event %d is NULL", i);
+    g_trace[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_trace_on = true;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
+  if (!ws) return fail(FMOE_ERR_WORKSPACE, "workspace is NULL");
+  if (ws_bytes < sizeof(WsControl)) return fail(FMOE_ERR_WORKSPACE, "workspace smaller than its control block");
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsControl), cs(stream));
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "cudaMemsetAsync");
+}
+
+fmoe_status fmoe_workspace_check(void* ws, fmoe_stream_t stream) {
+  if (!ws) return fail(FMOE_ERR_WORKSPACE, "workspace is NULL");
+  cudaError_t e = cudaStreamSynchronize(cs(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  WsControl* ctrl = static_cast<WsControl*>(ws);
+  int err = 0;
+  if ((e = cudaMemcpy(&err, &ctrl->err, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpy");
+  if (err == 0) return FMOE_OK;
+  const int zero = 0;
+  if ((e = cudaMemcpy(&ctrl->err, &zero, sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpy");
+  if (err == kDevBadIndex) return fail(FMOE_ERR_INVALID_ARG, "a kernel met an expert index outside the bank");
+  return fail(FMOE_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (code %d)", err);
+}
+
+}  // extern "C"

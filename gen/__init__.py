@@ -268,3 +268,72 @@ def device_normal_f32(k, std, dst, stream_ptr):
 
 def device_normal_bf16(k, std, dst, stream_ptr):
     _check(cuda_lib().fg_cuda_normal_bf16(k, std, dst.numel(), dst.data_ptr(), stream_ptr), "fg_cuda_normal_bf16")
+
+
+# ----------------------------------------------------------------------------------------------- device layers
+
+
+@dataclasses.dataclass
+class DeviceLayer:
+    spec: LayerSpec
+    bank: object          # torch uint8 [E * record]
+    shared: object        # torch uint8 [record]
+    w_router: object      # torch int16 (bf16 bits) [E][H]
+    w_shared_gate: object  # torch int16 [H]
+    gamma: object         # torch float32 [H]
+    logit_bias: object    # torch float32 [E] or None
+
+
+def upload_layer(hl, device="cuda"):
+    """Copies a fully drawn host layer to the device."""
+    import torch
+    spec = hl.spec
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    return DeviceLayer(spec, t(gen_bank_bytes(hl)), t(hl.shared), t(hl.w_router.view(np.int16)),
+                       t(hl.w_shared_gate.view(np.int16)), t(hl.gamma),
+                       None if hl.logit_bias is None else t(hl.logit_bias))
+
+
+def gen_bank_bytes(hl):
+    return bank_array(hl).reshape(-1)
+
+
+def device_layer(spec, seed=WEIGHT_SEED, layer=0, device="cuda"):
+    """Draws a whole layer directly in device memory (same bytes as host_layer)."""
+    import torch
+    stream = torch.cuda.current_stream().cuda_stream
+    nbytes = record_bytes(spec)
+    bank = torch.empty(spec.experts * nbytes, dtype=torch.uint8, device=device)
+    shared = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    device_fill_bank(spec, seed, layer, 0, spec.experts, bank, stream)
+    device_fill_bank(spec, seed, layer, EXPERT_SHARED, 1, shared, stream)
+    wr = torch.empty((spec.experts, spec.hidden), dtype=torch.int16, device=device)
+    device_normal_bf16(key(seed, layer, EXPERT_LAYER, KIND_ROUTER), spec.router_std, wr, stream)
+    wsg = torch.empty(spec.hidden, dtype=torch.int16, device=device)
+    device_normal_bf16(key(seed, layer, EXPERT_LAYER, KIND_SHARED_GATE), spec.shared_gate_std, wsg, stream)
+    gamma = torch.from_numpy(host_gamma(spec, seed, layer)).to(device)
+    bias = None
+    if spec.zipf > 0:
+        bias = torch.from_numpy(zipf_logit_bias(spec, seed, layer)).to(device)
+    return DeviceLayer(spec, bank, shared, wr, wsg, gamma, bias)
+
+
+def binding_layer(dl, top_k=None, use_gamma=True):
+    """Wraps a DeviceLayer as a layer of the product binding."""
+    import bit_dequant_expert_router_b200 as fmoe
+    spec = dl.spec
+    nbytes, off = record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    routed = fmoe.Bank(dl.bank, spec.bits, spec.hidden, spec.inter, spec.experts, nbytes, off, spec.group)
+    shared = fmoe.Bank(dl.shared, spec.bits, spec.hidden, spec.inter, 1, nbytes, off, spec.group)
+    return fmoe.Layer(routed, shared, dl.w_router, dl.w_shared_gate, dl.gamma if use_gamma else None, dl.logit_bias,
+                      spec.eps, spec.top_k if top_k is None else top_k)
+
+
+def device_tokens(t0, T, hidden, device="cuda"):
+    """Token hidden states drawn on the device (same values as host_tokens)."""
+    import torch
+    out = torch.empty((T, hidden), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream().cuda_stream
+    for i in range(T):
+        device_normal_f32(token_key(t0 + i), 1.0, out[i], stream)
+    return out

@@ -1,0 +1,187 @@
+/*
+ * fmoe.h -- C ABI of libfmoe.so: the routed Mixture-of-Experts FFN block at
+ * decode time, as hand-written CUDA kernels for sm_100a (B200).
+ *
+ * The block follows the Flash-MoE pages:
+ *   - "What is Flash-MoE" (a2a-mcp.org), MoE section: per layer a router picks
+ *     4 of 512 routed experts and one shared expert always runs;
+ *   - same page, section 2: group-wise affine codes, dequantised as
+ *     code * scale + bias (4-bit production, 2-bit experimental);
+ *   - same page, section 3 (hand-tuned Metal shaders): two-pass RMSNorm, fused
+ *     SwiGLU, and one combine pass of weighted experts + residual + sigmoid-gated
+ *     shared expert;
+ *   - "Flash-MoE" wiki summary (jeongsk), per-layer pipeline: routing projection,
+ *     softmax, top-K.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers owned by the caller unless stated; the
+ *     library never allocates or frees memory.
+ *   - Calls are stream-ordered and asynchronous: they validate their arguments
+ *     on the host, enqueue kernels on `stream` and return.  Errors in the
+ *     arguments are reported before anything is enqueued.  A failed launch
+ *     returns FMOE_ERR_CUDA.  Asynchronous device faults surface at the
+ *     caller's next synchronisation.
+ *   - No call aborts, throws or exits; fmoe_last_error() returns a message for
+ *     the last non-OK status of the calling host thread.
+ *   - Layouts are row-major.  bf16 values are passed as uint16_t bit patterns.
+ *
+ * Packed matrix [out][in] with b-bit codes (b = 2 or 4) and group size 64:
+ *   qw    uint32[out][in*b/32]  code of column c at word c/(32/b), bits
+ *                               [b*(c%(32/b)), +b) counted from the LSB;
+ *   scale bf16[out][in/64], bias bf16[out][in/64]: group g of row r covers
+ *                               columns [64g, 64g+63];
+ *   weight (r, c) = code(r, c) * scale[r][c/64] + bias[r][c/64].
+ * Expert record: gate [I][H] | up [I][H] | down [H][I], each {qw, scale, bias},
+ * every sub-array 16-byte aligned; at I = 1024, H = 4096 a record is
+ * 7,077,888 bytes at 4-bit (the pages' "6.75 MB per expert") and 3,932,160
+ * bytes at 2-bit (their "~3.9 MB").  A bank is `num_experts` records at a
+ * fixed stride.
+ */
+#ifndef FMOE_H
+#define FMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* fmoe_stream_t;
+
+typedef enum {
+  FMOE_OK = 0,
+  FMOE_ERR_INVALID_ARG = 1,   /* NULL pointer, bad shape or count */
+  FMOE_ERR_ALIGNMENT = 2,     /* a pointer, offset or stride is not 16-byte aligned */
+  FMOE_ERR_UNSUPPORTED = 3,   /* a shape or width these kernels do not handle */
+  FMOE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the size query returns */
+  FMOE_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  FMOE_ERR_DEVICE_TIMEOUT = 6 /* a kernel's bounded wait ran out (reported by fmoe_workspace_check) */
+} fmoe_status;
+
+/* A bank of expert records in device memory.
+ * bits: 2 or 4.  group_size: 64 (the only supported value).
+ * hidden (H), inter (I): model width and expert intermediate width.
+ * base: record 0 (16-byte aligned); stride: bytes between records (multiple of 16).
+ * off[9]: byte offsets inside a record of gate.qw, gate.scale, gate.bias,
+ *         up.qw, up.scale, up.bias, down.qw, down.scale, down.bias (multiples of 16). */
+typedef struct {
+  int32_t bits;
+  int32_t group_size;
+  int32_t hidden;
+  int32_t inter;
+  int32_t num_experts;
+  int32_t reserved;
+  const void* base;
+  int64_t stride;
+  int64_t off[9];
+} fmoe_bank;
+
+/* One MoE layer.
+ * routed: E = routed.num_experts experts.  shared: the always-on expert (record 0 used).
+ * w_router: bf16 [E][H].  router_bias: fp32 [E] added to the logits, or NULL.
+ * w_shared_gate: bf16 [H]; the shared expert's output is scaled by sigmoid(w_shared_gate . x).
+ * gamma: fp32 [H] RMSNorm weight; NULL skips the normalisation (x = h).
+ * eps: RMSNorm epsilon (1e-6 for the Qwen3.5-397B-A17B shapes).  top_k: K, 1 <= K <= min(E, 32). */
+typedef struct {
+  fmoe_bank routed;
+  fmoe_bank shared;
+  const uint16_t* w_router;
+  const float* router_bias;
+  const uint16_t* w_shared_gate;
+  const float* gamma;
+  float eps;
+  int32_t top_k;
+} fmoe_layer;
+
+/* Canonical record layout for (bits, group_size, hidden, inter): writes the
+ * record size and the nine sub-array offsets.  Host-only helper. */
+fmoe_status fmoe_bank_layout(int bits, int group_size, int hidden, int inter, int64_t* record_bytes, int64_t off[9]);
+
+/* Two-pass RMSNorm ("What is Flash-MoE", section 3: sum of squares, then apply):
+ *   y[t][i] = h[t][i] / sqrt(mean_i h[t][i]^2 + eps) * gamma[i].
+ * h, y: fp32 [T][H] (y may equal h).  gamma: fp32 [H] or NULL for unit weights.
+ * T >= 0 (T = 0 enqueues nothing), H >= 1. */
+fmoe_status fmoe_rmsnorm(const float* h, const float* gamma, float eps, int T, int H, float* y, fmoe_stream_t stream);
+
+/* Router GEMV + softmax + top-K ("Flash-MoE" wiki summary, per-layer pipeline:
+ * routing projection, then softmax and top-K; the pages run the selection on
+ * the CPU, here it stays on the GPU):
+ *   l[t][e] = sum_i w_router[e][i] x[t][i] (+ logit_bias[e]);  p = softmax_e(l);
+ *   idx[t][0..K-1] = the K largest p in descending order, ties to the lower index;
+ *   w[t][k] = p[idx[t][k]] / sum_k' p[idx[t][k']].
+ * x: fp32 [T][H] (already normalised).  w_router: bf16 [E][H].  logit_bias: fp32 [E] or NULL.
+ * idx: int32 [T][K]; w: fp32 [T][K]; probs: fp32 [T][E] or NULL.
+ * ws: device workspace of fmoe_router_topk_workspace_size(T, E) bytes, 256-byte
+ * aligned, zeroed once before first use (fmoe_workspace_init); every call
+ * leaves it ready for the next.  Requirements: H % 128 == 0, 1 <= K <= min(E, 32), E <= 4096. */
+fmoe_status fmoe_router_topk(const float* x, const uint16_t* w_router, const float* logit_bias, int T, int H, int E,
+                             int K, int32_t* idx, float* w, float* probs, void* ws, size_t ws_bytes,
+                             fmoe_stream_t stream);
+size_t fmoe_router_topk_workspace_size(int T, int E);
+
+/* One expert's FFN for one token ("What is Flash-MoE", sections 2-3: dequant
+ * matvec, fused SwiGLU):
+ *   g = Wg x, u = Wu x, a = silu(g) * u with silu(z) = z / (1 + exp(-z)), y = Wd a.
+ * bank: the expert bank; expert: record index in [0, num_experts).
+ * x: fp32 [H]; y: fp32 [H].  ws: fmoe_expert_ffn_workspace_size(bank) bytes,
+ * 256-byte aligned, zeroed once (fmoe_workspace_init).
+ * Requirements: bits 2 or 4, group 64, H % 128 == 0, I % 128 == 0,
+ * H*bits/128 and I*bits/128 powers of two no larger than 512. */
+fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, float* y, void* ws, size_t ws_bytes,
+                            fmoe_stream_t stream);
+size_t fmoe_expert_ffn_workspace_size(const fmoe_bank* bank);
+
+/* The whole block for T tokens (the MoE section and sections 2-3 of "What is
+ * Flash-MoE"; pipeline of the jeongsk wiki summary):
+ *   x = RMSNorm(h) (skipped when gamma is NULL); routing as fmoe_router_topk;
+ *   sigma = sigmoid(w_shared_gate . x);
+ *   out[t] = h[t] + sum_k w[t][k] FFN_{idx[t][k]}(x[t]) + sigma[t] FFN_shared(x[t]).
+ * h, out: fp32 [T][H]; out may equal h (in-place residual), no other overlap.
+ * topk_idx (int32 [T][K]) and topk_w (fp32 [T][K]) receive the routing, or NULL.
+ * ws: fmoe_moe_layer_workspace_size(layer, T) bytes, 256-byte aligned, zeroed
+ * once before first use (fmoe_workspace_init); calls on one workspace must be
+ * ordered on one stream.  Requirements: those of fmoe_expert_ffn for both
+ * banks (same bits, hidden, inter), 1 <= K <= min(E, 32), E <= 4096,
+ * (K+1) * I*bits/128 <= 512.  T = 0 enqueues nothing. */
+fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
+                           float* topk_w, void* ws, size_t ws_bytes, fmoe_stream_t stream);
+size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
+
+/* A stack of L layers applied in order, each block's output feeding the next
+ * (the 60-layer decode loop of the jeongsk wiki summary, without the attention
+ * layers): h_0 = h, h_{l+1} = block_l(h_l), out = h_L.  out may equal h.
+ * ws: max over l of fmoe_moe_layer_workspace_size(&layers[l], T) bytes. */
+fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int L, const float* h, int T, float* out, void* ws,
+                           size_t ws_bytes, fmoe_stream_t stream);
+
+/* Tracing hook for per-kernel timing: the next fmoe_moe_layer call made by
+ * this host thread records the caller's CUDA events (cudaEvent_t handles) on
+ * its stream: events[0] before the router kernel, events[1] after it,
+ * events[2] after the gate/up kernel, events[3] after the down/combine kernel
+ * (first token only when T > 1).  n must be 4; events = NULL cancels. */
+fmoe_status fmoe_trace_next_layer(void* const* events, int n);
+
+/* Zeroes the workspace's control words (enqueued on `stream`).  Call once after
+ * allocating a workspace, before its first use. */
+fmoe_status fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the workspace's device error
+ * word: FMOE_OK, or FMOE_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait. */
+fmoe_status fmoe_workspace_check(void* ws, fmoe_stream_t stream);
+
+/* Message for the last non-OK status returned to this host thread ("" if none). */
+const char* fmoe_last_error(void);
+
+/* Static name of a status code. */
+const char* fmoe_status_string(fmoe_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fmoe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMOE_H */

@@ -1,4 +1,6 @@
 """Test-side helpers: an independent numpy packer/dequantiser, the error metric and layer marshalling."""
+import math
+
 import numpy as np
 
 import gen
@@ -83,3 +85,38 @@ def oracle_layer_sparse(hl, top_k=None):
 
 def silu(z):
     return z / (1.0 + np.exp(-z))
+
+
+U32 = 2.0 ** -24
+
+
+def routing_margin(w_router_bf16, xhat, logit_bias=None, safety=8.0):
+    """Per-token bound on how far an fp32 logit may sit from the exact one: safety * u * sqrt(H) * sum_i |w x|.
+
+    Returns (exact logits [E] in fp64 from the fp64 x, delta)."""
+    W = bf16_to_f64(w_router_bf16)
+    l = W @ xhat + (0.0 if logit_bias is None else np.asarray(logit_bias, np.float64))
+    s = np.abs(W) @ np.abs(xhat)
+    return l, safety * U32 * math.sqrt(W.shape[1]) * float(s.max())
+
+
+def check_routing(gpu_idx, logits, K, delta):
+    """Compares one token's GPU top-K with the exact logits.
+
+    Returns True when the exact top K+1 logits are separated by more than delta (the
+    selection must then match exactly, in order); otherwise checks that every selected
+    expert is within delta of the exact K-th logit (a valid near-tie choice) and returns False."""
+    order = np.argsort(-logits, kind="stable")
+    top = logits[order[:K + 1]] if len(logits) > K else np.append(logits[order[:K]], -np.inf)
+    gaps = top[:-1] - top[1:]
+    gpu_idx = [int(i) for i in gpu_idx]
+    if np.all(gaps > delta):
+        assert gpu_idx == order[:K].tolist(), (gpu_idx, order[:K].tolist())
+        return True
+    assert len(set(gpu_idx)) == K
+    kth = logits[order[K - 1]]
+    for i in gpu_idx:
+        assert logits[i] >= kth - delta, (i, logits[i], kth)
+    sel = logits[gpu_idx]
+    assert np.all(sel[:-1] >= sel[1:] - delta)  # descending up to the near-tie margin
+    return False

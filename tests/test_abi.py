@@ -1,0 +1,110 @@
+"""The C ABI: library loads, exports every declared symbol, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_dequant_expert_router_b200 as fmoe
+from bit_dequant_expert_router_b200 import _abi
+import gen
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(fmoe_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = _declared()
+    assert len(names) >= 14
+    lib = ctypes.CDLL(_abi.SO_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert names == {s[0] for s in _abi.SIGNATURES}
+
+
+def test_version_and_status_strings():
+    L = fmoe.lib()
+    assert L.fmoe_version() >= 100
+    assert L.fmoe_status_string(0) == b"FMOE_OK"
+    assert L.fmoe_status_string(6) == b"FMOE_ERR_DEVICE_TIMEOUT"
+
+
+@pytest.mark.parametrize("bits,H,I", [(4, 4096, 1024), (2, 4096, 1024), (4, 256, 128), (2, 256, 128)])
+def test_bank_layout_matches_generator_layout(bits, H, I):
+    assert fmoe.bank_layout(bits, H, I) == gen.record_layout(bits, H, I)
+
+
+def _fake_bank(bits=4, H=4096, I=1024, E=512, base=0x10000000, stride=None, off=None):
+    nb, o = gen.record_layout(bits, H, I)
+    b = _abi.FmoeBank(bits, 64, H, I, E, 0, base, nb if stride is None else stride,
+                      (ctypes.c_int64 * 9)(*(o if off is None else off)))
+    return b
+
+
+def _fake_layer(**kw):
+    k = kw.pop("top_k", 4)
+    routed = _fake_bank(**kw)
+    shared = _fake_bank(**dict(kw, E=1))
+    return _abi.FmoeLayer(routed, shared, 0x20000000, None, 0x30000000, 0x40000000, 1e-6, k)
+
+
+def _call_layer(layer, T=1, ws=0x50000000, ws_bytes=1 << 30, h=0x60000000, out=0x60000000):
+    return fmoe.lib().fmoe_moe_layer(ctypes.byref(layer), h, T, out, None, None, ws, ws_bytes, None)
+
+
+def test_layer_validation_errors_are_reported_before_any_launch():
+    L = fmoe.lib()
+    assert L.fmoe_moe_layer(None, 0x1000, 1, 0x1000, None, None, 0x1000, 1 << 20, None) == 1
+    assert b"NULL" in L.fmoe_last_error()
+    assert _call_layer(_fake_layer(bits=3)) == 3
+    assert _call_layer(_fake_layer(top_k=0)) == 1
+    assert _call_layer(_fake_layer(top_k=513)) == 1
+    assert _call_layer(_fake_layer(top_k=33)) == 1
+    assert _call_layer(_fake_layer(H=4000)) == 3
+    assert _call_layer(_fake_layer(H=384)) == 3       # H*bits/128 not a power of two
+    assert _call_layer(_fake_layer(base=0x10000008)) == 2
+    assert _call_layer(_fake_layer(stride=7077888 + 8)) == 2
+    off = list(gen.record_layout(4, 4096, 1024)[1])
+    off[4] += 4
+    assert _call_layer(_fake_layer(off=off)) == 2
+    assert _call_layer(_fake_layer(), ws=0x50000010) == 2   # not 256-byte aligned
+    assert _call_layer(_fake_layer(), ws_bytes=1024) == 4
+    assert _call_layer(_fake_layer(), ws=None) == 4
+    assert _call_layer(_fake_layer(), h=0x60000004) == 2
+    assert _call_layer(_fake_layer(), T=-1) == 1
+    assert _call_layer(_fake_layer(), T=0) == 0            # empty batch: nothing enqueued
+    # (top_k + 1) * inter*bits/128 must fit one 512-thread CTA
+    assert _call_layer(_fake_layer(top_k=16)) == 3
+
+
+def test_workspace_size_query_is_positive_and_monotone():
+    L = fmoe.lib()
+    lay = _fake_layer()
+    n4 = L.fmoe_moe_layer_workspace_size(ctypes.byref(lay), 1)
+    lay8 = _fake_layer(top_k=8)
+    assert n4 > 0 and L.fmoe_moe_layer_workspace_size(ctypes.byref(lay8), 1) >= n4
+    assert L.fmoe_router_topk_workspace_size(64, 512) > L.fmoe_router_topk_workspace_size(1, 512)
+
+
+def test_other_entry_points_validate():
+    L = fmoe.lib()
+    assert L.fmoe_rmsnorm(0x1000, None, 1e-6, 0, 4096, 0x1000, None) == 0
+    assert L.fmoe_rmsnorm(None, None, 1e-6, 1, 4096, 0x1000, None) == 1
+    assert L.fmoe_router_topk(0x1000, 0x2000, None, 1, 4096, 512, 0, 0x3000, 0x4000, None, 0x5000, 1 << 20,
+                              None) == 1
+    assert L.fmoe_router_topk(0x1000, 0x2000, None, 1, 100, 512, 4, 0x3000, 0x4000, None, 0x5000, 1 << 20,
+                              None) == 3
+    b = _fake_bank()
+    assert L.fmoe_expert_ffn(ctypes.byref(b), 512, 0x1000, 0x2000, 0x5000, 1 << 20, None) == 1
+    assert L.fmoe_expert_ffn(ctypes.byref(b), -1, 0x1000, 0x2000, 0x5000, 1 << 20, None) == 1
+    assert L.fmoe_moe_stack(None, 1, 0x1000, 1, 0x1000, 0x5000, 1 << 20, None) == 1
+    assert L.fmoe_workspace_init(None, 100, None) == 4
