@@ -211,7 +211,8 @@ def main():
     with torch.cuda.graph(graph, stream=stream):
         for i in range(G):
             step(i, stream)
-    graph.replay()
+    with torch.cuda.stream(stream):
+        graph.replay()
     stream.synchronize()
 
     # ---- timed region: `steps` tokens, as steps / G graph replays
@@ -220,10 +221,11 @@ def main():
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for _ in range(steps // G):
-            graph.replay()
-        ev1.record(stream)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(steps // G):
+                graph.replay()
+            ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize(dev)
     ms = ev0.elapsed_time(ev1)
@@ -240,12 +242,18 @@ def main():
     # ---- per-kernel durations: a separate replay with trace events around each kernel
     tr = min(G, 500)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(tr)]
+    for e4 in evs:  # torch creates the CUDA event on its first record
+        for e in e4:
+            e.record(stream)
+    stream.synchronize()
+    # the library records these as external event nodes inside the captured graph
     tgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(tgraph, stream=stream):
         for i in range(tr):
             fmoe.trace_next_layer(evs[i])
             step(i, stream)
-    tgraph.replay()
+    with torch.cuda.stream(stream):
+        tgraph.replay()
     stream.synchronize()
     dur = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs]) * 1e3
     router_us, gateup_us, down_us = (float(np.mean(dur[:, k])) for k in range(3))
@@ -265,15 +273,17 @@ def main():
                 hd.copy_(hh[i], non_blocking=True)
                 fmoe.moe_layer(layers[i % ncopy], hd, out=od, ws=ws, stream=stream)
                 oh[i].copy_(od, non_blocking=True)
-        egraph.replay()
+        with torch.cuda.stream(stream):
+            egraph.replay()
         stream.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps // G):
-            egraph.replay()
-        e1.record(stream)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps // G):
+                egraph.replay()
+            e1.record(stream)
         e1.synchronize()
         ems = e0.elapsed_time(e1)
         if world > 1:

@@ -3,6 +3,7 @@
 // enqueuing anything and reports through fmoe_status (never aborts).
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -39,19 +40,27 @@ bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
 // Workspace regions (byte offsets), in this order.
 struct WsLayout {
-  size_t ctrl, xq_limbs, xq_cs, logits, idx, wts, act, total;
+  size_t ctrl, xq_limbs, xq_cs, logits, route_idx, route_w, act, act_limbs, act_cs, grp_cnt, total;
 };
 
+// Workspace: control words, digits of x (3 bytes per element + one float2 per
+// chunk of at most 32 elements), router logits [T][E+1], the routing [T][K]
+// and weights [T][K+1], the activations of the K+1 expert slots with their
+// digits, and per-group completion counters.
 WsLayout layout(int H, int E, int K, int I, int T) {
   WsLayout L;
+  const size_t ne = (size_t)K + 1;
   L.ctrl = 0;
   L.xq_limbs = up(sizeof(WsControl));
-  L.xq_cs = L.xq_limbs + up((size_t)T * 3 * H);       // 3 bytes of digits per element
-  L.logits = L.xq_cs + up((size_t)T * (H / 32) * 8);  // one float2 per chunk (at most H/32 chunks)
-  L.idx = L.logits + up((size_t)T * (E + 1) * 4);
-  L.wts = L.idx + up((size_t)T * (K > 0 ? K : 1) * 4);
-  L.act = L.wts + up((size_t)T * (K + 1) * 4);
-  L.total = L.act + up((size_t)(K + 1) * (I > 0 ? I : 1) * 4);
+  L.xq_cs = L.xq_limbs + up((size_t)T * 3 * H);
+  L.logits = L.xq_cs + up((size_t)T * (H / 32) * 8);
+  L.route_idx = L.logits + up((size_t)T * (E + 1) * 4);
+  L.route_w = L.route_idx + up((size_t)T * ne * 4);
+  L.act = L.route_w + up((size_t)T * ne * 4);
+  L.act_limbs = L.act + up(ne * I * 4);
+  L.act_cs = L.act_limbs + up(ne * 3 * I);
+  L.grp_cnt = L.act_cs + up(ne * (I / 32) * 8);
+  L.total = L.grp_cnt + up(ne * (I / 64 > 0 ? I / 64 : 1) * 4);
   return L;
 }
 
@@ -71,10 +80,11 @@ fmoe_status check_bank(const fmoe_bank* b, const char* name) {
   const int H = b->hidden, I = b->inter;
   if (H < 128 || I < 128 || H % 128 || I % 128)
     return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden %d and inter %d must be positive multiples of 128", name, H, I);
-  const int nch = H * b->bits / 128, ncd = I * b->bits / 128;
-  if (!pow2(nch) || nch > 512 || !pow2(ncd) || ncd > 512)
-    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden*bits/128 (%d) and inter*bits/128 (%d) must be powers of two <= 512",
-                name, nch, ncd);
+  if (!pow2(H / 64) || H > 8192 || !pow2(I / 64) || I > 8192)
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden %d and inter %d must be 64 times a power of two, at most 8192",
+                name, H, I);
+  if (!expert_shapes_supported(b->bits, H, I, 1))
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: shapes exceed the kernels' shared memory", name);
   if (!aligned16(b->base) || (b->stride & 15)) return fail(FMOE_ERR_ALIGNMENT, "%s bank: base/stride not 16-byte aligned", name);
   if (b->num_experts > 1 && b->stride <= 0) return fail(FMOE_ERR_INVALID_ARG, "%s bank: stride %lld", name, (long long)b->stride);
   for (int i = 0; i < 9; ++i)
@@ -93,6 +103,16 @@ BankRef ref(const fmoe_bank& b) {
 
 cudaStream_t cs(fmoe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Records a trace event; under stream capture it becomes an event-record node
+// of the graph (an external event), so the replay timestamps it.
+cudaError_t trace_record(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &st);
+  if (e != cudaSuccess) return e;
+  return cudaEventRecordWithFlags(ev, s, st == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                              : cudaEventRecordDefault);
+}
+
 }  // namespace
 
 int num_sms() {
@@ -105,6 +125,26 @@ int num_sms() {
     cache[dev] = n;
   }
   return cache[dev];
+}
+
+// L2 prefetch of the routed experts' down matrices from the gate/up kernel; FMOE_PREFETCH=0 turns it off.
+int prefetch_down() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("FMOE_PREFETCH");
+    on = (v && v[0] == '0') ? 0 : 1;
+  }
+  return on;
+}
+
+// Dependent launch between the block's kernels; FMOE_PDL=0 in the environment turns it off.
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("FMOE_PDL");
+    on = (v && v[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
 }
 
 }  // namespace fmoe
@@ -192,17 +232,19 @@ fmoe_status fmoe_router_topk(const float* x, const uint16_t* w_router, const flo
     p.T = n;
     p.H = H;
     p.E = E;
-    p.K = K;
     p.logits = reinterpret_cast<float*>(base + L.logits);
-    p.idx = reinterpret_cast<int32_t*>(base + L.idx);
-    p.wts = reinterpret_cast<float*>(base + L.wts);
-    p.idx_out = idx + (size_t)t0 * K;
-    p.w_out = w + (size_t)t0 * K;
-    p.probs_out = probs ? probs + (size_t)t0 * E : nullptr;
-    p.tickets = ctrl->tickets;
     p.err = &ctrl->err;
-    cudaError_t e = launch_router(p, 0, cs(stream));
+    cudaError_t e = launch_router(p, 0, false, cs(stream));
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    TopkParams q{};
+    q.logits = p.logits;
+    q.T = n;
+    q.E = E;
+    q.K = K;
+    q.idx = idx + (size_t)t0 * K;
+    q.w = w + (size_t)t0 * K;
+    q.probs = probs ? probs + (size_t)t0 * E : nullptr;
+    if ((e = launch_topk(q, cs(stream))) != cudaSuccess) return cuda_fail(e, "top-K launch");
   }
   return FMOE_OK;
 }
@@ -231,7 +273,9 @@ fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, f
   ExpertParams p{};
   p.routed = ref(*bank);
   p.shared = ref(*bank);
-  p.idx = nullptr;
+  p.route_idx = nullptr;
+  p.route_w = nullptr;
+  p.E = bank->num_experts;
   p.fixed_expert = expert;
   p.K = 1;
   p.has_shared = 0;
@@ -240,12 +284,15 @@ fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, f
   p.xq_limbs = reinterpret_cast<const uint32_t*>(base + L.xq_limbs);
   p.xq_cs = reinterpret_cast<const float2*>(base + L.xq_cs);
   p.act = reinterpret_cast<float*>(base + L.act);
-  p.wts = nullptr;
+  p.act_limbs = base + L.act_limbs;
+  p.act_cs = reinterpret_cast<float2*>(base + L.act_cs);
+  p.grp_cnt = reinterpret_cast<unsigned int*>(base + L.grp_cnt);
   p.resid = nullptr;
   p.out = y;
   p.err = &ctrl->err;
-  if ((e = launch_gateup(p, bits, cs(stream))) != cudaSuccess) return cuda_fail(e, "gate/up launch");
-  if ((e = launch_down(p, bits, cs(stream))) != cudaSuccess) return cuda_fail(e, "down launch");
+  const bool pdl = pdl_enabled();
+  if ((e = launch_gateup(p, bits, pdl, cs(stream))) != cudaSuccess) return cuda_fail(e, "gate/up launch");
+  if ((e = launch_down(p, bits, pdl, cs(stream))) != cudaSuccess) return cuda_fail(e, "down launch");
   return FMOE_OK;
 }
 
@@ -264,8 +311,9 @@ static fmoe_status check_layer(const fmoe_layer* layer) {
   if (E > 4096) return fail(FMOE_ERR_UNSUPPORTED, "E %d > 4096", E);
   if (r.hidden > 12288) return fail(FMOE_ERR_UNSUPPORTED, "hidden %d > 12288", r.hidden);
   if (K < 1 || K > E || K > 32) return fail(FMOE_ERR_INVALID_ARG, "top_k %d (1..min(E, 32))", K);
-  if ((K + 1) * (r.inter * r.bits / 128) > 512)
-    return fail(FMOE_ERR_UNSUPPORTED, "(top_k+1) * inter*bits/128 = %d > 512", (K + 1) * (r.inter * r.bits / 128));
+  if (!expert_shapes_supported(r.bits, r.hidden, r.inter, K + 1))
+    return fail(FMOE_ERR_UNSUPPORTED, "top_k %d with inter %d at %d bits exceeds the down kernel's shared memory", K,
+                r.inter, r.bits);
   if (!(layer->eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)layer->eps);
   return FMOE_OK;
 }
@@ -293,30 +341,32 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   rp.T = 1;
   rp.H = H;
   rp.E = E;
-  rp.K = K;
   rp.xq_limbs = base + L.xq_limbs;
   rp.xq_cs = reinterpret_cast<float2*>(base + L.xq_cs);
   rp.xq_limb_stride = 3LL * H;
   rp.xq_cs_stride = H / 32;
   rp.logits = reinterpret_cast<float*>(base + L.logits);
-  rp.idx = reinterpret_cast<int32_t*>(base + L.idx);
-  rp.wts = reinterpret_cast<float*>(base + L.wts);
+  rp.top_k = K;
+  rp.route_idx = reinterpret_cast<int32_t*>(base + L.route_idx);
+  rp.route_w = reinterpret_cast<float*>(base + L.route_w);
   rp.idx_out = idx_out;
   rp.w_out = w_out;
-  rp.probs_out = nullptr;
   rp.tickets = ctrl->tickets;
   rp.err = &ctrl->err;
   const bool trace = g_trace_on;
   g_trace_on = false;
+  const bool pdl = pdl_enabled() && !trace;
   cudaError_t e;
-  if (trace && (e = cudaEventRecord(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
-  e = launch_router(rp, bits, s);
+  if (trace && (e = trace_record(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  e = launch_router(rp, bits, pdl, s);
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
-  if (trace && (e = cudaEventRecord(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if (trace && (e = trace_record(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   ExpertParams p{};
   p.routed = ref(r);
   p.shared = ref(layer->shared);
-  p.idx = rp.idx;
+  p.route_idx = rp.route_idx;
+  p.route_w = rp.route_w;
+  p.E = E;
   p.fixed_expert = 0;
   p.K = K;
   p.has_shared = 1;
@@ -325,14 +375,17 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   p.xq_limbs = reinterpret_cast<const uint32_t*>(base + L.xq_limbs);
   p.xq_cs = reinterpret_cast<const float2*>(base + L.xq_cs);
   p.act = reinterpret_cast<float*>(base + L.act);
-  p.wts = rp.wts;
+  p.act_limbs = base + L.act_limbs;
+  p.act_cs = reinterpret_cast<float2*>(base + L.act_cs);
+  p.grp_cnt = reinterpret_cast<unsigned int*>(base + L.grp_cnt);
   p.resid = h;
   p.out = out;
+  p.prefetch_down = prefetch_down();
   p.err = &ctrl->err;
-  if ((e = launch_gateup(p, bits, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
-  if (trace && (e = cudaEventRecord(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
-  if ((e = launch_down(p, bits, s)) != cudaSuccess) return cuda_fail(e, "down launch");
-  if (trace && (e = cudaEventRecord(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if ((e = launch_gateup(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
+  if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if ((e = launch_down(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "down launch");
+  if (trace && (e = trace_record(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   return FMOE_OK;
 }
 
@@ -389,7 +442,7 @@ fmoe_status fmoe_trace_next_layer(void* const* events, int n) {
 fmoe_status fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
   if (!ws) return fail(FMOE_ERR_WORKSPACE, "workspace is NULL");
   if (ws_bytes < sizeof(WsControl)) return fail(FMOE_ERR_WORKSPACE, "workspace smaller than its control block");
-  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsControl), cs(stream));
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, cs(stream));
   return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "cudaMemsetAsync");
 }
 

@@ -45,6 +45,18 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// ------------------------------------------------------------------------------------------ dependent launch
+//
+// Kernels are launched with programmatic stream serialisation: a kernel may
+// start while its predecessor is still running, do work that reads only
+// constant data (weights), then pdl_wait() for the predecessor's results.
+// pdl_trigger() lets the successor start its own constant-data prologue.
+// Without the launch attribute both are no-ops.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------------ mbarrier + bulk copy
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -96,6 +108,15 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return p;
 }
 
+// Orders this thread's earlier generic-proxy accesses to shared memory before
+// later async-proxy (bulk copy) writes to the same bytes.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Asks L2 to fetch [src, src + bytes) ahead of use (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Bulk copy global -> this CTA's shared memory, completing `bytes` of
 // transaction count on barrier `bar`.  dst, src 16-byte aligned; bytes % 16 == 0.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar, uint64_t pol) {
@@ -108,16 +129,20 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 // ------------------------------------------------------------------------------------------ activation format
 //
-// The dot product sum_c code_c * x_c over one 16-byte chunk of codes runs on
-// integer dp4a units.  x is held per group of 64 as a fixed-point value:
+// The dot product sum_c code_c * x_c over a group of 64 codes runs on integer
+// dp4a units.  x is held per group of 64 as a fixed-point value:
 //   x_c ~= cscale * X_c,  X_c = rint(x_c * 2^(22-e)),  2^(e-1) <= max|x| < 2^e,
 // X_c = d0 * 2^16 + d1 * 2^8 + d2 with signed byte digits (|d0| <= 64).
-// The digits of one chunk are stored as 32-bit packs lined up with the way a
-// code word is split into bytes:
+// The digits are stored as 32-bit packs lined up with the way a code word is
+// split into bytes:
 //   4-bit: word w -> lo = w & 0x0F0F0F0F (codes 0,2,4,6), hi = (w >> 4) & ... (1,3,5,7)
 //   2-bit: word w -> pack m = (w >> 2m) & 0x03030303 (codes m, m+4, m+8, m+12)
-// Chunk layout: uint32 limbs[limb 0..2][word 0..3][pack 0..PPW-1], then per
-// chunk a float2 {cscale, sum of x over the chunk}.
+// One group is 48 words: chunk by chunk (a chunk is 16 bytes of codes: two per
+// group at 4-bit, one at 2-bit), and within a chunk [limb 0..2][word 0..3][pack].
+// Across a vector of NG groups the 16-byte pieces are interleaved, piece i of
+// group g at uint4 index i*NG + g, so that lanes reading consecutive groups hit
+// distinct shared-memory banks.  Per chunk there is a float2 {cscale, sum of x
+// over the chunk}, chunk-major.
 
 template <int BITS>
 struct Fmt {
@@ -127,11 +152,14 @@ struct Fmt {
   static constexpr int kLimbWords = 3 * 4 * kPacksPerWord; // 24 or 48 uint32 per chunk
 };
 
+constexpr int kGroupWords = 48;  // digit words of one group of 64
+
 // Quantises one group of 64 values held two per lane (lane l: elements 2l, 2l+1)
-// into the format above.  `limb_bytes` addresses chunk 0 of the vector, `cs` its
-// per-chunk scalars; g is the group index.  Whole warp participates.
+// into the format above.  `limb_bytes` addresses the vector's digits (NG
+// groups), `cs` its per-chunk scalars; g is the group index.  Whole warp participates.
 template <int BITS>
-__device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, uint8_t* limb_bytes, float2* cs) {
+__device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, int NG, uint8_t* limb_bytes,
+                                                  float2* cs) {
   const int lane = threadIdx.x & 31;
   const float m = warp_max(fmaxf(fabsf(v0), fabsf(v1)));
   int e = 0;
@@ -145,6 +173,7 @@ __device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, uin
   constexpr int CPC = Fmt<BITS>::kCodesPerChunk;
   constexpr int CPW = Fmt<BITS>::kCodesPerWord;
   constexpr int PPW = Fmt<BITS>::kPacksPerWord;
+  constexpr int LW = Fmt<BITS>::kLimbWords;
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const float v = k ? v1 : v0;
@@ -154,14 +183,15 @@ __device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, uin
     const int X1 = (X - d2) >> 8;
     const int d1 = ((X1 + 128) & 255) - 128;
     const int d0 = (X1 - d1) >> 8;
-    const int p = g * (kGroup / CPC) + i / CPC;  // chunk
-    const int ii = i % CPC;
+    const int ch = i / CPC, ii = i % CPC;
     const int wi = ii / CPW, j = ii % CPW;
     const int pack = j % PPW, byte = j / PPW;
-    const int base = ((p * 3 * 4 + wi) * PPW + pack) * 4 + byte;  // limb 0
-    limb_bytes[base] = (uint8_t)(int8_t)d0;
-    limb_bytes[base + 4 * PPW * 4] = (uint8_t)(int8_t)d1;
-    limb_bytes[base + 2 * 4 * PPW * 4] = (uint8_t)(int8_t)d2;
+    const int d[3] = {d0, d1, d2};
+#pragma unroll
+    for (int L = 0; L < 3; ++L) {
+      const int w = ch * LW + (L * 4 + wi) * PPW + pack;  // word within the group
+      limb_bytes[(((w >> 2) * NG + g) * 4 + (w & 3)) * 4 + byte] = (uint8_t)(int8_t)d[L];
+    }
   }
   float s = v0 + v1;
   if (BITS == 4) {  // two chunks of 32 per group: half-warp sums
@@ -175,39 +205,154 @@ __device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, uin
   }
 }
 
-// Integer dot product of one 16-byte chunk of codes with the chunk's digits L,
-// recombined into a float S with sum_c code_c * X_c == S (up to one rounding).
+// Integer dot product of one group of 64 codes (4-bit: two chunks q0, q1;
+// 2-bit: q0 only) with the group's digits L (chunk-major, as stored), returned
+// as a float S with sum_c code_c * X_c == S up to one rounding.
 template <int BITS>
-__device__ __forceinline__ float chunk_dot(const uint4 q, const uint32_t (&L)[Fmt<BITS>::kLimbWords]) {
-  constexpr int PPW = Fmt<BITS>::kPacksPerWord;
+__device__ __forceinline__ float group_dot(const uint4 q0, const uint4 q1, const uint32_t (&L)[48]) {
   int a0 = 0, a1 = 0, a2 = 0;
-  const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+  constexpr int PPW = Fmt<BITS>::kPacksPerWord;
+  constexpr int NCH = BITS == 4 ? 2 : 1;
+  constexpr int LWC = Fmt<BITS>::kLimbWords;  // words of one chunk
 #pragma unroll
-  for (int wi = 0; wi < 4; ++wi) {
-    const uint32_t w = w4[wi];
+  for (int ch = 0; ch < NCH; ++ch) {
+    const uint4 q = ch ? q1 : q0;
+    const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int pk = 0; pk < PPW; ++pk) {
-      const uint32_t c = BITS == 4 ? ((w >> (4 * pk)) & 0x0F0F0F0Fu) : ((w >> (2 * pk)) & 0x03030303u);
-      a0 = __dp4a((int)c, (int)L[(0 * 4 + wi) * PPW + pk], a0);
-      a1 = __dp4a((int)c, (int)L[(1 * 4 + wi) * PPW + pk], a1);
-      a2 = __dp4a((int)c, (int)L[(2 * 4 + wi) * PPW + pk], a2);
+    for (int wi = 0; wi < 4; ++wi) {
+      const uint32_t w = w4[wi];
+#pragma unroll
+      for (int pk = 0; pk < PPW; ++pk) {
+        const uint32_t c = BITS == 4 ? ((w >> (4 * pk)) & 0x0F0F0F0Fu) : ((w >> (2 * pk)) & 0x03030303u);
+        a0 = __dp4a((int)c, (int)L[ch * LWC + (0 * 4 + wi) * PPW + pk], a0);
+        a1 = __dp4a((int)c, (int)L[ch * LWC + (1 * 4 + wi) * PPW + pk], a1);
+        a2 = __dp4a((int)c, (int)L[ch * LWC + (2 * 4 + wi) * PPW + pk], a2);
+      }
     }
   }
-  const int A = a0 * 256 + a1;  // |A| < 2^23: exact in fp32
+  const int A = a0 * 256 + a1;  // |A| < 2^24: exact in fp32
   return fmaf((float)A, 256.0f, (float)a2);
 }
 
-// Loads one chunk's digits (uint4 granularity) from global or shared memory.
-template <int BITS>
-__device__ __forceinline__ void load_limbs(const uint32_t* src, uint32_t (&L)[Fmt<BITS>::kLimbWords]) {
+// Loads group g's 48 digit words from a vector of NG groups (interleaved pieces).
+__device__ __forceinline__ void load_group_limbs(const uint32_t* src, int g, int NG, uint32_t (&L)[48]) {
 #pragma unroll
-  for (int i = 0; i < Fmt<BITS>::kLimbWords / 4; ++i) {
-    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+  for (int i = 0; i < 12; ++i) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i * NG + g];
     L[4 * i] = v.x;
     L[4 * i + 1] = v.y;
     L[4 * i + 2] = v.z;
     L[4 * i + 3] = v.w;
   }
+}
+
+// Order-preserving key of (logit, index): larger value first, then lower index.
+__device__ __forceinline__ unsigned long long topk_key(float v, int e) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+
+__device__ __forceinline__ float topk_key_value(unsigned long long k) {
+  uint32_t u = (uint32_t)(k >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+  return __uint_as_float(u);
+}
+
+__device__ __forceinline__ int topk_key_index(unsigned long long k) { return (int)(0xFFFFFFFFu - (uint32_t)k); }
+
+// Largest key over the warp (every lane gets it).
+__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long k) {
+  const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(k >> 32));
+  const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(k >> 32) == hi ? (uint32_t)k : 0u);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
+// One warp: the K largest logits[0..E) in descending order (ties to the lower
+// index), their renormalised softmax weights w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0),
+// and, when has_gate, sigma = sigmoid(logits[E]).  Each lane keeps its logits
+// e = lane + 32 i (NV of them, E <= 32 * NV) in registers with its best
+// remaining key; each round takes the warp maximum and only the winning lane
+// rescans.  Lane k < K returns pick k in (idx_k, w_k); every lane gets sigma.
+template <int NV>
+__device__ __forceinline__ void warp_topk_impl(const float* logits, int E, int K, int has_gate, int& idx_k,
+                                               float& w_k, float& sigma) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long key[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? topk_key(__ldcg(logits + e), e) : 0ull;
+  }
+  const float zg = has_gate ? __ldcg(logits + E) : 0.0f;
+  unsigned long long best = 0ull;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
+  float top = 0.0f, mine_v = 0.0f;
+  idx_k = 0;
+  for (int k = 0; k < K; ++k) {
+    const unsigned long long w = warp_max_key(best);
+    int e = topk_key_index(w);
+    const float v = topk_key_value(w);
+    if (e < 0 || e >= E) e = 0;  // only with non-finite logits
+    if (k == 0) top = v;
+    if (lane == k) {
+      idx_k = e;
+      mine_v = v;
+    }
+    if (best == w) {  // the winning lane drops the pick and rescans its own logits
+      best = 0ull;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        key[i] = key[i] == w ? 0ull : key[i];
+        best = key[i] > best ? key[i] : best;
+      }
+    }
+  }
+  const float ek = lane < K ? expf(mine_v - top) : 0.0f;
+  w_k = ek / warp_sum(ek);
+  sigma = has_gate ? 1.0f / (1.0f + expf(-zg)) : 0.0f;
+}
+
+// Any E: the logits stay in memory and every round rescans them.
+__device__ __forceinline__ void warp_topk_mem(const float* logits, int E, int K, int has_gate, int& idx_k, float& w_k,
+                                              float& sigma) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long prev = ~0ull;
+  float top = 0.0f, mine_v = 0.0f;
+  idx_k = 0;
+  for (int k = 0; k < K; ++k) {
+    unsigned long long best = 0ull;
+    for (int e = lane; e < E; e += 32) {
+      const unsigned long long x = topk_key(__ldcg(logits + e), e);
+      best = (x < prev && x > best) ? x : best;
+    }
+    const unsigned long long w = warp_max_key(best);
+    int e = topk_key_index(w);
+    const float v = topk_key_value(w);
+    if (e < 0 || e >= E) e = 0;
+    if (k == 0) top = v;
+    if (lane == k) {
+      idx_k = e;
+      mine_v = v;
+    }
+    prev = w;
+  }
+  const float ek = lane < K ? expf(mine_v - top) : 0.0f;
+  w_k = ek / warp_sum(ek);
+  sigma = has_gate ? 1.0f / (1.0f + expf(-__ldcg(logits + E))) : 0.0f;
+}
+
+__device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int has_gate, int& idx_k, float& w_k,
+                                          float& sigma) {
+  if (E <= 256)
+    warp_topk_impl<8>(logits, E, K, has_gate, idx_k, w_k, sigma);
+  else if (E <= 512)
+    warp_topk_impl<16>(logits, E, K, has_gate, idx_k, w_k, sigma);
+  else if (E <= 1024)
+    warp_topk_impl<32>(logits, E, K, has_gate, idx_k, w_k, sigma);
+  else
+    warp_topk_mem(logits, E, K, has_gate, idx_k, w_k, sigma);
 }
 
 // Record base pointer for one expert slot.

@@ -9,7 +9,7 @@
 
 namespace fmoe {
 
-// Router GEMV + last-CTA softmax/top-K, one grid row (blockIdx.y) per token.
+// Router GEMV: logits[t][0..E) = Wr x_t (+ bias), logits[t][E] = wsg . x_t; one grid row per token.
 struct RouterParams {
   const float* h;             // [T][H] input (normalised in-kernel when norm != 0)
   const float* gamma;         // [H] or NULL (unit)
@@ -18,43 +18,80 @@ struct RouterParams {
   const uint16_t* w_router;   // bf16 [E][H]
   const float* bias;          // [E] or NULL
   const uint16_t* w_sgate;    // bf16 [H] or NULL (no shared-gate row)
-  int T, H, E, K;
+  int T, H, E;
+  int rows_per_cta;
   uint8_t* xq_limbs;          // per-token activation digits, or NULL
   float2* xq_cs;
   long long xq_limb_stride;   // bytes per token
   long long xq_cs_stride;     // float2 per token
   float* logits;              // [T][E+1]
-  int32_t* idx;               // [T][K]
-  float* wts;                 // [T][K+1]: routing weights, slot K = shared gate sigma
-  int32_t* idx_out;           // optional [T][K]
-  float* w_out;               // optional [T][K]
-  float* probs_out;           // optional [T][E]
-  unsigned int* tickets;      // [T], zero on entry, zero on exit
+  int top_k;                  // > 0: the last CTA of each token selects the top-K (route_* outputs)
+  int32_t* route_idx;         // [T][K] selected experts
+  float* route_w;             // [T][K+1]: renormalised weights, slot K = shared-gate sigma
+  int32_t* idx_out;           // optional user copies [T][K]
+  float* w_out;
+  unsigned int* tickets;      // [T], zero between calls
   int* err;
+};
+
+// Standalone selection from logits (the router_topk entry point).
+struct TopkParams {
+  const float* logits;        // [T][E+1]
+  int T, E, K;
+  int32_t* idx;               // [T][K]
+  float* w;                   // [T][K]
+  float* probs;               // [T][E] or NULL
 };
 
 struct ExpertParams {
   BankRef routed;
   BankRef shared;
-  const int32_t* idx;         // [K] routed slots, or NULL -> fixed_expert
+  const int32_t* route_idx;   // [K] selected experts (router output) or NULL (fixed_expert)
+  const float* route_w;       // [K+1] weights, slot K = shared-gate sigma; NULL: weight 1
+  int E;
   int fixed_expert;
   int K;                      // routed slots
   int has_shared;             // slot K is the shared expert
   int H, I;
   const uint32_t* xq_limbs;   // gate/up: digits of x (chunk-major)
   const float2* xq_cs;
-  float* act;                 // [K+has_shared][I]: gate/up output, down input
-  const float* wts;           // down: per-slot weights [K+1] or NULL (all 1)
+  float* act;                 // [K+has_shared][I]: gate/up output (SwiGLU activations)
+  uint8_t* act_limbs;         // digits of act, per slot [I*bits/128 chunks][limb words] (down input)
+  float2* act_cs;             // per slot [I*bits/128] chunk scalars
+  unsigned int* grp_cnt;      // [K+has_shared][I/64] rows finished per group of 64 (zero between calls)
   const float* resid;         // down: residual [H] or NULL
   float* out;                 // down: [H]
+  int prefetch_down;          // gate/up asks L2 for the routed experts' down matrices
   int* err;
 };
 
 cudaError_t launch_rmsnorm(const float* h, const float* gamma, float eps, int T, int H, float* y, cudaStream_t s);
-cudaError_t launch_router(const RouterParams& p, int xq_bits, cudaStream_t s);
-cudaError_t launch_gateup(const ExpertParams& p, int bits, cudaStream_t s);
-cudaError_t launch_down(const ExpertParams& p, int bits, cudaStream_t s);
+cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, cudaStream_t s);
+cudaError_t launch_router(RouterParams p, int xq_bits, bool pdl, cudaStream_t s);
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+cudaError_t launch_gateup(const ExpertParams& p, int bits, bool pdl, cudaStream_t s);
+cudaError_t launch_down(const ExpertParams& p, int bits, bool pdl, cudaStream_t s);
 
 int num_sms();
+bool expert_shapes_supported(int bits, int H, int I, int num_slots);
+bool pdl_enabled();
+cudaError_t set_smem(const void* kernel, size_t bytes);
+
+// Launch with optional programmatic stream serialisation (dependent launch).
+template <typename... Exp, typename... Act>
+cudaError_t launch_pdl(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                       Act&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Act&&>(args)...);
+}
 
 }  // namespace fmoe

@@ -8,307 +8,623 @@
 // one level up, per 16-byte chunk of codes:
 //     sum_c (q_c s + b) x_c = s * sum_c q_c x_c + b * sum_c x_c,
 // with sum_c x_c precomputed once per token and sum_c q_c x_c an exact integer
-// dp4a dot product against a 3-digit fixed-point x (see fmoe_device.cuh).
+// dp4a dot product against a 3-digit fixed-point x (fmoe_device.cuh).
 //
-// Both kernels are persistent (one 512-thread CTA per SM, static contiguous
-// share of the tiles) and stream their weight tiles through a ring of shared-
-// memory stages filled by bulk copies (TMA engine) that complete on mbarriers;
-// one thread refills a stage as soon as the CTA has consumed it.
+// Both kernels run in one wave.  Each warp owns one work unit (a few rows of
+// one expert, or a few output rows of every selected expert), bulk-copies the
+// unit's codes, scales and biases into its own shared-memory slice with the
+// TMA engine, waits once on its own mbarrier, reduces across its lanes and
+// writes its outputs: no CTA-wide barrier on the hot path, and every byte of
+// the phase is requested at the start.  Weight copies that do not depend on the
+// previous kernel (the shared expert; the down matrices, whose experts are known
+// from the router) are issued before griddepcontrol.wait, so they overlap the
+// previous kernel under programmatic dependent launch.
+#include <mutex>
+
 #include "fmoe_internal.h"
 
 namespace fmoe {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kRT = 4;   // gate/up tile: 4 rows of gate and the same 4 rows of up
-constexpr int kRD = 4;   // down tile: 4 output rows of every selected expert
-constexpr int kMaxNP = 16;
+// Lane geometry over rows of NG groups of 64 codes: LPR lanes per row, RPP rows
+// side by side in a warp, GPL groups per lane.
+template <int NG>
+struct Geo {
+  static constexpr int kLanesPerRow = NG < 32 ? NG : 32;
+  static constexpr int kRowsPerPass = 32 / kLanesPerRow;
+  static constexpr int kGroupsPerLane = NG / kLanesPerRow;
+};
 
-__device__ __forceinline__ const uint8_t* slot_record(const ExpertParams& p, int slot, int* err) {
-  if (slot < p.K) {
-    int e = p.idx ? p.idx[slot] : p.fixed_expert;
-    if (e < 0 || e >= p.routed.num_experts) {
-      atomicExch(err, kDevBadIndex);
-      e = 0;
-    }
-    return p.routed.base + (long long)e * p.routed.stride;
-  }
-  return p.shared.base;
+// One group's code words from a staged row (4-bit: 32 bytes, 2-bit: 16 bytes).
+template <int BITS>
+__device__ __forceinline__ void load_group_codes(const uint8_t* row, int g, uint4& q0, uint4& q1) {
+  constexpr int GB = kGroup * BITS / 8;
+  q0 = *reinterpret_cast<const uint4*>(row + g * GB);
+  q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(row + g * GB + 16) : q0;
 }
 
+// Chunk scalars of group g: {power-of-two scale of the digits, sum of x over the group}.
 template <int BITS>
-__global__ void __launch_bounds__(kThreads, 1) gateup_kernel(const ExpertParams p, int stages, int stage_bytes) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  using F = Fmt<BITS>;
-  const int tid = threadIdx.x;
-  const int H = p.H, I = p.I;
-  const int RB = H * BITS / 8;  // code bytes per row
-  const int SB = H / kGroup * 2;  // scale (or bias) bytes per row
-  const int NC = H * BITS / 128;  // 16-byte chunks per row
-  const int NP = NC >= 32 ? NC / 32 : 1;
-  const int NE = p.K + p.has_shared;
-  const int tps = I / kRT;
-  const int ntiles = NE * tps;
-  const int t0 = (int)((long long)blockIdx.x * ntiles / gridDim.x);
-  const int mine = (int)((long long)(blockIdx.x + 1) * ntiles / gridDim.x) - t0;
-  const uint32_t cb = kRT * RB, sb = kRT * SB;
+__device__ __forceinline__ float2 group_scalars(const float2* cs, int g) {
+  if (BITS == 4) {
+    const float2 a = cs[2 * g], b = cs[2 * g + 1];
+    return make_float2(a.x, a.y + b.y);
+  }
+  return cs[g];
+}
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + (size_t)stages * stage_bytes);
-  float* red = reinterpret_cast<float*>(bars + stages);  // [2][2*kRT][kMaxNP]
-  const uint8_t** rec = reinterpret_cast<const uint8_t**>(red + 2 * 2 * kRT * kMaxNP);
+// ------------------------------------------------------------------------------------------ gate/up
+
+constexpr int kGuWarps = 8;
+constexpr int kChunkUnits = 8;  // units per staged chunk
+
+template <int BITS, int NG>
+struct GuCfg {
+  using G = Geo<NG>;
+  static constexpr int kPasses = NG >= 32 ? (BITS == 4 ? 1 : 2) : 1;
+  static constexpr int kRowPairs = G::kRowsPerPass * kPasses;  // rows of gate (and of up) per unit
+  static constexpr int kRowBytes = NG * kGroup * BITS / 8;
+  static constexpr int kScaleBytes = NG * 2;
+  static constexpr int kChunkRows = kChunkUnits * kRowPairs;
+  // chunk buffer: gate codes | up codes | gate scales | gate biases | up scales | up biases
+  static constexpr int kChunkBytes = (2 * kChunkRows * (kRowBytes + 2 * kScaleBytes) + 127) / 128 * 128;
+  static constexpr int kChunks = NG * kGroup * BITS / 128;
+  static constexpr int kDigitBytes = NG * kGroupWords * 4 + kChunks * 8;  // x digits + chunk scalars
+  static constexpr int kHead = (kDigitBytes + 127) / 128 * 128;
+  static_assert(kRowPairs * kScaleBytes % 16 == 0 && kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
+};
+
+// Persistent: CTA b owns units [b*U/G, (b+1)*U/G) (a unit = kRowPairs rows of
+// gate and up of one expert slot), cut into chunks of up to kChunkUnits units
+// of one slot.  Thread 0 stages each chunk with six large bulk copies into a
+// ring of nbuf chunk buffers; warp w computes units w, w+8, .. of the chunk.
+// A lane always works on the same groups of 64 columns, so it keeps their
+// digits of x in registers for the whole kernel.
+template <int BITS, int NG>
+__global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertParams p, int nbuf) {
+  using G = Geo<NG>;
+  using C = GuCfg<BITS, NG>;
+  constexpr int RP = C::kRowPairs, PASSES = C::kPasses;
+  constexpr int LPR = G::kLanesPerRow, RPP = G::kRowsPerPass, GPL = G::kGroupsPerLane;
+  constexpr int RB = C::kRowBytes, SB = C::kScaleBytes, CR = C::kChunkRows, CHB = C::kChunkBytes;
+  constexpr int LW = Fmt<BITS>::kLimbWords;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t s_bar[8];
+  __shared__ __align__(8) uint64_t s_bar_x;
+  __shared__ int s_idx[32];
+  __shared__ int s_done[kGuWarps * 32];
   __shared__ int s_abort;
 
-  if (tid < NE) rec[tid] = slot_record(p, tid, p.err);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int I = p.I, NE = p.K + p.has_shared;
+  const int ups = I / RP, U = NE * ups;
+  const int u0 = (int)((long long)blockIdx.x * U / gridDim.x);
+  const int u1 = (int)((long long)(blockIdx.x + 1) * U / gridDim.x);
+  const uint32_t* xs = reinterpret_cast<const uint32_t*>(sm);
+  const float2* xcs = reinterpret_cast<const float2*>(sm + NG * kGroupWords * 4);
+
   if (tid == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&s_bar[b]), 1);
+    mbar_init(smem_addr(&s_bar_x), 1);
     mbar_fence_init();
     s_abort = 0;
   }
   __syncthreads();
 
-  const uint64_t pol_r = l2_policy_evict_first(), pol_s = l2_policy_evict_last();
-  auto issue = [&](int j) {
-    const int tile = t0 + j, slot = tile / tps, r0 = (tile % tps) * kRT;
-    const uint8_t* r = rec[slot];
-    const uint64_t pol = slot < p.K ? pol_r : pol_s;
-    const long long* off = slot < p.K ? p.routed.off : p.shared.off;
-    const int st = j % stages;
-    const uint32_t dst = smem_addr(sm + (size_t)st * stage_bytes), bar = smem_addr(&bars[st]);
+  // Chunk c covers units [cu, ce): up to kChunkUnits units, never across a slot boundary.
+  auto chunk_end = [&](int cu) { return min(min(cu + kChunkUnits, u1), (cu / ups + 1) * ups); };
+  auto issue = [&](int c, int cu, int ce) {  // thread 0
+    const int sl = cu / ups, r0 = (cu % ups) * RP, rows = (ce - cu) * RP;
+    const bool routed = sl < p.K;
+    const uint8_t* rec = routed ? p.routed.base + (long long)s_idx[sl] * p.routed.stride : p.shared.base;
+    const long long* off = routed ? p.routed.off : p.shared.off;
+    const uint64_t pol = routed ? l2_policy_evict_first() : l2_policy_evict_last();
+    uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
+    const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_bar[c % nbuf]);
+    const uint32_t cb = rows * RB, sb = rows * SB;
     mbar_expect_tx(bar, 2 * cb + 4 * sb);
-    bulk_g2s(dst, r + off[0] + (long long)r0 * RB, cb, bar, pol);
-    bulk_g2s(dst + cb, r + off[3] + (long long)r0 * RB, cb, bar, pol);
-    bulk_g2s(dst + 2 * cb, r + off[1] + (long long)r0 * SB, sb, bar, pol);
-    bulk_g2s(dst + 2 * cb + sb, r + off[2] + (long long)r0 * SB, sb, bar, pol);
-    bulk_g2s(dst + 2 * cb + 2 * sb, r + off[4] + (long long)r0 * SB, sb, bar, pol);
-    bulk_g2s(dst + 2 * cb + 3 * sb, r + off[5] + (long long)r0 * SB, sb, bar, pol);
+    bulk_g2s(dst, rec + off[0] + (long long)r0 * RB, cb, bar, pol);
+    bulk_g2s(dst + CR * RB, rec + off[3] + (long long)r0 * RB, cb, bar, pol);
+    bulk_g2s(dst + 2 * CR * RB, rec + off[1] + (long long)r0 * SB, sb, bar, pol);
+    bulk_g2s(dst + 2 * CR * RB + CR * SB, rec + off[2] + (long long)r0 * SB, sb, bar, pol);
+    bulk_g2s(dst + 2 * CR * RB + 2 * CR * SB, rec + off[4] + (long long)r0 * SB, sb, bar, pol);
+    bulk_g2s(dst + 2 * CR * RB + 3 * CR * SB, rec + off[5] + (long long)r0 * SB, sb, bar, pol);
   };
+
+  // Shared-expert chunks need nothing from the router: request them first.
+  if (tid == 0) {
+    int cu = u0;
+    for (int c = 0; c < nbuf && cu < u1; ++c) {
+      const int ce = chunk_end(cu);
+      if (cu / ups >= p.K) issue(c, cu, ce);
+      cu = ce;
+    }
+  }
+
+  pdl_wait();  // the router's logits, routing and x digits are complete
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane < p.K) {
+      int e = p.route_idx ? p.route_idx[lane] : p.fixed_expert;
+      if (e < 0 || e >= p.routed.num_experts) {
+        atomicExch(p.err, kDevBadIndex);
+        e = 0;
+      }
+      s_idx[lane] = e;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t bx = smem_addr(&s_bar_x);
+      mbar_expect_tx(bx, C::kDigitBytes);
+      bulk_g2s(smem_addr(sm), p.xq_limbs, NG * kGroupWords * 4, bx, l2_policy_evict_last());
+      bulk_g2s(smem_addr(sm + NG * kGroupWords * 4), p.xq_cs, C::kChunks * 8, bx, l2_policy_evict_last());
+      int cu = u0;
+      for (int c = 0; c < nbuf && cu < u1; ++c) {
+        const int ce = chunk_end(cu);
+        if (cu / ups < p.K) issue(c, cu, ce);
+        cu = ce;
+      }
+      if (p.prefetch_down && u0 / ups < p.K) {
+        // Warm L2 with this CTA's slice of each routed expert's down matrix.
+        const long long len[3] = {(long long)p.H * (I * BITS / 8), (long long)p.H * (I / kGroup) * 2,
+                                  (long long)p.H * (I / kGroup) * 2};
+        for (int k = 0; k < p.K; ++k) {
+          const uint8_t* rec = p.routed.base + (long long)s_idx[k] * p.routed.stride;
+          for (int m = 0; m < 3; ++m) {
+            const long long a0 = (len[m] * blockIdx.x / gridDim.x) & ~15LL;
+            const long long a1 = (len[m] * (blockIdx.x + 1) / gridDim.x) & ~15LL;
+            if (a1 > a0) prefetch_l2(rec + p.routed.off[6 + m] + a0, (uint32_t)(a1 - a0));
+          }
+        }
+      }
+    }
+  }
+
+  // This lane's groups and their digits of x, for the whole kernel.
+  const int sub = lane / LPR, gl = lane % LPR;
+  uint32_t L[GPL][48];
+  float2 cs[GPL];
+  bool ok = mbar_wait_bounded(smem_addr(&s_bar_x), 0, p.err);
+#pragma unroll
+  for (int j = 0; j < GPL; ++j) {
+    const int g = gl + LPR * j;
+    load_group_limbs(xs, g, NG, L[j]);
+    cs[j] = group_scalars<BITS>(xcs, g);
+  }
+
+  int cu = u0;
+  for (int c = 0; cu < u1; ++c) {
+    const int ce = chunk_end(cu);
+    const int sl = cu / ups, rbase = (cu % ups) * RP;
+    if (!mbar_wait_bounded(smem_addr(&s_bar[c % nbuf]), (uint32_t)((c / nbuf) & 1), p.err)) ok = false;
+    const uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
+    for (int k = warp; ok && k < ce - cu; k += kGuWarps) {
+      float accg[PASSES], accu[PASSES];
+#pragma unroll
+      for (int i = 0; i < PASSES; ++i) accg[i] = accu[i] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < GPL; ++j) {
+        const int g = gl + LPR * j;
+#pragma unroll
+        for (int i = 0; i < PASSES; ++i) {
+          const int r = k * RP + sub + RPP * i;  // row within the chunk
+          uint4 q0, q1, v0, v1;
+          load_group_codes<BITS>(buf + r * RB, g, q0, q1);
+          load_group_codes<BITS>(buf + CR * RB + r * RB, g, v0, v1);
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * CR * RB + r * SB);
+          const float gs = bf16_to_f32(sc[g]);
+          const float gb = bf16_to_f32(sc[CR * SB / 2 + g]);
+          const float us = bf16_to_f32(sc[CR * SB + g]);
+          const float ub = bf16_to_f32(sc[3 * CR * SB / 2 + g]);
+          const float Sg = group_dot<BITS>(q0, q1, L[j]);
+          const float Su = group_dot<BITS>(v0, v1, L[j]);
+          accg[i] = fmaf(gs, cs[j].x * Sg, fmaf(gb, cs[j].y, accg[i]));
+          accu[i] = fmaf(us, cs[j].x * Su, fmaf(ub, cs[j].y, accu[i]));
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < PASSES; ++i) {
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) {
+          accg[i] += __shfl_xor_sync(0xffffffffu, accg[i], o);
+          accu[i] += __shfl_xor_sync(0xffffffffu, accu[i], o);
+        }
+      }
+      if (gl == 0) {
+#pragma unroll
+        for (int i = 0; i < PASSES; ++i) {
+          const float g = accg[i], uu = accu[i];
+          p.act[(size_t)sl * I + rbase + k * RP + sub + RPP * i] = g / (1.0f + expf(-g)) * uu;
+        }
+      }
+    }
+    __syncthreads();  // every warp is done with this chunk buffer
+    if (!ok) s_abort = 1;
+    if (tid == 0) {  // refill the buffer with chunk c + nbuf
+      int nu = ce, nc = c + 1;
+      while (nc < c + nbuf && nu < u1) {
+        nu = chunk_end(nu);
+        ++nc;
+      }
+      if (nu < u1 && !s_abort) {
+        fence_proxy_async();
+        issue(c + nbuf, nu, chunk_end(nu));
+      }
+    }
+    cu = ce;
+  }
+
+  // Groups of 64 activations: the CTA that completes a group writes its digits
+  // for the down kernel (release: fence before the count; acquire: fence after).
+  __threadfence();
+  __syncthreads();
+  if (s_abort) {  // let copies still in flight land before the CTA exits
+    if (tid == 0)
+      for (int b = 0; b < nbuf; ++b) mbar_wait_bounded(smem_addr(&s_bar[b]), 0, p.err);
+    return;
+  }
+  const int g0 = u0 * RP / kGroup, ng = (u1 * RP - 1) / kGroup - g0 + 1;  // groups over concatenated slot rows
+  if (tid < ng) {
+    const int g = g0 + tid;
+    const int lo = max(u0 * RP, g * kGroup), hi = min(u1 * RP, (g + 1) * kGroup);
+    const unsigned prev = atomicAdd(&p.grp_cnt[g], (unsigned)(hi - lo));
+    s_done[tid] = prev + (unsigned)(hi - lo) == (unsigned)kGroup;
+  }
+  __syncthreads();
+  for (int t = warp; t < ng; t += kGuWarps) {
+    if (!s_done[t]) continue;
+    __threadfence();
+    const int g = g0 + t, slot = g * kGroup / I, gg = (g * kGroup % I) / kGroup;
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)g * kGroup) + lane);
+    const int ncd = I * BITS / 128;
+    xq_quantize_group<BITS>(v.x, v.y, gg, I / kGroup, p.act_limbs + (size_t)slot * ncd * LW * 4,
+                            p.act_cs + (size_t)slot * ncd);
+    if (lane == 0) p.grp_cnt[g] = 0u;
+  }
+}
+
+// ------------------------------------------------------------------------------------------ down + combine
+
+constexpr int kDnWarps = 8;
+
+template <int BITS, int NG>
+struct DnCfg {
+  static constexpr int kRowBytes = NG * kGroup * BITS / 8;
+  static constexpr int kScaleBytes = NG * 2;
+  // output rows per unit: 2, or more when a row's scales are too short for a 16-byte copy
+  static constexpr int kRows = kScaleBytes >= 8 ? 2 : 16 / kScaleBytes;
+  static constexpr int kChunks = NG * kGroup * BITS / 128;
+  static_assert(kRows * kScaleBytes % 16 == 0 && kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
+};
+
+// Persistent: CTA b owns units [b*U/G, (b+1)*U/G) of kRows output rows,
+// staged in chunks of up to `chunk_units` units: for every selected expert the
+// chunk's rows of its down matrix (codes, scales, biases: three bulk copies).
+// The experts are known from the router, so the first chunks are requested
+// before waiting on the gate/up kernel.  Lane l owns the (slot, group) pairs
+// q = l, l+32, .. (PPL of them) of every row and keeps their digits in
+// registers; the warp sums a row's pairs by shuffles.
+template <int BITS, int NG, int PPL>
+__global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertParams p, int chunk_units, int nbuf) {
+  using C = DnCfg<BITS, NG>;
+  constexpr int RD = C::kRows;
+  constexpr int RB = C::kRowBytes, SB = C::kScaleBytes;
+  constexpr int NCH = C::kChunks;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t s_bar[8];
+  __shared__ __align__(8) uint64_t s_bar_x;
+  __shared__ const uint8_t* s_src[33][3];
+  __shared__ float s_w[33];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NE = p.K + p.has_shared, NP = NE * NG;
+  const int U = p.H / RD;
+  const int u0 = (int)((long long)blockIdx.x * U / gridDim.x);
+  const int u1 = (int)((long long)(blockIdx.x + 1) * U / gridDim.x);
+  const int dwords = NE * NG * kGroupWords;  // digits of every slot's activations
+  const uint32_t* xs = reinterpret_cast<const uint32_t*>(sm);
+  const float2* xcs = reinterpret_cast<const float2*>(sm + (size_t)dwords * 4);
+  const int head = (dwords * 4 + NE * NCH * 8 + 127) / 128 * 128;
+  const int crows = chunk_units * RD;
+  const int slot_bytes = crows * (RB + 2 * SB);  // one expert's rows of a chunk
+  const int chb = (NE * slot_bytes + 127) / 128 * 128;
+
+  // Routing: the router has completed (the gate/up kernel signals this launch
+  // only after its own wait), so the experts and weights can be read now.
+  if (warp == 0) {
+    if (lane < p.K) {
+      int ik = p.route_idx ? p.route_idx[lane] : p.fixed_expert;
+      if (ik < 0 || ik >= p.routed.num_experts) {
+        atomicExch(p.err, kDevBadIndex);
+        ik = 0;
+      }
+      const uint8_t* rec = p.routed.base + (long long)ik * p.routed.stride;
+      s_src[lane][0] = rec + p.routed.off[6];
+      s_src[lane][1] = rec + p.routed.off[7];
+      s_src[lane][2] = rec + p.routed.off[8];
+      s_w[lane] = p.route_w ? p.route_w[lane] : 1.0f;
+    }
+    if (lane == 0 && p.has_shared) {
+      s_src[p.K][0] = p.shared.base + p.shared.off[6];
+      s_src[p.K][1] = p.shared.base + p.shared.off[7];
+      s_src[p.K][2] = p.shared.base + p.shared.off[8];
+      s_w[p.K] = p.route_w ? p.route_w[p.K] : 1.0f;
+    }
+    if (lane == 0) {
+      for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&s_bar[b]), 1);
+      mbar_init(smem_addr(&s_bar_x), 1);
+      mbar_fence_init();
+    }
+  }
+  __syncthreads();
+
+  auto issue = [&](int c) {  // chunk c: units [u0 + c*chunk_units, ..) of every slot, thread 0
+    const int cu = u0 + c * chunk_units, ce = min(cu + chunk_units, u1);
+    const long long j0 = (long long)cu * RD;
+    const uint32_t rows = (uint32_t)(ce - cu) * RD;
+    uint8_t* buf = sm + head + (size_t)(c % nbuf) * chb;
+    const uint32_t bar = smem_addr(&s_bar[c % nbuf]);
+    const uint64_t pol_r = l2_policy_evict_first(), pol_s = l2_policy_evict_last();
+    mbar_expect_tx(bar, (uint32_t)NE * rows * (RB + 2 * SB));
+    for (int s = 0; s < NE; ++s) {
+      const uint64_t pol = s < p.K ? pol_r : pol_s;
+      const uint32_t d = smem_addr(buf + (size_t)s * slot_bytes);
+      bulk_g2s(d, s_src[s][0] + j0 * RB, rows * RB, bar, pol);
+      bulk_g2s(d + crows * RB, s_src[s][1] + j0 * SB, rows * SB, bar, pol);
+      bulk_g2s(d + crows * RB + crows * SB, s_src[s][2] + j0 * SB, rows * SB, bar, pol);
+    }
+  };
+  const int nchunk = (u1 - u0 + chunk_units - 1) / chunk_units;
   if (tid == 0)
-    for (int j = 0; j < stages && j < mine; ++j) issue(j);
+    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c);
 
-  // This thread's chunk of every row and its digits of x.
-  const int pc = tid % NC, rs = tid / NC, RS = kThreads / NC;
-  uint32_t L[F::kLimbWords];
-  load_limbs<BITS>(p.xq_limbs + (size_t)pc * F::kLimbWords, L);
-  const float2 cs = p.xq_cs[pc];
-  const int grp = pc * F::kCodesPerChunk / kGroup;
-  const int nsub = (2 * kRT + RS - 1) / RS;  // streams per thread (uniform)
+  pdl_wait();  // the activations' digits are complete
+  pdl_trigger();
+  if (tid == 0) {  // every slot's digits, once per CTA
+    const uint32_t bx = smem_addr(&s_bar_x);
+    mbar_expect_tx(bx, (uint32_t)(dwords * 4 + NE * NCH * 8));
+    bulk_g2s(smem_addr(sm), p.act_limbs, (uint32_t)dwords * 4, bx, l2_policy_evict_first());
+    bulk_g2s(smem_addr(sm + (size_t)dwords * 4), p.act_cs, (uint32_t)(NE * NCH * 8), bx, l2_policy_evict_first());
+  }
 
-  int j = 0;
-  for (; j < mine; ++j) {
-    const int st = j % stages;
-    if (!mbar_wait_bounded(smem_addr(&bars[st]), (uint32_t)((j / stages) & 1), p.err)) s_abort = 1;
-    const uint8_t* sbuf = sm + (size_t)st * stage_bytes;
-    float* rb = red + (j & 1) * (2 * kRT * kMaxNP);
-    for (int k = 0; k < nsub; ++k) {
-      const int s = rs + k * RS;
-      const bool valid = s < 2 * kRT;
-      float part = 0.0f;
-      if (valid) {
-        const int m = s & 1, r = s >> 1;
-        const uint4 q = *reinterpret_cast<const uint4*>(sbuf + m * cb + r * RB + 16 * pc);
-        const float S = chunk_dot<BITS>(q, L);
-        const uint8_t* sc = sbuf + 2 * cb + 2 * m * sb + r * SB;
-        const float sf = bf16_to_f32(reinterpret_cast<const uint16_t*>(sc)[grp]);
-        const float bf = bf16_to_f32(reinterpret_cast<const uint16_t*>(sc + sb)[grp]);
-        part = fmaf(sf, cs.x * S, bf * cs.y);
+  // This lane's (slot, group) pairs and their digits.
+  uint32_t L[PPL][48];
+  float2 cs[PPL];
+  float wq[PPL];
+  int qoff[PPL], qg[PPL];
+  bool ok = mbar_wait_bounded(smem_addr(&s_bar_x), 0, p.err);
+#pragma unroll
+  for (int m = 0; m < PPL; ++m) {
+    const int q = lane + 32 * m;
+    const bool has = q < NP;
+    const int s = has ? q / NG : 0, g = has ? q % NG : 0;
+    load_group_limbs(xs + (size_t)s * NG * kGroupWords, g, NG, L[m]);
+    cs[m] = group_scalars<BITS>(xcs + s * NCH, g);
+    wq[m] = has ? s_w[s] : 0.0f;
+    qoff[m] = s * slot_bytes;
+    qg[m] = g;
+  }
+
+  for (int c = 0; c < nchunk; ++c) {
+    const int cu = u0 + c * chunk_units, ce = min(cu + chunk_units, u1);
+    if (!mbar_wait_bounded(smem_addr(&s_bar[c % nbuf]), (uint32_t)((c / nbuf) & 1), p.err)) ok = false;
+    const uint8_t* buf = sm + head + (size_t)(c % nbuf) * chb;
+    for (int k = warp; ok && k < ce - cu; k += kDnWarps) {
+      float acc[RD];
+#pragma unroll
+      for (int r = 0; r < RD; ++r) acc[r] = 0.0f;
+#pragma unroll
+      for (int m = 0; m < PPL; ++m) {
+        const uint8_t* sb = buf + qoff[m];
+#pragma unroll
+        for (int r = 0; r < RD; ++r) {
+          const int row = k * RD + r;  // row within the chunk
+          uint4 q0, q1;
+          load_group_codes<BITS>(sb + row * RB, qg[m], q0, q1);
+          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + crows * RB + row * SB)[qg[m]]);
+          const float bi =
+              bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + crows * RB + crows * SB + row * SB)[qg[m]]);
+          const float S = group_dot<BITS>(q0, q1, L[m]);
+          acc[r] = fmaf(wq[m], fmaf(sc, cs[m].x * S, bi * cs[m].y), acc[r]);
+        }
       }
-      for (int o = (NC >= 32 ? 16 : NC / 2); o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (valid && (pc & 31) == 0) rb[s * kMaxNP + (pc >> 5)] = part;
+#pragma unroll
+      for (int r = 0; r < RD; ++r) acc[r] = warp_sum(acc[r]);
+#pragma unroll
+      for (int r = 0; r < RD; ++r)
+        if (lane == r) {
+          const int row = (cu + k) * RD + r;
+          p.out[row] = (p.resid ? p.resid[row] : 0.0f) + acc[r];
+        }
     }
-    __syncthreads();
-    if (s_abort) break;
-    if (tid == 0 && j + stages < mine) issue(j + stages);
-    if (tid < kRT) {
-      const int tile = t0 + j, slot = tile / tps, row = (tile % tps) * kRT + tid;
-      float g = 0.0f, u = 0.0f;
-      for (int n = 0; n < NP; ++n) {
-        g += rb[(2 * tid) * kMaxNP + n];
-        u += rb[(2 * tid + 1) * kMaxNP + n];
-      }
-      p.act[(size_t)slot * I + row] = g / (1.0f + expf(-g)) * u;
+    __syncthreads();  // every warp is done with this chunk buffer
+    if (tid == 0 && c + nbuf < nchunk && ok) {
+      fence_proxy_async();
+      issue(c + nbuf);
     }
   }
-  if (s_abort && tid == 0) {  // let copies already in flight land before the CTA exits
-    for (int k = j; k < mine && k < j + stages; ++k)
-      mbar_wait_bounded(smem_addr(&bars[k % stages]), (uint32_t)((k / stages) & 1), p.err);
+  if (!ok && tid == 0)
+    for (int b = 0; b < nbuf; ++b) mbar_wait_bounded(smem_addr(&s_bar[b]), 0, p.err);
+}
+
+size_t round128(size_t v) { return (v + 127) / 128 * 128; }
+
+constexpr size_t kSmemBudget = 220 * 1024;
+
+template <int BITS, int NG>
+cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
+  using C = GuCfg<BITS, NG>;
+  const int NE = p.K + p.has_shared;
+  const int units = NE * (p.I / C::kRowPairs);
+  int grid = num_sms();
+  grid = grid > units ? units : grid;
+  // each CTA counts at most one block of threads' worth of activation groups
+  if ((long long)(units + grid - 1) / grid * C::kRowPairs / kGroup + 2 > kGuWarps * 32) return cudaErrorInvalidValue;
+  const int per_cta = (units + grid - 1) / grid;
+  int nbuf = (int)((kSmemBudget - C::kHead) / C::kChunkBytes);
+  const int need = (per_cta + kChunkUnits - 1) / kChunkUnits + 1;  // +1: a chunk may stop at a slot boundary
+  nbuf = nbuf > need ? need : nbuf;
+  nbuf = nbuf > 8 ? 8 : nbuf;
+  if (nbuf < 1) return cudaErrorInvalidValue;
+  const size_t smem = C::kHead + (size_t)nbuf * C::kChunkBytes;
+  void (*k)(const ExpertParams, int) = gateup_kernel<BITS, NG>;
+  cudaError_t e = set_smem((const void*)k, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(grid), dim3(kGuWarps * 32), smem, s, pdl, p, nbuf);
+}
+
+// Down-kernel staging: (chunk units, buffers, shared bytes) for NE slots, or false.
+template <int BITS, int NG>
+bool down_plan(int H, int NE, int& chunk_units, int& nbuf, size_t& smem) {
+  using C = DnCfg<BITS, NG>;
+  const int units = H / C::kRows;
+  int grid = num_sms();
+  grid = grid > units ? units : grid;
+  const int per_cta = (units + grid - 1) / grid;
+  const size_t head = round128((size_t)NE * NG * kGroupWords * 4 + (size_t)NE * C::kChunks * 8);
+  const size_t unit_bytes = (size_t)NE * C::kRows * (C::kRowBytes + 2 * C::kScaleBytes);
+  if (head + 2 * round128(unit_bytes) > kSmemBudget) return false;
+  // the whole share in one buffer when it fits, otherwise a ring of two
+  if (head + round128(per_cta * unit_bytes) <= kSmemBudget) {
+    chunk_units = per_cta;
+    nbuf = 1;
+  } else {
+    chunk_units = (int)((kSmemBudget - head) / 2 / unit_bytes);
+    nbuf = 2;
   }
+  smem = head + (size_t)nbuf * round128((size_t)chunk_units * unit_bytes);
+  return true;
+}
+
+template <int BITS, int NG>
+cudaError_t down_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
+  using C = DnCfg<BITS, NG>;
+  const int NE = p.K + p.has_shared;
+  int cu = 0, nbuf = 0;
+  size_t smem = 0;
+  const int ppl = (NE * NG + 31) / 32;
+  if (!down_plan<BITS, NG>(p.H, NE, cu, nbuf, smem) || ppl > 4) return cudaErrorInvalidValue;
+  const int units = p.H / C::kRows;
+  int grid = num_sms();
+  grid = grid > units ? units : grid;
+  void (*k)(const ExpertParams, int, int) = ppl == 1 ? down_kernel<BITS, NG, 1>
+                                          : ppl == 2 ? down_kernel<BITS, NG, 2>
+                                          : ppl == 3 ? down_kernel<BITS, NG, 3>
+                                                     : down_kernel<BITS, NG, 4>;
+  cudaError_t e = set_smem((const void*)k, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(grid), dim3(kDnWarps * 32), smem, s, pdl, p, cu, nbuf);
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kThreads, 1) down_kernel(const ExpertParams p, int stages, int stage_bytes) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  using F = Fmt<BITS>;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I;
-  const int RB = I * BITS / 8, SB = I / kGroup * 2, NC = I * BITS / 128;
-  const int NP = NC >= 32 ? NC / 32 : 1;
-  const int NE = p.K + p.has_shared;
-  const int sub = kRD * (RB + 2 * SB);  // bytes of one slot inside a stage
-  const int ntiles = H / kRD;
-  const int t0 = (int)((long long)blockIdx.x * ntiles / gridDim.x);
-  const int mine = (int)((long long)(blockIdx.x + 1) * ntiles / gridDim.x) - t0;
-
-  // [stages][digits NE*NC*LW u32][scalars NE*NC float2][red 2*kRD*NE*NP f32][bars][record pointers]
-  uint8_t* xl = sm + (size_t)stages * stage_bytes;
-  float2* xc = reinterpret_cast<float2*>(xl + (size_t)NE * NC * F::kLimbWords * 4);
-  float* red = reinterpret_cast<float*>(xc + NE * NC);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * kRD * NE * NP);
-  const uint8_t** rec = reinterpret_cast<const uint8_t**>(bars + stages);
-  __shared__ int s_abort;
-
-  if (tid < NE) rec[tid] = slot_record(p, tid, p.err);
-  if (tid == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
-    mbar_fence_init();
-    s_abort = 0;
+cudaError_t gateup_bits(const ExpertParams& p, bool pdl, cudaStream_t s) {
+  switch (p.H / kGroup) {
+    case 2: return gateup_dispatch<BITS, 2>(p, pdl, s);
+    case 4: return gateup_dispatch<BITS, 4>(p, pdl, s);
+    case 8: return gateup_dispatch<BITS, 8>(p, pdl, s);
+    case 16: return gateup_dispatch<BITS, 16>(p, pdl, s);
+    case 32: return gateup_dispatch<BITS, 32>(p, pdl, s);
+    case 64: return gateup_dispatch<BITS, 64>(p, pdl, s);
+    case 128: return gateup_dispatch<BITS, 128>(p, pdl, s);
   }
-  __syncthreads();
-
-  const uint64_t pol_r = l2_policy_evict_first(), pol_s = l2_policy_evict_last();
-  auto issue = [&](int j) {
-    const int r0 = (t0 + j) * kRD;
-    const int st = j % stages;
-    const uint32_t dst = smem_addr(sm + (size_t)st * stage_bytes), bar = smem_addr(&bars[st]);
-    mbar_expect_tx(bar, (uint32_t)(NE * sub));
-    for (int s = 0; s < NE; ++s) {
-      const uint8_t* r = rec[s];
-      const long long* off = s < p.K ? p.routed.off : p.shared.off;
-      const uint64_t pol = s < p.K ? pol_r : pol_s;
-      const uint32_t d = dst + s * sub;
-      bulk_g2s(d, r + off[6] + (long long)r0 * RB, kRD * RB, bar, pol);
-      bulk_g2s(d + kRD * RB, r + off[7] + (long long)r0 * SB, kRD * SB, bar, pol);
-      bulk_g2s(d + kRD * RB + kRD * SB, r + off[8] + (long long)r0 * SB, kRD * SB, bar, pol);
-    }
-  };
-  if (tid == 0)
-    for (int j = 0; j < stages && j < mine; ++j) issue(j);
-
-  // Digits of every slot's activation vector (all CTAs, while the first stages land).
-  for (int g = warp; g < NE * (I / kGroup); g += kThreads / 32) {
-    const int slot = g / (I / kGroup), gg = g % (I / kGroup);
-    const float2 v = reinterpret_cast<const float2*>(p.act + (size_t)slot * I + gg * kGroup)[lane];
-    xq_quantize_group<BITS>(v.x, v.y, gg, xl + (size_t)slot * NC * F::kLimbWords * 4, xc + slot * NC);
-  }
-  __syncthreads();
-
-  const int pc = tid % NC, q = tid / NC, s = q % NE, rg = q / NE;
-  const int RGN = (kThreads / NC) / NE;
-  const bool active = rg < RGN;
-  uint32_t L[F::kLimbWords];
-  float2 cs = make_float2(0.0f, 0.0f);
-  float wsl = 0.0f;
-  if (active) {
-    load_limbs<BITS>(reinterpret_cast<const uint32_t*>(xl) + ((size_t)s * NC + pc) * F::kLimbWords, L);
-    cs = xc[s * NC + pc];
-    wsl = p.wts ? p.wts[s] : 1.0f;
-  } else {
-#pragma unroll
-    for (int i = 0; i < F::kLimbWords; ++i) L[i] = 0u;
-  }
-  const int grp = pc * F::kCodesPerChunk / kGroup;
-  const int nsub = (kRD + RGN - 1) / RGN;
-
-  int j = 0;
-  for (; j < mine; ++j) {
-    const int st = j % stages;
-    if (!mbar_wait_bounded(smem_addr(&bars[st]), (uint32_t)((j / stages) & 1), p.err)) s_abort = 1;
-    const uint8_t* sbuf = sm + (size_t)st * stage_bytes + s * sub;
-    float* rb = red + (j & 1) * (kRD * NE * NP);
-    for (int k = 0; k < nsub; ++k) {
-      const int r = rg + k * RGN;
-      const bool valid = active && r < kRD;
-      float part = 0.0f;
-      if (valid) {
-        const uint4 qv = *reinterpret_cast<const uint4*>(sbuf + r * RB + 16 * pc);
-        const float S = chunk_dot<BITS>(qv, L);
-        const float sf = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbuf + kRD * RB + r * SB)[grp]);
-        const float bf = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbuf + kRD * RB + kRD * SB + r * SB)[grp]);
-        part = wsl * fmaf(sf, cs.x * S, bf * cs.y);
-      }
-      for (int o = (NC >= 32 ? 16 : NC / 2); o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (valid && (pc & 31) == 0) rb[r * NE * NP + s * NP + (pc >> 5)] = part;
-    }
-    __syncthreads();
-    if (s_abort) break;
-    if (tid == 0 && j + stages < mine) issue(j + stages);
-    if (tid < kRD) {
-      const int row = (t0 + j) * kRD + tid;
-      float acc = p.resid ? p.resid[row] : 0.0f;
-      for (int n = 0; n < NE * NP; ++n) acc += rb[tid * NE * NP + n];
-      p.out[row] = acc;
-    }
-  }
-  if (s_abort && tid == 0) {
-    for (int k = j; k < mine && k < j + stages; ++k)
-      mbar_wait_bounded(smem_addr(&bars[k % stages]), (uint32_t)((k / stages) & 1), p.err);
-  }
+  return cudaErrorInvalidValue;
 }
 
-constexpr size_t kSmemBudget = 200 * 1024;
-
-size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-// Raises a kernel's dynamic shared-memory limit once per device (and again only
-// if a larger size is asked for), so that captured launches make no attribute call.
-template <typename Kern>
-cudaError_t set_smem(Kern k, size_t bytes) {
-  static size_t done[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
-  return e;
+template <int BITS>
+cudaError_t down_bits(const ExpertParams& p, bool pdl, cudaStream_t s) {
+  switch (p.I / kGroup) {
+    case 2: return down_dispatch<BITS, 2>(p, pdl, s);
+    case 4: return down_dispatch<BITS, 4>(p, pdl, s);
+    case 8: return down_dispatch<BITS, 8>(p, pdl, s);
+    case 16: return down_dispatch<BITS, 16>(p, pdl, s);
+    case 32: return down_dispatch<BITS, 32>(p, pdl, s);
+    case 64: return down_dispatch<BITS, 64>(p, pdl, s);
+    case 128: return down_dispatch<BITS, 128>(p, pdl, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_gateup(const ExpertParams& p, int bits, cudaStream_t s) {
-  const int NE = p.K + p.has_shared;
-  const size_t stage = round_up((size_t)2 * kRT * (p.H * bits / 8) + (size_t)4 * kRT * (p.H / kGroup * 2), 128);
-  const size_t extra = 8 * 8 + sizeof(float) * 2 * 2 * kRT * kMaxNP + sizeof(void*) * (NE + 1) + 128;
-  int stages = (int)((kSmemBudget - extra) / stage);
-  stages = stages > 8 ? 8 : stages;
-  if (stages < 2) return cudaErrorInvalidValue;
-  const size_t bytes = stages * stage + extra;
-  const int ntiles = NE * (p.I / kRT);
-  int grid = num_sms();
-  grid = grid > ntiles ? ntiles : grid;
-  cudaError_t e;
-  if (bits == 4) {
-    if ((e = set_smem(gateup_kernel<4>, bytes)) != cudaSuccess) return e;
-    gateup_kernel<4><<<grid, kThreads, bytes, s>>>(p, stages, (int)stage);
-  } else {
-    if ((e = set_smem(gateup_kernel<2>, bytes)) != cudaSuccess) return e;
-    gateup_kernel<2><<<grid, kThreads, bytes, s>>>(p, stages, (int)stage);
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
+// again only if a larger size is asked for, so that launches captured into a
+// CUDA graph make no attribute call.
+cudaError_t set_smem(const void* kernel, size_t bytes) {
+  struct Entry {
+    const void* fn;
+    size_t bytes[64];
+  };
+  static Entry table[96] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (bytes <= 32 * 1024) return cudaSuccess;  // below the default limit even with static shared memory
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* slot = nullptr;
+  for (Entry& t : table) {
+    if (t.fn == kernel || t.fn == nullptr) {
+      slot = &t;
+      break;
+    }
   }
-  return cudaGetLastError();
+  if (slot && slot->fn == kernel && dev >= 0 && dev < 64 && slot->bytes[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && slot && dev >= 0 && dev < 64) {
+    slot->fn = kernel;
+    slot->bytes[dev] = bytes;
+  }
+  return e;
 }
 
-cudaError_t launch_down(const ExpertParams& p, int bits, cudaStream_t s) {
-  const int NE = p.K + p.has_shared;
-  const int NC = p.I * bits / 128, NP = NC >= 32 ? NC / 32 : 1;
-  const size_t sub = (size_t)kRD * (p.I * bits / 8 + 2 * (p.I / kGroup * 2));
-  const size_t stage = round_up(NE * sub, 128);
-  const size_t extra = 8 * 8 + (size_t)NE * NC * (3 * 4 * (8 / bits)) * 4 + (size_t)NE * NC * 8 +
-                       sizeof(float) * (2 * kRD * NE * NP + 2) + sizeof(void*) * (NE + 1) + 128;
-  int stages = (int)((kSmemBudget - extra) / stage);
-  stages = stages > 8 ? 8 : stages;
-  if (stages < 2) return cudaErrorInvalidValue;
-  const size_t bytes = stages * stage + extra;
-  const int ntiles = p.H / kRD;
-  int grid = num_sms();
-  grid = grid > ntiles ? ntiles : grid;
-  cudaError_t e;
-  if (bits == 4) {
-    if ((e = set_smem(down_kernel<4>, bytes)) != cudaSuccess) return e;
-    down_kernel<4><<<grid, kThreads, bytes, s>>>(p, stages, (int)stage);
-  } else {
-    if ((e = set_smem(down_kernel<2>, bytes)) != cudaSuccess) return e;
-    down_kernel<2><<<grid, kThreads, bytes, s>>>(p, stages, (int)stage);
+namespace {
+template <int BITS, int NGU, int NGD>
+bool fits(int ne) {
+  int cu, nb;
+  size_t sm;
+  return GuCfg<BITS, NGU>::kHead + GuCfg<BITS, NGU>::kChunkBytes <= kSmemBudget &&
+         down_plan<BITS, NGD>(1 << 20, ne, cu, nb, sm) && ne * NGD <= 4 * 32;
+}
+template <int BITS, int NGU>
+bool fits_d(int ngd, int ne) {
+  switch (ngd) {
+    case 2: return fits<BITS, NGU, 2>(ne);
+    case 4: return fits<BITS, NGU, 4>(ne);
+    case 8: return fits<BITS, NGU, 8>(ne);
+    case 16: return fits<BITS, NGU, 16>(ne);
+    case 32: return fits<BITS, NGU, 32>(ne);
+    case 64: return fits<BITS, NGU, 64>(ne);
+    case 128: return fits<BITS, NGU, 128>(ne);
   }
-  return cudaGetLastError();
+  return false;
+}
+template <int BITS>
+bool fits_u(int ngu, int ngd, int ne) {
+  switch (ngu) {
+    case 2: return fits_d<BITS, 2>(ngd, ne);
+    case 4: return fits_d<BITS, 4>(ngd, ne);
+    case 8: return fits_d<BITS, 8>(ngd, ne);
+    case 16: return fits_d<BITS, 16>(ngd, ne);
+    case 32: return fits_d<BITS, 32>(ngd, ne);
+    case 64: return fits_d<BITS, 64>(ngd, ne);
+    case 128: return fits_d<BITS, 128>(ngd, ne);
+  }
+  return false;
+}
+}  // namespace
+
+bool expert_shapes_supported(int bits, int H, int I, int ne) {
+  if (H % kGroup || I % kGroup) return false;
+  return bits == 4 ? fits_u<4>(H / kGroup, I / kGroup, ne) : fits_u<2>(H / kGroup, I / kGroup, ne);
+}
+
+cudaError_t launch_gateup(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {
+  return bits == 4 ? gateup_bits<4>(p, pdl, s) : gateup_bits<2>(p, pdl, s);
+}
+
+cudaError_t launch_down(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {
+  return bits == 4 ? down_bits<4>(p, pdl, s) : down_bits<2>(p, pdl, s);
 }
 
 }  // namespace fmoe

@@ -1,10 +1,12 @@
-// k_router.cu -- RMSNorm, activation digits, and the router GEMV with softmax / top-K.
+// k_router.cu -- RMSNorm, activation digits, the router GEMV and the standalone top-K.
 //
 // RMSNorm follows "What is Flash-MoE" (a2a-mcp.org), section 3: two passes,
 // sum of squares then apply.  Routing follows the "Flash-MoE" wiki summary
-// (jeongsk), per-layer pipeline: routing projection, softmax, top-K -- except
-// that the selection runs on the GPU in the last CTA to finish its rows, so no
-// host round trip sits between the router and the experts.
+// (jeongsk), per-layer pipeline: routing projection, then softmax and top-K.
+// The pages run the selection on the CPU; here the router kernel only writes
+// the logits and every expert kernel takes the top-K from them itself
+// (warp_topk), so no host round trip and no grid-wide handshake sits between
+// the router and the experts.
 #include "fmoe_internal.h"
 
 namespace fmoe {
@@ -44,36 +46,50 @@ __global__ void __launch_bounds__(256) xq_kernel(const float* __restrict__ x, in
   const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (g >= H / kGroup) return;  // warp-uniform
   const float2 v = reinterpret_cast<const float2*>(x + g * kGroup)[threadIdx.x & 31];
-  xq_quantize_group<BITS>(v.x, v.y, g, limbs, cs);
+  xq_quantize_group<BITS>(v.x, v.y, g, H / kGroup, limbs, cs);
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint4 ldg_nc(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// grid (NB, T).  Each CTA: x = RMSNorm(h_t) in shared memory; its share of the
-// activation digits; rows [b*rpc, b*rpc + rpc) of [Wr; wsg] as 8 warp tasks
-// (rows x segments).  The last CTA of token t (ticket) selects the top-K.
+// grid (NB, T).  Before waiting on the predecessor, each CTA bulk-copies its
+// rows [b*rpc, b*rpc + rpc) of [Wr; wsg] into shared memory (weights only).
+// Then x = RMSNorm(h_t) in shared memory, at most one group of the activation
+// digits per warp spread over the grid, and its logits as 8 warp tasks (rows x
+// segments).  When top_k > 0 the last CTA of the token (atomic ticket) selects
+// the experts once for every later kernel.
 template <int XQB>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterParams p) {
-  extern __shared__ __align__(16) float smem[];
+  extern __shared__ __align__(128) uint8_t sm[];
   __shared__ float s_red[8];
   __shared__ float s_part[8];
   __shared__ int s_last;
-  __shared__ int s_sel_idx[32];
-  __shared__ float s_sel_val[32];
+  __shared__ __align__(8) uint64_t s_bar;
   const int t = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, E = p.E, K = p.K;
-  float* xs = smem;
-  const float* h = p.h + (size_t)t * H;
+  const int H = p.H, E = p.E;
+  const int R = E + (p.w_sgate ? 1 : 0);
+  const int rpc = p.rows_per_cta;
+  const int r0 = blockIdx.x * rpc;
+  const int nrows = min(rpc, R - r0);
+  uint16_t* wrows = reinterpret_cast<uint16_t*>(sm);
+  float* xs = reinterpret_cast<float*>(sm + (size_t)rpc * H * 2);
+  const uint32_t bar = smem_addr(&s_bar);
 
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+    if (nrows > 0) {
+      const int nr = min(nrows, E - r0 > 0 ? E - r0 : 0);  // routed rows in range
+      const bool gate_row = p.w_sgate && r0 + nrows > E;
+      mbar_expect_tx(bar, (uint32_t)nrows * H * 2);
+      if (nr > 0) bulk_g2s(smem_addr(wrows), p.w_router + (size_t)r0 * H, (uint32_t)nr * H * 2, bar, l2_policy_evict_last());
+      if (gate_row) bulk_g2s(smem_addr(wrows + (size_t)nr * H), p.w_sgate, (uint32_t)H * 2, bar, l2_policy_evict_last());
+    }
+  }
+  pdl_wait();
+  pdl_trigger();
+
+  const float* h = p.h + (size_t)t * H;
   float ss = 0.0f;
   for (int i = tid * 4; i < H; i += kRouterThreads * 4) {
     const float4 v = *reinterpret_cast<const float4*>(h + i);
@@ -90,29 +106,25 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
   }
   __syncthreads();
 
-  if (XQB != 0 && p.xq_limbs != nullptr) {
-    for (int g = blockIdx.x * 8 + warp; g < H / kGroup; g += gridDim.x * 8) {
+  if (XQB != 0 && p.xq_limbs != nullptr) {  // group g by warp g / NB of CTA g % NB
+    for (int g = blockIdx.x + gridDim.x * warp; g < H / kGroup; g += gridDim.x * 8) {
       const float2 v = reinterpret_cast<const float2*>(xs + g * kGroup)[lane];
-      xq_quantize_group<XQB == 0 ? 4 : XQB>(v.x, v.y, g, p.xq_limbs + t * p.xq_limb_stride,
+      xq_quantize_group<XQB == 0 ? 4 : XQB>(v.x, v.y, g, H / kGroup, p.xq_limbs + t * p.xq_limb_stride,
                                             p.xq_cs + t * p.xq_cs_stride);
     }
   }
 
-  const int R = E + (p.w_sgate ? 1 : 0);
-  const int rpc = (R + gridDim.x - 1) / gridDim.x;
-  const int r0 = blockIdx.x * rpc;
-  const int nrows = min(rpc, R - r0);
-  const int S = rpc >= 8 ? 1 : 8 / rpc;  // segments per row: 8, 4, 2 or 1
-  if (nrows > 0 && warp < nrows * S) {
-    const int row = r0 + warp / S, seg = warp % S;
-    const uint16_t* wrow = row < E ? p.w_router + (size_t)row * H : p.w_sgate;
+  const int S = rpc >= 8 ? 1 : (rpc >= 4 ? 2 : (rpc >= 2 ? 4 : 8));  // segments per row
+  const bool ready = nrows > 0 && mbar_wait_bounded(bar, 0, p.err);
+  if (ready && warp < nrows * S) {
+    const int rl = warp / S, seg = warp % S;
     const int seglen = H / S;
-    const uint4* wv = reinterpret_cast<const uint4*>(wrow + seg * seglen);
+    const uint4* wv = reinterpret_cast<const uint4*>(wrows + (size_t)rl * H + seg * seglen);
     const float* xv = xs + seg * seglen;
     float acc = 0.0f;
 #pragma unroll 4
     for (int k = lane; k < seglen / 8; k += 32) {
-      const uint4 w = ldg_nc(wv + k);
+      const uint4 w = wv[k];
       const float4 xa = *reinterpret_cast<const float4*>(xv + 8 * k);
       const float4 xb = *reinterpret_cast<const float4*>(xv + 8 * k + 4);
       acc = fmaf(bf_lo(w.x), xa.x, acc);
@@ -129,73 +141,56 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
   }
   __syncthreads();
   float* logits = p.logits + (size_t)t * (E + 1);
-  if (tid < nrows) {
+  if (ready && tid < nrows) {
     float l = 0.0f;
     for (int s = 0; s < S; ++s) l += s_part[tid * S + s];
     const int row = r0 + tid;
     if (row < E && p.bias) l += p.bias[row];
     logits[row] = l;
   }
+  if (p.top_k <= 0) return;
 
-  // ---- last CTA of this token selects
+  // ---- the last CTA of this token selects the experts
+  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(&p.tickets[t], 1u);
-    s_last = prev == gridDim.x - 1;
-  }
+  if (tid == 0) s_last = atomicAdd(&p.tickets[t], 1u) == gridDim.x - 1;
   __syncthreads();
   if (!s_last || warp != 0) return;
   __threadfence();
-  float* sl = xs;  // x is no longer needed; smem holds max(H, E) floats
-  for (int e = lane; e < E; e += 32) sl[e] = __ldcg(logits + e);
-  __syncwarp();
-  for (int k = 0; k < K; ++k) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      const float v = sl[e];
-      if (v > bv || (v == bv && e < bi)) {
-        bv = v;
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi >= E) bi = 0;  // only reachable with non-finite logits
-    if (lane == 0) {
-      s_sel_idx[k] = bi;
-      s_sel_val[k] = bv;
-    }
-    if ((bi & 31) == lane) sl[bi] = -INFINITY;
-    __syncwarp();
-  }
-  const float m = s_sel_val[0];
-  const float ek = lane < K ? expf(s_sel_val[lane] - m) : 0.0f;
-  const float esum = warp_sum(ek);
+  const int K = p.top_k;
+  int ik;
+  float wk, sig;
+  warp_topk(logits, E, K, p.w_sgate != nullptr, ik, wk, sig);
   if (lane < K) {
-    const float wk = ek / esum;
-    const int ik = s_sel_idx[lane];
-    p.idx[t * K + lane] = ik;
-    p.wts[t * (K + 1) + lane] = wk;
-    if (p.idx_out) p.idx_out[t * K + lane] = ik;
-    if (p.w_out) p.w_out[t * K + lane] = wk;
+    p.route_idx[(size_t)t * K + lane] = ik;
+    p.route_w[(size_t)t * (K + 1) + lane] = wk;
+    if (p.idx_out) p.idx_out[(size_t)t * K + lane] = ik;
+    if (p.w_out) p.w_out[(size_t)t * K + lane] = wk;
   }
-  if (lane == 0) p.wts[t * (K + 1) + K] = p.w_sgate ? 1.0f / (1.0f + expf(-__ldcg(logits + E))) : 0.0f;
-  if (p.probs_out) {
+  if (lane == 0) {
+    p.route_w[(size_t)t * (K + 1) + K] = sig;
+    p.tickets[t] = 0u;
+  }
+}
+
+// One warp per token: top-K, renormalised weights and (optionally) full softmax.
+__global__ void __launch_bounds__(32) topk_kernel(const TopkParams p) {
+  const int t = blockIdx.x, lane = threadIdx.x;
+  const float* l = p.logits + (size_t)t * (p.E + 1);
+  int ik;
+  float wk, sig;
+  warp_topk(l, p.E, p.K, 0, ik, wk, sig);
+  if (lane < p.K) {
+    p.idx[(size_t)t * p.K + lane] = ik;
+    p.w[(size_t)t * p.K + lane] = wk;
+  }
+  if (p.probs) {
+    const float m = __shfl_sync(0xffffffffu, __ldcg(l + ik), 0);  // the largest logit
     float z = 0.0f;
-    for (int e = lane; e < E; e += 32) z += expf(__ldcg(logits + e) - m);
+    for (int e = lane; e < p.E; e += 32) z += expf(__ldcg(l + e) - m);
     z = warp_sum(z);
-    for (int e = lane; e < E; e += 32) p.probs_out[(size_t)t * E + e] = expf(__ldcg(logits + e) - m) / z;
+    for (int e = lane; e < p.E; e += 32) p.probs[(size_t)t * p.E + e] = expf(__ldcg(l + e) - m) / z;
   }
-  if (lane == 0) p.tickets[t] = 0u;
 }
 
 }  // namespace
@@ -215,19 +210,23 @@ cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* c
   return cudaGetLastError();
 }
 
-cudaError_t launch_router(const RouterParams& p, int xq_bits, cudaStream_t s) {
+cudaError_t launch_router(RouterParams p, int xq_bits, bool pdl, cudaStream_t s) {
   const int R = p.E + (p.w_sgate ? 1 : 0);
+  int rmax = 98304 / (2 * p.H);
+  rmax = rmax < 1 ? 1 : (rmax > 8 ? 8 : rmax);
   int nb = num_sms();
   if (nb > R) nb = R;
-  if ((R + nb - 1) / nb > 8 && nb < (R + 7) / 8) nb = (R + 7) / 8;
-  const size_t smem = sizeof(float) * (size_t)(p.H > p.E ? p.H : p.E);
-  dim3 grid(nb, p.T);
-  if (xq_bits == 4)
-    router_kernel<4><<<grid, kRouterThreads, smem, s>>>(p);
-  else if (xq_bits == 2)
-    router_kernel<2><<<grid, kRouterThreads, smem, s>>>(p);
-  else
-    router_kernel<0><<<grid, kRouterThreads, smem, s>>>(p);
+  if ((R + nb - 1) / nb > rmax) nb = (R + rmax - 1) / rmax;
+  p.rows_per_cta = (R + nb - 1) / nb;
+  const size_t smem = (size_t)p.rows_per_cta * p.H * 2 + (size_t)p.H * 4;
+  cudaError_t e;
+  void (*k)(RouterParams) = xq_bits == 4 ? router_kernel<4> : (xq_bits == 2 ? router_kernel<2> : router_kernel<0>);
+  if ((e = set_smem((const void*)k, smem)) != cudaSuccess) return e;
+  return launch_pdl(k, dim3(nb, p.T), dim3(kRouterThreads), smem, s, pdl, p);
+}
+
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
+  topk_kernel<<<p.T, 32, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -127,8 +127,8 @@ size_t fmoe_router_topk_workspace_size(int T, int E);
  * bank: the expert bank; expert: record index in [0, num_experts).
  * x: fp32 [H]; y: fp32 [H].  ws: fmoe_expert_ffn_workspace_size(bank) bytes,
  * 256-byte aligned, zeroed once (fmoe_workspace_init).
- * Requirements: bits 2 or 4, group 64, H % 128 == 0, I % 128 == 0,
- * H*bits/128 and I*bits/128 powers of two no larger than 512. */
+ * Requirements: bits 2 or 4, group 64, H and I each 64 times a power of two,
+ * 128 <= H, I <= 8192. */
 fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, float* y, void* ws, size_t ws_bytes,
                             fmoe_stream_t stream);
 size_t fmoe_expert_ffn_workspace_size(const fmoe_bank* bank);
@@ -144,7 +144,9 @@ size_t fmoe_expert_ffn_workspace_size(const fmoe_bank* bank);
  * once before first use (fmoe_workspace_init); calls on one workspace must be
  * ordered on one stream.  Requirements: those of fmoe_expert_ffn for both
  * banks (same bits, hidden, inter), 1 <= K <= min(E, 32), E <= 4096,
- * (K+1) * I*bits/128 <= 512.  T = 0 enqueues nothing. */
+ * hidden <= 8192, and K + 1 expert slots of the down kernel within its shared
+ * memory (K <= 9 at inter 1024, 4-bit; FMOE_ERR_UNSUPPORTED otherwise).
+ * T = 0 enqueues nothing. */
 fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
                            float* topk_w, void* ws, size_t ws_bytes, fmoe_stream_t stream);
 size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);

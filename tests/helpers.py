@@ -53,14 +53,25 @@ def dense_from_record(rec, spec_bits, hidden, inter, group=64):
     return out
 
 
-def max_rel_err(got, ref, floor=1e-2):
-    """max_i |g_i - r_i| / max(|r_i|, floor * rms(r)) over the last axis, maximised over rows."""
+def max_rel_err(got, ref, floor=1e-2, slack=None):
+    """max_i (|g_i - r_i| - slack_i)+ / max(|r_i|, floor * rms(r)) over the last axis, maximised over rows.
+
+    `slack` is an absolute allowance per element (default 0), used when `got` was
+    recovered from a stored fp32 value: out - h cannot be closer than one fp32 ulp of out."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
     den = np.maximum(np.abs(ref), floor * rms)
     den = np.where(den > 0, den, 1.0)
-    return float(np.max(np.abs(got - ref) / den)) if got.size else 0.0
+    diff = np.abs(got - ref)
+    if slack is not None:
+        diff = np.maximum(diff - np.asarray(slack, dtype=np.float64), 0.0)
+    return float(np.max(diff / den)) if got.size else 0.0
+
+
+def ulp32(a):
+    """One fp32 ulp of each element."""
+    return np.spacing(np.abs(np.asarray(a, dtype=np.float32))).astype(np.float64)
 
 
 def oracle_layer(hl, top_k=None, gamma=True):
