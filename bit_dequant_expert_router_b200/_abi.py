@@ -49,6 +49,7 @@ SIGNATURES = [
     ("fmoe_expert_ffn_workspace_size", _sz, [ctypes.POINTER(FmoeBank)]),
     ("fmoe_moe_layer", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("fmoe_moe_layer_workspace_size", _sz, [ctypes.POINTER(FmoeLayer), _i]),
+    ("fmoe_moe_layer_static", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _vp]),
     ("fmoe_moe_stack", _i, [ctypes.POINTER(FmoeLayer), _i, _vp, _i, _vp, _vp, _sz, _vp]),
     ("fmoe_trace_next_layer", _i, [ctypes.POINTER(ctypes.c_void_p), _i]),
     ("fmoe_workspace_init", _i, [_vp, _sz, _vp]),
@@ -212,6 +213,17 @@ def moe_layer(layer, h, out=None, topk_idx=None, topk_w=None, ws=None, stream=No
                                 _ptr(out, torch.float32, "out"), _ptr(topk_idx, torch.int32, "topk_idx"),
                                 _ptr(topk_w, torch.float32, "topk_w"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
                                 _stream(stream)))
+    return out
+
+
+def moe_layer_static(layer, h, out=None, topk_idx=None, topk_w=None, dev_err=None, stream=None):
+    """fmoe_moe_layer on the library's static scratch (no workspace argument)."""
+    T = h.shape[0] if h.dim() == 2 else 1
+    out = torch.empty_like(h) if out is None else out
+    _check(lib().fmoe_moe_layer_static(ctypes.byref(layer.s), _ptr(h, torch.float32, "h"), T,
+                                       _ptr(out, torch.float32, "out"), _ptr(topk_idx, torch.int32, "topk_idx"),
+                                       _ptr(topk_w, torch.float32, "topk_w"), _ptr(dev_err, torch.int32, "dev_err"),
+                                       _stream(stream)))
     return out
 
 

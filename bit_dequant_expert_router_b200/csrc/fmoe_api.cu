@@ -325,8 +325,9 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
 }
 
 // One token through the block: router (+RMSNorm, digits, top-K) -> gate/up -> down + combine.
+// err_word: where the kernels report a failed bounded wait; NULL means the workspace's own error word.
 static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
-                               uint8_t* base, const WsLayout& L, cudaStream_t s) {
+                               uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word = nullptr) {
   const fmoe_bank& r = layer->routed;
   const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
@@ -352,7 +353,7 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   rp.idx_out = idx_out;
   rp.w_out = w_out;
   rp.tickets = ctrl->tickets;
-  rp.err = &ctrl->err;
+  rp.err = err_word ? err_word : &ctrl->err;
   const bool trace = g_trace_on;
   g_trace_on = false;
   const bool pdl = pdl_enabled() && !trace;
@@ -381,7 +382,7 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   p.resid = h;
   p.out = out;
   p.prefetch_down = prefetch_down();
-  p.err = &ctrl->err;
+  p.err = rp.err;
   if ((e = launch_gateup(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
   if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   if ((e = launch_down(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "down launch");
@@ -404,6 +405,62 @@ fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float
   for (int t = 0; t < T; ++t) {
     st = layer_token(layer, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
                      topk_w ? topk_w + (size_t)t * K : nullptr, base, L, cs(stream));
+    if (st != FMOE_OK) return st;
+  }
+  return FMOE_OK;
+}
+
+// ---- fmoe_moe_layer_static: the same block with library-owned scratch.
+//
+// For callers that cannot hand over a workspace: a plain-C or FFI host that
+// keeps no device allocator of its own, or an engine whose memory planner has
+// already reserved every byte of the device and cannot grow.  The scratch is a
+// fixed file-scope device array, so the call allocates nothing.  Static device
+// memory starts zeroed when the module loads, which is the state the ticket and
+// group counters need; every call returns them to zero.
+
+constexpr size_t kStaticScratchBytes = FMOE_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device, looked up once per device.
+static fmoe_status static_scratch(uint8_t** out) {
+  static std::mutex mu;
+  static uint8_t* cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cache[dev]) {
+    *out = cache[dev];
+    return FMOE_OK;
+  }
+  void* p = nullptr;
+  if ((e = cudaGetSymbolAddress(&p, g_static_scratch)) != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+  if (dev >= 0 && dev < 64) cache[dev] = static_cast<uint8_t*>(p);
+  *out = static_cast<uint8_t*>(p);
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
+                                  float* topk_w, int* dev_err, fmoe_stream_t stream) {
+  fmoe_status st = check_layer(layer);
+  if (st != FMOE_OK) return st;
+  if (T < 0) return fail(FMOE_ERR_INVALID_ARG, "T %d", T);
+  if (T == 0) return FMOE_OK;
+  if (!h || !out) return fail(FMOE_ERR_INVALID_ARG, "h or out is NULL");
+  if (!aligned16(h) || !aligned16(out)) return fail(FMOE_ERR_ALIGNMENT, "h and out must be 16-byte aligned");
+  if (dev_err && ((uintptr_t)dev_err & 3u) != 0) return fail(FMOE_ERR_ALIGNMENT, "dev_err must be 4-byte aligned");
+  const int H = layer->routed.hidden, K = layer->top_k;
+  const WsLayout L = layout(H, layer->routed.num_experts, K, layer->routed.inter, 1);
+  if (L.total > kStaticScratchBytes)
+    return fail(FMOE_ERR_WORKSPACE,
+                "layer needs %zu bytes of scratch, the static scratch holds %zu (use fmoe_moe_layer with a workspace)",
+                L.total, kStaticScratchBytes);
+  uint8_t* base = nullptr;
+  if ((st = static_scratch(&base)) != FMOE_OK) return st;
+  for (int t = 0; t < T; ++t) {
+    st = layer_token(layer, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
+                     topk_w ? topk_w + (size_t)t * K : nullptr, base, L, cs(stream), dev_err);
     if (st != FMOE_OK) return st;
   }
   return FMOE_OK;

@@ -151,6 +151,38 @@ fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float
                            float* topk_w, void* ws, size_t ws_bytes, fmoe_stream_t stream);
 size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
 
+/* Bytes of the library's static scratch used by fmoe_moe_layer_static. */
+#define FMOE_STATIC_SCRATCH_BYTES 131072
+
+/* fmoe_moe_layer without a workspace argument: the pages have no counterpart
+ * (their engine owns all its buffers); this is an interface convenience.
+ * Computes exactly what fmoe_moe_layer computes, with the same kernels, but its
+ * scratch is a fixed device array inside libfmoe.so of FMOE_STATIC_SCRATCH_BYTES
+ * (128 KiB) per device, so the call allocates nothing.  It serves callers that
+ * cannot hand over a workspace: a plain-C or FFI host that keeps no device
+ * allocator, or an engine whose memory planner has reserved the whole device.
+ * Arguments as fmoe_moe_layer, plus:
+ *   dev_err: device int (caller-owned, 4-byte aligned) that the kernels set
+ *            non-zero when a bounded wait gives up or an expert index lies
+ *            outside the bank; it must start at zero and is never cleared by
+ *            the library.  NULL: such failures are recorded only inside the
+ *            static scratch, where no call reports them.
+ * The scratch needs no set-up: it is zero when the library's module loads on
+ * a device, and every call leaves its counters at zero again.  Its address is
+ * looked up (cudaGetSymbolAddress) on the first call on each device; make that
+ * first call outside any CUDA stream capture.
+ * One scratch per device is shared by every caller of this function: two calls
+ * on the same device whose kernels may overlap (different streams without an
+ * ordering between them, or different host threads) race on it and give wrong
+ * results.  Order all calls on a device on one stream.
+ * A layer whose scratch (fmoe_moe_layer_workspace_size(layer, T)) exceeds
+ * FMOE_STATIC_SCRATCH_BYTES is rejected with FMOE_ERR_WORKSPACE before
+ * anything is enqueued.  Every shape the other requirements admit needs at
+ * most 108,032 bytes (the Qwen3.5-397B-A17B layer 58,112), so today that
+ * check only guards against shapes later versions may admit. */
+fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
+                                  float* topk_w, int* dev_err, fmoe_stream_t stream);
+
 /* A stack of L layers applied in order, each block's output feeding the next
  * (the 60-layer decode loop of the jeongsk wiki summary, without the attention
  * layers): h_0 = h, h_{l+1} = block_l(h_l), out = h_L.  out may equal h.
