@@ -390,6 +390,105 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   return FMOE_OK;
 }
 
+// The single-kernel path (k_fused.cu) unless FMOE_FUSED=0 is set in the environment.
+static bool fused_enabled() {
+  const char* v = getenv("FMOE_FUSED");
+  return !(v && v[0] == '0');
+}
+
+static bool same_offsets(const fmoe_bank& a, const fmoe_bank& b) {
+  for (int i = 0; i < 9; ++i)
+    if (a.off[i] != b.off[i]) return false;
+  return true;
+}
+
+// Runs layers[0..nl) over T tokens as one launch of the single-kernel path, if
+// that path takes these shapes; `taken` tells whether it did.
+static fmoe_status run_fused(const fmoe_layer* layers, int nl, const float* h, int T, float* out, int32_t* idx_out,
+                             float* w_out, uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word,
+                             bool& taken) {
+  taken = false;
+  if (!fused_enabled() || nl < 1 || nl > kFusedMaxLayers) return FMOE_OK;
+  const fmoe_bank& r0 = layers[0].routed;
+  for (int l = 0; l < nl; ++l) {
+    const fmoe_layer& y = layers[l];
+    if (y.routed.bits != r0.bits || y.routed.hidden != r0.hidden || y.routed.inter != r0.inter ||
+        y.routed.num_experts != r0.num_experts || y.top_k != layers[0].top_k || !same_offsets(y.routed, r0) ||
+        !same_offsets(y.shared, r0))
+      return FMOE_OK;
+  }
+  const int H = r0.hidden, I = r0.inter, E = r0.num_experts, K = layers[0].top_k;
+  const FusedPlan pl = plan_fused(r0.bits, H, I, E, K);
+  if (!pl.ok) return FMOE_OK;
+  WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
+  FusedParams p{};
+  for (int l = 0; l < nl; ++l) {
+    const fmoe_layer& y = layers[l];
+    FusedLayer& f = p.layers[l];
+    f.routed = static_cast<const uint8_t*>(y.routed.base);
+    f.stride = y.routed.stride;
+    f.shared = static_cast<const uint8_t*>(y.shared.base);
+    f.w_router = y.w_router;
+    f.bias = y.router_bias;
+    f.w_sgate = y.w_shared_gate;
+    f.gamma = y.gamma;
+    f.eps = y.eps;
+  }
+  for (int i = 0; i < 9; ++i) p.off[i] = r0.off[i];
+  p.L = nl;
+  p.T = T;
+  p.H = H;
+  p.I = I;
+  p.E = E;
+  p.K = K;
+  p.h = h;
+  p.out = out;
+  p.idx_out = idx_out;
+  p.w_out = w_out;
+  p.logits = reinterpret_cast<float*>(base + L.logits);
+  p.act = reinterpret_cast<float*>(base + L.act);
+  p.act_limbs = base + L.act_limbs;
+  p.act_cs = reinterpret_cast<float2*>(base + L.act_cs);
+  p.grp_cnt = reinterpret_cast<unsigned*>(base + L.grp_cnt);
+  p.bar_cnt = &ctrl->grid_count;
+  p.bar_gen = &ctrl->grid_gen;
+  p.err = err_word ? err_word : &ctrl->err;
+  p.nbuf = pl.nbuf;
+  p.chb = pl.chb;
+  p.cu = pl.cu;
+  p.rt_rows = pl.rt_rows;
+  p.ru = pl.ru;
+  p.rd = pl.rd;
+  p.dn_rows_max = pl.dn_rows_max;
+  p.dn_slot_bytes = pl.dn_slot_bytes;
+  p.dn_off = pl.dn_off;
+  p.ring_off = pl.ring_off;
+  const bool trace = g_trace_on;
+  g_trace_on = false;
+  cudaError_t e;
+  if (trace && (e = trace_record(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if ((e = launch_fused(p, pl, r0.bits, pdl_enabled() && !trace, s)) != cudaSuccess) return cuda_fail(e, "fused launch");
+  for (int i = 1; trace && i < 4; ++i)
+    if ((e = trace_record(g_trace[i], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  taken = true;
+  return FMOE_OK;
+}
+
+// The block for T tokens of one layer on a checked workspace.
+static fmoe_status moe_layer_impl(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
+                                  float* topk_w, uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word) {
+  bool taken = false;
+  fmoe_status st = run_fused(layer, 1, h, T, out, topk_idx, topk_w, base, L, s, err_word, taken);
+  if (st != FMOE_OK || taken) return st;
+  const int H = layer->routed.hidden, K = layer->top_k;
+  for (int t = 0; t < T; ++t) {
+    st = layer_token(layer, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
+                     topk_w ? topk_w + (size_t)t * K : nullptr, base, L, s, err_word);
+    if (st != FMOE_OK) return st;
+  }
+  return FMOE_OK;
+}
+
 fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
                            float* topk_w, void* ws, size_t ws_bytes, fmoe_stream_t stream) {
   fmoe_status st = check_layer(layer);
@@ -401,13 +500,7 @@ fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float
   const int H = layer->routed.hidden, K = layer->top_k;
   const WsLayout L = layout(H, layer->routed.num_experts, K, layer->routed.inter, 1);
   if ((st = check_ws(ws, ws_bytes, L.total)) != FMOE_OK) return st;
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  for (int t = 0; t < T; ++t) {
-    st = layer_token(layer, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
-                     topk_w ? topk_w + (size_t)t * K : nullptr, base, L, cs(stream));
-    if (st != FMOE_OK) return st;
-  }
-  return FMOE_OK;
+  return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, static_cast<uint8_t*>(ws), L, cs(stream), nullptr);
 }
 
 // ---- fmoe_moe_layer_static: the same block with library-owned scratch.
@@ -458,12 +551,7 @@ fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T
                 L.total, kStaticScratchBytes);
   uint8_t* base = nullptr;
   if ((st = static_scratch(&base)) != FMOE_OK) return st;
-  for (int t = 0; t < T; ++t) {
-    st = layer_token(layer, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
-                     topk_w ? topk_w + (size_t)t * K : nullptr, base, L, cs(stream), dev_err);
-    if (st != FMOE_OK) return st;
-  }
-  return FMOE_OK;
+  return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, base, L, cs(stream), dev_err);
 }
 
 fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int nl, const float* h, int T, float* out, void* ws,
@@ -475,9 +563,34 @@ fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int nl, const float* h, int
     if (layers[l].routed.hidden != layers[0].routed.hidden)
       return fail(FMOE_ERR_INVALID_ARG, "layer %d: hidden differs from layer 0", l);
   }
+  if (T < 0) return fail(FMOE_ERR_INVALID_ARG, "T %d", T);
+  if (T == 0) return FMOE_OK;
+  if (!h || !out) return fail(FMOE_ERR_INVALID_ARG, "h or out is NULL");
+  if (!aligned16(h) || !aligned16(out)) return fail(FMOE_ERR_ALIGNMENT, "h and out must be 16-byte aligned");
+  // one launch per run of up to kFusedMaxLayers layers when the single-kernel path takes them
+  size_t need = 0;
   for (int l = 0; l < nl; ++l) {
-    fmoe_status st = fmoe_moe_layer(&layers[l], l == 0 ? h : out, T, out, nullptr, nullptr, ws, ws_bytes, stream);
+    const WsLayout Ll = layout(layers[l].routed.hidden, layers[l].routed.num_experts, layers[l].top_k,
+                               layers[l].routed.inter, 1);
+    need = Ll.total > need ? Ll.total : need;
+  }
+  fmoe_status st = check_ws(ws, ws_bytes, need);
+  if (st != FMOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  for (int l0 = 0; l0 < nl;) {
+    const int n = nl - l0 < kFusedMaxLayers ? nl - l0 : kFusedMaxLayers;
+    const WsLayout Ll = layout(layers[l0].routed.hidden, layers[l0].routed.num_experts, layers[l0].top_k,
+                               layers[l0].routed.inter, 1);
+    bool taken = false;
+    st = run_fused(&layers[l0], n, l0 == 0 ? h : out, T, out, nullptr, nullptr, base, Ll, cs(stream), nullptr, taken);
     if (st != FMOE_OK) return st;
+    if (taken) {
+      l0 += n;
+      continue;
+    }
+    st = fmoe_moe_layer(&layers[l0], l0 == 0 ? h : out, T, out, nullptr, nullptr, ws, ws_bytes, stream);
+    if (st != FMOE_OK) return st;
+    ++l0;
   }
   return FMOE_OK;
 }

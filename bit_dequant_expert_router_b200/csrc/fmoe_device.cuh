@@ -16,7 +16,11 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // bound on any device-si
 
 // Control words at the start of every workspace.
 struct WsControl {
-  unsigned int tickets[1024];  // last-CTA tickets, one per token
+  unsigned int tickets[960];   // last-CTA tickets, one per token
+  unsigned int grid_count;     // grid barrier of the single-kernel path: arrivals ...
+  unsigned int pad0[31];
+  unsigned int grid_gen;       // ... and generation (its own 128-byte line)
+  unsigned int pad1[31];
   int err;                     // nonzero once a bounded wait gave up
   int pad[63];
 };
@@ -67,6 +71,11 @@ __device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier
 
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Plain arrival (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -202,6 +211,71 @@ __device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, int
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) cs[g] = make_float2(csc, s);
+  }
+}
+
+// Same format, one block of 16 consecutive elements per lane: block `part`
+// (0..3) of group g, the four blocks of a group on lanes 4k..4k+3 of the warp.
+// Every lane of the warp calls it (shuffles); lanes with active == false take
+// part in the reductions with zeros and store nothing.  Bytes written are those
+// of xq_quantize_group; the chunk sums may differ in rounding order.
+template <int BITS>
+__device__ __forceinline__ void xq_quantize_block16(const float (&v)[16], int g, int part, int NG, uint8_t* limb_bytes,
+                                                   float2* cs, bool active) {
+  float m = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  int ex = 0;
+  if (m > 0.0f) {
+    const int ef = (int)((__float_as_uint(m) >> 23) & 0xFFu);
+    ex = ef == 0 ? -125 : ef - 126;  // m < 2^ex
+  }
+  ex = ex < -100 ? -100 : (ex > 100 ? 100 : ex);
+  const float inv = __uint_as_float((uint32_t)(127 + 22 - ex) << 23);
+  const float csc = __uint_as_float((uint32_t)(127 + ex - 22) << 23);
+  uint32_t d[3][16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int X = __float2int_rn(v[e] * inv);
+    const int d2 = ((X + 128) & 255) - 128;
+    const int X1 = (X - d2) >> 8;
+    const int d1 = ((X1 + 128) & 255) - 128;
+    const int d0 = (X1 - d1) >> 8;
+    d[0][e] = (uint32_t)d0 & 0xFFu;
+    d[1][e] = (uint32_t)d1 & 0xFFu;
+    d[2][e] = (uint32_t)d2 & 0xFFu;
+  }
+  if (active) {
+    uint4* dst = reinterpret_cast<uint4*>(limb_bytes);
+#pragma unroll
+    for (int L = 0; L < 3; ++L) {
+      uint32_t w[4];
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        // element of byte k of word wd (see the word/byte formula of xq_quantize_group)
+        uint32_t acc = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = BITS == 4 ? 8 * (wd >> 1) + (wd & 1) + 2 * k : 4 * k + wd;
+          acc |= d[L][e] << (8 * k);
+        }
+        w[wd] = acc;
+      }
+      const int piece = BITS == 4 ? 6 * (part >> 1) + 2 * L + (part & 1) : 4 * L + part;
+      dst[piece * NG + g] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  float sx = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) sx += v[e];
+  sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+  if (BITS == 4) {
+    if (active && (part & 1) == 0) cs[2 * g + (part >> 1)] = make_float2(csc, sx);
+  } else {
+    sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+    if (active && part == 0) cs[g] = make_float2(csc, sx);
   }
 }
 

@@ -65,6 +65,57 @@ struct ExpertParams {
   int* err;
 };
 
+// ---- single-kernel path (k_fused.cu): a sequence of T tokens x L layers, one CTA per SM
+
+constexpr int kFusedWarps = 8;
+constexpr int kFusedMaxRing = 16;        // chunk buffers
+constexpr int kFusedMaxItems = 64;       // staged items per CTA and step
+constexpr int kFusedMaxKS = 8;           // warps sharing one row
+constexpr int kFusedMaxChunkRows = 32;   // gate/up row pairs per chunk
+constexpr int kFusedMaxDnRows = 64;      // down rows per CTA
+constexpr int kFusedMaxLayers = 32;      // layers per launch
+constexpr long long kFusedSmemBudget = 223232;  // dynamic shared memory, bytes (static use is about 8.5 KiB)
+
+struct FusedLayer {                      // 64 bytes
+  const uint8_t* routed;                 // routed bank: record 0
+  long long stride;                      // bytes between records
+  const uint8_t* shared;                 // the shared expert's record
+  const uint16_t* w_router;              // bf16 [E][H]
+  const float* bias;                     // [E] or NULL
+  const uint16_t* w_sgate;               // bf16 [H]
+  const float* gamma;                    // [H] or NULL (no RMSNorm)
+  float eps;
+  int pad;
+};
+
+struct FusedParams {
+  FusedLayer layers[kFusedMaxLayers];
+  long long off[9];                      // record offsets, common to both banks of every layer
+  int L, T, H, I, E, K;
+  const float* h;                        // [T][H] input of layer 0
+  float* out;                            // [T][H] output of the last layer (also the stack's running state)
+  int32_t* idx_out;                      // [T][K] or NULL (single-layer calls)
+  float* w_out;
+  float* logits;                         // workspace: [E+1]
+  float* act;                            // [(K+1)][I]
+  uint8_t* act_limbs;                    // [(K+1)][3I] digits of act
+  float2* act_cs;                        // [(K+1)][I*bits/128]
+  unsigned* grp_cnt;                     // [(K+1)][I/64], zero between calls
+  unsigned* bar_cnt;                     // grid barrier words, zero before first use
+  unsigned* bar_gen;
+  int* err;
+  int nbuf, chb, cu, rt_rows, ru, rd, dn_rows_max, dn_slot_bytes, dn_off, ring_off;
+};
+
+struct FusedPlan {
+  bool ok;
+  int P, nbuf, chb, cu, rt_rows, ru, rd, dn_rows_max, dn_slot_bytes, dn_off, ring_off;
+  size_t smem;
+};
+
+FusedPlan plan_fused(int bits, int H, int I, int E, int K);
+cudaError_t launch_fused(const FusedParams& p, const FusedPlan& pl, int bits, bool pdl, cudaStream_t s);
+
 cudaError_t launch_rmsnorm(const float* h, const float* gamma, float eps, int T, int H, float* y, cudaStream_t s);
 cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, cudaStream_t s);
 cudaError_t launch_router(RouterParams p, int xq_bits, bool pdl, cudaStream_t s);

@@ -1,0 +1,634 @@
+// k_fused.cu -- the whole MoE block as one persistent kernel, for a sequence of steps.
+//
+// One step is one token through one layer: RMSNorm, router GEMV, softmax/top-K,
+// gate/up + SwiGLU of the K routed experts and the shared expert, down and the
+// weighted combine with the sigmoid-gated shared expert and the residual
+// ("What is Flash-MoE" (a2a-mcp.org), MoE section and sections 2-3; the
+// per-layer pipeline of the "Flash-MoE" wiki summary (jeongsk)).  The pages run
+// these as separate GPU dispatches with the top-K on the CPU in between; here
+// one CTA per SM carries every step of a sequence, and the data dependencies
+// between the block's phases become grid-wide barriers in global memory:
+//
+//   A: every CTA's router logits are written      -> each CTA selects the experts itself
+//   B: every SwiGLU activation group is quantised -> down projection
+//   C: every output row of the step is written    -> the next step reads it (stacked layers only)
+//
+// The bytes of a step fall into two kinds.  The router rows, the shared
+// expert's gate/up rows and the shared expert's down rows do not depend on the
+// routing, so a CTA requests its share of them for step s+1 as soon as its
+// gate/up work of step s is done, and for step s+1 that data is already in
+// shared memory.  The routed experts' gate/up rows stream through a ring of
+// chunk buffers, and their down rows land in a separate region while gate/up is
+// still running, so the down phase after barrier B computes from shared memory.
+//
+// Dot products use the per-group fold of fmoe_device.cuh:
+//   sum_c (q_c s + b) x_c = s * sum_c q_c x_c + b * sum_c x_c
+// with exact dp4a integer sums against a 3-digit fixed-point x.
+#include "fmoe_internal.h"
+
+namespace fmoe {
+namespace {
+
+constexpr int kFW = kFusedWarps;
+constexpr int kFT = kFW * 32;
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Grid barrier by generation count.  Thread 0 only, after a __syncthreads()
+// that orders the CTA's writes.  Arrive returns the generation to wait on;
+// the last CTA to arrive resets the count and publishes the next generation.
+__device__ __forceinline__ unsigned grid_arrive(unsigned* cnt, unsigned* gen, unsigned P) {
+  const unsigned g = ld_acquire_u32(gen);
+  __threadfence();
+  const unsigned old = atomicAdd(cnt, 1u);
+  if (old == P - 1) {
+    atomicExch(cnt, 0u);
+    __threadfence();
+    st_release_u32(gen, g + 1);
+  }
+  return g;
+}
+
+// Waits (at most kWaitNs) until the generation moves past g.
+__device__ __forceinline__ bool grid_wait(const unsigned* gen, unsigned g, int* err) {
+  bool ok = true;
+  if (ld_acquire_u32(gen) == g) {
+    const unsigned long long t0 = global_ns();
+    while (ld_acquire_u32(gen) == g) {
+      if (global_ns() - t0 > kWaitNs) {
+        atomicExch(err, kDevTimeout);
+        ok = false;
+        break;
+      }
+    }
+  }
+  __threadfence();
+  return ok;
+}
+
+struct Item {
+  int kind;  // 0: router rows, 1: gate/up rows
+  int slot;  // gate/up: expert slot (K = shared)
+  int row0;
+  int rows;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ FusedParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t s_full[kFusedMaxRing];
+  __shared__ __align__(8) uint64_t s_dnbar;
+  __shared__ __align__(8) uint64_t s_xbar;
+  __shared__ Item s_item[kFusedMaxItems];
+  __shared__ int s_pend[kFusedMaxRing];
+  __shared__ int s_idx[32];
+  __shared__ float s_w[33];
+  __shared__ float s_red[kFW];
+  __shared__ float s_rpart[2][8 * 8];
+  __shared__ float s_gpart[2][kFusedMaxKS * kFusedMaxChunkRows * 2];
+  __shared__ float s_dpart[kFusedMaxKS * kFusedMaxDnRows];
+  __shared__ int s_gdone[64];
+  __shared__ int s_abort;
+  __shared__ int s_nconst, s_nitems;
+  __shared__ int s_dnstate;  // down rows of the current step: 0 none in flight, 1 shared issued, 2 all issued
+  __shared__ int s_xstate;   // activation digits in flight
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int P = gridDim.x, b = blockIdx.x;
+  const int H = p.H, I = p.I, K = p.K, E = p.E, NE = K + 1;
+  const int NGH = H / kGroup, NGI = I / kGroup;
+  const int RB = H * BITS / 8, SB = NGH * 2;        // gate/up row: code bytes, scale bytes
+  const int RBd = I * BITS / 8, SBd = NGI * 2;      // down row
+  const int ncd = I * BITS / 128;  // chunk scalars of one activation vector
+  const int nbuf = p.nbuf, chb = p.chb, CU = p.cu;
+  uint8_t* xd = sm;
+  uint8_t* dn = sm + p.dn_off;
+  uint8_t* ring = sm + p.ring_off;
+  float* s_x = reinterpret_cast<float*>(xd);
+  uint8_t* s_xl = xd + (size_t)H * 4;
+  float2* s_xcs = reinterpret_cast<float2*>(xd + (size_t)H * 4 + (size_t)NGH * kGroupWords * 4);
+  const uint64_t pol = l2_policy_evict_first();
+
+  // ---- this CTA's share of every phase (the same for every step)
+  const int R = E + 1;  // router rows + the shared-gate row
+  const int rr0 = (int)((long long)b * R / P), rr1 = (int)((long long)(b + 1) * R / P);
+  const int US = I / p.ru, UR = K * I / p.ru, UD = H / p.rd;
+  const int sh0 = (int)((long long)b * US / P) * p.ru, sh1 = (int)((long long)(b + 1) * US / P) * p.ru;
+  const int rf0 = (int)((long long)b * UR / P) * p.ru, rf1 = (int)((long long)(b + 1) * UR / P) * p.ru;
+  const int d0 = (int)((long long)b * UD / P) * p.rd, d1 = (int)((long long)(b + 1) * UD / P) * p.rd;
+  const int nd = d1 - d0;
+  const int dn_slot = p.dn_slot_bytes, dmax = p.dn_rows_max;
+
+  if (tid == 0) {
+    int n = 0;
+    for (int r = rr0; r < rr1; r += p.rt_rows) s_item[n++] = Item{0, 0, r, min(p.rt_rows, rr1 - r)};
+    for (int r = sh0; r < sh1; r += CU) s_item[n++] = Item{1, K, r, min(CU, sh1 - r)};
+    s_nconst = n;
+    for (int f = rf0; f < rf1;) {
+      const int slot = f / I, r = f % I;
+      const int rows = min(min(CU, rf1 - f), I - r);
+      s_item[n++] = Item{1, slot, r, rows};
+      f += rows;
+    }
+    s_nitems = n;
+    for (int i = 0; i < nbuf; ++i) {
+      mbar_init(smem_addr(&s_full[i]), 1);
+      s_pend[i] = 0;
+    }
+    mbar_init(smem_addr(&s_dnbar), 2);
+    mbar_init(smem_addr(&s_xbar), 1);
+    mbar_fence_init();
+    s_abort = 0;
+    s_dnstate = 0;
+    s_xstate = 0;
+  }
+  __syncthreads();
+  const int n_const = s_nconst, n_items = s_nitems;
+  const int n_rt = (rr1 - rr0 + p.rt_rows - 1) / p.rt_rows;
+
+  // ---- copies (one thread per call)
+  auto issue_item = [&](int j, const FusedLayer& ly) {
+    const Item it = s_item[j];
+    const int bi = j % nbuf;
+    uint8_t* buf = ring + (size_t)bi * chb;
+    const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_full[bi]);
+    s_pend[bi] = 1;
+    if (it.kind == 0) {
+      const int nr = max(0, min(it.rows, E - it.row0));  // rows of w_router; the rest is the shared-gate row
+      mbar_expect_tx(bar, (uint32_t)it.rows * H * 2);
+      if (nr > 0) bulk_g2s(dst, ly.w_router + (size_t)it.row0 * H, (uint32_t)nr * H * 2, bar, pol);
+      if (nr < it.rows) bulk_g2s(dst + (uint32_t)nr * H * 2, ly.w_sgate, (uint32_t)H * 2, bar, pol);
+    } else {
+      const uint8_t* rec = it.slot < K ? ly.routed + (long long)s_idx[it.slot] * ly.stride : ly.shared;
+      const uint32_t cb = (uint32_t)it.rows * RB, sbb = (uint32_t)it.rows * SB;
+      mbar_expect_tx(bar, 2 * cb + 4 * sbb);
+      bulk_g2s(dst, rec + p.off[0] + (long long)it.row0 * RB, cb, bar, pol);
+      bulk_g2s(dst + CU * RB, rec + p.off[3] + (long long)it.row0 * RB, cb, bar, pol);
+      bulk_g2s(dst + 2 * CU * RB, rec + p.off[1] + (long long)it.row0 * SB, sbb, bar, pol);
+      bulk_g2s(dst + 2 * CU * RB + CU * SB, rec + p.off[2] + (long long)it.row0 * SB, sbb, bar, pol);
+      bulk_g2s(dst + 2 * CU * RB + 2 * CU * SB, rec + p.off[4] + (long long)it.row0 * SB, sbb, bar, pol);
+      bulk_g2s(dst + 2 * CU * RB + 3 * CU * SB, rec + p.off[5] + (long long)it.row0 * SB, sbb, bar, pol);
+    }
+  };
+  // Down rows [d0, d1) of one slot into its region of DN.
+  auto issue_down = [&](int slot, const uint8_t* rec) {
+    uint8_t* base = dn + (size_t)slot * dn_slot;
+    const uint32_t bar = smem_addr(&s_dnbar);
+    bulk_g2s(smem_addr(base), rec + p.off[6] + (long long)d0 * RBd, (uint32_t)nd * RBd, bar, pol);
+    bulk_g2s(smem_addr(base + (size_t)dmax * RBd), rec + p.off[7] + (long long)d0 * SBd, (uint32_t)nd * SBd, bar, pol);
+    bulk_g2s(smem_addr(base + (size_t)dmax * (RBd + SBd)), rec + p.off[8] + (long long)d0 * SBd, (uint32_t)nd * SBd,
+             bar, pol);
+  };
+  auto issue_shared_down = [&](const FusedLayer& ly) {
+    if (nd == 0) return;
+    s_dnstate = 1;
+    mbar_expect_tx(smem_addr(&s_dnbar), (uint32_t)nd * (RBd + 2 * SBd));
+    issue_down(K, ly.shared);
+  };
+
+  // ---- lane geometry
+  // gate/up: KS warps share a row (each lane one group of 64 columns), or RPP rows share a warp
+  const int KS = NGH >= 32 ? NGH / 32 : 1;
+  const int LPR = NGH >= 32 ? 32 : NGH, RPP = 32 / LPR;
+  const int gsub = lane / LPR, gl = lane % LPR;
+  const int kap = warp % KS;
+  const int xg = NGH >= 32 ? kap * 32 + lane : gl;  // this lane's group of x
+  // down: (slot, group) pairs, one per lane
+  const int NP = NE * NGI;
+  int np2 = 1;
+  while (np2 < NP) np2 <<= 1;
+  const int LPRd = np2 < 32 ? np2 : 32, RPPd = 32 / LPRd, KSd = np2 > 32 ? np2 / 32 : 1;
+  const int dsub = lane / LPRd, dl = lane % LPRd, kapd = warp % KSd;
+  const int q = kapd * 32 + dl;
+  const bool qon = q < NP;
+  const int qslot = qon ? q / NGI : 0, qg = qon ? q % NGI : 0;
+
+  uint32_t ph = 0;  // per ring buffer: parity of its next fill
+  bool ok = true;
+
+  // After a failed wait: let every copy in flight into this CTA's shared memory
+  // land (bounded), then leave.  `sp` is the step's parity.
+  auto abort_all = [&](int sp) {
+    __syncthreads();
+    if (tid == 0) {
+      for (int i = 0; i < nbuf; ++i)
+        if (s_pend[i]) mbar_wait_bounded(smem_addr(&s_full[i]), (ph >> i) & 1u, p.err);
+      if (s_dnstate == 1) mbar_arrive(smem_addr(&s_dnbar));  // the routed half never came
+      if (s_dnstate > 0) mbar_wait_bounded(smem_addr(&s_dnbar), (uint32_t)(sp & 1), p.err);
+      if (s_xstate) mbar_wait_bounded(smem_addr(&s_xbar), (uint32_t)(sp & 1), p.err);
+    }
+  };
+
+  const int S = p.T * p.L;
+  unsigned gen_c = 0;
+  bool wait_c = false;
+
+  // Step 0's routing-independent rows, before waiting on the previous kernel.
+  if (tid == 0) {
+    const FusedLayer& ly0 = p.layers[0];
+    for (int j = 0; j < n_const && j < nbuf; ++j) issue_item(j, ly0);
+    issue_shared_down(ly0);
+  }
+  pdl_wait();
+  pdl_trigger();  // the next kernel's CTAs start only once every CTA of this grid is running
+
+  int s = 0;
+  for (; s < S; ++s) {
+    const int t = s / p.L, l = s % p.L;
+    const FusedLayer& ly = p.layers[l];
+    const float* hin = (l == 0 ? p.h : p.out) + (size_t)t * H;
+    float* hout = p.out + (size_t)t * H;
+
+    if (s > 0 && tid == 0) issue_shared_down(ly);
+    if (wait_c && tid == 0 && !grid_wait(p.bar_gen, gen_c, p.err)) s_abort = 1;
+    wait_c = false;
+    __syncthreads();
+    if (s_abort) break;
+
+    // ---- x = RMSNorm(h), its digits (whole vector, in this CTA)
+    float ss = 0.0f;
+    for (int i = tid * 4; i < H; i += kFT * 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(hin + i));
+      *reinterpret_cast<float4*>(s_x + i) = v;
+      ss = fmaf(v.x, v.x, ss);
+      ss = fmaf(v.y, v.y, ss);
+      ss = fmaf(v.z, v.z, ss);
+      ss = fmaf(v.w, v.w, ss);
+    }
+    if (ly.gamma) {
+      ss = warp_sum(ss);
+      if (lane == 0) s_red[warp] = ss;
+      __syncthreads();
+      float tot = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kFW; ++w) tot += s_red[w];
+      const float rstd = 1.0f / sqrtf(tot / (float)H + ly.eps);
+      for (int i = tid; i < H; i += kFT) s_x[i] = s_x[i] * rstd * ly.gamma[i];
+    }
+    __syncthreads();
+    for (int g = warp; g < NGH; g += kFW) {
+      const float2 v = reinterpret_cast<const float2*>(s_x + g * kGroup)[lane];
+      xq_quantize_group<BITS>(v.x, v.y, g, NGH, s_xl, s_xcs);
+    }
+
+    // ---- router rows: logits of this CTA's rows (8 warp segments per row, fixed order)
+    int j = 0;
+    for (; j < n_rt; ++j) {
+      const int bi = j % nbuf;
+      if (!mbar_wait_bounded(smem_addr(&s_full[bi]), (ph >> bi) & 1u, p.err)) ok = false;
+      ph ^= 1u << bi;
+      const Item it = s_item[j];
+      const uint16_t* wr = reinterpret_cast<const uint16_t*>(ring + (size_t)bi * chb);
+      const int seg = H / 8;
+      float* part = s_rpart[j & 1];
+      for (int task = warp; ok && task < it.rows * 8; task += kFW) {
+        const int r = task >> 3, sg = task & 7;
+        const uint4* wv = reinterpret_cast<const uint4*>(wr + (size_t)r * H + sg * seg);
+        const float* xv = s_x + sg * seg;
+        float acc = 0.0f;
+        for (int k = lane; k < seg / 8; k += 32) {
+          const uint4 w = wv[k];
+          const float4 xa = *reinterpret_cast<const float4*>(xv + 8 * k);
+          const float4 xb = *reinterpret_cast<const float4*>(xv + 8 * k + 4);
+          acc = fmaf(__uint_as_float(w.x << 16), xa.x, acc);
+          acc = fmaf(__uint_as_float(w.x & 0xFFFF0000u), xa.y, acc);
+          acc = fmaf(__uint_as_float(w.y << 16), xa.z, acc);
+          acc = fmaf(__uint_as_float(w.y & 0xFFFF0000u), xa.w, acc);
+          acc = fmaf(__uint_as_float(w.z << 16), xb.x, acc);
+          acc = fmaf(__uint_as_float(w.z & 0xFFFF0000u), xb.y, acc);
+          acc = fmaf(__uint_as_float(w.w << 16), xb.z, acc);
+          acc = fmaf(__uint_as_float(w.w & 0xFFFF0000u), xb.w, acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) part[task] = acc;
+      }
+      __syncthreads();
+      if (tid < it.rows) {
+        float lg = 0.0f;
+#pragma unroll
+        for (int sg = 0; sg < 8; ++sg) lg += part[tid * 8 + sg];
+        const int row = it.row0 + tid;
+        if (row < E && ly.bias) lg += ly.bias[row];
+        p.logits[row] = lg;
+      }
+      if (tid == 0) {
+        s_pend[bi] = 0;
+        if (ok && j + nbuf < n_const) {  // more routing-independent rows than buffers
+          fence_proxy_async();
+          issue_item(j + nbuf, ly);
+        }
+      }
+    }
+    if (!ok) s_abort = 1;
+    __syncthreads();
+    if (s_abort) break;
+    unsigned gen_a = 0;
+    if (tid == 0) gen_a = grid_arrive(p.bar_cnt, p.bar_gen, P);
+
+    // ---- this lane's digits of x, for every gate/up row of the step
+    uint32_t L[48];
+    load_group_limbs(reinterpret_cast<const uint32_t*>(s_xl), xg, NGH, L);
+    float2 csx;
+    if (BITS == 4) {
+      const float2 a = s_xcs[2 * xg], c = s_xcs[2 * xg + 1];
+      csx = make_float2(a.x, a.y + c.y);
+    } else {
+      csx = s_xcs[xg];
+    }
+
+    // gate/up of one staged item: partial sums per (k-part, row) into s_gpart, then SwiGLU.
+    auto gateup_item = [&](int jj) {
+      const int bi = jj % nbuf;
+      if (!mbar_wait_bounded(smem_addr(&s_full[bi]), (ph >> bi) & 1u, p.err)) ok = false;
+      ph ^= 1u << bi;
+      const Item it = s_item[jj];
+      const uint8_t* buf = ring + (size_t)bi * chb;
+      float* part = s_gpart[jj & 1];
+      for (int pass = warp / KS; ok && pass * RPP < it.rows; pass += kFW / KS) {
+        const int r = pass * RPP + gsub;
+        float ag = 0.0f, au = 0.0f;
+        if (r < it.rows) {
+          uint4 q0, q1, v0, v1;
+          const uint8_t* gr = buf + (size_t)r * RB + xg * (kGroup * BITS / 8);
+          const uint8_t* ur = gr + (size_t)CU * RB;
+          q0 = *reinterpret_cast<const uint4*>(gr);
+          q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(gr + 16) : q0;
+          v0 = *reinterpret_cast<const uint4*>(ur);
+          v1 = BITS == 4 ? *reinterpret_cast<const uint4*>(ur + 16) : v0;
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * (size_t)CU * RB + (size_t)r * SB);
+          const int cs2 = CU * SB / 2;
+          const float gs = bf16_to_f32(sc[xg]), gb = bf16_to_f32(sc[cs2 + xg]);
+          const float us = bf16_to_f32(sc[2 * cs2 + xg]), ub = bf16_to_f32(sc[3 * cs2 + xg]);
+          const float Sg = group_dot<BITS>(q0, q1, L);
+          const float Su = group_dot<BITS>(v0, v1, L);
+          ag = fmaf(gs, csx.x * Sg, gb * csx.y);
+          au = fmaf(us, csx.x * Su, ub * csx.y);
+        }
+        for (int o = LPR / 2; o > 0; o >>= 1) {
+          ag += __shfl_xor_sync(0xffffffffu, ag, o);
+          au += __shfl_xor_sync(0xffffffffu, au, o);
+        }
+        if (gl == 0 && r < it.rows) {
+          part[(kap * kFusedMaxChunkRows + r) * 2] = ag;
+          part[(kap * kFusedMaxChunkRows + r) * 2 + 1] = au;
+        }
+      }
+      __syncthreads();  // every warp is done with the buffer and the partial sums are complete
+      if (tid < it.rows) {
+        float g = 0.0f, u = 0.0f;
+        for (int k = 0; k < KS; ++k) {
+          g += part[(k * kFusedMaxChunkRows + tid) * 2];
+          u += part[(k * kFusedMaxChunkRows + tid) * 2 + 1];
+        }
+        p.act[(size_t)it.slot * I + it.row0 + tid] = g / (1.0f + expf(-g)) * u;
+      }
+      if (tid == 0) s_pend[bi] = 0;
+    };
+
+    // ---- shared expert's gate/up while the other CTAs finish their logits
+    for (; j < n_const; ++j) {
+      gateup_item(j);
+      if (tid == 0 && ok && j + nbuf < n_const) {  // more routing-independent rows than buffers
+        fence_proxy_async();
+        issue_item(j + nbuf, ly);
+      }
+    }
+
+    // ---- barrier A, then the routing (each CTA selects the experts itself)
+    if (tid == 0 && !grid_wait(p.bar_gen, gen_a, p.err)) s_abort = 1;
+    if (!ok) s_abort = 1;
+    __syncthreads();
+    if (s_abort) break;
+    if (warp == 0) {
+      int ik;
+      float wk, sig;
+      warp_topk(p.logits, E, K, 1, ik, wk, sig);
+      if (ik < 0 || ik >= E) ik = 0;
+      if (lane < K) {
+        s_idx[lane] = ik;
+        s_w[lane] = wk;
+        if (b == 0 && p.idx_out) p.idx_out[(size_t)t * K + lane] = ik;
+        if (b == 0 && p.w_out) p.w_out[(size_t)t * K + lane] = wk;
+      }
+      if (lane == 0) s_w[K] = sig;
+      __syncwarp();
+      // routed gate/up rows into every buffer (all consumed by now), one item per lane
+      fence_proxy_async();
+      for (int jj = n_const + lane; jj < n_items && jj < n_const + nbuf; jj += 32) issue_item(jj, ly);
+      // routed down rows: one slot per lane
+      if (nd > 0 && lane < K) {
+        if (lane == 0) {
+          s_dnstate = 2;
+          mbar_expect_tx(smem_addr(&s_dnbar), (uint32_t)K * nd * (RBd + 2 * SBd));
+        }
+        __syncwarp(0xffffffffu >> (32 - K));
+        issue_down(lane, ly.routed + (long long)s_idx[lane] * ly.stride);
+      }
+    }
+    __syncthreads();
+
+    // ---- routed gate/up through the ring
+    for (; j < n_items; ++j) {
+      gateup_item(j);
+      if (tid == 0 && ok && j + nbuf < n_items) {
+        fence_proxy_async();
+        issue_item(j + nbuf, ly);
+      }
+    }
+
+    // ---- activation groups of 64: the CTA that completes a group writes its digits
+    __threadfence();
+    if (!ok) s_abort = 1;
+    __syncthreads();
+    if (s_abort) break;
+    // groups touched: shared rows [sh0, sh1) of slot K, routed flat rows [rf0, rf1)
+    const int gs0 = sh0 / kGroup, gs1 = sh1 > sh0 ? (sh1 - 1) / kGroup + 1 : gs0;
+    const int gr0 = rf0 / kGroup, gr1 = rf1 > rf0 ? (rf1 - 1) / kGroup + 1 : gr0;
+    const int ngs = gs1 - gs0, ngt = ngs + (gr1 - gr0);
+    if (tid < ngt) {
+      int fg, lo, hi;  // flat group over slot-major rows, and this CTA's rows in it
+      if (tid < ngs) {
+        const int g = gs0 + tid;
+        fg = K * NGI + g;
+        lo = max(sh0, g * kGroup);
+        hi = min(sh1, (g + 1) * kGroup);
+      } else {
+        const int g = gr0 + tid - ngs;
+        fg = g;
+        lo = max(rf0, g * kGroup);
+        hi = min(rf1, (g + 1) * kGroup);
+      }
+      const unsigned prev = atomicAdd(&p.grp_cnt[fg], (unsigned)(hi - lo));
+      s_gdone[tid] = prev + (unsigned)(hi - lo) == (unsigned)kGroup ? fg + 1 : 0;
+    }
+    __syncthreads();
+    for (int k = warp; k < ngt; k += kFW) {
+      const int fg1 = s_gdone[k];
+      if (!fg1) continue;
+      __threadfence();
+      const int fg = fg1 - 1, slot = fg / NGI, gg = fg % NGI;
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)fg * kGroup) + lane);
+      xq_quantize_group<BITS>(v.x, v.y, gg, NGI, p.act_limbs + (size_t)slot * NGI * kGroupWords * 4,
+                              p.act_cs + (size_t)slot * ncd);
+      if (lane == 0) p.grp_cnt[fg] = 0u;
+    }
+    __threadfence();
+    __syncthreads();
+
+    // ---- the next step's routing-independent rows, into the drained ring
+    if (tid == 0 && s + 1 < S) {
+      fence_proxy_async();
+      const FusedLayer& ln = p.layers[(s + 1) % p.L];
+      for (int jj = 0; jj < n_const && jj < nbuf; ++jj) issue_item(jj, ln);
+    }
+
+    // ---- barrier B, then down + combine from shared memory
+    if (tid == 0) {
+      const unsigned gb = grid_arrive(p.bar_cnt, p.bar_gen, P);
+      if (!grid_wait(p.bar_gen, gb, p.err)) s_abort = 1;
+      if (!s_abort) {
+        const uint32_t bx = smem_addr(&s_xbar);
+        const uint32_t lb = (uint32_t)NE * NGI * kGroupWords * 4, cb = (uint32_t)NE * ncd * 8;
+        fence_proxy_async();
+        s_xstate = 1;
+        mbar_expect_tx(bx, lb + cb);
+        bulk_g2s(smem_addr(xd), p.act_limbs, lb, bx, pol);
+        bulk_g2s(smem_addr(xd + lb), p.act_cs, cb, bx, pol);
+      }
+    }
+    __syncthreads();
+    if (s_abort) break;
+    if (!mbar_wait_bounded(smem_addr(&s_xbar), (uint32_t)(s & 1), p.err)) ok = false;
+    if (nd > 0 && !mbar_wait_bounded(smem_addr(&s_dnbar), (uint32_t)(s & 1), p.err)) ok = false;
+    if (!ok) s_abort = 1;
+    __syncthreads();
+    if (s_abort) break;
+    if (tid == 0) {
+      s_xstate = 0;
+      s_dnstate = 0;
+    }
+    {
+      uint32_t A[48];
+      const uint8_t* al = xd + (size_t)qslot * NGI * kGroupWords * 4;
+      load_group_limbs(reinterpret_cast<const uint32_t*>(al), qg, NGI, A);
+      const float2* acs = reinterpret_cast<const float2*>(xd + (size_t)NE * NGI * kGroupWords * 4) + qslot * ncd;
+      float2 csa;
+      if (BITS == 4) {
+        const float2 a = acs[2 * qg], c = acs[2 * qg + 1];
+        csa = make_float2(a.x, a.y + c.y);
+      } else {
+        csa = acs[qg];
+      }
+      const float wq = qon ? s_w[qslot] : 0.0f;
+      const uint8_t* sb = dn + (size_t)qslot * dn_slot;
+      for (int pass = warp / KSd; ok && pass * RPPd < nd; pass += kFW / KSd) {
+        const int r = pass * RPPd + dsub;
+        float acc = 0.0f;
+        if (qon && r < nd) {
+          const uint8_t* cr = sb + (size_t)r * RBd + qg * (kGroup * BITS / 8);
+          const uint4 q0 = *reinterpret_cast<const uint4*>(cr);
+          const uint4 q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(cr + 16) : q0;
+          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * RBd + (size_t)r * SBd)[qg]);
+          const float bi =
+              bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * (RBd + SBd) + (size_t)r * SBd)[qg]);
+          const float Sd = group_dot<BITS>(q0, q1, A);
+          acc = wq * fmaf(sc, csa.x * Sd, bi * csa.y);
+        }
+        for (int o = LPRd / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (dl == 0 && r < nd) s_dpart[kapd * kFusedMaxDnRows + r] = acc;
+      }
+    }
+    __syncthreads();
+    for (int r = tid; r < nd; r += kFT) {
+      float y = 0.0f;
+      for (int k = 0; k < KSd; ++k) y += s_dpart[k * kFusedMaxDnRows + r];
+      hout[d0 + r] = __ldcg(hin + d0 + r) + y;
+    }
+    // the next step reads this step's output when it is the next layer of a stack
+    if (s + 1 < S && (s + 1) % p.L != 0) {
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) gen_c = grid_arrive(p.bar_cnt, p.bar_gen, P);
+      wait_c = true;
+    }
+    __syncthreads();  // shared memory of this step (DN, XD) is free
+    if (tid == 0) fence_proxy_async();
+  }
+  if (s < S) abort_all(s);
+}
+
+}  // namespace
+
+FusedPlan plan_fused(int bits, int H, int I, int E, int K) {
+  FusedPlan pl{};
+  pl.ok = false;
+  if (H % kGroup || I % kGroup || K < 1 || K > 32 || E < K) return pl;
+  const int NGH = H / kGroup, NGI = I / kGroup, NE = K + 1;
+  if (NGH > 128 || NGI > 128) return pl;
+  const int RB = H * bits / 8, SB = NGH * 2, RBd = I * bits / 8, SBd = NGI * 2;
+  const int sms = num_sms();
+  int P = ((NE * I) + 31) / 32;
+  P = P < 2 ? 2 : P;
+  P = P > sms ? sms : P;
+  pl.P = P;
+  pl.ru = SB >= 16 ? 1 : 16 / SB;
+  pl.rd = SBd >= 16 ? 1 : 16 / SBd;
+  // down pairs per row: one per lane across at most 8 warps
+  int np2 = 1;
+  while (np2 < NE * NGI) np2 <<= 1;
+  if (np2 > 32 * kFusedMaxKS) return pl;
+  const int UD = H / pl.rd;
+  pl.dn_rows_max = (UD + P - 1) / P * pl.rd;
+  if (pl.dn_rows_max > kFusedMaxDnRows) return pl;
+  pl.dn_slot_bytes = (pl.dn_rows_max * (RBd + 2 * SBd) + 127) / 128 * 128;
+  const size_t xd1 = (size_t)H * 4 + (size_t)NGH * kGroupWords * 4 + (size_t)(H * bits / 128) * 8;
+  const size_t xd2 = (size_t)NE * NGI * kGroupWords * 4 + (size_t)NE * (I * bits / 128) * 8;
+  const size_t xd = ((xd1 > xd2 ? xd1 : xd2) + 127) / 128 * 128;
+  pl.dn_off = (int)xd;
+  pl.ring_off = (int)(xd + (size_t)NE * pl.dn_slot_bytes);
+  // gate/up chunks of about 18 KiB, a whole number of row units, at most kFusedMaxChunkRows rows
+  const int pair = 2 * (RB + 2 * SB);
+  int cu = 18432 / pair;
+  cu = cu < 1 ? 1 : cu;
+  cu = cu > kFusedMaxChunkRows ? kFusedMaxChunkRows : cu;
+  cu = cu / pl.ru * pl.ru;
+  if (cu < pl.ru) return pl;
+  pl.cu = cu;
+  pl.chb = ((cu * pair) + 127) / 128 * 128;
+  if (pl.chb < H * 2) pl.chb = (H * 2 + 127) / 128 * 128;  // at least one router row per buffer
+  int rt = pl.chb / (H * 2);
+  pl.rt_rows = rt > 8 ? 8 : rt;
+  const long long budget = kFusedSmemBudget - pl.ring_off;
+  if (budget < 2LL * pl.chb) return pl;
+  int nbuf = (int)(budget / pl.chb);
+  pl.nbuf = nbuf > kFusedMaxRing ? kFusedMaxRing : nbuf;
+  pl.smem = (size_t)pl.ring_off + (size_t)pl.nbuf * pl.chb;
+  // items per CTA must fit the item table
+  const int R = E + 1;
+  const int rt_items = ((R + P - 1) / P + pl.rt_rows - 1) / pl.rt_rows;
+  const int sh_items = ((I / pl.ru + P - 1) / P * pl.ru + cu - 1) / cu;
+  const int rf_items = ((K * I / pl.ru + P - 1) / P * pl.ru + cu - 1) / cu + 2;
+  if (rt_items + sh_items + rf_items > kFusedMaxItems) return pl;
+  // activation groups counted per CTA must fit s_gdone
+  const int gcount = ((I / pl.ru + P - 1) / P * pl.ru) / kGroup + 2 + ((K * I / pl.ru + P - 1) / P * pl.ru) / kGroup + 2;
+  if (gcount > 64) return pl;
+  pl.ok = true;
+  return pl;
+}
+
+cudaError_t launch_fused(const FusedParams& p, const FusedPlan& pl, int bits, bool pdl, cudaStream_t s) {
+  void (*k)(const FusedParams) = bits == 4 ? fused_kernel<4> : fused_kernel<2>;
+  cudaError_t e = set_smem((const void*)k, pl.smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(pl.P), dim3(kFT), pl.smem, s, pdl, p);
+}
+
+}  // namespace fmoe
