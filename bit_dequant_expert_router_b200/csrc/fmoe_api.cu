@@ -390,10 +390,10 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   return FMOE_OK;
 }
 
-// The single-kernel path (k_fused.cu) unless FMOE_FUSED=0 is set in the environment.
+// The single-kernel path (k_fused.cu) when FMOE_FUSED=1 is set in the environment.
 static bool fused_enabled() {
   const char* v = getenv("FMOE_FUSED");
-  return !(v && v[0] == '0');
+  return v && v[0] == '1';
 }
 
 static bool same_offsets(const fmoe_bank& a, const fmoe_bank& b) {

@@ -73,6 +73,8 @@ constexpr int kFusedMaxItems = 64;       // staged items per CTA and step
 constexpr int kFusedMaxKS = 8;           // warps sharing one row
 constexpr int kFusedMaxChunkRows = 32;   // gate/up row pairs per chunk
 constexpr int kFusedMaxDnRows = 64;      // down rows per CTA
+constexpr int kFusedMaxGuRows = 64;      // gate/up row pairs per CTA
+constexpr int kFusedMaxRtRows = 4;       // router rows per staged item
 constexpr int kFusedMaxLayers = 32;      // layers per launch
 constexpr long long kFusedSmemBudget = 223232;  // dynamic shared memory, bytes (static use is about 8.5 KiB)
 

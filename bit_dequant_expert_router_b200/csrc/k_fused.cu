@@ -31,6 +31,13 @@ namespace {
 
 constexpr int kFW = kFusedWarps;
 constexpr int kFT = kFW * 32;
+// A gpu-scope fence or release operation waits for every bulk copy that its own
+// thread still has in flight (measured on B200: about a microsecond with a 64 KiB
+// copy outstanding; a fence in another warp, or a CTA-scope fence, returns at
+// once).  Warp 0 issues the long-lived copies (routed down rows, the next step's
+// rows), so grid barriers run on thread kBarT of warp 1 and the release fences on
+// warps 1..7, never on warp 0.
+constexpr int kBarT = 32;
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
@@ -75,11 +82,125 @@ __device__ __forceinline__ bool grid_wait(const unsigned* gen, unsigned g, int* 
 }
 
 struct Item {
-  int kind;  // 0: router rows, 1: gate/up rows
-  int slot;  // gate/up: expert slot (K = shared)
+  int kind;   // 0: router rows, 1: gate/up rows
+  int slot;   // gate/up: expert slot (K = shared)
   int row0;
   int rows;
+  int rbase;  // gate/up: index of the item's first row among this CTA's gate/up rows
 };
+
+// Shapes the copy helpers need (kept out of line: the kernel runs each
+// phase once per step, so its code is kept small enough to stay in the
+// instruction cache).
+struct CopyShape {
+  int E, H, K, RB, SB, CU;
+  uint64_t pol;
+};
+
+// Stages one item into its ring buffer: router rows (the last may be the
+// shared-gate row), or `rows` rows of gate and of up of one expert with their
+// scales and biases.
+__device__ __noinline__ void issue_item_dev(const Item it, uint8_t* buf, uint32_t bar, const FusedLayer* ly,
+                                            const int* idx, const long long* off, const CopyShape cs) {
+  const uint32_t dst = smem_addr(buf);
+  if (it.kind == 0) {
+    const int nr = max(0, min(it.rows, cs.E - it.row0));  // rows of w_router; the rest is the shared-gate row
+    mbar_expect_tx(bar, (uint32_t)it.rows * cs.H * 2);
+    if (nr > 0) bulk_g2s(dst, ly->w_router + (size_t)it.row0 * cs.H, (uint32_t)nr * cs.H * 2, bar, cs.pol);
+    if (nr < it.rows) bulk_g2s(dst + (uint32_t)nr * cs.H * 2, ly->w_sgate, (uint32_t)cs.H * 2, bar, cs.pol);
+    return;
+  }
+  const uint8_t* rec = it.slot < cs.K ? ly->routed + (long long)idx[it.slot] * ly->stride : ly->shared;
+  const int RB = cs.RB, SB = cs.SB, CU = cs.CU;
+  const uint32_t cb = (uint32_t)it.rows * RB, sbb = (uint32_t)it.rows * SB;
+  mbar_expect_tx(bar, 2 * cb + 4 * sbb);
+  bulk_g2s(dst, rec + off[0] + (long long)it.row0 * RB, cb, bar, cs.pol);
+  bulk_g2s(dst + CU * RB, rec + off[3] + (long long)it.row0 * RB, cb, bar, cs.pol);
+  bulk_g2s(dst + 2 * CU * RB, rec + off[1] + (long long)it.row0 * SB, sbb, bar, cs.pol);
+  bulk_g2s(dst + 2 * CU * RB + CU * SB, rec + off[2] + (long long)it.row0 * SB, sbb, bar, cs.pol);
+  bulk_g2s(dst + 2 * CU * RB + 2 * CU * SB, rec + off[4] + (long long)it.row0 * SB, sbb, bar, cs.pol);
+  bulk_g2s(dst + 2 * CU * RB + 3 * CU * SB, rec + off[5] + (long long)it.row0 * SB, sbb, bar, cs.pol);
+}
+
+// Stages down rows [d0, d0 + nd) of one expert record (codes, scales, biases)
+// into its slot region of DN, which holds `dmax` rows.
+__device__ __noinline__ void issue_down_dev(uint8_t* base, uint32_t bar, const uint8_t* rec, const long long* off,
+                                            int d0, int nd, int dmax, int RBd, int SBd, uint64_t pol) {
+  bulk_g2s(smem_addr(base), rec + off[6] + (long long)d0 * RBd, (uint32_t)nd * RBd, bar, pol);
+  bulk_g2s(smem_addr(base + (size_t)dmax * RBd), rec + off[7] + (long long)d0 * SBd, (uint32_t)nd * SBd, bar, pol);
+  bulk_g2s(smem_addr(base + (size_t)dmax * (RBd + SBd)), rec + off[8] + (long long)d0 * SBd, (uint32_t)nd * SBd, bar,
+           pol);
+}
+
+// Routing of one token from its logits [E] (+ the shared-gate logit at E), E <= 512:
+// stage 1, every warp w takes the K largest keys of its slice of ceil(E/8)
+// logits (two per lane) into cand[w*K + k]; stage 2 (after a block barrier),
+// warp 0 takes the K largest of the 8K candidates.  Keys order by value, then
+// by lower index (topk_key), so the result is that of one sort of all E.
+__device__ __forceinline__ void topk_stage1(const float* logits, int E, int K, unsigned long long* cand) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ES = (E + kFW - 1) / kFW;
+  const int e0 = warp * ES + lane, e1 = e0 + 32;
+  unsigned long long k0 = (lane < ES && e0 < E) ? topk_key(__ldcg(logits + e0), e0) : 0ull;
+  unsigned long long k1 = (lane + 32 < ES && e1 < E) ? topk_key(__ldcg(logits + e1), e1) : 0ull;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    const unsigned long long m = warp_max_key(k0 > k1 ? k0 : k1);
+    if (lane == 0) cand[warp * K + k] = m;
+    k0 = k0 == m ? 0ull : k0;
+    k1 = k1 == m ? 0ull : k1;
+  }
+}
+
+// Stage 2, warp 0: picks, renormalised weights w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0)
+// and sigma = sigmoid(l_E) into idx[0..K), w[0..K], w[K] = sigma.
+__device__ __noinline__ void topk_stage2(const float* logits, int E, int K, const unsigned long long* cand, int* idx,
+                                         float* w) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long key[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) key[i] = lane + 32 * i < kFW * K ? cand[lane + 32 * i] : 0ull;
+  float top = 0.0f, mine = 0.0f;
+  int mi = 0;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) best = key[i] > best ? key[i] : best;
+    const unsigned long long m = warp_max_key(best);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) key[i] = key[i] == m ? 0ull : key[i];
+    int e = m ? topk_key_index(m) : 0;
+    const float v = topk_key_value(m);
+    if (e < 0 || e >= E) e = 0;  // only with non-finite logits
+    if (k == 0) top = v;
+    if (lane == k) {
+      mi = e;
+      mine = v;
+    }
+  }
+  const float ek = lane < K ? expf(mine - top) : 0.0f;
+  const float wk = ek / warp_sum(ek);
+  if (lane < K) {
+    idx[lane] = mi;
+    w[lane] = wk;
+  }
+  if (lane == 0) w[K] = 1.0f / (1.0f + expf(-__ldcg(logits + E)));
+}
+
+// Any E: one warp rescans the logits in memory for each pick.
+__device__ __noinline__ void topk_any(const float* logits, int E, int K, int* idx, float* w) {
+  int ik;
+  float wk, sig;
+  warp_topk_mem(logits, E, K, 1, ik, wk, sig);
+  const int lane = threadIdx.x & 31;
+  if (ik < 0 || ik >= E) ik = 0;
+  if (lane < K) {
+    idx[lane] = ik;
+    w[lane] = wk;
+  }
+  if (lane == 0) w[K] = sig;
+}
 
 template <int BITS>
 __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ FusedParams p) {
@@ -90,10 +211,12 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   __shared__ Item s_item[kFusedMaxItems];
   __shared__ int s_pend[kFusedMaxRing];
   __shared__ int s_idx[32];
+  __shared__ unsigned long long s_cand[kFW * 32];  // top-K candidates, K per warp
   __shared__ float s_w[33];
   __shared__ float s_red[kFW];
-  __shared__ float s_rpart[2][8 * 8];
-  __shared__ float s_gpart[2][kFusedMaxKS * kFusedMaxChunkRows * 2];
+  __shared__ float s_rpart[2][kFusedMaxRtRows * 8];
+  __shared__ float s_gacc[kFusedMaxGuRows * 4 * 2];  // gate/up partial sums [row][k-part][gate, up]
+  __shared__ int s_cnt[kFusedMaxRing];                // warps done with a buffer
   __shared__ float s_dpart[kFusedMaxKS * kFusedMaxDnRows];
   __shared__ int s_gdone[64];
   __shared__ int s_abort;
@@ -129,19 +252,25 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
 
   if (tid == 0) {
     int n = 0;
-    for (int r = rr0; r < rr1; r += p.rt_rows) s_item[n++] = Item{0, 0, r, min(p.rt_rows, rr1 - r)};
-    for (int r = sh0; r < sh1; r += CU) s_item[n++] = Item{1, K, r, min(CU, sh1 - r)};
+    int rb = 0;
+    for (int r = rr0; r < rr1; r += p.rt_rows) s_item[n++] = Item{0, 0, r, min(p.rt_rows, rr1 - r), 0};
+    for (int r = sh0; r < sh1; r += CU) {
+      s_item[n++] = Item{1, K, r, min(CU, sh1 - r), rb};
+      rb += min(CU, sh1 - r);
+    }
     s_nconst = n;
     for (int f = rf0; f < rf1;) {
       const int slot = f / I, r = f % I;
       const int rows = min(min(CU, rf1 - f), I - r);
-      s_item[n++] = Item{1, slot, r, rows};
+      s_item[n++] = Item{1, slot, r, rows, rb};
+      rb += rows;
       f += rows;
     }
     s_nitems = n;
     for (int i = 0; i < nbuf; ++i) {
       mbar_init(smem_addr(&s_full[i]), 1);
       s_pend[i] = 0;
+      s_cnt[i] = 0;
     }
     mbar_init(smem_addr(&s_dnbar), 2);
     mbar_init(smem_addr(&s_xbar), 1);
@@ -155,37 +284,14 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   const int n_rt = (rr1 - rr0 + p.rt_rows - 1) / p.rt_rows;
 
   // ---- copies (one thread per call)
+  const CopyShape cshape{E, H, K, RB, SB, CU, pol};
   auto issue_item = [&](int j, const FusedLayer& ly) {
-    const Item it = s_item[j];
     const int bi = j % nbuf;
-    uint8_t* buf = ring + (size_t)bi * chb;
-    const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_full[bi]);
     s_pend[bi] = 1;
-    if (it.kind == 0) {
-      const int nr = max(0, min(it.rows, E - it.row0));  // rows of w_router; the rest is the shared-gate row
-      mbar_expect_tx(bar, (uint32_t)it.rows * H * 2);
-      if (nr > 0) bulk_g2s(dst, ly.w_router + (size_t)it.row0 * H, (uint32_t)nr * H * 2, bar, pol);
-      if (nr < it.rows) bulk_g2s(dst + (uint32_t)nr * H * 2, ly.w_sgate, (uint32_t)H * 2, bar, pol);
-    } else {
-      const uint8_t* rec = it.slot < K ? ly.routed + (long long)s_idx[it.slot] * ly.stride : ly.shared;
-      const uint32_t cb = (uint32_t)it.rows * RB, sbb = (uint32_t)it.rows * SB;
-      mbar_expect_tx(bar, 2 * cb + 4 * sbb);
-      bulk_g2s(dst, rec + p.off[0] + (long long)it.row0 * RB, cb, bar, pol);
-      bulk_g2s(dst + CU * RB, rec + p.off[3] + (long long)it.row0 * RB, cb, bar, pol);
-      bulk_g2s(dst + 2 * CU * RB, rec + p.off[1] + (long long)it.row0 * SB, sbb, bar, pol);
-      bulk_g2s(dst + 2 * CU * RB + CU * SB, rec + p.off[2] + (long long)it.row0 * SB, sbb, bar, pol);
-      bulk_g2s(dst + 2 * CU * RB + 2 * CU * SB, rec + p.off[4] + (long long)it.row0 * SB, sbb, bar, pol);
-      bulk_g2s(dst + 2 * CU * RB + 3 * CU * SB, rec + p.off[5] + (long long)it.row0 * SB, sbb, bar, pol);
-    }
+    issue_item_dev(s_item[j], ring + (size_t)bi * chb, smem_addr(&s_full[bi]), &ly, s_idx, p.off, cshape);
   };
-  // Down rows [d0, d1) of one slot into its region of DN.
   auto issue_down = [&](int slot, const uint8_t* rec) {
-    uint8_t* base = dn + (size_t)slot * dn_slot;
-    const uint32_t bar = smem_addr(&s_dnbar);
-    bulk_g2s(smem_addr(base), rec + p.off[6] + (long long)d0 * RBd, (uint32_t)nd * RBd, bar, pol);
-    bulk_g2s(smem_addr(base + (size_t)dmax * RBd), rec + p.off[7] + (long long)d0 * SBd, (uint32_t)nd * SBd, bar, pol);
-    bulk_g2s(smem_addr(base + (size_t)dmax * (RBd + SBd)), rec + p.off[8] + (long long)d0 * SBd, (uint32_t)nd * SBd,
-             bar, pol);
+    issue_down_dev(dn + (size_t)slot * dn_slot, smem_addr(&s_dnbar), rec, p.off, d0, nd, dmax, RBd, SBd, pol);
   };
   auto issue_shared_down = [&](const FusedLayer& ly) {
     if (nd == 0) return;
@@ -248,68 +354,112 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     float* hout = p.out + (size_t)t * H;
 
     if (s > 0 && tid == 0) issue_shared_down(ly);
-    if (wait_c && tid == 0 && !grid_wait(p.bar_gen, gen_c, p.err)) s_abort = 1;
+    if (wait_c && tid == kBarT && !grid_wait(p.bar_gen, gen_c, p.err)) s_abort = 1;
     wait_c = false;
     __syncthreads();
     if (s_abort) break;
 
-    // ---- x = RMSNorm(h), its digits (whole vector, in this CTA)
+    // ---- x = RMSNorm(h) (two passes: sum of squares, then apply) and its digits,
+    // the whole vector in every CTA.  Pass 1 stages h in s_x.
     float ss = 0.0f;
+#pragma unroll 4
     for (int i = tid * 4; i < H; i += kFT * 4) {
       const float4 v = __ldcg(reinterpret_cast<const float4*>(hin + i));
       *reinterpret_cast<float4*>(s_x + i) = v;
-      ss = fmaf(v.x, v.x, ss);
-      ss = fmaf(v.y, v.y, ss);
-      ss = fmaf(v.z, v.z, ss);
-      ss = fmaf(v.w, v.w, ss);
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
     }
+    float rstd = 1.0f;
     if (ly.gamma) {
       ss = warp_sum(ss);
       if (lane == 0) s_red[warp] = ss;
-      __syncthreads();
+    }
+    __syncthreads();
+    if (ly.gamma) {
       float tot = 0.0f;
 #pragma unroll
       for (int w = 0; w < kFW; ++w) tot += s_red[w];
-      const float rstd = 1.0f / sqrtf(tot / (float)H + ly.eps);
-      for (int i = tid; i < H; i += kFT) s_x[i] = s_x[i] * rstd * ly.gamma[i];
+      rstd = 1.0f / sqrtf(tot / (float)H + ly.eps);
+    }
+    // Pass 2: lane l of a warp owns block (base + l) of 16 elements; the four
+    // blocks of a group of 64 sit on four neighbouring lanes.
+    const int NB = H / 16;
+#pragma unroll 1
+    for (int base = warp * 32; base < NB; base += kFT) {
+      const int blk = base + lane;
+      const bool act = blk < NB;
+      float xv[16];
+      if (act) {
+        const float4* xs4 = reinterpret_cast<const float4*>(s_x + blk * 16);
+        float4 v[4] = {xs4[0], xs4[1], xs4[2], xs4[3]};
+        if (ly.gamma) {
+          const float4* gp = reinterpret_cast<const float4*>(ly.gamma + blk * 16);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float4 g = __ldg(gp + k);
+            v[k] = make_float4(v[k].x * rstd * g.x, v[k].y * rstd * g.y, v[k].z * rstd * g.z, v[k].w * rstd * g.w);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          xv[4 * k] = v[k].x;
+          xv[4 * k + 1] = v[k].y;
+          xv[4 * k + 2] = v[k].z;
+          xv[4 * k + 3] = v[k].w;
+        }
+        float4* xo = reinterpret_cast<float4*>(s_x + blk * 16);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) xo[k] = v[k];
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) xv[k] = 0.0f;
+      }
+      xq_quantize_block16<BITS>(xv, blk >> 2, blk & 3, NGH, s_xl, s_xcs, act);
     }
     __syncthreads();
-    for (int g = warp; g < NGH; g += kFW) {
-      const float2 v = reinterpret_cast<const float2*>(s_x + g * kGroup)[lane];
-      xq_quantize_group<BITS>(v.x, v.y, g, NGH, s_xl, s_xcs);
-    }
 
-    // ---- router rows: logits of this CTA's rows (8 warp segments per row, fixed order)
+    // ---- router rows: logits of this CTA's rows.  Warp w sums segment w (H/8
+    // columns) of every row of a staged item; the 8 segments add in fixed order.
     int j = 0;
     for (; j < n_rt; ++j) {
       const int bi = j % nbuf;
       if (!mbar_wait_bounded(smem_addr(&s_full[bi]), (ph >> bi) & 1u, p.err)) ok = false;
       ph ^= 1u << bi;
       const Item it = s_item[j];
-      const uint16_t* wr = reinterpret_cast<const uint16_t*>(ring + (size_t)bi * chb);
-      const int seg = H / 8;
+      const uint16_t* wr = reinterpret_cast<const uint16_t*>(ring + (size_t)bi * chb) + warp * (H / 8);
+      const float* xs = s_x + warp * (H / 8);
       float* part = s_rpart[j & 1];
-      for (int task = warp; ok && task < it.rows * 8; task += kFW) {
-        const int r = task >> 3, sg = task & 7;
-        const uint4* wv = reinterpret_cast<const uint4*>(wr + (size_t)r * H + sg * seg);
-        const float* xv = s_x + sg * seg;
-        float acc = 0.0f;
-        for (int k = lane; k < seg / 8; k += 32) {
-          const uint4 w = wv[k];
-          const float4 xa = *reinterpret_cast<const float4*>(xv + 8 * k);
-          const float4 xb = *reinterpret_cast<const float4*>(xv + 8 * k + 4);
-          acc = fmaf(__uint_as_float(w.x << 16), xa.x, acc);
-          acc = fmaf(__uint_as_float(w.x & 0xFFFF0000u), xa.y, acc);
-          acc = fmaf(__uint_as_float(w.y << 16), xa.z, acc);
-          acc = fmaf(__uint_as_float(w.y & 0xFFFF0000u), xa.w, acc);
-          acc = fmaf(__uint_as_float(w.z << 16), xb.x, acc);
-          acc = fmaf(__uint_as_float(w.z & 0xFFFF0000u), xb.y, acc);
-          acc = fmaf(__uint_as_float(w.w << 16), xb.z, acc);
-          acc = fmaf(__uint_as_float(w.w & 0xFFFF0000u), xb.w, acc);
+      float acc[kFusedMaxRtRows];
+#pragma unroll
+      for (int r = 0; r < kFusedMaxRtRows; ++r) acc[r] = 0.0f;
+#pragma unroll 1
+      for (int k = lane; ok && k < H / 64; k += 32) {  // 8 columns per step
+        const float4 xa = *reinterpret_cast<const float4*>(xs + 8 * k);
+        const float4 xb = *reinterpret_cast<const float4*>(xs + 8 * k + 4);
+#pragma unroll
+        for (int r = 0; r < kFusedMaxRtRows; ++r) {
+          if (r < it.rows) {
+            const uint4 w = *reinterpret_cast<const uint4*>(wr + (size_t)r * H + 8 * k);
+            float a = acc[r];
+            a = fmaf(__uint_as_float(w.x << 16), xa.x, a);
+            a = fmaf(__uint_as_float(w.x & 0xFFFF0000u), xa.y, a);
+            a = fmaf(__uint_as_float(w.y << 16), xa.z, a);
+            a = fmaf(__uint_as_float(w.y & 0xFFFF0000u), xa.w, a);
+            a = fmaf(__uint_as_float(w.z << 16), xb.x, a);
+            a = fmaf(__uint_as_float(w.z & 0xFFFF0000u), xb.y, a);
+            a = fmaf(__uint_as_float(w.w << 16), xb.z, a);
+            a = fmaf(__uint_as_float(w.w & 0xFFFF0000u), xb.w, a);
+            acc[r] = a;
+          }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) part[task] = acc;
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int r = 0; r < kFusedMaxRtRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+      if (lane == 0)
+#pragma unroll
+        for (int r = 0; r < kFusedMaxRtRows; ++r)
+          if (r < it.rows) part[r * 8 + warp] = acc[r];
       __syncthreads();
       if (tid < it.rows) {
         float lg = 0.0f;
@@ -331,7 +481,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     __syncthreads();
     if (s_abort) break;
     unsigned gen_a = 0;
-    if (tid == 0) gen_a = grid_arrive(p.bar_cnt, p.bar_gen, P);
+    if (tid == kBarT) gen_a = grid_arrive(p.bar_cnt, p.bar_gen, P);
 
     // ---- this lane's digits of x, for every gate/up row of the step
     uint32_t L[48];
@@ -344,25 +494,69 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       csx = s_xcs[xg];
     }
 
-    // gate/up of one staged item: partial sums per (k-part, row) into s_gpart, then SwiGLU.
-    auto gateup_item = [&](int jj) {
-      const int bi = jj % nbuf;
+    // ---- gate/up of every staged item of the step: the shared expert's first
+    // (while the other CTAs finish their logits), then, after barrier A and the
+    // routing, the routed experts'.  Warp-level tasks (k-part, row pass) leave
+    // partial sums in s_gacc; warps move on independently, and the last warp
+    // done with a buffer refills it.
+    bool stop = false;
+    for (;; ++j) {
+      if (j == n_const) {
+        // ---- barrier A, then the routing (each CTA selects the experts itself)
+        if (tid == kBarT && !grid_wait(p.bar_gen, gen_a, p.err)) s_abort = 1;
+        if (!ok) s_abort = 1;
+        __syncthreads();
+        if (s_abort) {
+          stop = true;
+          break;
+        }
+        if (E <= kFW * 64) {
+          topk_stage1(p.logits, E, K, s_cand);
+          __syncthreads();
+          if (warp == 0) topk_stage2(p.logits, E, K, s_cand, s_idx, s_w);
+        } else if (warp == 0) {
+          topk_any(p.logits, E, K, s_idx, s_w);
+        }
+        __syncthreads();
+        // routed gate/up rows into every buffer (all consumed by now): item i by
+        // lane 0 of warp 1 + i % 7, so the copies go out from several warps at once
+        if (lane == 0 && warp > 0) {
+          fence_proxy_async();
+          for (int jj = n_const + warp - 1; jj < n_items && jj < n_const + nbuf; jj += kFW - 1) issue_item(jj, ly);
+        }
+        if (warp == 0) {
+          if (b == 0 && lane < K && p.idx_out) p.idx_out[(size_t)t * K + lane] = s_idx[lane];
+          if (b == 0 && lane < K && p.w_out) p.w_out[(size_t)t * K + lane] = s_w[lane];
+          // routed down rows: one slot per lane of warp 0
+          if (nd > 0 && lane < K) {
+            if (lane == 0) {
+              s_dnstate = 2;
+              mbar_expect_tx(smem_addr(&s_dnbar), (uint32_t)K * nd * (RBd + 2 * SBd));
+            }
+            __syncwarp(0xffffffffu >> (32 - K));
+            issue_down(lane, ly.routed + (long long)s_idx[lane] * ly.stride);
+          }
+        }
+      }
+      if (j >= n_items) break;
+      const int limit = j < n_const ? n_const : n_items;
+      const int bi = j % nbuf;
       if (!mbar_wait_bounded(smem_addr(&s_full[bi]), (ph >> bi) & 1u, p.err)) ok = false;
       ph ^= 1u << bi;
-      const Item it = s_item[jj];
+      const Item it = s_item[j];
       const uint8_t* buf = ring + (size_t)bi * chb;
-      float* part = s_gpart[jj & 1];
-      for (int pass = warp / KS; ok && pass * RPP < it.rows; pass += kFW / KS) {
-        const int r = pass * RPP + gsub;
+      const int ntask = (it.rows + RPP - 1) / RPP * KS;
+#pragma unroll 1
+      for (int task = warp; ok && task < ntask; task += kFW) {
+        const int r = (task / KS) * RPP + gsub;
         float ag = 0.0f, au = 0.0f;
         if (r < it.rows) {
-          uint4 q0, q1, v0, v1;
           const uint8_t* gr = buf + (size_t)r * RB + xg * (kGroup * BITS / 8);
           const uint8_t* ur = gr + (size_t)CU * RB;
-          q0 = *reinterpret_cast<const uint4*>(gr);
-          q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(gr + 16) : q0;
-          v0 = *reinterpret_cast<const uint4*>(ur);
-          v1 = BITS == 4 ? *reinterpret_cast<const uint4*>(ur + 16) : v0;
+          const uint4 q0 = *reinterpret_cast<const uint4*>(gr);
+          const uint4 q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(gr + 16) : q0;
+          const uint4 v0 = *reinterpret_cast<const uint4*>(ur);
+          const uint4 v1 = BITS == 4 ? *reinterpret_cast<const uint4*>(ur + 16) : v0;
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * (size_t)CU * RB + (size_t)r * SB);
           const int cs2 = CU * SB / 2;
           const float gs = bf16_to_f32(sc[xg]), gb = bf16_to_f32(sc[cs2 + xg]);
@@ -377,75 +571,42 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
           au += __shfl_xor_sync(0xffffffffu, au, o);
         }
         if (gl == 0 && r < it.rows) {
-          part[(kap * kFusedMaxChunkRows + r) * 2] = ag;
-          part[(kap * kFusedMaxChunkRows + r) * 2 + 1] = au;
+          s_gacc[((it.rbase + r) * 4 + kap) * 2] = ag;
+          s_gacc[((it.rbase + r) * 4 + kap) * 2 + 1] = au;
         }
       }
-      __syncthreads();  // every warp is done with the buffer and the partial sums are complete
-      if (tid < it.rows) {
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&s_cnt[bi], 1) == kFW - 1) {
+          s_cnt[bi] = 0;
+          __threadfence_block();
+          s_pend[bi] = 0;
+          if (ok && j + nbuf < limit) {
+            fence_proxy_async();
+            issue_item(j + nbuf, ly);
+          }
+        }
+      }
+    }
+    if (stop) break;
+    __syncthreads();  // every partial sum of the step is in s_gacc
+    // SwiGLU of every gate/up row of this CTA: silu(g) * u with silu(z) = z / (1 + exp(-z))
+    for (int jj = n_rt + warp; jj < n_items; jj += kFW) {
+      const Item it = s_item[jj];
+      if (lane < it.rows) {
         float g = 0.0f, u = 0.0f;
         for (int k = 0; k < KS; ++k) {
-          g += part[(k * kFusedMaxChunkRows + tid) * 2];
-          u += part[(k * kFusedMaxChunkRows + tid) * 2 + 1];
+          g += s_gacc[((it.rbase + lane) * 4 + k) * 2];
+          u += s_gacc[((it.rbase + lane) * 4 + k) * 2 + 1];
         }
-        p.act[(size_t)it.slot * I + it.row0 + tid] = g / (1.0f + expf(-g)) * u;
-      }
-      if (tid == 0) s_pend[bi] = 0;
-    };
-
-    // ---- shared expert's gate/up while the other CTAs finish their logits
-    for (; j < n_const; ++j) {
-      gateup_item(j);
-      if (tid == 0 && ok && j + nbuf < n_const) {  // more routing-independent rows than buffers
-        fence_proxy_async();
-        issue_item(j + nbuf, ly);
+        p.act[(size_t)it.slot * I + it.row0 + lane] = g / (1.0f + expf(-g)) * u;
       }
     }
 
-    // ---- barrier A, then the routing (each CTA selects the experts itself)
-    if (tid == 0 && !grid_wait(p.bar_gen, gen_a, p.err)) s_abort = 1;
-    if (!ok) s_abort = 1;
-    __syncthreads();
-    if (s_abort) break;
-    if (warp == 0) {
-      int ik;
-      float wk, sig;
-      warp_topk(p.logits, E, K, 1, ik, wk, sig);
-      if (ik < 0 || ik >= E) ik = 0;
-      if (lane < K) {
-        s_idx[lane] = ik;
-        s_w[lane] = wk;
-        if (b == 0 && p.idx_out) p.idx_out[(size_t)t * K + lane] = ik;
-        if (b == 0 && p.w_out) p.w_out[(size_t)t * K + lane] = wk;
-      }
-      if (lane == 0) s_w[K] = sig;
-      __syncwarp();
-      // routed gate/up rows into every buffer (all consumed by now), one item per lane
-      fence_proxy_async();
-      for (int jj = n_const + lane; jj < n_items && jj < n_const + nbuf; jj += 32) issue_item(jj, ly);
-      // routed down rows: one slot per lane
-      if (nd > 0 && lane < K) {
-        if (lane == 0) {
-          s_dnstate = 2;
-          mbar_expect_tx(smem_addr(&s_dnbar), (uint32_t)K * nd * (RBd + 2 * SBd));
-        }
-        __syncwarp(0xffffffffu >> (32 - K));
-        issue_down(lane, ly.routed + (long long)s_idx[lane] * ly.stride);
-      }
-    }
-    __syncthreads();
-
-    // ---- routed gate/up through the ring
-    for (; j < n_items; ++j) {
-      gateup_item(j);
-      if (tid == 0 && ok && j + nbuf < n_items) {
-        fence_proxy_async();
-        issue_item(j + nbuf, ly);
-      }
-    }
-
-    // ---- activation groups of 64: the CTA that completes a group writes its digits
-    __threadfence();
+    // ---- activation groups of 64: the CTA that completes a group writes its digits.
+    // Counting threads (warps 1..7) fence after the block barrier, which orders
+    // every act write of the CTA before their counts.
     if (!ok) s_abort = 1;
     __syncthreads();
     if (s_abort) break;
@@ -453,24 +614,26 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     const int gs0 = sh0 / kGroup, gs1 = sh1 > sh0 ? (sh1 - 1) / kGroup + 1 : gs0;
     const int gr0 = rf0 / kGroup, gr1 = rf1 > rf0 ? (rf1 - 1) / kGroup + 1 : gr0;
     const int ngs = gs1 - gs0, ngt = ngs + (gr1 - gr0);
-    if (tid < ngt) {
+    const int gt = tid - 32;  // counting thread's group
+    if (gt >= 0 && gt < ngt) {
       int fg, lo, hi;  // flat group over slot-major rows, and this CTA's rows in it
-      if (tid < ngs) {
-        const int g = gs0 + tid;
+      __threadfence();
+      if (gt < ngs) {
+        const int g = gs0 + gt;
         fg = K * NGI + g;
         lo = max(sh0, g * kGroup);
         hi = min(sh1, (g + 1) * kGroup);
       } else {
-        const int g = gr0 + tid - ngs;
+        const int g = gr0 + gt - ngs;
         fg = g;
         lo = max(rf0, g * kGroup);
         hi = min(rf1, (g + 1) * kGroup);
       }
       const unsigned prev = atomicAdd(&p.grp_cnt[fg], (unsigned)(hi - lo));
-      s_gdone[tid] = prev + (unsigned)(hi - lo) == (unsigned)kGroup ? fg + 1 : 0;
+      s_gdone[gt] = prev + (unsigned)(hi - lo) == (unsigned)kGroup ? fg + 1 : 0;
     }
     __syncthreads();
-    for (int k = warp; k < ngt; k += kFW) {
+    for (int k = warp - 1; warp > 0 && k < ngt; k += kFW - 1) {
       const int fg1 = s_gdone[k];
       if (!fg1) continue;
       __threadfence();
@@ -479,8 +642,8 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       xq_quantize_group<BITS>(v.x, v.y, gg, NGI, p.act_limbs + (size_t)slot * NGI * kGroupWords * 4,
                               p.act_cs + (size_t)slot * ncd);
       if (lane == 0) p.grp_cnt[fg] = 0u;
+      __threadfence();
     }
-    __threadfence();
     __syncthreads();
 
     // ---- the next step's routing-independent rows, into the drained ring
@@ -491,7 +654,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     }
 
     // ---- barrier B, then down + combine from shared memory
-    if (tid == 0) {
+    if (tid == kBarT) {
       const unsigned gb = grid_arrive(p.bar_cnt, p.bar_gen, P);
       if (!grid_wait(p.bar_gen, gb, p.err)) s_abort = 1;
       if (!s_abort) {
@@ -529,21 +692,34 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       }
       const float wq = qon ? s_w[qslot] : 0.0f;
       const uint8_t* sb = dn + (size_t)qslot * dn_slot;
-      for (int pass = warp / KSd; ok && pass * RPPd < nd; pass += kFW / KSd) {
-        const int r = pass * RPPd + dsub;
-        float acc = 0.0f;
-        if (qon && r < nd) {
-          const uint8_t* cr = sb + (size_t)r * RBd + qg * (kGroup * BITS / 8);
-          const uint4 q0 = *reinterpret_cast<const uint4*>(cr);
-          const uint4 q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(cr + 16) : q0;
-          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * RBd + (size_t)r * SBd)[qg]);
-          const float bi =
-              bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * (RBd + SBd) + (size_t)r * SBd)[qg]);
-          const float Sd = group_dot<BITS>(q0, q1, A);
-          acc = wq * fmaf(sc, csa.x * Sd, bi * csa.y);
+      // four row slots per pass: independent dot products, then one interleaved reduction
+      const uint16_t* scl = reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * RBd);
+      const uint16_t* bsl = reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * (RBd + SBd));
+      for (int pass = warp / KSd; ok && pass * 4 * RPPd < nd; pass += kFW / KSd) {
+        float acc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = (pass * 4 + u) * RPPd + dsub;
+          acc[u] = 0.0f;
+          if (qon && r < nd) {
+            const uint8_t* cr = sb + (size_t)r * RBd + qg * (kGroup * BITS / 8);
+            const uint4 q0 = *reinterpret_cast<const uint4*>(cr);
+            const uint4 q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(cr + 16) : q0;
+            const float sc = bf16_to_f32(scl[(size_t)r * NGI + qg]);
+            const float bi = bf16_to_f32(bsl[(size_t)r * NGI + qg]);
+            const float Sd = group_dot<BITS>(q0, q1, A);
+            acc[u] = wq * fmaf(sc, csa.x * Sd, bi * csa.y);
+          }
         }
-        for (int o = LPRd / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (dl == 0 && r < nd) s_dpart[kapd * kFusedMaxDnRows + r] = acc;
+        for (int o = LPRd / 2; o > 0; o >>= 1)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+        if (dl == 0)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = (pass * 4 + u) * RPPd + dsub;
+            if (r < nd) s_dpart[kapd * kFusedMaxDnRows + r] = acc[u];
+          }
       }
     }
     __syncthreads();
@@ -554,9 +730,8 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     }
     // the next step reads this step's output when it is the next layer of a stack
     if (s + 1 < S && (s + 1) % p.L != 0) {
-      __threadfence();
       __syncthreads();
-      if (tid == 0) gen_c = grid_arrive(p.bar_cnt, p.bar_gen, P);
+      if (tid == kBarT) gen_c = grid_arrive(p.bar_cnt, p.bar_gen, P);
       wait_c = true;
     }
     __syncthreads();  // shared memory of this step (DN, XD) is free
@@ -605,7 +780,7 @@ FusedPlan plan_fused(int bits, int H, int I, int E, int K) {
   pl.chb = ((cu * pair) + 127) / 128 * 128;
   if (pl.chb < H * 2) pl.chb = (H * 2 + 127) / 128 * 128;  // at least one router row per buffer
   int rt = pl.chb / (H * 2);
-  pl.rt_rows = rt > 8 ? 8 : rt;
+  pl.rt_rows = rt > kFusedMaxRtRows ? kFusedMaxRtRows : rt;
   const long long budget = kFusedSmemBudget - pl.ring_off;
   if (budget < 2LL * pl.chb) return pl;
   int nbuf = (int)(budget / pl.chb);
@@ -620,6 +795,8 @@ FusedPlan plan_fused(int bits, int H, int I, int E, int K) {
   // activation groups counted per CTA must fit s_gdone
   const int gcount = ((I / pl.ru + P - 1) / P * pl.ru) / kGroup + 2 + ((K * I / pl.ru + P - 1) / P * pl.ru) / kGroup + 2;
   if (gcount > 64) return pl;
+  const int gu_rows = (I / pl.ru + P - 1) / P * pl.ru + (K * I / pl.ru + P - 1) / P * pl.ru;
+  if (gu_rows > kFusedMaxGuRows || (NGH >= 32 && NGH / 32 > 4)) return pl;
   pl.ok = true;
   return pl;
 }
