@@ -27,6 +27,9 @@ import numpy as np  # noqa: E402
 
 METRIC = "MoE-layer decode tokens/s and effective weight GB/s (fraction of HBM peak), 1×B200"
 FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gate/up launch,
+# from one ncu capture of the current gateup_kernel per workload; None where none was taken.
+GATEUP_TRAFFIC = {"qwen397-4bit": 31243264}
 
 WORKLOADS = {
     # name: (spec factory, description)
@@ -322,7 +325,7 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "effective_gbs": eff, "frac_of_peak": eff / peak, "bytes_per_token": bytes_tok,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": None, "kernel": "gateup_kernel", "peak_kind": peak_kind,
+                         "traffic": GATEUP_TRAFFIC.get(args.workload), "kernel": "gateup_kernel", "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": gateup_bytes},
             "kernels_us": {"router": router_us, "gateup": gateup_us, "down": down_us},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * steps,

@@ -40,13 +40,15 @@ bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
 // Workspace regions (byte offsets), in this order.
 struct WsLayout {
-  size_t ctrl, xq_limbs, xq_cs, logits, route_idx, route_w, act, act_limbs, act_cs, grp_cnt, total;
+  size_t ctrl, xq_limbs, xq_cs, logits, route_idx, route_w, act, act_limbs, act_cs, grp_cnt, xlog, xact, xh, total;
 };
 
 // Workspace: control words, digits of x (3 bytes per element + one float2 per
 // chunk of at most 32 elements), router logits [T][E+1], the routing [T][K]
 // and weights [T][K+1], the activations of the K+1 expert slots with their
-// digits, and per-group completion counters.
+// digits, per-group completion counters, and the single-kernel path's
+// epoch-tagged exchange words (8 bytes each, two copies): logits [E+1],
+// activations [(K+1) I] and a stacked layer's output [H].
 WsLayout layout(int H, int E, int K, int I, int T) {
   WsLayout L;
   const size_t ne = (size_t)K + 1;
@@ -60,7 +62,10 @@ WsLayout layout(int H, int E, int K, int I, int T) {
   L.act_limbs = L.act + up(ne * I * 4);
   L.act_cs = L.act_limbs + up(ne * 3 * I);
   L.grp_cnt = L.act_cs + up(ne * (I / 32) * 8);
-  L.total = L.grp_cnt + up(ne * (I / 64 > 0 ? I / 64 : 1) * 4);
+  L.xlog = L.grp_cnt + up(ne * (I / 64 > 0 ? I / 64 : 1) * 4);
+  L.xact = L.xlog + up(2 * (size_t)(E + 1) * 8);
+  L.xh = L.xact + up(2 * ne * I * 8);
+  L.total = L.xh + up(2 * (size_t)H * 8);
   return L;
 }
 
@@ -445,13 +450,10 @@ static fmoe_status run_fused(const fmoe_layer* layers, int nl, const float* h, i
   p.out = out;
   p.idx_out = idx_out;
   p.w_out = w_out;
-  p.logits = reinterpret_cast<float*>(base + L.logits);
-  p.act = reinterpret_cast<float*>(base + L.act);
-  p.act_limbs = base + L.act_limbs;
-  p.act_cs = reinterpret_cast<float2*>(base + L.act_cs);
-  p.grp_cnt = reinterpret_cast<unsigned*>(base + L.grp_cnt);
-  p.bar_cnt = &ctrl->grid_count;
-  p.bar_gen = &ctrl->grid_gen;
+  p.xlog = reinterpret_cast<unsigned long long*>(base + L.xlog);
+  p.xact = reinterpret_cast<unsigned long long*>(base + L.xact);
+  p.xh = reinterpret_cast<unsigned long long*>(base + L.xh);
+  p.epoch = &ctrl->epoch;
   p.err = err_word ? err_word : &ctrl->err;
   p.nbuf = pl.nbuf;
   p.chb = pl.chb;

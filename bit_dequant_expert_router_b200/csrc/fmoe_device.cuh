@@ -16,11 +16,9 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // bound on any device-si
 
 // Control words at the start of every workspace.
 struct WsControl {
-  unsigned int tickets[960];   // last-CTA tickets, one per token
-  unsigned int grid_count;     // grid barrier of the single-kernel path: arrivals ...
+  unsigned int tickets[992];   // last-CTA tickets, one per token
+  unsigned int epoch;          // single-kernel path: steps run on this workspace (its own 128-byte line)
   unsigned int pad0[31];
-  unsigned int grid_gen;       // ... and generation (its own 128-byte line)
-  unsigned int pad1[31];
   int err;                     // nonzero once a bounded wait gave up
   int pad[63];
 };

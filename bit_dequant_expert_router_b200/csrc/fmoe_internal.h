@@ -98,13 +98,12 @@ struct FusedParams {
   float* out;                            // [T][H] output of the last layer (also the stack's running state)
   int32_t* idx_out;                      // [T][K] or NULL (single-layer calls)
   float* w_out;
-  float* logits;                         // workspace: [E+1]
-  float* act;                            // [(K+1)][I]
-  uint8_t* act_limbs;                    // [(K+1)][3I] digits of act
-  float2* act_cs;                        // [(K+1)][I*bits/128]
-  unsigned* grp_cnt;                     // [(K+1)][I/64], zero between calls
-  unsigned* bar_cnt;                     // grid barrier words, zero before first use
-  unsigned* bar_gen;
+  // workspace: epoch-tagged exchange words {value (low 32 bits), epoch (high 32 bits)},
+  // two copies each (step parity), zero before first use
+  unsigned long long* xlog;              // [2][E+1] router logits (+ the shared-gate logit)
+  unsigned long long* xact;              // [2][(K+1)*I] SwiGLU activations, slot-major
+  unsigned long long* xh;                // [2][H] a stacked layer's output, the next layer's input
+  unsigned* epoch;                       // steps run on this workspace so far
   int* err;
   int nbuf, chb, cu, rt_rows, ru, rd, dn_rows_max, dn_slot_bytes, dn_off, ring_off;
 };

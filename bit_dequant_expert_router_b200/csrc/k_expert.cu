@@ -179,6 +179,9 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
         }
       }
     }
+    // The other lanes wait here rather than spin on the digits' barrier, which
+    // would share the warp's issue slots with lane 0's copy issue.
+    __syncwarp();
   }
 
   // This lane's groups and their digits of x, for the whole kernel.
@@ -387,6 +390,7 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
     bulk_g2s(smem_addr(sm), p.act_limbs, (uint32_t)dwords * 4, bx, l2_policy_evict_first());
     bulk_g2s(smem_addr(sm + (size_t)dwords * 4), p.act_cs, (uint32_t)(NE * NCH * 8), bx, l2_policy_evict_first());
   }
+  __syncwarp();  // lanes 1..31 of warp 0 wait for the issue instead of spinning beside it
 
   // This lane's (slot, group) pairs and their digits.
   uint32_t L[PPL][48];

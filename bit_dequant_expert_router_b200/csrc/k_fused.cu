@@ -6,20 +6,27 @@
 // ("What is Flash-MoE" (a2a-mcp.org), MoE section and sections 2-3; the
 // per-layer pipeline of the "Flash-MoE" wiki summary (jeongsk)).  The pages run
 // these as separate GPU dispatches with the top-K on the CPU in between; here
-// one CTA per SM carries every step of a sequence, and the data dependencies
-// between the block's phases become grid-wide barriers in global memory:
+// one CTA per SM carries every step of a sequence.
 //
-//   A: every CTA's router logits are written      -> each CTA selects the experts itself
-//   B: every SwiGLU activation group is quantised -> down projection
-//   C: every output row of the step is written    -> the next step reads it (stacked layers only)
+// A step has three all-to-all exchanges between CTAs: the router logits (each
+// CTA computes a few rows, every CTA needs all of them for the top-K), the
+// SwiGLU activations (every CTA needs all of them for its down rows) and, in a
+// stack of layers, the output vector (the next layer's input).  Each goes
+// through a workspace array of 8-byte words {value, epoch}: the producer stores
+// the word once, consumers poll until the epoch of the step appears.  The word
+// is a single 64-bit access, so a matching epoch is its own proof that the
+// value is current: no grid barrier, counter or memory fence is on the path.
+// Arrays alternate by step parity; a CTA cannot run two steps ahead of another
+// (each step consumes data of every CTA), so two copies suffice.  Epochs are a
+// per-workspace count of steps (WsControl::epoch), advanced by CTA 0 on exit.
 //
 // The bytes of a step fall into two kinds.  The router rows, the shared
 // expert's gate/up rows and the shared expert's down rows do not depend on the
 // routing, so a CTA requests its share of them for step s+1 as soon as its
-// gate/up work of step s is done, and for step s+1 that data is already in
-// shared memory.  The routed experts' gate/up rows stream through a ring of
-// chunk buffers, and their down rows land in a separate region while gate/up is
-// still running, so the down phase after barrier B computes from shared memory.
+// gate/up work of step s is done.  The routed experts' gate/up rows stream
+// through a ring of chunk buffers, and their down rows land in a separate
+// region while gate/up is still running, so the down phase computes from
+// shared memory.
 //
 // Dot products use the per-group fold of fmoe_device.cuh:
 //   sum_c (q_c s + b) x_c = s * sum_c q_c x_c + b * sum_c x_c
@@ -31,54 +38,49 @@ namespace {
 
 constexpr int kFW = kFusedWarps;
 constexpr int kFT = kFW * 32;
-// A gpu-scope fence or release operation waits for every bulk copy that its own
-// thread still has in flight (measured on B200: about a microsecond with a 64 KiB
-// copy outstanding; a fence in another warp, or a CTA-scope fence, returns at
-// once).  Warp 0 issues the long-lived copies (routed down rows, the next step's
-// rows), so grid barriers run on thread kBarT of warp 1 and the release fences on
-// warps 1..7, never on warp 0.
-constexpr int kBarT = 32;
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+// ---- epoch-tagged words: low 32 bits the value, high 32 bits the epoch
+__device__ __forceinline__ void st_tagged(unsigned long long* p, float v, unsigned ep) {
+  const unsigned long long w = ((unsigned long long)ep << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 
-__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void ld_tagged2(const unsigned long long* p, unsigned long long& a, unsigned long long& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
 
-// Grid barrier by generation count.  Thread 0 only, after a __syncthreads()
-// that orders the CTA's writes.  Arrive returns the generation to wait on;
-// the last CTA to arrive resets the count and publishes the next generation.
-__device__ __forceinline__ unsigned grid_arrive(unsigned* cnt, unsigned* gen, unsigned P) {
-  const unsigned g = ld_acquire_u32(gen);
-  __threadfence();
-  const unsigned old = atomicAdd(cnt, 1u);
-  if (old == P - 1) {
-    atomicExch(cnt, 0u);
-    __threadfence();
-    st_release_u32(gen, g + 1);
-  }
-  return g;
+__device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
+  unsigned long long a;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(a) : "l"(p) : "memory");
+  return a;
 }
 
-// Waits (at most kWaitNs) until the generation moves past g.
-__device__ __forceinline__ bool grid_wait(const unsigned* gen, unsigned g, int* err) {
-  bool ok = true;
-  if (ld_acquire_u32(gen) == g) {
-    const unsigned long long t0 = global_ns();
-    while (ld_acquire_u32(gen) == g) {
-      if (global_ns() - t0 > kWaitNs) {
-        atomicExch(err, kDevTimeout);
-        ok = false;
-        break;
-      }
+__device__ __forceinline__ unsigned tag_of(unsigned long long w) { return (unsigned)(w >> 32); }
+__device__ __forceinline__ float val_of(unsigned long long w) { return __uint_as_float((unsigned)w); }
+
+// Polls n (even, 16-byte aligned) tagged words until all carry epoch ep; the
+// values go to v[0..n).  Bounded by kWaitNs; false (and the error word set) on timeout.
+template <int N>
+__device__ __forceinline__ bool poll_tagged(const unsigned long long* p, unsigned ep, float (&v)[N], int* err) {
+  unsigned long long t0 = 0;
+  for (;;) {
+    bool all = true;
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+      unsigned long long a, b;
+      ld_tagged2(p + i, a, b);
+      all = all && tag_of(a) == ep && tag_of(b) == ep;
+      v[i] = val_of(a);
+      v[i + 1] = val_of(b);
     }
+    if (all) return true;
+    if (t0 == 0) t0 = global_ns();
+    else if (global_ns() - t0 > kWaitNs) {
+      atomicExch(err, kDevTimeout);
+      return false;
+    }
+    __nanosleep(64);  // back off: polling loads compete with the copies and loads of other warps
   }
-  __threadfence();
-  return ok;
 }
 
 struct Item {
@@ -132,17 +134,34 @@ __device__ __noinline__ void issue_down_dev(uint8_t* base, uint32_t bar, const u
            pol);
 }
 
-// Routing of one token from its logits [E] (+ the shared-gate logit at E), E <= 512:
-// stage 1, every warp w takes the K largest keys of its slice of ceil(E/8)
-// logits (two per lane) into cand[w*K + k]; stage 2 (after a block barrier),
-// warp 0 takes the K largest of the 8K candidates.  Keys order by value, then
-// by lower index (topk_key), so the result is that of one sort of all E.
-__device__ __forceinline__ void topk_stage1(const float* logits, int E, int K, unsigned long long* cand) {
+// Routing of one token from its tagged logits [E] (+ the shared-gate logit at
+// E), E <= 8 * 64: stage 1, every warp w takes the K largest keys of its slice
+// of ceil(E/8) logits (two per lane) into cand[w*K + k]; stage 2 (after a block
+// barrier), warp 0 takes the K largest of the 8K candidates.  Keys order by
+// value, then by lower index (topk_key), so the result is that of one sort of
+// all E.  Returns false if the logits did not arrive in time.
+__device__ __forceinline__ bool topk_stage1(const unsigned long long* logits, unsigned ep, int E, int K,
+                                            unsigned long long* cand, int* err) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ES = (E + kFW - 1) / kFW;
   const int e0 = warp * ES + lane, e1 = e0 + 32;
-  unsigned long long k0 = (lane < ES && e0 < E) ? topk_key(__ldcg(logits + e0), e0) : 0ull;
-  unsigned long long k1 = (lane + 32 < ES && e1 < E) ? topk_key(__ldcg(logits + e1), e1) : 0ull;
+  const bool h0 = lane < ES && e0 < E, h1 = lane + 32 < ES && e1 < E;
+  unsigned long long w0 = 0, w1 = 0, t0 = 0;
+  bool ok = true;
+  for (;;) {
+    if (h0) w0 = ld_tagged(logits + e0);
+    if (h1) w1 = ld_tagged(logits + e1);
+    if ((!h0 || tag_of(w0) == ep) && (!h1 || tag_of(w1) == ep)) break;
+    if (t0 == 0) t0 = global_ns();
+    else if (global_ns() - t0 > kWaitNs) {
+      atomicExch(err, kDevTimeout);
+      ok = false;
+      break;
+    }
+    __nanosleep(64);
+  }
+  unsigned long long k0 = h0 ? topk_key(val_of(w0), e0) : 0ull;
+  unsigned long long k1 = h1 ? topk_key(val_of(w1), e1) : 0ull;
 #pragma unroll 1
   for (int k = 0; k < K; ++k) {
     const unsigned long long m = warp_max_key(k0 > k1 ? k0 : k1);
@@ -150,12 +169,13 @@ __device__ __forceinline__ void topk_stage1(const float* logits, int E, int K, u
     k0 = k0 == m ? 0ull : k0;
     k1 = k1 == m ? 0ull : k1;
   }
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Stage 2, warp 0: picks, renormalised weights w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0)
 // and sigma = sigmoid(l_E) into idx[0..K), w[0..K], w[K] = sigma.
-__device__ __noinline__ void topk_stage2(const float* logits, int E, int K, const unsigned long long* cand, int* idx,
-                                         float* w) {
+__device__ __noinline__ bool topk_stage2(const unsigned long long* logits, unsigned ep, int E, int K,
+                                         const unsigned long long* cand, int* idx, float* w, int* err) {
   const int lane = threadIdx.x & 31;
   unsigned long long key[8];
 #pragma unroll
@@ -185,21 +205,22 @@ __device__ __noinline__ void topk_stage2(const float* logits, int E, int K, cons
     idx[lane] = mi;
     w[lane] = wk;
   }
-  if (lane == 0) w[K] = 1.0f / (1.0f + expf(-__ldcg(logits + E)));
-}
-
-// Any E: one warp rescans the logits in memory for each pick.
-__device__ __noinline__ void topk_any(const float* logits, int E, int K, int* idx, float* w) {
-  int ik;
-  float wk, sig;
-  warp_topk_mem(logits, E, K, 1, ik, wk, sig);
-  const int lane = threadIdx.x & 31;
-  if (ik < 0 || ik >= E) ik = 0;
-  if (lane < K) {
-    idx[lane] = ik;
-    w[lane] = wk;
+  bool ok = true;
+  if (lane == 0) {  // the shared-gate logit
+    unsigned long long g = 0, t0 = 0;
+    for (;;) {
+      g = ld_tagged(logits + E);
+      if (tag_of(g) == ep) break;
+      if (t0 == 0) t0 = global_ns();
+      else if (global_ns() - t0 > kWaitNs) {
+        atomicExch(err, kDevTimeout);
+        ok = false;
+        break;
+      }
+    }
+    w[K] = 1.0f / (1.0f + expf(-val_of(g)));
   }
-  if (lane == 0) w[K] = sig;
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 template <int BITS>
@@ -207,7 +228,6 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ __align__(8) uint64_t s_full[kFusedMaxRing];
   __shared__ __align__(8) uint64_t s_dnbar;
-  __shared__ __align__(8) uint64_t s_xbar;
   __shared__ Item s_item[kFusedMaxItems];
   __shared__ int s_pend[kFusedMaxRing];
   __shared__ int s_idx[32];
@@ -218,11 +238,9 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   __shared__ float s_gacc[kFusedMaxGuRows * 4 * 2];  // gate/up partial sums [row][k-part][gate, up]
   __shared__ int s_cnt[kFusedMaxRing];                // warps done with a buffer
   __shared__ float s_dpart[kFusedMaxKS * kFusedMaxDnRows];
-  __shared__ int s_gdone[64];
   __shared__ int s_abort;
   __shared__ int s_nconst, s_nitems;
   __shared__ int s_dnstate;  // down rows of the current step: 0 none in flight, 1 shared issued, 2 all issued
-  __shared__ int s_xstate;   // activation digits in flight
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = gridDim.x, b = blockIdx.x;
@@ -230,7 +248,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   const int NGH = H / kGroup, NGI = I / kGroup;
   const int RB = H * BITS / 8, SB = NGH * 2;        // gate/up row: code bytes, scale bytes
   const int RBd = I * BITS / 8, SBd = NGI * 2;      // down row
-  const int ncd = I * BITS / 128;  // chunk scalars of one activation vector
+  const int ncd = I * BITS / 128;                   // chunk scalars of one activation vector
   const int nbuf = p.nbuf, chb = p.chb, CU = p.cu;
   uint8_t* xd = sm;
   uint8_t* dn = sm + p.dn_off;
@@ -238,6 +256,8 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   float* s_x = reinterpret_cast<float*>(xd);
   uint8_t* s_xl = xd + (size_t)H * 4;
   float2* s_xcs = reinterpret_cast<float2*>(xd + (size_t)H * 4 + (size_t)NGH * kGroupWords * 4);
+  uint8_t* s_al = xd;  // down phase: activation digits of every slot, then their chunk scalars
+  float2* s_acs = reinterpret_cast<float2*>(xd + (size_t)NE * NGI * kGroupWords * 4);
   const uint64_t pol = l2_policy_evict_first();
 
   // ---- this CTA's share of every phase (the same for every step)
@@ -273,11 +293,9 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       s_cnt[i] = 0;
     }
     mbar_init(smem_addr(&s_dnbar), 2);
-    mbar_init(smem_addr(&s_xbar), 1);
     mbar_fence_init();
     s_abort = 0;
     s_dnstate = 0;
-    s_xstate = 0;
   }
   __syncthreads();
   const int n_const = s_nconst, n_items = s_nitems;
@@ -329,13 +347,10 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
         if (s_pend[i]) mbar_wait_bounded(smem_addr(&s_full[i]), (ph >> i) & 1u, p.err);
       if (s_dnstate == 1) mbar_arrive(smem_addr(&s_dnbar));  // the routed half never came
       if (s_dnstate > 0) mbar_wait_bounded(smem_addr(&s_dnbar), (uint32_t)(sp & 1), p.err);
-      if (s_xstate) mbar_wait_bounded(smem_addr(&s_xbar), (uint32_t)(sp & 1), p.err);
     }
   };
 
   const int S = p.T * p.L;
-  unsigned gen_c = 0;
-  bool wait_c = false;
 
   // Step 0's routing-independent rows, before waiting on the previous kernel.
   if (tid == 0) {
@@ -345,35 +360,53 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
   }
   pdl_wait();
   pdl_trigger();  // the next kernel's CTAs start only once every CTA of this grid is running
+  // Epochs of this launch: base + s + 1 for step s.  Every CTA reads the base
+  // here; CTA 0 advances it on exit, after every CTA has consumed its data.
+  const unsigned ep_base = *reinterpret_cast<volatile const unsigned*>(p.epoch);
 
   int s = 0;
   for (; s < S; ++s) {
     const int t = s / p.L, l = s % p.L;
     const FusedLayer& ly = p.layers[l];
+    const unsigned ep = ep_base + (unsigned)s + 1u;
+    const int par = s & 1;
     const float* hin = (l == 0 ? p.h : p.out) + (size_t)t * H;
     float* hout = p.out + (size_t)t * H;
+    unsigned long long* xlog = p.xlog + (size_t)par * (E + 1);
+    unsigned long long* xact = p.xact + (size_t)par * NE * I;
 
     if (s > 0 && tid == 0) issue_shared_down(ly);
-    if (wait_c && tid == kBarT && !grid_wait(p.bar_gen, gen_c, p.err)) s_abort = 1;
-    wait_c = false;
-    __syncthreads();
-    if (s_abort) break;
+    __syncwarp();  // a single lane issuing copies keeps its warp-mates waiting, not spinning beside it
 
     // ---- x = RMSNorm(h) (two passes: sum of squares, then apply) and its digits,
-    // the whole vector in every CTA.  Pass 1 stages h in s_x.
+    // the whole vector in every CTA.  Pass 1 stages h in s_x: the user's input
+    // for the first layer, the previous step's tagged output inside a stack.
     float ss = 0.0f;
+    if (l == 0) {
 #pragma unroll 4
-    for (int i = tid * 4; i < H; i += kFT * 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(hin + i));
-      *reinterpret_cast<float4*>(s_x + i) = v;
-      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+      for (int i = tid * 4; i < H; i += kFT * 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(hin + i));
+        *reinterpret_cast<float4*>(s_x + i) = v;
+        ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+      }
+    } else {
+      const unsigned long long* xh = p.xh + (size_t)(par ^ 1) * H;
+#pragma unroll 1
+      for (int i = tid * 4; i < H; i += kFT * 4) {
+        float v[4];
+        if (!poll_tagged<4>(xh + i, ep - 1u, v, p.err)) ok = false;
+        *reinterpret_cast<float4*>(s_x + i) = make_float4(v[0], v[1], v[2], v[3]);
+        ss = fmaf(v[0], v[0], fmaf(v[1], v[1], fmaf(v[2], v[2], fmaf(v[3], v[3], ss))));
+      }
     }
     float rstd = 1.0f;
     if (ly.gamma) {
       ss = warp_sum(ss);
       if (lane == 0) s_red[warp] = ss;
     }
+    if (!ok) s_abort = 1;
     __syncthreads();
+    if (s_abort) break;
     if (ly.gamma) {
       float tot = 0.0f;
 #pragma unroll
@@ -417,8 +450,9 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     }
     __syncthreads();
 
-    // ---- router rows: logits of this CTA's rows.  Warp w sums segment w (H/8
-    // columns) of every row of a staged item; the 8 segments add in fixed order.
+    // ---- router rows: logits of this CTA's rows, published as tagged words.
+    // Warp w sums segment w (H/8 columns) of every row of a staged item; the 8
+    // segments add in fixed order.
     int j = 0;
     for (; j < n_rt; ++j) {
       const int bi = j % nbuf;
@@ -467,7 +501,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
         for (int sg = 0; sg < 8; ++sg) lg += part[tid * 8 + sg];
         const int row = it.row0 + tid;
         if (row < E && ly.bias) lg += ly.bias[row];
-        p.logits[row] = lg;
+        st_tagged(xlog + row, lg, ep);
       }
       if (tid == 0) {
         s_pend[bi] = 0;
@@ -476,12 +510,8 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
           issue_item(j + nbuf, ly);
         }
       }
+      __syncwarp();
     }
-    if (!ok) s_abort = 1;
-    __syncthreads();
-    if (s_abort) break;
-    unsigned gen_a = 0;
-    if (tid == kBarT) gen_a = grid_arrive(p.bar_cnt, p.bar_gen, P);
 
     // ---- this lane's digits of x, for every gate/up row of the step
     uint32_t L[48];
@@ -495,35 +525,34 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
     }
 
     // ---- gate/up of every staged item of the step: the shared expert's first
-    // (while the other CTAs finish their logits), then, after barrier A and the
-    // routing, the routed experts'.  Warp-level tasks (k-part, row pass) leave
-    // partial sums in s_gacc; warps move on independently, and the last warp
-    // done with a buffer refills it.
+    // (while the other CTAs finish their logits), then, once every logit is
+    // in and the routing is known, the routed experts'.  Warp-level tasks
+    // (k-part, row pass) leave partial sums in s_gacc; warps move on
+    // independently, and the last warp done with a buffer refills it.
     bool stop = false;
     for (;; ++j) {
       if (j == n_const) {
-        // ---- barrier A, then the routing (each CTA selects the experts itself)
-        if (tid == kBarT && !grid_wait(p.bar_gen, gen_a, p.err)) s_abort = 1;
+        // ---- the routing: every CTA selects the experts itself from the tagged logits
+        if (!topk_stage1(xlog, ep, E, K, s_cand, p.err)) ok = false;
         if (!ok) s_abort = 1;
         __syncthreads();
         if (s_abort) {
           stop = true;
           break;
         }
-        if (E <= kFW * 64) {
-          topk_stage1(p.logits, E, K, s_cand);
-          __syncthreads();
-          if (warp == 0) topk_stage2(p.logits, E, K, s_cand, s_idx, s_w);
-        } else if (warp == 0) {
-          topk_any(p.logits, E, K, s_idx, s_w);
-        }
+        if (warp == 0 && !topk_stage2(xlog, ep, E, K, s_cand, s_idx, s_w, p.err)) s_abort = 1;
         __syncthreads();
+        if (s_abort) {
+          stop = true;
+          break;
+        }
         // routed gate/up rows into every buffer (all consumed by now): item i by
         // lane 0 of warp 1 + i % 7, so the copies go out from several warps at once
         if (lane == 0 && warp > 0) {
           fence_proxy_async();
           for (int jj = n_const + warp - 1; jj < n_items && jj < n_const + nbuf; jj += kFW - 1) issue_item(jj, ly);
         }
+        __syncwarp();
         if (warp == 0) {
           if (b == 0 && lane < K && p.idx_out) p.idx_out[(size_t)t * K + lane] = s_idx[lane];
           if (b == 0 && lane < K && p.w_out) p.w_out[(size_t)t * K + lane] = s_w[lane];
@@ -536,6 +565,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
             __syncwarp(0xffffffffu >> (32 - K));
             issue_down(lane, ly.routed + (long long)s_idx[lane] * ly.stride);
           }
+          __syncwarp();
         }
       }
       if (j >= n_items) break;
@@ -588,10 +618,14 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
           }
         }
       }
+      __syncwarp();
     }
     if (stop) break;
+    if (!ok) s_abort = 1;
     __syncthreads();  // every partial sum of the step is in s_gacc
-    // SwiGLU of every gate/up row of this CTA: silu(g) * u with silu(z) = z / (1 + exp(-z))
+    if (s_abort) break;
+    // SwiGLU of every gate/up row of this CTA, silu(g) * u with silu(z) = z / (1 + exp(-z)),
+    // published as tagged words
     for (int jj = n_rt + warp; jj < n_items; jj += kFW) {
       const Item it = s_item[jj];
       if (lane < it.rows) {
@@ -600,51 +634,9 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
           g += s_gacc[((it.rbase + lane) * 4 + k) * 2];
           u += s_gacc[((it.rbase + lane) * 4 + k) * 2 + 1];
         }
-        p.act[(size_t)it.slot * I + it.row0 + lane] = g / (1.0f + expf(-g)) * u;
+        st_tagged(xact + (size_t)it.slot * I + it.row0 + lane, g / (1.0f + expf(-g)) * u, ep);
       }
     }
-
-    // ---- activation groups of 64: the CTA that completes a group writes its digits.
-    // Counting threads (warps 1..7) fence after the block barrier, which orders
-    // every act write of the CTA before their counts.
-    if (!ok) s_abort = 1;
-    __syncthreads();
-    if (s_abort) break;
-    // groups touched: shared rows [sh0, sh1) of slot K, routed flat rows [rf0, rf1)
-    const int gs0 = sh0 / kGroup, gs1 = sh1 > sh0 ? (sh1 - 1) / kGroup + 1 : gs0;
-    const int gr0 = rf0 / kGroup, gr1 = rf1 > rf0 ? (rf1 - 1) / kGroup + 1 : gr0;
-    const int ngs = gs1 - gs0, ngt = ngs + (gr1 - gr0);
-    const int gt = tid - 32;  // counting thread's group
-    if (gt >= 0 && gt < ngt) {
-      int fg, lo, hi;  // flat group over slot-major rows, and this CTA's rows in it
-      __threadfence();
-      if (gt < ngs) {
-        const int g = gs0 + gt;
-        fg = K * NGI + g;
-        lo = max(sh0, g * kGroup);
-        hi = min(sh1, (g + 1) * kGroup);
-      } else {
-        const int g = gr0 + gt - ngs;
-        fg = g;
-        lo = max(rf0, g * kGroup);
-        hi = min(rf1, (g + 1) * kGroup);
-      }
-      const unsigned prev = atomicAdd(&p.grp_cnt[fg], (unsigned)(hi - lo));
-      s_gdone[gt] = prev + (unsigned)(hi - lo) == (unsigned)kGroup ? fg + 1 : 0;
-    }
-    __syncthreads();
-    for (int k = warp - 1; warp > 0 && k < ngt; k += kFW - 1) {
-      const int fg1 = s_gdone[k];
-      if (!fg1) continue;
-      __threadfence();
-      const int fg = fg1 - 1, slot = fg / NGI, gg = fg % NGI;
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)fg * kGroup) + lane);
-      xq_quantize_group<BITS>(v.x, v.y, gg, NGI, p.act_limbs + (size_t)slot * NGI * kGroupWords * 4,
-                              p.act_cs + (size_t)slot * ncd);
-      if (lane == 0) p.grp_cnt[fg] = 0u;
-      __threadfence();
-    }
-    __syncthreads();
 
     // ---- the next step's routing-independent rows, into the drained ring
     if (tid == 0 && s + 1 < S) {
@@ -652,37 +644,38 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       const FusedLayer& ln = p.layers[(s + 1) % p.L];
       for (int jj = 0; jj < n_const && jj < nbuf; ++jj) issue_item(jj, ln);
     }
+    __syncwarp();
 
-    // ---- barrier B, then down + combine from shared memory
-    if (tid == kBarT) {
-      const unsigned gb = grid_arrive(p.bar_cnt, p.bar_gen, P);
-      if (!grid_wait(p.bar_gen, gb, p.err)) s_abort = 1;
-      if (!s_abort) {
-        const uint32_t bx = smem_addr(&s_xbar);
-        const uint32_t lb = (uint32_t)NE * NGI * kGroupWords * 4, cb = (uint32_t)NE * ncd * 8;
-        fence_proxy_async();
-        s_xstate = 1;
-        mbar_expect_tx(bx, lb + cb);
-        bulk_g2s(smem_addr(xd), p.act_limbs, lb, bx, pol);
-        bulk_g2s(smem_addr(xd + lb), p.act_cs, cb, bx, pol);
+    // ---- every CTA's activations: poll the tagged words of all K+1 slots and
+    // quantise them here (lane per block of 16, four lanes per group of 64)
+    const int nblk = NE * I / 16, bps = I / 16;
+#pragma unroll 1
+    for (int base = warp * 32; base < nblk; base += kFT) {
+      const int blk = base + lane;
+      const bool act = blk < nblk;
+      float av[16];
+      if (act) {
+        if (!poll_tagged<16>(xact + (size_t)blk * 16, ep, av, p.err)) ok = false;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) av[k] = 0.0f;
       }
+      const int slot = act ? blk / bps : 0, bb = act ? blk % bps : 0;
+      xq_quantize_block16<BITS>(av, bb >> 2, bb & 3, NGI, s_al + (size_t)slot * NGI * kGroupWords * 4,
+                                s_acs + (size_t)slot * ncd, act);
     }
-    __syncthreads();
-    if (s_abort) break;
-    if (!mbar_wait_bounded(smem_addr(&s_xbar), (uint32_t)(s & 1), p.err)) ok = false;
     if (nd > 0 && !mbar_wait_bounded(smem_addr(&s_dnbar), (uint32_t)(s & 1), p.err)) ok = false;
     if (!ok) s_abort = 1;
     __syncthreads();
     if (s_abort) break;
-    if (tid == 0) {
-      s_xstate = 0;
-      s_dnstate = 0;
-    }
+    if (tid == 0) s_dnstate = 0;
+
+    // ---- down + combine from shared memory: lane q owns one (slot, group) pair,
+    // four output rows per pass, then one interleaved reduction
     {
       uint32_t A[48];
-      const uint8_t* al = xd + (size_t)qslot * NGI * kGroupWords * 4;
-      load_group_limbs(reinterpret_cast<const uint32_t*>(al), qg, NGI, A);
-      const float2* acs = reinterpret_cast<const float2*>(xd + (size_t)NE * NGI * kGroupWords * 4) + qslot * ncd;
+      load_group_limbs(reinterpret_cast<const uint32_t*>(s_al + (size_t)qslot * NGI * kGroupWords * 4), qg, NGI, A);
+      const float2* acs = s_acs + qslot * ncd;
       float2 csa;
       if (BITS == 4) {
         const float2 a = acs[2 * qg], c = acs[2 * qg + 1];
@@ -692,10 +685,10 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       }
       const float wq = qon ? s_w[qslot] : 0.0f;
       const uint8_t* sb = dn + (size_t)qslot * dn_slot;
-      // four row slots per pass: independent dot products, then one interleaved reduction
       const uint16_t* scl = reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * RBd);
       const uint16_t* bsl = reinterpret_cast<const uint16_t*>(sb + (size_t)dmax * (RBd + SBd));
-      for (int pass = warp / KSd; ok && pass * 4 * RPPd < nd; pass += kFW / KSd) {
+#pragma unroll 1
+      for (int pass = warp / KSd; pass * 4 * RPPd < nd; pass += kFW / KSd) {
         float acc[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -723,21 +716,21 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
       }
     }
     __syncthreads();
+    // out = h + sum_k w_k y_k + sigma y_shared; inside a stack also the next layer's tagged input
+    const bool feed = s + 1 < S && (s + 1) % p.L != 0;
+    unsigned long long* xh = p.xh + (size_t)par * H;
     for (int r = tid; r < nd; r += kFT) {
       float y = 0.0f;
       for (int k = 0; k < KSd; ++k) y += s_dpart[k * kFusedMaxDnRows + r];
-      hout[d0 + r] = __ldcg(hin + d0 + r) + y;
+      const float o = __ldcg(hin + d0 + r) + y;
+      hout[d0 + r] = o;
+      if (feed) st_tagged(xh + d0 + r, o, ep);
     }
-    // the next step reads this step's output when it is the next layer of a stack
-    if (s + 1 < S && (s + 1) % p.L != 0) {
-      __syncthreads();
-      if (tid == kBarT) gen_c = grid_arrive(p.bar_cnt, p.bar_gen, P);
-      wait_c = true;
-    }
-    __syncthreads();  // shared memory of this step (DN, XD) is free
+    __syncthreads();  // shared memory of this step (XD, DN) is free
     if (tid == 0) fence_proxy_async();
   }
   if (s < S) abort_all(s);
+  if (b == 0 && tid == 0) *reinterpret_cast<volatile unsigned*>(p.epoch) = ep_base + (unsigned)S;
 }
 
 }  // namespace
@@ -745,7 +738,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
 FusedPlan plan_fused(int bits, int H, int I, int E, int K) {
   FusedPlan pl{};
   pl.ok = false;
-  if (H % kGroup || I % kGroup || K < 1 || K > 32 || E < K) return pl;
+  if (H % kGroup || I % kGroup || K < 1 || K > 32 || E < K || E > kFW * 64) return pl;
   const int NGH = H / kGroup, NGI = I / kGroup, NE = K + 1;
   if (NGH > 128 || NGI > 128) return pl;
   const int RB = H * bits / 8, SB = NGH * 2, RBd = I * bits / 8, SBd = NGI * 2;

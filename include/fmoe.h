@@ -152,13 +152,13 @@ fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float
 size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
 
 /* Bytes of the library's static scratch used by fmoe_moe_layer_static. */
-#define FMOE_STATIC_SCRATCH_BYTES 131072
+#define FMOE_STATIC_SCRATCH_BYTES 524288
 
 /* fmoe_moe_layer without a workspace argument: the pages have no counterpart
  * (their engine owns all its buffers); this is an interface convenience.
  * Computes exactly what fmoe_moe_layer computes, with the same kernels, but its
  * scratch is a fixed device array inside libfmoe.so of FMOE_STATIC_SCRATCH_BYTES
- * (128 KiB) per device, so the call allocates nothing.  It serves callers that
+ * (512 KiB) per device, so the call allocates nothing.  It serves callers that
  * cannot hand over a workspace: a plain-C or FFI host that keeps no device
  * allocator, or an engine whose memory planner has reserved the whole device.
  * Arguments as fmoe_moe_layer, plus:
@@ -178,7 +178,7 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
  * A layer whose scratch (fmoe_moe_layer_workspace_size(layer, T)) exceeds
  * FMOE_STATIC_SCRATCH_BYTES is rejected with FMOE_ERR_WORKSPACE before
  * anything is enqueued.  Every shape the other requirements admit needs at
- * most 108,032 bytes (the Qwen3.5-397B-A17B layer 58,112), so today that
+ * most 435,968 bytes (the Qwen3.5-397B-A17B layer 214,016), so today that
  * check only guards against shapes later versions may admit. */
 fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
                                   float* topk_w, int* dev_err, fmoe_stream_t stream);
