@@ -352,11 +352,7 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   rp.xq_limb_stride = 3LL * H;
   rp.xq_cs_stride = H / 32;
   rp.logits = reinterpret_cast<float*>(base + L.logits);
-  rp.top_k = K;
-  rp.route_idx = reinterpret_cast<int32_t*>(base + L.route_idx);
-  rp.route_w = reinterpret_cast<float*>(base + L.route_w);
-  rp.idx_out = idx_out;
-  rp.w_out = w_out;
+  rp.top_k = 0;  // the expert kernels select the experts from the logits themselves
   rp.tickets = ctrl->tickets;
   rp.err = err_word ? err_word : &ctrl->err;
   const bool trace = g_trace_on;
@@ -370,8 +366,9 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   ExpertParams p{};
   p.routed = ref(r);
   p.shared = ref(layer->shared);
-  p.route_idx = rp.route_idx;
-  p.route_w = rp.route_w;
+  p.logits = rp.logits;
+  p.idx_out = idx_out;
+  p.w_out = w_out;
   p.E = E;
   p.fixed_expert = 0;
   p.K = K;
@@ -388,9 +385,15 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   p.out = out;
   p.prefetch_down = prefetch_down();
   p.err = rp.err;
+  p.rt_idx = reinterpret_cast<int32_t*>(base + L.route_idx);
+  p.rt_w = reinterpret_cast<float*>(base + L.route_w);
   if ((e = launch_gateup(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
   if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
-  if ((e = launch_down(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "down launch");
+  ExpertParams pd = p;  // the down kernel reads the routing the gate/up kernel wrote
+  pd.logits = nullptr;
+  pd.route_idx = p.rt_idx;
+  pd.route_w = p.rt_w;
+  if ((e = launch_down(pd, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "down launch");
   if (trace && (e = trace_record(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   return FMOE_OK;
 }

@@ -428,6 +428,85 @@ __device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int
     warp_topk_mem(logits, E, K, has_gate, idx_k, w_k, sigma);
 }
 
+// Block-wide top-K of logits [E] (E <= 8 * 64) with 256 threads, in two stages.
+// Stage 1 (every warp w): the K largest keys of slice w of ceil(E/8) logits into
+// cand[w*K + k].  Stage 2 (warp 0, after a block barrier): the K largest of the
+// 8K candidates, the renormalised weights w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0)
+// into idx[0..K), w[0..K), and w[K] = sigmoid(logits[E]) when has_gate.  Keys
+// order by value, then by lower index (topk_key): the result is that of one sort.
+__device__ __forceinline__ void block_topk_stage1(const float* logits, int E, int K, unsigned long long* cand) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ES = (E + 7) / 8;
+  const int e0 = warp * ES + lane, e1 = e0 + 32;
+  unsigned long long k0 = (lane < ES && e0 < E) ? topk_key(__ldcg(logits + e0), e0) : 0ull;
+  unsigned long long k1 = (lane + 32 < ES && e1 < E) ? topk_key(__ldcg(logits + e1), e1) : 0ull;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    const unsigned long long m = warp_max_key(k0 > k1 ? k0 : k1);
+    if (lane == 0) cand[warp * K + k] = m;
+    k0 = k0 == m ? 0ull : k0;
+    k1 = k1 == m ? 0ull : k1;
+  }
+}
+
+__device__ __forceinline__ void block_topk_stage2(float zg, int E, int K, int has_gate,
+                                                  const unsigned long long* cand, int* idx, float* w) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long key[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) key[i] = lane + 32 * i < 8 * K ? cand[lane + 32 * i] : 0ull;
+  float top = 0.0f, mine = 0.0f;
+  int mi = 0;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) best = key[i] > best ? key[i] : best;
+    const unsigned long long m = warp_max_key(best);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) key[i] = key[i] == m ? 0ull : key[i];
+    int e = m ? topk_key_index(m) : 0;
+    const float v = topk_key_value(m);
+    if (e < 0 || e >= E) e = 0;  // only with non-finite logits
+    if (k == 0) top = v;
+    if (lane == k) {
+      mi = e;
+      mine = v;
+    }
+  }
+  const float ek = lane < K ? expf(mine - top) : 0.0f;
+  const float wk = ek / warp_sum(ek);
+  if (lane < K) {
+    idx[lane] = mi;
+    w[lane] = wk;
+  }
+  if (lane == 0) w[K] = has_gate ? 1.0f / (1.0f + expf(-zg)) : 0.0f;
+}
+
+// The routing of one token by the whole block (256 threads; contains block
+// barriers): the two-stage top-K for E <= 512, a single-warp rescan otherwise.
+__device__ __forceinline__ void block_topk(const float* logits, int E, int K, int has_gate, unsigned long long* cand,
+                                           int* idx, float* w) {
+  if (E <= 512) {
+    // thread 0 reads the shared-gate logit now, so that its latency overlaps stage 1
+    const float zg = (has_gate && threadIdx.x == 0) ? __ldcg(logits + E) : 0.0f;
+    block_topk_stage1(logits, E, K, cand);
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) block_topk_stage2(zg, E, K, has_gate, cand, idx, w);
+  } else if ((threadIdx.x >> 5) == 0) {
+    int ik;
+    float wk, sig;
+    warp_topk(logits, E, K, has_gate, ik, wk, sig);
+    const int lane = threadIdx.x & 31;
+    if (lane < K) {
+      idx[lane] = ik;
+      w[lane] = wk;
+    }
+    if (lane == 0) w[K] = sig;
+  }
+  __syncthreads();
+}
+
 // Record base pointer for one expert slot.
 struct BankRef {
   const uint8_t* base;

@@ -46,8 +46,14 @@ struct TopkParams {
 struct ExpertParams {
   BankRef routed;
   BankRef shared;
-  const int32_t* route_idx;   // [K] selected experts (router output) or NULL (fixed_expert)
+  const float* logits;        // [E+1] router logits (+ shared-gate logit): each kernel selects the
+                              // experts itself; NULL: the routing below
+  const int32_t* route_idx;   // [K] selected experts or NULL (fixed_expert)
   const float* route_w;       // [K+1] weights, slot K = shared-gate sigma; NULL: weight 1
+  int32_t* idx_out;           // with logits: the caller's copy of the routing [K], [K] (gate/up CTA 0), or NULL
+  float* w_out;
+  int32_t* rt_idx;            // with logits: gate/up CTA 0 writes the routing here for the down kernel
+  float* rt_w;                // [K+1], slot K = shared-gate sigma
   int E;
   int fixed_expert;
   int K;                      // routed slots

@@ -57,6 +57,7 @@ __device__ __forceinline__ float2 group_scalars(const float2* cs, int g) {
 
 constexpr int kGuWarps = 8;
 constexpr int kChunkUnits = 8;  // units per staged chunk
+constexpr size_t kGuSmemBudget = 220 * 1024;  // shared memory of the gate/up kernel
 
 template <int BITS, int NG>
 struct GuCfg {
@@ -76,10 +77,10 @@ struct GuCfg {
 
 // Persistent: CTA b owns units [b*U/G, (b+1)*U/G) (a unit = kRowPairs rows of
 // gate and up of one expert slot), cut into chunks of up to kChunkUnits units
-// of one slot.  Thread 0 stages each chunk with six large bulk copies into a
-// ring of nbuf chunk buffers; warp w computes units w, w+8, .. of the chunk.
-// A lane always works on the same groups of 64 columns, so it keeps their
-// digits of x in registers for the whole kernel.
+// of one slot, each staged with six bulk copies into a ring of nbuf chunk
+// buffers; warp w computes units w, w+8, .. of the chunk.  A lane always works
+// on the same groups of 64 columns, so it keeps their digits of x in registers
+// for the whole kernel.
 template <int BITS, int NG>
 __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertParams p, int nbuf) {
   using G = Geo<NG>;
@@ -92,6 +93,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
   __shared__ __align__(8) uint64_t s_bar[8];
   __shared__ __align__(8) uint64_t s_bar_x;
   __shared__ int s_idx[32];
+  __shared__ float s_wt[33];
+  __shared__ unsigned long long s_cand[8 * 32];
   __shared__ int s_done[kGuWarps * 32];
   __shared__ int s_abort;
 
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     const bool routed = sl < p.K;
     const uint8_t* rec = routed ? p.routed.base + (long long)s_idx[sl] * p.routed.stride : p.shared.base;
     const long long* off = routed ? p.routed.off : p.shared.off;
-    const uint64_t pol = routed ? l2_policy_evict_first() : l2_policy_evict_last();
+    const uint64_t pol = l2_policy_evict_first();  // weights come back only after a whole model pass
     uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
     const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_bar[c % nbuf]);
     const uint32_t cb = rows * RB, sb = rows * SB;
@@ -141,48 +144,62 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     }
   }
 
-  pdl_wait();  // the router's logits, routing and x digits are complete
+  pdl_wait();  // the router's logits and x digits are complete
   pdl_trigger();
 
-  if (warp == 0) {
-    if (lane < p.K) {
-      int e = p.route_idx ? p.route_idx[lane] : p.fixed_expert;
-      if (e < 0 || e >= p.routed.num_experts) {
-        atomicExch(p.err, kDevBadIndex);
-        e = 0;
-      }
-      s_idx[lane] = e;
+  // The routing: from the logits, by the whole block (every CTA the same), or given.
+  if (p.logits) {
+    block_topk(p.logits, p.E, p.K, 1, s_cand, s_idx, s_wt);
+  } else if (warp == 0 && lane < p.K) {
+    s_idx[lane] = p.route_idx ? p.route_idx[lane] : p.fixed_expert;
+  }
+  __syncthreads();
+  if (tid < p.K) {
+    const int e = s_idx[tid];
+    if (e < 0 || e >= p.routed.num_experts) {
+      atomicExch(p.err, kDevBadIndex);
+      s_idx[tid] = 0;
     }
-    __syncwarp();
-    if (lane == 0) {
+  }
+  __syncthreads();
+  if (p.logits && blockIdx.x == 0 && tid <= p.K) {  // the routing for the down kernel and the caller
+    if (tid < p.K) {
+      if (p.rt_idx) p.rt_idx[tid] = s_idx[tid];
+      if (p.idx_out) p.idx_out[tid] = s_idx[tid];
+      if (p.w_out) p.w_out[tid] = s_wt[tid];
+    }
+    if (p.rt_w) p.rt_w[tid] = s_wt[tid];
+  }
+  if (lane == 0) {
+    // x digits by warp 0; the first routed chunks one per warp (lane 0), so that
+    // their copies go out from several warps at once; the L2 warm-up by warp 7
+    if (warp == 0) {
       const uint32_t bx = smem_addr(&s_bar_x);
       mbar_expect_tx(bx, C::kDigitBytes);
       bulk_g2s(smem_addr(sm), p.xq_limbs, NG * kGroupWords * 4, bx, l2_policy_evict_last());
       bulk_g2s(smem_addr(sm + NG * kGroupWords * 4), p.xq_cs, C::kChunks * 8, bx, l2_policy_evict_last());
-      int cu = u0;
-      for (int c = 0; c < nbuf && cu < u1; ++c) {
-        const int ce = chunk_end(cu);
-        if (cu / ups < p.K) issue(c, cu, ce);
-        cu = ce;
-      }
-      if (p.prefetch_down && u0 / ups < p.K) {
-        // Warm L2 with this CTA's slice of each routed expert's down matrix.
-        const long long len[3] = {(long long)p.H * (I * BITS / 8), (long long)p.H * (I / kGroup) * 2,
-                                  (long long)p.H * (I / kGroup) * 2};
-        for (int k = 0; k < p.K; ++k) {
-          const uint8_t* rec = p.routed.base + (long long)s_idx[k] * p.routed.stride;
-          for (int m = 0; m < 3; ++m) {
-            const long long a0 = (len[m] * blockIdx.x / gridDim.x) & ~15LL;
-            const long long a1 = (len[m] * (blockIdx.x + 1) / gridDim.x) & ~15LL;
-            if (a1 > a0) prefetch_l2(rec + p.routed.off[6 + m] + a0, (uint32_t)(a1 - a0));
-          }
+    }
+    int cu = u0;
+    for (int c = 0; c < nbuf && cu < u1; ++c) {
+      const int ce = chunk_end(cu);
+      if (cu / ups < p.K && c % kGuWarps == warp) issue(c, cu, ce);
+      cu = ce;
+    }
+    if (warp == kGuWarps - 1 && p.prefetch_down && u0 / ups < p.K) {
+      // Warm L2 with this CTA's slice of each routed expert's down matrix.
+      const long long len[3] = {(long long)p.H * (I * BITS / 8), (long long)p.H * (I / kGroup) * 2,
+                                (long long)p.H * (I / kGroup) * 2};
+      for (int k = 0; k < p.K; ++k) {
+        const uint8_t* rec = p.routed.base + (long long)s_idx[k] * p.routed.stride;
+        for (int m = 0; m < 3; ++m) {
+          const long long a0 = (len[m] * blockIdx.x / gridDim.x) & ~15LL;
+          const long long a1 = (len[m] * (blockIdx.x + 1) / gridDim.x) & ~15LL;
+          if (a1 > a0) prefetch_l2(rec + p.routed.off[6 + m] + a0, (uint32_t)(a1 - a0));
         }
       }
     }
-    // The other lanes wait here rather than spin on the digits' barrier, which
-    // would share the warp's issue slots with lane 0's copy issue.
-    __syncwarp();
   }
+  __syncwarp();
 
   // This lane's groups and their digits of x, for the whole kernel.
   const int sub = lane / LPR, gl = lane % LPR;
@@ -259,8 +276,11 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
   }
 
   // Groups of 64 activations: the CTA that completes a group writes its digits
-  // for the down kernel (release: fence before the count; acquire: fence after).
-  __threadfence();
+  // for the down kernel.  The counting threads (warps 1..) fence after the block
+  // barrier (release of every act write of the CTA), the writing warps before
+  // reading (acquire).  Warp 7 lane 0 issued L2 prefetches and warp 0 nothing
+  // that matters here, but a gpu-scope fence waits for its own thread's copies,
+  // so neither takes part.
   __syncthreads();
   if (s_abort) {  // let copies still in flight land before the CTA exits
     if (tid == 0)
@@ -268,14 +288,16 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     return;
   }
   const int g0 = u0 * RP / kGroup, ng = (u1 * RP - 1) / kGroup - g0 + 1;  // groups over concatenated slot rows
-  if (tid < ng) {
-    const int g = g0 + tid;
+  const int ct = tid - 32;
+  if (ct >= 0 && ct < ng) {
+    const int g = g0 + ct;
     const int lo = max(u0 * RP, g * kGroup), hi = min(u1 * RP, (g + 1) * kGroup);
+    __threadfence();
     const unsigned prev = atomicAdd(&p.grp_cnt[g], (unsigned)(hi - lo));
-    s_done[tid] = prev + (unsigned)(hi - lo) == (unsigned)kGroup;
+    s_done[ct] = prev + (unsigned)(hi - lo) == (unsigned)kGroup;
   }
   __syncthreads();
-  for (int t = warp; t < ng; t += kGuWarps) {
+  for (int t = warp - 1; warp >= 1 && warp < kGuWarps - 1 && t < ng; t += kGuWarps - 2) {
     if (!s_done[t]) continue;
     __threadfence();
     const int g = g0 + t, slot = g * kGroup / I, gg = (g * kGroup % I) / kGroup;
@@ -304,8 +326,9 @@ struct DnCfg {
 // Persistent: CTA b owns units [b*U/G, (b+1)*U/G) of kRows output rows,
 // staged in chunks of up to `chunk_units` units: for every selected expert the
 // chunk's rows of its down matrix (codes, scales, biases: three bulk copies).
-// The experts are known from the router, so the first chunks are requested
-// before waiting on the gate/up kernel.  Lane l owns the (slot, group) pairs
+// The experts are known once the gate/up kernel (CTA 0) has written the
+// routing, i.e. after the wait; the gate/up kernel has warmed L2 with this
+// CTA's rows by then, so the copies come mostly from L2.  Lane l owns the (slot, group) pairs
 // q = l, l+32, .. (PPL of them) of every row and keeps their digits in
 // registers; the warp sums a row's pairs by shuffles.
 template <int BITS, int NG, int PPL>
@@ -333,11 +356,17 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
   const int slot_bytes = crows * (RB + 2 * SB);  // one expert's rows of a chunk
   const int chb = (NE * slot_bytes + 127) / 128 * 128;
 
-  // Routing: the router has completed (the gate/up kernel signals this launch
-  // only after its own wait), so the experts and weights can be read now.
+  // The routing is written by CTA 0 of the gate/up kernel: read it after the wait.
+  if (tid == 0) {
+    for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&s_bar[b]), 1);
+    mbar_init(smem_addr(&s_bar_x), 1);
+    mbar_fence_init();
+  }
+  pdl_wait();  // the activations' digits and the routing are complete
+  pdl_trigger();
   if (warp == 0) {
     if (lane < p.K) {
-      int ik = p.route_idx ? p.route_idx[lane] : p.fixed_expert;
+      int ik = p.route_idx ? __ldcg(p.route_idx + lane) : p.fixed_expert;
       if (ik < 0 || ik >= p.routed.num_experts) {
         atomicExch(p.err, kDevBadIndex);
         ik = 0;
@@ -346,18 +375,13 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
       s_src[lane][0] = rec + p.routed.off[6];
       s_src[lane][1] = rec + p.routed.off[7];
       s_src[lane][2] = rec + p.routed.off[8];
-      s_w[lane] = p.route_w ? p.route_w[lane] : 1.0f;
+      s_w[lane] = p.route_w ? __ldcg(p.route_w + lane) : 1.0f;
     }
     if (lane == 0 && p.has_shared) {
       s_src[p.K][0] = p.shared.base + p.shared.off[6];
       s_src[p.K][1] = p.shared.base + p.shared.off[7];
       s_src[p.K][2] = p.shared.base + p.shared.off[8];
-      s_w[p.K] = p.route_w ? p.route_w[p.K] : 1.0f;
-    }
-    if (lane == 0) {
-      for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&s_bar[b]), 1);
-      mbar_init(smem_addr(&s_bar_x), 1);
-      mbar_fence_init();
+      s_w[p.K] = p.route_w ? __ldcg(p.route_w + p.K) : 1.0f;
     }
   }
   __syncthreads();
@@ -379,16 +403,12 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
     }
   };
   const int nchunk = (u1 - u0 + chunk_units - 1) / chunk_units;
-  if (tid == 0)
-    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c);
-
-  pdl_wait();  // the activations' digits are complete
-  pdl_trigger();
-  if (tid == 0) {  // every slot's digits, once per CTA
+  if (tid == 0) {  // every slot's digits, once per CTA; then the first chunks (mostly from L2)
     const uint32_t bx = smem_addr(&s_bar_x);
     mbar_expect_tx(bx, (uint32_t)(dwords * 4 + NE * NCH * 8));
     bulk_g2s(smem_addr(sm), p.act_limbs, (uint32_t)dwords * 4, bx, l2_policy_evict_first());
     bulk_g2s(smem_addr(sm + (size_t)dwords * 4), p.act_cs, (uint32_t)(NE * NCH * 8), bx, l2_policy_evict_first());
+    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c);
   }
   __syncwarp();  // lanes 1..31 of warp 0 wait for the issue instead of spinning beside it
 
@@ -464,9 +484,9 @@ cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
   int grid = num_sms();
   grid = grid > units ? units : grid;
   // each CTA counts at most one block of threads' worth of activation groups
-  if ((long long)(units + grid - 1) / grid * C::kRowPairs / kGroup + 2 > kGuWarps * 32) return cudaErrorInvalidValue;
+  if ((long long)(units + grid - 1) / grid * C::kRowPairs / kGroup + 2 > kGuWarps * 32 - 32) return cudaErrorInvalidValue;
   const int per_cta = (units + grid - 1) / grid;
-  int nbuf = (int)((kSmemBudget - C::kHead) / C::kChunkBytes);
+  int nbuf = (int)((kGuSmemBudget - C::kHead) / C::kChunkBytes);
   const int need = (per_cta + kChunkUnits - 1) / kChunkUnits + 1;  // +1: a chunk may stop at a slot boundary
   nbuf = nbuf > need ? need : nbuf;
   nbuf = nbuf > 8 ? 8 : nbuf;
@@ -587,7 +607,7 @@ template <int BITS, int NGU, int NGD>
 bool fits(int ne) {
   int cu, nb;
   size_t sm;
-  return GuCfg<BITS, NGU>::kHead + GuCfg<BITS, NGU>::kChunkBytes <= kSmemBudget &&
+  return GuCfg<BITS, NGU>::kHead + GuCfg<BITS, NGU>::kChunkBytes <= kGuSmemBudget &&
          down_plan<BITS, NGD>(1 << 20, ne, cu, nb, sm) && ne * NGD <= 4 * 32;
 }
 template <int BITS, int NGU>

@@ -3,16 +3,18 @@
 // RMSNorm follows "What is Flash-MoE" (a2a-mcp.org), section 3: two passes,
 // sum of squares then apply.  Routing follows the "Flash-MoE" wiki summary
 // (jeongsk), per-layer pipeline: routing projection, then softmax and top-K.
-// The pages run the selection on the CPU; here the router kernel only writes
-// the logits and every expert kernel takes the top-K from them itself
-// (warp_topk), so no host round trip and no grid-wide handshake sits between
-// the router and the experts.
+// The pages run the selection on the CPU; here it stays on the GPU: in the
+// MoE block the router kernel writes the logits and every CTA of the expert
+// kernels selects the experts from them itself (block_topk), so neither a host
+// round trip nor a grid-wide handshake sits between the router and the experts.
+// The standalone router_topk entry point uses topk_kernel.
 #include "fmoe_internal.h"
 
 namespace fmoe {
 namespace {
 
 constexpr int kRouterThreads = 256;
+constexpr int kRouterMaxRows = 8;  // router rows per CTA
 
 // Block-wide sum of one value per thread (256 threads), same order every call.
 __device__ __forceinline__ float block_sum_256(float v, float* s_red) {
@@ -62,7 +64,7 @@ template <int XQB>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ float s_red[8];
-  __shared__ float s_part[8];
+  __shared__ float s_part[kRouterMaxRows * 8];
   __shared__ int s_last;
   __shared__ __align__(8) uint64_t s_bar;
   const int t = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -91,6 +93,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
 
   const float* h = p.h + (size_t)t * H;
   float ss = 0.0f;
+#pragma unroll 4
   for (int i = tid * 4; i < H; i += kRouterThreads * 4) {
     const float4 v = *reinterpret_cast<const float4*>(h + i);
     *reinterpret_cast<float4*>(xs + i) = v;
@@ -102,7 +105,13 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
   if (p.norm) {
     ss = block_sum_256(ss, s_red);
     const float rstd = 1.0f / sqrtf(ss / (float)H + p.eps);
-    for (int i = tid; i < H; i += kRouterThreads) xs[i] = xs[i] * rstd * (p.gamma ? p.gamma[i] : 1.0f);
+#pragma unroll 4
+    for (int i = tid * 4; i < H; i += kRouterThreads * 4) {
+      float4 v = *reinterpret_cast<const float4*>(xs + i);
+      const float4 g = p.gamma ? __ldg(reinterpret_cast<const float4*>(p.gamma + i)) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+      v = make_float4(v.x * rstd * g.x, v.y * rstd * g.y, v.z * rstd * g.z, v.w * rstd * g.w);
+      *reinterpret_cast<float4*>(xs + i) = v;
+    }
   }
   __syncthreads();
 
@@ -114,36 +123,52 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
     }
   }
 
-  const int S = rpc >= 8 ? 1 : (rpc >= 4 ? 2 : (rpc >= 2 ? 4 : 8));  // segments per row
+  // Warp w sums column slice w (H/8 columns) of every row of this CTA: x of the
+  // slice is read from shared memory once per 8 columns and reused for every
+  // row; the 8 slice sums of a row then add in fixed order.
   const bool ready = nrows > 0 && mbar_wait_bounded(bar, 0, p.err);
-  if (ready && warp < nrows * S) {
-    const int rl = warp / S, seg = warp % S;
-    const int seglen = H / S;
-    const uint4* wv = reinterpret_cast<const uint4*>(wrows + (size_t)rl * H + seg * seglen);
-    const float* xv = xs + seg * seglen;
-    float acc = 0.0f;
-#pragma unroll 4
-    for (int k = lane; k < seglen / 8; k += 32) {
-      const uint4 w = wv[k];
+  if (ready) {
+    const uint16_t* wr = wrows + warp * (H / 8);
+    const float* xv = xs + warp * (H / 8);
+    float acc[kRouterMaxRows];
+#pragma unroll
+    for (int r = 0; r < kRouterMaxRows; ++r) acc[r] = 0.0f;
+#pragma unroll 1
+    for (int k = lane; k < H / 64; k += 32) {  // 8 columns per step
       const float4 xa = *reinterpret_cast<const float4*>(xv + 8 * k);
       const float4 xb = *reinterpret_cast<const float4*>(xv + 8 * k + 4);
-      acc = fmaf(bf_lo(w.x), xa.x, acc);
-      acc = fmaf(bf_hi(w.x), xa.y, acc);
-      acc = fmaf(bf_lo(w.y), xa.z, acc);
-      acc = fmaf(bf_hi(w.y), xa.w, acc);
-      acc = fmaf(bf_lo(w.z), xb.x, acc);
-      acc = fmaf(bf_hi(w.z), xb.y, acc);
-      acc = fmaf(bf_lo(w.w), xb.z, acc);
-      acc = fmaf(bf_hi(w.w), xb.w, acc);
+#pragma unroll
+      for (int r = 0; r < kRouterMaxRows; ++r) {
+        if (r < nrows) {
+          const uint4 w = *reinterpret_cast<const uint4*>(wr + (size_t)r * H + 8 * k);
+          float a = acc[r];
+          a = fmaf(bf_lo(w.x), xa.x, a);
+          a = fmaf(bf_hi(w.x), xa.y, a);
+          a = fmaf(bf_lo(w.y), xa.z, a);
+          a = fmaf(bf_hi(w.y), xa.w, a);
+          a = fmaf(bf_lo(w.z), xb.x, a);
+          a = fmaf(bf_hi(w.z), xb.y, a);
+          a = fmaf(bf_lo(w.w), xb.z, a);
+          a = fmaf(bf_hi(w.w), xb.w, a);
+          acc[r] = a;
+        }
+      }
     }
-    acc = warp_sum(acc);
-    if (lane == 0) s_part[warp] = acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int r = 0; r < kRouterMaxRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+    if (lane == 0)
+#pragma unroll
+      for (int r = 0; r < kRouterMaxRows; ++r)
+        if (r < nrows) s_part[r * 8 + warp] = acc[r];
   }
   __syncthreads();
   float* logits = p.logits + (size_t)t * (E + 1);
   if (ready && tid < nrows) {
     float l = 0.0f;
-    for (int s = 0; s < S; ++s) l += s_part[tid * S + s];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) l += s_part[tid * 8 + w];
     const int row = r0 + tid;
     if (row < E && p.bias) l += p.bias[row];
     logits[row] = l;
