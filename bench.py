@@ -38,7 +38,13 @@ WORKLOADS = {
     "qwen397-2bit-zipf": (lambda: __import__("gen").qwen397_layer(2, zipf=1.1),
                           "Qwen3.5-397B-A17B-shaped MoE layer, 2-bit group-64 experts, Zipf(1.1) routing, batch-1 decode"),
     "tiny-4bit": (lambda: __import__("gen").tiny_layer(4), "tiny MoE layer (H256, E8, I128, top-2), 4-bit"),
+    "qwen397-2bit-stack60": (lambda: __import__("gen").qwen397_layer(2),
+                             "stack of 60 Qwen3.5-397B-A17B-shaped MoE blocks, 2-bit group-64 experts "
+                             "(all 60 x 513 experts resident), one token through all 60 per step"),
 }
+# Workloads that run a stack of distinct layers per token (fmoe_moe_stack); the
+# metric then counts layer-steps (one token through one layer) per second.
+STACK_LAYERS = {"qwen397-2bit-stack60": 60}
 
 
 def parse():
@@ -191,8 +197,13 @@ def main():
     fmoe.lib()
 
     # ---- resident inputs: layer copies and token states
-    ncopy = max(1, args.copies)
+    nstack = STACK_LAYERS.get(args.workload, 0)
+    ncopy = nstack if nstack else max(1, args.copies)
     layers = [gen.binding_layer(gen.device_layer(spec, seed=0, layer=c, device=dev)) for c in range(ncopy)]
+    if nstack:  # one step = one token through the whole stack: keep graphs and the run short
+        args.steps = min(args.steps, 200)
+        args.graph_tokens = min(args.graph_tokens, 50)
+        args.warmup = min(args.warmup, 5)
     G = min(args.graph_tokens, args.steps)
     steps = (args.steps + G - 1) // G * G
     h = gen.device_tokens(rank * 10_000_000, G, spec.hidden, device=dev)
@@ -202,7 +213,10 @@ def main():
     torch.cuda.synchronize(dev)
 
     def step(i, s):
-        fmoe.moe_layer(layers[i % ncopy], h[i % G], out=out[i % G], ws=ws, stream=s)
+        if nstack:
+            fmoe.moe_stack(layers, h[i % G:i % G + 1], out=out[i % G:i % G + 1], ws=ws, stream=s)
+        else:
+            fmoe.moe_layer(layers[i % ncopy], h[i % G], out=out[i % G], ws=ws, stream=s)
 
     with torch.cuda.stream(stream):
         for i in range(max(args.warmup, 3)):
@@ -238,8 +252,8 @@ def main():
         ms = float(t.item())
         dist.barrier()
     fmoe.workspace_check(ws, stream)
-    tokens = steps * world
-    value = tokens / (ms / 1e3)
+    per_step = nstack if nstack else 1  # layer-steps (one token through one layer) per step
+    value = steps * world * per_step / (ms / 1e3)
     ms_per_step = ms / steps
 
     # ---- per-kernel durations: a separate replay with trace events around each kernel
@@ -274,7 +288,10 @@ def main():
         with torch.cuda.graph(egraph, stream=stream):
             for i in range(G):
                 hd.copy_(hh[i], non_blocking=True)
-                fmoe.moe_layer(layers[i % ncopy], hd, out=od, ws=ws, stream=stream)
+                if nstack:
+                    fmoe.moe_stack(layers, hd.view(1, -1), out=od.view(1, -1), ws=ws, stream=stream)
+                else:
+                    fmoe.moe_layer(layers[i % ncopy], hd, out=od, ws=ws, stream=stream)
                 oh[i].copy_(od, non_blocking=True)
         with torch.cuda.stream(stream):
             egraph.replay()
@@ -294,7 +311,7 @@ def main():
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
         bpt = spec.hidden * 4
-        e2e = {"value": steps * world / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bpt,
+        e2e = {"value": steps * world * per_step / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bpt,
                "d2h_bytes_per_step": bpt}
         del egraph
 
@@ -320,15 +337,18 @@ def main():
             "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
                        "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": 1,
                        "layer_copies": ncopy, "graph_tokens": G,
-                       "l2": f"inputs larger than L2: {ncopy} resident layer copies "
-                             f"({ncopy * gen.record_bytes(spec) * (spec.experts + 1) / 1e9:.1f} GB) rotated per token",
+                       "l2": (f"inputs larger than L2: {ncopy} resident layers "
+                              f"({ncopy * gen.record_bytes(spec) * (spec.experts + 1) / 1e9:.1f} GB), each token "
+                              f"through all of them in order; value counts layer-steps" if nstack else
+                              f"inputs larger than L2: {ncopy} resident layer copies "
+                              f"({ncopy * gen.record_bytes(spec) * (spec.experts + 1) / 1e9:.1f} GB) rotated per token"),
                        "parallelism": f"replicas x{world}"},
             "effective_gbs": eff, "frac_of_peak": eff / peak, "bytes_per_token": bytes_tok,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": GATEUP_TRAFFIC.get(args.workload), "kernel": "gateup_kernel", "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": gateup_bytes},
             "kernels_us": {"router": router_us, "gateup": gateup_us, "down": down_us},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * steps,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * steps * per_step,
             "clocks": clk.record(),
         }
         print(json.dumps(line), flush=True)
