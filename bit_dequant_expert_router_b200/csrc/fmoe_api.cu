@@ -69,6 +69,38 @@ WsLayout layout(int H, int E, int K, int I, int T) {
   return L;
 }
 
+// Workspace of the expert-grouped path for T tokens: regions in this order,
+// placed after the whole per-token layout (whose counters must stay zero
+// between calls); the control block is the per-token one at offset 0.
+struct GLayout {
+  size_t ctrl, logits, xq_limbs, xq_cs, route_idx, route_w, n_active, act_expert, act_off, pair_tok, pair_pos, act,
+      act_limbs, act_cs, y, total;
+};
+
+GLayout glayout(int H, int E, int K, int I, int T) {
+  GLayout L;
+  const size_t np = (size_t)T * K, nr = np + T;
+  L.ctrl = 0;
+  L.logits = layout(H, E, K, I, 1).total;
+  L.xq_limbs = L.logits + up((size_t)T * (E + 1) * 4);
+  L.xq_cs = L.xq_limbs + up((size_t)T * 3 * H);
+  L.route_idx = L.xq_cs + up((size_t)T * (H / 32) * 8);
+  L.route_w = L.route_idx + up(np * 4);
+  L.n_active = L.route_w + up((size_t)T * (K + 1) * 4);
+  L.act_expert = L.n_active + up(4);
+  L.act_off = L.act_expert + up(np * 4);
+  L.pair_tok = L.act_off + up((np + 1) * 4);
+  L.pair_pos = L.pair_tok + up(np * 4);
+  L.act = L.pair_pos + up(np * 4);
+  L.act_limbs = L.act + up(nr * I * 4);
+  L.act_cs = L.act_limbs + up(nr * 3 * I);
+  L.y = L.act_cs + up(nr * (I / 32) * 8);
+  L.total = L.y + up(nr * H * 4);
+  return L;
+}
+
+constexpr int kGroupedMinT = 8;  // batches at least this large take the expert-grouped path
+
 fmoe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (!ws) return fail(FMOE_ERR_WORKSPACE, "workspace is NULL");
   if (((uintptr_t)ws & (kAlign - 1)) != 0) return fail(FMOE_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
@@ -324,9 +356,14 @@ static fmoe_status check_layer(const fmoe_layer* layer) {
 }
 
 size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
-  (void)T;
   if (!layer) return 0;
-  return layout(layer->routed.hidden, layer->routed.num_experts, layer->top_k, layer->routed.inter, 1).total;
+  const int H = layer->routed.hidden, E = layer->routed.num_experts, K = layer->top_k, I = layer->routed.inter;
+  size_t need = layout(H, E, K, I, 1).total;
+  if (T >= kGroupedMinT && K >= 1 && E >= 1 && H > 0 && I > 0) {
+    const size_t g = glayout(H, E, K, I, T).total;
+    need = g > need ? g : need;
+  }
+  return need;
 }
 
 // One token through the block: router (+RMSNorm, digits, top-K) -> gate/up -> down + combine.
@@ -479,10 +516,86 @@ static fmoe_status run_fused(const fmoe_layer* layers, int nl, const float* h, i
   return FMOE_OK;
 }
 
-// The block for T tokens of one layer on a checked workspace.
+// The expert-grouped path (k_grouped.cu) for T >= kGroupedMinT tokens, unless
+// FMOE_GROUPED=0 is set in the environment, the shapes are outside it, or the
+// workspace is too small for it; `taken` tells whether it ran.
+static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* idx_out,
+                               float* w_out, uint8_t* base, size_t ws_bytes, cudaStream_t s, int* err_word,
+                               bool& taken) {
+  taken = false;
+  const char* v = getenv("FMOE_GROUPED");
+  if (T < kGroupedMinT || (v && v[0] == '0')) return FMOE_OK;
+  const fmoe_bank& r = layer->routed;
+  const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
+  if (!grouped_shapes_supported(bits, H, I, E, K, T) || !same_offsets(r, layer->shared)) return FMOE_OK;
+  const GLayout G = glayout(H, E, K, I, T);
+  if (ws_bytes < G.total) return FMOE_OK;
+  WsControl* ctrl = reinterpret_cast<WsControl*>(base + G.ctrl);
+  int* err = err_word ? err_word : &ctrl->err;
+  RouterParams rp{};
+  rp.h = h;
+  rp.gamma = layer->gamma;
+  rp.eps = layer->eps;
+  rp.norm = layer->gamma != nullptr;
+  rp.w_router = layer->w_router;
+  rp.bias = layer->router_bias;
+  rp.w_sgate = layer->w_shared_gate;
+  rp.T = T;
+  rp.H = H;
+  rp.E = E;
+  rp.xq_limbs = base + G.xq_limbs;
+  rp.xq_cs = reinterpret_cast<float2*>(base + G.xq_cs);
+  rp.xq_limb_stride = 3LL * H;
+  rp.xq_cs_stride = H / 32;
+  rp.logits = reinterpret_cast<float*>(base + G.logits);
+  rp.top_k = 0;
+  rp.tickets = ctrl->tickets;
+  rp.err = err;
+  GroupedParams p{};
+  p.routed = ref(r);
+  p.shared = ref(layer->shared);
+  p.T = T;
+  p.E = E;
+  p.K = K;
+  p.H = H;
+  p.I = I;
+  p.logits = rp.logits;
+  p.xq_limbs = base + G.xq_limbs;
+  p.xq_cs = rp.xq_cs;
+  p.route_idx = reinterpret_cast<int32_t*>(base + G.route_idx);
+  p.route_w = reinterpret_cast<float*>(base + G.route_w);
+  p.idx_out = idx_out;
+  p.w_out = w_out;
+  p.n_active = reinterpret_cast<int32_t*>(base + G.n_active);
+  p.act_expert = reinterpret_cast<int32_t*>(base + G.act_expert);
+  p.act_off = reinterpret_cast<int32_t*>(base + G.act_off);
+  p.pair_tok = reinterpret_cast<int32_t*>(base + G.pair_tok);
+  p.pair_pos = reinterpret_cast<int32_t*>(base + G.pair_pos);
+  p.act = reinterpret_cast<float*>(base + G.act);
+  p.act_limbs = base + G.act_limbs;
+  p.act_cs = reinterpret_cast<float2*>(base + G.act_cs);
+  p.y = reinterpret_cast<float*>(base + G.y);
+  p.h = h;
+  p.out = out;
+  p.err = err;
+  cudaError_t e;
+  if ((e = launch_router(rp, bits, false, s)) != cudaSuccess) return cuda_fail(e, "router launch");
+  if ((e = launch_grouped_select(p, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  if ((e = launch_grouped_gateup(p, bits, s)) != cudaSuccess) return cuda_fail(e, "grouped gate/up launch");
+  if ((e = launch_grouped_actq(p, bits, s)) != cudaSuccess) return cuda_fail(e, "activation digits launch");
+  if ((e = launch_grouped_down(p, bits, s)) != cudaSuccess) return cuda_fail(e, "grouped down launch");
+  if ((e = launch_grouped_combine(p, s)) != cudaSuccess) return cuda_fail(e, "combine launch");
+  taken = true;
+  return FMOE_OK;
+}
+
+// The block for T tokens of one layer on a checked workspace of ws_bytes.
 static fmoe_status moe_layer_impl(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
-                                  float* topk_w, uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word) {
+                                  float* topk_w, uint8_t* base, size_t ws_bytes, const WsLayout& L, cudaStream_t s,
+                                  int* err_word) {
   bool taken = false;
+  fmoe_status gst = run_grouped(layer, h, T, out, topk_idx, topk_w, base, ws_bytes, s, err_word, taken);
+  if (gst != FMOE_OK || taken) return gst;
   fmoe_status st = run_fused(layer, 1, h, T, out, topk_idx, topk_w, base, L, s, err_word, taken);
   if (st != FMOE_OK || taken) return st;
   const int H = layer->routed.hidden, K = layer->top_k;
@@ -505,7 +618,8 @@ fmoe_status fmoe_moe_layer(const fmoe_layer* layer, const float* h, int T, float
   const int H = layer->routed.hidden, K = layer->top_k;
   const WsLayout L = layout(H, layer->routed.num_experts, K, layer->routed.inter, 1);
   if ((st = check_ws(ws, ws_bytes, L.total)) != FMOE_OK) return st;
-  return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, static_cast<uint8_t*>(ws), L, cs(stream), nullptr);
+  return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, static_cast<uint8_t*>(ws), ws_bytes, L, cs(stream),
+                        nullptr);
 }
 
 // ---- fmoe_moe_layer_static: the same block with library-owned scratch.
@@ -556,7 +670,7 @@ fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T
                 L.total, kStaticScratchBytes);
   uint8_t* base = nullptr;
   if ((st = static_scratch(&base)) != FMOE_OK) return st;
-  return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, base, L, cs(stream), dev_err);
+  return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, base, kStaticScratchBytes, L, cs(stream), dev_err);
 }
 
 fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int nl, const float* h, int T, float* out, void* ws,

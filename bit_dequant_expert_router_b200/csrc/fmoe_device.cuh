@@ -428,6 +428,33 @@ __device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int
     warp_topk_mem(logits, E, K, has_gate, idx_k, w_k, sigma);
 }
 
+// Lane geometry over rows of NG groups of 64 codes: LPR lanes per row, RPP rows
+// side by side in a warp, GPL groups per lane.
+template <int NG>
+struct Geo {
+  static constexpr int kLanesPerRow = NG < 32 ? NG : 32;
+  static constexpr int kRowsPerPass = 32 / kLanesPerRow;
+  static constexpr int kGroupsPerLane = NG / kLanesPerRow;
+};
+
+// One group's code words from a staged row (4-bit: 32 bytes, 2-bit: 16 bytes).
+template <int BITS>
+__device__ __forceinline__ void load_group_codes(const uint8_t* row, int g, uint4& q0, uint4& q1) {
+  constexpr int GB = kGroup * BITS / 8;
+  q0 = *reinterpret_cast<const uint4*>(row + g * GB);
+  q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(row + g * GB + 16) : q0;
+}
+
+// Chunk scalars of group g: {power-of-two scale of the digits, sum of x over the group}.
+template <int BITS>
+__device__ __forceinline__ float2 group_scalars(const float2* cs, int g) {
+  if (BITS == 4) {
+    const float2 a = cs[2 * g], b = cs[2 * g + 1];
+    return make_float2(a.x, a.y + b.y);
+  }
+  return cs[g];
+}
+
 // Block-wide top-K of logits [E] (E <= 8 * 64) with 256 threads, in two stages.
 // Stage 1 (every warp w): the K largest keys of slice w of ceil(E/8) logits into
 // cand[w*K + k].  Stage 2 (warp 0, after a block barrier): the K largest of the

@@ -71,6 +71,40 @@ struct ExpertParams {
   int* err;
 };
 
+// ---- expert-grouped path for batched decode (k_grouped.cu): T tokens, each active
+// expert's weights read once for all the tokens routed to it
+
+struct GroupedParams {
+  BankRef routed, shared;
+  int T, E, K, H, I;
+  const float* logits;        // [T][E+1] router logits (+ shared-gate logit)
+  const uint8_t* xq_limbs;    // [T][3H] digits of x per token
+  const float2* xq_cs;        // [T][H*bits/128]
+  int32_t* route_idx;         // [T][K]
+  float* route_w;             // [T][K+1], slot K = sigma
+  int32_t* idx_out;           // caller's copies [T][K] or NULL
+  float* w_out;
+  int32_t* n_active;          // [1] U: active experts
+  int32_t* act_expert;        // [T*K] active experts, increasing
+  int32_t* act_off;           // [T*K+1] first pair of each active expert in the sorted pair list
+  int32_t* pair_tok;          // [T*K] sorted pairs (expert, token, k): value t*K + k
+  int32_t* pair_pos;          // [T*K] position of pair t*K + k in the sorted list
+  float* act;                 // [(T*K + T)][I] SwiGLU outputs: sorted pairs, then the shared expert per token
+  uint8_t* act_limbs;         // [(T*K + T)][3I]
+  float2* act_cs;             // [(T*K + T)][I*bits/128]
+  float* y;                   // [(T*K + T)][H] down outputs (unweighted)
+  const float* h;             // [T][H] residual
+  float* out;                 // [T][H]
+  int* err;
+};
+
+cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s);
+cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, cudaStream_t s);
+cudaError_t launch_grouped_actq(const GroupedParams& p, int bits, cudaStream_t s);
+cudaError_t launch_grouped_down(const GroupedParams& p, int bits, cudaStream_t s);
+cudaError_t launch_grouped_combine(const GroupedParams& p, cudaStream_t s);
+bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T);
+
 // ---- single-kernel path (k_fused.cu): a sequence of T tokens x L layers, one CTA per SM
 
 constexpr int kFusedWarps = 8;

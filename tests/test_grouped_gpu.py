@@ -1,0 +1,94 @@
+"""The expert-grouped batched path (T >= 8 tokens of one layer) against the CPU oracle and the per-token path."""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from tests.helpers import max_rel_err, oracle_layer, oracle_layer_sparse, routing_margin, check_routing, ulp32
+from tests.test_parity_gpu import TOL, _compare_layer, _run_layer
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fmoe():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_dequant_expert_router_b200 as m
+    m.lib()
+    return m
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_grouped_tiny_batch_matches_oracle(fmoe, bits):
+    # 64 tokens over 8 experts: every expert's group is large (many digit batches per CTA)
+    spec = gen.LayerSpec(**{**gen.tiny_layer(bits).__dict__, "random_gamma": True})
+    hl = gen.host_layer(spec, seed=12)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(700, 64, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    exact, _ = _compare_layer(hl, h, out, idx, w)
+    assert exact >= 60
+
+
+def test_grouped_tiny_batch_top1_all_experts_and_odd_size(fmoe):
+    spec = gen.tiny_layer(4)
+    hl = gen.host_layer(spec, seed=13)
+    dl = gen.upload_layer(hl)
+    for top_k, T in ((1, 9), (8, 23)):
+        h = gen.host_tokens(900 + T, T, spec.hidden)
+        out, idx, w = _run_layer(fmoe, dl, h, top_k=top_k)
+        _compare_layer(hl, h, out, idx, w, L=oracle_layer(hl, top_k=top_k))
+
+
+def test_per_token_path_still_matches_oracle(fmoe, monkeypatch):
+    monkeypatch.setenv("FMOE_GROUPED", "0")
+    spec = gen.tiny_layer(2)
+    hl = gen.host_layer(spec, seed=14)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(1000, 16, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    _compare_layer(hl, h, out, idx, w)
+
+
+@pytest.mark.parametrize("bits,zipf", [(4, 0.0), (2, 1.1)])
+def test_grouped_full_size_batch(fmoe, monkeypatch, bits, zipf):
+    """64 tokens of the Qwen3.5-397B-A17B-shaped layer: sampled tokens against the
+    oracle, every token against the per-token path."""
+    spec = gen.qwen397_layer(bits, zipf=zipf)
+    dl = gen.device_layer(spec, seed=0, layer=0)
+    lay = gen.binding_layer(dl)
+    T, K = 64, spec.top_k
+    h_np = gen.host_tokens(2000, T, spec.hidden)
+    h = torch.from_numpy(h_np).cuda()
+    out = torch.empty_like(h)
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    ws = fmoe.workspace(fmoe.moe_layer_workspace_size(lay, T))
+    fmoe.moe_layer(lay, h, out=out, topk_idx=idx, topk_w=w, ws=ws)
+    fmoe.workspace_check(ws)
+    monkeypatch.setenv("FMOE_GROUPED", "0")
+    ref = torch.empty_like(h)
+    ref_idx = torch.empty_like(idx)
+    fmoe.moe_layer(lay, h, out=ref, topk_idx=ref_idx, ws=ws)
+    torch.cuda.synchronize()
+    o, r = out.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64)
+    gi, ri = idx.cpu().numpy(), ref_idx.cpu().numpy()
+    same = np.all(gi == ri, axis=1)
+    assert same.sum() >= T - 2   # routing agrees except where a logit near-tie flips
+    h64 = h_np.astype(np.float64)
+    assert max_rel_err(o[same] - h64[same], r[same] - h64[same], slack=ulp32(o[same])) <= TOL
+    # sampled tokens against the oracle (drawing only the experts they need)
+    sample = [0, 17, 40, 63]
+    hl0 = gen.host_layer(spec, seed=0, layer=0, experts=[])
+    need = set(gi[sample].reshape(-1).tolist())
+    for t in sample:
+        x = oracle.rmsnorm(h_np[t], hl0.gamma, spec.eps)
+        logits, _ = routing_margin(hl0.w_router, x, hl0.logit_bias)
+        need |= set(np.argsort(-logits, kind="stable")[:K].tolist())
+    hl = gen.host_layer(spec, seed=0, layer=0, experts=sorted(need))
+    _compare_layer(hl, h_np[sample], o[sample].astype(np.float64), gi[sample],
+                   w.cpu().numpy()[sample].astype(np.float64), L=oracle_layer_sparse(hl))
+    del dl, lay
+    torch.cuda.empty_cache()
