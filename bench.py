@@ -38,6 +38,9 @@ WORKLOADS = {
     "qwen397-2bit-zipf": (lambda: __import__("gen").qwen397_layer(2, zipf=1.1),
                           "Qwen3.5-397B-A17B-shaped MoE layer, 2-bit group-64 experts, Zipf(1.1) routing, batch-1 decode"),
     "tiny-4bit": (lambda: __import__("gen").tiny_layer(4), "tiny MoE layer (H256, E8, I128, top-2), 4-bit"),
+    "qwen397-4bit-batch64": (lambda: __import__("gen").qwen397_layer(4),
+                             "Qwen3.5-397B-A17B-shaped MoE layer, 4-bit group-64 experts, batched decode of 64 "
+                             "tokens per step grouped by expert"),
     "qwen397-2bit-stack60": (lambda: __import__("gen").qwen397_layer(2),
                              "stack of 60 Qwen3.5-397B-A17B-shaped MoE blocks, 2-bit group-64 experts "
                              "(all 60 x 513 experts resident), one token through all 60 per step"),
@@ -45,6 +48,8 @@ WORKLOADS = {
 # Workloads that run a stack of distinct layers per token (fmoe_moe_stack); the
 # metric then counts layer-steps (one token through one layer) per second.
 STACK_LAYERS = {"qwen397-2bit-stack60": 60}
+# Batched decode: tokens per step through one layer (the expert-grouped path).
+BATCH = {"qwen397-4bit-batch64": 64}
 
 
 def parse():
@@ -198,23 +203,32 @@ def main():
 
     # ---- resident inputs: layer copies and token states
     nstack = STACK_LAYERS.get(args.workload, 0)
-    ncopy = nstack if nstack else max(1, args.copies)
+    nbatch = BATCH.get(args.workload, 0)
+    ncopy = nstack if nstack else (min(4, max(1, args.copies)) if nbatch else max(1, args.copies))
     layers = [gen.binding_layer(gen.device_layer(spec, seed=0, layer=c, device=dev)) for c in range(ncopy)]
     if nstack:  # one step = one token through the whole stack: keep graphs and the run short
         args.steps = min(args.steps, 200)
         args.graph_tokens = min(args.graph_tokens, 50)
         args.warmup = min(args.warmup, 5)
+    if nbatch:  # one step = a batch of tokens through one layer (per-kernel trace skipped)
+        args.steps = min(args.steps, 500)
+        args.graph_tokens = min(args.graph_tokens, 20)
+        args.warmup = min(args.warmup, 5)
     G = min(args.graph_tokens, args.steps)
     steps = (args.steps + G - 1) // G * G
-    h = gen.device_tokens(rank * 10_000_000, G, spec.hidden, device=dev)
+    nb = nbatch if nbatch else 1
+    h = gen.device_tokens(rank * 10_000_000, G * nb, spec.hidden, device=dev).view(G, nb, spec.hidden) if nbatch else \
+        gen.device_tokens(rank * 10_000_000, G, spec.hidden, device=dev)
     out = torch.empty_like(h)
-    ws = fmoe.workspace(max(fmoe.moe_layer_workspace_size(l, 1) for l in layers), dev)
+    ws = fmoe.workspace(max(fmoe.moe_layer_workspace_size(l, nb) for l in layers), dev)
     stream = torch.cuda.Stream(dev)
     torch.cuda.synchronize(dev)
 
     def step(i, s):
         if nstack:
             fmoe.moe_stack(layers, h[i % G:i % G + 1], out=out[i % G:i % G + 1], ws=ws, stream=s)
+        elif nbatch:
+            fmoe.moe_layer(layers[i % ncopy], h[i % G], out=out[i % G], ws=ws, stream=s)
         else:
             fmoe.moe_layer(layers[i % ncopy], h[i % G], out=out[i % G], ws=ws, stream=s)
 
@@ -252,37 +266,50 @@ def main():
         ms = float(t.item())
         dist.barrier()
     fmoe.workspace_check(ws, stream)
-    per_step = nstack if nstack else 1  # layer-steps (one token through one layer) per step
+    per_step = nstack if nstack else (nbatch if nbatch else 1)  # layer-token steps per step
     value = steps * world * per_step / (ms / 1e3)
     ms_per_step = ms / steps
 
+    # ---- batched decode: active experts per step from one untimed pass (for the bytes a step moves)
+    n_active = None
+    if nbatch:
+        idx = torch.empty((nb, spec.top_k), dtype=torch.int32, device=dev)
+        act = []
+        for i in range(G):
+            fmoe.moe_layer(layers[i % ncopy], h[i], out=out[i], topk_idx=idx, ws=ws)
+            act.append(len(set(idx.cpu().numpy().reshape(-1).tolist())))
+        n_active = float(np.mean(act))
+
     # ---- per-kernel durations: a separate replay with trace events around each kernel
-    tr = min(G, 500)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(tr)]
-    for e4 in evs:  # torch creates the CUDA event on its first record
-        for e in e4:
-            e.record(stream)
-    stream.synchronize()
-    # the library records these as external event nodes inside the captured graph
-    tgraph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(tgraph, stream=stream):
-        for i in range(tr):
-            fmoe.trace_next_layer(evs[i])
-            step(i, stream)
-    with torch.cuda.stream(stream):
-        tgraph.replay()
-    stream.synchronize()
-    dur = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs]) * 1e3
-    router_us, gateup_us, down_us = (float(np.mean(dur[:, k])) for k in range(3))
-    del tgraph
+    # (the three-kernel per-token path; the batched path has no per-kernel trace)
+    tr = 0 if nbatch else min(G, 500)
+    router_us = gateup_us = down_us = None
+    if tr:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(tr)]
+        for e4 in evs:  # torch creates the CUDA event on its first record
+            for e in e4:
+                e.record(stream)
+        stream.synchronize()
+        # the library records these as external event nodes inside the captured graph
+        tgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tgraph, stream=stream):
+            for i in range(tr):
+                fmoe.trace_next_layer(evs[i])
+                step(i, stream)
+        with torch.cuda.stream(stream):
+            tgraph.replay()
+        stream.synchronize()
+        dur = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs]) * 1e3
+        router_us, gateup_us, down_us = (float(np.mean(dur[:, k])) for k in range(3))
+        del tgraph
 
     # ---- end to end through the C ABI with host buffers: H2D of h, the layer, D2H of out, every step
     e2e = None
     if not args.no_e2e:
-        hh = torch.empty((G, spec.hidden), dtype=torch.float32, pin_memory=True)
+        hh = torch.empty(tuple(h.shape), dtype=torch.float32, pin_memory=True)
         hh.copy_(h.cpu())
         oh = torch.empty_like(hh, pin_memory=True)
-        hd = torch.empty((spec.hidden,), dtype=torch.float32, device=dev)
+        hd = torch.empty(tuple(h.shape[1:]), dtype=torch.float32, device=dev)
         od = torch.empty_like(hd)
         egraph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(egraph, stream=stream):
@@ -310,7 +337,7 @@ def main():
             t = torch.tensor([ems], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
-        bpt = spec.hidden * 4
+        bpt = spec.hidden * 4 * nb  # the step's hidden states in, its outputs out
         e2e = {"value": steps * world * per_step / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bpt,
                "d2h_bytes_per_step": bpt}
         del egraph
@@ -318,9 +345,18 @@ def main():
     # ---- roofline of the dominant kernel (gate/up + SwiGLU over K routed + 1 shared expert)
     peak, peak_kind = peak_hbm()
     rec_mat = spec.inter * spec.hidden * spec.bits // 8 + 2 * spec.inter * (spec.hidden // spec.group) * 2
-    gateup_bytes = (spec.top_k + 1) * 2 * rec_mat
-    achieved = gateup_bytes / (gateup_us * 1e-6) / 1e9
-    bytes_tok = gen.algorithmic_bytes_per_token(spec)
+    if nbatch:
+        # a step moves the active experts' records, the shared expert's and the router, once each
+        rec = gen.record_bytes(spec)
+        step_bytes = (n_active + 1) * 3 * rec_mat + spec.experts * spec.hidden * 2
+        bytes_tok = step_bytes / nb
+        kernel, kbytes = "batched step (all kernels)", step_bytes
+        achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+        del rec
+    else:
+        kernel, kbytes = "gateup_kernel", (spec.top_k + 1) * 2 * rec_mat
+        achieved = kbytes / (gateup_us * 1e-6) / 1e9
+        bytes_tok = gen.algorithmic_bytes_per_token(spec)
     eff = bytes_tok * (value / world) / 1e9
 
     cpu = None
@@ -335,7 +371,8 @@ def main():
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32", "data": "synthetic",
             "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
-                       "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": 1,
+                       "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": nb,
+                       "active_experts_per_step": n_active,
                        "layer_copies": ncopy, "graph_tokens": G,
                        "l2": (f"inputs larger than L2: {ncopy} resident layers "
                               f"({ncopy * gen.record_bytes(spec) * (spec.experts + 1) / 1e9:.1f} GB), each token "
@@ -345,10 +382,10 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "effective_gbs": eff, "frac_of_peak": eff / peak, "bytes_per_token": bytes_tok,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": GATEUP_TRAFFIC.get(args.workload), "kernel": "gateup_kernel", "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": gateup_bytes},
+                         "traffic": GATEUP_TRAFFIC.get(args.workload), "kernel": kernel, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": kbytes},
             "kernels_us": {"router": router_us, "gateup": gateup_us, "down": down_us},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * steps * per_step,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (6 * steps if nbatch else 3 * steps * per_step),
             "clocks": clk.record(),
         }
         print(json.dumps(line), flush=True)
