@@ -129,6 +129,17 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (ms): every rank times its own replica, the job takes as long as the slowest."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -259,11 +270,8 @@ def main():
             ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize(dev)
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     fmoe.workspace_check(ws, stream)
     per_step = nstack if nstack else (nbatch if nbatch else 1)  # layer-token steps per step
@@ -332,11 +340,7 @@ def main():
                 egraph.replay()
             e1.record(stream)
         e1.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
         bpt = spec.hidden * 4 * nb  # the step's hidden states in, its outputs out
         e2e = {"value": steps * world * per_step / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bpt,
                "d2h_bytes_per_step": bpt}
