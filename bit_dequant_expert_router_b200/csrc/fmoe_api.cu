@@ -74,7 +74,7 @@ WsLayout layout(int H, int E, int K, int I, int T) {
 // between calls); the control block is the per-token one at offset 0.
 struct GLayout {
   size_t ctrl, logits, xq_limbs, xq_cs, route_idx, route_w, n_active, act_expert, act_off, pair_tok, pair_pos, act,
-      act_limbs, act_cs, y, total;
+      act_limbs, act_cs, y, x, total;
 };
 
 GLayout glayout(int H, int E, int K, int I, int T) {
@@ -95,7 +95,8 @@ GLayout glayout(int H, int E, int K, int I, int T) {
   L.act_limbs = L.act + up(nr * I * 4);
   L.act_cs = L.act_limbs + up(nr * 3 * I);
   L.y = L.act_cs + up(nr * (I / 32) * 8);
-  L.total = L.y + up(nr * H * 4);
+  L.x = L.y + up(nr * H * 4);
+  L.total = L.x + up((size_t)T * H * 4);
   return L;
 }
 
@@ -532,25 +533,13 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   if (ws_bytes < G.total) return FMOE_OK;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + G.ctrl);
   int* err = err_word ? err_word : &ctrl->err;
-  RouterParams rp{};
-  rp.h = h;
-  rp.gamma = layer->gamma;
-  rp.eps = layer->eps;
-  rp.norm = layer->gamma != nullptr;
-  rp.w_router = layer->w_router;
-  rp.bias = layer->router_bias;
-  rp.w_sgate = layer->w_shared_gate;
-  rp.T = T;
-  rp.H = H;
-  rp.E = E;
-  rp.xq_limbs = base + G.xq_limbs;
-  rp.xq_cs = reinterpret_cast<float2*>(base + G.xq_cs);
-  rp.xq_limb_stride = 3LL * H;
-  rp.xq_cs_stride = H / 32;
-  rp.logits = reinterpret_cast<float*>(base + G.logits);
-  rp.top_k = 0;
-  rp.tickets = ctrl->tickets;
-  rp.err = err;
+  RouterBatch rb{};
+  rb.gamma = layer->gamma;
+  rb.eps = layer->eps;
+  rb.w_router = layer->w_router;
+  rb.w_sgate = layer->w_shared_gate;
+  rb.bias = layer->router_bias;
+  rb.x = reinterpret_cast<float*>(base + G.x);
   GroupedParams p{};
   p.routed = ref(r);
   p.shared = ref(layer->shared);
@@ -559,9 +548,9 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   p.K = K;
   p.H = H;
   p.I = I;
-  p.logits = rp.logits;
+  p.logits = reinterpret_cast<float*>(base + G.logits);
   p.xq_limbs = base + G.xq_limbs;
-  p.xq_cs = rp.xq_cs;
+  p.xq_cs = reinterpret_cast<float2*>(base + G.xq_cs);
   p.route_idx = reinterpret_cast<int32_t*>(base + G.route_idx);
   p.route_w = reinterpret_cast<float*>(base + G.route_w);
   p.idx_out = idx_out;
@@ -579,7 +568,7 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   p.out = out;
   p.err = err;
   cudaError_t e;
-  if ((e = launch_router(rp, bits, false, s)) != cudaSuccess) return cuda_fail(e, "router launch");
+  if ((e = launch_grouped_router(p, rb, bits, s)) != cudaSuccess) return cuda_fail(e, "router launch");
   if ((e = launch_grouped_select(p, s)) != cudaSuccess) return cuda_fail(e, "select launch");
   if ((e = launch_grouped_gateup(p, bits, s)) != cudaSuccess) return cuda_fail(e, "grouped gate/up launch");
   if ((e = launch_grouped_actq(p, bits, s)) != cudaSuccess) return cuda_fail(e, "activation digits launch");

@@ -98,6 +98,17 @@ struct GroupedParams {
   int* err;
 };
 
+// The batched router: x = RMSNorm(h) and its digits per token, then the router GEMM.
+struct RouterBatch {
+  const float* gamma;         // [H] or NULL (no norm)
+  float eps;
+  const uint16_t* w_router;   // bf16 [E][H]
+  const uint16_t* w_sgate;    // bf16 [H]
+  const float* bias;          // [E] or NULL
+  float* x;                   // workspace [T][H]: x in fp32
+};
+
+cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s);
 cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s);
 cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, cudaStream_t s);
 cudaError_t launch_grouped_actq(const GroupedParams& p, int bits, cudaStream_t s);

@@ -30,54 +30,228 @@ constexpr int kGuTok = 2;         // tokens whose digits are staged at once (gat
 constexpr int kDnRows = 32;       // down output rows per CTA
 constexpr int kDnTok = 16;        // tokens whose activation digits are staged at once (down)
 constexpr int kMaxTK = 4096;      // T*K pairs
+constexpr int kRtRows = 8;        // router rows per CTA (batched router)
+constexpr int kRtTok = 16;        // tokens per CTA (batched router)
 
-// ---- selection: one CTA
-__global__ void __launch_bounds__(kGT) select_kernel(const GroupedParams p) {
-  extern __shared__ __align__(16) int s_cnt[];  // [E] counts, then [E] next free slot
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = p.T, E = p.E, K = p.K;
-  int* s_pos = s_cnt + E;
-  for (int e = tid; e < E; e += kGT) s_cnt[e] = 0;
-  // top-K of every token, one warp per token (ties to the lower index)
-  for (int t = warp; t < T; t += kGT / 32) {
-    int ik;
-    float wk, sig;
-    warp_topk(p.logits + (size_t)t * (E + 1), E, K, 1, ik, wk, sig);
-    if (ik < 0 || ik >= E) ik = 0;
-    if (lane < K) {
-      p.route_idx[(size_t)t * K + lane] = ik;
-      p.route_w[(size_t)t * (K + 1) + lane] = wk;
-      if (p.idx_out) p.idx_out[(size_t)t * K + lane] = ik;
-      if (p.w_out) p.w_out[(size_t)t * K + lane] = wk;
+// ---- selection, in two kernels.  topk: one CTA per token, the block-wide
+// two-stage top-K (ties to the lower index) with renormalised weights and the
+// shared-gate sigma.
+__global__ void __launch_bounds__(kGT) topk_tokens_kernel(const GroupedParams p) {
+  __shared__ int s_idx[32];
+  __shared__ float s_w[33];
+  __shared__ unsigned long long s_cand[8 * 32];
+  const int t = blockIdx.x, tid = threadIdx.x, K = p.K, E = p.E;
+  block_topk(p.logits + (size_t)t * (E + 1), E, K, 1, s_cand, s_idx, s_w);
+  if (tid < K) {
+    int e = s_idx[tid];
+    e = (e < 0 || e >= E) ? 0 : e;
+    p.route_idx[(size_t)t * K + tid] = e;
+    p.route_w[(size_t)t * (K + 1) + tid] = s_w[tid];
+    if (p.idx_out) p.idx_out[(size_t)t * K + tid] = e;
+    if (p.w_out) p.w_out[(size_t)t * K + tid] = s_w[tid];
+  }
+  if (tid == K) p.route_w[(size_t)t * (K + 1) + K] = s_w[K];
+}
+
+constexpr int kST = 1024;  // threads of the sort kernel
+
+// Exclusive block-wide scan of one value per thread (kST threads); returns the
+// exclusive prefix and writes the total to *total.
+__device__ __forceinline__ int block_scan_excl(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kST / 32 ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
     }
-    if (lane == 0) p.route_w[(size_t)t * (K + 1) + K] = sig;
+    if (lane < kST / 32) s_warp[lane] = w;  // inclusive warp totals
   }
   __syncthreads();
-  // counting sort of the T*K pairs by expert, stable in (token, k) order
-  if (tid == 0) {
-    for (int i = 0; i < T * K; ++i) ++s_cnt[p.route_idx[i]];
-    int u = 0, run = 0;
-    for (int e = 0; e < E; ++e) {
-      s_pos[e] = run;
-      if (s_cnt[e]) {
-        p.act_expert[u] = e;
-        p.act_off[u] = run;
-        ++u;
-        run += s_cnt[e];
+  const int before = warp ? s_warp[warp - 1] : 0;
+  *total = s_warp[kST / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// sort: one CTA.  Counting sort of the T*K pairs by expert, stable in (token, k)
+// order: the rank of pair i among the pairs of its expert is the number of
+// earlier pairs with the same expert.  Active experts in increasing order.
+__global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) {
+  extern __shared__ __align__(16) int s_mem[];  // [T*K] experts of the pairs, [E] counts, [E] starts
+  __shared__ int s_warp[kST / 32];
+  const int tid = threadIdx.x, N = p.T * p.K, E = p.E;
+  int* s_e = s_mem;
+  int* s_cnt = s_mem + N;
+  int* s_start = s_cnt + E;
+  for (int e = tid; e < E; e += kST) s_cnt[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < N; i += kST) {
+    const int e = __ldcg(p.route_idx + i);
+    s_e[i] = e;
+    atomicAdd(&s_cnt[e], 1);
+  }
+  __syncthreads();
+  // starts of the experts (exclusive scan of the counts) and slots of the active ones
+  const int per = (E + kST - 1) / kST;  // experts per thread, contiguous
+  int c = 0, a = 0;
+  for (int k = 0; k < per; ++k) {
+    const int e = tid * per + k;
+    if (e < E) {
+      c += s_cnt[e];
+      a += s_cnt[e] > 0;
+    }
+  }
+  int tot_c, tot_a;
+  int run = block_scan_excl(c, s_warp, &tot_c);
+  int slot = block_scan_excl(a, s_warp, &tot_a);
+  for (int k = 0; k < per; ++k) {
+    const int e = tid * per + k;
+    if (e < E) {
+      s_start[e] = run;
+      if (s_cnt[e] > 0) {
+        p.act_expert[slot] = e;
+        p.act_off[slot] = run;
+        ++slot;
       }
+      run += s_cnt[e];
     }
-    p.act_off[u] = run;
-    for (int i = 0; i < T * K; ++i) {
-      const int e = p.route_idx[i];
-      const int pos = s_pos[e]++;
-      p.pair_tok[pos] = i;
-      p.pair_pos[i] = pos;
-    }
-    *p.n_active = u;
+  }
+  if (tid == 0) {
+    p.act_off[tot_a] = tot_c;
+    *p.n_active = tot_a;
+  }
+  __syncthreads();
+  for (int i = tid; i < N; i += kST) {
+    const int e = s_e[i];
+    int rank = 0;
+    for (int j = 0; j < i; ++j) rank += s_e[j] == e;
+    const int pos = s_start[e] + rank;
+    p.pair_tok[pos] = i;
+    p.pair_pos[i] = pos;
   }
 }
 
-// The group of active expert slot u (u == U: the shared expert, every token):
+// ---- router for the batch.  norm_digits: one CTA per token, x = RMSNorm(h)
+// (two passes) in fp32 for the router and as digits for the experts.
+__global__ void __launch_bounds__(kGT) norm_digits_kernel(const GroupedParams p, const RouterBatch rb, int bits) {
+  __shared__ float s_red[kGT / 32];
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, H = p.H;
+  const float* h = p.h + (size_t)t * H;
+  float* x = rb.x + (size_t)t * H;
+  float ss = 0.0f;
+  for (int i = tid * 4; i < H; i += kGT * 4) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(h + i));
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+  }
+  float rstd = 1.0f;
+  if (rb.gamma) {
+    ss = warp_sum(ss);
+    if (lane == 0) s_red[warp] = ss;
+    __syncthreads();
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kGT / 32; ++w) tot += s_red[w];
+    rstd = 1.0f / sqrtf(tot / (float)H + rb.eps);
+  }
+  for (int i = tid * 4; i < H; i += kGT * 4) {
+    float4 v = __ldcg(reinterpret_cast<const float4*>(h + i));
+    if (rb.gamma) {
+      const float4 g = __ldg(reinterpret_cast<const float4*>(rb.gamma + i));
+      v = make_float4(v.x * rstd * g.x, v.y * rstd * g.y, v.z * rstd * g.z, v.w * rstd * g.w);
+    }
+    *reinterpret_cast<float4*>(x + i) = v;
+  }
+  __syncthreads();  // this CTA's x is written (read back through L1-bypassing loads below)
+  __threadfence_block();
+  uint8_t* limbs = const_cast<uint8_t*>(p.xq_limbs) + (size_t)t * 3 * H;
+  float2* cs = const_cast<float2*>(p.xq_cs) + (size_t)t * (H / 32);
+  for (int g = warp; g < H / kGroup; g += kGT / 32) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(x + g * kGroup) + lane);
+    if (bits == 4)
+      xq_quantize_group<4>(v.x, v.y, g, H / kGroup, limbs, cs);
+    else
+      xq_quantize_group<2>(v.x, v.y, g, H / kGroup, limbs, cs);
+  }
+}
+
+// router_gemm: CTA (a, b) computes logits of rows [8a, 8a+8) of [W_r; w_sg] for
+// tokens [16b, 16b+16): the rows are staged once, x of each token streams from
+// L2.  Warp w sums column slice w (H/8 columns); the 8 slice sums add in fixed order.
+__global__ void __launch_bounds__(kGT) router_gemm_kernel(const GroupedParams p, const RouterBatch rb) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ float s_part[kRtTok][kRtRows][kGT / 32];
+  __shared__ __align__(8) uint64_t s_bar;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, H = p.H, E = p.E;
+  const int r0 = blockIdx.x * kRtRows, n = min(kRtRows, E + 1 - r0);
+  const int t0 = blockIdx.y * kRtTok, nt = min(kRtTok, p.T - t0);
+  uint16_t* w = reinterpret_cast<uint16_t*>(sm);
+  if (tid == 0) {
+    const uint32_t bar = smem_addr(&s_bar);
+    mbar_init(bar, 1);
+    mbar_fence_init();
+    const int nr = max(0, min(n, E - r0));  // rows of w_router; the rest is the shared-gate row
+    mbar_expect_tx(bar, (uint32_t)n * H * 2);
+    if (nr > 0) bulk_g2s(smem_addr(w), rb.w_router + (size_t)r0 * H, (uint32_t)nr * H * 2, bar, l2_policy_evict_first());
+    if (nr < n) bulk_g2s(smem_addr(w + (size_t)nr * H), rb.w_sgate, (uint32_t)H * 2, bar, l2_policy_evict_first());
+  }
+  __syncthreads();
+  const bool ok = mbar_wait_bounded(smem_addr(&s_bar), 0, p.err);
+  const uint16_t* ws = w + warp * (H / 8);
+  for (int j = 0; ok && j < nt; ++j) {
+    const float* xs = rb.x + (size_t)(t0 + j) * H + warp * (H / 8);
+    float acc[kRtRows];
+#pragma unroll
+    for (int r = 0; r < kRtRows; ++r) acc[r] = 0.0f;
+    for (int k = lane; k < H / 64; k += 32) {
+      const float4 xa = __ldcg(reinterpret_cast<const float4*>(xs + 8 * k));
+      const float4 xb = __ldcg(reinterpret_cast<const float4*>(xs + 8 * k + 4));
+#pragma unroll
+      for (int r = 0; r < kRtRows; ++r) {
+        if (r < n) {
+          const uint4 q = *reinterpret_cast<const uint4*>(ws + (size_t)r * H + 8 * k);
+          float a = acc[r];
+          a = fmaf(__uint_as_float(q.x << 16), xa.x, a);
+          a = fmaf(__uint_as_float(q.x & 0xFFFF0000u), xa.y, a);
+          a = fmaf(__uint_as_float(q.y << 16), xa.z, a);
+          a = fmaf(__uint_as_float(q.y & 0xFFFF0000u), xa.w, a);
+          a = fmaf(__uint_as_float(q.z << 16), xb.x, a);
+          a = fmaf(__uint_as_float(q.z & 0xFFFF0000u), xb.y, a);
+          a = fmaf(__uint_as_float(q.w << 16), xb.z, a);
+          a = fmaf(__uint_as_float(q.w & 0xFFFF0000u), xb.w, a);
+          acc[r] = a;
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRtRows; ++r) acc[r] = warp_sum(acc[r]);
+    if (lane == 0)
+#pragma unroll
+      for (int r = 0; r < kRtRows; ++r) s_part[j][r][warp] = acc[r];
+  }
+  __syncthreads();
+  for (int i = tid; ok && i < nt * n; i += kGT) {
+    const int j = i / n, r = i % n;
+    float l = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kGT / 32; ++q) l += s_part[j][r][q];
+    const int row = r0 + r;
+    if (row < E && rb.bias) l += rb.bias[row];
+    const_cast<float*>(p.logits)[(size_t)(t0 + j) * (E + 1) + row] = l;
+  }
+}
+
+// The group of CTA slot u (u == 0: the shared expert, every token, scheduled
+// first because its groups are the largest; u >= 1: active expert u - 1):
 // record, number of tokens, and for token j its token index and output row.
 struct Group {
   const uint8_t* rec;
@@ -88,17 +262,18 @@ struct Group {
 
 __device__ __forceinline__ Group group_of(const GroupedParams& p, int u, int U) {
   Group g;
-  if (u == U) {
+  (void)U;
+  if (u == 0) {
     g.rec = p.shared.base;
     g.off = p.shared.off;
     g.n = p.T;
     g.first = -1;
   } else {
-    const int e = __ldcg(p.act_expert + u);
+    const int e = __ldcg(p.act_expert + u - 1);
     g.rec = p.routed.base + (long long)e * p.routed.stride;
     g.off = p.routed.off;
-    g.first = __ldcg(p.act_off + u);
-    g.n = __ldcg(p.act_off + u + 1) - g.first;
+    g.first = __ldcg(p.act_off + u - 1);
+    g.n = __ldcg(p.act_off + u) - g.first;
   }
   return g;
 }
@@ -385,14 +560,32 @@ cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
 }  // namespace
 
 bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T) {
-  if (T * K > kMaxTK || (size_t)2 * E * 4 > 48 * 1024) return false;
+  if (T * K > kMaxTK || ((size_t)T * K + 2 * (size_t)E) * 4 > 200 * 1024) return false;
+  if ((size_t)kRtRows * H * 2 > 200 * 1024) return false;
   if (H % kDnRows || I % kGuRows) return false;
   size_t smem = 0;
   return gu_smem(bits, H) <= 220 * 1024 && dn_tokens(bits, I, &smem) >= 1;
 }
 
 cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s) {
-  select_kernel<<<1, kGT, (size_t)2 * p.E * sizeof(int), s>>>(p);
+  topk_tokens_kernel<<<p.T, kGT, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = ((size_t)p.T * p.K + 2 * (size_t)p.E) * sizeof(int);
+  if ((e = set_smem((const void*)sort_pairs_kernel, smem)) != cudaSuccess) return e;
+  sort_pairs_kernel<<<1, kST, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s) {
+  norm_digits_kernel<<<p.T, kGT, 0, s>>>(p, rb, bits);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int R = p.E + 1;
+  const size_t smem = (size_t)kRtRows * p.H * 2;
+  void (*k)(const GroupedParams, const RouterBatch) = router_gemm_kernel;
+  if ((e = set_smem((const void*)k, smem)) != cudaSuccess) return e;
+  k<<<dim3((R + kRtRows - 1) / kRtRows, (p.T + kRtTok - 1) / kRtTok), kGT, smem, s>>>(p, rb);
   return cudaGetLastError();
 }
 
