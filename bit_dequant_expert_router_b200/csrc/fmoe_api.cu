@@ -73,8 +73,8 @@ WsLayout layout(int H, int E, int K, int I, int T) {
 // placed after the whole per-token layout (whose counters must stay zero
 // between calls); the control block is the per-token one at offset 0.
 struct GLayout {
-  size_t ctrl, logits, xq_limbs, xq_cs, route_idx, route_w, n_active, act_expert, act_off, pair_tok, pair_pos, act,
-      act_limbs, act_cs, y, x, total;
+  size_t ctrl, logits, xq_limbs, xq_cs, route_idx, route_w, n_active, act_expert, act_off, pair_tok, pair_pos, work,
+      act, act_limbs, act_cs, y, x, total;
 };
 
 GLayout glayout(int H, int E, int K, int I, int T) {
@@ -87,11 +87,12 @@ GLayout glayout(int H, int E, int K, int I, int T) {
   L.route_idx = L.xq_cs + up((size_t)T * (H / 32) * 8);
   L.route_w = L.route_idx + up(np * 4);
   L.n_active = L.route_w + up((size_t)T * (K + 1) * 4);
-  L.act_expert = L.n_active + up(4);
+  L.act_expert = L.n_active + up(8);
   L.act_off = L.act_expert + up(np * 4);
   L.pair_tok = L.act_off + up((np + 1) * 4);
   L.pair_pos = L.pair_tok + up(np * 4);
-  L.act = L.pair_pos + up(np * 4);
+  L.work = L.pair_pos + up(np * 4);
+  L.act = L.work + up(nr * sizeof(UnitDesc));
   L.act_limbs = L.act + up(nr * I * 4);
   L.act_cs = L.act_limbs + up(nr * 3 * I);
   L.y = L.act_cs + up(nr * (I / 32) * 8);
@@ -560,6 +561,7 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   p.act_off = reinterpret_cast<int32_t*>(base + G.act_off);
   p.pair_tok = reinterpret_cast<int32_t*>(base + G.pair_tok);
   p.pair_pos = reinterpret_cast<int32_t*>(base + G.pair_pos);
+  p.units = reinterpret_cast<UnitDesc*>(base + G.work);
   p.act = reinterpret_cast<float*>(base + G.act);
   p.act_limbs = base + G.act_limbs;
   p.act_cs = reinterpret_cast<float2*>(base + G.act_cs);

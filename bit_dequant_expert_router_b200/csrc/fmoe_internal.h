@@ -74,24 +74,37 @@ struct ExpertParams {
 // ---- expert-grouped path for batched decode (k_grouped.cu): T tokens, each active
 // expert's weights read once for all the tokens routed to it
 
+// A work unit of the grouped expert kernels: up to kUnitToks members of one
+// expert's group, whose rows in act / act_limbs / y are row0 .. row0 + n - 1.
+constexpr int kUnitToks = 2;
+struct alignas(16) UnitDesc {
+  int e;       // routed expert, -1 = the shared expert
+  int row0;    // first member row
+  int n;       // members
+  int pad;
+  int tok[4];  // token of each member (the first kUnitToks used)
+};
+static_assert(kUnitToks <= 4, "UnitDesc holds at most four members");
+
 struct GroupedParams {
   BankRef routed, shared;
   int T, E, K, H, I;
   const float* logits;        // [T][E+1] router logits (+ shared-gate logit)
-  const uint8_t* xq_limbs;    // [T][3H] digits of x per token
-  const float2* xq_cs;        // [T][H*bits/128]
+  const uint8_t* xq_limbs;    // [T][3H] digits of x per token, tensor-core layout
+  const float2* xq_cs;        // [T][H/64] per group {digit scale, sum of x}
   int32_t* route_idx;         // [T][K]
   float* route_w;             // [T][K+1], slot K = sigma
   int32_t* idx_out;           // caller's copies [T][K] or NULL
   float* w_out;
-  int32_t* n_active;          // [1] U: active experts
+  int32_t* n_active;          // [2] U: active experts, W: work units
+  UnitDesc* units;            // [T*K + T] work units of the expert kernels, the shared expert's first
   int32_t* act_expert;        // [T*K] active experts, increasing
   int32_t* act_off;           // [T*K+1] first pair of each active expert in the sorted pair list
   int32_t* pair_tok;          // [T*K] sorted pairs (expert, token, k): value t*K + k
   int32_t* pair_pos;          // [T*K] position of pair t*K + k in the sorted list
   float* act;                 // [(T*K + T)][I] SwiGLU outputs: sorted pairs, then the shared expert per token
-  uint8_t* act_limbs;         // [(T*K + T)][3I]
-  float2* act_cs;             // [(T*K + T)][I*bits/128]
+  uint8_t* act_limbs;         // [(T*K + T)][3I], tensor-core layout
+  float2* act_cs;             // [(T*K + T)][I/64]
   float* y;                   // [(T*K + T)][H] down outputs (unweighted)
   const float* h;             // [T][H] residual
   float* out;                 // [T][H]

@@ -25,13 +25,68 @@ namespace fmoe {
 namespace {
 
 constexpr int kGT = 256;          // threads per CTA
-constexpr int kGuRows = 16;       // gate/up row pairs per CTA
-constexpr int kGuTok = 2;         // tokens whose digits are staged at once (gate/up)
-constexpr int kDnRows = 32;       // down output rows per CTA
-constexpr int kDnTok = 16;        // tokens whose activation digits are staged at once (down)
 constexpr int kMaxTK = 4096;      // T*K pairs
 constexpr int kRtRows = 8;        // router rows per CTA (batched router)
 constexpr int kRtTok = 16;        // tokens per CTA (batched router)
+
+// ---- int8 tensor-core contraction of codes with activation digits.
+// The batched expert products run on mma.sync m16n8k32 (u8 codes x s8 digits,
+// s32 accumulate).  A tile is 16 weight rows x 8 columns, a column being one
+// limb of one token's digits (3 limbs per token, two tokens per tile); K runs
+// over one group of 64 in two k-blocks of 32, so that every group's int32 sums
+// are scaled on their own (s * cscale * S + b * sum x, per the fold above).
+//
+// Lane (gid, q) of the quad layout (gid = lane / 4, q = lane % 4) holds the A
+// registers {row gid k-lo, row gid+8 k-lo, row gid k-hi, row gid+8 k-hi} and the
+// B registers {k-lo, k-hi} of column gid, k-lo being k-slots 4q..4q+3 and k-hi
+// 16+4q..16+4q+3.  A code word unpacks into those byte registers directly:
+//   4-bit, k-block kb: word 2q+kb of the group's row; k-lo = low nibbles
+//     (columns 16q + 8kb + 2j), k-hi = high nibbles (the next column each);
+//   2-bit, k-block kb: word q; k-lo = 2-bit pack 2kb (columns 16q + 4j + 2kb),
+//     k-hi = pack 2kb+1 (the next column each).
+// The digits are stored so that each (k-block, limb, q) is one 8-byte pair
+// {k-lo, k-hi}: word ((kb*3 + L)*4 + q)*2 + {0, 1}, byte j; 192 bytes per group.
+// Per group one float2 {cscale, sum of x over the group}.
+
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Quantises one group of 64 values (lane l holds columns 2l, 2l+1) into the
+// layout above: the same fixed-point digits as the per-token format (cscale =
+// 2^(e-22) from the group's largest magnitude), only placed differently.
+template <int BITS>
+__device__ __forceinline__ void tc_quantize_group(float v0, float v1, uint8_t* glimbs, float2* gcs) {
+  const int lane = threadIdx.x & 31;
+  const float m = warp_max(fmaxf(fabsf(v0), fabsf(v1)));
+  int e = 0;
+  if (m > 0.0f) {
+    const int ef = (int)((__float_as_uint(m) >> 23) & 0xFFu);
+    e = ef == 0 ? -125 : ef - 126;  // m < 2^e
+  }
+  e = e < -100 ? -100 : (e > 100 ? 100 : e);
+  const float inv = __uint_as_float((uint32_t)(127 + 22 - e) << 23);  // 2^(22-e)
+  const float csc = __uint_as_float((uint32_t)(127 + e - 22) << 23);  // 2^(e-22)
+  const int c = 2 * lane;  // columns c (k-lo) and c + 1 (k-hi) share k-block, quad lane and byte
+  const int q = c >> 4;
+  const int kb = BITS == 4 ? (c >> 3) & 1 : (c & 3) >> 1;
+  const int j = BITS == 4 ? (c & 7) >> 1 : (c & 15) >> 2;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int X = __float2int_rn((r ? v1 : v0) * inv);
+    const int d2 = ((X + 128) & 255) - 128;
+    const int X1 = (X - d2) >> 8;
+    const int d1 = ((X1 + 128) & 255) - 128;
+    const int d0 = (X1 - d1) >> 8;
+    const int d[3] = {d0, d1, d2};
+#pragma unroll
+    for (int L = 0; L < 3; ++L) glimbs[((((kb * 3 + L) * 4 + q) * 2 + r) << 2) + j] = (uint8_t)(int8_t)d[L];
+  }
+  const float sx = warp_sum(v0 + v1);
+  if (lane == 0) *gcs = make_float2(csc, sx);
+}
 
 // ---- selection, in two kernels.  topk: one CTA per token, the block-wide
 // two-stage top-K (ties to the lower index) with renormalised weights and the
@@ -86,6 +141,11 @@ __device__ __forceinline__ int block_scan_excl(int v, int* s_warp, int* total) {
 // sort: one CTA.  Counting sort of the T*K pairs by expert, stable in (token, k)
 // order: the rank of pair i among the pairs of its expert is the number of
 // earlier pairs with the same expert.  Active experts in increasing order.
+// Then the work units of the expert kernels: each group (the shared expert's
+// T tokens first, then every active expert's pairs) cut into runs of at most
+// kUnitToks members, so that no unit of work is much heavier than another.
+// A unit is written out whole (UnitDesc) so that the expert kernels find it
+// with one load.
 __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) {
   extern __shared__ __align__(16) int s_mem[];  // [T*K] experts of the pairs, [E] counts, [E] starts
   __shared__ int s_warp[kST / 32];
@@ -103,17 +163,20 @@ __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) 
   __syncthreads();
   // starts of the experts (exclusive scan of the counts) and slots of the active ones
   const int per = (E + kST - 1) / kST;  // experts per thread, contiguous
-  int c = 0, a = 0;
+  const int C = kUnitToks, nsh = (p.T + C - 1) / C;
+  int c = 0, a = 0, w = 0;
   for (int k = 0; k < per; ++k) {
     const int e = tid * per + k;
     if (e < E) {
       c += s_cnt[e];
       a += s_cnt[e] > 0;
+      w += (s_cnt[e] + C - 1) / C;
     }
   }
-  int tot_c, tot_a;
+  int tot_c, tot_a, tot_w;
   int run = block_scan_excl(c, s_warp, &tot_c);
   int slot = block_scan_excl(a, s_warp, &tot_a);
+  int wpos = nsh + block_scan_excl(w, s_warp, &tot_w);
   for (int k = 0; k < per; ++k) {
     const int e = tid * per + k;
     if (e < E) {
@@ -122,13 +185,18 @@ __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) 
         p.act_expert[slot] = e;
         p.act_off[slot] = run;
         ++slot;
+        for (int j0 = 0; j0 < s_cnt[e]; j0 += C, ++wpos)
+          p.units[wpos] = UnitDesc{e, run + j0, min(C, s_cnt[e] - j0), 0, {0, 0, 0, 0}};
       }
       run += s_cnt[e];
     }
   }
+  for (int i = tid; i < nsh; i += kST)  // the shared expert's members are all T tokens, rows T*K + t
+    p.units[i] = UnitDesc{-1, N + i * C, min(C, p.T - i * C), 0, {0, 0, 0, 0}};
   if (tid == 0) {
     p.act_off[tot_a] = tot_c;
-    *p.n_active = tot_a;
+    p.n_active[0] = tot_a;
+    p.n_active[1] = nsh + tot_w;
   }
   __syncthreads();
   for (int i = tid; i < N; i += kST) {
@@ -138,6 +206,13 @@ __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) 
     const int pos = s_start[e] + rank;
     p.pair_tok[pos] = i;
     p.pair_pos[i] = pos;
+  }
+  __syncthreads();  // the units' tokens: from the sorted pairs (routed) or the row (shared)
+  const int NW = nsh + tot_w;
+  for (int i = tid; i < NW * kUnitToks; i += kST) {
+    UnitDesc& d = p.units[i / kUnitToks];
+    const int jj = i % kUnitToks;
+    if (jj < d.n) d.tok[jj] = d.e < 0 ? d.row0 - N + jj : p.pair_tok[d.row0 + jj] / p.K;
   }
 }
 
@@ -174,13 +249,13 @@ __global__ void __launch_bounds__(kGT) norm_digits_kernel(const GroupedParams p,
   __syncthreads();  // this CTA's x is written (read back through L1-bypassing loads below)
   __threadfence_block();
   uint8_t* limbs = const_cast<uint8_t*>(p.xq_limbs) + (size_t)t * 3 * H;
-  float2* cs = const_cast<float2*>(p.xq_cs) + (size_t)t * (H / 32);
+  float2* cs = const_cast<float2*>(p.xq_cs) + (size_t)t * (H / kGroup);
   for (int g = warp; g < H / kGroup; g += kGT / 32) {
     const float2 v = __ldcg(reinterpret_cast<const float2*>(x + g * kGroup) + lane);
     if (bits == 4)
-      xq_quantize_group<4>(v.x, v.y, g, H / kGroup, limbs, cs);
+      tc_quantize_group<4>(v.x, v.y, limbs + g * 192, cs + g);
     else
-      xq_quantize_group<2>(v.x, v.y, g, H / kGroup, limbs, cs);
+      tc_quantize_group<2>(v.x, v.y, limbs + g * 192, cs + g);
   }
 }
 
@@ -250,140 +325,367 @@ __global__ void __launch_bounds__(kGT) router_gemm_kernel(const GroupedParams p,
   }
 }
 
-// The group of CTA slot u (u == 0: the shared expert, every token, scheduled
-// first because its groups are the largest; u >= 1: active expert u - 1):
-// record, number of tokens, and for token j its token index and output row.
-struct Group {
-  const uint8_t* rec;
-  const long long* off;
-  int n;      // tokens in the group
-  int first;  // routed: first sorted pair; shared: -1
+// ---- the two expert kernels share one schedule.  Persistent, one CTA per SM,
+// 8 consumer warps and 1 producer warp.  The items are the row blocks of the
+// work units (item i = block i % NB of unit i / NB); CTA c takes the contiguous
+// range [c*N/P, (c+1)*N/P), so consecutive items read neighbouring rows of one
+// expert and share the unit's digits, which are staged once per unit.  The
+// producer stages each item's rows into a ring of `ns` buffers (full / empty
+// mbarriers per buffer) and each unit's digits into one of two slots; the
+// consumers sum, then reduce their partial tiles and write the outputs.
+constexpr int kConsumers = 8;                      // consumer warps
+constexpr int kThreads = (kConsumers + 1) * 32;    // + the producer warp
+constexpr int kRing = 16;                          // item descriptors in flight (> the largest ns)
+constexpr int kPad = 32;                           // bytes after each staged copy group of rows
+
+struct ItemDesc {
+  UnitDesc u;
+  int blk;    // row block within the unit
+  int useq;   // unit sequence number within this CTA: digit slot useq & 1
+  int first;  // first item of its unit here (consumers wait for the digits)
+  int last;   // last item of its unit here (consumers release the digit slot)
 };
 
-__device__ __forceinline__ Group group_of(const GroupedParams& p, int u, int U) {
-  Group g;
-  (void)U;
-  if (u == 0) {
-    g.rec = p.shared.base;
-    g.off = p.shared.off;
-    g.n = p.T;
-    g.first = -1;
-  } else {
-    const int e = __ldcg(p.act_expert + u - 1);
-    g.rec = p.routed.base + (long long)e * p.routed.stride;
-    g.off = p.routed.off;
-    g.first = __ldcg(p.act_off + u - 1);
-    g.n = __ldcg(p.act_off + u) - g.first;
-  }
-  return g;
+__device__ __forceinline__ UnitDesc load_unit(const GroupedParams& p, int wi) {
+  const int4* src = reinterpret_cast<const int4*>(p.units + wi);
+  const int4 a = __ldcg(src), b = __ldcg(src + 1);
+  return UnitDesc{a.x, a.y, a.z, a.w, {b.x, b.y, b.z, b.w}};
 }
 
-// token and output row (into act / y) of member j of a group
-__device__ __forceinline__ void member(const GroupedParams& p, const Group& g, int j, int& tok, int& row) {
-  if (g.first < 0) {
-    tok = j;
-    row = p.T * p.K + j;
-  } else {
-    const int pr = __ldcg(p.pair_tok + g.first + j);
-    tok = pr / p.K;
-    row = g.first + j;
+__device__ __forceinline__ const uint8_t* unit_record(const GroupedParams& p, int e) {
+  return e < 0 ? p.shared.base : p.routed.base + (long long)e * p.routed.stride;
+}
+
+// this CTA's items [i0, i0 + count)
+__device__ __forceinline__ void item_range(const GroupedParams& p, int NB, int& i0, int& count) {
+  const long long n = (long long)__ldcg(p.n_active + 1) * NB, P = gridDim.x, c = blockIdx.x;
+  i0 = (int)(c * n / P);
+  count = (int)((c + 1) * n / P) - i0;
+}
+
+// barrier of the consumer warps that also ORs a predicate over them
+__device__ __forceinline__ bool named_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, 1, %2, p; selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kConsumers * 32)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive_one(uint32_t bar) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(bar) : "memory");
+}
+
+// The producer loop (lane 0 plans and waits; `issue_w(it, stage)` and
+// `issue_d(unit, slot)` are called by the whole warp and arm their barrier on
+// lane 0 first).  On a timeout, or when the consumers gave up, it stops
+// issuing and waits (bounded) for the copies it has in flight, then returns.
+template <typename IW, typename ID>
+__device__ __forceinline__ void producer_loop(const GroupedParams& p, int NB, int i0, int count, int ns,
+                                              ItemDesc* s_item, uint64_t* wfull, uint64_t* wempty, uint64_t* dfull,
+                                              uint64_t* dempty, volatile int* s_abort, IW issue_w, ID issue_d) {
+  const int lane = threadIdx.x & 31;
+  int prev = -1, useq = -1, issued = 0, dissued = 0;
+  bool ok = true;
+  UnitDesc u{};
+  for (int k = 0; k < count && ok; ++k) {
+    const int item = i0 + k, wi = item / NB, blk = item % NB;
+    if (lane == 0 && k >= ns) ok = mbar_wait_bounded(smem_addr(&wempty[k % ns]), (uint32_t)(((k / ns) - 1) & 1), p.err);
+    if (lane == 0 && *s_abort) ok = false;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    const bool first = wi != prev;
+    if (first) {
+      ++useq;
+      prev = wi;
+      if (lane == 0) {
+        u = load_unit(p, wi);
+        if (useq >= 2) ok = mbar_wait_bounded(smem_addr(&dempty[useq & 1]), (uint32_t)(((useq >> 1) - 1) & 1), p.err);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+    }
+    const bool last = k + 1 == count || (item + 1) / NB != wi;
+    if (lane == 0) s_item[k % kRing] = ItemDesc{u, blk, useq, first ? 1 : 0, last ? 1 : 0};
+    __syncwarp();
+    if (first) {
+      issue_d(s_item[k % kRing].u, useq & 1);
+      dissued = useq + 1;
+    }
+    issue_w(s_item[k % kRing], k % ns);  // its arrive releases the descriptor to the consumers
+    issued = k + 1;
+  }
+  if (!ok && lane == 0) {  // let every copy in flight land before the CTA can leave
+    *s_abort = 1;
+    for (int k = issued - ns > 0 ? issued - ns : 0; k < issued; ++k)
+      mbar_wait_bounded(smem_addr(&wfull[k % ns]), (uint32_t)((k / ns) & 1), p.err);
+    for (int q = dissued - 2 > 0 ? dissued - 2 : 0; q < dissued; ++q)
+      mbar_wait_bounded(smem_addr(&dfull[q & 1]), (uint32_t)((q >> 1) & 1), p.err);
   }
 }
 
-
-// ---- gate/up + SwiGLU: CTA (u, b) = active expert slot u, row pairs [16b, 16b+16).
-// The rows are staged once; the digits of x of kGuTok tokens of the group at a
-// time.  Lane geometry as in the per-token kernel (Geo<NG>): a lane owns GPL
-// groups of 64 columns, a warp one row pair per pass (RPP when NG < 32).
+// Shapes of one staged row and of one token's (or activation row's) digits.
 template <int BITS, int NG>
-__global__ void __launch_bounds__(kGT) grouped_gateup_kernel(const GroupedParams p) {
-  using G = Geo<NG>;
-  constexpr int LPR = G::kLanesPerRow, RPP = G::kRowsPerPass, GPL = G::kGroupsPerLane;
-  constexpr int RB = NG * kGroup * BITS / 8, SB = NG * 2;
-  constexpr int NCX = NG * kGroup * BITS / 128;              // chunk scalars of x
-  constexpr int DIG = NG * kGroupWords * 4 + NCX * 8;        // staged bytes per token
-  constexpr int WB = kGuRows * (2 * RB + 4 * SB);            // staged weight bytes
+struct TcRows {
+  static constexpr int RB = NG * kGroup * BITS / 8;
+  static constexpr int GPW = NG >= 8 ? NG / 8 : 1;  // groups per warp (K is split over the 8 warps)
+  static constexpr int LB = NG * 192;               // digit bytes of one token / activation row
+  static constexpr int CB = NG * 8;                 // its per-group scalars
+};
+
+// A registers of rows (gid, gid + 8) for k-block kb of group g from staged rows.
+template <int BITS>
+__device__ __forceinline__ void tc_load_a(const uint8_t* r_lo, const uint8_t* r_hi, int g, int q, uint32_t (&w)[2][2]) {
+  if (BITS == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(r_lo + g * 32 + 8 * q);
+    const uint2 y = *reinterpret_cast<const uint2*>(r_hi + g * 32 + 8 * q);
+    w[0][0] = x.x; w[0][1] = x.y; w[1][0] = y.x; w[1][1] = y.y;
+  } else {
+    const uint32_t x = *reinterpret_cast<const uint32_t*>(r_lo + g * 16 + 4 * q);
+    const uint32_t y = *reinterpret_cast<const uint32_t*>(r_hi + g * 16 + 4 * q);
+    w[0][0] = w[0][1] = x; w[1][0] = w[1][1] = y;
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void tc_unpack_a(const uint32_t (&w)[2][2], int kb, uint32_t (&a)[4]) {
+  if (BITS == 4) {
+    a[0] = w[0][kb] & 0x0F0F0F0Fu;
+    a[1] = w[1][kb] & 0x0F0F0F0Fu;
+    a[2] = (w[0][kb] >> 4) & 0x0F0F0F0Fu;
+    a[3] = (w[1][kb] >> 4) & 0x0F0F0F0Fu;
+  } else {
+    a[0] = (w[0][kb] >> (4 * kb)) & 0x03030303u;
+    a[1] = (w[1][kb] >> (4 * kb)) & 0x03030303u;
+    a[2] = (w[0][kb] >> (4 * kb + 2)) & 0x03030303u;
+    a[3] = (w[1][kb] >> (4 * kb + 2)) & 0x03030303u;
+  }
+}
+
+// GPW consecutive bf16 values (a warp's groups of one staged scale row) into
+// packed registers, two per word.
+template <int GPW>
+__device__ __forceinline__ void tc_load_scales(const uint16_t* src, uint32_t (&v)[(GPW + 1) / 2]) {
+  if constexpr (GPW == 1) {
+    v[0] = src[0];
+  } else if constexpr (GPW == 2) {
+    v[0] = *reinterpret_cast<const uint32_t*>(src);
+  } else if constexpr (GPW == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(src);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < GPW / 8; ++i) {
+      const uint4 x = reinterpret_cast<const uint4*>(src)[i];
+      v[4 * i] = x.x;
+      v[4 * i + 1] = x.y;
+      v[4 * i + 2] = x.z;
+      v[4 * i + 3] = x.w;
+    }
+  }
+}
+
+template <int GPW>
+__device__ __forceinline__ float tc_scale(const uint32_t (&v)[(GPW + 1) / 2], int gi) {
+  return __uint_as_float((gi & 1) ? (v[gi >> 1] & 0xFFFF0000u) : (v[gi >> 1] << 16));
+}
+
+// The quad lane's two columns: column c = 3 t + L (token t of the tile, limb
+// L), columns 6 and 7 unused.  Per group: the scale of the int32 sum and the
+// bias factor (sum of x / 2^16 on limb 0, whose weight 2^16 is applied last).
+struct TcCol {
+  int t;     // token of the tile, -1 = unused column
+  bool l0;   // limb 0
+};
+
+__device__ __forceinline__ TcCol tc_col(int c, int n) {
+  TcCol k;
+  k.t = (c < 6 && c / 3 < n) ? c / 3 : -1;
+  k.l0 = c % 3 == 0;
+  return k;
+}
+
+// ---- gate/up + SwiGLU.  An item is 8*RPC (gate, up) row pairs, staged as 8
+// copy groups of RPC consecutive rows per matrix (plus kPad bytes each), so
+// that the 8 rows one quad-layout load reads sit in 8 distinct groups.  Tile
+// mt pairs gate row RPC*gid + mt (A rows 0-7) with the same up row (rows 8-15).
+// The digits are those of x for each member token.  Warp w sums groups
+// [w*GPW, w*GPW + GPW); the eight partial tiles add in warp order.
+// act[row][r] = silu(g) * u.
+template <int BITS, int NG, int RPC>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const GroupedParams p, int ns) {
+  using R = TcRows<BITS, NG>;
+  constexpr int RB = R::RB, GPW = R::GPW, LB = R::LB, CB = R::CB, SB = NG * 2;
+  constexpr int ROWS = 8 * RPC;                     // row pairs per item
+  constexpr int GP = RPC * RB + kPad;               // one staged copy group
+  constexpr int WB = 16 * GP + 4 * ROWS * SB;       // gate groups, up groups, gate s, gate b, up s, up b
+  constexpr int DB = kUnitToks * (LB + CB);
+  constexpr int TP = 2 * ROWS * 8 + 4;              // floats per warp's partial tiles (gate rows, then up rows)
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ __align__(8) uint64_t s_wbar;
-  __shared__ __align__(8) uint64_t s_dbar;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int U = __ldcg(p.n_active);
-  const int u = blockIdx.x;
-  if (u > U) return;  // block-uniform
-  const Group grp = group_of(p, u, U);
-  const int H = p.H, I = p.I;
-  const int r0 = blockIdx.y * kGuRows;
-  uint8_t* dbuf = sm + WB;
-  const uint64_t pol = l2_policy_evict_first();
+  __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
+  __shared__ ItemDesc s_item[kRing];
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, q = lane & 3;
+  const int I = p.I, NB = I / ROWS;
+  int i0, count;
+  item_range(p, NB, i0, count);
+  uint8_t* dbase = sm + (size_t)ns * WB;
+  float* red = reinterpret_cast<float*>(dbase + 2 * DB);  // [2][kConsumers][TP]
   if (tid == 0) {
-    mbar_init(smem_addr(&s_wbar), 1);
-    mbar_init(smem_addr(&s_dbar), 1);
+    for (int i = 0; i < ns; ++i) {
+      mbar_init(smem_addr(&s_wfull[i]), 1);
+      mbar_init(smem_addr(&s_wempty[i]), kConsumers);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&s_dfull[i]), 1);
+      mbar_init(smem_addr(&s_dempty[i]), kConsumers);
+    }
     mbar_fence_init();
-    const uint32_t bw = smem_addr(&s_wbar), dst = smem_addr(sm);
-    const uint32_t cb = kGuRows * RB, sbb = kGuRows * SB;
-    mbar_expect_tx(bw, 2 * cb + 4 * sbb);
-    bulk_g2s(dst, grp.rec + grp.off[0] + (long long)r0 * RB, cb, bw, pol);
-    bulk_g2s(dst + cb, grp.rec + grp.off[3] + (long long)r0 * RB, cb, bw, pol);
-    bulk_g2s(dst + 2 * cb, grp.rec + grp.off[1] + (long long)r0 * SB, sbb, bw, pol);
-    bulk_g2s(dst + 2 * cb + sbb, grp.rec + grp.off[2] + (long long)r0 * SB, sbb, bw, pol);
-    bulk_g2s(dst + 2 * cb + 2 * sbb, grp.rec + grp.off[4] + (long long)r0 * SB, sbb, bw, pol);
-    bulk_g2s(dst + 2 * cb + 3 * sbb, grp.rec + grp.off[5] + (long long)r0 * SB, sbb, bw, pol);
+    s_abort = 0;
   }
   __syncthreads();
-  bool ok = mbar_wait_bounded(smem_addr(&s_wbar), 0, p.err);
-  const int sub = lane / LPR, gl = lane % LPR;
-  const uint16_t* scl = reinterpret_cast<const uint16_t*>(sm + 2 * kGuRows * RB);
-  for (int j0 = 0, it = 0; j0 < grp.n; j0 += kGuTok, ++it) {
-    const int nb = min(kGuTok, grp.n - j0);
-    if (tid == 0) {
-      const uint32_t bd = smem_addr(&s_dbar);
-      fence_proxy_async();
-      mbar_expect_tx(bd, (uint32_t)nb * DIG);
-      for (int jj = 0; jj < nb; ++jj) {
-        int tok, row;
-        member(p, grp, j0 + jj, tok, row);
-        bulk_g2s(smem_addr(dbuf + jj * DIG), p.xq_limbs + (size_t)tok * 3 * H, NG * kGroupWords * 4, bd, pol);
-        bulk_g2s(smem_addr(dbuf + jj * DIG + NG * kGroupWords * 4), p.xq_cs + (size_t)tok * (H / 32), NCX * 8, bd, pol);
+
+  if (warp == kConsumers) {  // the producer
+    const uint64_t pol_w = l2_policy_evict_first(), pol_d = l2_policy_evict_last();
+    auto issue_w = [&](const ItemDesc& it, int st) {
+      const uint8_t* rec = unit_record(p, it.u.e);
+      const long long r0 = (long long)it.blk * ROWS;
+      const uint32_t bw = smem_addr(&s_wfull[st]), dst = smem_addr(sm + (size_t)st * WB);
+      if (lane == 0) mbar_expect_tx(bw, 2 * ROWS * RB + 4 * ROWS * SB);
+      __syncwarp();
+      if (lane < 16) {  // copy group lane % 8 of the gate (lanes 0-7) or up (8-15) rows
+        const int j = lane & 7;
+        const long long off = lane < 8 ? p.routed.off[0] : p.routed.off[3];
+        bulk_g2s(dst + (lane >> 3) * 8 * GP + j * GP, rec + off + (r0 + RPC * j) * RB, RPC * RB, bw, pol_w);
+      } else if (lane < 20) {  // gate s, gate b, up s, up b
+        const int a = lane - 16;
+        const long long off = p.routed.off[a == 0 ? 1 : a == 1 ? 2 : a == 2 ? 4 : 5];
+        bulk_g2s(dst + 16 * GP + a * ROWS * SB, rec + off + r0 * SB, ROWS * SB, bw, pol_w);
+      }
+    };
+    auto issue_d = [&](const UnitDesc& u, int slot) {
+      const uint32_t bd = smem_addr(&s_dfull[slot]);
+      uint8_t* dst = dbase + (size_t)slot * DB;
+      if (lane == 0) mbar_expect_tx(bd, (uint32_t)u.n * (LB + CB));
+      __syncwarp();
+      if (lane < u.n) {
+        const int tok = u.tok[lane];
+        bulk_g2s(smem_addr(dst + lane * LB), p.xq_limbs + (size_t)tok * LB, LB, bd, pol_d);
+        bulk_g2s(smem_addr(dst + kUnitToks * LB + lane * CB), p.xq_cs + (size_t)tok * NG, CB, bd, pol_d);
+      }
+    };
+    producer_loop(p, NB, i0, count, ns, s_item, s_wfull, s_wempty, s_dfull, s_dempty, &s_abort, issue_w, issue_d);
+    return;
+  }
+
+  const int g0 = warp * GPW;
+  const bool kwarp = g0 < NG;  // this warp has groups to sum
+  for (int k = 0; k < count; ++k) {
+    const int st = k % ns;
+    bool ok = mbar_wait_bounded(smem_addr(&s_wfull[st]), (uint32_t)((k / ns) & 1), p.err);
+    const ItemDesc it = s_item[k % kRing];
+    const int slot = it.useq & 1;
+    if (ok && it.first) ok = mbar_wait_bounded(smem_addr(&s_dfull[slot]), (uint32_t)((it.useq >> 1) & 1), p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    const uint8_t* wb = sm + (size_t)st * WB;
+    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + 16 * GP);
+    const uint8_t* db = dbase + (size_t)slot * DB;
+    float acc[RPC][4];
+#pragma unroll
+    for (int mt = 0; mt < RPC; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+    if (ok && kwarp) {
+      const int n = it.u.n;
+      const TcCol ca = tc_col(2 * q, n), cb = tc_col(2 * q + 1, n);
+      const int bt = gid / 3, bl = gid % 3;  // this lane's B column: token, limb
+      const bool bvalid = gid < 6 && bt < n;
+      const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
+      const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);
+      uint32_t sv[RPC][4][(GPW + 1) / 2];  // gate s, gate b, up s, up b of row pair RPC*gid + mt, this warp's groups
+#pragma unroll
+      for (int mt = 0; mt < RPC; ++mt)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) tc_load_scales<GPW>(scl + (a * ROWS + RPC * gid + mt) * NG + g0, sv[mt][a]);
+#pragma unroll
+      for (int gi = 0; gi < GPW; ++gi) {
+        const int g = g0 + gi;
+        uint2 b[2];
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+          b[kb] = bvalid ? *reinterpret_cast<const uint2*>(bsrc + g * 192 + kb * 96) : make_uint2(0u, 0u);
+        float sa = 0.0f, ba = 0.0f, sb_ = 0.0f, bb = 0.0f;
+        if (ca.t >= 0) {
+          const float2 v = csv[ca.t * NG + g];
+          sa = v.x;
+          ba = ca.l0 ? v.y * 0x1p-16f : 0.0f;
+        }
+        if (cb.t >= 0) {
+          const float2 v = csv[cb.t * NG + g];
+          sb_ = v.x;
+          bb = cb.l0 ? v.y * 0x1p-16f : 0.0f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < RPC; ++mt) {
+          uint32_t w[2][2];
+          tc_load_a<BITS>(wb + gid * GP + mt * RB, wb + 8 * GP + gid * GP + mt * RB, g, q, w);
+          int c[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            uint32_t a[4];
+            tc_unpack_a<BITS>(w, kb, a);
+            mma_u8s8(c, a, b[kb].x, b[kb].y);
+          }
+          const float gs = tc_scale<GPW>(sv[mt][0], gi), gb = tc_scale<GPW>(sv[mt][1], gi);
+          const float us = tc_scale<GPW>(sv[mt][2], gi), ub = tc_scale<GPW>(sv[mt][3], gi);
+          acc[mt][0] = fmaf(gs * sa, (float)c[0], fmaf(gb, ba, acc[mt][0]));
+          acc[mt][1] = fmaf(gs * sb_, (float)c[1], fmaf(gb, bb, acc[mt][1]));
+          acc[mt][2] = fmaf(us * sa, (float)c[2], fmaf(ub, ba, acc[mt][2]));
+          acc[mt][3] = fmaf(us * sb_, (float)c[3], fmaf(ub, bb, acc[mt][3]));
+        }
       }
     }
-    if (!mbar_wait_bounded(smem_addr(&s_dbar), (uint32_t)(it & 1), p.err)) ok = false;
-    for (int jj = 0; ok && jj < nb; ++jj) {
-      int tok, row;
-      member(p, grp, j0 + jj, tok, row);
-      const uint32_t* xl = reinterpret_cast<const uint32_t*>(dbuf + jj * DIG);
-      const float2* xc = reinterpret_cast<const float2*>(dbuf + jj * DIG + NG * kGroupWords * 4);
-      uint32_t L[GPL][48];
-      float2 cs[GPL];
+    __syncwarp();
+    if (lane == 0) {  // this warp is done with the item's rows (and, on its last item, the unit's digits)
+      mbar_arrive_one(smem_addr(&s_wempty[st]));
+      if (it.last) mbar_arrive_one(smem_addr(&s_dempty[slot]));
+    }
+    float* rw = red + ((k & 1) * kConsumers + warp) * TP;
 #pragma unroll
-      for (int q = 0; q < GPL; ++q) {
-        load_group_limbs(xl, gl + LPR * q, NG, L[q]);
-        cs[q] = group_scalars<BITS>(xc, gl + LPR * q);
-      }
-      for (int pr = warp; pr * RPP < kGuRows; pr += kGT / 32) {
-        const int r = pr * RPP + sub;  // row pair within the block
-        float ag = 0.0f, au = 0.0f;
+    for (int mt = 0; mt < RPC; ++mt) {
+      const int r = RPC * gid + mt;
+      *reinterpret_cast<float2*>(rw + r * 8 + 2 * q) = make_float2(acc[mt][0], acc[mt][1]);
+      *reinterpret_cast<float2*>(rw + (ROWS + r) * 8 + 2 * q) = make_float2(acc[mt][2], acc[mt][3]);
+    }
+    // partial tiles in place (double-buffered: item k + 2 writes these only after
+    // the next barrier); a wait that ran out anywhere ends every consumer here
+    if (named_sync_or(!ok)) {
+      if (tid == 0) s_abort = 1;
+      return;
+    }
+    const int r0 = it.blk * ROWS;
 #pragma unroll
-        for (int q = 0; q < GPL; ++q) {
-          const int g = gl + LPR * q;
-          uint4 q0, q1, v0, v1;
-          load_group_codes<BITS>(sm + r * RB, g, q0, q1);
-          load_group_codes<BITS>(sm + kGuRows * RB + r * RB, g, v0, v1);
-          const float gs = bf16_to_f32(scl[r * NG + g]), gb = bf16_to_f32(scl[kGuRows * NG + r * NG + g]);
-          const float us = bf16_to_f32(scl[2 * kGuRows * NG + r * NG + g]);
-          const float ub = bf16_to_f32(scl[3 * kGuRows * NG + r * NG + g]);
-          const float Sg = group_dot<BITS>(q0, q1, L[q]);
-          const float Su = group_dot<BITS>(v0, v1, L[q]);
-          ag = fmaf(gs, cs[q].x * Sg, fmaf(gb, cs[q].y, ag));
-          au = fmaf(us, cs[q].x * Su, fmaf(ub, cs[q].y, au));
+    for (int pass = 0; pass < (16 * ROWS + kConsumers * 32 - 1) / (kConsumers * 32); ++pass) {
+      const int idx = pass * kConsumers * 32 + tid;
+      if (idx < 16 * ROWS) {  // output (row pair r, token t) from warp slice ws, then the slices in order
+        const int o = idx >> 3, ws = idx & 7, r = o >> 1, t = o & 1;
+        const float* rs = red + ((k & 1) * kConsumers + ws) * TP + 3 * t;
+        float gv = 0.0f, uv = 0.0f;
+#pragma unroll
+        for (int L = 0; L < 3; ++L) {
+          const float f = L == 0 ? 65536.0f : L == 1 ? 256.0f : 1.0f;
+          gv = fmaf(f, rs[r * 8 + L], gv);
+          uv = fmaf(f, rs[(ROWS + r) * 8 + L], uv);
         }
-        for (int o = LPR / 2; o > 0; o >>= 1) {
-          ag += __shfl_xor_sync(0xffffffffu, ag, o);
-          au += __shfl_xor_sync(0xffffffffu, au, o);
+#pragma unroll
+        for (int o2 = 1; o2 < 8; o2 <<= 1) {
+          gv += __shfl_xor_sync(0xffffffffu, gv, o2);
+          uv += __shfl_xor_sync(0xffffffffu, uv, o2);
         }
-        if (gl == 0) p.act[(size_t)row * I + r0 + r] = ag / (1.0f + expf(-ag)) * au;
+        if (ws == 0 && t < it.u.n) p.act[(size_t)(it.u.row0 + t) * I + r0 + r] = gv / (1.0f + expf(-gv)) * uv;
       }
     }
-    __syncthreads();  // the digit buffer is free for the next tokens
   }
 }
 
@@ -395,91 +697,174 @@ __global__ void __launch_bounds__(kGT) grouped_actq_kernel(const GroupedParams p
   if (gw >= (p.T * p.K + p.T) * NGI) return;  // warp-uniform
   const int row = gw / NGI, g = gw % NGI;
   const float2 v = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)row * I + g * kGroup) + (threadIdx.x & 31));
-  xq_quantize_group<BITS>(v.x, v.y, g, NGI, p.act_limbs + (size_t)row * 3 * I, p.act_cs + (size_t)row * (I / 32));
+  tc_quantize_group<BITS>(v.x, v.y, p.act_limbs + (size_t)row * 3 * I + g * 192, p.act_cs + (size_t)row * NGI + g);
 }
 
-// ---- down: CTA (u, b) = active expert slot u, output rows [32b, 32b+32).  The
-// rows are staged once, the activation digits of up to `tb` group members at a
-// time; y[member row][h] holds the unweighted down output.
-template <int BITS, int NG>
-__global__ void __launch_bounds__(kGT) grouped_down_kernel(const GroupedParams p, int tb) {
-  using G = Geo<NG>;
-  constexpr int LPR = G::kLanesPerRow, RPP = G::kRowsPerPass, GPL = G::kGroupsPerLane;
-  constexpr int RB = NG * kGroup * BITS / 8, SB = NG * 2;
-  constexpr int NCA = NG * kGroup * BITS / 128;
-  constexpr int DIG = NG * kGroupWords * 4 + NCA * 8;
-  constexpr int WB = kDnRows * (RB + 2 * SB);
+// ---- down.  An item is 8*RPC output rows (RPC even), staged as 8 copy groups
+// of RPC rows (plus kPad bytes each); tile mt takes rows RPC*gid + 2mt (A rows
+// 0-7) and RPC*gid + 2mt + 1 (rows 8-15), so that each quad-layout load reads 8
+// distinct groups.  The digits are those of the members' activations, whose
+// rows are consecutive (two copies per unit).  K is split over the warps as in
+// gate/up.  y[member row][h] holds the unweighted down output.
+template <int BITS, int NG, int RPC>
+__global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const GroupedParams p, int ns) {
+  using R = TcRows<BITS, NG>;
+  constexpr int RB = R::RB, GPW = R::GPW, LB = R::LB, CB = R::CB, SB = NG * 2;
+  constexpr int ROWS = 8 * RPC, MT = RPC / 2;
+  constexpr int GP = RPC * RB + kPad;
+  constexpr int WB = 8 * GP + 2 * ROWS * SB;  // row groups, then s, b ([ROWS][NG] bf16 each)
+  constexpr int DB = kUnitToks * (LB + CB);
+  constexpr int TP = ROWS * 8 + 4;
+  static_assert(RPC % 2 == 0, "down tiles pair rows within a copy group");
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ __align__(8) uint64_t s_wbar;
-  __shared__ __align__(8) uint64_t s_dbar;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int U = __ldcg(p.n_active);
-  const int u = blockIdx.x;
-  if (u > U) return;
-  const Group grp = group_of(p, u, U);
-  const int H = p.H, I = p.I;
-  const int d0 = blockIdx.y * kDnRows;
-  uint8_t* dbuf = sm + WB;
-  const uint64_t pol = l2_policy_evict_first();
+  __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
+  __shared__ ItemDesc s_item[kRing];
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, q = lane & 3;
+  const int H = p.H, I = p.I, NB = H / ROWS;
+  int i0, count;
+  item_range(p, NB, i0, count);
+  uint8_t* dbase = sm + (size_t)ns * WB;
+  float* red = reinterpret_cast<float*>(dbase + 2 * DB);
   if (tid == 0) {
-    mbar_init(smem_addr(&s_wbar), 1);
-    mbar_init(smem_addr(&s_dbar), 1);
+    for (int i = 0; i < ns; ++i) {
+      mbar_init(smem_addr(&s_wfull[i]), 1);
+      mbar_init(smem_addr(&s_wempty[i]), kConsumers);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&s_dfull[i]), 1);
+      mbar_init(smem_addr(&s_dempty[i]), kConsumers);
+    }
     mbar_fence_init();
-    const uint32_t bw = smem_addr(&s_wbar), dst = smem_addr(sm);
-    mbar_expect_tx(bw, kDnRows * (RB + 2 * SB));
-    bulk_g2s(dst, grp.rec + grp.off[6] + (long long)d0 * RB, kDnRows * RB, bw, pol);
-    bulk_g2s(dst + kDnRows * RB, grp.rec + grp.off[7] + (long long)d0 * SB, kDnRows * SB, bw, pol);
-    bulk_g2s(dst + kDnRows * (RB + SB), grp.rec + grp.off[8] + (long long)d0 * SB, kDnRows * SB, bw, pol);
+    s_abort = 0;
   }
   __syncthreads();
-  bool ok = mbar_wait_bounded(smem_addr(&s_wbar), 0, p.err);
-  const int sub = lane / LPR, gl = lane % LPR;
-  const uint16_t* scl = reinterpret_cast<const uint16_t*>(sm + kDnRows * RB);
-  const uint16_t* bsl = reinterpret_cast<const uint16_t*>(sm + kDnRows * (RB + SB));
-  for (int j0 = 0, it = 0; j0 < grp.n; j0 += tb, ++it) {
-    const int nb = min(tb, grp.n - j0);
-    if (tid == 0) {
-      const uint32_t bd = smem_addr(&s_dbar);
-      fence_proxy_async();
-      mbar_expect_tx(bd, (uint32_t)nb * DIG);
-      for (int jj = 0; jj < nb; ++jj) {
-        int tok, row;
-        member(p, grp, j0 + jj, tok, row);
-        bulk_g2s(smem_addr(dbuf + jj * DIG), p.act_limbs + (size_t)row * 3 * I, NG * kGroupWords * 4, bd, pol);
-        bulk_g2s(smem_addr(dbuf + jj * DIG + NG * kGroupWords * 4), p.act_cs + (size_t)row * (I / 32), NCA * 8, bd, pol);
+
+  if (warp == kConsumers) {  // the producer
+    const uint64_t pol_w = l2_policy_evict_first(), pol_d = l2_policy_evict_last();
+    auto issue_w = [&](const ItemDesc& it, int st) {
+      const uint8_t* rec = unit_record(p, it.u.e);
+      const long long d0 = (long long)it.blk * ROWS;
+      const uint32_t bw = smem_addr(&s_wfull[st]), dst = smem_addr(sm + (size_t)st * WB);
+      if (lane == 0) mbar_expect_tx(bw, ROWS * RB + 2 * ROWS * SB);
+      __syncwarp();
+      if (lane < 8)
+        bulk_g2s(dst + lane * GP, rec + p.routed.off[6] + (d0 + RPC * lane) * RB, RPC * RB, bw, pol_w);
+      else if (lane < 10)
+        bulk_g2s(dst + 8 * GP + (lane - 8) * ROWS * SB, rec + p.routed.off[lane - 1] + d0 * SB, ROWS * SB, bw, pol_w);
+    };
+    auto issue_d = [&](const UnitDesc& u, int slot) {
+      const uint32_t bd = smem_addr(&s_dfull[slot]);
+      uint8_t* dst = dbase + (size_t)slot * DB;
+      if (lane == 0) {
+        mbar_expect_tx(bd, (uint32_t)u.n * (LB + CB));
+        bulk_g2s(smem_addr(dst), p.act_limbs + (size_t)u.row0 * LB, u.n * LB, bd, pol_d);
+        bulk_g2s(smem_addr(dst + kUnitToks * LB), p.act_cs + (size_t)u.row0 * NG, u.n * CB, bd, pol_d);
       }
-    }
-    if (!mbar_wait_bounded(smem_addr(&s_dbar), (uint32_t)(it & 1), p.err)) ok = false;
-    for (int jj = 0; ok && jj < nb; ++jj) {
-      int tok, row;
-      member(p, grp, j0 + jj, tok, row);
-      const uint32_t* al = reinterpret_cast<const uint32_t*>(dbuf + jj * DIG);
-      const float2* ac = reinterpret_cast<const float2*>(dbuf + jj * DIG + NG * kGroupWords * 4);
-      uint32_t L[GPL][48];
-      float2 cs[GPL];
-#pragma unroll
-      for (int q = 0; q < GPL; ++q) {
-        load_group_limbs(al, gl + LPR * q, NG, L[q]);
-        cs[q] = group_scalars<BITS>(ac, gl + LPR * q);
-      }
-      for (int pr = warp; pr * RPP < kDnRows; pr += kGT / 32) {
-        const int r = pr * RPP + sub;
-        float acc = 0.0f;
-#pragma unroll
-        for (int q = 0; q < GPL; ++q) {
-          const int g = gl + LPR * q;
-          uint4 q0, q1;
-          load_group_codes<BITS>(sm + r * RB, g, q0, q1);
-          const float sc = bf16_to_f32(scl[r * NG + g]), bi = bf16_to_f32(bsl[r * NG + g]);
-          const float S = group_dot<BITS>(q0, q1, L[q]);
-          acc = fmaf(sc, cs[q].x * S, fmaf(bi, cs[q].y, acc));
-        }
-        for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (gl == 0) p.y[(size_t)row * H + d0 + r] = acc;
-      }
-    }
-    __syncthreads();
+    };
+    producer_loop(p, NB, i0, count, ns, s_item, s_wfull, s_wempty, s_dfull, s_dempty, &s_abort, issue_w, issue_d);
+    return;
   }
+
+  const int g0 = warp * GPW;
+  const bool kwarp = g0 < NG;
+  for (int k = 0; k < count; ++k) {
+    const int st = k % ns;
+    bool ok = mbar_wait_bounded(smem_addr(&s_wfull[st]), (uint32_t)((k / ns) & 1), p.err);
+    const ItemDesc it = s_item[k % kRing];
+    const int slot = it.useq & 1;
+    if (ok && it.first) ok = mbar_wait_bounded(smem_addr(&s_dfull[slot]), (uint32_t)((it.useq >> 1) & 1), p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    const uint8_t* wb = sm + (size_t)st * WB;
+    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + 8 * GP);
+    const uint8_t* db = dbase + (size_t)slot * DB;
+    float acc[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+    if (ok && kwarp) {
+      const int n = it.u.n;
+      const TcCol ca = tc_col(2 * q, n), cb = tc_col(2 * q + 1, n);
+      const int bt = gid / 3, bl = gid % 3;
+      const bool bvalid = gid < 6 && bt < n;
+      const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
+      const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);
+      uint32_t sv[MT][2][2][(GPW + 1) / 2];  // [tile][row lo / hi][s, b]
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+            tc_load_scales<GPW>(scl + (a * ROWS + RPC * gid + 2 * mt + h) * NG + g0, sv[mt][h][a]);
+#pragma unroll
+      for (int gi = 0; gi < GPW; ++gi) {
+        const int g = g0 + gi;
+        uint2 b[2];
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+          b[kb] = bvalid ? *reinterpret_cast<const uint2*>(bsrc + g * 192 + kb * 96) : make_uint2(0u, 0u);
+        float sa = 0.0f, ba = 0.0f, sb_ = 0.0f, bb = 0.0f;
+        if (ca.t >= 0) {
+          const float2 v = csv[ca.t * NG + g];
+          sa = v.x;
+          ba = ca.l0 ? v.y * 0x1p-16f : 0.0f;
+        }
+        if (cb.t >= 0) {
+          const float2 v = csv[cb.t * NG + g];
+          sb_ = v.x;
+          bb = cb.l0 ? v.y * 0x1p-16f : 0.0f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          uint32_t w[2][2];
+          tc_load_a<BITS>(wb + gid * GP + 2 * mt * RB, wb + gid * GP + (2 * mt + 1) * RB, g, q, w);
+          int c[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            uint32_t a[4];
+            tc_unpack_a<BITS>(w, kb, a);
+            mma_u8s8(c, a, b[kb].x, b[kb].y);
+          }
+          const float s0 = tc_scale<GPW>(sv[mt][0][0], gi), b0 = tc_scale<GPW>(sv[mt][0][1], gi);
+          const float s1 = tc_scale<GPW>(sv[mt][1][0], gi), b1 = tc_scale<GPW>(sv[mt][1][1], gi);
+          acc[mt][0] = fmaf(s0 * sa, (float)c[0], fmaf(b0, ba, acc[mt][0]));
+          acc[mt][1] = fmaf(s0 * sb_, (float)c[1], fmaf(b0, bb, acc[mt][1]));
+          acc[mt][2] = fmaf(s1 * sa, (float)c[2], fmaf(b1, ba, acc[mt][2]));
+          acc[mt][3] = fmaf(s1 * sb_, (float)c[3], fmaf(b1, bb, acc[mt][3]));
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_one(smem_addr(&s_wempty[st]));
+      if (it.last) mbar_arrive_one(smem_addr(&s_dempty[slot]));
+    }
+    float* rw = red + ((k & 1) * kConsumers + warp) * TP;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int r = RPC * gid + 2 * mt;
+      *reinterpret_cast<float2*>(rw + r * 8 + 2 * q) = make_float2(acc[mt][0], acc[mt][1]);
+      *reinterpret_cast<float2*>(rw + (r + 1) * 8 + 2 * q) = make_float2(acc[mt][2], acc[mt][3]);
+    }
+    if (named_sync_or(!ok)) {
+      if (tid == 0) s_abort = 1;
+      return;
+    }
+    const int d0 = it.blk * ROWS;
+#pragma unroll
+    for (int pass = 0; pass < (16 * ROWS + kConsumers * 32 - 1) / (kConsumers * 32); ++pass) {
+      const int idx = pass * kConsumers * 32 + tid;
+      if (idx < 16 * ROWS) {  // output (row r, token t) from warp slice ws, then the slices in order
+        const int o = idx >> 3, ws = idx & 7, r = o >> 1, t = o & 1;
+        const float* rs = red + ((k & 1) * kConsumers + ws) * TP + r * 8 + 3 * t;
+        float v = fmaf(65536.0f, rs[0], fmaf(256.0f, rs[1], rs[2]));
+#pragma unroll
+        for (int o2 = 1; o2 < 8; o2 <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+        if (ws == 0 && t < it.u.n) p.y[(size_t)(it.u.row0 + t) * H + d0 + r] = v;
+      }
+    }
+  }
+  (void)I;
 }
 
 // ---- combine, fixed k order: out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t]
@@ -496,65 +881,100 @@ __global__ void __launch_bounds__(kGT) grouped_combine_kernel(const GroupedParam
   p.out[(size_t)t * p.H + h] = p.h[(size_t)t * p.H + h] + acc;
 }
 
-size_t gu_smem(int bits, int H) {
-  const int NG = H / kGroup, RB = H * bits / 8, SB = NG * 2;
-  return (size_t)kGuRows * (2 * RB + 4 * SB) + (size_t)kGuTok * (NG * kGroupWords * 4 + (H * bits / 128) * 8);
+constexpr size_t kSmemBudget = 220 * 1024;
+
+// Shared memory of an expert kernel: `ns` staged items of `wb` bytes, two digit
+// slots of kUnitToks members and the double-buffered partial tiles (tp floats
+// per consumer warp).
+size_t tc_smem(int ns, size_t wb, int NG, size_t tp) {
+  return (size_t)ns * wb + 2 * (size_t)kUnitToks * NG * 200 + 2 * (size_t)kConsumers * tp * 4;
 }
 
-// down: staged rows + as many members' digits as fit (at most kDnTok)
-int dn_tokens(int bits, int I, size_t* smem) {
+struct TcConfig {
+  int rpc, ns;
+  size_t smem;
+};
+
+// gate/up: the most rows per item (RPC 2, else 1) whose ring keeps at least
+// 64 KiB of rows in flight, with as many stages (<= 6) as fit.
+TcConfig gu_config(int bits, int H) {
+  const int NG = H / kGroup, RB = H * bits / 8, SB = NG * 2;
+  for (int rpc : {2, 1}) {
+    const size_t wb = 16 * (size_t)(rpc * RB + kPad) + 32 * (size_t)rpc * SB;
+    const size_t tp = 2 * 8 * (size_t)rpc * 8 + 4;
+    for (int n = 6; n >= 2; --n) {
+      const size_t sm = tc_smem(n, wb, NG, tp);
+      if (sm <= kSmemBudget && ((n - 1) * wb >= 64 * 1024 || rpc == 1)) return TcConfig{rpc, n, sm};
+    }
+  }
+  return TcConfig{0, 0, 0};
+}
+
+// down: RPC 8, 4 or 2 (64, 32 or 16 rows per item), the first with at least 3 stages (<= 8).
+TcConfig dn_config(int bits, int I) {
   const int NG = I / kGroup, RB = I * bits / 8, SB = NG * 2;
-  const size_t wb = (size_t)kDnRows * (RB + 2 * SB), dig = (size_t)NG * kGroupWords * 4 + (size_t)(I * bits / 128) * 8;
-  const size_t budget = 220 * 1024;
-  if (wb + dig > budget) return 0;
-  size_t tb = (budget - wb) / dig;
-  tb = tb > (size_t)kDnTok ? (size_t)kDnTok : tb;
-  *smem = wb + tb * dig;
-  return (int)tb;
+  for (int rpc : {8, 4, 2}) {
+    const size_t wb = 8 * (size_t)(rpc * RB + kPad) + 2 * 8 * (size_t)rpc * SB;
+    const size_t tp = 8 * (size_t)rpc * 8 + 4;
+    for (int n = 8; n >= 3; --n) {
+      const size_t sm = tc_smem(n, wb, NG, tp);
+      if (sm <= kSmemBudget) return TcConfig{rpc, n, sm};
+    }
+  }
+  return TcConfig{0, 0, 0};
+}
+
+template <int BITS, int NG>
+cudaError_t gateup_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
+  void (*k)(const GroupedParams, int) =
+      c.rpc == 2 ? grouped_gateup_kernel<BITS, NG, 2> : grouped_gateup_kernel<BITS, NG, 1>;
+  cudaError_t e = set_smem((const void*)k, c.smem);
+  if (e != cudaSuccess) return e;
+  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns);
+  return cudaGetLastError();
+}
+
+template <int BITS, int NG>
+cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
+  void (*k)(const GroupedParams, int) = c.rpc == 8   ? grouped_down_kernel<BITS, NG, 8>
+                                        : c.rpc == 4 ? grouped_down_kernel<BITS, NG, 4>
+                                                     : grouped_down_kernel<BITS, NG, 2>;
+  cudaError_t e = set_smem((const void*)k, c.smem);
+  if (e != cudaSuccess) return e;
+  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns);
+  return cudaGetLastError();
 }
 
 template <int BITS>
 cudaError_t gateup_bits_g(const GroupedParams& p, cudaStream_t s) {
-  void (*k)(const GroupedParams) = nullptr;
+  const TcConfig c = gu_config(BITS, p.H);
+  if (c.rpc == 0) return cudaErrorInvalidValue;
   switch (p.H / kGroup) {
-    case 2: k = grouped_gateup_kernel<BITS, 2>; break;
-    case 4: k = grouped_gateup_kernel<BITS, 4>; break;
-    case 8: k = grouped_gateup_kernel<BITS, 8>; break;
-    case 16: k = grouped_gateup_kernel<BITS, 16>; break;
-    case 32: k = grouped_gateup_kernel<BITS, 32>; break;
-    case 64: k = grouped_gateup_kernel<BITS, 64>; break;
-    case 128: k = grouped_gateup_kernel<BITS, 128>; break;
+    case 2: return gateup_ng<BITS, 2>(p, c, s);
+    case 4: return gateup_ng<BITS, 4>(p, c, s);
+    case 8: return gateup_ng<BITS, 8>(p, c, s);
+    case 16: return gateup_ng<BITS, 16>(p, c, s);
+    case 32: return gateup_ng<BITS, 32>(p, c, s);
+    case 64: return gateup_ng<BITS, 64>(p, c, s);
+    case 128: return gateup_ng<BITS, 128>(p, c, s);
     default: return cudaErrorInvalidValue;
   }
-  const size_t smem = gu_smem(BITS, p.H);
-  cudaError_t e = set_smem((const void*)k, smem);
-  if (e != cudaSuccess) return e;
-  const int umax = (p.E < p.T * p.K ? p.E : p.T * p.K) + 1;
-  k<<<dim3(umax, p.I / kGuRows), kGT, smem, s>>>(p);
-  return cudaGetLastError();
 }
 
 template <int BITS>
 cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
-  void (*k)(const GroupedParams, int) = nullptr;
+  const TcConfig c = dn_config(BITS, p.I);
+  if (c.rpc == 0 || p.H % (8 * c.rpc)) return cudaErrorInvalidValue;
   switch (p.I / kGroup) {
-    case 2: k = grouped_down_kernel<BITS, 2>; break;
-    case 4: k = grouped_down_kernel<BITS, 4>; break;
-    case 8: k = grouped_down_kernel<BITS, 8>; break;
-    case 16: k = grouped_down_kernel<BITS, 16>; break;
-    case 32: k = grouped_down_kernel<BITS, 32>; break;
-    case 64: k = grouped_down_kernel<BITS, 64>; break;
-    case 128: k = grouped_down_kernel<BITS, 128>; break;
+    case 2: return down_ng<BITS, 2>(p, c, s);
+    case 4: return down_ng<BITS, 4>(p, c, s);
+    case 8: return down_ng<BITS, 8>(p, c, s);
+    case 16: return down_ng<BITS, 16>(p, c, s);
+    case 32: return down_ng<BITS, 32>(p, c, s);
+    case 64: return down_ng<BITS, 64>(p, c, s);
+    case 128: return down_ng<BITS, 128>(p, c, s);
     default: return cudaErrorInvalidValue;
   }
-  size_t smem = 0;
-  const int tb = dn_tokens(BITS, p.I, &smem);
-  if (tb < 1) return cudaErrorInvalidValue;
-  cudaError_t e = set_smem((const void*)k, smem);
-  if (e != cudaSuccess) return e;
-  const int umax = (p.E < p.T * p.K ? p.E : p.T * p.K) + 1;
-  k<<<dim3(umax, p.H / kDnRows), kGT, smem, s>>>(p, tb);
-  return cudaGetLastError();
 }
 
 }  // namespace
@@ -562,9 +982,8 @@ cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
 bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T) {
   if (T * K > kMaxTK || ((size_t)T * K + 2 * (size_t)E) * 4 > 200 * 1024) return false;
   if ((size_t)kRtRows * H * 2 > 200 * 1024) return false;
-  if (H % kDnRows || I % kGuRows) return false;
-  size_t smem = 0;
-  return gu_smem(bits, H) <= 220 * 1024 && dn_tokens(bits, I, &smem) >= 1;
+  const TcConfig gu = gu_config(bits, H), dn = dn_config(bits, I);
+  return gu.rpc > 0 && I % (8 * gu.rpc) == 0 && dn.rpc > 0 && H % (8 * dn.rpc) == 0;
 }
 
 cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s) {
