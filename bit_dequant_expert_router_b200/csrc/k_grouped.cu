@@ -19,6 +19,11 @@
 //   combine : out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t]
 // Dequant dot products use the per-group fold sum_c (q s + b) x = s*sum q x + b*sum x
 // with exact dp4a sums ("What is Flash-MoE", sections 2-3, for the block itself).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "fmoe_internal.h"
 
 namespace fmoe {
@@ -336,7 +341,6 @@ __global__ void __launch_bounds__(kGT) router_gemm_kernel(const GroupedParams p,
 constexpr int kConsumers = 8;                      // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;    // + the producer warp
 constexpr int kRing = 16;                          // item descriptors in flight (> the largest ns)
-constexpr int kPad = 32;                           // bytes after each staged copy group of rows
 
 struct ItemDesc {
   UnitDesc u;
@@ -430,21 +434,39 @@ __device__ __forceinline__ void producer_loop(const GroupedParams& p, int NB, in
 template <int BITS, int NG>
 struct TcRows {
   static constexpr int RB = NG * kGroup * BITS / 8;
-  static constexpr int GPW = NG >= 8 ? NG / 8 : 1;  // groups per warp (K is split over the 8 warps)
   static constexpr int LB = NG * 192;               // digit bytes of one token / activation row
   static constexpr int CB = NG * 8;                 // its per-group scalars
 };
 
-// A registers of rows (gid, gid + 8) for k-block kb of group g from staged rows.
-template <int BITS>
-__device__ __forceinline__ void tc_load_a(const uint8_t* r_lo, const uint8_t* r_hi, int g, int q, uint32_t (&w)[2][2]) {
+// Staged code rows: one tensor copy per matrix brings an item's ROWS rows as
+// lines of LW = min(128, RB) bytes ordered (column block, row), with the copy's
+// swizzle: the 16-byte chunk index of byte X is XORed with bits 7.. of X
+// (128-byte swizzle: 3 bits, 64-byte: 2, 32-byte: 1).  Rows gid = 0..7 of a
+// tile are consecutive, so the eight rows a quad-layout load reads land in
+// distinct chunks.
+template <int BITS, int NG, int ROWS>
+struct TcSw {
+  static constexpr int RB = NG * kGroup * BITS / 8;
+  static constexpr int LW = RB >= 128 ? 128 : RB;
+  static constexpr int M = LW == 128 ? 7 : LW == 64 ? 3 : 1;
+  __device__ static __forceinline__ const uint8_t* at(const uint8_t* buf, int row, int c) {
+    const int X = ((c / LW) * ROWS + row) * LW + c % LW;
+    return buf + (X ^ (((X >> 7) & M) << 4));
+  }
+};
+
+// A registers of staged rows row_lo (A rows 0-7) and row_hi (rows 8-15) for group g.
+template <int BITS, int NG, int ROWS>
+__device__ __forceinline__ void tc_load_a(const uint8_t* buf_lo, int row_lo, const uint8_t* buf_hi, int row_hi, int g,
+                                          int q, uint32_t (&w)[2][2]) {
+  using S = TcSw<BITS, NG, ROWS>;
   if (BITS == 4) {
-    const uint2 x = *reinterpret_cast<const uint2*>(r_lo + g * 32 + 8 * q);
-    const uint2 y = *reinterpret_cast<const uint2*>(r_hi + g * 32 + 8 * q);
+    const uint2 x = *reinterpret_cast<const uint2*>(S::at(buf_lo, row_lo, g * 32 + 8 * q));
+    const uint2 y = *reinterpret_cast<const uint2*>(S::at(buf_hi, row_hi, g * 32 + 8 * q));
     w[0][0] = x.x; w[0][1] = x.y; w[1][0] = y.x; w[1][1] = y.y;
   } else {
-    const uint32_t x = *reinterpret_cast<const uint32_t*>(r_lo + g * 16 + 4 * q);
-    const uint32_t y = *reinterpret_cast<const uint32_t*>(r_hi + g * 16 + 4 * q);
+    const uint32_t x = *reinterpret_cast<const uint32_t*>(S::at(buf_lo, row_lo, g * 16 + 4 * q));
+    const uint32_t y = *reinterpret_cast<const uint32_t*>(S::at(buf_hi, row_hi, g * 16 + 4 * q));
     w[0][0] = w[0][1] = x; w[1][0] = w[1][1] = y;
   }
 }
@@ -493,38 +515,162 @@ __device__ __forceinline__ float tc_scale(const uint32_t (&v)[(GPW + 1) / 2], in
   return __uint_as_float((gi & 1) ? (v[gi >> 1] & 0xFFFF0000u) : (v[gi >> 1] << 16));
 }
 
-// The quad lane's two columns: column c = 3 t + L (token t of the tile, limb
-// L), columns 6 and 7 unused.  Per group: the scale of the int32 sum and the
-// bias factor (sum of x / 2^16 on limb 0, whose weight 2^16 is applied last).
-struct TcCol {
-  int t;     // token of the tile, -1 = unused column
-  bool l0;   // limb 0
+// The quad lane's two C columns are 2q and 2q + 1; column c = 3t + L is limb L
+// of the tile's token t, columns 6 and 7 unused.  Per group the lane needs each
+// column's digit scale (0 for a column without a token), and for the limb-0
+// column it holds (lane q = 0: column 0, token 0; q = 1: column 3, token 1) the
+// token's group sum of x, for the bias term b * sum x (added on limb 0, whose
+// weight 2^16 is applied last).  B registers of a column without a token read
+// whatever the digit slot holds: any byte is a digit, and the column's scale is 0.
+struct TcLane {
+  int ta, tb;    // tokens of columns 2q and 2q + 1, clamped to a slot that exists
+  bool va, vb;   // whether those columns have a token
+  bool bias_a;   // column 2q is limb 0 of a token (q == 0)
+  bool bias_b;   // column 2q + 1 is limb 0 of a token (q == 1 with two tokens)
 };
 
-__device__ __forceinline__ TcCol tc_col(int c, int n) {
-  TcCol k;
-  k.t = (c < 6 && c / 3 < n) ? c / 3 : -1;
-  k.l0 = c % 3 == 0;
-  return k;
+__device__ __forceinline__ TcLane tc_lane(int q, int n) {
+  TcLane l;
+  const int ca = 2 * q, cb = 2 * q + 1;
+  l.va = ca < 6 && ca / 3 < n;
+  l.vb = cb < 6 && cb / 3 < n;
+  l.ta = l.va ? ca / 3 : 0;
+  l.tb = l.vb ? cb / 3 : 0;
+  l.bias_a = q == 0;
+  l.bias_b = q == 1 && l.vb;
+  return l;
 }
 
-// ---- gate/up + SwiGLU.  An item is 8*RPC (gate, up) row pairs, staged as 8
-// copy groups of RPC consecutive rows per matrix (plus kPad bytes each), so
-// that the 8 rows one quad-layout load reads sit in 8 distinct groups.  Tile
-// mt pairs gate row RPC*gid + mt (A rows 0-7) with the same up row (rows 8-15).
-// The digits are those of x for each member token.  Warp w sums groups
-// [w*GPW, w*GPW + GPW); the eight partial tiles add in warp order.
-// act[row][r] = silu(g) * u.
-template <int BITS, int NG, int RPC>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const GroupedParams p, int ns) {
+// The int32 sums are read as floats through a biased accumulator: the mma
+// starts from the bits of 1.5 * 2^23, so that (for |sum| < 2^22, here below
+// 15 * 128 * 64) the result's bits are those of the float 1.5 * 2^23 + sum.
+// With a power-of-two digit scale s, fma(f, s, -1.5 * 2^23 * s) is then
+// exactly sum * s.
+constexpr int kMagicBits = 0x4B400000;
+constexpr float kMagic = 12582912.0f;
+
+struct TcColScale {
+  float sa, sb;  // digit scales of the two columns
+  float na, nb;  // -kMagic * scale
+  float bx;      // group sum of x / 2^16 for this lane's limb-0 column, else 0
+};
+
+__device__ __forceinline__ TcColScale tc_colscale(const float2* csv, int NG, int g, const TcLane& l) {
+  const float2 va = csv[l.ta * NG + g], vb = csv[l.tb * NG + g];
+  TcColScale c;
+  c.sa = l.va ? va.x : 0.0f;
+  c.sb = l.vb ? vb.x : 0.0f;
+  c.na = -kMagic * c.sa;
+  c.nb = -kMagic * c.sb;
+  c.bx = (l.bias_a ? va.y : l.bias_b ? vb.y : 0.0f) * 0x1p-16f;
+  return c;
+}
+
+// One group of one 16-row tile from its A words, with row scales s_lo / s_hi
+// and biases b_lo / b_hi.
+template <int BITS>
+__device__ __forceinline__ void tc_tile_group(const uint32_t (&w)[2][2], const uint2 (&b)[2], const TcColScale& cs,
+                                              float s_lo, float s_hi, float b_lo, float b_hi, float (&acc)[4],
+                                              float (&accb)[2]) {
+  int c[4] = {kMagicBits, kMagicBits, kMagicBits, kMagicBits};
+#pragma unroll
+  for (int kb = 0; kb < 2; ++kb) {
+    uint32_t a[4];
+    tc_unpack_a<BITS>(w, kb, a);
+    mma_u8s8(c, a, b[kb].x, b[kb].y);
+  }
+  acc[0] = fmaf(s_lo, fmaf(__int_as_float(c[0]), cs.sa, cs.na), acc[0]);
+  acc[1] = fmaf(s_lo, fmaf(__int_as_float(c[1]), cs.sb, cs.nb), acc[1]);
+  acc[2] = fmaf(s_hi, fmaf(__int_as_float(c[2]), cs.sa, cs.na), acc[2]);
+  acc[3] = fmaf(s_hi, fmaf(__int_as_float(c[3]), cs.sb, cs.nb), acc[3]);
+  accb[0] = fmaf(b_lo, cs.bx, accb[0]);
+  accb[1] = fmaf(b_hi, cs.bx, accb[1]);
+}
+
+// Sums TPW tiles over groups [g0, g0 + GPW) into acc (each tile's C layout,
+// bias folded into the limb-0 columns).  Tile i reads rows rlo[i] of buf_lo and
+// rhi[i] of buf_hi (staged, ROWS rows each); sc[i] = its scale rows
+// {s_lo, b_lo, s_hi, b_hi} at group 0.  B and the column scales are shared by
+// the tiles.
+template <int BITS, int NG, int ROWS, int GPW, int TPW>
+__device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf_hi, const int (&rlo)[TPW],
+                                       const int (&rhi)[TPW], const uint16_t* const (&sc)[TPW][4], const uint8_t* db, int n,
+                                       int g0, float (&acc)[TPW][4]) {
+  constexpr int LB = NG * 192;
+  constexpr int GPC = GPW < 8 ? GPW : 8;  // groups whose scales are held at once
+  const int lane = threadIdx.x & 31, gid = lane >> 2, q = lane & 3;
+  const TcLane ln = tc_lane(q, n);
+  const int bt = gid < 6 ? gid / 3 : 0, bl = gid % 3;  // this lane's B column: token slot, limb
+  const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
+  const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);
+  float accb[TPW][2];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) accb[i][0] = accb[i][1] = 0.0f;
+#pragma unroll
+  for (int gc = 0; gc < GPW; gc += GPC) {
+    uint32_t sv[TPW][4][(GPC + 1) / 2];
+#pragma unroll
+    for (int i = 0; i < TPW; ++i)
+#pragma unroll
+      for (int a = 0; a < 4; ++a) tc_load_scales<GPC>(sc[i][a] + g0 + gc, sv[i][a]);
+#pragma unroll
+    for (int gi = 0; gi < GPC; ++gi) {
+      const int g = g0 + gc + gi;
+      uint2 b[2];
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) b[kb] = *reinterpret_cast<const uint2*>(bsrc + g * 192 + kb * 96);
+      const TcColScale cs = tc_colscale(csv, NG, g, ln);
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+        uint32_t w[2][2];
+        tc_load_a<BITS, NG, ROWS>(buf_lo, rlo[i], buf_hi, rhi[i], g, q, w);
+        tc_tile_group<BITS>(w, b, cs, tc_scale<GPC>(sv[i][0], gi), tc_scale<GPC>(sv[i][2], gi),
+                            tc_scale<GPC>(sv[i][1], gi), tc_scale<GPC>(sv[i][3], gi), acc[i], accb[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    if (q == 0) {
+      acc[i][0] += accb[i][0];
+      acc[i][2] += accb[i][1];
+    } else if (q == 1) {
+      acc[i][1] += accb[i][0];
+      acc[i][3] += accb[i][1];
+    }
+  }
+}
+
+// cp.async.bulk.tensor of a 4-D box at (0, row, 0, expert) into shared memory.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, int row, int expert, uint32_t bar,
+                                            uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(tm), "r"(0), "r"(row), "r"(0), "r"(expert), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+// ---- gate/up + SwiGLU.  An item is ROWS = 8*TL (gate, up) row pairs: one
+// tensor copy per matrix stages the rows (swizzled, see TcSw), four bulk copies
+// the scale arrays.  Tile t pairs gate row 8t + gid (A rows 0-7) with the same
+// up row (rows 8-15).  The digits are those of x for each member token.  Warp
+// w sums tiles [TPW*(w / KS), +TPW) over K slice w % KS; the KS partial tiles
+// add in slice order.  act[row][r] = silu(g) * u.
+template <int BITS, int NG, int TL>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gateup_kernel(const GroupedParams p, int ns, const __grid_constant__ CUtensorMap tm_rg,
+                          const __grid_constant__ CUtensorMap tm_ru, const __grid_constant__ CUtensorMap tm_sg,
+                          const __grid_constant__ CUtensorMap tm_su) {
   using R = TcRows<BITS, NG>;
-  constexpr int RB = R::RB, GPW = R::GPW, LB = R::LB, CB = R::CB, SB = NG * 2;
-  constexpr int ROWS = 8 * RPC;                     // row pairs per item
-  constexpr int GP = RPC * RB + kPad;               // one staged copy group
-  constexpr int WB = 16 * GP + 4 * ROWS * SB;       // gate groups, up groups, gate s, gate b, up s, up b
+  constexpr int RB = R::RB, LB = R::LB, CB = R::CB, SB = NG * 2;
+  constexpr int ROWS = 8 * TL, TPW = TL < 2 ? TL : 2, KS = 8 * TPW / TL;
+  constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;  // groups per K slice
+  constexpr int CODE = ROWS * RB;                   // one matrix's staged rows
+  constexpr int WB = (2 * CODE + 4 * ROWS * SB + 1023) / 1024 * 1024;
   constexpr int DB = kUnitToks * (LB + CB);
-  constexpr int TP = 2 * ROWS * 8 + 4;              // floats per warp's partial tiles (gate rows, then up rows)
-  extern __shared__ __align__(128) uint8_t sm[];
+  constexpr int TP = 2 * ROWS * 8 + 4;              // floats per slice's partial tiles (gate rows, then up rows)
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
   __shared__ ItemDesc s_item[kRing];
   __shared__ int s_abort;
@@ -532,8 +678,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const Group
   const int I = p.I, NB = I / ROWS;
   int i0, count;
   item_range(p, NB, i0, count);
+  uint8_t* sm = sm_raw + ((1024u - (smem_addr(sm_raw) & 1023u)) & 1023u);  // swizzled copies want 1 KiB alignment
   uint8_t* dbase = sm + (size_t)ns * WB;
-  float* red = reinterpret_cast<float*>(dbase + 2 * DB);  // [2][kConsumers][TP]
+  float* red = reinterpret_cast<float*>(dbase + 2 * DB);  // [2][KS][TP]
   if (tid == 0) {
     for (int i = 0; i < ns; ++i) {
       mbar_init(smem_addr(&s_wfull[i]), 1);
@@ -551,19 +698,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const Group
   if (warp == kConsumers) {  // the producer
     const uint64_t pol_w = l2_policy_evict_first(), pol_d = l2_policy_evict_last();
     auto issue_w = [&](const ItemDesc& it, int st) {
-      const uint8_t* rec = unit_record(p, it.u.e);
-      const long long r0 = (long long)it.blk * ROWS;
+      const int r0 = it.blk * ROWS;
       const uint32_t bw = smem_addr(&s_wfull[st]), dst = smem_addr(sm + (size_t)st * WB);
-      if (lane == 0) mbar_expect_tx(bw, 2 * ROWS * RB + 4 * ROWS * SB);
+      if (lane == 0) {
+        mbar_expect_tx(bw, 2 * CODE + 4 * ROWS * SB);
+        const bool sh = it.u.e < 0;
+        tma_load_4d(dst, sh ? &tm_sg : &tm_rg, r0, sh ? 0 : it.u.e, bw, pol_w);
+        tma_load_4d(dst + CODE, sh ? &tm_su : &tm_ru, r0, sh ? 0 : it.u.e, bw, pol_w);
+      }
       __syncwarp();
-      if (lane < 16) {  // copy group lane % 8 of the gate (lanes 0-7) or up (8-15) rows
-        const int j = lane & 7;
-        const long long off = lane < 8 ? p.routed.off[0] : p.routed.off[3];
-        bulk_g2s(dst + (lane >> 3) * 8 * GP + j * GP, rec + off + (r0 + RPC * j) * RB, RPC * RB, bw, pol_w);
-      } else if (lane < 20) {  // gate s, gate b, up s, up b
-        const int a = lane - 16;
+      if (lane >= 1 && lane <= 4) {  // gate s, gate b, up s, up b
+        const int a = lane - 1;
         const long long off = p.routed.off[a == 0 ? 1 : a == 1 ? 2 : a == 2 ? 4 : 5];
-        bulk_g2s(dst + 16 * GP + a * ROWS * SB, rec + off + r0 * SB, ROWS * SB, bw, pol_w);
+        bulk_g2s(dst + 2 * CODE + a * ROWS * SB, unit_record(p, it.u.e) + off + (long long)r0 * SB, ROWS * SB, bw,
+                 pol_w);
       }
     };
     auto issue_d = [&](const UnitDesc& u, int slot) {
@@ -581,8 +729,32 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const Group
     return;
   }
 
-  const int g0 = warp * GPW;
+  const int tg = warp / KS, kp = warp % KS, g0 = kp * GPW;
   const bool kwarp = g0 < NG;  // this warp has groups to sum
+  int rows[TPW];               // this lane's row pair in each of its tiles
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) rows[i] = 8 * (tg * TPW + i) + gid;
+  // output (row pair r, token t) of item k from slice ks, then the KS slices in order
+  auto reduce = [&](int k, int row0, int n, int r0) {
+    if (tid < 2 * ROWS * KS) {
+      const int o = tid / KS, ks = tid % KS, r = o >> 1, t = o & 1;
+      const float* rs = red + ((k & 1) * KS + ks) * TP + 3 * t;
+      float gv = 0.0f, uv = 0.0f;
+#pragma unroll
+      for (int L = 0; L < 3; ++L) {
+        const float f = L == 0 ? 65536.0f : L == 1 ? 256.0f : 1.0f;
+        gv = fmaf(f, rs[r * 8 + L], gv);
+        uv = fmaf(f, rs[(ROWS + r) * 8 + L], uv);
+      }
+#pragma unroll
+      for (int o2 = 1; o2 < KS; o2 <<= 1) {
+        gv += __shfl_xor_sync(0xffffffffu, gv, o2);
+        uv += __shfl_xor_sync(0xffffffffu, uv, o2);
+      }
+      if (ks == 0 && t < n) p.act[(size_t)(row0 + t) * I + r0 + r] = gv / (1.0f + expf(-gv)) * uv;
+    }
+  };
+  int p_row0 = 0, p_n = 0, p_r0 = 0;  // the previous item, reduced one step late
   for (int k = 0; k < count; ++k) {
     const int st = k % ns;
     bool ok = mbar_wait_bounded(smem_addr(&s_wfull[st]), (uint32_t)((k / ns) & 1), p.err);
@@ -591,102 +763,42 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const Group
     if (ok && it.first) ok = mbar_wait_bounded(smem_addr(&s_dfull[slot]), (uint32_t)((it.useq >> 1) & 1), p.err);
     ok = __all_sync(0xffffffffu, ok);
     const uint8_t* wb = sm + (size_t)st * WB;
-    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + 16 * GP);
-    const uint8_t* db = dbase + (size_t)slot * DB;
-    float acc[RPC][4];
+    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + 2 * CODE);
+    float acc[TPW][4];
 #pragma unroll
-    for (int mt = 0; mt < RPC; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+    for (int i = 0; i < TPW; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
     if (ok && kwarp) {
-      const int n = it.u.n;
-      const TcCol ca = tc_col(2 * q, n), cb = tc_col(2 * q + 1, n);
-      const int bt = gid / 3, bl = gid % 3;  // this lane's B column: token, limb
-      const bool bvalid = gid < 6 && bt < n;
-      const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
-      const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);
-      uint32_t sv[RPC][4][(GPW + 1) / 2];  // gate s, gate b, up s, up b of row pair RPC*gid + mt, this warp's groups
+      const uint16_t* sc[TPW][4];
 #pragma unroll
-      for (int mt = 0; mt < RPC; ++mt)
+      for (int i = 0; i < TPW; ++i)
 #pragma unroll
-        for (int a = 0; a < 4; ++a) tc_load_scales<GPW>(scl + (a * ROWS + RPC * gid + mt) * NG + g0, sv[mt][a]);
-#pragma unroll
-      for (int gi = 0; gi < GPW; ++gi) {
-        const int g = g0 + gi;
-        uint2 b[2];
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-          b[kb] = bvalid ? *reinterpret_cast<const uint2*>(bsrc + g * 192 + kb * 96) : make_uint2(0u, 0u);
-        float sa = 0.0f, ba = 0.0f, sb_ = 0.0f, bb = 0.0f;
-        if (ca.t >= 0) {
-          const float2 v = csv[ca.t * NG + g];
-          sa = v.x;
-          ba = ca.l0 ? v.y * 0x1p-16f : 0.0f;
-        }
-        if (cb.t >= 0) {
-          const float2 v = csv[cb.t * NG + g];
-          sb_ = v.x;
-          bb = cb.l0 ? v.y * 0x1p-16f : 0.0f;
-        }
-#pragma unroll
-        for (int mt = 0; mt < RPC; ++mt) {
-          uint32_t w[2][2];
-          tc_load_a<BITS>(wb + gid * GP + mt * RB, wb + 8 * GP + gid * GP + mt * RB, g, q, w);
-          int c[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            uint32_t a[4];
-            tc_unpack_a<BITS>(w, kb, a);
-            mma_u8s8(c, a, b[kb].x, b[kb].y);
-          }
-          const float gs = tc_scale<GPW>(sv[mt][0], gi), gb = tc_scale<GPW>(sv[mt][1], gi);
-          const float us = tc_scale<GPW>(sv[mt][2], gi), ub = tc_scale<GPW>(sv[mt][3], gi);
-          acc[mt][0] = fmaf(gs * sa, (float)c[0], fmaf(gb, ba, acc[mt][0]));
-          acc[mt][1] = fmaf(gs * sb_, (float)c[1], fmaf(gb, bb, acc[mt][1]));
-          acc[mt][2] = fmaf(us * sa, (float)c[2], fmaf(ub, ba, acc[mt][2]));
-          acc[mt][3] = fmaf(us * sb_, (float)c[3], fmaf(ub, bb, acc[mt][3]));
-        }
-      }
+        for (int a = 0; a < 4; ++a) sc[i][a] = scl + (size_t)(a * ROWS + rows[i]) * NG;
+      tc_sum<BITS, NG, ROWS, GPW, TPW>(wb, wb + CODE, rows, rows, sc, dbase + (size_t)slot * DB, it.u.n, g0, acc);
     }
     __syncwarp();
     if (lane == 0) {  // this warp is done with the item's rows (and, on its last item, the unit's digits)
       mbar_arrive_one(smem_addr(&s_wempty[st]));
       if (it.last) mbar_arrive_one(smem_addr(&s_dempty[slot]));
     }
-    float* rw = red + ((k & 1) * kConsumers + warp) * TP;
+    if (k > 0) reduce(k - 1, p_row0, p_n, p_r0);  // its tiles were complete at the last barrier
+    float* rw = red + ((k & 1) * KS + kp) * TP;
 #pragma unroll
-    for (int mt = 0; mt < RPC; ++mt) {
-      const int r = RPC * gid + mt;
-      *reinterpret_cast<float2*>(rw + r * 8 + 2 * q) = make_float2(acc[mt][0], acc[mt][1]);
-      *reinterpret_cast<float2*>(rw + (ROWS + r) * 8 + 2 * q) = make_float2(acc[mt][2], acc[mt][3]);
+    for (int i = 0; i < TPW; ++i) {
+      *reinterpret_cast<float2*>(rw + rows[i] * 8 + 2 * q) = make_float2(acc[i][0], acc[i][1]);
+      *reinterpret_cast<float2*>(rw + (ROWS + rows[i]) * 8 + 2 * q) = make_float2(acc[i][2], acc[i][3]);
     }
-    // partial tiles in place (double-buffered: item k + 2 writes these only after
-    // the next barrier); a wait that ran out anywhere ends every consumer here
+    // the tiles of item k are in place; item k + 2 writes them again only after the
+    // next barrier, by which every thread has reduced them.  A wait that ran out
+    // anywhere ends every consumer here.
     if (named_sync_or(!ok)) {
       if (tid == 0) s_abort = 1;
       return;
     }
-    const int r0 = it.blk * ROWS;
-#pragma unroll
-    for (int pass = 0; pass < (16 * ROWS + kConsumers * 32 - 1) / (kConsumers * 32); ++pass) {
-      const int idx = pass * kConsumers * 32 + tid;
-      if (idx < 16 * ROWS) {  // output (row pair r, token t) from warp slice ws, then the slices in order
-        const int o = idx >> 3, ws = idx & 7, r = o >> 1, t = o & 1;
-        const float* rs = red + ((k & 1) * kConsumers + ws) * TP + 3 * t;
-        float gv = 0.0f, uv = 0.0f;
-#pragma unroll
-        for (int L = 0; L < 3; ++L) {
-          const float f = L == 0 ? 65536.0f : L == 1 ? 256.0f : 1.0f;
-          gv = fmaf(f, rs[r * 8 + L], gv);
-          uv = fmaf(f, rs[(ROWS + r) * 8 + L], uv);
-        }
-#pragma unroll
-        for (int o2 = 1; o2 < 8; o2 <<= 1) {
-          gv += __shfl_xor_sync(0xffffffffu, gv, o2);
-          uv += __shfl_xor_sync(0xffffffffu, uv, o2);
-        }
-        if (ws == 0 && t < it.u.n) p.act[(size_t)(it.u.row0 + t) * I + r0 + r] = gv / (1.0f + expf(-gv)) * uv;
-      }
-    }
+    p_row0 = it.u.row0;
+    p_n = it.u.n;
+    p_r0 = it.blk * ROWS;
   }
+  if (count > 0) reduce(count - 1, p_row0, p_n, p_r0);
 }
 
 // ---- activation digits of every sorted pair and every shared-expert token: one warp per group of 64
@@ -700,30 +812,33 @@ __global__ void __launch_bounds__(kGT) grouped_actq_kernel(const GroupedParams p
   tc_quantize_group<BITS>(v.x, v.y, p.act_limbs + (size_t)row * 3 * I + g * 192, p.act_cs + (size_t)row * NGI + g);
 }
 
-// ---- down.  An item is 8*RPC output rows (RPC even), staged as 8 copy groups
-// of RPC rows (plus kPad bytes each); tile mt takes rows RPC*gid + 2mt (A rows
-// 0-7) and RPC*gid + 2mt + 1 (rows 8-15), so that each quad-layout load reads 8
-// distinct groups.  The digits are those of the members' activations, whose
-// rows are consecutive (two copies per unit).  K is split over the warps as in
-// gate/up.  y[member row][h] holds the unweighted down output.
-template <int BITS, int NG, int RPC>
-__global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const GroupedParams p, int ns) {
+// ---- down.  An item is ROWS = 16*TL output rows: one tensor copy stages the
+// rows (swizzled, see TcSw), two bulk copies the scale arrays.  Tile t takes
+// rows 16t + gid (A rows 0-7) and 16t + 8 + gid (rows 8-15).  The digits are
+// those of the members' activations, whose rows are consecutive (two copies
+// per unit).  Warps split tiles and K as in gate/up.  y[member row][h] holds the
+// unweighted down output.
+template <int BITS, int NG, int TL>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_down_kernel(const GroupedParams p, int ns, const __grid_constant__ CUtensorMap tm_rd,
+                        const __grid_constant__ CUtensorMap tm_sd) {
   using R = TcRows<BITS, NG>;
-  constexpr int RB = R::RB, GPW = R::GPW, LB = R::LB, CB = R::CB, SB = NG * 2;
-  constexpr int ROWS = 8 * RPC, MT = RPC / 2;
-  constexpr int GP = RPC * RB + kPad;
-  constexpr int WB = 8 * GP + 2 * ROWS * SB;  // row groups, then s, b ([ROWS][NG] bf16 each)
+  constexpr int RB = R::RB, LB = R::LB, CB = R::CB, SB = NG * 2;
+  constexpr int ROWS = 16 * TL, TPW = TL < 2 ? TL : 2, KS = 8 * TPW / TL;
+  constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;
+  constexpr int CODE = ROWS * RB;
+  constexpr int WB = (CODE + 2 * ROWS * SB + 1023) / 1024 * 1024;
   constexpr int DB = kUnitToks * (LB + CB);
   constexpr int TP = ROWS * 8 + 4;
-  static_assert(RPC % 2 == 0, "down tiles pair rows within a copy group");
-  extern __shared__ __align__(128) uint8_t sm[];
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
   __shared__ ItemDesc s_item[kRing];
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, q = lane & 3;
-  const int H = p.H, I = p.I, NB = H / ROWS;
+  const int H = p.H, NB = H / ROWS;
   int i0, count;
   item_range(p, NB, i0, count);
+  uint8_t* sm = sm_raw + ((1024u - (smem_addr(sm_raw) & 1023u)) & 1023u);
   uint8_t* dbase = sm + (size_t)ns * WB;
   float* red = reinterpret_cast<float*>(dbase + 2 * DB);
   if (tid == 0) {
@@ -743,15 +858,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const Grouped
   if (warp == kConsumers) {  // the producer
     const uint64_t pol_w = l2_policy_evict_first(), pol_d = l2_policy_evict_last();
     auto issue_w = [&](const ItemDesc& it, int st) {
-      const uint8_t* rec = unit_record(p, it.u.e);
-      const long long d0 = (long long)it.blk * ROWS;
+      const int d0 = it.blk * ROWS;
       const uint32_t bw = smem_addr(&s_wfull[st]), dst = smem_addr(sm + (size_t)st * WB);
-      if (lane == 0) mbar_expect_tx(bw, ROWS * RB + 2 * ROWS * SB);
+      if (lane == 0) {
+        mbar_expect_tx(bw, CODE + 2 * ROWS * SB);
+        tma_load_4d(dst, it.u.e < 0 ? &tm_sd : &tm_rd, d0, it.u.e < 0 ? 0 : it.u.e, bw, pol_w);
+      }
       __syncwarp();
-      if (lane < 8)
-        bulk_g2s(dst + lane * GP, rec + p.routed.off[6] + (d0 + RPC * lane) * RB, RPC * RB, bw, pol_w);
-      else if (lane < 10)
-        bulk_g2s(dst + 8 * GP + (lane - 8) * ROWS * SB, rec + p.routed.off[lane - 1] + d0 * SB, ROWS * SB, bw, pol_w);
+      if (lane >= 1 && lane <= 2)  // s, b
+        bulk_g2s(dst + CODE + (lane - 1) * ROWS * SB, unit_record(p, it.u.e) + p.routed.off[6 + lane] + (long long)d0 * SB,
+                 ROWS * SB, bw, pol_w);
     };
     auto issue_d = [&](const UnitDesc& u, int slot) {
       const uint32_t bd = smem_addr(&s_dfull[slot]);
@@ -766,8 +882,30 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const Grouped
     return;
   }
 
-  const int g0 = warp * GPW;
+  const int tg = warp / KS, kp = warp % KS, g0 = kp * GPW;
   const bool kwarp = g0 < NG;
+  int rlo[TPW], rhi[TPW];  // this lane's rows in each of its tiles
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    rlo[i] = 16 * (tg * TPW + i) + gid;
+    rhi[i] = rlo[i] + 8;
+  }
+  // output (row r, token t) of item k from slice ks, then the KS slices in order
+  auto reduce = [&](int k, int row0, int n, int d0) {
+#pragma unroll
+    for (int pass = 0; pass < (2 * ROWS * KS + kConsumers * 32 - 1) / (kConsumers * 32); ++pass) {
+      const int idx = pass * kConsumers * 32 + tid;
+      if (idx < 2 * ROWS * KS) {
+        const int o = idx / KS, ks = idx % KS, r = o >> 1, t = o & 1;
+        const float* rs = red + ((k & 1) * KS + ks) * TP + r * 8 + 3 * t;
+        float v = fmaf(65536.0f, rs[0], fmaf(256.0f, rs[1], rs[2]));
+#pragma unroll
+        for (int o2 = 1; o2 < KS; o2 <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+        if (ks == 0 && t < n) p.y[(size_t)(row0 + t) * H + d0 + r] = v;
+      }
+    }
+  };
+  int p_row0 = 0, p_n = 0, p_d0 = 0;
   for (int k = 0; k < count; ++k) {
     const int st = k % ns;
     bool ok = mbar_wait_bounded(smem_addr(&s_wfull[st]), (uint32_t)((k / ns) & 1), p.err);
@@ -776,95 +914,42 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const Grouped
     if (ok && it.first) ok = mbar_wait_bounded(smem_addr(&s_dfull[slot]), (uint32_t)((it.useq >> 1) & 1), p.err);
     ok = __all_sync(0xffffffffu, ok);
     const uint8_t* wb = sm + (size_t)st * WB;
-    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + 8 * GP);
-    const uint8_t* db = dbase + (size_t)slot * DB;
-    float acc[MT][4];
+    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + CODE);
+    float acc[TPW][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+    for (int i = 0; i < TPW; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
     if (ok && kwarp) {
-      const int n = it.u.n;
-      const TcCol ca = tc_col(2 * q, n), cb = tc_col(2 * q + 1, n);
-      const int bt = gid / 3, bl = gid % 3;
-      const bool bvalid = gid < 6 && bt < n;
-      const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
-      const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);
-      uint32_t sv[MT][2][2][(GPW + 1) / 2];  // [tile][row lo / hi][s, b]
+      const uint16_t* sc[TPW][4];
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int a = 0; a < 2; ++a)
-            tc_load_scales<GPW>(scl + (a * ROWS + RPC * gid + 2 * mt + h) * NG + g0, sv[mt][h][a]);
-#pragma unroll
-      for (int gi = 0; gi < GPW; ++gi) {
-        const int g = g0 + gi;
-        uint2 b[2];
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-          b[kb] = bvalid ? *reinterpret_cast<const uint2*>(bsrc + g * 192 + kb * 96) : make_uint2(0u, 0u);
-        float sa = 0.0f, ba = 0.0f, sb_ = 0.0f, bb = 0.0f;
-        if (ca.t >= 0) {
-          const float2 v = csv[ca.t * NG + g];
-          sa = v.x;
-          ba = ca.l0 ? v.y * 0x1p-16f : 0.0f;
-        }
-        if (cb.t >= 0) {
-          const float2 v = csv[cb.t * NG + g];
-          sb_ = v.x;
-          bb = cb.l0 ? v.y * 0x1p-16f : 0.0f;
-        }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          uint32_t w[2][2];
-          tc_load_a<BITS>(wb + gid * GP + 2 * mt * RB, wb + gid * GP + (2 * mt + 1) * RB, g, q, w);
-          int c[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            uint32_t a[4];
-            tc_unpack_a<BITS>(w, kb, a);
-            mma_u8s8(c, a, b[kb].x, b[kb].y);
-          }
-          const float s0 = tc_scale<GPW>(sv[mt][0][0], gi), b0 = tc_scale<GPW>(sv[mt][0][1], gi);
-          const float s1 = tc_scale<GPW>(sv[mt][1][0], gi), b1 = tc_scale<GPW>(sv[mt][1][1], gi);
-          acc[mt][0] = fmaf(s0 * sa, (float)c[0], fmaf(b0, ba, acc[mt][0]));
-          acc[mt][1] = fmaf(s0 * sb_, (float)c[1], fmaf(b0, bb, acc[mt][1]));
-          acc[mt][2] = fmaf(s1 * sa, (float)c[2], fmaf(b1, ba, acc[mt][2]));
-          acc[mt][3] = fmaf(s1 * sb_, (float)c[3], fmaf(b1, bb, acc[mt][3]));
-        }
+      for (int i = 0; i < TPW; ++i) {
+        sc[i][0] = scl + (size_t)rlo[i] * NG;
+        sc[i][1] = scl + (size_t)(ROWS + rlo[i]) * NG;
+        sc[i][2] = scl + (size_t)rhi[i] * NG;
+        sc[i][3] = scl + (size_t)(ROWS + rhi[i]) * NG;
       }
+      tc_sum<BITS, NG, ROWS, GPW, TPW>(wb, wb, rlo, rhi, sc, dbase + (size_t)slot * DB, it.u.n, g0, acc);
     }
     __syncwarp();
     if (lane == 0) {
       mbar_arrive_one(smem_addr(&s_wempty[st]));
       if (it.last) mbar_arrive_one(smem_addr(&s_dempty[slot]));
     }
-    float* rw = red + ((k & 1) * kConsumers + warp) * TP;
+    if (k > 0) reduce(k - 1, p_row0, p_n, p_d0);
+    float* rw = red + ((k & 1) * KS + kp) * TP;
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int r = RPC * gid + 2 * mt;
-      *reinterpret_cast<float2*>(rw + r * 8 + 2 * q) = make_float2(acc[mt][0], acc[mt][1]);
-      *reinterpret_cast<float2*>(rw + (r + 1) * 8 + 2 * q) = make_float2(acc[mt][2], acc[mt][3]);
+    for (int i = 0; i < TPW; ++i) {
+      *reinterpret_cast<float2*>(rw + rlo[i] * 8 + 2 * q) = make_float2(acc[i][0], acc[i][1]);
+      *reinterpret_cast<float2*>(rw + rhi[i] * 8 + 2 * q) = make_float2(acc[i][2], acc[i][3]);
     }
     if (named_sync_or(!ok)) {
       if (tid == 0) s_abort = 1;
       return;
     }
-    const int d0 = it.blk * ROWS;
-#pragma unroll
-    for (int pass = 0; pass < (16 * ROWS + kConsumers * 32 - 1) / (kConsumers * 32); ++pass) {
-      const int idx = pass * kConsumers * 32 + tid;
-      if (idx < 16 * ROWS) {  // output (row r, token t) from warp slice ws, then the slices in order
-        const int o = idx >> 3, ws = idx & 7, r = o >> 1, t = o & 1;
-        const float* rs = red + ((k & 1) * kConsumers + ws) * TP + r * 8 + 3 * t;
-        float v = fmaf(65536.0f, rs[0], fmaf(256.0f, rs[1], rs[2]));
-#pragma unroll
-        for (int o2 = 1; o2 < 8; o2 <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-        if (ws == 0 && t < it.u.n) p.y[(size_t)(it.u.row0 + t) * H + d0 + r] = v;
-      }
-    }
+    p_row0 = it.u.row0;
+    p_n = it.u.n;
+    p_d0 = it.blk * ROWS;
   }
-  (void)I;
+  if (count > 0) reduce(count - 1, p_row0, p_n, p_d0);
 }
 
 // ---- combine, fixed k order: out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t]
@@ -884,71 +969,116 @@ __global__ void __launch_bounds__(kGT) grouped_combine_kernel(const GroupedParam
 constexpr size_t kSmemBudget = 220 * 1024;
 
 // Shared memory of an expert kernel: `ns` staged items of `wb` bytes, two digit
-// slots of kUnitToks members and the double-buffered partial tiles (tp floats
-// per consumer warp).
+// slots of kUnitToks members, the double-buffered partial tiles (tp floats per
+// buffer, all K slices) and 1 KiB to align the staging ring.
 size_t tc_smem(int ns, size_t wb, int NG, size_t tp) {
-  return (size_t)ns * wb + 2 * (size_t)kUnitToks * NG * 200 + 2 * (size_t)kConsumers * tp * 4;
+  return (size_t)ns * wb + 2 * (size_t)kUnitToks * NG * 200 + 2 * tp * 4 + 1024;
 }
 
+size_t round_kib(size_t v) { return (v + 1023) / 1024 * 1024; }
+
 struct TcConfig {
-  int rpc, ns;
+  int tl, ns;
   size_t smem;
 };
 
-// gate/up: the most rows per item (RPC 2, else 1) whose ring keeps at least
-// 64 KiB of rows in flight, with as many stages (<= 6) as fit.
+// gate/up: 16 row pairs per item (TL 2) while two stages fit, else 8 (TL 1),
+// with as many stages (<= 6) as fit.
 TcConfig gu_config(int bits, int H) {
   const int NG = H / kGroup, RB = H * bits / 8, SB = NG * 2;
-  for (int rpc : {2, 1}) {
-    const size_t wb = 16 * (size_t)(rpc * RB + kPad) + 32 * (size_t)rpc * SB;
-    const size_t tp = 2 * 8 * (size_t)rpc * 8 + 4;
+  for (int tl : {2, 1}) {
+    const int rows = 8 * tl, tpw = tl < 2 ? tl : 2, ks = 8 * tpw / tl;
+    const size_t wb = round_kib(2 * (size_t)rows * RB + 4 * (size_t)rows * SB);
+    const size_t tp = (size_t)ks * (2 * rows * 8 + 4);
     for (int n = 6; n >= 2; --n) {
       const size_t sm = tc_smem(n, wb, NG, tp);
-      if (sm <= kSmemBudget && ((n - 1) * wb >= 64 * 1024 || rpc == 1)) return TcConfig{rpc, n, sm};
+      if (sm <= kSmemBudget) return TcConfig{tl, n, sm};
     }
   }
   return TcConfig{0, 0, 0};
 }
 
-// down: RPC 8, 4 or 2 (64, 32 or 16 rows per item), the first with at least 3 stages (<= 8).
+// down: 64, 32 or 16 rows per item (TL 4, 2, 1), the first with at least 3 stages (<= 8).
 TcConfig dn_config(int bits, int I) {
   const int NG = I / kGroup, RB = I * bits / 8, SB = NG * 2;
-  for (int rpc : {8, 4, 2}) {
-    const size_t wb = 8 * (size_t)(rpc * RB + kPad) + 2 * 8 * (size_t)rpc * SB;
-    const size_t tp = 8 * (size_t)rpc * 8 + 4;
+  for (int tl : {4, 2, 1}) {
+    const int rows = 16 * tl, tpw = tl < 2 ? tl : 2, ks = 8 * tpw / tl;
+    const size_t wb = round_kib((size_t)rows * RB + 2 * (size_t)rows * SB);
+    const size_t tp = (size_t)ks * (rows * 8 + 4);
     for (int n = 8; n >= 3; --n) {
       const size_t sm = tc_smem(n, wb, NG, tp);
-      if (sm <= kSmemBudget) return TcConfig{rpc, n, sm};
+      if (sm <= kSmemBudget) return TcConfig{tl, n, sm};
     }
   }
   return TcConfig{0, 0, 0};
+}
+
+// The tensor map of one code matrix of a bank: `rows` rows of RB bytes per
+// expert, seen as (LW bytes, rows, RB / LW column blocks, experts) so that a
+// box of box_rows rows lands as (column block, row) lines; swizzled as TcSw
+// assumes.
+cudaError_t encode_codes(CUtensorMap* m, const uint8_t* base, int rows, int RB, int nexp, long long stride,
+                         int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!enc) return cudaErrorNotSupported;
+  const int LW = RB >= 128 ? 128 : RB;
+  const cuuint64_t dims[4] = {(cuuint64_t)LW, (cuuint64_t)rows, (cuuint64_t)(RB / LW), (cuuint64_t)nexp};
+  const cuuint64_t strides[3] = {(cuuint64_t)RB, (cuuint64_t)LW,
+                                 (cuuint64_t)(nexp > 1 ? stride : (long long)rows * RB)};
+  const cuuint32_t box[4] = {(cuuint32_t)LW, (cuuint32_t)box_rows, (cuuint32_t)(RB / LW), 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUtensorMapSwizzle sw =
+      LW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : LW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int BITS, int NG>
 cudaError_t gateup_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
-  void (*k)(const GroupedParams, int) =
-      c.rpc == 2 ? grouped_gateup_kernel<BITS, NG, 2> : grouped_gateup_kernel<BITS, NG, 1>;
-  cudaError_t e = set_smem((const void*)k, c.smem);
-  if (e != cudaSuccess) return e;
-  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns);
+  const int RB = p.H * BITS / 8, rows = 8 * c.tl;
+  alignas(64) CUtensorMap m[4];
+  cudaError_t e;
+  if ((e = encode_codes(&m[0], p.routed.base + p.routed.off[0], p.I, RB, p.E, p.routed.stride, rows)) != cudaSuccess ||
+      (e = encode_codes(&m[1], p.routed.base + p.routed.off[3], p.I, RB, p.E, p.routed.stride, rows)) != cudaSuccess ||
+      (e = encode_codes(&m[2], p.shared.base + p.shared.off[0], p.I, RB, 1, 0, rows)) != cudaSuccess ||
+      (e = encode_codes(&m[3], p.shared.base + p.shared.off[3], p.I, RB, 1, 0, rows)) != cudaSuccess)
+    return e;
+  auto k = c.tl == 2 ? grouped_gateup_kernel<BITS, NG, 2> : grouped_gateup_kernel<BITS, NG, 1>;
+  if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
+  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m[0], m[1], m[2], m[3]);
   return cudaGetLastError();
 }
 
 template <int BITS, int NG>
 cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
-  void (*k)(const GroupedParams, int) = c.rpc == 8   ? grouped_down_kernel<BITS, NG, 8>
-                                        : c.rpc == 4 ? grouped_down_kernel<BITS, NG, 4>
-                                                     : grouped_down_kernel<BITS, NG, 2>;
-  cudaError_t e = set_smem((const void*)k, c.smem);
-  if (e != cudaSuccess) return e;
-  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns);
+  const int RB = p.I * BITS / 8, rows = 16 * c.tl;
+  alignas(64) CUtensorMap m[2];
+  cudaError_t e;
+  if ((e = encode_codes(&m[0], p.routed.base + p.routed.off[6], p.H, RB, p.E, p.routed.stride, rows)) != cudaSuccess ||
+      (e = encode_codes(&m[1], p.shared.base + p.shared.off[6], p.H, RB, 1, 0, rows)) != cudaSuccess)
+    return e;
+  auto k = c.tl == 4 ? grouped_down_kernel<BITS, NG, 4>
+           : c.tl == 2 ? grouped_down_kernel<BITS, NG, 2>
+                       : grouped_down_kernel<BITS, NG, 1>;
+  if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
+  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m[0], m[1]);
   return cudaGetLastError();
 }
 
 template <int BITS>
 cudaError_t gateup_bits_g(const GroupedParams& p, cudaStream_t s) {
   const TcConfig c = gu_config(BITS, p.H);
-  if (c.rpc == 0) return cudaErrorInvalidValue;
+  if (c.tl == 0 || p.I % (8 * c.tl)) return cudaErrorInvalidValue;
   switch (p.H / kGroup) {
     case 2: return gateup_ng<BITS, 2>(p, c, s);
     case 4: return gateup_ng<BITS, 4>(p, c, s);
@@ -964,7 +1094,7 @@ cudaError_t gateup_bits_g(const GroupedParams& p, cudaStream_t s) {
 template <int BITS>
 cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
   const TcConfig c = dn_config(BITS, p.I);
-  if (c.rpc == 0 || p.H % (8 * c.rpc)) return cudaErrorInvalidValue;
+  if (c.tl == 0 || p.H % (16 * c.tl)) return cudaErrorInvalidValue;
   switch (p.I / kGroup) {
     case 2: return down_ng<BITS, 2>(p, c, s);
     case 4: return down_ng<BITS, 4>(p, c, s);
@@ -983,7 +1113,7 @@ bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T) {
   if (T * K > kMaxTK || ((size_t)T * K + 2 * (size_t)E) * 4 > 200 * 1024) return false;
   if ((size_t)kRtRows * H * 2 > 200 * 1024) return false;
   const TcConfig gu = gu_config(bits, H), dn = dn_config(bits, I);
-  return gu.rpc > 0 && I % (8 * gu.rpc) == 0 && dn.rpc > 0 && H % (8 * dn.rpc) == 0;
+  return gu.tl > 0 && I % (8 * gu.tl) == 0 && dn.tl > 0 && H % (16 * dn.tl) == 0;
 }
 
 cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s) {
