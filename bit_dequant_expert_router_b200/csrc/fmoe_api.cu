@@ -74,7 +74,7 @@ WsLayout layout(int H, int E, int K, int I, int T) {
 // between calls); the control block is the per-token one at offset 0.
 struct GLayout {
   size_t ctrl, logits, xq_limbs, xq_cs, route_idx, route_w, n_active, act_expert, act_off, pair_tok, pair_pos, work,
-      act, act_limbs, act_cs, y, x, total;
+      act, act_limbs, act_cs, y, x, rt_part, total;
 };
 
 GLayout glayout(int H, int E, int K, int I, int T) {
@@ -97,7 +97,8 @@ GLayout glayout(int H, int E, int K, int I, int T) {
   L.act_cs = L.act_limbs + up(nr * 3 * I);
   L.y = L.act_cs + up(nr * (I / 32) * 8);
   L.x = L.y + up(nr * H * 4);
-  L.total = L.x + up((size_t)T * H * 4);
+  L.rt_part = L.x + up((size_t)T * H * 4);
+  L.total = L.rt_part + up((size_t)grouped_router_split(H, E, T) * (E + 1) * T * 4);
   return L;
 }
 
@@ -562,6 +563,9 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   p.pair_tok = reinterpret_cast<int32_t*>(base + G.pair_tok);
   p.pair_pos = reinterpret_cast<int32_t*>(base + G.pair_pos);
   p.units = reinterpret_cast<UnitDesc*>(base + G.work);
+  p.rt_part = reinterpret_cast<float*>(base + G.rt_part);
+  p.rt_split = grouped_router_split(H, E, T);
+  p.rt_bias = layer->router_bias;
   p.act = reinterpret_cast<float*>(base + G.act);
   p.act_limbs = base + G.act_limbs;
   p.act_cs = reinterpret_cast<float2*>(base + G.act_cs);
@@ -570,7 +574,8 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   p.out = out;
   p.err = err;
   cudaError_t e;
-  if ((e = launch_grouped_router(p, rb, bits, s)) != cudaSuccess) return cuda_fail(e, "router launch");
+  if ((e = launch_grouped_router(p, rb, bits, s)) != cudaSuccess)
+    return cuda_fail(e, "router launch");
   if ((e = launch_grouped_select(p, s)) != cudaSuccess) return cuda_fail(e, "select launch");
   if ((e = launch_grouped_gateup(p, bits, s)) != cudaSuccess) return cuda_fail(e, "grouped gate/up launch");
   if ((e = launch_grouped_actq(p, bits, s)) != cudaSuccess) return cuda_fail(e, "activation digits launch");

@@ -98,6 +98,9 @@ struct GroupedParams {
   float* w_out;
   int32_t* n_active;          // [2] U: active experts, W: work units
   UnitDesc* units;            // [T*K + T] work units of the expert kernels, the shared expert's first
+  float* rt_part;             // [rt_split][T][E+1] the router's slice sums
+  int rt_split;
+  const float* rt_bias;       // [E] or NULL
   int32_t* act_expert;        // [T*K] active experts, increasing
   int32_t* act_off;           // [T*K+1] first pair of each active expert in the sorted pair list
   int32_t* pair_tok;          // [T*K] sorted pairs (expert, token, k): value t*K + k
@@ -121,6 +124,8 @@ struct RouterBatch {
   float* x;                   // workspace [T][H]: x in fp32
 };
 
+// The batched router's split-K factor: the workspace holds split * T * (E+1) partial logits.
+int grouped_router_split(int H, int E, int T);
 cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s);
 cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s);
 cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, cudaStream_t s);

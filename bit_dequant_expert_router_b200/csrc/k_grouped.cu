@@ -31,8 +31,6 @@ namespace {
 
 constexpr int kGT = 256;          // threads per CTA
 constexpr int kMaxTK = 4096;      // T*K pairs
-constexpr int kRtRows = 8;        // router rows per CTA (batched router)
-constexpr int kRtTok = 16;        // tokens per CTA (batched router)
 
 // ---- int8 tensor-core contraction of codes with activation digits.
 // The batched expert products run on mma.sync m16n8k32 (u8 codes x s8 digits,
@@ -100,8 +98,20 @@ __global__ void __launch_bounds__(kGT) topk_tokens_kernel(const GroupedParams p)
   __shared__ int s_idx[32];
   __shared__ float s_w[33];
   __shared__ unsigned long long s_cand[8 * 32];
-  const int t = blockIdx.x, tid = threadIdx.x, K = p.K, E = p.E;
-  block_topk(p.logits + (size_t)t * (E + 1), E, K, 1, s_cand, s_idx, s_w);
+  const int t = blockIdx.x, tid = threadIdx.x, K = p.K, E = p.E, R = E + 1, T = p.T, ns = p.rt_split;
+  float* lg = const_cast<float*>(p.logits) + (size_t)t * R;
+  for (int r = tid; r < R; r += kGT) {  // the router's slice sums, in slice order, then the bias
+    float v[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) v[c] = c < ns ? __ldcg(p.rt_part + ((size_t)c * T + t) * R + r) : 0.0f;
+    float l = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) l += v[c];
+    if (r < E && p.rt_bias) l += p.rt_bias[r];
+    lg[r] = l;
+  }
+  __syncthreads();  // the block's own global writes are visible to it after the barrier
+  block_topk(lg, E, K, 1, s_cand, s_idx, s_w);
   if (tid < K) {
     int e = s_idx[tid];
     e = (e < 0 || e >= E) ? 0 : e;
@@ -264,70 +274,63 @@ __global__ void __launch_bounds__(kGT) norm_digits_kernel(const GroupedParams p,
   }
 }
 
-// router_gemm: CTA (a, b) computes logits of rows [8a, 8a+8) of [W_r; w_sg] for
-// tokens [16b, 16b+16): the rows are staged once, x of each token streams from
-// L2.  Warp w sums column slice w (H/8 columns); the 8 slice sums add in fixed order.
+// router_gemm: partial logits of [W_r; w_sg] . x[t] as a split-K tiled product.
+// CTA (a, b, c) takes rows [64a, 64a+64), tokens [64b, 64b+64) and the c-th of
+// p.rt_split slices of H, staged 256 columns at a time (cp.async); thread
+// (ty, tx) sums rows ty + 16i and tokens tx + 16j.  The slice sums go to
+// rt_part[c][t][row]; the top-K kernel adds the slices in order and the bias.
+constexpr int kRtR = 64, kRtT = 64, kRtK = 256;  // rows, tokens and columns per staged tile
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
 __global__ void __launch_bounds__(kGT) router_gemm_kernel(const GroupedParams p, const RouterBatch rb) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ float s_part[kRtTok][kRtRows][kGT / 32];
-  __shared__ __align__(8) uint64_t s_bar;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, H = p.H, E = p.E;
-  const int r0 = blockIdx.x * kRtRows, n = min(kRtRows, E + 1 - r0);
-  const int t0 = blockIdx.y * kRtTok, nt = min(kRtTok, p.T - t0);
-  uint16_t* w = reinterpret_cast<uint16_t*>(sm);
-  if (tid == 0) {
-    const uint32_t bar = smem_addr(&s_bar);
-    mbar_init(bar, 1);
-    mbar_fence_init();
-    const int nr = max(0, min(n, E - r0));  // rows of w_router; the rest is the shared-gate row
-    mbar_expect_tx(bar, (uint32_t)n * H * 2);
-    if (nr > 0) bulk_g2s(smem_addr(w), rb.w_router + (size_t)r0 * H, (uint32_t)nr * H * 2, bar, l2_policy_evict_first());
-    if (nr < n) bulk_g2s(smem_addr(w + (size_t)nr * H), rb.w_sgate, (uint32_t)H * 2, bar, l2_policy_evict_first());
-  }
-  __syncthreads();
-  const bool ok = mbar_wait_bounded(smem_addr(&s_bar), 0, p.err);
-  const uint16_t* ws = w + warp * (H / 8);
-  for (int j = 0; ok && j < nt; ++j) {
-    const float* xs = rb.x + (size_t)(t0 + j) * H + warp * (H / 8);
-    float acc[kRtRows];
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15, H = p.H, E = p.E, T = p.T, R = E + 1;
+  const int r0 = blockIdx.x * kRtR, t0 = blockIdx.y * kRtT, kc = blockIdx.z, KC = H / p.rt_split;
+  constexpr int WP = kRtK + 8, XP = kRtK + 4;  // padded row pitches (bf16, fp32)
+  uint16_t* ws = reinterpret_cast<uint16_t*>(sm);
+  float* xs = reinterpret_cast<float*>(sm + (size_t)kRtR * WP * 2);
+  float acc[4][4] = {};
+  for (int k0 = kc * KC; k0 < (kc + 1) * KC; k0 += kRtK) {
+    const int kn = min(kRtK, (kc + 1) * KC - k0);  // a multiple of 64
+    if (k0 != kc * KC) __syncthreads();          // the previous columns are summed
+    for (int i = tid; i < kRtR * (kn / 8); i += kGT) {  // rows: W_r, then the shared-gate row, then zeros
+      const int r = i / (kn / 8), c = (i % (kn / 8)) * 8, row = r0 + r;
+      const uint16_t* src = row < E ? rb.w_router + (size_t)row * H + k0 + c : rb.w_sgate + k0 + c;
+      cp_async16(ws + (size_t)r * WP + c, src, row <= E);
+    }
+    for (int i = tid; i < kRtT * (kn / 4); i += kGT) {
+      const int t = i / (kn / 4), c = (i % (kn / 4)) * 4;
+      cp_async16(xs + (size_t)t * XP + c, rb.x + (size_t)min(t0 + t, T - 1) * H + k0 + c, t0 + t < T);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    for (int k = 0; k < kn; k += 4) {
+      float4 xv[4];
 #pragma unroll
-    for (int r = 0; r < kRtRows; ++r) acc[r] = 0.0f;
-    for (int k = lane; k < H / 64; k += 32) {
-      const float4 xa = __ldcg(reinterpret_cast<const float4*>(xs + 8 * k));
-      const float4 xb = __ldcg(reinterpret_cast<const float4*>(xs + 8 * k + 4));
+      for (int j = 0; j < 4; ++j) xv[j] = *reinterpret_cast<const float4*>(xs + (size_t)(tx + 16 * j) * XP + k);
 #pragma unroll
-      for (int r = 0; r < kRtRows; ++r) {
-        if (r < n) {
-          const uint4 q = *reinterpret_cast<const uint4*>(ws + (size_t)r * H + 8 * k);
-          float a = acc[r];
-          a = fmaf(__uint_as_float(q.x << 16), xa.x, a);
-          a = fmaf(__uint_as_float(q.x & 0xFFFF0000u), xa.y, a);
-          a = fmaf(__uint_as_float(q.y << 16), xa.z, a);
-          a = fmaf(__uint_as_float(q.y & 0xFFFF0000u), xa.w, a);
-          a = fmaf(__uint_as_float(q.z << 16), xb.x, a);
-          a = fmaf(__uint_as_float(q.z & 0xFFFF0000u), xb.y, a);
-          a = fmaf(__uint_as_float(q.w << 16), xb.z, a);
-          a = fmaf(__uint_as_float(q.w & 0xFFFF0000u), xb.w, a);
-          acc[r] = a;
-        }
+      for (int i = 0; i < 4; ++i) {
+        const uint2 wv = *reinterpret_cast<const uint2*>(ws + (size_t)(ty + 16 * i) * WP + k);
+        const float w0 = __uint_as_float(wv.x << 16), w1 = __uint_as_float(wv.x & 0xFFFF0000u);
+        const float w2 = __uint_as_float(wv.y << 16), w3 = __uint_as_float(wv.y & 0xFFFF0000u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          acc[i][j] = fmaf(w3, xv[j].w, fmaf(w2, xv[j].z, fmaf(w1, xv[j].y, fmaf(w0, xv[j].x, acc[i][j]))));
       }
     }
-#pragma unroll
-    for (int r = 0; r < kRtRows; ++r) acc[r] = warp_sum(acc[r]);
-    if (lane == 0)
-#pragma unroll
-      for (int r = 0; r < kRtRows; ++r) s_part[j][r][warp] = acc[r];
   }
-  __syncthreads();
-  for (int i = tid; ok && i < nt * n; i += kGT) {
-    const int j = i / n, r = i % n;
-    float l = 0.0f;
+  float* pc = p.rt_part + (size_t)kc * T * R;  // this slice's partials [T][R]
 #pragma unroll
-    for (int q = 0; q < kGT / 32; ++q) l += s_part[j][r][q];
-    const int row = r0 + r;
-    if (row < E && rb.bias) l += rb.bias[row];
-    const_cast<float*>(p.logits)[(size_t)(t0 + j) * (E + 1) + row] = l;
-  }
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = r0 + ty + 16 * i, t = t0 + tx + 16 * j;
+      if (row < R && t < T) pc[(size_t)t * R + row] = acc[i][j];
+    }
 }
 
 // ---- the two expert kernels share one schedule.  Persistent, one CTA per SM,
@@ -438,22 +441,25 @@ struct TcRows {
   static constexpr int CB = NG * 8;                 // its per-group scalars
 };
 
-// Staged code rows: one tensor copy per matrix brings an item's ROWS rows as
-// lines of LW = min(128, RB) bytes ordered (column block, row), with the copy's
-// swizzle: the 16-byte chunk index of byte X is XORed with bits 7.. of X
-// (128-byte swizzle: 3 bits, 64-byte: 2, 32-byte: 1).  Rows gid = 0..7 of a
-// tile are consecutive, so the eight rows a quad-layout load reads land in
+// Staged rows (codes, and the per-group scale arrays): one tensor copy per array
+// brings an item's ROWS rows of RB bytes as lines of LW = min(128, RB) bytes
+// ordered (column block, row), with the copy's swizzle: the 16-byte chunk
+// index of byte X is XORed with bits 7.. of X (128-byte swizzle: 3 bits,
+// 64-byte: 2, 32-byte: 1; 16-byte lines are not swizzled).  Rows gid = 0..7 of
+// a tile are consecutive, so the eight rows a quad-layout load reads land in
 // distinct chunks.
-template <int BITS, int NG, int ROWS>
-struct TcSw {
-  static constexpr int RB = NG * kGroup * BITS / 8;
+template <int RB, int ROWS>
+struct Sw {
   static constexpr int LW = RB >= 128 ? 128 : RB;
-  static constexpr int M = LW == 128 ? 7 : LW == 64 ? 3 : 1;
+  static constexpr int M = LW == 128 ? 7 : LW == 64 ? 3 : LW == 32 ? 1 : 0;
   __device__ static __forceinline__ const uint8_t* at(const uint8_t* buf, int row, int c) {
     const int X = ((c / LW) * ROWS + row) * LW + c % LW;
     return buf + (X ^ (((X >> 7) & M) << 4));
   }
 };
+
+template <int BITS, int NG, int ROWS>
+using TcSw = Sw<NG * kGroup * BITS / 8, ROWS>;
 
 // A registers of staged rows row_lo (A rows 0-7) and row_hi (rows 8-15) for group g.
 template <int BITS, int NG, int ROWS>
@@ -556,7 +562,7 @@ struct TcColScale {
 };
 
 __device__ __forceinline__ TcColScale tc_colscale(const float2* csv, int NG, int g, const TcLane& l) {
-  const float2 va = csv[l.ta * NG + g], vb = csv[l.tb * NG + g];
+  const float2 va = csv[l.ta * (NG + 2) + g], vb = csv[l.tb * (NG + 2) + g];
   TcColScale c;
   c.sa = l.va ? va.x : 0.0f;
   c.sb = l.vb ? vb.x : 0.0f;
@@ -589,12 +595,13 @@ __device__ __forceinline__ void tc_tile_group(const uint32_t (&w)[2][2], const u
 
 // Sums TPW tiles over groups [g0, g0 + GPW) into acc (each tile's C layout,
 // bias folded into the limb-0 columns).  Tile i reads rows rlo[i] of buf_lo and
-// rhi[i] of buf_hi (staged, ROWS rows each); sc[i] = its scale rows
-// {s_lo, b_lo, s_hi, b_hi} at group 0.  B and the column scales are shared by
-// the tiles.
+// rhi[i] of buf_hi (staged, ROWS rows each); its row scales and biases come
+// from the staged scale arrays sarr = {s_lo, b_lo, s_hi, b_hi} (row rlo[i] for
+// the first two, rhi[i] for the others).  B and the column scales are shared
+// by the tiles.
 template <int BITS, int NG, int ROWS, int GPW, int TPW>
 __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf_hi, const int (&rlo)[TPW],
-                                       const int (&rhi)[TPW], const uint16_t* const (&sc)[TPW][4], const uint8_t* db, int n,
+                                       const int (&rhi)[TPW], const uint8_t* const (&sarr)[4], const uint8_t* db, int n,
                                        int g0, float (&acc)[TPW][4]) {
   constexpr int LB = NG * 192;
   constexpr int GPC = GPW < 8 ? GPW : 8;  // groups whose scales are held at once
@@ -602,7 +609,7 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
   const TcLane ln = tc_lane(q, n);
   const int bt = gid < 6 ? gid / 3 : 0, bl = gid % 3;  // this lane's B column: token slot, limb
   const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
-  const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);
+  const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);  // [token][NG + 2] (padded pitch)
   float accb[TPW][2];
 #pragma unroll
   for (int i = 0; i < TPW; ++i) accb[i][0] = accb[i][1] = 0.0f;
@@ -612,7 +619,10 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
 #pragma unroll
     for (int i = 0; i < TPW; ++i)
 #pragma unroll
-      for (int a = 0; a < 4; ++a) tc_load_scales<GPC>(sc[i][a] + g0 + gc, sv[i][a]);
+      for (int a = 0; a < 4; ++a)
+        tc_load_scales<GPC>(
+            reinterpret_cast<const uint16_t*>(Sw<NG * 2, ROWS>::at(sarr[a], a < 2 ? rlo[i] : rhi[i], (g0 + gc) * 2)),
+            sv[i][a]);
 #pragma unroll
     for (int gi = 0; gi < GPC; ++gi) {
       const int g = g0 + gc + gi;
@@ -641,6 +651,12 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
   }
 }
 
+// The tensor maps of a kernel's staged arrays: routed bank first, then the shared expert's.
+template <int N>
+struct TcMaps {
+  CUtensorMap m[N];
+};
+
 // cp.async.bulk.tensor of a 4-D box at (0, row, 0, expert) into shared memory.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, int row, int expert, uint32_t bar,
                                             uint64_t pol) {
@@ -659,17 +675,17 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
 // add in slice order.  act[row][r] = silu(g) * u.
 template <int BITS, int NG, int TL>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gateup_kernel(const GroupedParams p, int ns, const __grid_constant__ CUtensorMap tm_rg,
-                          const __grid_constant__ CUtensorMap tm_ru, const __grid_constant__ CUtensorMap tm_sg,
-                          const __grid_constant__ CUtensorMap tm_su) {
+    grouped_gateup_kernel(const GroupedParams p, int ns, const __grid_constant__ TcMaps<12> maps) {
   using R = TcRows<BITS, NG>;
   constexpr int RB = R::RB, LB = R::LB, CB = R::CB, SB = NG * 2;
-  constexpr int ROWS = 8 * TL, TPW = TL < 2 ? TL : 2, KS = 8 * TPW / TL;
-  constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;  // groups per K slice
-  constexpr int CODE = ROWS * RB;                   // one matrix's staged rows
-  constexpr int WB = (2 * CODE + 4 * ROWS * SB + 1023) / 1024 * 1024;
-  constexpr int DB = kUnitToks * (LB + CB);
-  constexpr int TP = 2 * ROWS * 8 + 4;              // floats per slice's partial tiles (gate rows, then up rows)
+  constexpr int ROWS = 8 * TL, TPW = TL < 2 ? TL : 2, KS = kConsumers * TPW / TL;  // TPW tiles per warp, KS K slices
+  constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;                                  // groups per K slice
+  constexpr int CODE = (ROWS * RB + 1023) / 1024 * 1024;  // one matrix's staged rows
+  constexpr int SA = (ROWS * SB + 1023) / 1024 * 1024;    // one staged scale array
+  constexpr int WB = 2 * CODE + 4 * SA;                   // gate rows, up rows, gate s, gate b, up s, up b
+  constexpr int CBP = CB + 16;                            // a token's scalars, padded apart in shared memory
+  constexpr int DB = kUnitToks * (LB + CBP);
+  constexpr int TP = 2 * ROWS * 8 + 4;  // floats per slice's partial tiles (gate rows, then up rows)
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
   __shared__ ItemDesc s_item[kRing];
@@ -697,21 +713,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kConsumers) {  // the producer
     const uint64_t pol_w = l2_policy_evict_first(), pol_d = l2_policy_evict_last();
-    auto issue_w = [&](const ItemDesc& it, int st) {
+    auto issue_w = [&](const ItemDesc& it, int st) {  // gate rows, up rows, then the four scale arrays
       const int r0 = it.blk * ROWS;
       const uint32_t bw = smem_addr(&s_wfull[st]), dst = smem_addr(sm + (size_t)st * WB);
-      if (lane == 0) {
-        mbar_expect_tx(bw, 2 * CODE + 4 * ROWS * SB);
-        const bool sh = it.u.e < 0;
-        tma_load_4d(dst, sh ? &tm_sg : &tm_rg, r0, sh ? 0 : it.u.e, bw, pol_w);
-        tma_load_4d(dst + CODE, sh ? &tm_su : &tm_ru, r0, sh ? 0 : it.u.e, bw, pol_w);
-      }
+      if (lane == 0) mbar_expect_tx(bw, 2 * ROWS * RB + 4 * ROWS * SB);
       __syncwarp();
-      if (lane >= 1 && lane <= 4) {  // gate s, gate b, up s, up b
-        const int a = lane - 1;
-        const long long off = p.routed.off[a == 0 ? 1 : a == 1 ? 2 : a == 2 ? 4 : 5];
-        bulk_g2s(dst + 2 * CODE + a * ROWS * SB, unit_record(p, it.u.e) + off + (long long)r0 * SB, ROWS * SB, bw,
-                 pol_w);
+      if (lane < 6) {
+        const bool sh = it.u.e < 0;
+        const uint32_t off = lane == 0 ? 0u : lane == 1 ? (uint32_t)CODE : (uint32_t)(2 * CODE + (lane - 2) * SA);
+        tma_load_4d(dst + off, &maps.m[(sh ? 6 : 0) + lane], r0, sh ? 0 : it.u.e, bw, pol_w);
       }
     };
     auto issue_d = [&](const UnitDesc& u, int slot) {
@@ -722,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane < u.n) {
         const int tok = u.tok[lane];
         bulk_g2s(smem_addr(dst + lane * LB), p.xq_limbs + (size_t)tok * LB, LB, bd, pol_d);
-        bulk_g2s(smem_addr(dst + kUnitToks * LB + lane * CB), p.xq_cs + (size_t)tok * NG, CB, bd, pol_d);
+        bulk_g2s(smem_addr(dst + kUnitToks * LB + lane * CBP), p.xq_cs + (size_t)tok * NG, CB, bd, pol_d);
       }
     };
     producer_loop(p, NB, i0, count, ns, s_item, s_wfull, s_wempty, s_dfull, s_dempty, &s_abort, issue_w, issue_d);
@@ -763,17 +773,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && it.first) ok = mbar_wait_bounded(smem_addr(&s_dfull[slot]), (uint32_t)((it.useq >> 1) & 1), p.err);
     ok = __all_sync(0xffffffffu, ok);
     const uint8_t* wb = sm + (size_t)st * WB;
-    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + 2 * CODE);
     float acc[TPW][4];
 #pragma unroll
     for (int i = 0; i < TPW; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
     if (ok && kwarp) {
-      const uint16_t* sc[TPW][4];
-#pragma unroll
-      for (int i = 0; i < TPW; ++i)
-#pragma unroll
-        for (int a = 0; a < 4; ++a) sc[i][a] = scl + (size_t)(a * ROWS + rows[i]) * NG;
-      tc_sum<BITS, NG, ROWS, GPW, TPW>(wb, wb + CODE, rows, rows, sc, dbase + (size_t)slot * DB, it.u.n, g0, acc);
+      const uint8_t* const sarr[4] = {wb + 2 * CODE, wb + 2 * CODE + SA, wb + 2 * CODE + 2 * SA, wb + 2 * CODE + 3 * SA};
+      tc_sum<BITS, NG, ROWS, GPW, TPW>(wb, wb + CODE, rows, rows, sarr, dbase + (size_t)slot * DB, it.u.n, g0, acc);
     }
     __syncwarp();
     if (lane == 0) {  // this warp is done with the item's rows (and, on its last item, the unit's digits)
@@ -820,15 +825,16 @@ __global__ void __launch_bounds__(kGT) grouped_actq_kernel(const GroupedParams p
 // unweighted down output.
 template <int BITS, int NG, int TL>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_down_kernel(const GroupedParams p, int ns, const __grid_constant__ CUtensorMap tm_rd,
-                        const __grid_constant__ CUtensorMap tm_sd) {
+    grouped_down_kernel(const GroupedParams p, int ns, const __grid_constant__ TcMaps<6> maps) {
   using R = TcRows<BITS, NG>;
   constexpr int RB = R::RB, LB = R::LB, CB = R::CB, SB = NG * 2;
-  constexpr int ROWS = 16 * TL, TPW = TL < 2 ? TL : 2, KS = 8 * TPW / TL;
+  constexpr int ROWS = 16 * TL, TPW = TL < 2 ? TL : 2, KS = kConsumers * TPW / TL;
   constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;
-  constexpr int CODE = ROWS * RB;
-  constexpr int WB = (CODE + 2 * ROWS * SB + 1023) / 1024 * 1024;
-  constexpr int DB = kUnitToks * (LB + CB);
+  constexpr int CODE = (ROWS * RB + 1023) / 1024 * 1024;
+  constexpr int SA = (ROWS * SB + 1023) / 1024 * 1024;
+  constexpr int WB = CODE + 2 * SA;  // rows, then s, b
+  constexpr int CBP = CB + 16;
+  constexpr int DB = kUnitToks * (LB + CBP);
   constexpr int TP = ROWS * 8 + 4;
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
@@ -857,17 +863,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kConsumers) {  // the producer
     const uint64_t pol_w = l2_policy_evict_first(), pol_d = l2_policy_evict_last();
-    auto issue_w = [&](const ItemDesc& it, int st) {
+    auto issue_w = [&](const ItemDesc& it, int st) {  // rows, then the scale arrays s, b
       const int d0 = it.blk * ROWS;
       const uint32_t bw = smem_addr(&s_wfull[st]), dst = smem_addr(sm + (size_t)st * WB);
-      if (lane == 0) {
-        mbar_expect_tx(bw, CODE + 2 * ROWS * SB);
-        tma_load_4d(dst, it.u.e < 0 ? &tm_sd : &tm_rd, d0, it.u.e < 0 ? 0 : it.u.e, bw, pol_w);
-      }
+      if (lane == 0) mbar_expect_tx(bw, ROWS * RB + 2 * ROWS * SB);
       __syncwarp();
-      if (lane >= 1 && lane <= 2)  // s, b
-        bulk_g2s(dst + CODE + (lane - 1) * ROWS * SB, unit_record(p, it.u.e) + p.routed.off[6 + lane] + (long long)d0 * SB,
-                 ROWS * SB, bw, pol_w);
+      if (lane < 3) {
+        const bool sh = it.u.e < 0;
+        const uint32_t off = lane == 0 ? 0u : (uint32_t)(CODE + (lane - 1) * SA);
+        tma_load_4d(dst + off, &maps.m[(sh ? 3 : 0) + lane], d0, sh ? 0 : it.u.e, bw, pol_w);
+      }
     };
     auto issue_d = [&](const UnitDesc& u, int slot) {
       const uint32_t bd = smem_addr(&s_dfull[slot]);
@@ -875,8 +880,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         mbar_expect_tx(bd, (uint32_t)u.n * (LB + CB));
         bulk_g2s(smem_addr(dst), p.act_limbs + (size_t)u.row0 * LB, u.n * LB, bd, pol_d);
-        bulk_g2s(smem_addr(dst + kUnitToks * LB), p.act_cs + (size_t)u.row0 * NG, u.n * CB, bd, pol_d);
       }
+      __syncwarp();
+      if (lane < u.n)
+        bulk_g2s(smem_addr(dst + kUnitToks * LB + lane * CBP), p.act_cs + (size_t)(u.row0 + lane) * NG, CB, bd, pol_d);
     };
     producer_loop(p, NB, i0, count, ns, s_item, s_wfull, s_wempty, s_dfull, s_dempty, &s_abort, issue_w, issue_d);
     return;
@@ -914,20 +921,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && it.first) ok = mbar_wait_bounded(smem_addr(&s_dfull[slot]), (uint32_t)((it.useq >> 1) & 1), p.err);
     ok = __all_sync(0xffffffffu, ok);
     const uint8_t* wb = sm + (size_t)st * WB;
-    const uint16_t* scl = reinterpret_cast<const uint16_t*>(wb + CODE);
     float acc[TPW][4];
 #pragma unroll
     for (int i = 0; i < TPW; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
     if (ok && kwarp) {
-      const uint16_t* sc[TPW][4];
-#pragma unroll
-      for (int i = 0; i < TPW; ++i) {
-        sc[i][0] = scl + (size_t)rlo[i] * NG;
-        sc[i][1] = scl + (size_t)(ROWS + rlo[i]) * NG;
-        sc[i][2] = scl + (size_t)rhi[i] * NG;
-        sc[i][3] = scl + (size_t)(ROWS + rhi[i]) * NG;
-      }
-      tc_sum<BITS, NG, ROWS, GPW, TPW>(wb, wb, rlo, rhi, sc, dbase + (size_t)slot * DB, it.u.n, g0, acc);
+      const uint8_t* const sarr[4] = {wb + CODE, wb + CODE + SA, wb + CODE, wb + CODE + SA};
+      tc_sum<BITS, NG, ROWS, GPW, TPW>(wb, wb, rlo, rhi, sarr, dbase + (size_t)slot * DB, it.u.n, g0, acc);
     }
     __syncwarp();
     if (lane == 0) {
@@ -972,7 +971,7 @@ constexpr size_t kSmemBudget = 220 * 1024;
 // slots of kUnitToks members, the double-buffered partial tiles (tp floats per
 // buffer, all K slices) and 1 KiB to align the staging ring.
 size_t tc_smem(int ns, size_t wb, int NG, size_t tp) {
-  return (size_t)ns * wb + 2 * (size_t)kUnitToks * NG * 200 + 2 * tp * 4 + 1024;
+  return (size_t)ns * wb + 2 * (size_t)kUnitToks * ((size_t)NG * 200 + 16) + 2 * tp * 4 + 1024;
 }
 
 size_t round_kib(size_t v) { return (v + 1023) / 1024 * 1024; }
@@ -987,8 +986,8 @@ struct TcConfig {
 TcConfig gu_config(int bits, int H) {
   const int NG = H / kGroup, RB = H * bits / 8, SB = NG * 2;
   for (int tl : {2, 1}) {
-    const int rows = 8 * tl, tpw = tl < 2 ? tl : 2, ks = 8 * tpw / tl;
-    const size_t wb = round_kib(2 * (size_t)rows * RB + 4 * (size_t)rows * SB);
+    const int rows = 8 * tl, ks = kConsumers * (tl < 2 ? tl : 2) / tl;
+    const size_t wb = 2 * round_kib((size_t)rows * RB) + 4 * round_kib((size_t)rows * SB);
     const size_t tp = (size_t)ks * (2 * rows * 8 + 4);
     for (int n = 6; n >= 2; --n) {
       const size_t sm = tc_smem(n, wb, NG, tp);
@@ -1002,8 +1001,8 @@ TcConfig gu_config(int bits, int H) {
 TcConfig dn_config(int bits, int I) {
   const int NG = I / kGroup, RB = I * bits / 8, SB = NG * 2;
   for (int tl : {4, 2, 1}) {
-    const int rows = 16 * tl, tpw = tl < 2 ? tl : 2, ks = 8 * tpw / tl;
-    const size_t wb = round_kib((size_t)rows * RB + 2 * (size_t)rows * SB);
+    const int rows = 16 * tl, ks = kConsumers * (tl < 2 ? tl : 2) / tl;
+    const size_t wb = round_kib((size_t)rows * RB) + 2 * round_kib((size_t)rows * SB);
     const size_t tp = (size_t)ks * (rows * 8 + 4);
     for (int n = 8; n >= 3; --n) {
       const size_t sm = tc_smem(n, wb, NG, tp);
@@ -1013,10 +1012,10 @@ TcConfig dn_config(int bits, int I) {
   return TcConfig{0, 0, 0};
 }
 
-// The tensor map of one code matrix of a bank: `rows` rows of RB bytes per
-// expert, seen as (LW bytes, rows, RB / LW column blocks, experts) so that a
-// box of box_rows rows lands as (column block, row) lines; swizzled as TcSw
-// assumes.
+// The tensor map of one staged array of a bank (a code matrix, or a per-group
+// scale array): `rows` rows of RB bytes per expert, seen as (LW bytes, rows,
+// RB / LW column blocks, experts) so that a box of box_rows rows lands as
+// (column block, row) lines; swizzled as Sw assumes.
 cudaError_t encode_codes(CUtensorMap* m, const uint8_t* base, int rows, int RB, int nexp, long long stride,
                          int box_rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
@@ -1035,43 +1034,56 @@ cudaError_t encode_codes(CUtensorMap* m, const uint8_t* base, int rows, int RB, 
                                  (cuuint64_t)(nexp > 1 ? stride : (long long)rows * RB)};
   const cuuint32_t box[4] = {(cuuint32_t)LW, (cuuint32_t)box_rows, (cuuint32_t)(RB / LW), 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
-  const CUtensorMapSwizzle sw =
-      LW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : LW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  const CUtensorMapSwizzle sw = LW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : LW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : LW == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                           : CU_TENSOR_MAP_SWIZZLE_NONE;
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(base), dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Maps of the arrays `subs` (record sub-array indices) of both banks: rows of
+// the codes are rb bytes, of the scale arrays 2 * NG bytes.
+template <int N>
+cudaError_t encode_maps(TcMaps<N>& m, const GroupedParams& p, const int (&subs)[N / 2], bool codes_first, int rows,
+                        int rb, int NG, int box_rows) {
+  for (int b = 0; b < 2; ++b) {
+    const BankRef& bk = b == 0 ? p.routed : p.shared;
+    for (int j = 0; j < N / 2; ++j) {
+      const int w = (codes_first && j == 0) || (!codes_first && j < 2) ? rb : 2 * NG;
+      const cudaError_t e = encode_codes(&m.m[b * (N / 2) + j], bk.base + bk.off[subs[j]], rows, w, b == 0 ? p.E : 1,
+                                         b == 0 ? bk.stride : 0, box_rows);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  return cudaSuccess;
+}
+
 template <int BITS, int NG>
 cudaError_t gateup_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
-  const int RB = p.H * BITS / 8, rows = 8 * c.tl;
-  alignas(64) CUtensorMap m[4];
-  cudaError_t e;
-  if ((e = encode_codes(&m[0], p.routed.base + p.routed.off[0], p.I, RB, p.E, p.routed.stride, rows)) != cudaSuccess ||
-      (e = encode_codes(&m[1], p.routed.base + p.routed.off[3], p.I, RB, p.E, p.routed.stride, rows)) != cudaSuccess ||
-      (e = encode_codes(&m[2], p.shared.base + p.shared.off[0], p.I, RB, 1, 0, rows)) != cudaSuccess ||
-      (e = encode_codes(&m[3], p.shared.base + p.shared.off[3], p.I, RB, 1, 0, rows)) != cudaSuccess)
-    return e;
+  TcMaps<12> m;
+  static constexpr int subs[6] = {0, 3, 1, 2, 4, 5};  // gate rows, up rows, gate s, gate b, up s, up b
+  cudaError_t e = encode_maps(m, p, subs, false, p.I, p.H * BITS / 8, NG, 8 * c.tl);
+  if (e != cudaSuccess) return e;
   auto k = c.tl == 2 ? grouped_gateup_kernel<BITS, NG, 2> : grouped_gateup_kernel<BITS, NG, 1>;
   if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
-  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m[0], m[1], m[2], m[3]);
+  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m);
   return cudaGetLastError();
 }
 
 template <int BITS, int NG>
 cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
-  const int RB = p.I * BITS / 8, rows = 16 * c.tl;
-  alignas(64) CUtensorMap m[2];
-  cudaError_t e;
-  if ((e = encode_codes(&m[0], p.routed.base + p.routed.off[6], p.H, RB, p.E, p.routed.stride, rows)) != cudaSuccess ||
-      (e = encode_codes(&m[1], p.shared.base + p.shared.off[6], p.H, RB, 1, 0, rows)) != cudaSuccess)
-    return e;
+  TcMaps<6> m;
+  static constexpr int subs[3] = {6, 7, 8};  // rows, s, b
+  cudaError_t e = encode_maps(m, p, subs, true, p.H, p.I * BITS / 8, NG, 16 * c.tl);
+  if (e != cudaSuccess) return e;
   auto k = c.tl == 4 ? grouped_down_kernel<BITS, NG, 4>
            : c.tl == 2 ? grouped_down_kernel<BITS, NG, 2>
                        : grouped_down_kernel<BITS, NG, 1>;
   if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
-  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m[0], m[1]);
+  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m);
   return cudaGetLastError();
 }
 
@@ -1080,8 +1092,6 @@ cudaError_t gateup_bits_g(const GroupedParams& p, cudaStream_t s) {
   const TcConfig c = gu_config(BITS, p.H);
   if (c.tl == 0 || p.I % (8 * c.tl)) return cudaErrorInvalidValue;
   switch (p.H / kGroup) {
-    case 2: return gateup_ng<BITS, 2>(p, c, s);
-    case 4: return gateup_ng<BITS, 4>(p, c, s);
     case 8: return gateup_ng<BITS, 8>(p, c, s);
     case 16: return gateup_ng<BITS, 16>(p, c, s);
     case 32: return gateup_ng<BITS, 32>(p, c, s);
@@ -1096,8 +1106,6 @@ cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
   const TcConfig c = dn_config(BITS, p.I);
   if (c.tl == 0 || p.H % (16 * c.tl)) return cudaErrorInvalidValue;
   switch (p.I / kGroup) {
-    case 2: return down_ng<BITS, 2>(p, c, s);
-    case 4: return down_ng<BITS, 4>(p, c, s);
     case 8: return down_ng<BITS, 8>(p, c, s);
     case 16: return down_ng<BITS, 16>(p, c, s);
     case 32: return down_ng<BITS, 32>(p, c, s);
@@ -1110,8 +1118,8 @@ cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
 }  // namespace
 
 bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T) {
+  if (H < 512 || I < 512) return false;  // scale rows of at least 16 bytes (one tensor-copy line)
   if (T * K > kMaxTK || ((size_t)T * K + 2 * (size_t)E) * 4 > 200 * 1024) return false;
-  if ((size_t)kRtRows * H * 2 > 200 * 1024) return false;
   const TcConfig gu = gu_config(bits, H), dn = dn_config(bits, I);
   return gu.tl > 0 && I % (8 * gu.tl) == 0 && dn.tl > 0 && H % (16 * dn.tl) == 0;
 }
@@ -1126,15 +1134,21 @@ cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+int grouped_router_split(int H, int E, int T) {
+  const int blocks = ((E + 1 + kRtR - 1) / kRtR) * ((T + kRtT - 1) / kRtT);
+  int n = 1;
+  while (n < 16 && blocks * n * 2 <= 148 && H % (2 * n * 64) == 0) n *= 2;
+  return n;
+}
+
 cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s) {
   norm_digits_kernel<<<p.T, kGT, 0, s>>>(p, rb, bits);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int R = p.E + 1;
-  const size_t smem = (size_t)kRtRows * p.H * 2;
+  const size_t smem = (size_t)kRtR * (kRtK + 8) * 2 + (size_t)kRtT * (kRtK + 4) * 4;
   void (*k)(const GroupedParams, const RouterBatch) = router_gemm_kernel;
   if ((e = set_smem((const void*)k, smem)) != cudaSuccess) return e;
-  k<<<dim3((R + kRtRows - 1) / kRtRows, (p.T + kRtTok - 1) / kRtTok), kGT, smem, s>>>(p, rb);
+  k<<<dim3((p.E + 1 + kRtR - 1) / kRtR, (p.T + kRtT - 1) / kRtT, p.rt_split), kGT, smem, s>>>(p, rb);
   return cudaGetLastError();
 }
 

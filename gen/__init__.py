@@ -106,6 +106,12 @@ def tiny_layer(bits=4):
     return LayerSpec(hidden=256, experts=8, inter=128, top_k=2, bits=bits, router_std=1.0 / math.sqrt(256))
 
 
+def small_layer(bits=4, experts=16, top_k=4):
+    """Small layer for batched-path tests: hidden 512, intermediate 512 (8 groups of 64 per row)."""
+    return LayerSpec(hidden=512, experts=experts, inter=512, top_k=top_k, bits=bits,
+                     router_std=1.0 / math.sqrt(512))
+
+
 def qwen397_layer(bits=4, zipf=0.0):
     """Qwen3.5-397B-A17B-shaped MoE layer: hidden 4096, 512 experts of intermediate 1024, top-4 + shared."""
     return LayerSpec(hidden=4096, experts=512, inter=1024, top_k=4, bits=bits, zipf=zipf)

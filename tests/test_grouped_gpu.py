@@ -21,9 +21,9 @@ def fmoe():
 
 
 @pytest.mark.parametrize("bits", [4, 2])
-def test_grouped_tiny_batch_matches_oracle(fmoe, bits):
-    # 64 tokens over 8 experts: every expert's group is large (many digit batches per CTA)
-    spec = gen.LayerSpec(**{**gen.tiny_layer(bits).__dict__, "random_gamma": True})
+def test_grouped_small_batch_matches_oracle(fmoe, bits):
+    # 64 tokens over 16 experts: every expert's group spans many work units
+    spec = gen.LayerSpec(**{**gen.small_layer(bits).__dict__, "random_gamma": True})
     hl = gen.host_layer(spec, seed=12)
     dl = gen.upload_layer(hl)
     h = gen.host_tokens(700, 64, spec.hidden)
@@ -32,14 +32,25 @@ def test_grouped_tiny_batch_matches_oracle(fmoe, bits):
     assert exact >= 60
 
 
-def test_grouped_tiny_batch_top1_all_experts_and_odd_size(fmoe):
-    spec = gen.tiny_layer(4)
+def test_grouped_small_batch_top1_all_experts_and_odd_size(fmoe):
+    spec = gen.small_layer(4, experts=8, top_k=2)
     hl = gen.host_layer(spec, seed=13)
     dl = gen.upload_layer(hl)
     for top_k, T in ((1, 9), (8, 23)):
         h = gen.host_tokens(900 + T, T, spec.hidden)
         out, idx, w = _run_layer(fmoe, dl, h, top_k=top_k)
         _compare_layer(hl, h, out, idx, w, L=oracle_layer(hl, top_k=top_k))
+
+
+def test_tiny_layer_batch_takes_the_per_token_path(fmoe):
+    # hidden 256: scale rows of 8 bytes are below the batched path's staging line, so the
+    # call falls back to the per-token kernels; the result must not change
+    spec = gen.tiny_layer(4)
+    hl = gen.host_layer(spec, seed=15)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(1100, 12, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    _compare_layer(hl, h, out, idx, w)
 
 
 def test_per_token_path_still_matches_oracle(fmoe, monkeypatch):
