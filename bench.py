@@ -30,6 +30,12 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gate/up launch,
 # from one ncu capture of the current gateup_kernel per workload; None where none was taken.
 GATEUP_TRAFFIC = {"qwen397-4bit": 31243264}
+# grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
+# (+ the shared expert): 1,050,211,840 B over 207.5 experts
+GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5061262}
+DTYPE_TOKEN = "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32"
+DTYPE_BATCH = "i32 mma.sync (u4/u2 codes as u8 x 24-bit fixed-point x as three s8 limbs) + f32"
+BATCH_KERNELS = 8  # norm+digits, router GEMM, top-K, sort, gate/up, activation digits, down, combine
 
 WORKLOADS = {
     # name: (spec factory, description)
@@ -289,8 +295,9 @@ def main():
         n_active = float(np.mean(act))
 
     # ---- per-kernel durations: a separate replay with trace events around each kernel
-    # (the three-kernel per-token path; the batched path has no per-kernel trace)
-    tr = 0 if nbatch else min(G, 500)
+    # (per-token path: router, gate/up, down; batched path: router + selection, gate/up,
+    # activation digits + down + combine)
+    tr = min(G, 500)
     router_us = gateup_us = down_us = None
     if tr:
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(tr)]
@@ -350,13 +357,12 @@ def main():
     peak, peak_kind = peak_hbm()
     rec_mat = spec.inter * spec.hidden * spec.bits // 8 + 2 * spec.inter * (spec.hidden // spec.group) * 2
     if nbatch:
-        # a step moves the active experts' records, the shared expert's and the router, once each
-        rec = gen.record_bytes(spec)
+        # a step moves the active experts' records, the shared expert's and the router, once each;
+        # the dominant kernel is the grouped gate/up (gate and up of the active + shared experts)
         step_bytes = (n_active + 1) * 3 * rec_mat + spec.experts * spec.hidden * 2
         bytes_tok = step_bytes / nb
-        kernel, kbytes = "batched step (all kernels)", step_bytes
-        achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
-        del rec
+        kernel, kbytes = "grouped_gateup_kernel", (n_active + 1) * 2 * rec_mat
+        achieved = kbytes / (gateup_us * 1e-6) / 1e9 if gateup_us else step_bytes / (ms_per_step * 1e-3) / 1e9
     else:
         kernel, kbytes = "gateup_kernel", (spec.top_k + 1) * 2 * rec_mat
         achieved = kbytes / (gateup_us * 1e-6) / 1e9
@@ -373,7 +379,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": DTYPE_BATCH if nbatch else DTYPE_TOKEN, "data": "synthetic",
             "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
                        "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": nb,
                        "active_experts_per_step": n_active,
@@ -386,10 +392,13 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "effective_gbs": eff, "frac_of_peak": eff / peak, "bytes_per_token": bytes_tok,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": GATEUP_TRAFFIC.get(args.workload), "kernel": kernel, "peak_kind": peak_kind,
+                         "traffic": (GROUPED_GATEUP_TRAFFIC_PER_EXPERT[args.workload] * (n_active + 1)
+                                     if nbatch and args.workload in GROUPED_GATEUP_TRAFFIC_PER_EXPERT
+                                     else GATEUP_TRAFFIC.get(args.workload)),
+                         "kernel": kernel, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": kbytes},
             "kernels_us": {"router": router_us, "gateup": gateup_us, "down": down_us},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (6 * steps if nbatch else 3 * steps * per_step),
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (BATCH_KERNELS * steps if nbatch else 3 * steps * per_step),
             "clocks": clk.record(),
         }
         print(json.dumps(line), flush=True)

@@ -194,7 +194,10 @@ fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int L, const float* h, int 
  * this host thread records the caller's CUDA events (cudaEvent_t handles) on
  * its stream: events[0] before the router kernel, events[1] after it,
  * events[2] after the gate/up kernel, events[3] after the down/combine kernel
- * (first token only when T > 1).  n must be 4; events = NULL cancels. */
+ * (first token only when T > 1).  On the expert-grouped path (T >= 8) the
+ * events bracket the whole batch: [0] before the router, [1] after the
+ * selection and sort, [2] after the grouped gate/up kernel, [3] after the
+ * combine.  n must be 4; events = NULL cancels. */
 fmoe_status fmoe_trace_next_layer(void* const* events, int n);
 
 /* Zeroes the workspace's control words (enqueued on `stream`).  Call once after
