@@ -57,6 +57,13 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
                : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// d = a * b + c with c a separate (unchanged) input, e.g. a constant start value.
+__device__ __forceinline__ void mma_u8s8_c(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, int c) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c));
+}
+
 // Quantises one group of 64 values (lane l holds columns 2l, 2l+1) into the
 // layout above: the same fixed-point digits as the per-token format (cscale =
 // 2^(e-22) from the group's largest magnitude), only placed differently.
@@ -578,13 +585,12 @@ template <int BITS>
 __device__ __forceinline__ void tc_tile_group(const uint32_t (&w)[2][2], const uint2 (&b)[2], const TcColScale& cs,
                                               float s_lo, float s_hi, float b_lo, float b_hi, float (&acc)[4],
                                               float (&accb)[2]) {
-  int c[4] = {kMagicBits, kMagicBits, kMagicBits, kMagicBits};
-#pragma unroll
-  for (int kb = 0; kb < 2; ++kb) {
-    uint32_t a[4];
-    tc_unpack_a<BITS>(w, kb, a);
-    mma_u8s8(c, a, b[kb].x, b[kb].y);
-  }
+  int c[4];
+  uint32_t a[4];
+  tc_unpack_a<BITS>(w, 0, a);
+  mma_u8s8_c(c, a, b[0].x, b[0].y, kMagicBits);  // starts from the biased accumulator
+  tc_unpack_a<BITS>(w, 1, a);
+  mma_u8s8(c, a, b[1].x, b[1].y);
   acc[0] = fmaf(s_lo, fmaf(__int_as_float(c[0]), cs.sa, cs.na), acc[0]);
   acc[1] = fmaf(s_lo, fmaf(__int_as_float(c[1]), cs.sb, cs.nb), acc[1]);
   acc[2] = fmaf(s_hi, fmaf(__int_as_float(c[2]), cs.sa, cs.na), acc[2]);
@@ -610,6 +616,23 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
   const int bt = gid < 6 ? gid / 3 : 0, bl = gid % 3;  // this lane's B column: token slot, limb
   const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
   const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);  // [token][NG + 2] (padded pitch)
+  // A addresses.  With 128-byte lines and g0 a multiple of the groups per line
+  // (4 at 4-bit, 8 at 2-bit), a lane's rows all have row % 8 == gid, so the
+  // swizzled byte of group g is row*128 + (g / PER)*ROWS*128 + vx[g % PER], with
+  // vx a lane constant: one add per load.  Otherwise the general formula (Sw).
+  using SA = TcSw<BITS, NG, ROWS>;
+  constexpr int PER = BITS == 4 ? 4 : 8;  // groups per 128-byte line
+  constexpr bool FAST = SA::LW == 128 && GPW % PER == 0;
+  uint32_t vx[PER];
+#pragma unroll
+  for (int m = 0; m < PER; ++m) vx[m] = (uint32_t)((BITS == 4 ? (m << 5) | (8 * q) : (m << 4) | (4 * q)) ^ (gid << 4));
+  const uint8_t* blo[TPW];
+  const uint8_t* bhi[TPW];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    blo[i] = buf_lo + (size_t)rlo[i] * 128 + (size_t)(g0 / PER) * ROWS * 128;
+    bhi[i] = buf_hi + (size_t)rhi[i] * 128 + (size_t)(g0 / PER) * ROWS * 128;
+  }
   float accb[TPW][2];
 #pragma unroll
   for (int i = 0; i < TPW; ++i) accb[i][0] = accb[i][1] = 0.0f;
@@ -633,7 +656,21 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
 #pragma unroll
       for (int i = 0; i < TPW; ++i) {
         uint32_t w[2][2];
-        tc_load_a<BITS, NG, ROWS>(buf_lo, rlo[i], buf_hi, rhi[i], g, q, w);
+        if constexpr (FAST) {
+          const int gg = gc + gi;  // compile-time after unrolling
+          const size_t off = (size_t)(gg / PER) * ROWS * 128;
+          if (BITS == 4) {
+            const uint2 x = *reinterpret_cast<const uint2*>(blo[i] + off + vx[gg % PER]);
+            const uint2 y = *reinterpret_cast<const uint2*>(bhi[i] + off + vx[gg % PER]);
+            w[0][0] = x.x; w[0][1] = x.y; w[1][0] = y.x; w[1][1] = y.y;
+          } else {
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(blo[i] + off + vx[gg % PER]);
+            const uint32_t y = *reinterpret_cast<const uint32_t*>(bhi[i] + off + vx[gg % PER]);
+            w[0][0] = w[0][1] = x; w[1][0] = w[1][1] = y;
+          }
+        } else {
+          tc_load_a<BITS, NG, ROWS>(buf_lo, rlo[i], buf_hi, rhi[i], g, q, w);
+        }
         tc_tile_group<BITS>(w, b, cs, tc_scale<GPC>(sv[i][0], gi), tc_scale<GPC>(sv[i][2], gi),
                             tc_scale<GPC>(sv[i][1], gi), tc_scale<GPC>(sv[i][3], gi), acc[i], accb[i]);
       }
