@@ -142,7 +142,11 @@ size_t fmoe_expert_ffn_workspace_size(const fmoe_bank* bank);
  * topk_idx (int32 [T][K]) and topk_w (fp32 [T][K]) receive the routing, or NULL.
  * ws: fmoe_moe_layer_workspace_size(layer, T) bytes, 256-byte aligned, zeroed
  * once before first use (fmoe_workspace_init); calls on one workspace must be
- * ordered on one stream.  Requirements: those of fmoe_expert_ffn for both
+ * ordered on one stream.  T >= 8 tokens run expert-grouped (each active
+ * expert's rows read once for its token group) when the workspace holds the
+ * T-token size, hidden and inter are >= 512 and FMOE_GROUPED is not "0";
+ * otherwise token by token, for which the T = 1 size suffices (a smaller
+ * workspace gives FMOE_ERR_WORKSPACE).  Requirements: those of fmoe_expert_ffn for both
  * banks (same bits, hidden, inter), 1 <= K <= min(E, 32), E <= 4096,
  * hidden <= 8192, and K + 1 expert slots of the down kernel within its shared
  * memory (K <= 9 at inter 1024, 4-bit; FMOE_ERR_UNSUPPORTED otherwise).

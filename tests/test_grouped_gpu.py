@@ -42,6 +42,54 @@ def test_grouped_small_batch_top1_all_experts_and_odd_size(fmoe):
         _compare_layer(hl, h, out, idx, w, L=oracle_layer(hl, top_k=top_k))
 
 
+def test_grouped_many_token_tiles_and_repeated_calls(fmoe):
+    """200 tokens: the router's grid spans four token tiles, the sort 800 pairs; a second
+    call on the same workspace (tickets, counters and slots reused) gives the same bytes."""
+    spec = gen.LayerSpec(**{**gen.small_layer(4, experts=16, top_k=4).__dict__, "random_gamma": True})
+    hl = gen.host_layer(spec, seed=16)
+    dl = gen.upload_layer(hl)
+    lay = gen.binding_layer(dl)
+    T, K = 200, spec.top_k
+    h_np = gen.host_tokens(1300, T, spec.hidden)
+    h = torch.from_numpy(h_np).cuda()
+    ws = fmoe.workspace(fmoe.moe_layer_workspace_size(lay, T))
+    outs = []
+    for _ in range(2):
+        out = torch.empty_like(h)
+        idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+        fmoe.moe_layer(lay, h, out=out, topk_idx=idx, topk_w=w, ws=ws)
+        outs.append((out, idx, w))
+    fmoe.workspace_check(ws)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    out, idx, w = (x.cpu().numpy() for x in outs[0])
+    _compare_layer(hl, h_np, out.astype(np.float64), idx, w.astype(np.float64))
+
+
+def test_small_workspace_falls_back_to_the_per_token_path(fmoe):
+    """A workspace sized for one token cannot hold the grouped path's regions: a 16-token
+    call then runs token by token and must give the oracle's results."""
+    spec = gen.small_layer(2)
+    hl = gen.host_layer(spec, seed=17)
+    dl = gen.upload_layer(hl)
+    lay = gen.binding_layer(dl)
+    T, K = 16, spec.top_k
+    h_np = gen.host_tokens(1500, T, spec.hidden)
+    h = torch.from_numpy(h_np).cuda()
+    small = fmoe.moe_layer_workspace_size(lay, 1)
+    assert small < fmoe.moe_layer_workspace_size(lay, T)
+    ws = fmoe.workspace(small)
+    out = torch.empty_like(h)
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    fmoe.moe_layer(lay, h, out=out, topk_idx=idx, topk_w=w, ws=ws)
+    fmoe.workspace_check(ws)
+    torch.cuda.synchronize()
+    _compare_layer(hl, h_np, out.cpu().numpy().astype(np.float64), idx.cpu().numpy(),
+                   w.cpu().numpy().astype(np.float64))
+
+
 def test_tiny_layer_batch_takes_the_per_token_path(fmoe):
     # hidden 256: scale rows of 8 bytes are below the batched path's staging line, so the
     # call falls back to the per-token kernels; the result must not change
