@@ -329,11 +329,38 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
   const int slot_bytes = crows * (RB + 2 * SB);  // one expert's rows of a chunk
   const int chb = (NE * slot_bytes + 127) / 128 * 128;
 
-  // The routing is written by CTA 0 of the gate/up kernel: read it after the wait.
+  // The shared expert's rows are weights: thread 0 requests them for the first
+  // chunks before the wait.  The routing is written by CTA 0 of the gate/up
+  // kernel: it is read, and the routed rows requested, after the wait.
+  if (tid == 0 && p.has_shared) {
+    s_src[p.K][0] = p.shared.base + p.shared.off[6];
+    s_src[p.K][1] = p.shared.base + p.shared.off[7];
+    s_src[p.K][2] = p.shared.base + p.shared.off[8];
+  }
+  // chunk c, slots [s0, s1): units [u0 + c*chunk_units, ..) of each slot (thread 0);
+  // `expect` arms the chunk's barrier for all NE slots
+  auto issue = [&](int c, int s0, int s1, bool expect) {
+    const int cu = u0 + c * chunk_units, ce = min(cu + chunk_units, u1);
+    const long long j0 = (long long)cu * RD;
+    const uint32_t rows = (uint32_t)(ce - cu) * RD;
+    uint8_t* buf = sm + head + (size_t)(c % nbuf) * chb;
+    const uint32_t bar = smem_addr(&s_bar[c % nbuf]);
+    const uint64_t pol_r = l2_policy_evict_first(), pol_s = l2_policy_evict_last();
+    if (expect) mbar_expect_tx(bar, (uint32_t)NE * rows * (RB + 2 * SB));
+    for (int s = s0; s < s1; ++s) {
+      const uint64_t pol = s < p.K ? pol_r : pol_s;
+      const uint32_t d = smem_addr(buf + (size_t)s * slot_bytes);
+      bulk_g2s(d, s_src[s][0] + j0 * RB, rows * RB, bar, pol);
+      bulk_g2s(d + crows * RB, s_src[s][1] + j0 * SB, rows * SB, bar, pol);
+      bulk_g2s(d + crows * RB + crows * SB, s_src[s][2] + j0 * SB, rows * SB, bar, pol);
+    }
+  };
+  const int nchunk = (u1 - u0 + chunk_units - 1) / chunk_units;
   if (tid == 0) {
     for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&s_bar[b]), 1);
     mbar_init(smem_addr(&s_bar_x), 1);
     mbar_fence_init();
+    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c, p.K, NE, true);  // the shared slot (if any)
   }
   pdl_wait();  // the activations' digits and the routing are complete
   pdl_trigger();
@@ -350,38 +377,16 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
       s_src[lane][2] = rec + p.routed.off[8];
       s_w[lane] = p.route_w ? __ldcg(p.route_w + lane) : 1.0f;
     }
-    if (lane == 0 && p.has_shared) {
-      s_src[p.K][0] = p.shared.base + p.shared.off[6];
-      s_src[p.K][1] = p.shared.base + p.shared.off[7];
-      s_src[p.K][2] = p.shared.base + p.shared.off[8];
-      s_w[p.K] = p.route_w ? __ldcg(p.route_w + p.K) : 1.0f;
-    }
+    if (lane == 0 && p.has_shared) s_w[p.K] = p.route_w ? __ldcg(p.route_w + p.K) : 1.0f;
   }
   __syncthreads();
 
-  auto issue = [&](int c) {  // chunk c: units [u0 + c*chunk_units, ..) of every slot, thread 0
-    const int cu = u0 + c * chunk_units, ce = min(cu + chunk_units, u1);
-    const long long j0 = (long long)cu * RD;
-    const uint32_t rows = (uint32_t)(ce - cu) * RD;
-    uint8_t* buf = sm + head + (size_t)(c % nbuf) * chb;
-    const uint32_t bar = smem_addr(&s_bar[c % nbuf]);
-    const uint64_t pol_r = l2_policy_evict_first(), pol_s = l2_policy_evict_last();
-    mbar_expect_tx(bar, (uint32_t)NE * rows * (RB + 2 * SB));
-    for (int s = 0; s < NE; ++s) {
-      const uint64_t pol = s < p.K ? pol_r : pol_s;
-      const uint32_t d = smem_addr(buf + (size_t)s * slot_bytes);
-      bulk_g2s(d, s_src[s][0] + j0 * RB, rows * RB, bar, pol);
-      bulk_g2s(d + crows * RB, s_src[s][1] + j0 * SB, rows * SB, bar, pol);
-      bulk_g2s(d + crows * RB + crows * SB, s_src[s][2] + j0 * SB, rows * SB, bar, pol);
-    }
-  };
-  const int nchunk = (u1 - u0 + chunk_units - 1) / chunk_units;
-  if (tid == 0) {  // every slot's digits, once per CTA; then the first chunks (mostly from L2)
+  if (tid == 0) {  // every slot's digits, once per CTA; then the routed rows of the first chunks (mostly from L2)
     const uint32_t bx = smem_addr(&s_bar_x);
     mbar_expect_tx(bx, (uint32_t)(dwords * 4 + NE * NCH * 8));
     bulk_g2s(smem_addr(sm), p.act_limbs, (uint32_t)dwords * 4, bx, l2_policy_evict_first());
     bulk_g2s(smem_addr(sm + (size_t)dwords * 4), p.act_cs, (uint32_t)(NE * NCH * 8), bx, l2_policy_evict_first());
-    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c);
+    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c, 0, p.K, false);
   }
   __syncwarp();  // lanes 1..31 of warp 0 wait for the issue instead of spinning beside it
 
@@ -438,7 +443,7 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
     __syncthreads();  // every warp is done with this chunk buffer
     if (tid == 0 && c + nbuf < nchunk && ok) {
       fence_proxy_async();
-      issue(c + nbuf);
+      issue(c + nbuf, 0, NE, true);
     }
   }
   if (!ok && tid == 0)

@@ -88,6 +88,15 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
       if (gate_row) bulk_g2s(smem_addr(wrows + (size_t)nr * H), p.w_sgate, (uint32_t)H * 2, bar, l2_policy_evict_last());
     }
   }
+  // gamma is a weight: read it (this thread's float4s, H <= 8192) before the wait
+  constexpr int kGv = 8192 / (kRouterThreads * 4);
+  float4 gv[kGv];
+#pragma unroll
+  for (int j = 0; j < kGv; ++j) {
+    const int i = (tid + j * kRouterThreads) * 4;
+    gv[j] = (p.norm && p.gamma && i < H) ? __ldg(reinterpret_cast<const float4*>(p.gamma + i))
+                                         : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+  }
   pdl_wait();
   pdl_trigger();
 
@@ -105,12 +114,15 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
   if (p.norm) {
     ss = block_sum_256(ss, s_red);
     const float rstd = 1.0f / sqrtf(ss / (float)H + p.eps);
-#pragma unroll 4
-    for (int i = tid * 4; i < H; i += kRouterThreads * 4) {
-      float4 v = *reinterpret_cast<const float4*>(xs + i);
-      const float4 g = p.gamma ? __ldg(reinterpret_cast<const float4*>(p.gamma + i)) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-      v = make_float4(v.x * rstd * g.x, v.y * rstd * g.y, v.z * rstd * g.z, v.w * rstd * g.w);
-      *reinterpret_cast<float4*>(xs + i) = v;
+#pragma unroll
+    for (int j = 0; j < kGv; ++j) {
+      const int i = (tid + j * kRouterThreads) * 4;
+      if (i < H) {
+        float4 v = *reinterpret_cast<const float4*>(xs + i);
+        const float4 g = gv[j];
+        v = make_float4(v.x * rstd * g.x, v.y * rstd * g.y, v.z * rstd * g.z, v.w * rstd * g.w);
+        *reinterpret_cast<float4*>(xs + i) = v;
+      }
     }
   }
   __syncthreads();
