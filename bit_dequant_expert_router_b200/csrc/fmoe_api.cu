@@ -394,6 +394,7 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   rp.logits = reinterpret_cast<float*>(base + L.logits);
   rp.top_k = 0;  // the expert kernels select the experts from the logits themselves
   rp.tickets = ctrl->tickets;
+  rp.route_ready = &ctrl->route_ready;
   rp.err = err_word ? err_word : &ctrl->err;
   const bool trace = g_trace_on;
   g_trace_on = false;
@@ -427,6 +428,7 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   p.err = rp.err;
   p.rt_idx = reinterpret_cast<int32_t*>(base + L.route_idx);
   p.rt_w = reinterpret_cast<float*>(base + L.route_w);
+  p.route_ready = &ctrl->route_ready;  // gate/up CTA 0 sets it once rt_idx / rt_w are written
   if ((e = launch_gateup(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
   if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   ExpertParams pd = p;  // the down kernel reads the routing the gate/up kernel wrote

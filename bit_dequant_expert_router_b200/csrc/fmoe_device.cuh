@@ -18,7 +18,8 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // bound on any device-si
 struct WsControl {
   unsigned int tickets[992];   // last-CTA tickets, one per token
   unsigned int epoch;          // single-kernel path: steps run on this workspace (its own 128-byte line)
-  unsigned int pad0[31];
+  unsigned int route_ready;    // three-kernel path: 1 once the gate/up kernel has published this token's routing
+  unsigned int pad0[30];
   int err;                     // nonzero once a bounded wait gave up
   int pad[63];
 };
@@ -26,6 +27,16 @@ struct WsControl {
 // ------------------------------------------------------------------------------------------ small helpers
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 

@@ -31,6 +31,7 @@ struct RouterParams {
   int32_t* idx_out;           // optional user copies [T][K]
   float* w_out;
   unsigned int* tickets;      // [T], zero between calls
+  unsigned int* route_ready;  // or NULL: cleared once the predecessor is complete (see ExpertParams)
   int* err;
 };
 
@@ -68,6 +69,9 @@ struct ExpertParams {
   const float* resid;         // down: residual [H] or NULL
   float* out;                 // down: [H]
   int prefetch_down;          // gate/up asks L2 for the routed experts' down matrices
+  unsigned int* route_ready;  // or NULL.  Gate/up CTA 0 sets it (release) after writing rt_idx / rt_w;
+                              // the down kernel, seeing it set (acquire), reads the routing and requests
+                              // the routed rows before its dependency wait; the next router clears it
   int* err;
 };
 

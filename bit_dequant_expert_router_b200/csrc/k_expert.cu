@@ -143,6 +143,15 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     }
     if (p.rt_w) p.rt_w[tid] = s_wt[tid];
   }
+  if (p.logits && p.route_ready && blockIdx.x == 0) {
+    // publish it: lane 1 of warp 1 has no copies in flight, so its release does not
+    // wait for any (a gpu-scope release waits for the issuing thread's own bulk copies)
+    __syncthreads();
+    if (tid == 33) {
+      __threadfence();
+      st_release_gpu(p.route_ready, 1u);
+    }
+  }
   if (lane == 0) {
     // x digits by warp 0; the first routed chunks one per warp (lane 0), so that
     // their copies go out from several warps at once; the L2 warm-up by warp 7
@@ -356,15 +365,15 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
     }
   };
   const int nchunk = (u1 - u0 + chunk_units - 1) / chunk_units;
+  __shared__ int s_early;
   if (tid == 0) {
     for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&s_bar[b]), 1);
     mbar_init(smem_addr(&s_bar_x), 1);
     mbar_fence_init();
     for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c, p.K, NE, true);  // the shared slot (if any)
   }
-  pdl_wait();  // the activations' digits and the routing are complete
-  pdl_trigger();
-  if (warp == 0) {
+  // the routing, from the slots the gate/up kernel wrote (or given)
+  auto read_routing = [&]() {  // warp 1
     if (lane < p.K) {
       int ik = p.route_idx ? __ldcg(p.route_idx + lane) : p.fixed_expert;
       if (ik < 0 || ik >= p.routed.num_experts) {
@@ -378,16 +387,38 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
       s_w[lane] = p.route_w ? __ldcg(p.route_w + lane) : 1.0f;
     }
     if (lane == 0 && p.has_shared) s_w[p.K] = p.route_w ? __ldcg(p.route_w + p.K) : 1.0f;
+  };
+  // Published already (gate/up CTA 0 finished its selection long before this grid
+  // starts, in practice)?  Warp 1 has no copies in flight, so its acquire does not wait.
+  if (warp == 1) {  // every lane acquires, so that its own reads of the routing follow
+    const bool seen = p.route_ready && ld_acquire_gpu(p.route_ready) == 1u;
+    const bool early = __all_sync(0xffffffffu, seen);
+    if (early) read_routing();
+    if (lane == 0) s_early = early ? 1 : 0;
   }
   __syncthreads();
+  const bool early = s_early != 0;
+  // the routed rows of the first chunks (mostly from L2; their barriers are armed): one
+  // (chunk, slot) per issuing lane, lane 0 of warps 1.., so that the requests go out side by side
+  auto issue_routed = [&]() {
+    if (lane == 0 && warp > 0)
+      for (int cs = warp - 1; cs < min(nbuf, nchunk) * p.K; cs += kDnWarps - 1) issue(cs / p.K, cs % p.K, cs % p.K + 1, false);
+  };
+  if (early) issue_routed();
+  pdl_wait();  // the activations' digits (and the routing) are complete
+  pdl_trigger();
+  if (!early) {
+    if (warp == 1) read_routing();
+    __syncthreads();
+  }
 
-  if (tid == 0) {  // every slot's digits, once per CTA; then the routed rows of the first chunks (mostly from L2)
+  if (tid == 0) {  // every slot's digits, once per CTA
     const uint32_t bx = smem_addr(&s_bar_x);
     mbar_expect_tx(bx, (uint32_t)(dwords * 4 + NE * NCH * 8));
     bulk_g2s(smem_addr(sm), p.act_limbs, (uint32_t)dwords * 4, bx, l2_policy_evict_first());
     bulk_g2s(smem_addr(sm + (size_t)dwords * 4), p.act_cs, (uint32_t)(NE * NCH * 8), bx, l2_policy_evict_first());
-    for (int c = 0; c < nbuf && c < nchunk; ++c) issue(c, 0, p.K, false);
   }
+  if (!early) issue_routed();
   __syncwarp();  // lanes 1..31 of warp 0 wait for the issue instead of spinning beside it
 
   // This lane's (slot, group) pairs and their digits.

@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
   }
   pdl_wait();
   pdl_trigger();
+  // every kernel of the previous token is complete: its routing flag is spent
+  if (p.route_ready && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *p.route_ready = 0u;
 
   const float* h = p.h + (size_t)t * H;
   float ss = 0.0f;
