@@ -1034,14 +1034,15 @@ TcConfig gu_config(int bits, int H) {
   return TcConfig{0, 0, 0};
 }
 
-// down: 64, 32 or 16 rows per item (TL 4, 2, 1), the first with at least 3 stages (<= 8).
+// down: 128 rows per item (TL 8) with at least 2 stages, else 64, 32 or 16 rows
+// (TL 4, 2, 1) with at least 3; at most 8 stages.
 TcConfig dn_config(int bits, int I) {
   const int NG = I / kGroup, RB = I * bits / 8, SB = NG * 2;
-  for (int tl : {4, 2, 1}) {
+  for (int tl : {8, 4, 2, 1}) {
     const int rows = 16 * tl, ks = kConsumers * (tl < 2 ? tl : 2) / tl;
     const size_t wb = round_kib((size_t)rows * RB) + 2 * round_kib((size_t)rows * SB);
     const size_t tp = (size_t)ks * (rows * 8 + 4);
-    for (int n = 8; n >= 3; --n) {
+    for (int n = 8; n >= (tl == 8 ? 2 : 3); --n) {
       const size_t sm = tc_smem(n, wb, NG, tp);
       if (sm <= kSmemBudget) return TcConfig{tl, n, sm};
     }
@@ -1116,7 +1117,8 @@ cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
   static constexpr int subs[3] = {6, 7, 8};  // rows, s, b
   cudaError_t e = encode_maps(m, p, subs, true, p.H, p.I * BITS / 8, NG, 16 * c.tl);
   if (e != cudaSuccess) return e;
-  auto k = c.tl == 4 ? grouped_down_kernel<BITS, NG, 4>
+  auto k = c.tl == 8   ? grouped_down_kernel<BITS, NG, 8>
+           : c.tl == 4 ? grouped_down_kernel<BITS, NG, 4>
            : c.tl == 2 ? grouped_down_kernel<BITS, NG, 2>
                        : grouped_down_kernel<BITS, NG, 1>;
   if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
