@@ -223,8 +223,13 @@ __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) 
   __syncthreads();
   for (int i = tid; i < N; i += kST) {
     const int e = s_e[i];
-    int rank = 0;
-    for (int j = 0; j < i; ++j) rank += s_e[j] == e;
+    int rank = 0, j = 0;
+#pragma unroll 4
+    for (; j + 4 <= i; j += 4) {
+      const int4 v = *reinterpret_cast<const int4*>(s_e + j);
+      rank += (v.x == e) + (v.y == e) + (v.z == e) + (v.w == e);
+    }
+    for (; j < i; ++j) rank += s_e[j] == e;
     const int pos = s_start[e] + rank;
     p.pair_tok[pos] = i;
     p.pair_pos[i] = pos;
@@ -238,20 +243,24 @@ __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) 
   }
 }
 
-// ---- router for the batch.  norm_digits: one CTA per token, x = RMSNorm(h)
-// (two passes) in fp32 for the router and as digits for the experts.
+// ---- router for the batch.  norm_digits: x = RMSNorm(h) in fp32 for the
+// router and as digits for the experts.  CTA (c, t) takes groups
+// [c*NG/kNormSplit, (c+1)*NG/kNormSplit) of token t, one warp per group; every
+// CTA of the token sums the squares of the whole row (the same order in each).
+constexpr int kNormSplit = 4;
+
 __global__ void __launch_bounds__(kGT) norm_digits_kernel(const GroupedParams p, const RouterBatch rb, int bits) {
   __shared__ float s_red[kGT / 32];
-  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, H = p.H;
+  const int t = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, H = p.H, NG = H / kGroup;
   const float* h = p.h + (size_t)t * H;
   float* x = rb.x + (size_t)t * H;
-  float ss = 0.0f;
-  for (int i = tid * 4; i < H; i += kGT * 4) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(h + i));
-    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-  }
   float rstd = 1.0f;
   if (rb.gamma) {
+    float ss = 0.0f;
+    for (int i = tid * 4; i < H; i += kGT * 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(h + i));
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
     ss = warp_sum(ss);
     if (lane == 0) s_red[warp] = ss;
     __syncthreads();
@@ -260,20 +269,17 @@ __global__ void __launch_bounds__(kGT) norm_digits_kernel(const GroupedParams p,
     for (int w = 0; w < kGT / 32; ++w) tot += s_red[w];
     rstd = 1.0f / sqrtf(tot / (float)H + rb.eps);
   }
-  for (int i = tid * 4; i < H; i += kGT * 4) {
-    float4 v = __ldcg(reinterpret_cast<const float4*>(h + i));
-    if (rb.gamma) {
-      const float4 g = __ldg(reinterpret_cast<const float4*>(rb.gamma + i));
-      v = make_float4(v.x * rstd * g.x, v.y * rstd * g.y, v.z * rstd * g.z, v.w * rstd * g.w);
-    }
-    *reinterpret_cast<float4*>(x + i) = v;
-  }
-  __syncthreads();  // this CTA's x is written (read back through L1-bypassing loads below)
-  __threadfence_block();
+  const int per = (NG + kNormSplit - 1) / kNormSplit, ge = min(NG, (int)(blockIdx.x + 1) * per);
   uint8_t* limbs = const_cast<uint8_t*>(p.xq_limbs) + (size_t)t * 3 * H;
-  float2* cs = const_cast<float2*>(p.xq_cs) + (size_t)t * (H / kGroup);
-  for (int g = warp; g < H / kGroup; g += kGT / 32) {
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(x + g * kGroup) + lane);
+  float2* cs = const_cast<float2*>(p.xq_cs) + (size_t)t * NG;
+  for (int g = blockIdx.x * per + warp; g < ge; g += kGT / 32) {
+    const int i = g * kGroup + 2 * lane;
+    float2 v = __ldcg(reinterpret_cast<const float2*>(h + i));
+    if (rb.gamma) {
+      const float2 gm = __ldg(reinterpret_cast<const float2*>(rb.gamma + i));
+      v = make_float2(v.x * rstd * gm.x, v.y * rstd * gm.y);
+    }
+    *reinterpret_cast<float2*>(x + i) = v;
     if (bits == 4)
       tc_quantize_group<4>(v.x, v.y, limbs + g * 192, cs + g);
     else
@@ -445,8 +451,15 @@ template <int BITS, int NG>
 struct TcRows {
   static constexpr int RB = NG * kGroup * BITS / 8;
   static constexpr int LB = NG * 192;               // digit bytes of one token / activation row
+  static constexpr int LBP = LB + 96;               // a member's pitch in a digit slot (see tc_sum)
   static constexpr int CB = NG * 8;                 // its per-group scalars
 };
+
+// The staged row that mma row gid (and gid + 8) of a tile reads: even rows for
+// lanes 0-15, odd rows for lanes 16-31.  An 8-byte shared load is served per
+// half-warp; with the 128-byte swizzle (chunk ^= row % 8) rows r and r ^ 1 share
+// their pair of chunks, so a half-warp must read rows of distinct r >> 1.
+__device__ __forceinline__ int tc_row(int gid) { return ((gid & 3) << 1) | (gid >> 2); }
 
 // Staged rows (codes, and the per-group scale arrays): one tensor copy per array
 // brings an item's ROWS rows of RB bytes as lines of LW = min(128, RB) bytes
@@ -609,15 +622,20 @@ template <int BITS, int NG, int ROWS, int GPW, int TPW>
 __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf_hi, const int (&rlo)[TPW],
                                        const int (&rhi)[TPW], const uint8_t* const (&sarr)[4], const uint8_t* db, int n,
                                        int g0, float (&acc)[TPW][4]) {
-  constexpr int LB = NG * 192;
+  constexpr int LBP = TcRows<BITS, NG>::LBP;
   constexpr int GPC = GPW < 8 ? GPW : 8;  // groups whose scales are held at once
   const int lane = threadIdx.x & 31, gid = lane >> 2, q = lane & 3;
   const TcLane ln = tc_lane(q, n);
-  const int bt = gid < 6 ? gid / 3 : 0, bl = gid % 3;  // this lane's B column: token slot, limb
-  const uint8_t* bsrc = db + bt * LB + (size_t)((bl * 4 + q) * 8);
-  const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LB);  // [token][NG + 2] (padded pitch)
+  // This lane's B column: member slot and limb.  Half-warp 0 reads member 0's
+  // three limbs and member 1's limb 0, half-warp 1 member 1's limbs 1 and 2
+  // (columns 6 and 7, unused, repeat 4 and 5).  A member's 96 bytes of a group
+  // are limb-major; with the members 96 bytes apart modulo 128 (pitch LBP),
+  // each half-warp's 8-byte loads fall in distinct banks.
+  const int bt = gid < 3 ? 0 : 1, bl = gid < 6 ? gid % 3 : gid - 5;
+  const uint8_t* bsrc = db + bt * LBP + (size_t)((bl * 4 + q) * 8);
+  const float2* csv = reinterpret_cast<const float2*>(db + kUnitToks * LBP);  // [token][NG + 2] (padded pitch)
   // A addresses.  With 128-byte lines and g0 a multiple of the groups per line
-  // (4 at 4-bit, 8 at 2-bit), a lane's rows all have row % 8 == gid, so the
+  // (4 at 4-bit, 8 at 2-bit), a lane's rows all have row % 8 == tc_row(gid), so the
   // swizzled byte of group g is row*128 + (g / PER)*ROWS*128 + vx[g % PER], with
   // vx a lane constant: one add per load.  Otherwise the general formula (Sw).
   using SA = TcSw<BITS, NG, ROWS>;
@@ -625,7 +643,8 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
   constexpr bool FAST = SA::LW == 128 && GPW % PER == 0;
   uint32_t vx[PER];
 #pragma unroll
-  for (int m = 0; m < PER; ++m) vx[m] = (uint32_t)((BITS == 4 ? (m << 5) | (8 * q) : (m << 4) | (4 * q)) ^ (gid << 4));
+  for (int m = 0; m < PER; ++m)
+    vx[m] = (uint32_t)((BITS == 4 ? (m << 5) | (8 * q) : (m << 4) | (4 * q)) ^ (tc_row(gid) << 4));
   const uint8_t* blo[TPW];
   const uint8_t* bhi[TPW];
 #pragma unroll
@@ -706,22 +725,22 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
 
 // ---- gate/up + SwiGLU.  An item is ROWS = 8*TL (gate, up) row pairs: one
 // tensor copy per matrix stages the rows (swizzled, see TcSw), four bulk copies
-// the scale arrays.  Tile t pairs gate row 8t + gid (A rows 0-7) with the same
-// up row (rows 8-15).  The digits are those of x for each member token.  Warp
+// the scale arrays.  Tile t pairs gate row 8t + tc_row(gid) (A rows 0-7) with
+// the same up row (rows 8-15).  The digits are those of x for each member token.  Warp
 // w sums tiles [TPW*(w / KS), +TPW) over K slice w % KS; the KS partial tiles
 // add in slice order.  act[row][r] = silu(g) * u.
 template <int BITS, int NG, int TL>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gateup_kernel(const GroupedParams p, int ns, const __grid_constant__ TcMaps<12> maps) {
   using R = TcRows<BITS, NG>;
-  constexpr int RB = R::RB, LB = R::LB, CB = R::CB, SB = NG * 2;
+  constexpr int RB = R::RB, LB = R::LB, LBP = R::LBP, CB = R::CB, SB = NG * 2;
   constexpr int ROWS = 8 * TL, TPW = TL < 2 ? TL : 2, KS = kConsumers * TPW / TL;  // TPW tiles per warp, KS K slices
   constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;                                  // groups per K slice
   constexpr int CODE = (ROWS * RB + 1023) / 1024 * 1024;  // one matrix's staged rows
   constexpr int SA = (ROWS * SB + 1023) / 1024 * 1024;    // one staged scale array
   constexpr int WB = 2 * CODE + 4 * SA;                   // gate rows, up rows, gate s, gate b, up s, up b
   constexpr int CBP = CB + 16;                            // a token's scalars, padded apart in shared memory
-  constexpr int DB = kUnitToks * (LB + CBP);
+  constexpr int DB = kUnitToks * (LBP + CBP);
   constexpr int TP = 2 * ROWS * 8 + 4;  // floats per slice's partial tiles (gate rows, then up rows)
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
@@ -768,8 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane < u.n) {
         const int tok = u.tok[lane];
-        bulk_g2s(smem_addr(dst + lane * LB), p.xq_limbs + (size_t)tok * LB, LB, bd, pol_d);
-        bulk_g2s(smem_addr(dst + kUnitToks * LB + lane * CBP), p.xq_cs + (size_t)tok * NG, CB, bd, pol_d);
+        bulk_g2s(smem_addr(dst + lane * LBP), p.xq_limbs + (size_t)tok * LB, LB, bd, pol_d);
+        bulk_g2s(smem_addr(dst + kUnitToks * LBP + lane * CBP), p.xq_cs + (size_t)tok * NG, CB, bd, pol_d);
       }
     };
     producer_loop(p, NB, i0, count, ns, s_item, s_wfull, s_wempty, s_dfull, s_dempty, &s_abort, issue_w, issue_d);
@@ -780,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool kwarp = g0 < NG;  // this warp has groups to sum
   int rows[TPW];               // this lane's row pair in each of its tiles
 #pragma unroll
-  for (int i = 0; i < TPW; ++i) rows[i] = 8 * (tg * TPW + i) + gid;
+  for (int i = 0; i < TPW; ++i) rows[i] = 8 * (tg * TPW + i) + tc_row(gid);
   // output (row pair r, token t) of item k from slice ks, then the KS slices in order
   auto reduce = [&](int k, int row0, int n, int r0) {
     if (tid < 2 * ROWS * KS) {
@@ -856,22 +875,22 @@ __global__ void __launch_bounds__(kGT) grouped_actq_kernel(const GroupedParams p
 
 // ---- down.  An item is ROWS = 16*TL output rows: one tensor copy stages the
 // rows (swizzled, see TcSw), two bulk copies the scale arrays.  Tile t takes
-// rows 16t + gid (A rows 0-7) and 16t + 8 + gid (rows 8-15).  The digits are
-// those of the members' activations, whose rows are consecutive (two copies
-// per unit).  Warps split tiles and K as in gate/up.  y[member row][h] holds the
-// unweighted down output.
+// rows 16t + tc_row(gid) (A rows 0-7) and 16t + 8 + tc_row(gid) (rows 8-15).
+// The digits are those of the members' activations (two copies per member).
+// Warps split tiles and K as in gate/up.  y[member row][h] holds the unweighted
+// down output.
 template <int BITS, int NG, int TL>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_down_kernel(const GroupedParams p, int ns, const __grid_constant__ TcMaps<6> maps) {
   using R = TcRows<BITS, NG>;
-  constexpr int RB = R::RB, LB = R::LB, CB = R::CB, SB = NG * 2;
+  constexpr int RB = R::RB, LB = R::LB, LBP = R::LBP, CB = R::CB, SB = NG * 2;
   constexpr int ROWS = 16 * TL, TPW = TL < 2 ? TL : 2, KS = kConsumers * TPW / TL;
   constexpr int GPW = NG / KS >= 1 ? NG / KS : 1;
   constexpr int CODE = (ROWS * RB + 1023) / 1024 * 1024;
   constexpr int SA = (ROWS * SB + 1023) / 1024 * 1024;
   constexpr int WB = CODE + 2 * SA;  // rows, then s, b
   constexpr int CBP = CB + 16;
-  constexpr int DB = kUnitToks * (LB + CBP);
+  constexpr int DB = kUnitToks * (LBP + CBP);
   constexpr int TP = ROWS * 8 + 4;
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t s_wfull[kRing], s_wempty[kRing], s_dfull[2], s_dempty[2];
@@ -914,13 +933,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_d = [&](const UnitDesc& u, int slot) {
       const uint32_t bd = smem_addr(&s_dfull[slot]);
       uint8_t* dst = dbase + (size_t)slot * DB;
-      if (lane == 0) {
-        mbar_expect_tx(bd, (uint32_t)u.n * (LB + CB));
-        bulk_g2s(smem_addr(dst), p.act_limbs + (size_t)u.row0 * LB, u.n * LB, bd, pol_d);
-      }
+      if (lane == 0) mbar_expect_tx(bd, (uint32_t)u.n * (LB + CB));
       __syncwarp();
-      if (lane < u.n)
-        bulk_g2s(smem_addr(dst + kUnitToks * LB + lane * CBP), p.act_cs + (size_t)(u.row0 + lane) * NG, CB, bd, pol_d);
+      if (lane < u.n) {
+        bulk_g2s(smem_addr(dst + lane * LBP), p.act_limbs + (size_t)(u.row0 + lane) * LB, LB, bd, pol_d);
+        bulk_g2s(smem_addr(dst + kUnitToks * LBP + lane * CBP), p.act_cs + (size_t)(u.row0 + lane) * NG, CB, bd, pol_d);
+      }
     };
     producer_loop(p, NB, i0, count, ns, s_item, s_wfull, s_wempty, s_dfull, s_dempty, &s_abort, issue_w, issue_d);
     return;
@@ -931,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int rlo[TPW], rhi[TPW];  // this lane's rows in each of its tiles
 #pragma unroll
   for (int i = 0; i < TPW; ++i) {
-    rlo[i] = 16 * (tg * TPW + i) + gid;
+    rlo[i] = 16 * (tg * TPW + i) + tc_row(gid);
     rhi[i] = rlo[i] + 8;
   }
   // output (row r, token t) of item k from slice ks, then the KS slices in order
@@ -988,18 +1006,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (count > 0) reduce(count - 1, p_row0, p_n, p_d0);
 }
 
-// ---- combine, fixed k order: out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t]
+// ---- combine, fixed k order: out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t].
+// CTA (c, t) takes columns [4*kGT*c, 4*kGT*(c+1)) of token t, four per thread;
+// the member rows and weights are read once per CTA, and the rows' loads are
+// issued eight at a time before their terms are added in k order.
 __global__ void __launch_bounds__(kGT) grouped_combine_kernel(const GroupedParams p) {
-  const int t = blockIdx.y, h = blockIdx.x * kGT + threadIdx.x;
-  if (h >= p.H) return;
-  const int K = p.K;
-  float acc = 0.0f;
-  for (int k = 0; k < K; ++k) {
-    const int pos = __ldcg(p.pair_pos + (size_t)t * K + k);
-    acc = fmaf(__ldcg(p.route_w + (size_t)t * (K + 1) + k), __ldcg(p.y + (size_t)pos * p.H + h), acc);
+  __shared__ int s_pos[33];
+  __shared__ float s_w[33];
+  const int t = blockIdx.y, tid = threadIdx.x, K = p.K, H = p.H;
+  if (tid <= K) {
+    s_pos[tid] = tid < K ? __ldcg(p.pair_pos + (size_t)t * K + tid) : p.T * K + t;
+    s_w[tid] = __ldcg(p.route_w + (size_t)t * (K + 1) + tid);
   }
-  acc = fmaf(__ldcg(p.route_w + (size_t)t * (K + 1) + K), __ldcg(p.y + (size_t)(p.T * K + t) * p.H + h), acc);
-  p.out[(size_t)t * p.H + h] = p.h[(size_t)t * p.H + h] + acc;
+  __syncthreads();
+  const int h = (blockIdx.x * kGT + tid) * 4;
+  if (h >= H) return;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int k0 = 0; k0 <= K; k0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (k0 + j <= K) v[j] = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)s_pos[k0 + j] * H + h));
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (k0 + j <= K) {
+        const float w = s_w[k0 + j];
+        acc = make_float4(fmaf(w, v[j].x, acc.x), fmaf(w, v[j].y, acc.y), fmaf(w, v[j].z, acc.z), fmaf(w, v[j].w, acc.w));
+      }
+  }
+  const float4 hv = __ldcg(reinterpret_cast<const float4*>(p.h + (size_t)t * H + h));
+  *reinterpret_cast<float4*>(p.out + (size_t)t * H + h) =
+      make_float4(hv.x + acc.x, hv.y + acc.y, hv.z + acc.z, hv.w + acc.w);
 }
 
 constexpr size_t kSmemBudget = 220 * 1024;
@@ -1008,7 +1045,7 @@ constexpr size_t kSmemBudget = 220 * 1024;
 // slots of kUnitToks members, the double-buffered partial tiles (tp floats per
 // buffer, all K slices) and 1 KiB to align the staging ring.
 size_t tc_smem(int ns, size_t wb, int NG, size_t tp) {
-  return (size_t)ns * wb + 2 * (size_t)kUnitToks * ((size_t)NG * 200 + 16) + 2 * tp * 4 + 1024;
+  return (size_t)ns * wb + 2 * (size_t)kUnitToks * ((size_t)NG * 200 + 96 + 16) + 2 * tp * 4 + 1024;
 }
 
 size_t round_kib(size_t v) { return (v + 1023) / 1024 * 1024; }
@@ -1181,7 +1218,7 @@ int grouped_router_split(int H, int E, int T) {
 }
 
 cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s) {
-  norm_digits_kernel<<<p.T, kGT, 0, s>>>(p, rb, bits);
+  norm_digits_kernel<<<dim3(kNormSplit, p.T), kGT, 0, s>>>(p, rb, bits);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)kRtR * (kRtK + 8) * 2 + (size_t)kRtT * (kRtK + 4) * 4;
@@ -1210,7 +1247,7 @@ cudaError_t launch_grouped_down(const GroupedParams& p, int bits, cudaStream_t s
 }
 
 cudaError_t launch_grouped_combine(const GroupedParams& p, cudaStream_t s) {
-  grouped_combine_kernel<<<dim3((p.H + kGT - 1) / kGT, p.T), kGT, 0, s>>>(p);
+  grouped_combine_kernel<<<dim3((p.H / 4 + kGT - 1) / kGT, p.T), kGT, 0, s>>>(p);
   return cudaGetLastError();
 }
 
