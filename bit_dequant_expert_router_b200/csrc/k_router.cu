@@ -97,6 +97,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
     gv[j] = (p.norm && p.gamma && i < H) ? __ldg(reinterpret_cast<const float4*>(p.gamma + i))
                                          : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
   }
+  // h may still be written by the kernel waited on below.  An L2 prefetch of it
+  // cannot leave stale data behind (every global write lands in L2); when h was
+  // written earlier it hides the DRAM latency of the first read after the wait.
+  if (blockIdx.x == 0 && tid == 0) prefetch_l2(p.h + (size_t)t * H, (uint32_t)H * 4);
   pdl_wait();
   pdl_trigger();
   // every kernel of the previous token is complete: its routing flag is spent
