@@ -497,13 +497,16 @@ __device__ __forceinline__ void tc_load_a(const uint8_t* buf_lo, int row_lo, con
   }
 }
 
+// A registers of k-block kb.  At 4 bits the u8 operands are 16 * code (the low
+// nibble moved up, the high nibble masked in place), so the sums come out 16x;
+// the column scales carry the 1/16 (tc_colscale).
 template <int BITS>
 __device__ __forceinline__ void tc_unpack_a(const uint32_t (&w)[2][2], int kb, uint32_t (&a)[4]) {
   if (BITS == 4) {
-    a[0] = w[0][kb] & 0x0F0F0F0Fu;
-    a[1] = w[1][kb] & 0x0F0F0F0Fu;
-    a[2] = (w[0][kb] >> 4) & 0x0F0F0F0Fu;
-    a[3] = (w[1][kb] >> 4) & 0x0F0F0F0Fu;
+    a[0] = (w[0][kb] << 4) & 0xF0F0F0F0u;
+    a[1] = (w[1][kb] << 4) & 0xF0F0F0F0u;
+    a[2] = w[0][kb] & 0xF0F0F0F0u;
+    a[3] = w[1][kb] & 0xF0F0F0F0u;
   } else {
     a[0] = (w[0][kb] >> (4 * kb)) & 0x03030303u;
     a[1] = (w[1][kb] >> (4 * kb)) & 0x03030303u;
@@ -569,7 +572,7 @@ __device__ __forceinline__ TcLane tc_lane(int q, int n) {
 
 // The int32 sums are read as floats through a biased accumulator: the mma
 // starts from the bits of 1.5 * 2^23, so that (for |sum| < 2^22, here below
-// 15 * 128 * 64) the result's bits are those of the float 1.5 * 2^23 + sum.
+// 16 * 15 * 128 * 64 at 4 bits) the result's bits are those of the float 1.5 * 2^23 + sum.
 // With a power-of-two digit scale s, fma(f, s, -1.5 * 2^23 * s) is then
 // exactly sum * s.
 constexpr int kMagicBits = 0x4B400000;
@@ -581,11 +584,12 @@ struct TcColScale {
   float bx;      // group sum of x / 2^16 for this lane's limb-0 column, else 0
 };
 
-__device__ __forceinline__ TcColScale tc_colscale(const float2* csv, int NG, int g, const TcLane& l) {
+// cf: the factor of the codes in the A operand's sums (1/16 at 4 bits, see tc_unpack_a).
+__device__ __forceinline__ TcColScale tc_colscale(const float2* csv, int NG, int g, const TcLane& l, float cf) {
   const float2 va = csv[l.ta * (NG + 2) + g], vb = csv[l.tb * (NG + 2) + g];
   TcColScale c;
-  c.sa = l.va ? va.x : 0.0f;
-  c.sb = l.vb ? vb.x : 0.0f;
+  c.sa = l.va ? va.x * cf : 0.0f;
+  c.sb = l.vb ? vb.x * cf : 0.0f;
   c.na = -kMagic * c.sa;
   c.nb = -kMagic * c.sb;
   c.bx = (l.bias_a ? va.y : l.bias_b ? vb.y : 0.0f) * 0x1p-16f;
@@ -655,7 +659,7 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
   float accb[TPW][2];
 #pragma unroll
   for (int i = 0; i < TPW; ++i) accb[i][0] = accb[i][1] = 0.0f;
-#pragma unroll
+#pragma unroll 1  // chunks of GPC groups (more than one only for long rows: keeps registers in bounds)
   for (int gc = 0; gc < GPW; gc += GPC) {
     uint32_t sv[TPW][4][(GPC + 1) / 2];
 #pragma unroll
@@ -671,20 +675,20 @@ __device__ __forceinline__ void tc_sum(const uint8_t* buf_lo, const uint8_t* buf
       uint2 b[2];
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) b[kb] = *reinterpret_cast<const uint2*>(bsrc + g * 192 + kb * 96);
-      const TcColScale cs = tc_colscale(csv, NG, g, ln);
+      const TcColScale cs = tc_colscale(csv, NG, g, ln, BITS == 4 ? 0.0625f : 1.0f);
 #pragma unroll
       for (int i = 0; i < TPW; ++i) {
         uint32_t w[2][2];
         if constexpr (FAST) {
-          const int gg = gc + gi;  // compile-time after unrolling
-          const size_t off = (size_t)(gg / PER) * ROWS * 128;
+          // GPC is a multiple of PER here, so gi % PER is the line position
+          const size_t off = (size_t)(gc / PER + gi / PER) * ROWS * 128;
           if (BITS == 4) {
-            const uint2 x = *reinterpret_cast<const uint2*>(blo[i] + off + vx[gg % PER]);
-            const uint2 y = *reinterpret_cast<const uint2*>(bhi[i] + off + vx[gg % PER]);
+            const uint2 x = *reinterpret_cast<const uint2*>(blo[i] + off + vx[gi % PER]);
+            const uint2 y = *reinterpret_cast<const uint2*>(bhi[i] + off + vx[gi % PER]);
             w[0][0] = x.x; w[0][1] = x.y; w[1][0] = y.x; w[1][1] = y.y;
           } else {
-            const uint32_t x = *reinterpret_cast<const uint32_t*>(blo[i] + off + vx[gg % PER]);
-            const uint32_t y = *reinterpret_cast<const uint32_t*>(bhi[i] + off + vx[gg % PER]);
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(blo[i] + off + vx[gi % PER]);
+            const uint32_t y = *reinterpret_cast<const uint32_t*>(bhi[i] + off + vx[gi % PER]);
             w[0][0] = w[0][1] = x; w[1][0] = w[1][1] = y;
           }
         } else {

@@ -32,6 +32,24 @@ def test_grouped_small_batch_matches_oracle(fmoe, bits):
     assert exact >= 60
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+def test_grouped_longer_rows(fmoe, monkeypatch, bits):
+    """hidden 1024 and intermediate 2048: other staged-row widths, items and K slices than
+    the 512-wide layer (gate/up 16 groups per row, down 32).  The per-token path gives the
+    same routing and, summing in another order, not the same bits: the batch ran grouped."""
+    # (top-2: the per-token down kernel holds (K + 1) * 32 groups of digits, at most 128)
+    spec = gen.LayerSpec(hidden=1024, experts=16, inter=2048, top_k=2, bits=bits, router_std=1.0 / 32.0,
+                         random_gamma=True)
+    hl = gen.host_layer(spec, seed=17)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(1700, 24, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    _compare_layer(hl, h, out, idx, w)
+    monkeypatch.setenv("FMOE_GROUPED", "0")
+    out1, idx1, _ = _run_layer(fmoe, dl, h)
+    assert np.array_equal(idx, idx1) and not np.array_equal(out, out1)
+
+
 def test_grouped_small_batch_top1_all_experts_and_odd_size(fmoe):
     spec = gen.small_layer(4, experts=8, top_k=2)
     hl = gen.host_layer(spec, seed=13)
