@@ -57,6 +57,17 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
                : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Two fp32 fmas in one instruction (element-wise, each rounded once: the same
+// results as two fmaf).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{ .reg .b64 a, b, c, d; mov.b64 a, {%2, %3}; mov.b64 b, {%4, %5}; mov.b64 c, {%6, %7};"
+      " fma.rn.f32x2 d, a, b, c; mov.b64 {%0, %1}, d; }"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 // d = a * b + c with c a separate (unchanged) input, e.g. a constant start value.
 __device__ __forceinline__ void mma_u8s8_c(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, int c) {
   asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
@@ -608,12 +619,20 @@ __device__ __forceinline__ void tc_tile_group(const uint32_t (&w)[2][2], const u
   mma_u8s8_c(c, a, b[0].x, b[0].y, kMagicBits);  // starts from the biased accumulator
   tc_unpack_a<BITS>(w, 1, a);
   mma_u8s8(c, a, b[1].x, b[1].y);
-  acc[0] = fmaf(s_lo, fmaf(__int_as_float(c[0]), cs.sa, cs.na), acc[0]);
-  acc[1] = fmaf(s_lo, fmaf(__int_as_float(c[1]), cs.sb, cs.nb), acc[1]);
-  acc[2] = fmaf(s_hi, fmaf(__int_as_float(c[2]), cs.sa, cs.na), acc[2]);
-  acc[3] = fmaf(s_hi, fmaf(__int_as_float(c[3]), cs.sb, cs.nb), acc[3]);
-  accb[0] = fmaf(b_lo, cs.bx, accb[0]);
-  accb[1] = fmaf(b_hi, cs.bx, accb[1]);
+  // the lane's two columns pair up: digit scales {sa, sb}, row scale s_lo (A rows
+  // 0-7) or s_hi (rows 8-15)
+  const float2 sc = make_float2(cs.sa, cs.sb), nc = make_float2(cs.na, cs.nb);
+  const float2 ilo = ffma2(make_float2(__int_as_float(c[0]), __int_as_float(c[1])), sc, nc);
+  const float2 ihi = ffma2(make_float2(__int_as_float(c[2]), __int_as_float(c[3])), sc, nc);
+  const float2 alo = ffma2(make_float2(s_lo, s_lo), ilo, make_float2(acc[0], acc[1]));
+  const float2 ahi = ffma2(make_float2(s_hi, s_hi), ihi, make_float2(acc[2], acc[3]));
+  const float2 ab = ffma2(make_float2(b_lo, b_hi), make_float2(cs.bx, cs.bx), make_float2(accb[0], accb[1]));
+  acc[0] = alo.x;
+  acc[1] = alo.y;
+  acc[2] = ahi.x;
+  acc[3] = ahi.y;
+  accb[0] = ab.x;
+  accb[1] = ab.y;
 }
 
 // Sums TPW tiles over groups [g0, g0 + GPW) into acc (each tile's C layout,
