@@ -31,8 +31,8 @@ FALLBACK_HBM_GBS = 6650.0
 # from one ncu capture of the current gateup_kernel per workload; None where none was taken.
 GATEUP_TRAFFIC = {"qwen397-4bit": 30697472}  # ncu capture of the per-token gate/up kernel
 # grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
-# (+ the shared expert): 1,050,211,840 B over 207.5 experts
-GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5061262}
+# (+ the shared expert): 1,051,820,288 B over 207.5 experts
+GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5069013}
 DTYPE_TOKEN = "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32"
 DTYPE_BATCH = "i32 mma.sync (u4/u2 codes as u8 x 24-bit fixed-point x as three s8 limbs) + f32"
 BATCH_KERNELS = 8  # norm+digits, router GEMM, top-K, sort, gate/up, activation digits, down, combine
