@@ -383,10 +383,6 @@ __device__ __forceinline__ UnitDesc load_unit(const GroupedParams& p, int wi) {
   return UnitDesc{a.x, a.y, a.z, a.w, {b.x, b.y, b.z, b.w}};
 }
 
-__device__ __forceinline__ const uint8_t* unit_record(const GroupedParams& p, int e) {
-  return e < 0 ? p.shared.base : p.routed.base + (long long)e * p.routed.stride;
-}
-
 // this CTA's items [i0, i0 + count)
 __device__ __forceinline__ void item_range(const GroupedParams& p, int NB, int& i0, int& count) {
   const long long n = (long long)__ldcg(p.n_active + 1) * NB, P = gridDim.x, c = blockIdx.x;
@@ -482,8 +478,8 @@ __device__ __forceinline__ int tc_row(int gid) { return ((gid & 3) << 1) | (gid 
 template <int RB, int ROWS>
 struct Sw {
   static constexpr int LW = RB >= 128 ? 128 : RB;
-  static constexpr int M = LW == 128 ? 7 : LW == 64 ? 3 : LW == 32 ? 1 : 0;
   __device__ static __forceinline__ const uint8_t* at(const uint8_t* buf, int row, int c) {
+    constexpr int M = LW == 128 ? 7 : LW == 64 ? 3 : LW == 32 ? 1 : 0;  // swizzle mask of the line index
     const int X = ((c / LW) * ROWS + row) * LW + c % LW;
     return buf + (X ^ (((X >> 7) & M) << 4));
   }
