@@ -490,19 +490,9 @@ __device__ __forceinline__ void block_topk_stage1(const float* logits, int E, in
 __device__ __forceinline__ void block_topk_stage2(float zg, int E, int K, int has_gate,
                                                   const unsigned long long* cand, int* idx, float* w) {
   const int lane = threadIdx.x & 31;
-  unsigned long long key[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) key[i] = lane + 32 * i < 8 * K ? cand[lane + 32 * i] : 0ull;
   float top = 0.0f, mine = 0.0f;
   int mi = 0;
-#pragma unroll 1
-  for (int k = 0; k < K; ++k) {
-    unsigned long long best = 0ull;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) best = key[i] > best ? key[i] : best;
-    const unsigned long long m = warp_max_key(best);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) key[i] = key[i] == m ? 0ull : key[i];
+  auto take = [&](int k, unsigned long long m) {
     int e = m ? topk_key_index(m) : 0;
     const float v = topk_key_value(m);
     if (e < 0 || e >= E) e = 0;  // only with non-finite logits
@@ -510,6 +500,29 @@ __device__ __forceinline__ void block_topk_stage2(float zg, int E, int K, int ha
     if (lane == k) {
       mi = e;
       mine = v;
+    }
+  };
+  if (8 * K <= 32) {  // at most one candidate per lane
+    unsigned long long key = lane < 8 * K ? cand[lane] : 0ull;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      const unsigned long long m = warp_max_key(key);
+      key = key == m ? 0ull : key;
+      take(k, m);
+    }
+  } else {
+    unsigned long long key[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) key[i] = lane + 32 * i < 8 * K ? cand[lane + 32 * i] : 0ull;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) best = key[i] > best ? key[i] : best;
+      const unsigned long long m = warp_max_key(best);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) key[i] = key[i] == m ? 0ull : key[i];
+      take(k, m);
     }
   }
   const float ek = lane < K ? expf(mine - top) : 0.0f;

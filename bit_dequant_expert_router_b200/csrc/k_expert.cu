@@ -29,7 +29,7 @@ namespace {
 // ------------------------------------------------------------------------------------------ gate/up
 
 constexpr int kGuWarps = 8;
-constexpr int kChunkUnits = 8;  // units per staged chunk
+constexpr int kChunkUnits = 20;  // units per staged chunk (few, large copies: each costs issue time)
 constexpr size_t kGuSmemBudget = 220 * 1024;  // shared memory of the gate/up kernel
 
 template <int BITS, int NG>
