@@ -29,7 +29,7 @@ METRIC = "MoE-layer decode tokens/s and effective weight GB/s (fraction of HBM p
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gate/up launch,
 # from one ncu capture of the current gateup_kernel per workload; None where none was taken.
-GATEUP_TRAFFIC = {}  # ncu capture of the per-token gate/up kernel (none yet of the 20-unit-chunk build)
+GATEUP_TRAFFIC = {"qwen397-4bit": 30658048}  # ncu capture of the per-token gate/up kernel (mean of 2 launches)
 # grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
 # (+ the shared expert): 1,051,820,288 B over 207.5 experts
 GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5069013}
