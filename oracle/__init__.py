@@ -5,6 +5,7 @@ this package.  It shares no code with the CUDA path; inputs are numpy arrays in
 host memory (bf16 values as uint16 bit patterns).
 """
 import ctypes
+import os
 
 import numpy as np
 
@@ -33,8 +34,13 @@ class OrLayer(ctypes.Structure):
 def lib():
     global _lib
     if _lib is None:
-        _build.build()
-        L = ctypes.CDLL(_build.SO)
+        # FMOE_ORACLE_SO: load another build of the oracle source instead (the mutation
+        # tests point it at copies with a planted mistake, to show that the pins fail)
+        so = os.environ.get("FMOE_ORACLE_SO")
+        if not so:
+            _build.build()
+            so = _build.SO
+        L = ctypes.CDLL(so)
         vp, ci, cd = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         L.or_bf16.restype = cd
         L.or_bf16.argtypes = [ctypes.c_uint16]

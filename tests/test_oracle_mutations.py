@@ -1,0 +1,102 @@
+"""The oracle's pins catch plausible mistakes (no GPU needed).
+
+Each case plants one slip in a copy of the oracle's C source: a wrong code
+order, a dropped or mis-signed term, a wrong group index, a transposed operand,
+a missing normalisation, a reversed tie-break, swapped SwiGLU operands, a
+missing residual or shared term.  The copy is compiled with the oracle's own
+flags into a temporary directory, the pin suite (test_oracle_pins.py) runs
+against it in a child process, and at least one pin must fail.  The real
+oracle is never touched.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(ROOT, "oracle", "fmoe_oracle.c")
+
+# (name, text in the oracle source, the slip that replaces it)
+MUTATIONS = [
+    ("code order msb-first",
+     "return (w >> (bits * (c % per_word))) & ((1u << bits) - 1u);",
+     "return (w >> (32 - bits * (1 + c % per_word))) & ((1u << bits) - 1u);"),
+    ("bias dropped",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]) + or_bf16(m->bias[(int64_t)r * gpr + g]);",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]);"),
+    ("bias sign",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]) + or_bf16(m->bias[(int64_t)r * gpr + g]);",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]) - or_bf16(m->bias[(int64_t)r * gpr + g]);"),
+    ("group index of the first group only",
+     "const int g = c / m->group;",
+     "const int g = 0 * (c / m->group);"),
+    ("group index by column modulo",
+     "const int g = c / m->group;",
+     "const int g = c % gpr;"),
+    ("matvec transposed",
+     "for (int c = 0; c < m->cols; ++c) acc += or_weight(m, r, c) * x[c];",
+     "for (int c = 0; c < m->cols; ++c) acc += or_weight(m, c % m->rows, r % m->cols) * x[c];"),
+    ("rmsnorm without the mean",
+     "const double denom = sqrt(ss / (double)H + eps);",
+     "const double denom = sqrt(ss + eps);"),
+    ("rmsnorm ignores gamma",
+     "x[i] = (double)h[i] / denom * (gamma ? (double)gamma[i] : 1.0);",
+     "x[i] = (double)h[i] / denom;"),
+    ("router bias dropped",
+     "logits[e] = acc + (bias ? (double)bias[e] : 0.0);",
+     "logits[e] = acc;"),
+    ("softmax not normalised",
+     "for (int i = 0; i < n; ++i) p[i] /= s;",
+     "for (int i = 0; i < n; ++i) p[i] /= 1.0;"),
+    ("top-k ties to the higher index",
+     "return (x->i > y->i) - (x->i < y->i);",
+     "return (x->i < y->i) - (x->i > y->i);"),
+    ("top-k ascending",
+     "if (x->v > y->v) return -1;\n  if (x->v < y->v) return 1;",
+     "if (x->v > y->v) return 1;\n  if (x->v < y->v) return -1;"),
+    ("swiglu operands swapped",
+     "g[r] = g[r] / (1.0 + exp(-g[r])) * u[r];",
+     "g[r] = u[r] / (1.0 + exp(-u[r])) * g[r];"),
+    ("silu sign",
+     "g[r] = g[r] / (1.0 + exp(-g[r])) * u[r];",
+     "g[r] = g[r] / (1.0 + exp(g[r])) * u[r];"),
+    ("weights not renormalised",
+     "const double wk = p[idx[k]] / psum;",
+     "const double wk = p[idx[k]];"),
+    ("shared gate sign",
+     "const double sigma = 1.0 / (1.0 + exp(-zs));",
+     "const double sigma = 1.0 / (1.0 + exp(zs));"),
+    ("shared gate on h instead of the normalised x",
+     "for (int i = 0; i < H; ++i) zs += or_bf16(L->w_shared_gate[i]) * x[i];",
+     "for (int i = 0; i < H; ++i) zs += or_bf16(L->w_shared_gate[i]) * (double)ht[i];"),
+    ("down fed the up projection",
+     "or_matvec(&md, g, y);",
+     "or_matvec(&md, u, y);"),
+    ("eps outside the root",
+     "const double denom = sqrt(ss / (double)H + eps);",
+     "const double denom = sqrt(ss / (double)H) + eps;"),
+    ("residual dropped",
+     "for (int i = 0; i < H; ++i) ot[i] = (double)ht[i];",
+     "for (int i = 0; i < H; ++i) ot[i] = 0.0;"),
+    ("shared expert dropped",
+     "for (int i = 0; i < H; ++i) ot[i] += sigma * y[i];",
+     "for (int i = 0; i < H; ++i) ot[i] += 0.0 * sigma * y[i];"),
+]
+
+
+@pytest.mark.parametrize("name,orig,slip", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(tmp_path, name, orig, slip):
+    src = open(SRC).read()
+    assert src.count(orig) == 1, f"the oracle source no longer holds the text this case mutates: {name}"
+    mutated = tmp_path / "fmoe_oracle_mutated.c"
+    mutated.write_text(src.replace(orig, slip))
+    so = tmp_path / "liboracle_mutated.so"
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+                           "-std=c11", str(mutated), "-o", str(so), "-lm"])
+    env = dict(os.environ, FMOE_ORACLE_SO=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(HERE, "test_oracle_pins.py"), "-q", "-x",
+                        "-p", "no:cacheprovider", "-m", "not gpu"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 1, f"no pin failed with the planted mistake '{name}':\n{r.stdout[-2000:]}"

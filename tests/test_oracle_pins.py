@@ -4,7 +4,8 @@ Each test is chosen so that a plausible slip in the oracle fails it: a wrong
 code order or field width (worked examples), a dropped or mis-signed bias term
 (worked examples, closed forms), a wrong group index or a transposed operand
 (brute force on non-square shapes with distinct per-group scales), a missing
-renormalisation or wrong sort order (top-K/softmax), swapped SwiGLU operands or
+renormalisation or wrong sort order (top-K/softmax), a dropped router bias
+(one-hot router rows), swapped SwiGLU operands or
 sigmoid sign (closed-form constant experts), and a missing residual or shared
 term (K = E invariant and closed-form combine).
 """
@@ -106,6 +107,19 @@ def test_topk_is_full_sort_with_ties_to_lower_index():
         assert oracle.topk(p, k).tolist() == np.argsort(-p, kind="stable")[:k].tolist()
     tied = np.array([0.1, 0.3, 0.3, 0.2, 0.3, 0.05])
     assert oracle.topk(tied, 4).tolist() == [1, 2, 4, 3]
+
+
+def test_router_logits_closed_forms():
+    # one-hot bf16 rows (W[e, i] = 1 if i == e): l_e = x_e + bias_e exactly; zero rows: l = bias
+    E, H = 8, 64
+    x = np.random.default_rng(6).standard_normal(H)
+    bias = (np.arange(E, dtype=np.float32) - 3.5) / 4.0
+    one = f32_to_bf16_exact([1.0])[0]
+    w = np.zeros((E, H), np.uint16)
+    w[np.arange(E), np.arange(E)] = one
+    assert oracle.router_logits(w, bias, x).tolist() == (x[:E] + bias.astype(np.float64)).tolist()
+    assert oracle.router_logits(w, None, x).tolist() == x[:E].tolist()
+    assert oracle.router_logits(np.zeros((E, H), np.uint16), bias, x).tolist() == bias.astype(np.float64).tolist()
 
 
 def test_softmax_closed_form_and_sum():
