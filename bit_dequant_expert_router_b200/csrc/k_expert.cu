@@ -29,7 +29,7 @@ namespace {
 // ------------------------------------------------------------------------------------------ gate/up
 
 constexpr int kGuWarps = 8;
-constexpr int kChunkUnits = 20;  // units per staged chunk (few, large copies: each costs issue time)
+constexpr int kMaxChunkUnits = 20;  // units per staged chunk, at most (few, large copies: each costs issue time)
 constexpr size_t kGuSmemBudget = 220 * 1024;  // shared memory of the gate/up kernel
 
 template <int BITS, int NG>
@@ -39,17 +39,21 @@ struct GuCfg {
   static constexpr int kRowPairs = G::kRowsPerPass * kPasses;  // rows of gate (and of up) per unit
   static constexpr int kRowBytes = NG * kGroup * BITS / 8;
   static constexpr int kScaleBytes = NG * 2;
-  static constexpr int kChunkRows = kChunkUnits * kRowPairs;
-  // chunk buffer: gate codes | up codes | gate scales | gate biases | up scales | up biases
-  static constexpr int kChunkBytes = (2 * kChunkRows * (kRowBytes + 2 * kScaleBytes) + 127) / 128 * 128;
   static constexpr int kChunks = NG * kGroup * BITS / 128;
   static constexpr int kDigitBytes = NG * kGroupWords * 4 + kChunks * 8;  // x digits + chunk scalars
   static constexpr int kHead = (kDigitBytes + 127) / 128 * 128;
+  // units per chunk: kMaxChunkUnits, or fewer where two chunk buffers would not fit
+  static constexpr int kUnitBytes = 2 * kRowPairs * (kRowBytes + 2 * kScaleBytes);
+  static constexpr int kFit = (int)((kGuSmemBudget - kHead - 256) / (2 * (size_t)kUnitBytes));
+  static constexpr int kChunkUnits = kFit < 1 ? 1 : kFit < kMaxChunkUnits ? kFit : kMaxChunkUnits;
+  static constexpr int kChunkRows = kChunkUnits * kRowPairs;
+  // chunk buffer: gate codes | up codes | gate scales | gate biases | up scales | up biases
+  static constexpr int kChunkBytes = (2 * kChunkRows * (kRowBytes + 2 * kScaleBytes) + 127) / 128 * 128;
   static_assert(kRowPairs * kScaleBytes % 16 == 0 && kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
 };
 
 // Persistent: CTA b owns units [b*U/G, (b+1)*U/G) (a unit = kRowPairs rows of
-// gate and up of one expert slot), cut into chunks of up to kChunkUnits units
+// gate and up of one expert slot), cut into chunks of up to C::kChunkUnits units
 // of one slot, each staged with six bulk copies into a ring of nbuf chunk
 // buffers; warp w computes units w, w+8, .. of the chunk.  A lane always works
 // on the same groups of 64 columns, so it keeps their digits of x in registers
@@ -87,8 +91,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
   }
   __syncthreads();
 
-  // Chunk c covers units [cu, ce): up to kChunkUnits units, never across a slot boundary.
-  auto chunk_end = [&](int cu) { return min(min(cu + kChunkUnits, u1), (cu / ups + 1) * ups); };
+  // Chunk c covers units [cu, ce): up to C::kChunkUnits units, never across a slot boundary.
+  auto chunk_end = [&](int cu) { return min(min(cu + C::kChunkUnits, u1), (cu / ups + 1) * ups); };
   auto issue = [&](int c, int cu, int ce) {  // thread 0
     const int sl = cu / ups, r0 = (cu % ups) * RP, rows = (ce - cu) * RP;
     const bool routed = sl < p.K;
@@ -496,7 +500,7 @@ cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
   if ((long long)(units + grid - 1) / grid * C::kRowPairs / kGroup + 2 > kGuWarps * 32 - 32) return cudaErrorInvalidValue;
   const int per_cta = (units + grid - 1) / grid;
   int nbuf = (int)((kGuSmemBudget - C::kHead) / C::kChunkBytes);
-  const int need = (per_cta + kChunkUnits - 1) / kChunkUnits + 1;  // +1: a chunk may stop at a slot boundary
+  const int need = (per_cta + C::kChunkUnits - 1) / C::kChunkUnits + 1;  // +1: a chunk may stop at a slot boundary
   nbuf = nbuf > need ? need : nbuf;
   nbuf = nbuf > 8 ? 8 : nbuf;
   if (nbuf < 1) return cudaErrorInvalidValue;
