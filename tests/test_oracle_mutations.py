@@ -77,6 +77,17 @@ MUTATIONS = [
     ("eps outside the root",
      "const double denom = sqrt(ss / (double)H + eps);",
      "const double denom = sqrt(ss / (double)H) + eps;"),
+    ("gate and up matrices swapped",
+     "m.qw = (const uint32_t*)(rec + b->off[3 * which]);\n  m.scale = (const uint16_t*)(rec + b->off[3 * which + 1]);\n"
+     "  m.bias = (const uint16_t*)(rec + b->off[3 * which + 2]);",
+     "const int wh = which == 2 ? 2 : 1 - which;\n  m.qw = (const uint32_t*)(rec + b->off[3 * wh]);\n"
+     "  m.scale = (const uint16_t*)(rec + b->off[3 * wh + 1]);\n  m.bias = (const uint16_t*)(rec + b->off[3 * wh + 2]);"),
+    ("scales and biases of a matrix swapped",
+     "m.scale = (const uint16_t*)(rec + b->off[3 * which + 1]);\n  m.bias = (const uint16_t*)(rec + b->off[3 * which + 2]);",
+     "m.scale = (const uint16_t*)(rec + b->off[3 * which + 2]);\n  m.bias = (const uint16_t*)(rec + b->off[3 * which + 1]);"),
+    ("expert record of the next expert",
+     "const uint8_t* rec = b->records ? b->records[e] : b->base + (int64_t)e * b->stride;",
+     "const uint8_t* rec = b->records ? b->records[(e + 1) % b->num_experts] : b->base + (int64_t)((e + 1) % b->num_experts) * b->stride;"),
     ("residual dropped",
      "for (int i = 0; i < H; ++i) ot[i] = (double)ht[i];",
      "for (int i = 0; i < H; ++i) ot[i] = 0.0;"),
