@@ -9,16 +9,22 @@
 // Results are scattered back with the renormalised top-K weights in fixed k
 // order, so the output does not depend on the grouping.
 //
-// Kernels, in stream order after the router (which already writes the logits
-// and the digits of x of every token):
-//   select  : top-K per token, the sorted pair list and the active experts
-//   gate/up : one CTA per (active expert, block of rows): stage the rows once,
-//             then gate/up + SwiGLU for each token of the group
-//   actq    : digits of every pair's activations (fmoe_device.cuh format)
-//   down    : one CTA per (active expert, block of output rows), same scheme
-//   combine : out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t]
-// Dequant dot products use the per-group fold sum_c (q s + b) x = s*sum q x + b*sum x
-// with exact dp4a sums ("What is Flash-MoE", sections 2-3, for the block itself).
+// Kernels, in stream order:
+//   norm_digits : x = RMSNorm(h) per token (fp32 for the router) and its digits
+//   router_gemm : partial logits of [W_r; w_sg] x as a split-K tiled product
+//   topk_tokens : the slice sums in order, the top-K and weights per token
+//   sort_pairs  : the sorted pair list, the active experts and the work units
+//                 (runs of at most kUnitToks members of one expert's group)
+//   gate/up     : persistent, one CTA per SM; a producer warp stages each item
+//                 (a block of rows of one unit's expert) by TMA tensor copies,
+//                 eight consumer warps contract it with the members' digits
+//                 on the int8 tensor cores (mma.sync) and apply SwiGLU
+//   actq        : digits of every member's activations
+//   down        : the same scheme over blocks of output rows
+//   combine     : out[t] = h[t] + sum_k w_tk y[pair(t,k)] + sigma_t y_shared[t]
+// The dequant products use the per-group fold sum_c (q s + b) x = s*sum q x + b*sum x
+// with exact integer sums of codes times fixed-point digits of x ("What is
+// Flash-MoE", sections 2-3, for the block itself).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
