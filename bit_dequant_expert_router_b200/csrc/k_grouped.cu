@@ -48,9 +48,11 @@ constexpr int kMaxTK = 4096;      // T*K pairs
 // Lane (gid, q) of the quad layout (gid = lane / 4, q = lane % 4) holds the A
 // registers {row gid k-lo, row gid+8 k-lo, row gid k-hi, row gid+8 k-hi} and the
 // B registers {k-lo, k-hi} of column gid, k-lo being k-slots 4q..4q+3 and k-hi
-// 16+4q..16+4q+3.  A code word unpacks into those byte registers directly:
+// 16+4q..16+4q+3 (A row r is staged row tc_row(r) of its 8-row half).  A code
+// word unpacks into those byte registers directly:
 //   4-bit, k-block kb: word 2q+kb of the group's row; k-lo = low nibbles
-//     (columns 16q + 8kb + 2j), k-hi = high nibbles (the next column each);
+//     (columns 16q + 8kb + 2j), k-hi = high nibbles (the next column each),
+//     both entering as 16 x code (tc_unpack_a);
 //   2-bit, k-block kb: word q; k-lo = 2-bit pack 2kb (columns 16q + 4j + 2kb),
 //     k-hi = pack 2kb+1 (the next column each).
 // The digits are stored so that each (k-block, limb, q) is one 8-byte pair
