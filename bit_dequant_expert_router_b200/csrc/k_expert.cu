@@ -10,15 +10,17 @@
 // with sum_c x_c precomputed once per token and sum_c q_c x_c an exact integer
 // dp4a dot product against a 3-digit fixed-point x (fmoe_device.cuh).
 //
-// Both kernels run in one wave.  Each warp owns one work unit (a few rows of
-// one expert, or a few output rows of every selected expert), bulk-copies the
-// unit's codes, scales and biases into its own shared-memory slice with the
-// TMA engine, waits once on its own mbarrier, reduces across its lanes and
-// writes its outputs: no CTA-wide barrier on the hot path, and every byte of
-// the phase is requested at the start.  Weight copies that do not depend on the
-// previous kernel (the shared expert; the down matrices, whose experts are known
-// from the router) are issued before griddepcontrol.wait, so they overlap the
-// previous kernel under programmatic dependent launch.
+// Both kernels run in one wave, one CTA per SM.  Each CTA owns a contiguous
+// range of work units (gate/up: a row pair of gate and up of one expert slot;
+// down: a few output rows of every selected expert) and stages them with bulk
+// copies on the TMA engine in a few large chunks, each completing on its own
+// mbarrier: a copy costs issue time on the SM's copy engine, so there are few
+// of them, and as much of the CTA's share as fits is requested at once.  Lanes
+// keep their groups' digits in registers; warps reduce across their lanes.
+// Weight copies that do not depend on the previous kernel (the shared expert's
+// rows; the routed down rows once the routing is published) are issued before
+// griddepcontrol.wait, so they overlap the previous kernel under programmatic
+// dependent launch.
 #include <mutex>
 
 #include "fmoe_internal.h"
