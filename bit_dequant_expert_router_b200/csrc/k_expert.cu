@@ -346,7 +346,8 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
 
   // The shared expert's rows are weights: thread 0 requests them for the first
   // chunks before the wait.  The routing is written by CTA 0 of the gate/up
-  // kernel: it is read, and the routed rows requested, after the wait.
+  // kernel: if it is published already (route_ready), it is read and the routed
+  // rows requested before the wait, otherwise after it.
   if (tid == 0 && p.has_shared) {
     s_src[p.K][0] = p.shared.base + p.shared.off[6];
     s_src[p.K][1] = p.shared.base + p.shared.off[7];
