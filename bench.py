@@ -70,6 +70,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--reps", type=int, default=5, help="timed repetitions of the steps-token region (median)")
     return ap.parse_args()
 
 
@@ -136,14 +137,16 @@ class ClockSampler:
 
 
 def max_over_ranks(ms, world, device):
-    """The slowest rank's time (ms): every rank times its own replica, the job takes as long as the slowest."""
+    """The slowest rank's time (ms), or element-wise for a list of repetitions: every rank
+    times its own replica, the job takes as long as the slowest."""
     if world <= 1:
         return ms
     import torch
     import torch.distributed as dist
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    one = not isinstance(ms, (list, tuple))
+    t = torch.tensor([ms] if one else list(ms), dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return float(t[0].item()) if one else t.tolist()
 
 
 def dist_setup(args):
@@ -263,22 +266,31 @@ def main():
         graph.replay()
     stream.synchronize()
 
-    # ---- timed region: `steps` tokens, as steps / G graph replays
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    # ---- timed region: `steps` tokens, as steps / G graph replays, repeated `reps` times
+    # (at least 5, and enough to cover about 0.3 s for the clock record); the reported
+    # time is the median over repetitions of the slowest rank's time
+    def timed(g):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            ev0.record(stream)
+            e0.record(stream)
             for _ in range(steps // G):
-                graph.replay()
-            ev1.record(stream)
-        ev1.synchronize()
-    torch.cuda.synchronize(dev)
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    if world > 1:
-        dist.barrier()
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    def repeat(g):
+        first = max_over_ranks(timed(g), world, dev)  # every rank agrees on the count
+        reps = max(args.reps, min(1000, int(0.3e3 / max(first, 1e-3)) + 1))
+        times = [first] + max_over_ranks([timed(g) for _ in range(reps - 1)], world, dev)
+        return statistics.median(times), len(times)
+
+    with ClockSampler(local) as clk:
+        ms, nreps = repeat(graph)
     fmoe.workspace_check(ws, stream)
     per_step = nstack if nstack else (nbatch if nbatch else 1)  # layer-token steps per step
     value = steps * world * per_step / (ms / 1e3)
@@ -338,16 +350,7 @@ def main():
         with torch.cuda.stream(stream):
             egraph.replay()
         stream.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(steps // G):
-                egraph.replay()
-            e1.record(stream)
-        e1.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        ems, _ = repeat(egraph)
         bpt = spec.hidden * 4 * nb  # the step's hidden states in, its outputs out
         e2e = {"value": steps * world * per_step / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bpt,
                "d2h_bytes_per_step": bpt}
@@ -378,7 +381,7 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "reps": nreps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": DTYPE_BATCH if nbatch else DTYPE_TOKEN, "data": "synthetic",
             "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
                        "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": nb,

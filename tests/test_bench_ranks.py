@@ -23,7 +23,9 @@ def _worker(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        q.put((rank, bench.max_over_ranks(1.0 + 2.0 * rank, world, "cpu")))
+        one = bench.max_over_ranks(1.0 + 2.0 * rank, world, "cpu")
+        reps = bench.max_over_ranks([1.0 + rank, 5.0 - rank, 2.0], world, "cpu")
+        q.put((rank, one, reps))
     finally:
         dist.destroy_process_group()
 
@@ -36,11 +38,15 @@ def test_max_over_ranks_takes_the_slowest_rank():
     procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    got = dict(q.get(timeout=120) for _ in procs)
+    got = {}
+    for _ in procs:
+        r, one, reps = q.get(timeout=120)
+        got[r] = (one, reps)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert got == {0: 3.0, 1: 3.0}
+    # one time, and repetition by repetition (the bench's median runs over these)
+    assert got == {0: (3.0, [2.0, 5.0, 2.0]), 1: (3.0, [2.0, 5.0, 2.0])}
 
 
 def test_single_rank_returns_its_own_time():

@@ -131,8 +131,12 @@ def test_per_token_path_still_matches_oracle(fmoe, monkeypatch):
 
 @pytest.mark.parametrize("bits,zipf", [(4, 0.0), (2, 1.1)])
 def test_grouped_full_size_batch(fmoe, monkeypatch, bits, zipf):
-    """64 tokens of the Qwen3.5-397B-A17B-shaped layer: sampled tokens against the
-    oracle, every token against the per-token path."""
+    """64 tokens of the Qwen3.5-397B-A17B-shaped layer on the grouped path, every token
+    against the oracle: routing exact wherever the top K+1 logits are separated (at
+    least 60 of 64), outputs and out - h within 2e-3.  The oracle holds every record
+    that the GPU or the exact routing selects (about 200 at 4-bit), so each active
+    expert's work units, row items and K slices are compared."""
+    from tests.test_parity_gpu import full_size_oracle_layer
     spec = gen.qwen397_layer(bits, zipf=zipf)
     dl = gen.device_layer(spec, seed=0, layer=0)
     lay = gen.binding_layer(dl)
@@ -145,27 +149,17 @@ def test_grouped_full_size_batch(fmoe, monkeypatch, bits, zipf):
     ws = fmoe.workspace(fmoe.moe_layer_workspace_size(lay, T))
     fmoe.moe_layer(lay, h, out=out, topk_idx=idx, topk_w=w, ws=ws)
     fmoe.workspace_check(ws)
-    monkeypatch.setenv("FMOE_GROUPED", "0")
-    ref = torch.empty_like(h)
-    ref_idx = torch.empty_like(idx)
-    fmoe.moe_layer(lay, h, out=ref, topk_idx=ref_idx, ws=ws)
     torch.cuda.synchronize()
-    o, r = out.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64)
-    gi, ri = idx.cpu().numpy(), ref_idx.cpu().numpy()
-    same = np.all(gi == ri, axis=1)
-    assert same.sum() >= T - 2   # routing agrees except where a logit near-tie flips
-    h64 = h_np.astype(np.float64)
-    assert max_rel_err(o[same] - h64[same], r[same] - h64[same], slack=ulp32(o[same])) <= TOL
-    # sampled tokens against the oracle (drawing only the experts they need)
-    sample = [0, 17, 40, 63]
-    hl0 = gen.host_layer(spec, seed=0, layer=0, experts=[])
-    need = set(gi[sample].reshape(-1).tolist())
-    for t in sample:
-        x = oracle.rmsnorm(h_np[t], hl0.gamma, spec.eps)
-        logits, _ = routing_margin(hl0.w_router, x, hl0.logit_bias)
-        need |= set(np.argsort(-logits, kind="stable")[:K].tolist())
-    hl = gen.host_layer(spec, seed=0, layer=0, experts=sorted(need))
-    _compare_layer(hl, h_np[sample], o[sample].astype(np.float64), gi[sample],
-                   w.cpu().numpy()[sample].astype(np.float64), L=oracle_layer_sparse(hl))
+    o = out.cpu().numpy().astype(np.float64)
+    gi = idx.cpu().numpy()
+    hl, L = full_size_oracle_layer(spec, h_np, gi)
+    exact, _ = _compare_layer(hl, h_np, o, gi, w.cpu().numpy().astype(np.float64), L=L)
+    assert exact >= 60, exact
+    # the per-token path on the same batch: same routing where not near-tied (an extra check)
+    monkeypatch.setenv("FMOE_GROUPED", "0")
+    ref_idx = torch.empty_like(idx)
+    fmoe.moe_layer(lay, h, topk_idx=ref_idx, ws=ws)
+    torch.cuda.synchronize()
+    assert np.sum(np.all(gi == ref_idx.cpu().numpy(), axis=1)) >= T - 2
     del dl, lay
     torch.cuda.empty_cache()
