@@ -123,7 +123,7 @@ fmoe_status check_bank(const fmoe_bank* b, const char* name) {
   if (!pow2(H / 64) || H > 8192 || !pow2(I / 64) || I > 8192)
     return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden %d and inter %d must be 64 times a power of two, at most 8192",
                 name, H, I);
-  if (!expert_shapes_supported(b->bits, H, I, 1))
+  if (!expert_shapes_supported(b->bits, H, I, 1) || !plan_token(b->bits, H, I, 1, 0).ok)
     return fail(FMOE_ERR_UNSUPPORTED, "%s bank: shapes exceed the kernels' shared memory", name);
   if (!aligned16(b->base) || (b->stride & 15)) return fail(FMOE_ERR_ALIGNMENT, "%s bank: base/stride not 16-byte aligned", name);
   if (b->num_experts > 1 && b->stride <= 0) return fail(FMOE_ERR_INVALID_ARG, "%s bank: stride %lld", name, (long long)b->stride);
@@ -175,6 +175,12 @@ int prefetch_down() {
     on = (v && v[0] == '0') ? 0 : 1;
   }
   return on;
+}
+
+// TMA tensor-map staging in the per-token expert kernel; FMOE_TMA_MAPS=0 turns it off (bulk copies).
+bool token_maps_enabled() {
+  const char* v = getenv("FMOE_TMA_MAPS");
+  return !(v && v[0] == '0');
 }
 
 // Dependent launch between the block's kernels; FMOE_PDL=0 in the environment turns it off.
@@ -237,6 +243,13 @@ fmoe_status fmoe_rmsnorm(const float* h, const float* gamma, float eps, int T, i
   if (!(eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)eps);
   cudaError_t e = launch_rmsnorm(h, gamma, eps, T, H, y, cs(stream));
   return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "rmsnorm launch");
+}
+
+// The per-token path: three kernels (router, gate/up, down) unless FMOE_TOKEN_KERNELS=2
+// selects the two-kernel path (router, fused expert kernel).
+static bool three_kernel_path() {
+  const char* v = getenv("FMOE_TOKEN_KERNELS");
+  return !(v && v[0] == '2');
 }
 
 size_t fmoe_router_topk_workspace_size(int T, int E) {
@@ -307,6 +320,29 @@ fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, f
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
   const int bits = bank->bits;
+  if (!three_kernel_path()) {
+    const bool pdl = pdl_enabled();
+    cudaError_t e = launch_tok_xq(x, bank->hidden, bits, base + L.xq_limbs, reinterpret_cast<float2*>(base + L.xq_cs),
+                                  &ctrl->tok_count, pdl, cs(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "digits launch");
+    TokExpertParams p{};
+    p.routed = ref(*bank);
+    p.shared = ref(*bank);
+    p.fixed_expert = expert;
+    p.E = bank->num_experts;
+    p.K = 1;
+    p.has_shared = 0;
+    p.H = bank->hidden;
+    p.I = bank->inter;
+    p.xq_limbs = base + L.xq_limbs;
+    p.xq_cs = reinterpret_cast<const float2*>(base + L.xq_cs);
+    p.act = reinterpret_cast<float*>(base + L.act);
+    p.count = &ctrl->tok_count;
+    p.out = y;
+    p.err = &ctrl->err;
+    if ((e = launch_tok_expert(p, bits, pdl, cs(stream))) != cudaSuccess) return cuda_fail(e, "expert launch");
+    return FMOE_OK;
+  }
   cudaError_t e = launch_xq(x, bank->hidden, bits, base + L.xq_limbs, reinterpret_cast<float2*>(base + L.xq_cs),
                             cs(stream));
   if (e != cudaSuccess) return cuda_fail(e, "digits launch");
@@ -351,7 +387,7 @@ static fmoe_status check_layer(const fmoe_layer* layer) {
   if (E > 4096) return fail(FMOE_ERR_UNSUPPORTED, "E %d > 4096", E);
   if (r.hidden > 12288) return fail(FMOE_ERR_UNSUPPORTED, "hidden %d > 12288", r.hidden);
   if (K < 1 || K > E || K > 32) return fail(FMOE_ERR_INVALID_ARG, "top_k %d (1..min(E, 32))", K);
-  if (!expert_shapes_supported(r.bits, r.hidden, r.inter, K + 1))
+  if (!expert_shapes_supported(r.bits, r.hidden, r.inter, K + 1) || !plan_token(r.bits, r.hidden, r.inter, K, 1).ok)
     return fail(FMOE_ERR_UNSUPPORTED, "top_k %d with inter %d at %d bits exceeds the down kernel's shared memory", K,
                 r.inter, r.bits);
   if (!(layer->eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)layer->eps);
@@ -369,10 +405,67 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
   return need;
 }
 
-// One token through the block: router (+RMSNorm, digits, top-K) -> gate/up -> down + combine.
+static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
+                                  uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word);
+
+// One token through the block: router kernel (RMSNorm, logits, digits of x), then
+// the expert kernel (top-K, gate/up + SwiGLU, down + combine + residual).
 // err_word: where the kernels report a failed bounded wait; NULL means the workspace's own error word.
 static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
                                uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word = nullptr) {
+  if (three_kernel_path()) return layer_token_3k(layer, h, out, idx_out, w_out, base, L, s, err_word);
+  const fmoe_bank& r = layer->routed;
+  const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
+  WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
+  TokRouterParams rp{};
+  rp.h = h;
+  rp.gamma = layer->gamma;
+  rp.eps = layer->eps;
+  rp.norm = layer->gamma != nullptr;
+  rp.w_router = layer->w_router;
+  rp.bias = layer->router_bias;
+  rp.w_sgate = layer->w_shared_gate;
+  rp.H = H;
+  rp.E = E;
+  rp.row0 = 0;
+  rp.xq_limbs = base + L.xq_limbs;
+  rp.xq_cs = reinterpret_cast<float2*>(base + L.xq_cs);
+  rp.logits = reinterpret_cast<float*>(base + L.logits);
+  rp.count = &ctrl->tok_count;
+  rp.err = err_word ? err_word : &ctrl->err;
+  const bool trace = g_trace_on;
+  g_trace_on = false;
+  const bool pdl = pdl_enabled() && !trace;
+  cudaError_t e;
+  if (trace && (e = trace_record(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if ((e = launch_tok_router(rp, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "router launch");
+  if (trace && (e = trace_record(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  TokExpertParams p{};
+  p.routed = ref(r);
+  p.shared = ref(layer->shared);
+  p.logits = rp.logits;
+  p.idx_out = idx_out;
+  p.w_out = w_out;
+  p.E = E;
+  p.K = K;
+  p.has_shared = 1;
+  p.H = H;
+  p.I = I;
+  p.xq_limbs = base + L.xq_limbs;
+  p.xq_cs = reinterpret_cast<const float2*>(base + L.xq_cs);
+  p.act = reinterpret_cast<float*>(base + L.act);
+  p.count = &ctrl->tok_count;
+  p.resid = h;
+  p.out = out;
+  p.err = rp.err;
+  if ((e = launch_tok_expert(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "expert launch");
+  if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if (trace && (e = trace_record(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  return FMOE_OK;
+}
+
+static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
+                                  uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word) {
   const fmoe_bank& r = layer->routed;
   const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);

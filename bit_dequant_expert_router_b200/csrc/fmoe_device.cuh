@@ -21,8 +21,11 @@ struct WsControl {
   unsigned int route_ready;    // three-kernel path: 1 once the gate/up kernel has published this token's routing
   unsigned int pad0[30];
   int err;                     // nonzero once a bounded wait gave up
-  int pad[63];
+  int pad[31];
+  unsigned int tok_count;      // per-token path: expert-kernel CTAs whose activations are written
+  unsigned int pad1[31];       // (its own 128-byte line; cleared by the first kernel of each token)
 };
+constexpr int kMaxTokenCtas = 256;
 
 // ------------------------------------------------------------------------------------------ small helpers
 
@@ -34,11 +37,24 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
   return v;
 }
 
+__device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Barrier `id` (1..15) over the first `n` threads of the block (n a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
@@ -114,6 +130,45 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
   }
 }
+
+// Waits until *flag == value (acquire, gpu scope), at most limit_ns; on timeout
+// records the error and returns false.
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned int* flag, unsigned int value, unsigned long long limit_ns,
+                                                  int* err) {
+  if (ld_acquire_gpu(flag) == value) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (ld_acquire_gpu(flag) == value) return true;
+    if (global_ns() - t0 > limit_ns) {
+      atomicExch(err, kDevTimeout);
+      return false;
+    }
+  }
+}
+
+// One thread waits until *count >= target (relaxed reads with a short sleep between
+// them, then one acquire fence), at most kWaitNs; on timeout records the error and
+// returns false.  One thread per CTA polls one word, so waiting CTAs do not flood L2.
+__device__ __forceinline__ bool count_wait_bounded(const unsigned int* count, unsigned int target, int* err) {
+  unsigned long long t0 = 0;
+  for (int round = 0;; ++round) {
+    if (ld_relaxed_gpu(count) >= target) {
+      fence_acq_rel_gpu();
+      return true;
+    }
+    if (round == 0) t0 = global_ns();
+    else if (global_ns() - t0 > kWaitNs) {
+      atomicExch(err, kDevTimeout);
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
+// Asks L1 for the 128-byte line holding p.
+__device__ __forceinline__ void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
@@ -330,6 +385,18 @@ __device__ __forceinline__ void load_group_limbs(const uint32_t* src, int g, int
   }
 }
 
+// load_group_limbs from global memory (through L2: the digits are written by the previous kernel).
+__device__ __forceinline__ void load_group_limbs_global(const uint32_t* src, int g, int NG, uint32_t (&L)[48]) {
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src) + i * NG + g);
+    L[4 * i] = v.x;
+    L[4 * i + 1] = v.y;
+    L[4 * i + 2] = v.z;
+    L[4 * i + 3] = v.w;
+  }
+}
+
 // Order-preserving key of (logit, index): larger value first, then lower index.
 __device__ __forceinline__ unsigned long long topk_key(float v, int e) {
   uint32_t u = __float_as_uint(v);
@@ -464,6 +531,15 @@ __device__ __forceinline__ float2 group_scalars(const float2* cs, int g) {
     return make_float2(a.x, a.y + b.y);
   }
   return cs[g];
+}
+
+template <int BITS>
+__device__ __forceinline__ float2 group_scalars_global(const float2* cs, int g) {
+  if (BITS == 4) {
+    const float2 a = __ldcg(cs + 2 * g), b = __ldcg(cs + 2 * g + 1);
+    return make_float2(a.x, a.y + b.y);
+  }
+  return __ldcg(cs + g);
 }
 
 // Block-wide top-K of logits [E] (E <= 8 * 64) with 256 threads, in two stages.

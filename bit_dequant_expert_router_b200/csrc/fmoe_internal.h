@@ -190,6 +190,62 @@ struct FusedPlan {
 FusedPlan plan_fused(int bits, int H, int I, int E, int K);
 cudaError_t launch_fused(const FusedParams& p, const FusedPlan& pl, int bits, bool pdl, cudaStream_t s);
 
+// ---- per-token path (k_token.cu): a router kernel and one expert kernel per token
+
+struct TokRouterParams {
+  const float* h;             // [H] the block's input
+  const float* gamma;         // [H] RMSNorm weight, or NULL
+  float eps;
+  int norm;                   // 1: x = RMSNorm(h); 0: x = h
+  const uint16_t* w_router;   // bf16 [E][H]
+  const float* bias;          // [E] or NULL
+  const uint16_t* w_sgate;    // bf16 [H]: row E of the router's output
+  int H, E;
+  int row0;                   // first output row: 0, or E (the shared-gate row alone)
+  int rpc;                    // rows per CTA (set by the launcher)
+  uint8_t* xq_limbs;          // digits of x for the expert kernel
+  float2* xq_cs;
+  float* logits;              // [E + 1]
+  unsigned int* count;        // the expert kernel's arrival counter, cleared once per token
+  int* err;
+};
+
+struct TokExpertParams {
+  BankRef routed, shared;
+  const float* logits;        // [E + 1]: the routing is the top-K of logits[0, E) unless route_idx is
+                              // given; sigma = sigmoid(logits[E])
+  const int32_t* route_idx;   // [K] given routing, or NULL
+  const float* route_w;       // [K] given weights, or NULL (weight 1)
+  int fixed_expert;           // the routing when logits and route_idx are both NULL (K = 1)
+  int32_t* idx_out;           // the caller's copy of the routing [K] (CTA 0), or NULL
+  float* w_out;
+  int E, K, has_shared, H, I;
+  const uint8_t* xq_limbs;    // digits of x
+  const float2* xq_cs;
+  float* act;                 // [K + has_shared][I] SwiGLU activations, exchanged between CTAs
+  unsigned int* count;        // CTAs whose activations are written (cleared by the kernel before this one)
+  const float* resid;         // [H] residual, or NULL
+  float* out;                 // [H]
+  int* err;
+  // set by the launcher
+  int gmax_s, gmax_r, dmax;   // units per shared / routed gate/up chunk, per down range
+  int xd_bytes, ring_bytes;   // shared-memory regions
+  int use_maps;               // stage by TMA tensor copies (else bulk copies)
+};
+
+struct TokPlan {
+  bool ok;
+  int grid, gmax_s, gmax_r, dmax, xd_bytes, ring_bytes, dppl;
+  size_t smem;
+};
+
+TokPlan plan_token(int bits, int H, int I, int K, int has_shared);
+cudaError_t launch_tok_router(TokRouterParams p, int bits, bool pdl, cudaStream_t s);
+cudaError_t launch_tok_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, unsigned int* count, bool pdl,
+                          cudaStream_t s);
+bool token_maps_enabled();
+cudaError_t launch_tok_expert(TokExpertParams p, int bits, bool pdl, cudaStream_t s);
+
 cudaError_t launch_rmsnorm(const float* h, const float* gamma, float eps, int T, int H, float* y, cudaStream_t s);
 cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, cudaStream_t s);
 cudaError_t launch_router(RouterParams p, int xq_bits, bool pdl, cudaStream_t s);
@@ -201,6 +257,7 @@ int num_sms();
 bool expert_shapes_supported(int bits, int H, int I, int num_slots);
 bool pdl_enabled();
 cudaError_t set_smem(const void* kernel, size_t bytes);
+cudaError_t set_carveout_max(const void* kernel);
 
 // Launch with optional programmatic stream serialisation (dependent launch).
 template <typename... Exp, typename... Act>

@@ -590,6 +590,28 @@ cudaError_t down_bits(const ExpertParams& p, bool pdl, cudaStream_t s) {
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
 // again only if a larger size is asked for, so that launches captured into a
 // CUDA graph make no attribute call.
+// Asks for the largest shared-memory carveout for a kernel, once per (kernel, device):
+// kernels that sit on an SM together under dependent launch must run with the same
+// carveout, else the later one waits for the SM to drain before it can start there.
+cudaError_t set_carveout_max(const void* kernel) {
+  static const void* done[64][32] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  for (const void*& k : done[dev]) {
+    if (k == kernel) return cudaSuccess;
+    if (k == nullptr) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e == cudaSuccess) k = kernel;
+      return e;
+    }
+  }
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+}
+
 cudaError_t set_smem(const void* kernel, size_t bytes) {
   struct Entry {
     const void* fn;

@@ -1,0 +1,1026 @@
+// k_token.cu -- the MoE block for one token: a router kernel and one expert kernel.
+//
+// What is computed follows the Flash-MoE pages: "What is Flash-MoE"
+// (a2a-mcp.org), MoE section (4 of 512 routed experts + one shared expert per
+// layer), section 2 (group-wise affine codes, weight = code * scale + bias),
+// section 3 (two-pass RMSNorm, fused SwiGLU, one combine pass of the weighted
+// experts, the residual and the sigmoid-gated shared expert); the "Flash-MoE"
+// wiki summary (jeongsk), per-layer pipeline (routing projection, softmax,
+// top-K).
+//
+// tok_router_kernel: every CTA stages its rows of [W_r; w_sg] before the
+// dependency wait, then computes sum(h^2) and its rows' dot products with
+// gamma * h in one pass over h (the first pass of the RMSNorm), so that a
+// logit is rsqrt(mean(h^2) + eps) * (w . (gamma * h)); the second pass
+// applies the scale to the groups of x whose digits this CTA writes.  Its
+// shared memory is small, so that under programmatic dependent launch its
+// CTAs sit beside the previous token's expert kernel and their row copies
+// overlap it.
+//
+// tok_expert_kernel: one CTA per SM, eight consumer warps and one producer
+// warp.  Every CTA selects the experts from the logits itself (block-wide
+// top-K), computes an equal share of the shared expert's and of the routed
+// experts' gate/up rows (SwiGLU activations out to global memory), publishes
+// that by an epoch-tagged flag, waits for every CTA's flag, turns all
+// activations into digits, and computes its share of the output rows: down
+// projection of every slot, weighted sum, sigma * shared, residual.  The
+// producer streams the CTA's rows through a byte ring of shared memory with
+// bulk copies (TMA engine): one chunk = a row range of one slot's gate and up
+// (six copies) or of every slot's down matrix (three copies per slot); each
+// chunk completes on its own "full" mbarrier and is handed back by the
+// consumer warps on its "empty" mbarrier, so no block-wide barrier sits in the
+// stream.  The shared expert's rows are requested before the dependency wait,
+// the routed rows as soon as the routing is known, and the routed down rows
+// are asked of L2 right after, to be copied into the ring as gate/up chunks
+// free it.
+//
+// Dot products: sum_c (q_c s + b) x_c = s * sum_c q_c X_c * cscale + b * sum_c x_c
+// per group of 64, with the integer sum on dp4a against 24-bit fixed-point
+// digits of x (fmoe_device.cuh).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "fmoe_internal.h"
+
+namespace fmoe {
+namespace {
+
+// ------------------------------------------------------------------------------------------ router
+
+constexpr int kRtThreads = 128;
+constexpr int kRtMaxRows = 8;
+constexpr int kRtSmemBudget = 32 * 1024;  // rows of the router per CTA, bf16
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// grid (ceil((E + 1 - row0) / rpc)): CTA b computes rows [row0 + b*rpc, +rpc) of [W_r; w_sg]
+// (row E is the shared-gate vector), and the digits of groups b, b + grid, .. of x.
+// kRtMaxF4: float4s of h per thread (H <= kRtMaxF4 * 512).
+template <int BITS, int kRtMaxF4>
+__global__ void __launch_bounds__(kRtThreads) tok_router_kernel(const TokRouterParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ float s_red[kRtThreads / 32][kRtMaxRows + 1];
+  __shared__ __align__(16) float s_x[kRtThreads / 32][kGroup];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = p.H, E = p.E;
+  const int r0 = p.row0 + blockIdx.x * p.rpc;
+  const int nrows = max(0, min(p.rpc, E + 1 - r0));
+  const uint32_t bar = smem_addr(&s_bar);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+    if (nrows > 0) {  // weights: staged before the dependency wait
+      const int nr = max(0, min(nrows, E - r0));  // routed rows; the rest is the shared-gate row
+      const uint64_t pol = l2_policy_evict_first();
+      mbar_expect_tx(bar, (uint32_t)nrows * H * 2);
+      if (nr > 0) bulk_g2s(smem_addr(sm), p.w_router + (size_t)r0 * H, (uint32_t)nr * H * 2, bar, pol);
+      if (nr < nrows) bulk_g2s(smem_addr(sm + (size_t)nr * H * 2), p.w_sgate, (uint32_t)H * 2, bar, pol);
+    }
+  }
+  // pass 1: sum of squares of h, and each row's dot product with gamma * h.  Every
+  // load is issued before any is used (a use waits for its load, and a warp issues in
+  // order); columns past H read a clamped address and count 0.  gamma is a weight:
+  // loaded before the wait.
+  float4 hv[kRtMaxF4], gv[kRtMaxF4];
+  if (p.gamma) {
+#pragma unroll
+    for (int j = 0; j < kRtMaxF4; ++j)
+      gv[j] = __ldg(reinterpret_cast<const float4*>(p.gamma + min((tid + j * kRtThreads) * 4, H - 4)));
+  } else {
+#pragma unroll
+    for (int j = 0; j < kRtMaxF4; ++j) gv[j] = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+  }
+  __syncthreads();
+  pdl_wait();  // h may be the previous kernel's output
+  const float* h = p.h;
+#pragma unroll
+  for (int j = 0; j < kRtMaxF4; ++j)
+    hv[j] = __ldcg(reinterpret_cast<const float4*>(h + min((tid + j * kRtThreads) * 4, H - 4)));
+  pdl_trigger();  // after the loads of h, so that they go out before the next kernel's weight copies
+  if (blockIdx.x == 0 && tid == 0) *p.count = 0u;  // every kernel of the previous token is complete
+  float ss = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kRtMaxF4; ++j) {
+    if ((tid + j * kRtThreads) * 4 >= H) hv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    ss = fmaf(hv[j].x, hv[j].x, ss);
+    ss = fmaf(hv[j].y, hv[j].y, ss);
+    ss = fmaf(hv[j].z, hv[j].z, ss);
+    ss = fmaf(hv[j].w, hv[j].w, ss);
+  }
+  float acc[kRtMaxRows];
+#pragma unroll
+  for (int r = 0; r < kRtMaxRows; ++r) acc[r] = 0.0f;
+  const bool ready = nrows == 0 || mbar_wait_bounded(bar, 0, p.err);
+  if (ready) {
+    const uint16_t* wr = reinterpret_cast<const uint16_t*>(sm);
+#pragma unroll
+    for (int j = 0; j < kRtMaxF4; ++j) {
+      const int cc = min((tid + j * kRtThreads) * 4, H - 4);  // columns past H: v is 0 there
+      const float4 g = gv[j];
+      const float4 v = make_float4(hv[j].x * g.x, hv[j].y * g.y, hv[j].z * g.z, hv[j].w * g.w);
+#pragma unroll
+      for (int r = 0; r < kRtMaxRows; ++r) {
+        if (r < nrows) {
+          const uint2 w = *reinterpret_cast<const uint2*>(wr + (size_t)r * H + cc);
+          float a = acc[r];
+          a = fmaf(bf_lo(w.x), v.x, a);
+          a = fmaf(bf_hi(w.x), v.y, a);
+          a = fmaf(bf_lo(w.y), v.z, a);
+          a = fmaf(bf_hi(w.y), v.w, a);
+          acc[r] = a;
+        }
+      }
+    }
+  }
+  ss = warp_sum(ss);
+#pragma unroll
+  for (int r = 0; r < kRtMaxRows; ++r)
+    if (r < nrows) acc[r] = warp_sum(acc[r]);
+  if (lane == 0) {
+    s_red[warp][kRtMaxRows] = ss;
+#pragma unroll
+    for (int r = 0; r < kRtMaxRows; ++r) s_red[warp][r] = acc[r];
+  }
+  __syncthreads();
+  float sst = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kRtThreads / 32; ++w) sst += s_red[w][kRtMaxRows];  // same order in every CTA
+  const float rstd = p.norm ? 1.0f / sqrtf(sst / (float)H + p.eps) : 1.0f;
+  if (ready && tid < nrows) {
+    float d = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kRtThreads / 32; ++w) d += s_red[w][tid];
+    const int row = r0 + tid;
+    p.logits[row] = fmaf(rstd, d, (row < E && p.bias) ? p.bias[row] : 0.0f);
+  }
+  // pass 2: x = h * rstd * gamma for the groups whose digits this CTA writes (group b,
+  // b + grid, ..), from the registers of pass 1: thread tid holds columns
+  // 4 tid + 512 j, i.e. elements 4 (tid % 16) .. + 3 of group tid / 16 + 8 j.  Up to
+  // four groups per round are staged in shared memory, then one warp digitises each.
+  const int NG = H / kGroup;
+  for (int g0 = blockIdx.x; g0 < NG; g0 += gridDim.x * (kRtThreads / 32)) {
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kRtThreads / 32; ++w) {
+      const int g = g0 + gridDim.x * w;
+      if (g < NG && tid / 16 == g % 8) {
+#pragma unroll
+        for (int j = 0; j < kRtMaxF4; ++j)
+          if (j == g / 8) {
+            const float4 hx = hv[j], gx = gv[j];
+            *reinterpret_cast<float4*>(&s_x[w][4 * (tid % 16)]) =
+                make_float4(hx.x * rstd * gx.x, hx.y * rstd * gx.y, hx.z * rstd * gx.z, hx.w * rstd * gx.w);
+          }
+      }
+    }
+    __syncthreads();
+    const int g = g0 + gridDim.x * warp;
+    if (g < NG) {
+      const float2 v = *reinterpret_cast<const float2*>(&s_x[warp][2 * lane]);
+      xq_quantize_group<BITS>(v.x, v.y, g, NG, p.xq_limbs, p.xq_cs);
+    }
+  }
+}
+
+// Digits of a given x (the single-expert entry point); one warp per group.  CTA 0
+// clears the expert kernel's arrival counter, as the router kernel does.
+template <int BITS>
+__global__ void __launch_bounds__(kRtThreads) tok_xq_kernel(const float* __restrict__ x, int H, uint8_t* limbs,
+                                                           float2* cs, unsigned int* count) {
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *count = 0u;
+  const int g = blockIdx.x * (kRtThreads / 32) + (threadIdx.x >> 5);
+  if (g >= H / kGroup) return;  // warp-uniform
+  const float2 v = __ldcg(reinterpret_cast<const float2*>(x + g * kGroup) + (threadIdx.x & 31));
+  xq_quantize_group<BITS>(v.x, v.y, g, H / kGroup, limbs, cs);
+}
+
+// ------------------------------------------------------------------------------------------ expert kernel
+
+constexpr int kXWarps = 8;                     // consumer warps
+constexpr int kXThreads = (kXWarps + 1) * 32;  // + the producer warp
+constexpr int kXSlots = 48;                    // chunks in flight at most (barrier pairs); >= 33 + a few
+constexpr int kBarCons = 1;                    // named barrier of the consumer warps
+constexpr int kBarAll = 2;                     // named barrier of consumers + producer
+constexpr int kXMaxDRows = 128;                // output rows per down range
+constexpr int kMaxSlots = 33;                  // K + shared
+constexpr size_t kXSmemBudget = 184 * 1024;    // dynamic shared memory of the expert kernel
+constexpr size_t kXChunkTarget = 32 * 1024;    // bytes per gate/up chunk, about
+
+// The tensor maps of the staged arrays, [0] the routed bank, [1] the shared expert:
+//   gu_codes  (RB / 8 u64, I rows, {gate, up}, experts)           box (RB / 8, gbox, 2, 1)
+//   gu_sb     (SB / 8 u64, I rows, {scale, bias}, {gate, up}, experts) box (SB / 8, gbox, 2, 2, 1)
+//   dn_codes  (RBD / 8 u64, H rows, experts)                     box (RBD / 8, dbox, 1)
+//   dn_sb     (SBD / 8 u64, H rows, {scale, bias}, experts)       box (SBD / 8, dbox, 2, 1)
+// A box lands as [outer dims][rows][row bytes]: for gate/up gate rows then up rows,
+// then gate scales, gate biases, up scales, up biases, which is the chunk layout below.
+struct TokMaps {
+  CUtensorMap gu_codes[2];
+  CUtensorMap gu_sb[2];
+  CUtensorMap dn_codes[2];
+  CUtensorMap dn_sb[2];
+};
+
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, int c1, int c2, uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap* m, int c1, int c2, int c3, uint32_t bar,
+                                       uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_5d(uint32_t dst, const CUtensorMap* m, int c1, int c2, int c3, int c4, uint32_t bar,
+                                       uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+// Block-wide top-K of logits [E] by the 256 consumer threads (E <= 1024), in two
+// stages: each warp's K largest keys of its logits e = tid + 256 i into cand,
+// then warp 0 the K largest candidates, the renormalised weights
+// w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0) and, with has_gate, w[K] =
+// sigmoid(logits[E]).  Keys order by value, then lower index: one sort's result.
+// Larger E: warp 0 alone (rescans).  Ends before the caller's next barrier.
+__device__ __forceinline__ void consumer_topk(const float* logits, int E, int K, int has_gate, unsigned long long* cand,
+                                              int* idx, float* w) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (E > 1024) {
+    if (warp == 0) {
+      int ik;
+      float wk, sig;
+      warp_topk(logits, E, K, has_gate, ik, wk, sig);
+      if (lane < K) {
+        idx[lane] = ik;
+        w[lane] = wk;
+      }
+      if (lane == 0) w[K] = sig;
+    }
+    return;
+  }
+  // every load first (clamped index), then the keys: a use waits for its load
+  const float zg = __ldcg(logits + E);
+  float lv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lv[i] = __ldcg(logits + min(tid + 256 * i, E - 1));
+  unsigned long long key[4], best = 0ull;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + 256 * i;
+    key[i] = e < E ? topk_key(lv[i], e) : 0ull;
+    best = key[i] > best ? key[i] : best;
+  }
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    const unsigned long long m = warp_max_key(best);
+    if (lane == 0) cand[warp * K + k] = m;
+    if (best == m && m != 0ull) {
+      best = 0ull;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        key[i] = key[i] == m ? 0ull : key[i];
+        best = key[i] > best ? key[i] : best;
+      }
+    }
+  }
+  named_bar_sync(kBarCons, kXWarps * 32);
+  if (warp != 0) return;
+  const int NC = kXWarps * K;  // candidates, <= 256
+  unsigned long long ck[8];
+  best = 0ull;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    ck[i] = lane + 32 * i < NC ? cand[lane + 32 * i] : 0ull;
+    best = ck[i] > best ? ck[i] : best;
+  }
+  float top = 0.0f, mine = 0.0f;
+  int mi = 0;
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    const unsigned long long m = warp_max_key(best);
+    int e = m ? topk_key_index(m) : 0;
+    const float v = topk_key_value(m);
+    if (e < 0 || e >= E) e = 0;  // only with non-finite logits
+    if (k == 0) top = v;
+    if (lane == k) {
+      mi = e;
+      mine = v;
+    }
+    if (best == m && m != 0ull) {
+      best = 0ull;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ck[i] = ck[i] == m ? 0ull : ck[i];
+        best = ck[i] > best ? ck[i] : best;
+      }
+    }
+  }
+  const float ek = lane < K ? expf(mine - top) : 0.0f;
+  const float wk = ek / warp_sum(ek);
+  if (lane < K) {
+    idx[lane] = mi;
+    w[lane] = wk;
+  }
+  if (lane == 0) w[K] = has_gate ? 1.0f / (1.0f + expf(-zg)) : 0.0f;
+}
+
+// The CTA's work ranges, in units: shared-expert gate/up units [sh0, sh1) (a unit =
+// RPP rows of gate and of up), routed gate/up units [rt0, rt1) over the K slots
+// concatenated (ups units per slot), output-row units [d0, d1) (a unit = DR rows).
+struct Ranges {
+  int sh0, sh1, rt0, rt1, d0, d1;
+};
+
+// A gate/up chunk: n units of one slot (K = the shared expert), from unit u0 of the slot.
+struct GChunk {
+  int slot, u0, n;
+};
+
+// The CTA's gate/up chunks in order: the shared expert's, then the routed ones
+// (never across a slot).
+struct GChunkIt {
+  int phase, u;
+  __device__ __forceinline__ explicit GChunkIt(const Ranges& r) : phase(0), u(r.sh0) {}
+  __device__ __forceinline__ bool next(GChunk& c, const Ranges& r, int K, int ups, int gmax_s, int gmax_r) {
+    if (phase == 0) {
+      if (u < r.sh1) {
+        c = GChunk{K, u, min(gmax_s, r.sh1 - u)};
+        u += c.n;
+        return true;
+      }
+      phase = 1;
+      u = r.rt0;
+    }
+    if (phase == 1 && u < r.rt1) {
+      const int sl = u / ups, ui = u - sl * ups;
+      c = GChunk{sl, ui, min(gmax_r, min(r.rt1 - u, ups - ui))};
+      u += c.n;
+      return true;
+    }
+    phase = 2;
+    return false;
+  }
+};
+
+// Down chunk jd of the CTA: output-row range jd / NE (rows [d0*DR + range*dbox, +dbox),
+// clipped to the CTA's rows), slot order within a range: the shared expert first.
+__device__ __forceinline__ int down_slot(int pos, int K, int has_shared) {
+  return has_shared ? (pos == 0 ? K : pos - 1) : pos;
+}
+
+// Ring placement: a chunk takes the virtual byte range [vs, vs + len), vs the end of
+// the previous chunk padded so that the chunk never wraps; its buffer is
+// ring + vs % RING.  Placement depends on the lengths only, so producer and
+// consumers replay it alike.
+struct RingPos {
+  uint32_t vhead = 0;
+  __device__ __forceinline__ uint32_t place(uint32_t len, uint32_t RING) {
+    uint32_t vs = vhead;
+    if (vs % RING + len > RING) vs = (vs / RING + 1) * RING;
+    vhead = vs + len;
+    return vs;
+  }
+};
+
+// A producer's view of one ring: chunk j uses barrier pair j % NS, and may be issued
+// once chunk j - NS is handed back and every older chunk still in use starts at most
+// RING bytes before its end.  Every producer lane keeps the same state.
+template <int NS>
+struct RingProd {
+  RingPos rp;
+  uint32_t vstart[NS] = {};
+  int tail = 0, j = 0;
+  uint32_t RING;
+  uint64_t* empty;
+  // Places a chunk of len bytes; with may_wait false gives up (returns false) instead of
+  // waiting; ok turns false when a wait runs out.
+  __device__ __forceinline__ bool reserve(uint32_t len, bool may_wait, uint32_t& vs, bool& ok, int* err) {
+    RingPos trial = rp;
+    vs = trial.place(len, RING);
+    while (tail < j && (tail <= j - NS || vs + len > vstart[tail % NS] + RING)) {
+      if (!may_wait) return false;
+      if (!mbar_wait_bounded(smem_addr(&empty[tail % NS]), (uint32_t)((tail / NS) & 1), err)) {
+        ok = false;
+        return false;
+      }
+      ++tail;
+    }
+    rp = trial;
+    vstart[j % NS] = vs;
+    return true;
+  }
+};
+
+template <int BITS, int NG>
+struct XCfg {
+  using G = Geo<NG>;
+  static constexpr int kLPR = G::kLanesPerRow, kRPP = G::kRowsPerPass, kGPL = G::kGroupsPerLane;
+  static constexpr bool kRegDigits = kGPL <= 2;  // this lane's digits of x in registers (else read per group)
+  static constexpr int kRB = NG * kGroup * BITS / 8;  // bytes of codes per gate/up row
+  static constexpr int kSB = NG * 2;                 // bytes of scales per gate/up row
+  static constexpr int kXChunks = NG * kGroup * BITS / 128;
+  static constexpr int kXDigitBytes = NG * kGroupWords * 4;
+};
+
+// Staged layouts.  Gate/up chunk (box of gbox rows): gate codes [gbox][RB] | up codes |
+// gate s [gbox][SB] | gate b | up s | up b.  Down chunk (one slot, dbox rows): codes
+// [dbox][RBD] | s [dbox][SBD] | b [dbox][SBD], each part 128-byte aligned.
+__device__ __forceinline__ uint32_t r128(uint32_t v) { return (v + 127u) & ~127u; }
+
+template <int BITS, int NG, int DPPL>
+__global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExpertParams p,
+                                                                  const __grid_constant__ TokMaps maps) {
+  using C = XCfg<BITS, NG>;
+  constexpr int LPR = C::kLPR, RPP = C::kRPP, GPL = C::kGPL;
+  constexpr int RB = C::kRB, SB = C::kSB;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t s_full[kXSlots], s_empty[kXSlots];
+  __shared__ __align__(8) uint64_t s_xbar;
+  __shared__ int s_idx[32];
+  __shared__ float s_w[kMaxSlots];
+  __shared__ unsigned long long s_cand[kXWarps * 32];
+  __shared__ float s_dpart[2][kXMaxDRows];
+  __shared__ int s_abort;
+  __shared__ int s_issued;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = p.K, NE = K + p.has_shared, H = p.H, I = p.I;
+  const int NGD = I / kGroup;
+  const int ups = I / RPP;                        // gate/up units per slot
+  const int DR = NGD >= 8 ? 1 : 8 / NGD;          // output rows per down unit (16-byte scale copies)
+  const int RBD = I * BITS / 8, SBD = NGD * 2;     // bytes of codes / scales per down row
+  const int chD = I * BITS / 128;                  // digit chunk scalars per slot
+  const int dbox = p.dmax * DR;
+  // a gate/up chunk's box: gmax_s units for the shared expert, gmax_r for the routed ones
+  auto gbox_of = [&](int slot) { return (slot < K ? p.gmax_r : p.gmax_s) * RPP; };
+  auto glen_of = [&](int gbox) { return r128(2u * gbox * RB) + 4u * r128((uint32_t)gbox * SB); };
+  const uint32_t dcode = r128((uint32_t)dbox * RBD), dsb = r128((uint32_t)dbox * SBD);
+  const uint32_t dlen = dcode + 2 * dsb;
+  const int G = gridDim.x, b = blockIdx.x;
+  Ranges rg;
+  {
+    const int US = p.has_shared ? ups : 0, UR = K * ups, UD = H / DR;
+    rg.sh0 = (int)((long long)b * US / G);
+    rg.sh1 = (int)((long long)(b + 1) * US / G);
+    rg.rt0 = (int)((long long)b * UR / G);
+    rg.rt1 = (int)((long long)(b + 1) * UR / G);
+    rg.d0 = (int)((long long)b * UD / G);
+    rg.d1 = (int)((long long)(b + 1) * UD / G);
+  }
+  const int drows_all = (rg.d1 - rg.d0) * DR;                // this CTA's output rows
+  const int nranges = (drows_all + dbox - 1) / dbox;
+  const int nd = nranges * NE;                               // down chunks (one per slot and row range)
+  uint8_t* xd = sm;                                          // digits of x, then of the activations
+  uint8_t* ring = sm + p.xd_bytes;
+  const uint32_t RING = (uint32_t)p.ring_bytes;
+
+  if (tid == 0) {
+    for (int i = 0; i < kXSlots; ++i) {
+      mbar_init(smem_addr(&s_full[i]), 1);
+      mbar_init(smem_addr(&s_empty[i]), kXWarps);
+    }
+    mbar_init(smem_addr(&s_xbar), 1);
+    mbar_fence_init();
+    s_abort = 0;
+    s_issued = 0;
+  }
+  __syncthreads();
+
+  if (warp == kXWarps) {
+    // ================================================================ producer warp
+    // One ring, chunks in order: the gate/up chunks (shared expert, then routed), then
+    // the down chunks (per row range, one per slot, the shared expert's first).
+    const uint64_t pol = l2_policy_evict_first();
+    bool ok = true;
+    RingProd<kXSlots> rpr;
+    rpr.RING = RING;
+    rpr.empty = s_empty;
+    GChunkIt git(rg);
+    GChunk gc;
+    bool ghave = git.next(gc, rg, K, ups, p.gmax_s, p.gmax_r);
+    auto issue_g = [&](const GChunk& c, uint32_t vs) {
+      const uint32_t d = smem_addr(ring + vs % RING);
+      const uint32_t bar = smem_addr(&s_full[rpr.j % kXSlots]);
+      const int rows = c.n * RPP, r0 = c.u0 * RPP, gbox = gbox_of(c.slot);
+      const bool routed = c.slot < K;
+      const int e = routed ? s_idx[c.slot] : 0;
+      const uint32_t cpart = r128(2u * gbox * RB), spart = r128((uint32_t)gbox * SB);
+      if (p.use_maps) {  // two tensor copies: gate+up codes, and the four scale arrays (whole boxes)
+        if (lane == 0) {
+          mbar_expect_tx(bar, 2u * gbox * RB + 4u * gbox * SB);
+          tma_4d(d, &maps.gu_codes[routed ? 0 : 1], r0, 0, e, bar, pol);
+          tma_5d(d + cpart, &maps.gu_sb[routed ? 0 : 1], r0, 0, 0, e, bar, pol);
+        }
+      } else {  // six bulk copies of the chunk's rows
+        if (lane == 0) mbar_expect_tx(bar, (uint32_t)rows * 2 * (RB + 2 * SB));
+        __syncwarp();
+        const uint8_t* rec = routed ? p.routed.base + (long long)e * p.routed.stride : p.shared.base;
+        const long long* off = routed ? p.routed.off : p.shared.off;
+        if (lane < 2) {
+          bulk_g2s(d + lane * (uint32_t)gbox * RB, rec + off[lane == 0 ? 0 : 3] + (long long)r0 * RB,
+                   (uint32_t)rows * RB, bar, pol);
+        } else if (lane < 6) {
+          const int i = lane - 2;
+          bulk_g2s(d + cpart + i * spart, rec + off[i == 0 ? 1 : i == 1 ? 2 : i == 2 ? 4 : 5] + (long long)r0 * SB,
+                   (uint32_t)rows * SB, bar, pol);
+        }
+      }
+      __syncwarp();
+      ++rpr.j;
+    };
+    auto issue_d = [&](int jd, uint32_t vs) {
+      const uint32_t d = smem_addr(ring + vs % RING);
+      const uint32_t bar = smem_addr(&s_full[rpr.j % kXSlots]);
+      const int range = jd / NE, slot = down_slot(jd % NE, K, p.has_shared);
+      const int row0 = rg.d0 * DR + range * dbox, rows = min(dbox, drows_all - range * dbox);
+      const bool routed = slot < K;
+      const int e = routed ? s_idx[slot] : 0;
+      if (p.use_maps) {  // two tensor copies: codes, scales + biases (whole boxes)
+        if (lane == 0) {
+          mbar_expect_tx(bar, (uint32_t)dbox * (RBD + 2 * SBD));
+          tma_3d(d, &maps.dn_codes[routed ? 0 : 1], row0, e, bar, pol);
+          tma_4d(d + dcode, &maps.dn_sb[routed ? 0 : 1], row0, 0, e, bar, pol);
+        }
+      } else {
+        if (lane == 0) mbar_expect_tx(bar, (uint32_t)rows * (RBD + 2 * SBD));
+        __syncwarp();
+        const uint8_t* rec = routed ? p.routed.base + (long long)e * p.routed.stride : p.shared.base;
+        const long long* off = routed ? p.routed.off : p.shared.off;
+        if (lane < 3) {
+          const uint32_t unit = lane == 0 ? RBD : SBD;
+          bulk_g2s(d + (lane == 0 ? 0u : dcode + (lane - 1) * dsb), rec + off[6 + lane] + (long long)row0 * unit,
+                   (uint32_t)rows * unit, bar, pol);
+        }
+      }
+      __syncwarp();
+      ++rpr.j;
+    };
+    // L2 requests for this CTA's down rows of slot `slot` (codes, scales, biases), lanes base..base+2
+    auto ask_l2_down = [&](int slot, int base) {
+      if (lane >= base && lane < base + 3 && drows_all > 0) {
+        const int m = lane - base;
+        const bool routed = slot < K;
+        const uint8_t* rec = routed ? p.routed.base + (long long)s_idx[slot] * p.routed.stride : p.shared.base;
+        const long long* off = routed ? p.routed.off : p.shared.off;
+        const long long unit = m == 0 ? RBD : SBD;
+        prefetch_l2(rec + off[6 + m] + (long long)rg.d0 * DR * unit, (uint32_t)(drows_all * unit));
+      }
+    };
+    // Before the dependency wait (weights only): the shared expert's gate/up chunks as far
+    // as they fit without waiting, and an L2 request for its down rows.
+    uint32_t vs;
+    while (ghave && gc.slot == K && rpr.reserve(glen_of(gbox_of(gc.slot)), false, vs, ok, p.err)) {
+      issue_g(gc, vs);
+      ghave = git.next(gc, rg, K, ups, p.gmax_s, p.gmax_r);
+    }
+    if (p.has_shared) ask_l2_down(K, 0);
+    pdl_wait();
+    pdl_trigger();
+    if (lane == 0) {  // the digits of x, written by the previous kernel
+      const uint32_t bx = smem_addr(&s_xbar);
+      mbar_expect_tx(bx, (uint32_t)(C::kXDigitBytes + C::kXChunks * 8));
+      bulk_g2s(smem_addr(xd), p.xq_limbs, C::kXDigitBytes, bx, l2_policy_evict_last());
+      bulk_g2s(smem_addr(xd + C::kXDigitBytes), p.xq_cs, C::kXChunks * 8, bx, l2_policy_evict_last());
+    }
+    named_bar_sync(kBarAll, kXThreads);  // the routing is in s_idx
+    while (ok && ghave && rpr.reserve(glen_of(gbox_of(gc.slot)), true, vs, ok, p.err)) {
+      issue_g(gc, vs);
+      ghave = git.next(gc, rg, K, ups, p.gmax_s, p.gmax_r);
+    }
+    // every gate/up chunk is out: ask L2 for the routed down rows, then stage the down chunks
+    for (int k = 0; k < K && 3 * k < 32; ++k) ask_l2_down(k, 3 * k);
+    for (int jd = 0; ok && jd < nd && rpr.reserve(dlen, true, vs, ok, p.err); ++jd) issue_d(jd, vs);
+    if (lane == 0) {
+      s_issued = rpr.j;
+      if (!ok) s_abort = 1;
+    }
+  } else {
+    // ================================================================ consumer warps
+    pdl_wait();  // the router's logits and the digits of x are complete
+    pdl_trigger();
+    if (p.logits && !p.route_idx) {
+      consumer_topk(p.logits, p.E, K, p.has_shared, s_cand, s_idx, s_w);
+    } else if (warp == 0) {
+      int e = 0;
+      float wv = 1.0f;
+      if (lane < K) {
+        e = p.route_idx ? __ldcg(p.route_idx + lane) : p.fixed_expert;
+        wv = p.route_w ? __ldcg(p.route_w + lane) : 1.0f;
+      }
+      const float zg = (p.has_shared && p.logits) ? __ldcg(p.logits + p.E) : 0.0f;
+      if (lane < K) {
+        s_idx[lane] = e;
+        s_w[lane] = wv;
+      }
+      if (lane == 0) s_w[K] = p.has_shared ? (p.logits ? 1.0f / (1.0f + expf(-zg)) : 1.0f) : 0.0f;
+    }
+    if (warp == 0 && lane < K) {
+      const int e = s_idx[lane];
+      if (e < 0 || e >= p.routed.num_experts) {
+        atomicExch(p.err, kDevBadIndex);
+        s_idx[lane] = 0;
+      }
+    }
+    __syncwarp();
+    named_bar_sync(kBarAll, kXThreads);
+    if (b == 0 && tid < K) {
+      if (p.idx_out) p.idx_out[tid] = s_idx[tid];
+      if (p.w_out) p.w_out[tid] = s_w[tid];
+    }
+
+    // this lane's groups of x and their digits, for every gate/up row it computes
+    const int sub = lane / LPR, gl = lane % LPR;
+    bool ok = mbar_wait_bounded(smem_addr(&s_xbar), 0, p.err);
+    const uint32_t* xs = reinterpret_cast<const uint32_t*>(xd);
+    const float2* xcs = reinterpret_cast<const float2*>(xd + C::kXDigitBytes);
+    uint32_t L[C::kRegDigits ? GPL : 1][48];
+    float2 cs[GPL];
+#pragma unroll
+    for (int q = 0; q < GPL; ++q) {
+      const int g = gl + LPR * q;
+      if constexpr (C::kRegDigits) load_group_limbs(xs, g, NG, L[q]);
+      cs[q] = group_scalars<BITS>(xcs, g);
+    }
+
+    // ---- gate/up + SwiGLU: warp w takes tasks w, w + 8, .. of a chunk (a task = RPP rows)
+    RingPos rp;
+    int jc = 0;  // chunk index (both kinds)
+    {
+      GChunkIt git(rg);
+      GChunk c;
+      for (; git.next(c, rg, K, ups, p.gmax_s, p.gmax_r); ++jc) {
+        const int gbox = gbox_of(c.slot);
+        const uint32_t vs = rp.place(glen_of(gbox), RING);
+        if (ok && !mbar_wait_bounded(smem_addr(&s_full[jc % kXSlots]), (uint32_t)((jc / kXSlots) & 1), p.err))
+          ok = false;
+        const uint8_t* buf = ring + vs % RING;
+        const uint8_t* sbase = buf + r128(2u * gbox * RB);
+        const uint32_t spart = r128((uint32_t)gbox * SB);
+        for (int t = warp; ok && t < c.n; t += kXWarps) {
+          const int rr = t * RPP + sub;  // row within the chunk
+          float ag = 0.0f, au = 0.0f;
+#pragma unroll
+          for (int q = 0; q < GPL; ++q) {
+            const int g = gl + LPR * q;
+            uint4 q0, q1, v0, v1;
+            load_group_codes<BITS>(buf + rr * RB, g, q0, q1);
+            load_group_codes<BITS>(buf + gbox * RB + rr * RB, g, v0, v1);
+            const float gs = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + rr * SB)[g]);
+            const float gb = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + spart + rr * SB)[g]);
+            const float us = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + 2 * spart + rr * SB)[g]);
+            const float ub = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + 3 * spart + rr * SB)[g]);
+            float Sg, Su;
+            if constexpr (C::kRegDigits) {
+              Sg = group_dot<BITS>(q0, q1, L[q]);
+              Su = group_dot<BITS>(v0, v1, L[q]);
+            } else {
+              uint32_t Lt[48];
+              load_group_limbs(xs, g, NG, Lt);
+              Sg = group_dot<BITS>(q0, q1, Lt);
+              Su = group_dot<BITS>(v0, v1, Lt);
+            }
+            ag = fmaf(gs, cs[q].x * Sg, fmaf(gb, cs[q].y, ag));
+            au = fmaf(us, cs[q].x * Su, fmaf(ub, cs[q].y, au));
+          }
+#pragma unroll
+          for (int o = LPR / 2; o > 0; o >>= 1) {
+            ag += __shfl_xor_sync(0xffffffffu, ag, o);
+            au += __shfl_xor_sync(0xffffffffu, au, o);
+          }
+          if (gl == 0) p.act[(size_t)c.slot * I + (size_t)c.u0 * RPP + rr] = ag / (1.0f + expf(-ag)) * au;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&s_empty[jc % kXSlots]));
+      }
+    }
+
+    // ---- hand-off: count this CTA in, wait until every CTA is in.  One thread each
+    // (consumer threads issue no bulk copies, so their fences do not wait on any).
+    named_bar_sync(kBarCons, kXWarps * 32);
+    if (tid == 0) {
+      __threadfence();
+      atomicAdd(p.count, 1u);
+      if (!count_wait_bounded(p.count, (unsigned)G, p.err)) s_abort = 1;
+    }
+    named_bar_sync(kBarCons, kXWarps * 32);
+    if (s_abort) ok = false;
+
+    // ---- digits of every slot's activations, into the digits region (x is in registers now)
+    uint8_t* dl = xd;                                                                  // [NE][NGD * 192]
+    float2* dcs = reinterpret_cast<float2*>(xd + (size_t)NE * NGD * kGroupWords * 4);  // [NE][chD]
+    {
+      constexpr int kQ = 128 / kXWarps;  // groups per warp at most (NE * NGD <= 128)
+      float2 v[kQ];
+#pragma unroll
+      for (int i = 0; i < kQ; ++i) {
+        const int q = warp + kXWarps * i;
+        v[i] = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)min(q, NE * NGD - 1) * kGroup) + lane);
+      }
+#pragma unroll
+      for (int i = 0; i < kQ; ++i) {
+        const int q = warp + kXWarps * i;
+        if (q < NE * NGD) {
+          const int s = q / NGD, g = q - s * NGD;
+          xq_quantize_group<BITS>(v[i].x, v[i].y, g, NGD, dl + (size_t)s * NGD * kGroupWords * 4, dcs + (size_t)s * chD);
+        }
+      }
+    }
+    named_bar_sync(kBarCons, kXWarps * 32);
+
+    // ---- down + combine.  The (slot, group) pairs split into P parts of at most 64,
+    // each taken by 8 / P warps; lane l owns pairs l and l + 32 of its part.
+    const int NP = NE * NGD;
+    const int P = NP > 64 ? 2 : 1;
+    const int part = warp / (kXWarps / P), wi = warp % (kXWarps / P), nw = kXWarps / P;
+    const int pb = part == 0 ? 0 : (NP + 1) / 2, pe = P == 1 ? NP : (part == 0 ? (NP + 1) / 2 : NP);
+    uint32_t LD[DPPL][48];
+    float2 csd[DPPL];
+    float wq[DPPL];
+    int qs[DPPL], qg[DPPL];
+#pragma unroll
+    for (int m = 0; m < DPPL; ++m) {
+      const int q = pb + lane + 32 * m;
+      const bool has = q < pe;
+      const int s = has ? q / NGD : 0, g = has ? q - (q / NGD) * NGD : 0;
+      load_group_limbs(reinterpret_cast<const uint32_t*>(dl + (size_t)s * NGD * kGroupWords * 4), g, NGD, LD[m]);
+      csd[m] = group_scalars<BITS>(dcs + (size_t)s * chD, g);
+      wq[m] = has ? s_w[s] : 0.0f;
+      qs[m] = s;
+      qg[m] = g;
+    }
+    for (int range = 0; range < nranges; ++range) {
+      // the range's NE chunks, in issue order; this lane's slots' buffers
+      const uint8_t* sbuf[DPPL];
+#pragma unroll
+      for (int m = 0; m < DPPL; ++m) sbuf[m] = ring;
+      const int j0 = jc;
+      for (int k = 0; k < NE; ++k, ++jc) {
+        const uint32_t vs = rp.place(dlen, RING);
+        const int slot = down_slot(k, K, p.has_shared);
+#pragma unroll
+        for (int m = 0; m < DPPL; ++m)
+          if (qs[m] == slot) sbuf[m] = ring + vs % RING;
+        if (ok && !mbar_wait_bounded(smem_addr(&s_full[jc % kXSlots]), (uint32_t)((jc / kXSlots) & 1), p.err))
+          ok = false;
+      }
+      const int rows = min(dbox, drows_all - range * dbox);
+      for (int rr = wi; ok && rr < rows; rr += nw) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int m = 0; m < DPPL; ++m) {
+          const uint8_t* sb = sbuf[m];
+          const int g = qg[m];
+          const uint4 q0 = *reinterpret_cast<const uint4*>(sb + rr * RBD + g * (kGroup * BITS / 8));
+          const uint4 q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(sb + rr * RBD + g * (kGroup * BITS / 8) + 16) : q0;
+          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + dcode + rr * SBD)[g]);
+          const float bi = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + dcode + dsb + rr * SBD)[g]);
+          const float S = group_dot<BITS>(q0, q1, LD[m]);
+          acc = fmaf(wq[m], fmaf(sc, csd[m].x * S, bi * csd[m].y), acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) s_dpart[part][rr] = acc;
+      }
+      __syncwarp();
+      if (lane == 0)
+        for (int k = 0; k < NE; ++k) mbar_arrive(smem_addr(&s_empty[(j0 + k) % kXSlots]));
+      named_bar_sync(kBarCons, kXWarps * 32);
+      if (ok)
+        for (int rr = tid; rr < rows; rr += kXWarps * 32) {
+          const int row = rg.d0 * DR + range * dbox + rr;
+          const float y = P == 2 ? s_dpart[0][rr] + s_dpart[1][rr] : s_dpart[0][rr];
+          p.out[row] = (p.resid ? __ldcg(p.resid + row) : 0.0f) + y;
+        }
+      named_bar_sync(kBarCons, kXWarps * 32);
+    }
+    if (!ok && tid == 0) s_abort = 1;
+  }
+  // A CTA that gave up a wait lets the copies it issued land before it exits.
+  __syncthreads();
+  if (s_abort && tid == 0) {
+    for (int q = s_issued > kXSlots ? s_issued - kXSlots : 0; q < s_issued; ++q)
+      mbar_wait_bounded(smem_addr(&s_full[q % kXSlots]), (uint32_t)((q / kXSlots) & 1), p.err);
+    mbar_wait_bounded(smem_addr(&s_xbar), 0, p.err);
+  }
+}
+
+size_t round128(size_t v) { return (v + 127) / 128 * 128; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return enc;
+}
+
+// One map over 8-byte elements: dims[0] elements per row, then the outer dims with
+// their byte strides; box: dims[0] x box_rows x the outer dims' full extents (last: 1).
+bool encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                const cuuint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, rank, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The maps of both banks, or false when the layout does not allow them (then the kernel
+// takes bulk copies): gate and up (and scale and bias) sub-arrays must sit at uniform
+// distances inside a record, rows of at most 2048 bytes of codes and at least 16 of scales.
+bool encode_tok_maps(TokMaps& M, const TokExpertParams& p, int bits) {
+  const int H = p.H, I = p.I, NG = H / kGroup, NGD = I / kGroup;
+  const long long RB = (long long)H * bits / 8, SB = NG * 2, RBD = (long long)I * bits / 8, SBD = NGD * 2;
+  if (RB > 2048 || RBD > 2048 || SB < 16 || SBD < 16) return false;
+  const int LPR = NG < 32 ? NG : 32, RPP = 32 / LPR, DR = NGD >= 8 ? 1 : 8 / NGD;
+  const int dbox = p.dmax * DR;
+  if (p.gmax_r * RPP > 256 || p.gmax_s * RPP > 256 || dbox > 256) return false;
+  for (int bk = 0; bk < 2; ++bk) {
+    const int gbox = (bk == 0 ? p.gmax_r : p.gmax_s) * RPP;
+    const BankRef& r = bk == 0 ? p.routed : p.shared;
+    const long long* o = r.off;
+    const long long gu = o[3] - o[0], sbd = o[2] - o[1];
+    if (o[4] - o[1] != gu || o[5] - o[2] != gu || o[5] - o[4] != sbd || gu <= 0 || sbd <= 0) return false;
+    const long long dsb = o[8] - o[7];
+    if (dsb <= 0) return false;
+    const cuuint64_t ne = bk == 0 ? (cuuint64_t)p.routed.num_experts : 1;
+    const cuuint64_t est = bk == 0 ? (cuuint64_t)r.stride : 16;
+    {
+      const cuuint64_t dims[4] = {(cuuint64_t)(RB / 8), (cuuint64_t)I, 2, ne};
+      const cuuint64_t st[3] = {(cuuint64_t)RB, (cuuint64_t)gu, est};
+      const cuuint32_t box[4] = {(cuuint32_t)(RB / 8), (cuuint32_t)gbox, 2, 1};
+      if (!encode_map(&M.gu_codes[bk], r.base + o[0], 4, dims, st, box)) return false;
+    }
+    {
+      const cuuint64_t dims[5] = {(cuuint64_t)(SB / 8), (cuuint64_t)I, 2, 2, ne};
+      const cuuint64_t st[4] = {(cuuint64_t)SB, (cuuint64_t)sbd, (cuuint64_t)gu, est};
+      const cuuint32_t box[5] = {(cuuint32_t)(SB / 8), (cuuint32_t)gbox, 2, 2, 1};
+      if (!encode_map(&M.gu_sb[bk], r.base + o[1], 5, dims, st, box)) return false;
+    }
+    {
+      const cuuint64_t dims[3] = {(cuuint64_t)(RBD / 8), (cuuint64_t)H, ne};
+      const cuuint64_t st[2] = {(cuuint64_t)RBD, est};
+      const cuuint32_t box[3] = {(cuuint32_t)(RBD / 8), (cuuint32_t)dbox, 1};
+      if (!encode_map(&M.dn_codes[bk], r.base + o[6], 3, dims, st, box)) return false;
+    }
+    {
+      const cuuint64_t dims[4] = {(cuuint64_t)(SBD / 8), (cuuint64_t)H, 2, ne};
+      const cuuint64_t st[3] = {(cuuint64_t)SBD, (cuuint64_t)dsb, est};
+      const cuuint32_t box[4] = {(cuuint32_t)(SBD / 8), (cuuint32_t)dbox, 2, 1};
+      if (!encode_map(&M.dn_sb[bk], r.base + o[7], 4, dims, st, box)) return false;
+    }
+  }
+  return true;
+}
+
+template <int BITS, int NG>
+cudaError_t expert_ng(const TokExpertParams& p, const TokMaps& m, int dppl, size_t smem, int grid, bool pdl,
+                      cudaStream_t s) {
+  void (*k)(const TokExpertParams, const TokMaps) =
+      dppl == 1 ? tok_expert_kernel<BITS, NG, 1> : tok_expert_kernel<BITS, NG, 2>;
+  cudaError_t e = set_smem((const void*)k, smem);
+  if (e == cudaSuccess) e = set_carveout_max((const void*)k);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(grid), dim3(kXThreads), smem, s, pdl, p, m);
+}
+
+template <int BITS>
+cudaError_t expert_bits(const TokExpertParams& p, const TokMaps& m, int dppl, size_t smem, int grid, bool pdl,
+                        cudaStream_t s) {
+  switch (p.H / kGroup) {
+    case 2: return expert_ng<BITS, 2>(p, m, dppl, smem, grid, pdl, s);
+    case 4: return expert_ng<BITS, 4>(p, m, dppl, smem, grid, pdl, s);
+    case 8: return expert_ng<BITS, 8>(p, m, dppl, smem, grid, pdl, s);
+    case 16: return expert_ng<BITS, 16>(p, m, dppl, smem, grid, pdl, s);
+    case 32: return expert_ng<BITS, 32>(p, m, dppl, smem, grid, pdl, s);
+    case 64: return expert_ng<BITS, 64>(p, m, dppl, smem, grid, pdl, s);
+    case 128: return expert_ng<BITS, 128>(p, m, dppl, smem, grid, pdl, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+// Shared memory of the expert kernel: the digits region (x, later the activations) and
+// one ring for the staged chunks.  A down range's NE chunks are in the ring together,
+// so a range holds at most half of it.
+TokPlan plan_token(int bits, int H, int I, int K, int has_shared) {
+  TokPlan pl{};
+  if (H % kGroup || I % kGroup || H < 2 * kGroup || I < 2 * kGroup || K < 1 || K > 32) return pl;
+  const int NG = H / kGroup, NGD = I / kGroup, NE = K + has_shared;
+  const int LPR = NG < 32 ? NG : 32, RPP = 32 / LPR;
+  const size_t RB = (size_t)H * bits / 8, SB = (size_t)NG * 2;
+  const size_t chX = (size_t)H * bits / 128, chD = (size_t)I * bits / 128;
+  const size_t xd = round128(std::max((size_t)NG * kGroupWords * 4 + chX * 8,
+                                      (size_t)NE * ((size_t)NGD * kGroupWords * 4 + chD * 8)));
+  if (xd + 4096 > kXSmemBudget || NE + 4 > kXSlots) return pl;
+  const size_t ring = (kXSmemBudget - xd) / 128 * 128;
+  int grid = num_sms();
+  if (grid > kMaxTokenCtas) grid = kMaxTokenCtas;
+  const int DR = NGD >= 8 ? 1 : 8 / NGD;
+  const size_t RBD = (size_t)I * bits / 8, SBD = (size_t)NGD * 2;
+  // gate/up chunks: at most about kXChunkTarget bytes, the CTA's average range split
+  // into equal chunks (a tensor copy moves a whole box, so uneven tails would fetch
+  // rows of the next range)
+  const size_t unitG = RPP * 2 * (RB + 2 * SB);
+  const int cap = (int)std::max<size_t>(1, std::min<size_t>(std::min(kXChunkTarget, ring / 4) / unitG, 256 / RPP));
+  const int ups = I / RPP;
+  auto even = [&](int units_total) {
+    const int avg = std::max(1, (units_total + grid - 1) / grid);
+    const int n = (avg + cap - 1) / cap;
+    return (avg + n - 1) / n;
+  };
+  const int gmax_r = even(K * ups), gmax_s = has_shared ? even(ups) : 1;
+  const size_t glen = round128(2 * (size_t)std::max(gmax_r, gmax_s) * RPP * RB) +
+                      4 * round128((size_t)std::max(gmax_r, gmax_s) * RPP * SB);
+  // down ranges: the CTA's whole share when its NE chunks fit in half the ring
+  auto dlen_of = [&](int dm) {
+    const size_t rows = (size_t)dm * DR;
+    return round128(rows * RBD) + 2 * round128(rows * SBD);
+  };
+  const int UD = H / DR, dshare = (UD + grid - 1) / grid;
+  int dmax = std::min(dshare, std::min(kXMaxDRows, 256) / DR);
+  while (dmax > 1 && (size_t)NE * dlen_of(dmax) > ring / 2) --dmax;
+  const int NP = NE * NGD, part = NP > 64 ? (NP + 1) / 2 : NP;
+  if (glen > ring || (size_t)NE * dlen_of(dmax) > ring || NP > 128) return pl;
+  pl.ok = true;
+  pl.grid = grid;
+  pl.gmax_s = gmax_s;
+  pl.gmax_r = gmax_r;
+  pl.dmax = dmax;
+  pl.xd_bytes = (int)xd;
+  pl.ring_bytes = (int)ring;
+  pl.dppl = (part + 31) / 32;
+  pl.smem = xd + ring;
+  return pl;
+}
+
+cudaError_t launch_tok_router(TokRouterParams p, int bits, bool pdl, cudaStream_t s) {
+  const int rows = p.E + 1 - p.row0;
+  int rmax = kRtSmemBudget / (2 * p.H);
+  rmax = rmax < 1 ? 1 : (rmax > kRtMaxRows ? kRtMaxRows : rmax);
+  const int nsm = num_sms();
+  int rpc = (rows + nsm - 1) / nsm;
+  rpc = rpc < 1 ? 1 : (rpc > rmax ? rmax : rpc);
+  int grid = (rows + rpc - 1) / rpc;
+  const int NG = p.H / kGroup;
+  if (grid < NG && grid < nsm) grid = NG < nsm ? NG : nsm;  // spread the digit groups too
+  p.rpc = rpc;
+  const size_t smem = (size_t)rpc * p.H * 2;
+  void (*k)(const TokRouterParams) = p.H <= 8 * 4 * kRtThreads
+                                        ? (bits == 4 ? tok_router_kernel<4, 8> : tok_router_kernel<2, 8>)
+                                        : (bits == 4 ? tok_router_kernel<4, 16> : tok_router_kernel<2, 16>);
+  cudaError_t e = set_smem((const void*)k, smem);
+  if (e == cudaSuccess) e = set_carveout_max((const void*)k);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(grid), dim3(kRtThreads), smem, s, pdl, p);
+}
+
+cudaError_t launch_tok_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, unsigned int* count, bool pdl,
+                          cudaStream_t s) {
+  const int grid = (H / kGroup + kRtThreads / 32 - 1) / (kRtThreads / 32);
+  void (*k)(const float*, int, uint8_t*, float2*, unsigned int*) = bits == 4 ? tok_xq_kernel<4> : tok_xq_kernel<2>;
+  cudaError_t e = set_carveout_max((const void*)k);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(grid), dim3(kRtThreads), 0, s, pdl, x, H, limbs, cs, count);
+}
+
+cudaError_t launch_tok_expert(TokExpertParams p, int bits, bool pdl, cudaStream_t s) {
+  const TokPlan pl = plan_token(bits, p.H, p.I, p.K, p.has_shared);
+  if (!pl.ok) return cudaErrorInvalidValue;
+  p.gmax_s = pl.gmax_s;
+  p.gmax_r = pl.gmax_r;
+  p.dmax = pl.dmax;
+  p.xd_bytes = pl.xd_bytes;
+  p.ring_bytes = pl.ring_bytes;
+  TokMaps m;
+  memset(&m, 0, sizeof(m));
+  p.use_maps = token_maps_enabled() && encode_tok_maps(m, p, bits) ? 1 : 0;
+  return bits == 4 ? expert_bits<4>(p, m, pl.dppl, pl.smem, pl.grid, pdl, s)
+                   : expert_bits<2>(p, m, pl.dppl, pl.smem, pl.grid, pdl, s);
+}
+
+}  // namespace fmoe

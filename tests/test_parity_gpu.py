@@ -232,3 +232,58 @@ def test_stack_of_layers_matches_oracle(fmoe):
         ref = oracle_layer(hl).forward(ref.astype(np.float32))["out"]
     # fp32 inputs between layers on the oracle side; routing of this seed has no near-ties
     assert max_rel_err(out, ref) <= TOL
+
+
+# --------------------------------------------------------------------------- the two-kernel per-token path
+
+
+@pytest.fixture
+def two_kernels(monkeypatch):
+    monkeypatch.setenv("FMOE_TOKEN_KERNELS", "2")
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_two_kernel_path_tiny_layer(fmoe, two_kernels, bits):
+    spec = gen.LayerSpec(**{**gen.tiny_layer(bits).__dict__, "random_gamma": True})
+    hl = gen.host_layer(spec, seed=21)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(2100, 24, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    exact, _ = _compare_layer(hl, h, out, idx, w)
+    assert exact >= 22
+
+
+@pytest.mark.parametrize("top_k", [1, 8])
+def test_two_kernel_path_top1_and_all_experts(fmoe, two_kernels, top_k):
+    spec = gen.tiny_layer(4)
+    hl = gen.host_layer(spec, seed=22)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(2200, 8, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h, top_k=top_k)
+    _compare_layer(hl, h, out, idx, w, L=oracle_layer(hl, top_k=top_k))
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_two_kernel_path_expert_ffn(fmoe, two_kernels, bits):
+    spec = gen.tiny_layer(bits)
+    hl = gen.host_layer(spec, seed=23)
+    dl = gen.upload_layer(hl)
+    lay = gen.binding_layer(dl)
+    L = oracle_layer(hl)
+    rng = np.random.default_rng(23)
+    for e in (0, 7):
+        x = rng.standard_normal(spec.hidden).astype(np.float32)
+        y = fmoe.expert_ffn(lay.routed, e, torch.from_numpy(x).cuda()).cpu().numpy()
+        assert max_rel_err(y, oracle.expert_ffn(L.routed, e, x)) <= TOL
+
+
+def test_two_kernel_path_full_size(fmoe, big, two_kernels):
+    """The Qwen3.5-397B-A17B-shaped layer (4-bit; 2-bit with Zipf routing), 16 fresh
+    tokens against the oracle."""
+    spec, dl = big
+    T = 16
+    h = gen.host_tokens(2500, T, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    hl, L = full_size_oracle_layer(spec, h, idx)
+    exact, _ = _compare_layer(hl, h, out, idx, w, L=L)
+    assert exact >= 14, exact
