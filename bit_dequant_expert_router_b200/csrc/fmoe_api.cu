@@ -123,7 +123,7 @@ fmoe_status check_bank(const fmoe_bank* b, const char* name) {
   if (!pow2(H / 64) || H > 8192 || !pow2(I / 64) || I > 8192)
     return fail(FMOE_ERR_UNSUPPORTED, "%s bank: hidden %d and inter %d must be 64 times a power of two, at most 8192",
                 name, H, I);
-  if (!expert_shapes_supported(b->bits, H, I, 1) || !plan_token(b->bits, H, I, 1, 0).ok)
+  if (!expert_shapes_supported(b->bits, H, I, 1))
     return fail(FMOE_ERR_UNSUPPORTED, "%s bank: shapes exceed the kernels' shared memory", name);
   if (!aligned16(b->base) || (b->stride & 15)) return fail(FMOE_ERR_ALIGNMENT, "%s bank: base/stride not 16-byte aligned", name);
   if (b->num_experts > 1 && b->stride <= 0) return fail(FMOE_ERR_INVALID_ARG, "%s bank: stride %lld", name, (long long)b->stride);
@@ -175,12 +175,6 @@ int prefetch_down() {
     on = (v && v[0] == '0') ? 0 : 1;
   }
   return on;
-}
-
-// TMA tensor-map staging in the per-token expert kernel; FMOE_TMA_MAPS=0 turns it off (bulk copies).
-bool token_maps_enabled() {
-  const char* v = getenv("FMOE_TMA_MAPS");
-  return !(v && v[0] == '0');
 }
 
 // Dependent launch between the block's kernels; FMOE_PDL=0 in the environment turns it off.
@@ -320,7 +314,7 @@ fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, f
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
   const int bits = bank->bits;
-  if (!three_kernel_path()) {
+  if (!three_kernel_path() && token_path_supported(bits, bank->hidden, bank->inter, 1, 0, ref(*bank), ref(*bank))) {
     const bool pdl = pdl_enabled();
     cudaError_t e = launch_tok_xq(x, bank->hidden, bits, base + L.xq_limbs, reinterpret_cast<float2*>(base + L.xq_cs),
                                   &ctrl->tok_count, pdl, cs(stream));
@@ -387,7 +381,7 @@ static fmoe_status check_layer(const fmoe_layer* layer) {
   if (E > 4096) return fail(FMOE_ERR_UNSUPPORTED, "E %d > 4096", E);
   if (r.hidden > 12288) return fail(FMOE_ERR_UNSUPPORTED, "hidden %d > 12288", r.hidden);
   if (K < 1 || K > E || K > 32) return fail(FMOE_ERR_INVALID_ARG, "top_k %d (1..min(E, 32))", K);
-  if (!expert_shapes_supported(r.bits, r.hidden, r.inter, K + 1) || !plan_token(r.bits, r.hidden, r.inter, K, 1).ok)
+  if (!expert_shapes_supported(r.bits, r.hidden, r.inter, K + 1))
     return fail(FMOE_ERR_UNSUPPORTED, "top_k %d with inter %d at %d bits exceeds the down kernel's shared memory", K,
                 r.inter, r.bits);
   if (!(layer->eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)layer->eps);
@@ -413,8 +407,10 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
 // err_word: where the kernels report a failed bounded wait; NULL means the workspace's own error word.
 static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
                                uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word = nullptr) {
-  if (three_kernel_path()) return layer_token_3k(layer, h, out, idx_out, w_out, base, L, s, err_word);
   const fmoe_bank& r = layer->routed;
+  if (three_kernel_path() ||
+      !token_path_supported(r.bits, r.hidden, r.inter, layer->top_k, 1, ref(r), ref(layer->shared)))
+    return layer_token_3k(layer, h, out, idx_out, w_out, base, L, s, err_word);
   const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
   TokRouterParams rp{};

@@ -201,6 +201,24 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared on the load path (not the TMA engine,
+// whose fixed cost per copy makes small copies slow); dst, src 16-byte aligned.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// The barrier receives one arrival once every cp.async this thread issued so far has
+// landed (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Copies `bytes` (a multiple of 16) from src to shared dst with cp_async16, the pieces
+// spread over the 32 lanes of the calling warp.
+__device__ __forceinline__ void cp_async_warp(uint32_t dst, const uint8_t* src, uint32_t bytes, int lane) {
+  for (uint32_t o = 16u * lane; o < bytes; o += 512u) cp_async16(dst + o, src + o);
+}
+
 // ------------------------------------------------------------------------------------------ activation format
 //
 // The dot product sum_c code_c * x_c over a group of 64 codes runs on integer

@@ -229,13 +229,13 @@ struct TokExpertParams {
   int* err;
   // set by the launcher
   int gmax_s, gmax_r, dmax;   // units per shared / routed gate/up chunk, per down range
-  int xd_bytes, ring_bytes;   // shared-memory regions
-  int use_maps;               // stage by TMA tensor copies (else bulk copies)
+  int xd_bytes, sc_bytes, ring_bytes;  // shared-memory regions: digits, scales, staged codes
+  int sbox_s, sbox_r, drows;  // staged scale rows: shared and routed gate/up, down (per CTA, at most)
 };
 
 struct TokPlan {
   bool ok;
-  int grid, gmax_s, gmax_r, dmax, xd_bytes, ring_bytes, dppl;
+  int grid, gmax_s, gmax_r, dmax, xd_bytes, sc_bytes, sbox_s, sbox_r, drows, ring_bytes, dppl;
   size_t smem;
 };
 
@@ -243,8 +243,9 @@ TokPlan plan_token(int bits, int H, int I, int K, int has_shared);
 cudaError_t launch_tok_router(TokRouterParams p, int bits, bool pdl, cudaStream_t s);
 cudaError_t launch_tok_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, unsigned int* count, bool pdl,
                           cudaStream_t s);
-bool token_maps_enabled();
 cudaError_t launch_tok_expert(TokExpertParams p, int bits, bool pdl, cudaStream_t s);
+// Whether the two-kernel path takes these shapes and record layouts.
+bool token_path_supported(int bits, int H, int I, int K, int has_shared, const BankRef& routed, const BankRef& shared);
 
 cudaError_t launch_rmsnorm(const float* h, const float* gamma, float eps, int T, int H, float* y, cudaStream_t s);
 cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, cudaStream_t s);

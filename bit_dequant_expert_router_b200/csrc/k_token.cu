@@ -112,39 +112,32 @@ __global__ void __launch_bounds__(kRtThreads) tok_router_kernel(const TokRouterP
     ss = fmaf(hv[j].z, hv[j].z, ss);
     ss = fmaf(hv[j].w, hv[j].w, ss);
   }
-  float acc[kRtMaxRows];
+  // v = gamma * h, kept in hv (pass 2 scales it by rstd)
 #pragma unroll
-  for (int r = 0; r < kRtMaxRows; ++r) acc[r] = 0.0f;
+  for (int j = 0; j < kRtMaxF4; ++j)
+    hv[j] = make_float4(hv[j].x * gv[j].x, hv[j].y * gv[j].y, hv[j].z * gv[j].z, hv[j].w * gv[j].w);
+  ss = warp_sum(ss);
+  if (lane == 0) s_red[warp][kRtMaxRows] = ss;
   const bool ready = nrows == 0 || mbar_wait_bounded(bar, 0, p.err);
   if (ready) {
+    // one row at a time in a loop that is not unrolled over the rows: this code runs
+    // once per token, so it is kept short (it is fetched cold every time)
     const uint16_t* wr = reinterpret_cast<const uint16_t*>(sm);
+#pragma unroll 1
+    for (int r = 0; r < nrows; ++r) {
+      float a = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kRtMaxF4; ++j) {
-      const int cc = min((tid + j * kRtThreads) * 4, H - 4);  // columns past H: v is 0 there
-      const float4 g = gv[j];
-      const float4 v = make_float4(hv[j].x * g.x, hv[j].y * g.y, hv[j].z * g.z, hv[j].w * g.w);
-#pragma unroll
-      for (int r = 0; r < kRtMaxRows; ++r) {
-        if (r < nrows) {
-          const uint2 w = *reinterpret_cast<const uint2*>(wr + (size_t)r * H + cc);
-          float a = acc[r];
-          a = fmaf(bf_lo(w.x), v.x, a);
-          a = fmaf(bf_hi(w.x), v.y, a);
-          a = fmaf(bf_lo(w.y), v.z, a);
-          a = fmaf(bf_hi(w.y), v.w, a);
-          acc[r] = a;
-        }
+      for (int j = 0; j < kRtMaxF4; ++j) {
+        const int cc = min((tid + j * kRtThreads) * 4, H - 4);  // columns past H: v is 0 there
+        const uint2 w = *reinterpret_cast<const uint2*>(wr + (size_t)r * H + cc);
+        a = fmaf(bf_lo(w.x), hv[j].x, a);
+        a = fmaf(bf_hi(w.x), hv[j].y, a);
+        a = fmaf(bf_lo(w.y), hv[j].z, a);
+        a = fmaf(bf_hi(w.y), hv[j].w, a);
       }
+      a = warp_sum(a);
+      if (lane == 0) s_red[warp][r] = a;
     }
-  }
-  ss = warp_sum(ss);
-#pragma unroll
-  for (int r = 0; r < kRtMaxRows; ++r)
-    if (r < nrows) acc[r] = warp_sum(acc[r]);
-  if (lane == 0) {
-    s_red[warp][kRtMaxRows] = ss;
-#pragma unroll
-    for (int r = 0; r < kRtMaxRows; ++r) s_red[warp][r] = acc[r];
   }
   __syncthreads();
   float sst = 0.0f;
@@ -172,9 +165,9 @@ __global__ void __launch_bounds__(kRtThreads) tok_router_kernel(const TokRouterP
 #pragma unroll
         for (int j = 0; j < kRtMaxF4; ++j)
           if (j == g / 8) {
-            const float4 hx = hv[j], gx = gv[j];
+            const float4 v = hv[j];
             *reinterpret_cast<float4*>(&s_x[w][4 * (tid % 16)]) =
-                make_float4(hx.x * rstd * gx.x, hx.y * rstd * gx.y, hx.z * rstd * gx.z, hx.w * rstd * gx.w);
+                make_float4(v.x * rstd, v.y * rstd, v.z * rstd, v.w * rstd);
           }
       }
     }
@@ -214,17 +207,15 @@ constexpr size_t kXSmemBudget = 184 * 1024;    // dynamic shared memory of the e
 constexpr size_t kXChunkTarget = 32 * 1024;    // bytes per gate/up chunk, about
 
 // The tensor maps of the staged arrays, [0] the routed bank, [1] the shared expert:
-//   gu_codes  (RB / 8 u64, I rows, {gate, up}, experts)           box (RB / 8, gbox, 2, 1)
-//   gu_sb     (SB / 8 u64, I rows, {scale, bias}, {gate, up}, experts) box (SB / 8, gbox, 2, 2, 1)
-//   dn_codes  (RBD / 8 u64, H rows, experts)                     box (RBD / 8, dbox, 1)
-//   dn_sb     (SBD / 8 u64, H rows, {scale, bias}, experts)       box (SBD / 8, dbox, 2, 1)
-// A box lands as [outer dims][rows][row bytes]: for gate/up gate rows then up rows,
-// then gate scales, gate biases, up scales, up biases, which is the chunk layout below.
+//   gu_codes  (RB / 8 u64, I rows, {gate, up}, experts)                 box (RB / 8, gbox, 2, 1)
+//   gu_sb     (SB / 8 u64, {scale, bias}, {gate, up}, I rows, experts)  box (SB / 8, 2, 2, sbox, 1)
+//   dn_codes  (RBD / 8 u64, H rows, experts)                           box (RBD / 8, dbox, 1)
+// A box lands as [outer dims][..][row bytes]: gate/up codes as gate rows then up rows;
+// the scale box row by row, each row as gate scales, gate biases, up scales, up biases.
 struct TokMaps {
   CUtensorMap gu_codes[2];
   CUtensorMap gu_sb[2];
   CUtensorMap dn_codes[2];
-  CUtensorMap dn_sb[2];
 };
 
 __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, int c1, int c2, uint32_t bar, uint64_t pol) {
@@ -342,23 +333,38 @@ __device__ __forceinline__ void consumer_topk(const float* logits, int E, int K,
 }
 
 // The CTA's work ranges, in units: shared-expert gate/up units [sh0, sh1) (a unit =
-// RPP rows of gate and of up), routed gate/up units [rt0, rt1) over the K slots
-// concatenated (ups units per slot), output-row units [d0, d1) (a unit = DR rows).
+// RPP rows of gate and of up); routed gate/up units [rt0, rt1) of one slot, rslot
+// (the CTAs are dealt out to the K slots in equal runs, so that a CTA's routed rows
+// belong to one expert); output-row units [d0, d1) (a unit = DR rows).
 struct Ranges {
-  int sh0, sh1, rt0, rt1, d0, d1;
+  int sh0, sh1, rslot, rt0, rt1, d0, d1;
 };
+
+__device__ __forceinline__ Ranges cta_ranges(int b, int G, int K, int ups, int has_shared, int UD) {
+  Ranges r;
+  const int US = has_shared ? ups : 0;
+  r.sh0 = (int)((long long)b * US / G);
+  r.sh1 = (int)((long long)(b + 1) * US / G);
+  r.rslot = (int)((long long)b * K / G);
+  const int c0 = (int)(((long long)r.rslot * G + K - 1) / K);        // first CTA of the slot
+  const int c1 = (int)(((long long)(r.rslot + 1) * G + K - 1) / K);  // one past its last
+  r.rt0 = (int)((long long)(b - c0) * ups / (c1 - c0));
+  r.rt1 = (int)((long long)(b - c0 + 1) * ups / (c1 - c0));
+  r.d0 = (int)((long long)b * UD / G);
+  r.d1 = (int)((long long)(b + 1) * UD / G);
+  return r;
+}
 
 // A gate/up chunk: n units of one slot (K = the shared expert), from unit u0 of the slot.
 struct GChunk {
   int slot, u0, n;
 };
 
-// The CTA's gate/up chunks in order: the shared expert's, then the routed ones
-// (never across a slot).
+// The CTA's gate/up chunks in order: the shared expert's, then its routed slot's.
 struct GChunkIt {
   int phase, u;
   __device__ __forceinline__ explicit GChunkIt(const Ranges& r) : phase(0), u(r.sh0) {}
-  __device__ __forceinline__ bool next(GChunk& c, const Ranges& r, int K, int ups, int gmax_s, int gmax_r) {
+  __device__ __forceinline__ bool next(GChunk& c, const Ranges& r, int K, int gmax_s, int gmax_r) {
     if (phase == 0) {
       if (u < r.sh1) {
         c = GChunk{K, u, min(gmax_s, r.sh1 - u)};
@@ -369,8 +375,7 @@ struct GChunkIt {
       u = r.rt0;
     }
     if (phase == 1 && u < r.rt1) {
-      const int sl = u / ups, ui = u - sl * ups;
-      c = GChunk{sl, ui, min(gmax_r, min(r.rt1 - u, ups - ui))};
+      c = GChunk{r.rslot, u, min(gmax_r, r.rt1 - u)};
       u += c.n;
       return true;
     }
@@ -453,6 +458,8 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ __align__(8) uint64_t s_full[kXSlots], s_empty[kXSlots];
   __shared__ __align__(8) uint64_t s_xbar;
+  __shared__ __align__(8) uint64_t s_gss, s_gsr;   // gate/up scales: the shared expert's, the routed slot's
+  __shared__ __align__(8) uint64_t s_dsp, s_dsr;   // down scales: the shared expert's, the routed ones
   __shared__ int s_idx[32];
   __shared__ float s_w[kMaxSlots];
   __shared__ unsigned long long s_cand[kXWarps * 32];
@@ -464,32 +471,27 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
   const int K = p.K, NE = K + p.has_shared, H = p.H, I = p.I;
   const int NGD = I / kGroup;
   const int ups = I / RPP;                        // gate/up units per slot
-  const int DR = NGD >= 8 ? 1 : 8 / NGD;          // output rows per down unit (16-byte scale copies)
+  const int DR = NGD >= 8 ? 1 : 8 / NGD;          // output rows per down unit (16-byte scale rows)
   const int RBD = I * BITS / 8, SBD = NGD * 2;     // bytes of codes / scales per down row
   const int chD = I * BITS / 128;                  // digit chunk scalars per slot
   const int dbox = p.dmax * DR;
-  // a gate/up chunk's box: gmax_s units for the shared expert, gmax_r for the routed ones
+  // a gate/up chunk's box: gmax_s units for the shared expert, gmax_r for the routed slot
   auto gbox_of = [&](int slot) { return (slot < K ? p.gmax_r : p.gmax_s) * RPP; };
-  auto glen_of = [&](int gbox) { return r128(2u * gbox * RB) + 4u * r128((uint32_t)gbox * SB); };
-  const uint32_t dcode = r128((uint32_t)dbox * RBD), dsb = r128((uint32_t)dbox * SBD);
-  const uint32_t dlen = dcode + 2 * dsb;
+  auto glen_of = [&](int gbox) { return r128(2u * gbox * RB); };
+  const uint32_t dlen = r128((uint32_t)dbox * RBD);
   const int G = gridDim.x, b = blockIdx.x;
-  Ranges rg;
-  {
-    const int US = p.has_shared ? ups : 0, UR = K * ups, UD = H / DR;
-    rg.sh0 = (int)((long long)b * US / G);
-    rg.sh1 = (int)((long long)(b + 1) * US / G);
-    rg.rt0 = (int)((long long)b * UR / G);
-    rg.rt1 = (int)((long long)(b + 1) * UR / G);
-    rg.d0 = (int)((long long)b * UD / G);
-    rg.d1 = (int)((long long)(b + 1) * UD / G);
-  }
+  const Ranges rg = cta_ranges(b, G, K, ups, p.has_shared, H / DR);
   const int drows_all = (rg.d1 - rg.d0) * DR;                // this CTA's output rows
   const int nranges = (drows_all + dbox - 1) / dbox;
   const int nd = nranges * NE;                               // down chunks (one per slot and row range)
   uint8_t* xd = sm;                                          // digits of x, then of the activations
-  uint8_t* ring = sm + p.xd_bytes;
+  // scales: gate/up rows [sbox_s shared rows + sbox_r routed rows][4][SB] (gate s, gate b,
+  // up s, up b of a row together), down [NE][scale, bias][drows][SBD]
+  uint8_t* gsc = sm + p.xd_bytes;
+  uint8_t* dsc = gsc + r128(4u * (p.sbox_s + p.sbox_r) * SB);
+  uint8_t* ring = sm + p.xd_bytes + p.sc_bytes;
   const uint32_t RING = (uint32_t)p.ring_bytes;
+  const uint32_t dslot = 2u * p.drows * SBD;                 // bytes per slot in the down scales
 
   if (tid == 0) {
     for (int i = 0; i < kXSlots; ++i) {
@@ -497,6 +499,10 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
       mbar_init(smem_addr(&s_empty[i]), kXWarps);
     }
     mbar_init(smem_addr(&s_xbar), 1);
+    mbar_init(smem_addr(&s_gss), 1);
+    mbar_init(smem_addr(&s_gsr), 1);
+    mbar_init(smem_addr(&s_dsp), kXWarps * 32);  // one cp.async arrival per consumer thread
+    mbar_init(smem_addr(&s_dsr), kXWarps * 32);
     mbar_fence_init();
     s_abort = 0;
     s_issued = 0;
@@ -504,9 +510,11 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
   __syncthreads();
 
   if (warp == kXWarps) {
-    // ================================================================ producer warp
-    // One ring, chunks in order: the gate/up chunks (shared expert, then routed), then
-    // the down chunks (per row range, one per slot, the shared expert's first).
+    // ================================================================ producer warp (lane 0 issues)
+    // One ring, chunks in order: the gate/up chunks (shared expert, then the routed slot),
+    // then the down chunks (per row range, one per slot, the shared expert's first).
+    // Every copy is a tensor copy of a whole box: the TMA engine spends about as long on
+    // a small copy as on a large one, so copies are few and large.
     const uint64_t pol = l2_policy_evict_first();
     bool ok = true;
     RingProd<kXSlots> rpr;
@@ -514,63 +522,40 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
     rpr.empty = s_empty;
     GChunkIt git(rg);
     GChunk gc;
-    bool ghave = git.next(gc, rg, K, ups, p.gmax_s, p.gmax_r);
+    bool ghave = git.next(gc, rg, K, p.gmax_s, p.gmax_r);
     auto issue_g = [&](const GChunk& c, uint32_t vs) {
-      const uint32_t d = smem_addr(ring + vs % RING);
-      const uint32_t bar = smem_addr(&s_full[rpr.j % kXSlots]);
-      const int rows = c.n * RPP, r0 = c.u0 * RPP, gbox = gbox_of(c.slot);
+      const int gbox = gbox_of(c.slot);
       const bool routed = c.slot < K;
-      const int e = routed ? s_idx[c.slot] : 0;
-      const uint32_t cpart = r128(2u * gbox * RB), spart = r128((uint32_t)gbox * SB);
-      if (p.use_maps) {  // two tensor copies: gate+up codes, and the four scale arrays (whole boxes)
-        if (lane == 0) {
-          mbar_expect_tx(bar, 2u * gbox * RB + 4u * gbox * SB);
-          tma_4d(d, &maps.gu_codes[routed ? 0 : 1], r0, 0, e, bar, pol);
-          tma_5d(d + cpart, &maps.gu_sb[routed ? 0 : 1], r0, 0, 0, e, bar, pol);
-        }
-      } else {  // six bulk copies of the chunk's rows
-        if (lane == 0) mbar_expect_tx(bar, (uint32_t)rows * 2 * (RB + 2 * SB));
-        __syncwarp();
-        const uint8_t* rec = routed ? p.routed.base + (long long)e * p.routed.stride : p.shared.base;
-        const long long* off = routed ? p.routed.off : p.shared.off;
-        if (lane < 2) {
-          bulk_g2s(d + lane * (uint32_t)gbox * RB, rec + off[lane == 0 ? 0 : 3] + (long long)r0 * RB,
-                   (uint32_t)rows * RB, bar, pol);
-        } else if (lane < 6) {
-          const int i = lane - 2;
-          bulk_g2s(d + cpart + i * spart, rec + off[i == 0 ? 1 : i == 1 ? 2 : i == 2 ? 4 : 5] + (long long)r0 * SB,
-                   (uint32_t)rows * SB, bar, pol);
-        }
+      if (lane == 0) {
+        const uint32_t bar = smem_addr(&s_full[rpr.j % kXSlots]);
+        mbar_expect_tx(bar, 2u * gbox * RB);
+        tma_4d(smem_addr(ring + vs % RING), &maps.gu_codes[routed ? 0 : 1], c.u0 * RPP, 0, routed ? s_idx[c.slot] : 0,
+               bar, pol);
       }
       __syncwarp();
       ++rpr.j;
     };
     auto issue_d = [&](int jd, uint32_t vs) {
-      const uint32_t d = smem_addr(ring + vs % RING);
-      const uint32_t bar = smem_addr(&s_full[rpr.j % kXSlots]);
       const int range = jd / NE, slot = down_slot(jd % NE, K, p.has_shared);
-      const int row0 = rg.d0 * DR + range * dbox, rows = min(dbox, drows_all - range * dbox);
       const bool routed = slot < K;
-      const int e = routed ? s_idx[slot] : 0;
-      if (p.use_maps) {  // two tensor copies: codes, scales + biases (whole boxes)
-        if (lane == 0) {
-          mbar_expect_tx(bar, (uint32_t)dbox * (RBD + 2 * SBD));
-          tma_3d(d, &maps.dn_codes[routed ? 0 : 1], row0, e, bar, pol);
-          tma_4d(d + dcode, &maps.dn_sb[routed ? 0 : 1], row0, 0, e, bar, pol);
-        }
-      } else {
-        if (lane == 0) mbar_expect_tx(bar, (uint32_t)rows * (RBD + 2 * SBD));
-        __syncwarp();
-        const uint8_t* rec = routed ? p.routed.base + (long long)e * p.routed.stride : p.shared.base;
-        const long long* off = routed ? p.routed.off : p.shared.off;
-        if (lane < 3) {
-          const uint32_t unit = lane == 0 ? RBD : SBD;
-          bulk_g2s(d + (lane == 0 ? 0u : dcode + (lane - 1) * dsb), rec + off[6 + lane] + (long long)row0 * unit,
-                   (uint32_t)rows * unit, bar, pol);
-        }
+      if (lane == 0) {
+        const uint32_t bar = smem_addr(&s_full[rpr.j % kXSlots]);
+        mbar_expect_tx(bar, (uint32_t)dbox * RBD);
+        tma_3d(smem_addr(ring + vs % RING), &maps.dn_codes[routed ? 0 : 1], rg.d0 * DR + range * dbox,
+               routed ? s_idx[slot] : 0, bar, pol);
       }
       __syncwarp();
       ++rpr.j;
+    };
+    // gate/up scales of a segment: one tensor copy of the segment's rows (whole box)
+    auto issue_gs = [&](bool routed, int row0, uint32_t dst, uint64_t* bar_) {
+      if (lane == 0) {
+        const int box = routed ? p.sbox_r : p.sbox_s;
+        const uint32_t bar = smem_addr(bar_);
+        mbar_expect_tx(bar, 4u * box * SB);
+        tma_5d(dst, &maps.gu_sb[routed ? 0 : 1], 0, 0, row0, routed ? s_idx[rg.rslot] : 0, bar, pol);
+      }
+      __syncwarp();
     };
     // L2 requests for this CTA's down rows of slot `slot` (codes, scales, biases), lanes base..base+2
     auto ask_l2_down = [&](int slot, int base) {
@@ -583,12 +568,13 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
         prefetch_l2(rec + off[6 + m] + (long long)rg.d0 * DR * unit, (uint32_t)(drows_all * unit));
       }
     };
-    // Before the dependency wait (weights only): the shared expert's gate/up chunks as far
-    // as they fit without waiting, and an L2 request for its down rows.
+    // Before the dependency wait (weights only): the shared expert's gate/up scales and
+    // chunks as far as they fit without waiting, and an L2 request for its down rows.
     uint32_t vs;
+    if (p.has_shared && rg.sh1 > rg.sh0) issue_gs(false, rg.sh0 * RPP, smem_addr(gsc), &s_gss);
     while (ghave && gc.slot == K && rpr.reserve(glen_of(gbox_of(gc.slot)), false, vs, ok, p.err)) {
       issue_g(gc, vs);
-      ghave = git.next(gc, rg, K, ups, p.gmax_s, p.gmax_r);
+      ghave = git.next(gc, rg, K, p.gmax_s, p.gmax_r);
     }
     if (p.has_shared) ask_l2_down(K, 0);
     pdl_wait();
@@ -600,9 +586,11 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
       bulk_g2s(smem_addr(xd + C::kXDigitBytes), p.xq_cs, C::kXChunks * 8, bx, l2_policy_evict_last());
     }
     named_bar_sync(kBarAll, kXThreads);  // the routing is in s_idx
+    if (rg.rt1 > rg.rt0)
+      issue_gs(true, rg.rt0 * RPP, smem_addr(gsc + 4u * p.sbox_s * SB), &s_gsr);
     while (ok && ghave && rpr.reserve(glen_of(gbox_of(gc.slot)), true, vs, ok, p.err)) {
       issue_g(gc, vs);
-      ghave = git.next(gc, rg, K, ups, p.gmax_s, p.gmax_r);
+      ghave = git.next(gc, rg, K, p.gmax_s, p.gmax_r);
     }
     // every gate/up chunk is out: ask L2 for the routed down rows, then stage the down chunks
     for (int k = 0; k < K && 3 * k < 32; ++k) ask_l2_down(k, 3 * k);
@@ -613,6 +601,24 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
     }
   } else {
     // ================================================================ consumer warps
+    // Down scale arrays of the CTA's output rows, by cp.async from every consumer thread
+    // (the shared expert's before the dependency wait, the routed ones once gate/up is
+    // done, while the CTAs wait for one another).  Each thread arrives once per batch.
+    const uint32_t dsa = smem_addr(dsc);
+    auto cp_rows = [&](uint32_t dst, const uint8_t* src, uint32_t bytes) {
+      for (uint32_t o = 16u * tid; o < bytes; o += 16u * kXWarps * 32) cp_async16(dst + o, src + o);
+    };
+    auto cp_down_scales = [&](int slot) {
+      const bool routed = slot < K;
+      const uint8_t* rec = routed ? p.routed.base + (long long)s_idx[slot] * p.routed.stride : p.shared.base;
+      const long long* off = routed ? p.routed.off : p.shared.off;
+#pragma unroll 1
+      for (int m = 0; m < 2; ++m)
+        cp_rows(dsa + slot * dslot + m * p.drows * SBD, rec + off[7 + m] + (long long)rg.d0 * DR * SBD,
+                (uint32_t)drows_all * SBD);
+    };
+    if (p.has_shared) cp_down_scales(K);
+    cp_async_arrive(smem_addr(&s_dsp));
     pdl_wait();  // the router's logits and the digits of x are complete
     pdl_trigger();
     if (p.logits && !p.route_idx) {
@@ -665,16 +671,19 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
     {
       GChunkIt git(rg);
       GChunk c;
-      for (; git.next(c, rg, K, ups, p.gmax_s, p.gmax_r); ++jc) {
+      for (; git.next(c, rg, K, p.gmax_s, p.gmax_r); ++jc) {
         const int gbox = gbox_of(c.slot);
         const uint32_t vs = rp.place(glen_of(gbox), RING);
+        const bool routed_c = c.slot < K;
+        if (ok && !mbar_wait_bounded(smem_addr(routed_c ? &s_gsr : &s_gss), 0, p.err)) ok = false;
         if (ok && !mbar_wait_bounded(smem_addr(&s_full[jc % kXSlots]), (uint32_t)((jc / kXSlots) & 1), p.err))
           ok = false;
         const uint8_t* buf = ring + vs % RING;
-        const uint8_t* sbase = buf + r128(2u * gbox * RB);
-        const uint32_t spart = r128((uint32_t)gbox * SB);
+        // this chunk's rows among the CTA's staged scale rows
+        const int crow = routed_c ? p.sbox_s + (c.u0 - rg.rt0) * RPP : (c.u0 - rg.sh0) * RPP;
         for (int t = warp; ok && t < c.n; t += kXWarps) {
           const int rr = t * RPP + sub;  // row within the chunk
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(gsc + (size_t)(crow + rr) * 4 * SB);
           float ag = 0.0f, au = 0.0f;
 #pragma unroll
           for (int q = 0; q < GPL; ++q) {
@@ -682,10 +691,10 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
             uint4 q0, q1, v0, v1;
             load_group_codes<BITS>(buf + rr * RB, g, q0, q1);
             load_group_codes<BITS>(buf + gbox * RB + rr * RB, g, v0, v1);
-            const float gs = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + rr * SB)[g]);
-            const float gb = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + spart + rr * SB)[g]);
-            const float us = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + 2 * spart + rr * SB)[g]);
-            const float ub = bf16_to_f32(reinterpret_cast<const uint16_t*>(sbase + 3 * spart + rr * SB)[g]);
+            const float gs = bf16_to_f32(sc[g]);
+            const float gb = bf16_to_f32(sc[SB / 2 + g]);
+            const float us = bf16_to_f32(sc[SB + g]);
+            const float ub = bf16_to_f32(sc[3 * SB / 2 + g]);
             float Sg, Su;
             if constexpr (C::kRegDigits) {
               Sg = group_dot<BITS>(q0, q1, L[q]);
@@ -711,8 +720,12 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
       }
     }
 
-    // ---- hand-off: count this CTA in, wait until every CTA is in.  One thread each
-    // (consumer threads issue no bulk copies, so their fences do not wait on any).
+    // ---- the routed down scales (needed only after the hand-off), then the hand-off:
+    // count this CTA in, wait until every CTA is in.  One thread each (consumer threads
+    // issue no bulk copies, so their fences do not wait on any).
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) cp_down_scales(k);
+    cp_async_arrive(smem_addr(&s_dsr));
     named_bar_sync(kBarCons, kXWarps * 32);
     if (tid == 0) {
       __threadfence();
@@ -726,20 +739,31 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
     uint8_t* dl = xd;                                                                  // [NE][NGD * 192]
     float2* dcs = reinterpret_cast<float2*>(xd + (size_t)NE * NGD * kGroupWords * 4);  // [NE][chD]
     {
-      constexpr int kQ = 128 / kXWarps;  // groups per warp at most (NE * NGD <= 128)
-      float2 v[kQ];
+      // this warp's groups q = warp + 8 i, four at a time; the next four are loaded before
+      // the current four are digitised (a use waits for its load)
+      const int nq = NE * NGD, mine = (nq - warp + kXWarps - 1) / kXWarps;
+      float2 cur[4], nxt[4];
+      auto load4 = [&](int i0, float2 (&v)[4]) {
 #pragma unroll
-      for (int i = 0; i < kQ; ++i) {
-        const int q = warp + kXWarps * i;
-        v[i] = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)min(q, NE * NGD - 1) * kGroup) + lane);
-      }
-#pragma unroll
-      for (int i = 0; i < kQ; ++i) {
-        const int q = warp + kXWarps * i;
-        if (q < NE * NGD) {
-          const int s = q / NGD, g = q - s * NGD;
-          xq_quantize_group<BITS>(v[i].x, v[i].y, g, NGD, dl + (size_t)s * NGD * kGroupWords * 4, dcs + (size_t)s * chD);
+        for (int k = 0; k < 4; ++k) {
+          const int q = min(warp + kXWarps * (i0 + k), nq - 1);
+          v[k] = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)q * kGroup) + lane);
         }
+      };
+      load4(0, cur);
+#pragma unroll 1
+      for (int i0 = 0; i0 < mine; i0 += 4) {
+        if (i0 + 4 < mine) load4(i0 + 4, nxt);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (i0 + k < mine) {
+            const int q = warp + kXWarps * (i0 + k), s = q / NGD, g = q - s * NGD;
+            xq_quantize_group<BITS>(cur[k].x, cur[k].y, g, NGD, dl + (size_t)s * NGD * kGroupWords * 4,
+                                    dcs + (size_t)s * chD);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cur[k] = nxt[k];
       }
     }
     named_bar_sync(kBarCons, kXWarps * 32);
@@ -765,6 +789,8 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
       qs[m] = s;
       qg[m] = g;
     }
+    if (ok && !(mbar_wait_bounded(smem_addr(&s_dsp), 0, p.err) && mbar_wait_bounded(smem_addr(&s_dsr), 0, p.err)))
+      ok = false;
     for (int range = 0; range < nranges; ++range) {
       // the range's NE chunks, in issue order; this lane's slots' buffers
       const uint8_t* sbuf[DPPL];
@@ -789,8 +815,9 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
           const int g = qg[m];
           const uint4 q0 = *reinterpret_cast<const uint4*>(sb + rr * RBD + g * (kGroup * BITS / 8));
           const uint4 q1 = BITS == 4 ? *reinterpret_cast<const uint4*>(sb + rr * RBD + g * (kGroup * BITS / 8) + 16) : q0;
-          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + dcode + rr * SBD)[g]);
-          const float bi = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + dcode + dsb + rr * SBD)[g]);
+          const uint8_t* ss_ = dsc + qs[m] * dslot + (size_t)(range * dbox + rr) * SBD;
+          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(ss_)[g]);
+          const float bi = bf16_to_f32(reinterpret_cast<const uint16_t*>(ss_ + p.drows * SBD)[g]);
           const float S = group_dot<BITS>(q0, q1, LD[m]);
           acc = fmaf(wq[m], fmaf(sc, csd[m].x * S, bi * csd[m].y), acc);
         }
@@ -817,6 +844,12 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
     for (int q = s_issued > kXSlots ? s_issued - kXSlots : 0; q < s_issued; ++q)
       mbar_wait_bounded(smem_addr(&s_full[q % kXSlots]), (uint32_t)((q / kXSlots) & 1), p.err);
     mbar_wait_bounded(smem_addr(&s_xbar), 0, p.err);
+    if (p.has_shared && rg.sh1 > rg.sh0) mbar_wait_bounded(smem_addr(&s_gss), 0, p.err);
+    if (rg.rt1 > rg.rt0) mbar_wait_bounded(smem_addr(&s_gsr), 0, p.err);
+  }
+  if (s_abort && tid < kXWarps * 32) {  // every consumer thread's cp.async copies
+    mbar_wait_bounded(smem_addr(&s_dsp), 0, p.err);
+    mbar_wait_bounded(smem_addr(&s_dsr), 0, p.err);
   }
 }
 
@@ -848,36 +881,42 @@ bool encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* di
   return r == CUDA_SUCCESS;
 }
 
-// The maps of both banks, or false when the layout does not allow them (then the kernel
-// takes bulk copies): gate and up (and scale and bias) sub-arrays must sit at uniform
-// distances inside a record, rows of at most 2048 bytes of codes and at least 16 of scales.
+// The two-kernel path stages every array by tensor copies of whole boxes, which needs:
+// rows of at most 2048 bytes of codes, at least 16 bytes of scales, and a record
+// layout in which up's arrays sit at one distance from gate's, and each bias array at
+// one distance from its scale array.
+bool tok_layout_ok(const BankRef& r, int bits, int H, int I) {
+  const long long NG = H / kGroup, NGD = I / kGroup;
+  if ((long long)H * bits / 8 > 2048 || (long long)I * bits / 8 > 2048 || NG * 2 < 16 || NGD * 2 < 16) return false;
+  const long long* o = r.off;
+  const long long gu = o[3] - o[0], gus = o[4] - o[1], sb = o[2] - o[1];
+  return gu > 0 && gus > 0 && sb > 0 && o[5] - o[2] == gus && o[5] - o[4] == sb && o[8] > o[7];
+}
+
 bool encode_tok_maps(TokMaps& M, const TokExpertParams& p, int bits) {
   const int H = p.H, I = p.I, NG = H / kGroup, NGD = I / kGroup;
-  const long long RB = (long long)H * bits / 8, SB = NG * 2, RBD = (long long)I * bits / 8, SBD = NGD * 2;
-  if (RB > 2048 || RBD > 2048 || SB < 16 || SBD < 16) return false;
+  const long long RB = (long long)H * bits / 8, SB = NG * 2, RBD = (long long)I * bits / 8;
   const int LPR = NG < 32 ? NG : 32, RPP = 32 / LPR, DR = NGD >= 8 ? 1 : 8 / NGD;
   const int dbox = p.dmax * DR;
-  if (p.gmax_r * RPP > 256 || p.gmax_s * RPP > 256 || dbox > 256) return false;
+  if (p.gmax_r * RPP > 256 || p.gmax_s * RPP > 256 || dbox > 256 || p.sbox_r > 256 || p.sbox_s > 256) return false;
   for (int bk = 0; bk < 2; ++bk) {
-    const int gbox = (bk == 0 ? p.gmax_r : p.gmax_s) * RPP;
     const BankRef& r = bk == 0 ? p.routed : p.shared;
+    if (!tok_layout_ok(r, bits, H, I)) return false;
     const long long* o = r.off;
-    const long long gu = o[3] - o[0], sbd = o[2] - o[1];
-    if (o[4] - o[1] != gu || o[5] - o[2] != gu || o[5] - o[4] != sbd || gu <= 0 || sbd <= 0) return false;
-    const long long dsb = o[8] - o[7];
-    if (dsb <= 0) return false;
     const cuuint64_t ne = bk == 0 ? (cuuint64_t)p.routed.num_experts : 1;
     const cuuint64_t est = bk == 0 ? (cuuint64_t)r.stride : 16;
     {
+      const int gbox = (bk == 0 ? p.gmax_r : p.gmax_s) * RPP;
       const cuuint64_t dims[4] = {(cuuint64_t)(RB / 8), (cuuint64_t)I, 2, ne};
-      const cuuint64_t st[3] = {(cuuint64_t)RB, (cuuint64_t)gu, est};
+      const cuuint64_t st[3] = {(cuuint64_t)RB, (cuuint64_t)(o[3] - o[0]), est};
       const cuuint32_t box[4] = {(cuuint32_t)(RB / 8), (cuuint32_t)gbox, 2, 1};
       if (!encode_map(&M.gu_codes[bk], r.base + o[0], 4, dims, st, box)) return false;
     }
     {
-      const cuuint64_t dims[5] = {(cuuint64_t)(SB / 8), (cuuint64_t)I, 2, 2, ne};
-      const cuuint64_t st[4] = {(cuuint64_t)SB, (cuuint64_t)sbd, (cuuint64_t)gu, est};
-      const cuuint32_t box[5] = {(cuuint32_t)(SB / 8), (cuuint32_t)gbox, 2, 2, 1};
+      const int sbox = bk == 0 ? p.sbox_r : p.sbox_s;
+      const cuuint64_t dims[5] = {(cuuint64_t)(SB / 8), 2, 2, (cuuint64_t)I, ne};
+      const cuuint64_t st[4] = {(cuuint64_t)(o[2] - o[1]), (cuuint64_t)(o[4] - o[1]), (cuuint64_t)SB, est};
+      const cuuint32_t box[5] = {(cuuint32_t)(SB / 8), 2, 2, (cuuint32_t)(sbox > 0 ? sbox : 1), 1};
       if (!encode_map(&M.gu_sb[bk], r.base + o[1], 5, dims, st, box)) return false;
     }
     {
@@ -885,12 +924,6 @@ bool encode_tok_maps(TokMaps& M, const TokExpertParams& p, int bits) {
       const cuuint64_t st[2] = {(cuuint64_t)RBD, est};
       const cuuint32_t box[3] = {(cuuint32_t)(RBD / 8), (cuuint32_t)dbox, 1};
       if (!encode_map(&M.dn_codes[bk], r.base + o[6], 3, dims, st, box)) return false;
-    }
-    {
-      const cuuint64_t dims[4] = {(cuuint64_t)(SBD / 8), (cuuint64_t)H, 2, ne};
-      const cuuint64_t st[3] = {(cuuint64_t)SBD, (cuuint64_t)dsb, est};
-      const cuuint32_t box[4] = {(cuuint32_t)(SBD / 8), (cuuint32_t)dbox, 2, 1};
-      if (!encode_map(&M.dn_sb[bk], r.base + o[7], 4, dims, st, box)) return false;
     }
   }
   return true;
@@ -937,7 +970,7 @@ TokPlan plan_token(int bits, int H, int I, int K, int has_shared) {
   const size_t xd = round128(std::max((size_t)NG * kGroupWords * 4 + chX * 8,
                                       (size_t)NE * ((size_t)NGD * kGroupWords * 4 + chD * 8)));
   if (xd + 4096 > kXSmemBudget || NE + 4 > kXSlots) return pl;
-  const size_t ring = (kXSmemBudget - xd) / 128 * 128;
+  size_t ring = (kXSmemBudget - xd) / 128 * 128;
   int grid = num_sms();
   if (grid > kMaxTokenCtas) grid = kMaxTokenCtas;
   const int DR = NGD >= 8 ? 1 : 8 / NGD;
@@ -948,20 +981,25 @@ TokPlan plan_token(int bits, int H, int I, int K, int has_shared) {
   const size_t unitG = RPP * 2 * (RB + 2 * SB);
   const int cap = (int)std::max<size_t>(1, std::min<size_t>(std::min(kXChunkTarget, ring / 4) / unitG, 256 / RPP));
   const int ups = I / RPP;
-  auto even = [&](int units_total) {
-    const int avg = std::max(1, (units_total + grid - 1) / grid);
+  if (grid < K) return pl;
+  // the routed units of a slot are dealt out to its run of grid / K CTAs
+  const int per_r = (ups + grid / K - 1) / (grid / K), per_s = has_shared ? (ups + grid - 1) / grid : 0;
+  auto even_r = [&](int avg) {
+    avg = std::max(1, avg);
     const int n = (avg + cap - 1) / cap;
     return (avg + n - 1) / n;
   };
-  const int gmax_r = even(K * ups), gmax_s = has_shared ? even(ups) : 1;
-  const size_t glen = round128(2 * (size_t)std::max(gmax_r, gmax_s) * RPP * RB) +
-                      4 * round128((size_t)std::max(gmax_r, gmax_s) * RPP * SB);
-  // down ranges: the CTA's whole share when its NE chunks fit in half the ring
-  auto dlen_of = [&](int dm) {
-    const size_t rows = (size_t)dm * DR;
-    return round128(rows * RBD) + 2 * round128(rows * SBD);
-  };
+  const int gmax_r = even_r(per_r), gmax_s = has_shared ? even_r(per_s) : 1;
+  const size_t glen = round128(2 * (size_t)std::max(gmax_r, gmax_s) * RPP * RB);
+  // scales of the CTA's rows: gate/up [sbox_s + sbox_r rows][4][SB], down [NE][2][drows][SBD]
   const int UD = H / DR, dshare = (UD + grid - 1) / grid;
+  const int sbox_s = per_s * RPP, sbox_r = per_r * RPP;
+  const int drows = dshare * DR;
+  const size_t sc = round128(4 * (size_t)(sbox_s + sbox_r) * SB) + round128((size_t)NE * 2 * drows * SBD);
+  if (xd + sc + glen > kXSmemBudget) return pl;
+  ring = (kXSmemBudget - xd - sc) / 128 * 128;
+  // down ranges: the CTA's whole share when its NE chunks fit in half the ring
+  auto dlen_of = [&](int dm) { return round128((size_t)dm * DR * RBD); };
   int dmax = std::min(dshare, std::min(kXMaxDRows, 256) / DR);
   while (dmax > 1 && (size_t)NE * dlen_of(dmax) > ring / 2) --dmax;
   const int NP = NE * NGD, part = NP > 64 ? (NP + 1) / 2 : NP;
@@ -972,10 +1010,19 @@ TokPlan plan_token(int bits, int H, int I, int K, int has_shared) {
   pl.gmax_r = gmax_r;
   pl.dmax = dmax;
   pl.xd_bytes = (int)xd;
+  pl.sc_bytes = (int)sc;
+  pl.sbox_s = sbox_s;
+  pl.sbox_r = sbox_r;
+  pl.drows = drows;
   pl.ring_bytes = (int)ring;
   pl.dppl = (part + 31) / 32;
-  pl.smem = xd + ring;
+  pl.smem = xd + sc + ring;
   return pl;
+}
+
+bool token_path_supported(int bits, int H, int I, int K, int has_shared, const BankRef& routed, const BankRef& shared) {
+  return plan_token(bits, H, I, K, has_shared).ok && tok_layout_ok(routed, bits, H, I) &&
+         tok_layout_ok(shared, bits, H, I);
 }
 
 cudaError_t launch_tok_router(TokRouterParams p, int bits, bool pdl, cudaStream_t s) {
@@ -1015,10 +1062,14 @@ cudaError_t launch_tok_expert(TokExpertParams p, int bits, bool pdl, cudaStream_
   p.gmax_r = pl.gmax_r;
   p.dmax = pl.dmax;
   p.xd_bytes = pl.xd_bytes;
+  p.sc_bytes = pl.sc_bytes;
+  p.sbox_s = pl.sbox_s;
+  p.sbox_r = pl.sbox_r;
+  p.drows = pl.drows;
   p.ring_bytes = pl.ring_bytes;
   TokMaps m;
   memset(&m, 0, sizeof(m));
-  p.use_maps = token_maps_enabled() && encode_tok_maps(m, p, bits) ? 1 : 0;
+  if (!encode_tok_maps(m, p, bits)) return cudaErrorNotSupported;
   return bits == 4 ? expert_bits<4>(p, m, pl.dppl, pl.smem, pl.grid, pdl, s)
                    : expert_bits<2>(p, m, pl.dppl, pl.smem, pl.grid, pdl, s);
 }
