@@ -50,6 +50,8 @@ SIGNATURES = [
     ("fmoe_moe_layer", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("fmoe_moe_layer_workspace_size", _sz, [ctypes.POINTER(FmoeLayer), _i]),
     ("fmoe_moe_layer_static", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _vp]),
+    ("fmoe_moe_layer_routed", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    ("fmoe_wait_flag", _i, [_vp, ctypes.c_uint32, ctypes.c_int64, _vp, _vp]),
     ("fmoe_moe_stack", _i, [ctypes.POINTER(FmoeLayer), _i, _vp, _i, _vp, _vp, _sz, _vp]),
     ("fmoe_trace_next_layer", _i, [ctypes.POINTER(ctypes.c_void_p), _i]),
     ("fmoe_workspace_init", _i, [_vp, _sz, _vp]),
@@ -225,6 +227,25 @@ def moe_layer_static(layer, h, out=None, topk_idx=None, topk_w=None, dev_err=Non
                                        _ptr(topk_w, torch.float32, "topk_w"), _ptr(dev_err, torch.int32, "dev_err"),
                                        _stream(stream)))
     return out
+
+
+def moe_layer_routed(layer, h, topk_idx, topk_w, out=None, ws=None, stream=None):
+    """The block with the caller's routing (int32 [T][K] experts, fp32 [T][K] weights)."""
+    T = h.shape[0] if h.dim() == 2 else 1
+    out = torch.empty_like(h) if out is None else out
+    if ws is None:
+        ws = workspace(moe_layer_workspace_size(layer, 1), h.device, stream)
+    _check(lib().fmoe_moe_layer_routed(ctypes.byref(layer.s), _ptr(h, torch.float32, "h"), T,
+                                       _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
+                                       _ptr(out, torch.float32, "out"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                       _stream(stream)))
+    return out
+
+
+def wait_flag(flag, value, limit_ns, ws, stream=None):
+    """Bounded stream-ordered wait until flag (int32/uint32 device tensor of one element) == value."""
+    _check(lib().fmoe_wait_flag(_ptr(flag, None, "flag"), int(value), int(limit_ns), _ptr(ws, torch.uint8, "ws"),
+                                _stream(stream)))
 
 
 def moe_stack(layers, h, out=None, ws=None, stream=None):

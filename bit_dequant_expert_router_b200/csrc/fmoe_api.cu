@@ -400,7 +400,8 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
 }
 
 static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
-                                  uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word);
+                                  uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word,
+                                  const int32_t* given_idx = nullptr, const float* given_w = nullptr);
 
 // One token through the block: router kernel (RMSNorm, logits, digits of x), then
 // the expert kernel (top-K, gate/up + SwiGLU, down + combine + residual).
@@ -460,8 +461,11 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
   return FMOE_OK;
 }
 
+// given_idx / given_w ([K] each, device): the routing given by the caller instead of the
+// top-K of the logits (the router still runs, for x, its digits and the shared gate).
 static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
-                                  uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word) {
+                                  uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word,
+                                  const int32_t* given_idx, const float* given_w) {
   const fmoe_bank& r = layer->routed;
   const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
@@ -484,6 +488,8 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
   rp.top_k = 0;  // the expert kernels select the experts from the logits themselves
   rp.tickets = ctrl->tickets;
   rp.route_ready = &ctrl->route_ready;
+  rp.clear = reinterpret_cast<unsigned int*>(base + L.grp_cnt);
+  rp.nclear = (K + 1) * (I / 64 > 0 ? I / 64 : 1);
   rp.err = err_word ? err_word : &ctrl->err;
   const bool trace = g_trace_on;
   g_trace_on = false;
@@ -518,12 +524,25 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
   p.rt_idx = reinterpret_cast<int32_t*>(base + L.route_idx);
   p.rt_w = reinterpret_cast<float*>(base + L.route_w);
   p.route_ready = &ctrl->route_ready;  // gate/up CTA 0 sets it once rt_idx / rt_w are written
+  if (given_idx) {
+    p.logits = nullptr;
+    p.route_idx = given_idx;
+    p.idx_out = nullptr;
+    p.w_out = nullptr;
+    p.route_ready = nullptr;
+  }
   if ((e = launch_gateup(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "gate/up launch");
   if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   ExpertParams pd = p;  // the down kernel reads the routing the gate/up kernel wrote
   pd.logits = nullptr;
   pd.route_idx = p.rt_idx;
   pd.route_w = p.rt_w;
+  if (given_idx) {  // launched below with the caller's routing
+    pd.route_idx = given_idx;
+    pd.route_w = given_w;
+    pd.sigma_logit = rp.logits + E;
+    pd.route_ready = nullptr;
+  }
   if ((e = launch_down(pd, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "down launch");
   if (trace && (e = trace_record(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   return FMOE_OK;
@@ -766,6 +785,40 @@ fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T
   uint8_t* base = nullptr;
   if ((st = static_scratch(&base)) != FMOE_OK) return st;
   return moe_layer_impl(layer, h, T, out, topk_idx, topk_w, base, kStaticScratchBytes, L, cs(stream), dev_err);
+}
+
+fmoe_status fmoe_moe_layer_routed(const fmoe_layer* layer, const float* h, int T, const int32_t* topk_idx,
+                                  const float* topk_w, float* out, void* ws, size_t ws_bytes, fmoe_stream_t stream) {
+  fmoe_status st = check_layer(layer);
+  if (st != FMOE_OK) return st;
+  if (T < 0) return fail(FMOE_ERR_INVALID_ARG, "T %d", T);
+  if (T == 0) return FMOE_OK;
+  if (!h || !out || !topk_idx || !topk_w) return fail(FMOE_ERR_INVALID_ARG, "h, out, topk_idx or topk_w is NULL");
+  if (!aligned16(h) || !aligned16(out)) return fail(FMOE_ERR_ALIGNMENT, "h and out must be 16-byte aligned");
+  if (((uintptr_t)topk_idx & 3u) || ((uintptr_t)topk_w & 3u))
+    return fail(FMOE_ERR_ALIGNMENT, "topk_idx and topk_w must be 4-byte aligned");
+  const int H = layer->routed.hidden, K = layer->top_k;
+  const WsLayout L = layout(H, layer->routed.num_experts, K, layer->routed.inter, 1);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != FMOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  for (int t = 0; t < T; ++t) {
+    st = layer_token_3k(layer, h + (size_t)t * H, out + (size_t)t * H, nullptr, nullptr, base, L, cs(stream), nullptr,
+                        topk_idx + (size_t)t * K, topk_w + (size_t)t * K);
+    if (st != FMOE_OK) return st;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_wait_flag(const uint32_t* flag, uint32_t value, int64_t limit_ns, void* ws, fmoe_stream_t stream) {
+  if (!flag) return fail(FMOE_ERR_INVALID_ARG, "flag is NULL");
+  if (((uintptr_t)flag & 3u) != 0) return fail(FMOE_ERR_ALIGNMENT, "flag must be 4-byte aligned");
+  if (limit_ns <= 0 || limit_ns > 60000000000LL) return fail(FMOE_ERR_INVALID_ARG, "limit_ns %lld (1 ns .. 60 s)",
+                                                             (long long)limit_ns);
+  if (!ws) return fail(FMOE_ERR_WORKSPACE, "workspace is NULL");
+  if (((uintptr_t)ws & (kAlign - 1)) != 0) return fail(FMOE_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  WsControl* ctrl = static_cast<WsControl*>(ws);
+  cudaError_t e = launch_wait_flag(flag, value, (unsigned long long)limit_ns, &ctrl->err, cs(stream));
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "wait launch");
 }
 
 fmoe_status fmoe_moe_stack(const fmoe_layer* layers, int nl, const float* h, int T, float* out, void* ws,

@@ -32,6 +32,9 @@ struct RouterParams {
   float* w_out;
   unsigned int* tickets;      // [T], zero between calls
   unsigned int* route_ready;  // or NULL: cleared once the predecessor is complete (see ExpertParams)
+  unsigned int* clear;        // or NULL: nclear counters that CTA 0 zeroes once the predecessor is
+  int nclear;                 // complete (the gate/up kernel's group counters, so that a call never
+                              // depends on the previous one having finished cleanly)
   int* err;
 };
 
@@ -51,6 +54,8 @@ struct ExpertParams {
                               // experts itself; NULL: the routing below
   const int32_t* route_idx;   // [K] selected experts or NULL (fixed_expert)
   const float* route_w;       // [K+1] weights, slot K = shared-gate sigma; NULL: weight 1
+  const float* sigma_logit;   // or NULL; when set, the down kernel takes the routed weights from route_w
+                              // [K] and sigma = sigmoid(*sigma_logit) (the routing given by the caller)
   int32_t* idx_out;           // with logits: the caller's copy of the routing [K], [K] (gate/up CTA 0), or NULL
   float* w_out;
   int32_t* rt_idx;            // with logits: gate/up CTA 0 writes the routing here for the down kernel
@@ -257,6 +262,8 @@ cudaError_t launch_down(const ExpertParams& p, int bits, bool pdl, cudaStream_t 
 int num_sms();
 bool expert_shapes_supported(int bits, int H, int I, int num_slots);
 bool pdl_enabled();
+cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err,
+                             cudaStream_t s);
 cudaError_t set_smem(const void* kernel, size_t bytes);
 cudaError_t set_carveout_max(const void* kernel);
 

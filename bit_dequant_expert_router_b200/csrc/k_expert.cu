@@ -393,7 +393,9 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
       s_src[lane][2] = rec + p.routed.off[8];
       s_w[lane] = p.route_w ? __ldcg(p.route_w + lane) : 1.0f;
     }
-    if (lane == 0 && p.has_shared) s_w[p.K] = p.route_w ? __ldcg(p.route_w + p.K) : 1.0f;
+    if (lane == 0 && p.has_shared)
+      s_w[p.K] = p.sigma_logit ? 1.0f / (1.0f + expf(-__ldcg(p.sigma_logit)))
+                               : (p.route_w ? __ldcg(p.route_w + p.K) : 1.0f);
   };
   // Published already (gate/up CTA 0 finished its selection long before this grid
   // starts, in practice)?  Warp 1 has no copies in flight, so its acquire does not wait.
@@ -486,6 +488,12 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
   }
   if (!ok && tid == 0)
     for (int b = 0; b < nbuf; ++b) mbar_wait_bounded(smem_addr(&s_bar[b]), 0, p.err);
+}
+
+// One thread waits until *flag == value, at most limit_ns; on timeout it records
+// FMOE_ERR_DEVICE_TIMEOUT in *err and returns.
+__global__ void wait_flag_kernel(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err) {
+  flag_wait_bounded(flag, value, limit_ns, err);
 }
 
 size_t round128(size_t v) { return (v + 127) / 128 * 128; }
@@ -679,6 +687,12 @@ bool fits_u(int ngu, int ngd, int ne) {
 bool expert_shapes_supported(int bits, int H, int I, int ne) {
   if (H % kGroup || I % kGroup) return false;
   return bits == 4 ? fits_u<4>(H / kGroup, I / kGroup, ne) : fits_u<2>(H / kGroup, I / kGroup, ne);
+}
+
+cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err,
+                             cudaStream_t s) {
+  wait_flag_kernel<<<1, 1, 0, s>>>(flag, value, limit_ns, err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gateup(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {

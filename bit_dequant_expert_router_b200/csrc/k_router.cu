@@ -103,8 +103,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
   if (blockIdx.x == 0 && tid == 0) prefetch_l2(p.h + (size_t)t * H, (uint32_t)H * 4);
   pdl_wait();
   pdl_trigger();
-  // every kernel of the previous token is complete: its routing flag is spent
+  // every kernel of the previous token is complete: its routing flag is spent, and the
+  // gate/up kernel's group counters are cleared (they return to zero by themselves unless
+  // a bounded wait gave up part-way)
   if (p.route_ready && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *p.route_ready = 0u;
+  if (p.clear && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = tid; i < p.nclear; i += kRouterThreads) p.clear[i] = 0u;
 
   const float* h = p.h + (size_t)t * H;
   float ss = 0.0f;

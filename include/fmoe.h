@@ -160,9 +160,12 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
 
 /* fmoe_moe_layer without a workspace argument: the pages have no counterpart
  * (their engine owns all its buffers); this is an interface convenience.
- * Computes exactly what fmoe_moe_layer computes, with the same kernels, but its
- * scratch is a fixed device array inside libfmoe.so of FMOE_STATIC_SCRATCH_BYTES
- * (512 KiB) per device, so the call allocates nothing.  It serves callers that
+ * Computes what fmoe_moe_layer computes, but its scratch is a fixed device array
+ * inside libfmoe.so of FMOE_STATIC_SCRATCH_BYTES (512 KiB) per device, so the call
+ * allocates nothing.  Batches of T >= 8 tokens take the expert-grouped kernels only
+ * when their grouped layout fits the scratch (small layers); otherwise, e.g. for the
+ * Qwen3.5-397B-A17B shapes, they run token by token, which reads every selected
+ * expert's rows once per token.  It serves callers that
  * cannot hand over a workspace: a plain-C or FFI host that keeps no device
  * allocator, or an engine whose memory planner has reserved the whole device.
  * Arguments as fmoe_moe_layer, plus:
@@ -172,7 +175,9 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
  *            the library.  NULL: such failures are recorded only inside the
  *            static scratch, where no call reports them.
  * The scratch needs no set-up: it is zero when the library's module loads on
- * a device, and every call leaves its counters at zero again.  Its address is
+ * a device, and the first kernel of every token clears the counters the later
+ * ones use.  A call after which dev_err is non-zero has invalid outputs; the
+ * scratch itself needs no reset, since the next call clears its counters again.  Its address is
  * looked up (cudaGetSymbolAddress) on the first call on each device; make that
  * first call outside any CUDA stream capture.
  * One scratch per device is shared by every caller of this function: two calls
@@ -186,6 +191,28 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
  * check only guards against shapes later versions may admit. */
 fmoe_status fmoe_moe_layer_static(const fmoe_layer* layer, const float* h, int T, float* out, int32_t* topk_idx,
                                   float* topk_w, int* dev_err, fmoe_stream_t stream);
+
+/* The block with the routing given by the caller instead of selected from the logits
+ * (for a routing recorded earlier or made elsewhere; the pages' engine selects on the
+ * CPU and hands the choice to the GPU, "Flash-MoE" wiki summary, per-layer pipeline):
+ *   out[t] = h[t] + sum_k topk_w[t][k] FFN_{topk_idx[t][k]}(x[t]) + sigma[t] FFN_shared(x[t]),
+ * with x = RMSNorm(h) and sigma = sigmoid(w_shared_gate . x) as in fmoe_moe_layer; the
+ * weights are used as given (not renormalised).
+ * topk_idx: device int32 [T][K]; topk_w: device fp32 [T][K] (4-byte aligned).  Other
+ * arguments and requirements as fmoe_moe_layer (token by token; the T = 1 workspace
+ * size suffices).  An index outside [0, num_experts) is not checked on the host: the
+ * kernels replace it by expert 0 and record it, and fmoe_workspace_check then returns
+ * FMOE_ERR_INVALID_ARG. */
+fmoe_status fmoe_moe_layer_routed(const fmoe_layer* layer, const float* h, int T, const int32_t* topk_idx,
+                                  const float* topk_w, float* out, void* ws, size_t ws_bytes, fmoe_stream_t stream);
+
+/* Stream-ordered, bounded wait: work enqueued on `stream` after this call starts once
+ * *flag == value (a device word, or mapped host memory, set by another stream, the host
+ * or a peer), or once limit_ns (1 ns .. 60 s) have passed; in that case the workspace's
+ * error word records it and fmoe_workspace_check returns FMOE_ERR_DEVICE_TIMEOUT.  The
+ * kernels of this library bound every wait the same way.  ws: any workspace of this
+ * library (its control words are used).  flag: 4-byte aligned. */
+fmoe_status fmoe_wait_flag(const uint32_t* flag, uint32_t value, int64_t limit_ns, void* ws, fmoe_stream_t stream);
 
 /* A stack of L layers applied in order, each block's output feeding the next
  * (the 60-layer decode loop of the jeongsk wiki summary, without the attention

@@ -108,3 +108,25 @@ def test_other_entry_points_validate():
     assert L.fmoe_expert_ffn(ctypes.byref(b), -1, 0x1000, 0x2000, 0x5000, 1 << 20, None) == 1
     assert L.fmoe_moe_stack(None, 1, 0x1000, 1, 0x1000, 0x5000, 1 << 20, None) == 1
     assert L.fmoe_workspace_init(None, 100, None) == 4
+
+
+def test_routed_layer_and_wait_flag_reject_bad_arguments_before_any_launch():
+    L = fmoe.lib()
+    lay = _fake_layer()
+    ok = (ctypes.byref(lay), 0x60000000, 1, 0x70000000, 0x70001000, 0x60000000, 0x50000000, 1 << 30, None)
+    # NULL routing, misaligned routing, misaligned h, workspace too small
+    assert L.fmoe_moe_layer_routed(ctypes.byref(lay), 0x60000000, 1, None, 0x70001000, 0x60000000, 0x50000000,
+                                   1 << 30, None) == 1
+    assert L.fmoe_moe_layer_routed(ctypes.byref(lay), 0x60000000, 1, 0x70000002, 0x70001000, 0x60000000, 0x50000000,
+                                   1 << 30, None) == 2
+    assert L.fmoe_moe_layer_routed(ctypes.byref(lay), 0x60000008, 1, 0x70000000, 0x70001000, 0x60000000, 0x50000000,
+                                   1 << 30, None) == 2
+    assert L.fmoe_moe_layer_routed(ctypes.byref(lay), 0x60000000, 1, 0x70000000, 0x70001000, 0x60000000, 0x50000000,
+                                   1024, None) == 4
+    assert L.fmoe_moe_layer_routed(ctypes.byref(lay), 0x60000000, 0, *ok[3:]) == 0
+    # the bounded wait: limits outside 1 ns .. 60 s, NULL or misaligned flag or workspace
+    assert L.fmoe_wait_flag(0x70000000, 1, 0, 0x50000000, None) == 1
+    assert L.fmoe_wait_flag(0x70000000, 1, 61 * 10 ** 9, 0x50000000, None) == 1
+    assert L.fmoe_wait_flag(None, 1, 1000, 0x50000000, None) == 1
+    assert L.fmoe_wait_flag(0x70000002, 1, 1000, 0x50000000, None) == 2
+    assert L.fmoe_wait_flag(0x70000000, 1, 1000, 0x50000010, None) == 2

@@ -103,3 +103,50 @@ def test_static_scratch_matches_workspace_entry_point_full_size():
     _both(m, lay, h, lay.top_k)
     del dl
     torch.cuda.empty_cache()
+
+
+@pytest.mark.gpu
+def test_static_scratch_grouped_and_token_by_token_batches():
+    """hidden 512: a T = 8 batch's grouped layout fits the static scratch, so it runs
+    expert-grouped there; T = 16 does not fit and runs token by token.  Two static calls
+    in a row with different T share the scratch.  Both against fmoe_moe_layer."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_dequant_expert_router_b200 as m
+    L = m.lib()
+    spec = gen.small_layer(4)
+    dl = gen.upload_layer(gen.host_layer(spec, seed=41))
+    lay = gen.binding_layer(dl)
+    assert L.fmoe_moe_layer_workspace_size(ctypes.byref(lay.s), 8) <= STATIC_BYTES
+    assert L.fmoe_moe_layer_workspace_size(ctypes.byref(lay.s), 16) > STATIC_BYTES
+    _both(m, lay, torch.from_numpy(gen.host_tokens(4100, 8, spec.hidden)).cuda(), lay.top_k)
+    _both(m, lay, torch.from_numpy(gen.host_tokens(4200, 16, spec.hidden)).cuda(), lay.top_k)
+
+
+@pytest.mark.gpu
+def test_static_scratch_full_size_batch_runs_token_by_token():
+    """The Qwen3.5-397B-A17B-shaped layer with T = 8: the grouped layout exceeds the static
+    scratch, so the batch runs token by token, with the results of fmoe_moe_layer."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_dequant_expert_router_b200 as m
+    spec = gen.qwen397_layer(4)
+    dl = gen.device_layer(spec)
+    lay = gen.binding_layer(dl)
+    h = gen.device_tokens(4300, 8, spec.hidden)
+    # the caller workspace holds only the per-token layout, so both calls run token by token
+    T, K = 8, lay.top_k
+    ref = torch.empty_like(h)
+    ref_idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    ws = m.workspace(m.moe_layer_workspace_size(lay, 1))
+    m.moe_layer(lay, h, out=ref, topk_idx=ref_idx, ws=ws)
+    m.workspace_check(ws)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(h)
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    m.moe_layer_static(lay, h, out=out, topk_idx=idx, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(idx, ref_idx) and torch.equal(out, ref)
+    del dl
+    torch.cuda.empty_cache()
