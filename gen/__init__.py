@@ -1,4 +1,5 @@
-"""Seeded synthetic inputs for the routed-MoE block: shapes, layouts and generators.
+"""Seeded synthetic inputs for the routed-MoE block and the Gated DeltaNet state update:
+shapes, layouts and generators.
 
 Both the CPU oracle (through the host library) and the GPU path (through the
 device library) consume the bytes drawn here; this module holds none of the
@@ -342,4 +343,69 @@ def device_tokens(t0, T, hidden, device="cuda"):
     stream = torch.cuda.current_stream().cuda_stream
     for i in range(T):
         device_normal_f32(token_key(t0 + i), 1.0, out[i], stream)
+    return out
+
+
+# ----------------------------------------------------------------------------------------------- Gated DeltaNet
+# Inputs of the linear-attention state update (64 heads x 128 x 128 in the Qwen3.5-397B-A17B
+# description of the Flash-MoE pages).  Recipe: state entries N(0, 0.1^2) fp32; k a fresh
+# N(0,1) draw per head scaled to unit L2 norm; q the same, times dk^-1/2; v N(0,1); the
+# decay gate alpha uniform in [0.8, 1.0) and the write strength beta uniform in [0, 1),
+# both on a 2^-24 grid.  Every token draws fresh q, k, v, alpha, beta.
+
+GDN_SEED = 2
+GDN_Q, GDN_K, GDN_V, GDN_ALPHA, GDN_BETA, GDN_STATE = range(6)
+
+
+@dataclasses.dataclass(frozen=True)
+class GdnSpec:
+    """n independent heads (batch x heads), each a dv x dk fp32 state."""
+    heads: int
+    dk: int
+    dv: int
+    state_std: float = 0.1
+
+
+def gdn_qwen397(batch=1):
+    """Qwen3.5-397B-A17B linear-attention layer: 64 heads of 128 x 128, `batch` sequences."""
+    return GdnSpec(heads=64 * batch, dk=128, dv=128)
+
+
+def gdn_key(layer, t, kind):
+    return int(host_lib().fg_host_key(GDN_SEED, (int(layer) << 40) | (int(t) << 4) | int(kind)))
+
+
+def _gdn_uniform(k, n):
+    u = np.empty(n, dtype=np.uint32)
+    host_lib().fg_host_uniform_u32(k, 1 << 24, n, u.ctypes.data)
+    return u.astype(np.float32) * np.float32(2.0 ** -24)
+
+
+def _unit_rows(a):
+    return (a / np.sqrt(np.sum(a.astype(np.float64) ** 2, axis=1, keepdims=True))).astype(np.float32)
+
+
+def host_gdn_state(spec, layer=0):
+    """Initial state of one layer: fp32 [heads][dv][dk]."""
+    n = spec.heads * spec.dv * spec.dk
+    return host_normal_f32(gdn_key(layer, 0, GDN_STATE), spec.state_std, n).reshape(spec.heads, spec.dv, spec.dk)
+
+
+def host_gdn_token(spec, layer, t):
+    """Token t's inputs to one layer: q, k fp32 [heads][dk], v [heads][dv], alpha, beta [heads]."""
+    n, dk, dv = spec.heads, spec.dk, spec.dv
+    k = _unit_rows(host_normal_f32(gdn_key(layer, t, GDN_K), 1.0, n * dk).reshape(n, dk))
+    q = (_unit_rows(host_normal_f32(gdn_key(layer, t, GDN_Q), 1.0, n * dk).reshape(n, dk))
+         * np.float32(1.0 / math.sqrt(dk))).astype(np.float32)
+    v = host_normal_f32(gdn_key(layer, t, GDN_V), 1.0, n * dv).reshape(n, dv)
+    alpha = (np.float32(0.8) + np.float32(0.2) * _gdn_uniform(gdn_key(layer, t, GDN_ALPHA), n)).astype(np.float32)
+    beta = _gdn_uniform(gdn_key(layer, t, GDN_BETA), n)
+    return dict(q=q, k=k, v=v, alpha=alpha, beta=beta)
+
+
+def device_gdn_state(spec, layer=0, device="cuda"):
+    """The same initial state as host_gdn_state, drawn on the device."""
+    import torch
+    out = torch.empty((spec.heads, spec.dv, spec.dk), dtype=torch.float32, device=device)
+    device_normal_f32(gdn_key(layer, 0, GDN_STATE), spec.state_std, out, torch.cuda.current_stream().cuda_stream)
     return out

@@ -1,4 +1,5 @@
-"""CPU oracle of the routed-MoE decode block (fp64, plain C) -- TEST INFRASTRUCTURE ONLY.
+"""CPU oracle of the routed-MoE decode block and of the Gated DeltaNet state update
+(fp64, plain C) -- TEST INFRASTRUCTURE ONLY.
 
 Only the tests, the smoke check and the benchmark's CPU-baseline leg may import
 this package.  It shares no code with the CUDA path; inputs are numpy arrays in
@@ -55,6 +56,7 @@ def lib():
         L.or_topk.argtypes = [vp, ci, ci, vp]
         L.or_expert_ffn.argtypes = [ctypes.POINTER(OrBank), ci, vp, vp, vp]
         L.or_moe_layer.argtypes = [ctypes.POINTER(OrLayer), vp, ci, vp, vp, vp, vp, vp, vp, vp]
+        L.or_gdn_step.argtypes = [ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
         L.or_set_threads.argtypes = [ci]
         L.or_get_threads.restype = ci
         L.or_max_threads.restype = ci
@@ -195,3 +197,18 @@ class Layer:
         lib().or_moe_layer(ctypes.byref(self.s), h.ctypes.data, T, _p(fi), out.ctypes.data, idx.ctypes.data,
                            w.ctypes.data, probs.ctypes.data, logits.ctypes.data, sigma.ctypes.data)
         return dict(out=out, idx=idx, w=w, probs=probs, logits=logits, sigma=sigma)
+
+
+def gdn_step(S, q, k, v, alpha, beta):
+    """One gated-delta-rule step of n heads (or_gdn_step): S [n][dv][dk], q/k [n][dk], v [n][dv],
+    alpha/beta [n], any float dtype (widened to fp64).  Returns (new state, o [n][dv]) in fp64;
+    the inputs are not modified."""
+    S = np.array(S, dtype=np.float64, order="C", copy=True)
+    n, dv, dk = S.shape
+    q, k = _c(q, np.float64).reshape(n, dk), _c(k, np.float64).reshape(n, dk)
+    v = _c(v, np.float64).reshape(n, dv)
+    alpha, beta = _c(alpha, np.float64).reshape(n), _c(beta, np.float64).reshape(n)
+    o = np.empty((n, dv), dtype=np.float64)
+    lib().or_gdn_step(n, dk, dv, S.ctypes.data, q.ctypes.data, k.ctypes.data, v.ctypes.data, alpha.ctypes.data,
+                      beta.ctypes.data, o.ctypes.data)
+    return S, o

@@ -1,5 +1,6 @@
 /*
- * fmoe_oracle.c -- plain, slow, fp64 CPU oracle of the routed-MoE decode block.
+ * fmoe_oracle.c -- plain, slow, fp64 CPU oracle of the routed-MoE decode block
+ * and of the Gated DeltaNet state update.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
  * call this file; only the tests, the smoke check and the benchmark's CPU
@@ -15,7 +16,10 @@
  *     squares, then apply), fused SwiGLU, and one combine pass of the weighted
  *     expert outputs, the residual and the sigmoid-gated shared expert;
  *   - "Flash-MoE" wiki summary (jeongsk), per-layer pipeline: routing
- *     projection, then softmax and top-K selection.
+ *     projection, then softmax and top-K selection;
+ *   - same page section 4 and the wiki summary's key technique 4: the Gated
+ *     DeltaNet state update of the linear-attention layers (or_gdn_step, at
+ *     the end of this file).
  * Readings where the pages are silent (code order LSB-first, unsigned codes,
  * groups of 64 along the input dimension, router [E][H] in bf16, softmax over
  * all E then top-K then renormalisation, ties to the lower index, eps 1e-6)
@@ -248,4 +252,49 @@ void or_moe_layer(const or_layer* L, const float* h, int T, const int* force_idx
   free(l);
   free(p);
   free(idx);
+}
+
+/* ------------------------------------------------------------------------------------
+ * Gated DeltaNet state update, one decode step.
+ *
+ * "What is Flash-MoE" (a2a-mcp.org), section 4 (Accelerate BLAS for the Gated DeltaNet
+ * layers), and the "Flash-MoE" wiki summary (jeongsk), key technique 4: each of the 45
+ * linear-attention layers keeps a 128 x 128 state matrix per head, 64 heads, and updates
+ * it with three single-precision BLAS calls: a scaling (sscal), a matrix-vector product
+ * (sgemv) and a rank-1 update (sger).  Read as the gated delta rule, per head and in
+ * that order:
+ *   S <- alpha S                    scaling: the gate decays the whole memory
+ *   u  = S k                        matrix-vector: what the memory returns for key k
+ *   S <- S + beta (v - u) k^T       rank-1 update: move the answer for k toward v
+ *   o  = S q                        matrix-vector: the read-out for query q
+ * S: [n][dv][dk] (row i of a head is value coordinate i, column j key coordinate j),
+ * updated in place; q, k: [n][dk]; v, o: [n][dv]; alpha, beta: [n].  Each step is its
+ * own loop, in the order above; OpenMP runs heads (independent) in parallel.
+ * ------------------------------------------------------------------------------------ */
+void or_gdn_step(int n, int dk, int dv, double* S, const double* q, const double* k, const double* v,
+                 const double* alpha, const double* beta, double* o) {
+#pragma omp parallel for schedule(dynamic, 1) num_threads(g_threads)
+  for (int h = 0; h < n; ++h) {
+    double* Sh = S + (int64_t)h * dv * dk;
+    const double* qh = q + (int64_t)h * dk;
+    const double* kh = k + (int64_t)h * dk;
+    const double* vh = v + (int64_t)h * dv;
+    const double a = alpha[h], b = beta[h];
+    double* u = (double*)malloc(sizeof(double) * (size_t)dv);
+    for (int i = 0; i < dv; ++i)
+      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= a;
+    for (int i = 0; i < dv; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * kh[j];
+      u[i] = acc;
+    }
+    for (int i = 0; i < dv; ++i)
+      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];
+    for (int i = 0; i < dv; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * qh[j];
+      o[(int64_t)h * dv + i] = acc;
+    }
+    free(u);
+  }
 }

@@ -3,8 +3,10 @@
 Each case plants one slip in a copy of the oracle's C source: a wrong code
 order, a dropped or mis-signed term, a wrong group index, a transposed operand,
 a missing normalisation, a reversed tie-break, swapped SwiGLU operands, a
-missing residual or shared term.  The copy is compiled with the oracle's own
-flags into a temporary directory, the pin suite (test_oracle_pins.py) runs
+missing residual or shared term; in the Gated DeltaNet step a skipped decay, a
+recall from the undecayed state, a wrong delta sign or a missing delta term, a
+dropped write strength, a transposed rank-1 update, a read-out with the wrong
+vector.  The copy is compiled with the oracle's own flags into a temporary directory, the pin suite (test_oracle_pins.py) runs
 against it in a child process, and at least one pin must fail.  The real
 oracle is never touched.
 """
@@ -94,6 +96,27 @@ MUTATIONS = [
     ("shared expert dropped",
      "for (int i = 0; i < H; ++i) ot[i] += sigma * y[i];",
      "for (int i = 0; i < H; ++i) ot[i] += 0.0 * sigma * y[i];"),
+    ("gdn decay skipped",
+     "for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= a;",
+     "for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= 1.0;"),
+    ("gdn recall from the undecayed state",
+     "for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * kh[j];",
+     "for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] / a * kh[j];"),
+    ("gdn delta sign",
+     "Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];",
+     "Sh[(int64_t)i * dk + j] += b * (u[i] - vh[i]) * kh[j];"),
+    ("gdn no delta term (plain linear attention)",
+     "Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];",
+     "Sh[(int64_t)i * dk + j] += b * vh[i] * kh[j];"),
+    ("gdn write strength dropped",
+     "Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];",
+     "Sh[(int64_t)i * dk + j] += (vh[i] - u[i]) * kh[j];"),
+    ("gdn outer product transposed",
+     "Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];",
+     "Sh[(int64_t)i * dk + j] += b * (vh[j % dv] - u[j % dv]) * kh[i % dk];"),
+    ("gdn read-out with the key",
+     "for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * qh[j];",
+     "for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * kh[j];"),
 ]
 
 

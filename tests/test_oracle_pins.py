@@ -275,3 +275,97 @@ def test_sparse_record_table_equals_full_bank():
     from tests.helpers import oracle_layer_sparse
     part = oracle_layer_sparse(sub).forward(h, force_idx=full["idx"])
     assert np.array_equal(full["out"], part["out"])
+
+
+# ----------------------------------------------------------------------------------------------- Gated DeltaNet
+# The state update of the linear-attention layers ("What is Flash-MoE", section 4; "Flash-MoE"
+# wiki summary, key technique 4).  The oracle takes the three BLAS steps one by one; the pins
+# below fix it by the gated delta rule's product form, by what the delta rule guarantees
+# (writing v at a unit key k and reading k back returns v; directions orthogonal to k only
+# decay), and by its special cases.  Shapes are non-square (dv != dk) so that a transposed
+# operand cannot pass.
+
+def _gdn_case(seed, n=3, dk=8, dv=5):
+    rng = np.random.default_rng(seed)
+    S = rng.standard_normal((n, dv, dk))
+    q = rng.standard_normal((n, dk))
+    k = rng.standard_normal((n, dk))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((n, dv))
+    alpha = rng.uniform(0.5, 1.0, n)
+    beta = rng.uniform(0.1, 1.0, n)
+    return S, q, k, v, alpha, beta
+
+
+def test_gdn_equals_the_gated_delta_rule_product_form():
+    # S' = alpha S (I - beta k k^T) + beta v k^T and o = S' q, for keys of any norm
+    S, q, k, v, alpha, beta = _gdn_case(0)
+    k = k * np.array([[0.5], [1.0], [2.0]])
+    S2, o = oracle.gdn_step(S, q, k, v, alpha, beta)
+    for h in range(S.shape[0]):
+        P = alpha[h] * S[h] @ (np.eye(S.shape[2]) - beta[h] * np.outer(k[h], k[h])) + beta[h] * np.outer(v[h], k[h])
+        assert np.allclose(S2[h], P, rtol=0, atol=1e-13)
+        assert np.allclose(o[h], P @ q[h], rtol=0, atol=1e-13)
+
+
+def test_gdn_full_write_at_a_unit_key_reads_back_the_value():
+    S, q, k, v, alpha, _ = _gdn_case(1)
+    S2, o = oracle.gdn_step(S, k, k, v, alpha, np.ones(3))   # query = key
+    for h in range(3):
+        assert np.allclose(S2[h] @ k[h], v[h], rtol=0, atol=1e-13)
+        assert np.allclose(o[h], v[h], rtol=0, atol=1e-13)
+
+
+def test_gdn_directions_orthogonal_to_the_key_only_decay():
+    S, q, k, v, alpha, beta = _gdn_case(2)
+    S2, _ = oracle.gdn_step(S, q, k, v, alpha, beta)
+    rng = np.random.default_rng(3)
+    for h in range(3):
+        w = rng.standard_normal(S.shape[2])
+        w -= np.dot(w, k[h]) * k[h]
+        assert np.allclose(S2[h] @ w, alpha[h] * (S[h] @ w), rtol=0, atol=1e-13)
+        # and along k: S' k = alpha (1 - beta) S k + beta v
+        assert np.allclose(S2[h] @ k[h], alpha[h] * (1 - beta[h]) * (S[h] @ k[h]) + beta[h] * v[h], rtol=0,
+                           atol=1e-13)
+
+
+def test_gdn_special_cases():
+    S, q, k, v, alpha, beta = _gdn_case(4)
+    zero, one = np.zeros(3), np.ones(3)
+    S2, o = oracle.gdn_step(S, q, k, v, zero, beta)          # no memory left: a single write
+    for h in range(3):
+        assert np.allclose(S2[h], beta[h] * np.outer(v[h], k[h]), rtol=0, atol=1e-14)
+        assert np.allclose(o[h], beta[h] * np.dot(k[h], q[h]) * v[h], rtol=0, atol=1e-14)
+    S2, o = oracle.gdn_step(S, q, k, v, one, zero)           # no decay, no write
+    assert np.array_equal(S2, S)
+    assert np.allclose(o, np.einsum("hij,hj->hi", S, q), rtol=0, atol=1e-13)
+    S2, _ = oracle.gdn_step(S, q, k, v, alpha, zero)         # decay only
+    assert np.allclose(S2, alpha[:, None, None] * S, rtol=0, atol=1e-15)
+
+
+def test_gdn_orthonormal_keys_form_an_associative_memory_with_overwrite():
+    # from an empty state, full writes at orthonormal keys store every value; writing a new
+    # value at an old key replaces it and leaves the others alone (plain linear attention,
+    # without the delta term, would add the two values instead)
+    dk, dv, m = 6, 4, 5
+    rng = np.random.default_rng(5)
+    keys = np.linalg.qr(rng.standard_normal((dk, dk)))[0][:, :m].T
+    vals = rng.standard_normal((m, dv))
+    S = np.zeros((1, dv, dk))
+    for i in range(m):
+        S, _ = oracle.gdn_step(S, keys[i:i + 1], keys[i:i + 1], vals[i:i + 1], np.ones(1), np.ones(1))
+    for i in range(m):
+        assert np.allclose(S[0] @ keys[i], vals[i], rtol=0, atol=1e-13)
+    new = rng.standard_normal((1, dv))
+    S, o = oracle.gdn_step(S, keys[1:2], keys[1:2], new, np.ones(1), np.ones(1))
+    assert np.allclose(o[0], new[0], rtol=0, atol=1e-13)
+    for i in range(m):
+        assert np.allclose(S[0] @ keys[i], new[0] if i == 1 else vals[i], rtol=0, atol=1e-13)
+
+
+def test_gdn_heads_are_independent():
+    S, q, k, v, alpha, beta = _gdn_case(6)
+    S2, o = oracle.gdn_step(S, q, k, v, alpha, beta)
+    for h in range(3):
+        Sh, oh = oracle.gdn_step(S[h:h + 1], q[h:h + 1], k[h:h + 1], v[h:h + 1], alpha[h:h + 1], beta[h:h + 1])
+        assert np.array_equal(Sh[0], S2[h]) and np.array_equal(oh[0], o[h])
