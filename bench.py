@@ -28,7 +28,7 @@ import numpy as np  # noqa: E402
 METRIC = "MoE-layer decode tokens/s and effective weight GB/s (fraction of HBM peak), 1×B200"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the per-token
-# expert kernel, from one ncu capture of the current build per workload; absent where none was taken.
+# gate/up kernel, from one ncu capture of the current build per workload; absent where none was taken.
 EXPERT_TRAFFIC = {}
 # grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
 # (+ the shared expert): 1,051,820,288 B over 207.5 experts
@@ -36,7 +36,10 @@ GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5069013}
 DTYPE_TOKEN = "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32"
 DTYPE_BATCH = "i32 mma.sync (u4/u2 codes as u8 x 24-bit fixed-point x as three s8 limbs) + f32"
 BATCH_KERNELS = 8  # norm+digits, router GEMM, top-K, sort, gate/up, activation digits, down, combine
-TOKEN_KERNELS = 2  # router, expert (gate/up + SwiGLU + down + combine)
+# Per-token path: router, gate/up + SwiGLU, down + combine (three dependent launches);
+# FMOE_TOKEN_KERNELS=2 selects the two-kernel variant: router, expert (gate/up + SwiGLU
+# + down + combine in one kernel).
+TOKEN_KERNELS = 2 if os.environ.get("FMOE_TOKEN_KERNELS") == "2" else 3
 
 WORKLOADS = {
     # name: (spec factory, description)
@@ -368,8 +371,10 @@ def main():
         kernel, kbytes = "grouped_gateup_kernel", (n_active + 1) * 2 * rec_mat
         achieved = kbytes / (gateup_us * 1e-6) / 1e9 if gateup_us else step_bytes / (ms_per_step * 1e-3) / 1e9
     else:
-        # the expert kernel streams gate, up and down of the K routed experts and the shared one
-        kernel, kbytes = "tok_expert_kernel", (spec.top_k + 1) * 3 * rec_mat
+        if TOKEN_KERNELS == 2:  # one kernel streams gate, up and down of the K routed + shared experts
+            kernel, kbytes = "tok_expert_kernel", (spec.top_k + 1) * 3 * rec_mat
+        else:  # the gate/up kernel streams gate and up of the K routed + shared experts
+            kernel, kbytes = "gateup_kernel", (spec.top_k + 1) * 2 * rec_mat
         achieved = kbytes / (gateup_us * 1e-6) / 1e9
         bytes_tok = gen.algorithmic_bytes_per_token(spec)
     eff = bytes_tok * (value / world) / 1e9
@@ -399,11 +404,13 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": (GROUPED_GATEUP_TRAFFIC_PER_EXPERT[args.workload] * (n_active + 1)
                                      if nbatch and args.workload in GROUPED_GATEUP_TRAFFIC_PER_EXPERT
-                                     else EXPERT_TRAFFIC.get(args.workload)),
+                                     else EXPERT_TRAFFIC.get(args.workload) if TOKEN_KERNELS == 3 and not nbatch
+                                     else None),
                          "kernel": kernel, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": kbytes},
             "kernels_us": ({"router_and_selection": router_us, "gateup": gateup_us, "down_and_combine": down_us}
-                           if nbatch else {"router": router_us, "expert": gateup_us}),
+                           if nbatch else {"router": router_us, "expert": gateup_us} if TOKEN_KERNELS == 2
+                           else {"router": router_us, "gateup": gateup_us, "down_and_combine": down_us}),
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (BATCH_KERNELS * steps if nbatch else TOKEN_KERNELS * steps * per_step),
             "clocks": clk.record(),
         }

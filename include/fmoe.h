@@ -211,7 +211,8 @@ fmoe_status fmoe_moe_layer_routed(const fmoe_layer* layer, const float* h, int T
  * or a peer), or once limit_ns (1 ns .. 60 s) have passed; in that case the workspace's
  * error word records it and fmoe_workspace_check returns FMOE_ERR_DEVICE_TIMEOUT.  The
  * kernels of this library bound every wait the same way.  ws: any workspace of this
- * library (its control words are used).  flag: 4-byte aligned. */
+ * library, initialised by fmoe_workspace_init (its control words are used; every size
+ * query of this library returns at least their size).  flag: 4-byte aligned. */
 fmoe_status fmoe_wait_flag(const uint32_t* flag, uint32_t value, int64_t limit_ns, void* ws, fmoe_stream_t stream);
 
 /* A stack of L layers applied in order, each block's output feeding the next

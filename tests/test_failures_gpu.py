@@ -24,7 +24,10 @@ def fmoe():
 
 
 def test_bounded_wait_on_a_flag_that_is_never_set_reports_a_timeout(fmoe):
-    ws = fmoe.workspace(4096)
+    spec = gen.tiny_layer(4)
+    hl = gen.host_layer(spec, seed=31)
+    lay = gen.binding_layer(gen.upload_layer(hl))
+    ws = fmoe.workspace(fmoe.moe_layer_workspace_size(lay, 1))
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     fmoe.wait_flag(flag, 1, 5_000_000, ws)   # 5 ms, nothing sets the flag
     with pytest.raises(fmoe.FmoeError) as e:
@@ -35,11 +38,9 @@ def test_bounded_wait_on_a_flag_that_is_never_set_reports_a_timeout(fmoe):
     fmoe.wait_flag(flag, 1, 5_000_000, ws)   # already set: returns at once, no error
     fmoe.workspace_check(ws)
     # the context is still usable: a layer call after the timeout gives the oracle's result
-    spec = gen.tiny_layer(4)
-    hl = gen.host_layer(spec, seed=31)
-    lay = gen.binding_layer(gen.upload_layer(hl))
     h = gen.host_tokens(3100, 2, spec.hidden)
-    out = fmoe.moe_layer(lay, torch.from_numpy(h).cuda()).cpu().numpy()
+    out = fmoe.moe_layer(lay, torch.from_numpy(h).cuda(), ws=ws).cpu().numpy()
+    fmoe.workspace_check(ws)
     assert max_rel_err(out, oracle_layer(hl).forward(h)["out"]) <= TOL
 
 
