@@ -55,6 +55,13 @@ WORKLOADS = {
                              "stack of 60 Qwen3.5-397B-A17B-shaped MoE blocks, 2-bit group-64 experts "
                              "(all 60 x 513 experts resident), one token through all 60 per step"),
 }
+# Gated DeltaNet state update of the linear-attention layers: (batch, layers whose states
+# are resident and stepped in turn, description); one step = one layer's update for one token.
+GDN_WORKLOADS = {
+    "qwen397-gdn": (1, 45, "Qwen3.5-397B-A17B linear-attention state update: 64 heads x 128 x 128 fp32 state, "
+                           "45 layers' states resident, one token through each in turn (batch-1 decode)"),
+}
+GDN_METRIC = "Gated DeltaNet decode state updates/s (one layer, 64 heads x 128x128 fp32) and GB/s, 1xB200"
 # Workloads that run a stack of distinct layers per token (fmoe_moe_stack); the
 # metric then counts layer-steps (one token through one layer) per second.
 STACK_LAYERS = {"qwen397-2bit-stack60": 60}
@@ -68,7 +75,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="fmoe", choices=["fmoe", "reference"])
-    ap.add_argument("--workload", default="qwen397-4bit", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="qwen397-4bit", choices=sorted(WORKLOADS) + sorted(GDN_WORKLOADS))
     ap.add_argument("--copies", type=int, default=16, help="resident layer copies rotated per token")
     ap.add_argument("--graph-tokens", type=int, default=1000, help="tokens per captured CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
@@ -206,9 +213,178 @@ def run_reference(args, spec, desc, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def gdn_bytes_per_step(spec):
+    """Algorithmic bytes of one layer's update: the state read and written once, q, k, v,
+    alpha, beta read and o written once."""
+    n, dk, dv = spec.heads, spec.dk, spec.dv
+    return 4 * (2 * n * dv * dk + n * (2 * dk + dv + 2) + n * dv)
+
+
+def cpu_oracle_gdn_rate(spec, layers, budget_s):
+    """Times the CPU oracle's gated-delta-rule step (all host cores) on a bounded sample of
+    layer-steps; drawing the inputs is not timed."""
+    import gen
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    states = {}
+    n, spent = 0, 0.0
+    while spent < budget_s and n < 100 * layers:
+        l = n % layers
+        if l not in states:
+            states[l] = gen.host_gdn_state(spec, layer=l).astype(np.float64)
+        t = gen.host_gdn_token(spec, l, n // layers)
+        s = time.perf_counter()
+        states[l], _ = oracle.gdn_step(states[l], t["q"], t["k"], t["v"], t["alpha"], t["beta"])
+        spent += time.perf_counter() - s
+        n += 1
+    return n / spent, cores, n, spent
+
+
+def run_gdn(args, world, rank, local):
+    import gen
+    batch, nlayers, desc = GDN_WORKLOADS[args.workload]
+    spec = gen.gdn_qwen397(batch)
+    bytes_step = gdn_bytes_per_step(spec)
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        rate, cores, n, spent = cpu_oracle_gdn_rate(spec, nlayers, max(args.cpu_seconds, 5.0))
+        line = {"metric": GDN_METRIC, "impl": "reference", "value": rate, "unit": "layer-steps/s",
+                "n_gpus": args.gpus, "steps": n, "warmup": 0, "ms_per_step": 1e3 / rate, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": desc},
+                "cpu_baseline": {"value": rate, "unit": "layer-steps/s", "cores": cores, "kind": "oracle",
+                                 "sample": f"{n} layer-steps ({spent:.1f} s of oracle time)"},
+                "e2e": {"value": rate, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import bit_dequant_expert_router_b200 as fmoe
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    fmoe.lib()
+    # resident: every layer's state (above L2 in total); NT token input sets per layer
+    states = [gen.device_gdn_state(spec, layer=l, device=dev) for l in range(nlayers)]
+    NT = 4
+    toks = [[{k: torch.from_numpy(v).to(dev) for k, v in gen.host_gdn_token(spec, l, rank * 1000 + t).items()}
+             for t in range(NT)] for l in range(nlayers)]
+    outs = torch.empty((nlayers, spec.heads, spec.dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    G = min(args.graph_tokens, args.steps, 900)
+    G = max(nlayers, G // nlayers * nlayers)
+    steps = (args.steps + G - 1) // G * G
+
+    def step(i, s):
+        l = i % nlayers
+        d = toks[l][(i // nlayers) % NT]
+        fmoe.gdn_step(states[l], d["q"], d["k"], d["v"], d["alpha"], d["beta"], o=outs[l], early=nlayers > 1,
+                      stream=s)
+
+    torch.cuda.synchronize(dev)
+    # warm-up in whole rounds of the layers, so that no two consecutive launches (here, into
+    # the graph, or from one replay to the next) step the same state: the early state read
+    # relies on that
+    warm = (max(args.warmup, 3) + nlayers - 1) // nlayers * nlayers
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            step(i, stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            step(i, stream)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    stream.synchronize()
+
+    def timed(g):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps // G):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+
+    def repeat(g):
+        first = max_over_ranks(timed(g), world, dev)
+        reps = max(args.reps, min(1000, int(0.3e3 / max(first, 1e-3)) + 1))
+        times = [first] + max_over_ranks([timed(g) for _ in range(reps - 1)], world, dev)
+        return statistics.median(times), len(times)
+
+    with ClockSampler(local) as clk:
+        ms, nreps = repeat(graph)
+    value = steps * world / (ms / 1e3)
+    us_launch = ms * 1e3 / steps          # every launch in the region is the update kernel
+    peak, peak_kind = peak_hbm()
+    achieved = bytes_step / (us_launch * 1e-6) / 1e9
+
+    # end to end: each step's q, k, v, alpha, beta from pinned host memory, o back to the host
+    e2e = None
+    if not args.no_e2e:
+        hin = [{k: v.cpu().pin_memory() for k, v in toks[l][0].items()} for l in range(nlayers)]
+        din = {k: torch.empty_like(v) for k, v in toks[0][0].items()}
+        hout = torch.empty((G, spec.heads, spec.dv), dtype=torch.float32).pin_memory()
+        egraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(egraph, stream=stream):
+            for i in range(G):
+                l = i % nlayers
+                for k in din:
+                    din[k].copy_(hin[l][k], non_blocking=True)
+                fmoe.gdn_step(states[l], din["q"], din["k"], din["v"], din["alpha"], din["beta"], o=outs[l],
+                              stream=stream)
+                hout[i].copy_(outs[l], non_blocking=True)
+        with torch.cuda.stream(stream):
+            egraph.replay()
+        stream.synchronize()
+        ems, _ = repeat(egraph)
+        h2d = sum(v.numel() * 4 for v in din.values())
+        e2e = {"value": steps * world / (ems / 1e3), "unit": "layer-steps/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": spec.heads * spec.dv * 4}
+        del egraph
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, n, spent = cpu_oracle_gdn_rate(spec, nlayers, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "layer-steps/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} layer-steps of this workload ({spent:.1f} s of oracle time)"}
+    if rank == 0:
+        line = {
+            "metric": GDN_METRIC, "value": value, "unit": "layer-steps/s", "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": ms / steps, "reps": nreps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": desc, "heads": spec.heads, "dk": spec.dk, "dv": spec.dv, "layers": nlayers,
+                       "graph_steps": G,
+                       "l2": f"inputs larger than L2: {nlayers} resident states "
+                             f"({nlayers * spec.heads * spec.dv * spec.dk * 4 / 1e6:.0f} MB) stepped in turn",
+                       "parallelism": f"replicas x{world}"},
+            "effective_gbs": achieved, "bytes_per_step": bytes_step,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "gdn_step_kernel",
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_step},
+            "kernels_us": {"gdn_step": us_launch},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": steps, "clocks": clk.record(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
+    if args.workload in GDN_WORKLOADS:
+        return run_gdn(args, world, rank, local)
     import gen
     spec = WORKLOADS[args.workload][0]()
     desc = WORKLOADS[args.workload][1]

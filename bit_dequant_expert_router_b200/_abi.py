@@ -52,6 +52,7 @@ SIGNATURES = [
     ("fmoe_moe_layer_static", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _vp]),
     ("fmoe_moe_layer_routed", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("fmoe_wait_flag", _i, [_vp, ctypes.c_uint32, ctypes.c_int64, _vp, _vp]),
+    ("fmoe_gdn_step", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, ctypes.c_uint32, _vp]),
     ("fmoe_moe_stack", _i, [ctypes.POINTER(FmoeLayer), _i, _vp, _i, _vp, _vp, _sz, _vp]),
     ("fmoe_trace_next_layer", _i, [ctypes.POINTER(ctypes.c_void_p), _i]),
     ("fmoe_workspace_init", _i, [_vp, _sz, _vp]),
@@ -246,6 +247,22 @@ def wait_flag(flag, value, limit_ns, ws, stream=None):
     """Bounded stream-ordered wait until flag (int32/uint32 device tensor of one element) == value."""
     _check(lib().fmoe_wait_flag(_ptr(flag, None, "flag"), int(value), int(limit_ns), _ptr(ws, torch.uint8, "ws"),
                                 _stream(stream)))
+
+
+GDN_STATE_EARLY = 1
+
+
+def gdn_step(state, q, k, v, alpha, beta, o=None, early=False, stream=None):
+    """One Gated DeltaNet decode step of n heads (fmoe_gdn_step): state fp32 [n][dv][dk] is
+    updated in place; q, k [n][dk], v [n][dv], alpha, beta [n]; returns o [n][dv].
+    early: the previous launch on the stream does not write `state` (FMOE_GDN_STATE_EARLY)."""
+    n, dv, dk = state.shape
+    o = torch.empty((n, dv), dtype=torch.float32, device=state.device) if o is None else o
+    f32 = torch.float32
+    _check(lib().fmoe_gdn_step(_ptr(state, f32, "state"), _ptr(q, f32, "q"), _ptr(k, f32, "k"), _ptr(v, f32, "v"),
+                               _ptr(alpha, f32, "alpha"), _ptr(beta, f32, "beta"), _ptr(o, f32, "o"), n, dk, dv,
+                               GDN_STATE_EARLY if early else 0, _stream(stream)))
+    return o
 
 
 def moe_stack(layers, h, out=None, ws=None, stream=None):

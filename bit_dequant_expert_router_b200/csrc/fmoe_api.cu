@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "fmoe.h"
+#include "fmoe_gdn.h"
 #include "fmoe_internal.h"
 
 namespace fmoe {
@@ -237,6 +238,35 @@ fmoe_status fmoe_rmsnorm(const float* h, const float* gamma, float eps, int T, i
   if (!(eps >= 0.0f)) return fail(FMOE_ERR_INVALID_ARG, "eps %g", (double)eps);
   cudaError_t e = launch_rmsnorm(h, gamma, eps, T, H, y, cs(stream));
   return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "rmsnorm launch");
+}
+
+fmoe_status fmoe_gdn_step(float* state, const float* q, const float* k, const float* v, const float* alpha,
+                          const float* beta, float* o, int n, int dk, int dv, unsigned flags, fmoe_stream_t stream) {
+  if (n < 0 || dv < 1) return fail(FMOE_ERR_INVALID_ARG, "n %d, dv %d", n, dv);
+  if (flags & ~FMOE_GDN_STATE_EARLY) return fail(FMOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (!gdn_shape_supported(dk)) return fail(FMOE_ERR_UNSUPPORTED, "dk %d (128, 256, 384 or 512)", dk);
+  if ((long long)n * dv > 0x7fffffffLL) return fail(FMOE_ERR_UNSUPPORTED, "n * dv = %lld rows", (long long)n * dv);
+  if (n == 0) return FMOE_OK;
+  if (!state || !q || !k || !v || !alpha || !beta || !o)
+    return fail(FMOE_ERR_INVALID_ARG, "state, q, k, v, alpha, beta and o must be non-NULL");
+  if (!aligned16(state) || !aligned16(q) || !aligned16(k))
+    return fail(FMOE_ERR_ALIGNMENT, "state, q and k must be 16-byte aligned");
+  if ((((uintptr_t)v | (uintptr_t)alpha | (uintptr_t)beta | (uintptr_t)o) & 3u) != 0)
+    return fail(FMOE_ERR_ALIGNMENT, "v, alpha, beta and o must be 4-byte aligned");
+  GdnParams p{};
+  p.state = state;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.rows = n * dv;
+  p.dk = dk;
+  p.dv = dv;
+  p.early = (flags & FMOE_GDN_STATE_EARLY) ? 1 : 0;
+  cudaError_t e = launch_gdn_step(p, pdl_enabled(), cs(stream));
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "gdn step launch");
 }
 
 // The per-token path: three kernels (router, gate/up, down) unless FMOE_TOKEN_KERNELS=2

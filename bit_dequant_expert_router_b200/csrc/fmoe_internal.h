@@ -261,6 +261,22 @@ cudaError_t launch_down(const ExpertParams& p, int bits, bool pdl, cudaStream_t 
 
 int num_sms();
 bool expert_shapes_supported(int bits, int H, int I, int num_slots);
+
+// Gated DeltaNet state update, one decode step of `rows / dv` heads (k_gdn.cu).
+struct GdnParams {
+  float* state;               // [n][dv][dk], updated in place
+  const float* q;             // [n][dk]
+  const float* k;             // [n][dk]
+  const float* v;             // [n][dv]
+  const float* alpha;         // [n]
+  const float* beta;          // [n]
+  float* o;                   // [n][dv]
+  int rows;                   // n * dv
+  int dk, dv;
+  int early;                  // 1: read the state before the dependency wait
+};
+bool gdn_shape_supported(int dk);
+cudaError_t launch_gdn_step(const GdnParams& p, bool pdl, cudaStream_t s);
 bool pdl_enabled();
 cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err,
                              cudaStream_t s);

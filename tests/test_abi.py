@@ -130,3 +130,22 @@ def test_routed_layer_and_wait_flag_reject_bad_arguments_before_any_launch():
     assert L.fmoe_wait_flag(None, 1, 1000, 0x50000000, None) == 1
     assert L.fmoe_wait_flag(0x70000002, 1, 1000, 0x50000000, None) == 2
     assert L.fmoe_wait_flag(0x70000000, 1, 1000, 0x50000010, None) == 2
+
+
+def test_gdn_step_rejects_bad_arguments_before_any_launch():
+    L = fmoe.lib()
+    S, q, k, v, a, b, o = 0x60000000, 0x61000000, 0x62000000, 0x63000000, 0x64000000, 0x65000000, 0x66000000
+    good = (S, q, k, v, a, b, o)
+    assert L.fmoe_gdn_step(*good, 0, 128, 128, 0, None) == 0          # n = 0: nothing enqueued
+    assert L.fmoe_gdn_step(*good, -1, 128, 128, 0, None) == 1         # negative n
+    assert L.fmoe_gdn_step(*good, 64, 128, 0, 0, None) == 1           # dv < 1
+    assert L.fmoe_gdn_step(*good, 64, 128, 128, 2, None) == 1         # unknown flag
+    assert L.fmoe_gdn_step(None, *good[1:], 64, 128, 128, 0, None) == 1
+    assert L.fmoe_gdn_step(*good[:6], None, 64, 128, 128, 1, None) == 1
+    for dk in (64, 96, 200, 640):
+        assert L.fmoe_gdn_step(*good, 64, dk, 128, 0, None) == 3      # unsupported key width
+    assert L.fmoe_gdn_step(*good, 1 << 20, 128, 4096, 0, None) == 3   # rows beyond 2^31
+    assert L.fmoe_gdn_step(S + 8, *good[1:], 64, 128, 128, 0, None) == 2
+    assert L.fmoe_gdn_step(S, q + 4, *good[2:], 64, 128, 128, 0, None) == 2
+    assert L.fmoe_gdn_step(*good[:3], v + 2, *good[4:], 64, 128, 128, 0, None) == 2
+    assert L.fmoe_gdn_step(*good[:6], o + 1, 64, 128, 128, 0, None) == 2
