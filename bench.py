@@ -29,7 +29,7 @@ METRIC = "MoE-layer decode tokens/s and effective weight GB/s (fraction of HBM p
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the per-token
 # gate/up kernel, from one ncu capture of the current build per workload; absent where none was taken.
-EXPERT_TRAFFIC = {}
+EXPERT_TRAFFIC = {"qwen397-4bit": 30657536}
 # grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
 # (+ the shared expert): 1,051,820,288 B over 207.5 experts
 GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5069013}
@@ -82,6 +82,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--reps", type=int, default=5, help="timed repetitions of the steps-token region (median)")
+    ap.add_argument("--min-seconds", type=float, default=0.3,
+                    help="repeat the timed region until it covers this long in total (for the clock record)")
     return ap.parse_args()
 
 
@@ -317,7 +319,7 @@ def run_gdn(args, world, rank, local):
 
     def repeat(g):
         first = max_over_ranks(timed(g), world, dev)
-        reps = max(args.reps, min(1000, int(0.3e3 / max(first, 1e-3)) + 1))
+        reps = max(args.reps, min(1000, int(args.min_seconds * 1e3 / max(first, 1e-3)) + 1))
         times = [first] + max_over_ranks([timed(g) for _ in range(reps - 1)], world, dev)
         return statistics.median(times), len(times)
 
@@ -465,7 +467,7 @@ def main():
 
     def repeat(g):
         first = max_over_ranks(timed(g), world, dev)  # every rank agrees on the count
-        reps = max(args.reps, min(1000, int(0.3e3 / max(first, 1e-3)) + 1))
+        reps = max(args.reps, min(1000, int(args.min_seconds * 1e3 / max(first, 1e-3)) + 1))
         times = [first] + max_over_ranks([timed(g) for _ in range(reps - 1)], world, dev)
         return statistics.median(times), len(times)
 
