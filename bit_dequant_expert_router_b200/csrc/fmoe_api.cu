@@ -719,15 +719,16 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   g_trace_on = false;
   cudaError_t e;
   if (trace && (e = trace_record(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
-  if ((e = launch_grouped_router(p, rb, bits, s)) != cudaSuccess)
+  const bool pdl = pdl_enabled() && !trace;
+  if ((e = launch_grouped_router(p, rb, bits, pdl, s)) != cudaSuccess)
     return cuda_fail(e, "router launch");
-  if ((e = launch_grouped_select(p, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  if ((e = launch_grouped_select(p, pdl, s)) != cudaSuccess) return cuda_fail(e, "select launch");
   if (trace && (e = trace_record(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
-  if ((e = launch_grouped_gateup(p, bits, s)) != cudaSuccess) return cuda_fail(e, "grouped gate/up launch");
+  if ((e = launch_grouped_gateup(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "grouped gate/up launch");
   if (trace && (e = trace_record(g_trace[2], s)) != cudaSuccess) return cuda_fail(e, "trace event");
-  if ((e = launch_grouped_actq(p, bits, s)) != cudaSuccess) return cuda_fail(e, "activation digits launch");
-  if ((e = launch_grouped_down(p, bits, s)) != cudaSuccess) return cuda_fail(e, "grouped down launch");
-  if ((e = launch_grouped_combine(p, s)) != cudaSuccess) return cuda_fail(e, "combine launch");
+  if ((e = launch_grouped_actq(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "activation digits launch");
+  if ((e = launch_grouped_down(p, bits, pdl, s)) != cudaSuccess) return cuda_fail(e, "grouped down launch");
+  if ((e = launch_grouped_combine(p, pdl, s)) != cudaSuccess) return cuda_fail(e, "combine launch");
   if (trace && (e = trace_record(g_trace[3], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   taken = true;
   return FMOE_OK;

@@ -135,12 +135,14 @@ struct RouterBatch {
 
 // The batched router's split-K factor: the workspace holds split * T * (E+1) partial logits.
 int grouped_router_split(int H, int E, int T);
-cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s);
-cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s);
-cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, cudaStream_t s);
-cudaError_t launch_grouped_actq(const GroupedParams& p, int bits, cudaStream_t s);
-cudaError_t launch_grouped_down(const GroupedParams& p, int bits, cudaStream_t s);
-cudaError_t launch_grouped_combine(const GroupedParams& p, cudaStream_t s);
+// pdl: chain each launch to its predecessor by dependent launch (every grouped kernel
+// waits for its predecessor at entry, then lets its successor launch).
+cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, bool pdl, cudaStream_t s);
+cudaError_t launch_grouped_select(const GroupedParams& p, bool pdl, cudaStream_t s);
+cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, bool pdl, cudaStream_t s);
+cudaError_t launch_grouped_actq(const GroupedParams& p, int bits, bool pdl, cudaStream_t s);
+cudaError_t launch_grouped_down(const GroupedParams& p, int bits, bool pdl, cudaStream_t s);
+cudaError_t launch_grouped_combine(const GroupedParams& p, bool pdl, cudaStream_t s);
 bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T);
 
 // ---- single-kernel path (k_fused.cu): a sequence of T tokens x L layers, one CTA per SM

@@ -59,38 +59,50 @@ __global__ void __launch_bounds__(kGdnWarps * 32) gdn_step_kernel(const GdnParam
   pdl_wait();
   if (!p.early) load_rows();
 
+  // this warp's small operands, all requested before any arithmetic (one L2 round trip)
+  float a[R], b[R], vi[R];
+  float4 kk[R][NC], qq[R][NC];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const long long row = row0 + r;
+    if (row < p.rows) {
+      const int head = (int)(row / p.dv);
+      a[r] = __ldg(p.alpha + head);
+      b[r] = __ldg(p.beta + head);
+      vi[r] = __ldg(p.v + row);
+      const float4* k4 = reinterpret_cast<const float4*>(p.k + (long long)head * p.dk) + lane;
+      const float4* q4 = reinterpret_cast<const float4*>(p.q + (long long)head * p.dk) + lane;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        kk[r][c] = __ldg(k4 + 32 * c);
+        qq[r][c] = __ldg(q4 + 32 * c);
+      }
+    }
+  }
+
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const long long row = row0 + r;
     if (row >= p.rows) break;  // uniform over the warp
-    const int head = (int)(row / p.dv);
-    const float a = __ldg(p.alpha + head);
-    const float b = __ldg(p.beta + head);
-    const float vi = __ldg(p.v + row);
-    const float4* k4 = reinterpret_cast<const float4*>(p.k + (long long)head * p.dk) + lane;
-    const float4* q4 = reinterpret_cast<const float4*>(p.q + (long long)head * p.dk) + lane;
-    float4 kk[NC];
     float part = 0.0f;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-      kk[c] = __ldg(k4 + 32 * c);
-      s[r][c].x *= a;  // S <- alpha S
-      s[r][c].y *= a;
-      s[r][c].z *= a;
-      s[r][c].w *= a;
-      part = dot4(s[r][c], kk[c], part);
+      s[r][c].x *= a[r];  // S <- alpha S
+      s[r][c].y *= a[r];
+      s[r][c].z *= a[r];
+      s[r][c].w *= a[r];
+      part = dot4(s[r][c], kk[r][c], part);
     }
     const float u = warp_sum(part);  // u_i = S[i] . k
-    const float d = b * (vi - u);
+    const float d = b[r] * (vi[r] - u);
     part = 0.0f;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-      const float4 qq = __ldg(q4 + 32 * c);
-      s[r][c].x = fmaf(d, kk[c].x, s[r][c].x);  // S[i] <- S[i] + beta (v_i - u_i) k
-      s[r][c].y = fmaf(d, kk[c].y, s[r][c].y);
-      s[r][c].z = fmaf(d, kk[c].z, s[r][c].z);
-      s[r][c].w = fmaf(d, kk[c].w, s[r][c].w);
-      part = dot4(s[r][c], qq, part);
+      s[r][c].x = fmaf(d, kk[r][c].x, s[r][c].x);  // S[i] <- S[i] + beta (v_i - u_i) k
+      s[r][c].y = fmaf(d, kk[r][c].y, s[r][c].y);
+      s[r][c].z = fmaf(d, kk[r][c].z, s[r][c].z);
+      s[r][c].w = fmaf(d, kk[r][c].w, s[r][c].w);
+      part = dot4(s[r][c], qq[r][c], part);
     }
     const float oi = warp_sum(part);  // o_i = S[i] . q
     float4* dst = reinterpret_cast<float4*>(p.state + row * p.dk) + lane;
@@ -111,7 +123,7 @@ int rows_per_warp() {
   static int r = -1;
   if (r < 0) {
     const char* e = getenv("FMOE_GDN_RPW");
-    r = (e && (e[0] == '1' || e[0] == '2' || e[0] == '4')) ? e[0] - '0' : 2;
+    r = (e && (e[0] == '1' || e[0] == '2' || e[0] == '4')) ? e[0] - '0' : 1;
   }
   return r;
 }

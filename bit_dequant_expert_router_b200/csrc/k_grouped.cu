@@ -35,6 +35,16 @@
 namespace fmoe {
 namespace {
 
+// The grouped path's kernels are chained by dependent launch: each waits for its
+// predecessor to complete (its writes visible) before anything else, and only then lets
+// its successor launch.  At most two kernels of the chain are resident, and the waiting
+// one never holds resources that a CTA of its predecessor still needs; what is saved is
+// the successor's launch latency.  Every kernel waits, so completion is transitive.
+__device__ __forceinline__ void pdl_chain() {
+  pdl_wait();
+  pdl_trigger();
+}
+
 constexpr int kGT = 256;          // threads per CTA
 constexpr int kMaxTK = 4096;      // T*K pairs
 
@@ -121,6 +131,7 @@ __device__ __forceinline__ void tc_quantize_group(float v0, float v1, uint8_t* g
 // two-stage top-K (ties to the lower index) with renormalised weights and the
 // shared-gate sigma.
 __global__ void __launch_bounds__(kGT) topk_tokens_kernel(const GroupedParams p) {
+  pdl_chain();
   __shared__ int s_idx[32];
   __shared__ float s_w[33];
   __shared__ unsigned long long s_cand[8 * 32];
@@ -188,6 +199,7 @@ __device__ __forceinline__ int block_scan_excl(int v, int* s_warp, int* total) {
 // A unit is written out whole (UnitDesc) so that the expert kernels find it
 // with one load.
 __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) {
+  pdl_chain();
   extern __shared__ __align__(16) int s_mem[];  // [T*K] experts of the pairs, [E] counts, [E] starts
   __shared__ int s_warp[kST / 32];
   const int tid = threadIdx.x, N = p.T * p.K, E = p.E;
@@ -269,6 +281,7 @@ __global__ void __launch_bounds__(kST) sort_pairs_kernel(const GroupedParams p) 
 constexpr int kNormSplit = 4;
 
 __global__ void __launch_bounds__(kGT) norm_digits_kernel(const GroupedParams p, const RouterBatch rb, int bits) {
+  pdl_chain();
   __shared__ float s_red[kGT / 32];
   const int t = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, H = p.H, NG = H / kGroup;
   const float* h = p.h + (size_t)t * H;
@@ -319,6 +332,7 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool vali
 }
 
 __global__ void __launch_bounds__(kGT) router_gemm_kernel(const GroupedParams p, const RouterBatch rb) {
+  pdl_chain();
   extern __shared__ __align__(16) uint8_t sm[];
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15, H = p.H, E = p.E, T = p.T, R = E + 1;
   const int r0 = blockIdx.x * kRtR, t0 = blockIdx.y * kRtT, kc = blockIdx.z, KC = H / p.rt_split;
@@ -759,6 +773,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
 template <int BITS, int NG, int TL>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gateup_kernel(const GroupedParams p, int ns, const __grid_constant__ TcMaps<12> maps) {
+  pdl_chain();
   using R = TcRows<BITS, NG>;
   constexpr int RB = R::RB, LB = R::LB, LBP = R::LBP, CB = R::CB, SB = NG * 2;
   constexpr int ROWS = 8 * TL, TPW = TL < 2 ? TL : 2, KS = kConsumers * TPW / TL;  // TPW tiles per warp, KS K slices
@@ -892,6 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---- activation digits of every sorted pair and every shared-expert token: one warp per group of 64
 template <int BITS>
 __global__ void __launch_bounds__(kGT) grouped_actq_kernel(const GroupedParams p) {
+  pdl_chain();
   const int I = p.I, NGI = I / kGroup;
   const int gw = blockIdx.x * (kGT / 32) + (threadIdx.x >> 5);
   if (gw >= (p.T * p.K + p.T) * NGI) return;  // warp-uniform
@@ -909,6 +925,7 @@ __global__ void __launch_bounds__(kGT) grouped_actq_kernel(const GroupedParams p
 template <int BITS, int NG, int TL>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_down_kernel(const GroupedParams p, int ns, const __grid_constant__ TcMaps<6> maps) {
+  pdl_chain();
   using R = TcRows<BITS, NG>;
   constexpr int RB = R::RB, LB = R::LB, LBP = R::LBP, CB = R::CB, SB = NG * 2;
   constexpr int ROWS = 16 * TL, TPW = TL < 2 ? TL : 2, KS = kConsumers * TPW / TL;
@@ -1038,6 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // the member rows and weights are read once per CTA, and the rows' loads are
 // issued eight at a time before their terms are added in k order.
 __global__ void __launch_bounds__(kGT) grouped_combine_kernel(const GroupedParams p) {
+  pdl_chain();
   __shared__ int s_pos[33];
   __shared__ float s_w[33];
   const int t = blockIdx.y, tid = threadIdx.x, K = p.K, H = p.H;
@@ -1164,19 +1182,19 @@ cudaError_t encode_maps(TcMaps<N>& m, const GroupedParams& p, const int (&subs)[
 }
 
 template <int BITS, int NG>
-cudaError_t gateup_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
+cudaError_t gateup_ng(const GroupedParams& p, const TcConfig& c, bool pdl, cudaStream_t s) {
   TcMaps<12> m;
   static constexpr int subs[6] = {0, 3, 1, 2, 4, 5};  // gate rows, up rows, gate s, gate b, up s, up b
   cudaError_t e = encode_maps(m, p, subs, false, p.I, p.H * BITS / 8, NG, 8 * c.tl);
   if (e != cudaSuccess) return e;
   auto k = c.tl == 2 ? grouped_gateup_kernel<BITS, NG, 2> : grouped_gateup_kernel<BITS, NG, 1>;
   if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
-  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m);
-  return cudaGetLastError();
+  if ((e = set_carveout_max((const void*)k)) != cudaSuccess) return e;
+  return launch_pdl(k, dim3(num_sms()), dim3(kThreads), c.smem, s, pdl, p, c.ns, m);
 }
 
 template <int BITS, int NG>
-cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
+cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, bool pdl, cudaStream_t s) {
   TcMaps<6> m;
   static constexpr int subs[3] = {6, 7, 8};  // rows, s, b
   cudaError_t e = encode_maps(m, p, subs, true, p.H, p.I * BITS / 8, NG, 16 * c.tl);
@@ -1186,34 +1204,34 @@ cudaError_t down_ng(const GroupedParams& p, const TcConfig& c, cudaStream_t s) {
            : c.tl == 2 ? grouped_down_kernel<BITS, NG, 2>
                        : grouped_down_kernel<BITS, NG, 1>;
   if ((e = set_smem((const void*)k, c.smem)) != cudaSuccess) return e;
-  k<<<num_sms(), kThreads, c.smem, s>>>(p, c.ns, m);
-  return cudaGetLastError();
+  if ((e = set_carveout_max((const void*)k)) != cudaSuccess) return e;
+  return launch_pdl(k, dim3(num_sms()), dim3(kThreads), c.smem, s, pdl, p, c.ns, m);
 }
 
 template <int BITS>
-cudaError_t gateup_bits_g(const GroupedParams& p, cudaStream_t s) {
+cudaError_t gateup_bits_g(const GroupedParams& p, bool pdl, cudaStream_t s) {
   const TcConfig c = gu_config(BITS, p.H);
   if (c.tl == 0 || p.I % (8 * c.tl)) return cudaErrorInvalidValue;
   switch (p.H / kGroup) {
-    case 8: return gateup_ng<BITS, 8>(p, c, s);
-    case 16: return gateup_ng<BITS, 16>(p, c, s);
-    case 32: return gateup_ng<BITS, 32>(p, c, s);
-    case 64: return gateup_ng<BITS, 64>(p, c, s);
-    case 128: return gateup_ng<BITS, 128>(p, c, s);
+    case 8: return gateup_ng<BITS, 8>(p, c, pdl, s);
+    case 16: return gateup_ng<BITS, 16>(p, c, pdl, s);
+    case 32: return gateup_ng<BITS, 32>(p, c, pdl, s);
+    case 64: return gateup_ng<BITS, 64>(p, c, pdl, s);
+    case 128: return gateup_ng<BITS, 128>(p, c, pdl, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int BITS>
-cudaError_t down_bits_g(const GroupedParams& p, cudaStream_t s) {
+cudaError_t down_bits_g(const GroupedParams& p, bool pdl, cudaStream_t s) {
   const TcConfig c = dn_config(BITS, p.I);
   if (c.tl == 0 || p.H % (16 * c.tl)) return cudaErrorInvalidValue;
   switch (p.I / kGroup) {
-    case 8: return down_ng<BITS, 8>(p, c, s);
-    case 16: return down_ng<BITS, 16>(p, c, s);
-    case 32: return down_ng<BITS, 32>(p, c, s);
-    case 64: return down_ng<BITS, 64>(p, c, s);
-    case 128: return down_ng<BITS, 128>(p, c, s);
+    case 8: return down_ng<BITS, 8>(p, c, pdl, s);
+    case 16: return down_ng<BITS, 16>(p, c, pdl, s);
+    case 32: return down_ng<BITS, 32>(p, c, pdl, s);
+    case 64: return down_ng<BITS, 64>(p, c, pdl, s);
+    case 128: return down_ng<BITS, 128>(p, c, pdl, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1227,14 +1245,14 @@ bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T) {
   return gu.tl > 0 && I % (8 * gu.tl) == 0 && dn.tl > 0 && H % (16 * dn.tl) == 0;
 }
 
-cudaError_t launch_grouped_select(const GroupedParams& p, cudaStream_t s) {
-  topk_tokens_kernel<<<p.T, kGT, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
+cudaError_t launch_grouped_select(const GroupedParams& p, bool pdl, cudaStream_t s) {
+  cudaError_t e = set_carveout_max((const void*)topk_tokens_kernel);
   if (e != cudaSuccess) return e;
+  if ((e = launch_pdl(topk_tokens_kernel, dim3(p.T), dim3(kGT), 0, s, pdl, p)) != cudaSuccess) return e;
   const size_t smem = ((size_t)p.T * p.K + 2 * (size_t)p.E) * sizeof(int);
   if ((e = set_smem((const void*)sort_pairs_kernel, smem)) != cudaSuccess) return e;
-  sort_pairs_kernel<<<1, kST, smem, s>>>(p);
-  return cudaGetLastError();
+  if ((e = set_carveout_max((const void*)sort_pairs_kernel)) != cudaSuccess) return e;
+  return launch_pdl(sort_pairs_kernel, dim3(1), dim3(kST), smem, s, pdl, p);
 }
 
 int grouped_router_split(int H, int E, int T) {
@@ -1244,38 +1262,40 @@ int grouped_router_split(int H, int E, int T) {
   return n;
 }
 
-cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, cudaStream_t s) {
-  norm_digits_kernel<<<dim3(kNormSplit, p.T), kGT, 0, s>>>(p, rb, bits);
-  cudaError_t e = cudaGetLastError();
+cudaError_t launch_grouped_router(const GroupedParams& p, const RouterBatch& rb, int bits, bool pdl, cudaStream_t s) {
+  cudaError_t e = set_carveout_max((const void*)norm_digits_kernel);
   if (e != cudaSuccess) return e;
+  if ((e = launch_pdl(norm_digits_kernel, dim3(kNormSplit, p.T), dim3(kGT), 0, s, pdl, p, rb, bits)) != cudaSuccess)
+    return e;
   const size_t smem = (size_t)kRtR * (kRtK + 8) * 2 + (size_t)kRtT * (kRtK + 4) * 4;
   void (*k)(const GroupedParams, const RouterBatch) = router_gemm_kernel;
   if ((e = set_smem((const void*)k, smem)) != cudaSuccess) return e;
-  k<<<dim3((p.E + 1 + kRtR - 1) / kRtR, (p.T + kRtT - 1) / kRtT, p.rt_split), kGT, smem, s>>>(p, rb);
-  return cudaGetLastError();
+  if ((e = set_carveout_max((const void*)k)) != cudaSuccess) return e;
+  return launch_pdl(k, dim3((p.E + 1 + kRtR - 1) / kRtR, (p.T + kRtT - 1) / kRtT, p.rt_split), dim3(kGT), smem, s,
+                    pdl, p, rb);
 }
 
-cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, cudaStream_t s) {
-  return bits == 4 ? gateup_bits_g<4>(p, s) : gateup_bits_g<2>(p, s);
+cudaError_t launch_grouped_gateup(const GroupedParams& p, int bits, bool pdl, cudaStream_t s) {
+  return bits == 4 ? gateup_bits_g<4>(p, pdl, s) : gateup_bits_g<2>(p, pdl, s);
 }
 
-cudaError_t launch_grouped_actq(const GroupedParams& p, int bits, cudaStream_t s) {
+cudaError_t launch_grouped_actq(const GroupedParams& p, int bits, bool pdl, cudaStream_t s) {
   const int warps = (p.T * p.K + p.T) * (p.I / kGroup);
   const int grid = (warps + kGT / 32 - 1) / (kGT / 32);
-  if (bits == 4)
-    grouped_actq_kernel<4><<<grid, kGT, 0, s>>>(p);
-  else
-    grouped_actq_kernel<2><<<grid, kGT, 0, s>>>(p);
-  return cudaGetLastError();
+  void (*k)(const GroupedParams) = bits == 4 ? grouped_actq_kernel<4> : grouped_actq_kernel<2>;
+  const cudaError_t e = set_carveout_max((const void*)k);
+  return e != cudaSuccess ? e : launch_pdl(k, dim3(grid), dim3(kGT), 0, s, pdl, p);
 }
 
-cudaError_t launch_grouped_down(const GroupedParams& p, int bits, cudaStream_t s) {
-  return bits == 4 ? down_bits_g<4>(p, s) : down_bits_g<2>(p, s);
+cudaError_t launch_grouped_down(const GroupedParams& p, int bits, bool pdl, cudaStream_t s) {
+  return bits == 4 ? down_bits_g<4>(p, pdl, s) : down_bits_g<2>(p, pdl, s);
 }
 
-cudaError_t launch_grouped_combine(const GroupedParams& p, cudaStream_t s) {
-  grouped_combine_kernel<<<dim3((p.H / 4 + kGT - 1) / kGT, p.T), kGT, 0, s>>>(p);
-  return cudaGetLastError();
+cudaError_t launch_grouped_combine(const GroupedParams& p, bool pdl, cudaStream_t s) {
+  const cudaError_t e = set_carveout_max((const void*)grouped_combine_kernel);
+  return e != cudaSuccess ? e
+                          : launch_pdl(grouped_combine_kernel, dim3((p.H / 4 + kGT - 1) / kGT, p.T), dim3(kGT), 0, s,
+                                       pdl, p);
 }
 
 }  // namespace fmoe

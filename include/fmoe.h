@@ -63,6 +63,8 @@ typedef enum {
 /* A bank of expert records in device memory.
  * bits: 2 or 4.  group_size: 64 (the only supported value).
  * hidden (H), inter (I): model width and expert intermediate width.
+ * reserved: set to 0 (it spells out the padding before `base`, so that the layout is
+ * the same under every compiler).
  * base: record 0 (16-byte aligned); stride: bytes between records (multiple of 16).
  * off[9]: byte offsets inside a record of gate.qw, gate.scale, gate.bias,
  *         up.qw, up.scale, up.bias, down.qw, down.scale, down.bias (multiples of 16). */
