@@ -62,6 +62,13 @@ GDN_WORKLOADS = {
                            "45 layers' states resident, one token through each in turn (batch-1 decode)"),
 }
 GDN_METRIC = "Gated DeltaNet decode state updates/s (one layer, 64 heads x 128x128 fp32) and GB/s, 1xB200"
+# Routed experts in pinned host memory behind an HBM expert cache: (bits, Zipf exponent,
+# cache slots, description); one step = one token through the layer.
+CACHED_WORKLOADS = {
+    "qwen397-4bit-cached": (4, 1.1, 64, "Qwen3.5-397B-A17B-shaped MoE layer, 4-bit group-64 experts, all 512 in "
+                                        "pinned host memory behind a 64-slot HBM expert cache, Zipf(1.1) routing, "
+                                        "batch-1 decode"),
+}
 # Workloads that run a stack of distinct layers per token (fmoe_moe_stack); the
 # metric then counts layer-steps (one token through one layer) per second.
 STACK_LAYERS = {"qwen397-2bit-stack60": 60}
@@ -75,7 +82,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="fmoe", choices=["fmoe", "reference"])
-    ap.add_argument("--workload", default="qwen397-4bit", choices=sorted(WORKLOADS) + sorted(GDN_WORKLOADS))
+    ap.add_argument("--workload", default="qwen397-4bit",
+                    choices=sorted(WORKLOADS) + sorted(GDN_WORKLOADS) + sorted(CACHED_WORKLOADS))
     ap.add_argument("--copies", type=int, default=16, help="resident layer copies rotated per token")
     ap.add_argument("--graph-tokens", type=int, default=1000, help="tokens per captured CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
@@ -399,11 +407,178 @@ def run_gdn(args, world, rank, local):
         dist.destroy_process_group()
 
 
+def run_cached(args, world, rank, local):
+    import gen
+    bits, zipf, C, desc = CACHED_WORKLOADS[args.workload]
+    spec = gen.qwen397_layer(bits, zipf=zipf)
+    if args.impl == "reference":  # the oracle computes the same layer; where the experts live does not matter to it
+        return run_reference(args, spec, desc, world, rank)
+    import torch
+    import torch.distributed as dist
+    import bit_dequant_expert_router_b200 as fmoe
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    fmoe.lib()
+    nbytes, off = gen.record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
+    dl = gen.device_layer(spec, seed=0, layer=0, device=dev)
+    host_bank = torch.empty(dl.bank.numel(), dtype=torch.uint8, pin_memory=True)
+    host_bank.copy_(dl.bank)
+    dl.bank = None  # the routed experts live in host memory only
+    torch.cuda.empty_cache()
+    routed = fmoe.Bank(None, spec.bits, spec.hidden, spec.inter, spec.experts, nbytes, off, spec.group)
+    shared = fmoe.Bank(dl.shared, spec.bits, spec.hidden, spec.inter, 1, nbytes, off, spec.group)
+    lay = fmoe.Layer(routed, shared, dl.w_router, dl.w_shared_gate, dl.gamma, dl.logit_bias, spec.eps, spec.top_k)
+    cache = fmoe.ExpertCache(host_bank, spec.experts, nbytes, nbytes, C, device=dev)
+    # every token of the timed region is a fresh one (the cache sees a realistic stream):
+    # `steps` distinct tokens, captured as steps / G graphs of G tokens each
+    G = min(args.graph_tokens, args.steps, 200)
+    steps = (min(args.steps, 2000) + G - 1) // G * G
+    h = gen.device_tokens(rank * 10_000_000, steps, spec.hidden, device=dev)
+    out = torch.empty_like(h)
+    ws = fmoe.workspace(fmoe.moe_layer_workspace_size(lay, 1), dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step(i, s):
+        fmoe.moe_layer_cached(lay, cache, h[i % steps], out=out[i % steps], ws=ws, stream=s)
+
+    with torch.cuda.stream(stream):  # warm-up: the cache reaches its steady state
+        for i in range(max(args.warmup, 3, 4 * C // spec.top_k)):
+            step(steps - 1 - i, stream)
+    stream.synchronize()
+    fmoe.workspace_check(ws, stream)
+    graphs = []
+    for j in range(steps // G):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(j * G, (j + 1) * G):
+                step(i, stream)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            g.replay()
+    stream.synchronize()
+
+    def timed(gs):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for g in gs:
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+
+    h0, m0, b0 = cache.stats(stream)
+    with ClockSampler(local) as clk:
+        times = [max_over_ranks(timed(graphs), world, dev) for _ in range(max(args.reps, 3))]
+    h1, m1, b1 = cache.stats(stream)
+    fmoe.workspace_check(ws, stream)
+    ms = statistics.median(times)
+    value = steps * world / (ms / 1e3)
+    lookups = (h1 - h0) + (m1 - m0)
+    copied_per_token = (b1 - b0) / (steps * len(times))
+
+    # the copy kernel alone: lookups that all miss (fresh experts each time), against the
+    # copy engine's pinned host -> device rate on the same bytes
+    cache.reset(stream)
+    K = spec.top_k
+    miss_idx = torch.arange(0, spec.experts, dtype=torch.int32, device=dev)
+    nl = spec.experts // K
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        cache.fetch(miss_idx[:K], stream=stream)
+        stream.synchronize()
+        cache.reset(stream)
+        e0.record(stream)
+        for j in range(nl):
+            cache.fetch(miss_idx[j * K:(j + 1) * K], stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    fetch_gbs = nl * K * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    dst = torch.empty(64 * nbytes, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        dst.copy_(host_bank[:64 * nbytes], non_blocking=True)
+        e0.record(stream)
+        for _ in range(3):
+            dst.copy_(host_bank[:64 * nbytes], non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    ce_gbs = 3 * 64 * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del dst
+    cache.reset(stream)
+
+    e2e = None
+    if not args.no_e2e:
+        hh = h.cpu().pin_memory()
+        oh = torch.empty_like(hh).pin_memory()
+        hd = torch.empty(spec.hidden, dtype=torch.float32, device=dev)
+        od = torch.empty_like(hd)
+        del graphs
+        with torch.cuda.stream(stream):
+            for i in range(4 * C // spec.top_k):
+                step(steps - 1 - i, stream)
+        egraphs = []
+        for j in range(steps // G):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(j * G, (j + 1) * G):
+                    hd.copy_(hh[i], non_blocking=True)
+                    fmoe.moe_layer_cached(lay, cache, hd, out=od, ws=ws, stream=stream)
+                    oh[i].copy_(od, non_blocking=True)
+            egraphs.append(g)
+        with torch.cuda.stream(stream):
+            for g in egraphs:
+                g.replay()
+        stream.synchronize()
+        ems = statistics.median([max_over_ranks(timed(egraphs), world, dev) for _ in range(3)])
+        e2e = {"value": steps * world / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": spec.hidden * 4,
+               "d2h_bytes_per_step": spec.hidden * 4}
+        del egraphs
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, n, spent = cpu_oracle_rate(spec, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} tokens of this workload, layer copy 0 ({spent:.1f} s of oracle time)"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": max(args.warmup, 3, 4 * C // spec.top_k), "ms_per_step": ms / steps, "reps": len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_TOKEN,
+            "data": "synthetic",
+            "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
+                       "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": 1, "cache_slots": C,
+                       "l2": "the experts stream from host memory on a miss; a hit reads a slot in HBM",
+                       "parallelism": f"replicas x{world}"},
+            "cache": {"hit_rate": (h1 - h0) / lookups if lookups else None, "lookups": lookups,
+                      "host_bytes_per_token": copied_per_token,
+                      "host_link_gbs": copied_per_token * value / world / 1e9},
+            "roofline": {"bound": "host_link", "achieved": fetch_gbs, "peak": ce_gbs, "unit": "GB/s",
+                         "frac": fetch_gbs / ce_gbs, "traffic": None, "kernel": "cache_copy_kernel",
+                         "peak_kind": "measured here: copy-engine pinned host -> device rate on 64 records",
+                         "algorithmic_bytes_per_launch": spec.top_k * nbytes},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * steps, "clocks": clk.record(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     if args.workload in GDN_WORKLOADS:
         return run_gdn(args, world, rank, local)
+    if args.workload in CACHED_WORKLOADS:
+        return run_cached(args, world, rank, local)
     import gen
     spec = WORKLOADS[args.workload][0]()
     desc = WORKLOADS[args.workload][1]

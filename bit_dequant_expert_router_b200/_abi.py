@@ -1,4 +1,4 @@
-"""ctypes binding of libfmoe.so (include/fmoe.h): argument marshalling only.
+"""ctypes binding of libfmoe.so (include/fmoe.h, fmoe_gdn.h, fmoe_cache.h): argument marshalling only.
 
 Every function takes torch tensors that already live on the GPU, passes their
 device pointers and the current torch stream to the C ABI, and raises
@@ -36,6 +36,12 @@ class FmoeLayer(ctypes.Structure):
                 ("eps", ctypes.c_float), ("top_k", ctypes.c_int32)]
 
 
+class FmoeExpertCache(ctypes.Structure):
+    _fields_ = [("host_base", ctypes.c_void_p), ("host_stride", ctypes.c_int64), ("slots", ctypes.c_void_p),
+                ("slot_stride", ctypes.c_int64), ("record_bytes", ctypes.c_int64), ("num_experts", ctypes.c_int32),
+                ("num_slots", ctypes.c_int32), ("state", ctypes.c_void_p)]
+
+
 _lib = None
 
 # (name, restype, argtypes) of every entry point declared in include/fmoe.h
@@ -53,6 +59,13 @@ SIGNATURES = [
     ("fmoe_moe_layer_routed", _i, [ctypes.POINTER(FmoeLayer), _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("fmoe_wait_flag", _i, [_vp, ctypes.c_uint32, ctypes.c_int64, _vp, _vp]),
     ("fmoe_gdn_step", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, ctypes.c_uint32, _vp]),
+    ("fmoe_expert_cache_state_size", _sz, [_i, _i]),
+    ("fmoe_expert_cache_reset", _i, [ctypes.POINTER(FmoeExpertCache), _vp]),
+    ("fmoe_expert_cache_fetch", _i, [ctypes.POINTER(FmoeExpertCache), _vp, _i, _vp, _vp]),
+    ("fmoe_expert_cache_stats", _i, [ctypes.POINTER(FmoeExpertCache), ctypes.POINTER(ctypes.c_int64),
+                                     ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), _vp]),
+    ("fmoe_moe_layer_cached", _i, [ctypes.POINTER(FmoeLayer), ctypes.POINTER(FmoeExpertCache), _vp, _i, _vp, _vp, _vp,
+                                   _vp, _sz, _vp]),
     ("fmoe_moe_stack", _i, [ctypes.POINTER(FmoeLayer), _i, _vp, _i, _vp, _vp, _sz, _vp]),
     ("fmoe_trace_next_layer", _i, [ctypes.POINTER(ctypes.c_void_p), _i]),
     ("fmoe_workspace_init", _i, [_vp, _sz, _vp]),
@@ -114,9 +127,9 @@ class Bank:
     """A bank of expert records held in one device tensor (uint8)."""
 
     def __init__(self, storage, bits, hidden, inter, num_experts, stride, off, group_size=64):
-        self.storage = storage
-        self.s = FmoeBank(bits, group_size, hidden, inter, num_experts, 0,
-                          _ptr(storage, torch.uint8, "bank storage").value, stride, (ctypes.c_int64 * 9)(*off))
+        self.storage = storage   # None: the records live elsewhere (an expert cache's host store)
+        base = None if storage is None else _ptr(storage, torch.uint8, "bank storage").value
+        self.s = FmoeBank(bits, group_size, hidden, inter, num_experts, 0, base, stride, (ctypes.c_int64 * 9)(*off))
 
 
 class Layer:
@@ -263,6 +276,57 @@ def gdn_step(state, q, k, v, alpha, beta, o=None, early=False, stream=None):
                                _ptr(alpha, f32, "alpha"), _ptr(beta, f32, "beta"), _ptr(o, f32, "o"), n, dk, dv,
                                GDN_STATE_EARLY if early else 0, _stream(stream)))
     return o
+
+
+class ExpertCache:
+    """An HBM cache of `num_slots` expert records in front of `host_records`, a pinned host
+    tensor (uint8) holding `num_experts` records at `stride` bytes (fmoe_cache.h)."""
+
+    def __init__(self, host_records, num_experts, stride, record_bytes, num_slots, device=None, stream=None):
+        if host_records.is_cuda or not host_records.is_pinned():
+            raise ValueError("host_records must be a pinned host tensor")
+        if host_records.dtype != torch.uint8 or not host_records.is_contiguous():
+            raise TypeError("host_records must be a contiguous uint8 tensor")
+        if host_records.numel() < num_experts * stride:
+            raise ValueError("host_records holds fewer than num_experts records")
+        device = device or "cuda"
+        self.host = host_records
+        self.slots = torch.empty(num_slots * stride, dtype=torch.uint8, device=device)
+        self.state = torch.empty(max(1, lib().fmoe_expert_cache_state_size(num_experts, num_slots)),
+                                 dtype=torch.uint8, device=device)
+        self.s = FmoeExpertCache(host_records.data_ptr(), stride, self.slots.data_ptr(), stride, record_bytes,
+                                 num_experts, num_slots, self.state.data_ptr())
+        self.reset(stream)
+
+    def reset(self, stream=None):
+        _check(lib().fmoe_expert_cache_reset(ctypes.byref(self.s), _stream(stream)))
+
+    def fetch(self, idx, slot=None, stream=None):
+        """One lookup of the experts idx (device int32 [K]); returns their slots (device int32 [K])."""
+        slot = torch.empty_like(idx) if slot is None else slot
+        _check(lib().fmoe_expert_cache_fetch(ctypes.byref(self.s), _ptr(idx, torch.int32, "idx"), idx.numel(),
+                                             _ptr(slot, torch.int32, "slot"), _stream(stream)))
+        return slot
+
+    def stats(self, stream=None):
+        """(hits, misses, bytes copied) since the last reset; synchronises the stream."""
+        h, m, b = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().fmoe_expert_cache_stats(ctypes.byref(self.s), ctypes.byref(h), ctypes.byref(m), ctypes.byref(b),
+                                             _stream(stream)))
+        return h.value, m.value, b.value
+
+
+def moe_layer_cached(layer, cache, h, out=None, topk_idx=None, topk_w=None, ws=None, stream=None):
+    """fmoe_moe_layer_cached: the block with the routed experts behind `cache`."""
+    T = h.shape[0] if h.dim() == 2 else 1
+    out = torch.empty_like(h) if out is None else out
+    if ws is None:
+        ws = workspace(moe_layer_workspace_size(layer, 1), h.device, stream)
+    _check(lib().fmoe_moe_layer_cached(ctypes.byref(layer.s), ctypes.byref(cache.s), _ptr(h, torch.float32, "h"), T,
+                                       _ptr(out, torch.float32, "out"), _ptr(topk_idx, torch.int32, "topk_idx"),
+                                       _ptr(topk_w, torch.float32, "topk_w"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                       _stream(stream)))
+    return out
 
 
 def moe_stack(layers, h, out=None, ws=None, stream=None):

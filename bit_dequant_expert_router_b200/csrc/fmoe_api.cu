@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "fmoe.h"
+#include "fmoe_cache.h"
 #include "fmoe_gdn.h"
 #include "fmoe_internal.h"
 
@@ -431,7 +432,8 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
 
 static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
                                   uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word,
-                                  const int32_t* given_idx = nullptr, const float* given_w = nullptr);
+                                  const int32_t* given_idx = nullptr, const float* given_w = nullptr,
+                                  const CacheParams* cache = nullptr);
 
 // One token through the block: router kernel (RMSNorm, logits, digits of x), then
 // the expert kernel (top-K, gate/up + SwiGLU, down + combine + residual).
@@ -493,11 +495,14 @@ static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* o
 
 // given_idx / given_w ([K] each, device): the routing given by the caller instead of the
 // top-K of the logits (the router still runs, for x, its digits and the shared gate).
+// cache: the routed experts sit behind an expert cache; the router's last CTA selects the
+// top-K, one cache lookup maps them to slots, and the expert kernels read the slots with
+// that routing (layer->routed then describes the slots).
 static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
                                   uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word,
-                                  const int32_t* given_idx, const float* given_w) {
+                                  const int32_t* given_idx, const float* given_w, const CacheParams* cache) {
   const fmoe_bank& r = layer->routed;
-  const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
+  const int H = r.hidden, E = cache ? cache->E : r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
   RouterParams rp{};
   rp.h = h;
@@ -526,8 +531,19 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
   const bool pdl = pdl_enabled() && !trace;
   cudaError_t e;
   if (trace && (e = trace_record(g_trace[0], s)) != cudaSuccess) return cuda_fail(e, "trace event");
+  if (cache) {  // the router's last CTA selects; the lookup maps the experts to slots
+    rp.top_k = K;
+    rp.route_idx = reinterpret_cast<int32_t*>(base + L.route_idx);
+    rp.route_w = reinterpret_cast<float*>(base + L.route_w);
+    rp.idx_out = idx_out;
+    rp.w_out = w_out;
+    given_idx = cache_slot_out(*cache);
+    given_w = rp.route_w;
+  }
   e = launch_router(rp, bits, pdl, s);
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  if (cache && (e = launch_cache_lookup(*cache, rp.route_idx, K, cache_slot_out(*cache), rp.err, pdl, s)) != cudaSuccess)
+    return cuda_fail(e, "cache lookup launch");
   if (trace && (e = trace_record(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   ExpertParams p{};
   p.routed = ref(r);
@@ -835,6 +851,139 @@ fmoe_status fmoe_moe_layer_routed(const fmoe_layer* layer, const float* h, int T
   for (int t = 0; t < T; ++t) {
     st = layer_token_3k(layer, h + (size_t)t * H, out + (size_t)t * H, nullptr, nullptr, base, L, cs(stream), nullptr,
                         topk_idx + (size_t)t * K, topk_w + (size_t)t * K);
+    if (st != FMOE_OK) return st;
+  }
+  return FMOE_OK;
+}
+
+// ---- expert cache (fmoe_cache.h)
+
+// True if p is pinned host memory that the device reads at the same address.
+static bool host_mapped(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost && a.devicePointer == p;
+}
+
+static bool device_memory(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+static fmoe_status check_cache(const fmoe_expert_cache* c, CacheParams& cp) {
+  if (!c) return fail(FMOE_ERR_INVALID_ARG, "cache is NULL");
+  if (!c->host_base || !c->slots || !c->state) return fail(FMOE_ERR_INVALID_ARG, "host_base, slots or state is NULL");
+  if (c->num_experts < 1 || c->num_experts > (1 << 24) || c->num_slots < 1 || c->num_slots > (1 << 24))
+    return fail(FMOE_ERR_INVALID_ARG, "num_experts %d, num_slots %d", c->num_experts, c->num_slots);
+  if (c->record_bytes < 16 || (c->record_bytes & 15) || (c->host_stride & 15) || (c->slot_stride & 15) ||
+      !aligned16(c->host_base) || !aligned16(c->slots) || !aligned16(c->state))
+    return fail(FMOE_ERR_ALIGNMENT, "record_bytes, strides, host_base, slots and state must be multiples of 16");
+  if (c->host_stride < c->record_bytes || c->slot_stride < c->record_bytes)
+    return fail(FMOE_ERR_INVALID_ARG, "a stride is smaller than record_bytes");
+  if (!host_mapped(c->host_base))
+    return fail(FMOE_ERR_INVALID_ARG, "host_base is not pinned host memory mapped at the same device address");
+  if (!device_memory(c->slots) || !device_memory(c->state))
+    return fail(FMOE_ERR_INVALID_ARG, "slots and state must be device memory");
+  cp.host = static_cast<const uint8_t*>(c->host_base);
+  cp.host_stride = c->host_stride;
+  cp.slots = static_cast<uint8_t*>(c->slots);
+  cp.slot_stride = c->slot_stride;
+  cp.rec = c->record_bytes;
+  cp.E = c->num_experts;
+  cp.C = c->num_slots;
+  cp.state = static_cast<uint8_t*>(c->state);
+  return FMOE_OK;
+}
+
+size_t fmoe_expert_cache_state_size(int num_experts, int num_slots) {
+  if (num_experts < 1 || num_slots < 1) return 0;
+  return cache_state_bytes(num_experts, num_slots);
+}
+
+fmoe_status fmoe_expert_cache_reset(const fmoe_expert_cache* cache, fmoe_stream_t stream) {
+  CacheParams cp{};
+  fmoe_status st = check_cache(cache, cp);
+  if (st != FMOE_OK) return st;
+  cudaError_t e = launch_cache_reset(cp, cs(stream));
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "cache reset launch");
+}
+
+fmoe_status fmoe_expert_cache_fetch(const fmoe_expert_cache* cache, const int32_t* idx, int K, int32_t* slot,
+                                    fmoe_stream_t stream) {
+  CacheParams cp{};
+  fmoe_status st = check_cache(cache, cp);
+  if (st != FMOE_OK) return st;
+  if (!idx) return fail(FMOE_ERR_INVALID_ARG, "idx is NULL");
+  if (K < 1 || K > kCacheMaxK || K > cp.C) return fail(FMOE_ERR_INVALID_ARG, "K %d (1..min(num_slots, 32))", K);
+  if (((uintptr_t)idx & 3u) || ((uintptr_t)slot & 3u)) return fail(FMOE_ERR_ALIGNMENT, "idx and slot must be 4-byte aligned");
+  CacheHeader* hd = reinterpret_cast<CacheHeader*>(cp.state);
+  cudaError_t e = launch_cache_lookup(cp, idx, K, slot, &hd->err, pdl_enabled(), cs(stream));
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e, "cache lookup launch");
+}
+
+fmoe_status fmoe_expert_cache_stats(const fmoe_expert_cache* cache, int64_t* hits, int64_t* misses, int64_t* bytes,
+                                    fmoe_stream_t stream) {
+  CacheParams cp{};
+  fmoe_status st = check_cache(cache, cp);
+  if (st != FMOE_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(cs(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  CacheHeader hd{};
+  if ((e = cudaMemcpy(&hd, cp.state, sizeof(hd), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpy");
+  if (hits) *hits = (int64_t)hd.hits;
+  if (misses) *misses = (int64_t)hd.misses;
+  if (bytes) *bytes = (int64_t)hd.bytes;
+  if (hd.err != 0) {
+    const int zero = 0;
+    if ((e = cudaMemcpy(&reinterpret_cast<CacheHeader*>(cp.state)->err, &zero, sizeof(int), cudaMemcpyHostToDevice)) !=
+        cudaSuccess)
+      return cuda_fail(e, "cudaMemcpy");
+    return fail(FMOE_ERR_INVALID_ARG, "a lookup met an expert index outside the bank");
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_moe_layer_cached(const fmoe_layer* layer, const fmoe_expert_cache* cache, const float* h, int T,
+                                  float* out, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                                  fmoe_stream_t stream) {
+  if (!layer) return fail(FMOE_ERR_INVALID_ARG, "layer is NULL");
+  CacheParams cp{};
+  fmoe_status st = check_cache(cache, cp);
+  if (st != FMOE_OK) return st;
+  if (layer->routed.num_experts != cp.E)
+    return fail(FMOE_ERR_INVALID_ARG, "layer E %d differs from the cache's %d", layer->routed.num_experts, cp.E);
+  // the routed bank as the expert kernels see it: the cache's slots
+  fmoe_layer lc = *layer;
+  lc.routed.base = cp.slots;
+  lc.routed.stride = cp.slot_stride;
+  if ((st = check_layer(&lc)) != FMOE_OK) return st;
+  const int H = lc.routed.hidden, I = lc.routed.inter, K = lc.top_k, b = lc.routed.bits;
+  if (K > cp.C) return fail(FMOE_ERR_INVALID_ARG, "top_k %d > num_slots %d", K, cp.C);
+  const int64_t qg = (int64_t)I * H * b / 8, sg = (int64_t)I * (H / 64) * 2, sd = (int64_t)H * (I / 64) * 2;
+  const int64_t len[9] = {qg, sg, sg, qg, sg, sg, qg, sd, sd};
+  for (int i = 0; i < 9; ++i)
+    if (lc.routed.off[i] + len[i] > cp.rec)
+      return fail(FMOE_ERR_INVALID_ARG, "record_bytes %lld does not cover sub-array %d", (long long)cp.rec, i);
+  lc.routed.num_experts = cp.C;
+  if (T < 0) return fail(FMOE_ERR_INVALID_ARG, "T %d", T);
+  if (T == 0) return FMOE_OK;
+  if (!h || !out) return fail(FMOE_ERR_INVALID_ARG, "h or out is NULL");
+  if (!aligned16(h) || !aligned16(out)) return fail(FMOE_ERR_ALIGNMENT, "h and out must be 16-byte aligned");
+  const WsLayout L = layout(H, cp.E, K, I, 1);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != FMOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  for (int t = 0; t < T; ++t) {
+    st = layer_token_3k(&lc, h + (size_t)t * H, out + (size_t)t * H, topk_idx ? topk_idx + (size_t)t * K : nullptr,
+                        topk_w ? topk_w + (size_t)t * K : nullptr, base, L, cs(stream), nullptr, nullptr, nullptr,
+                        &cp);
     if (st != FMOE_OK) return st;
   }
   return FMOE_OK;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace fmoe {
@@ -227,21 +228,23 @@ __device__ __forceinline__ void cp_async_warp(uint32_t dst, const uint8_t* src, 
 // X_c = d0 * 2^16 + d1 * 2^8 + d2 with signed byte digits (|d0| <= 64).
 // The digits are stored as 32-bit packs lined up with the way a code word is
 // split into bytes:
+//   8-bit: word w is one pack itself (codes 0,1,2,3)
 //   4-bit: word w -> lo = w & 0x0F0F0F0F (codes 0,2,4,6), hi = (w >> 4) & ... (1,3,5,7)
 //   2-bit: word w -> pack m = (w >> 2m) & 0x03030303 (codes m, m+4, m+8, m+12)
-// One group is 48 words: chunk by chunk (a chunk is 16 bytes of codes: two per
-// group at 4-bit, one at 2-bit), and within a chunk [limb 0..2][word 0..3][pack].
-// Across a vector of NG groups the 16-byte pieces are interleaved, piece i of
-// group g at uint4 index i*NG + g, so that lanes reading consecutive groups hit
-// distinct shared-memory banks.  Per chunk there is a float2 {cscale, sum of x
-// over the chunk}, chunk-major.
+// One group is 48 words: chunk by chunk (a chunk is 16 bytes of codes: four per
+// group at 8-bit, two at 4-bit, one at 2-bit), and within a chunk [limb 0..2][word
+// 0..3][pack].  Across a vector of NG groups the 16-byte pieces are interleaved, piece
+// i of group g at uint4 index i*NG + g, so that lanes reading consecutive groups hit
+// distinct shared-memory banks.  Per 32 elements (4- and 8-bit; per group at 2-bit)
+// there is a float2 {cscale, sum of x over the 32}, in element order.
 
 template <int BITS>
 struct Fmt {
-  static constexpr int kCodesPerWord = 32 / BITS;          // 8 or 16
-  static constexpr int kCodesPerChunk = 4 * kCodesPerWord;  // 32 or 64
-  static constexpr int kPacksPerWord = 8 / BITS;           // 2 or 4
-  static constexpr int kLimbWords = 3 * 4 * kPacksPerWord; // 24 or 48 uint32 per chunk
+  static constexpr int kCodesPerWord = 32 / BITS;          // 4, 8 or 16
+  static constexpr int kCodesPerChunk = 4 * kCodesPerWord;  // 16, 32 or 64
+  static constexpr int kPacksPerWord = 8 / BITS;           // 1, 2 or 4
+  static constexpr int kLimbWords = 3 * 4 * kPacksPerWord; // 12, 24 or 48 uint32 per chunk
+  static constexpr int kCsPerGroup = BITS == 2 ? 1 : 2;    // {cscale, sum x} pairs per group of 64
 };
 
 constexpr int kGroupWords = 48;  // digit words of one group of 64
@@ -286,7 +289,7 @@ __device__ __forceinline__ void xq_quantize_group(float v0, float v1, int g, int
     }
   }
   float s = v0 + v1;
-  if (BITS == 4) {  // two chunks of 32 per group: half-warp sums
+  if (BITS != 2) {  // two halves of 32 per group: half-warp sums
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if ((lane & 15) == 0) cs[2 * g + (lane >> 4)] = make_float2(csc, s);
@@ -341,12 +344,12 @@ __device__ __forceinline__ void xq_quantize_block16(const float (&v)[16], int g,
         uint32_t acc = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int e = BITS == 4 ? 8 * (wd >> 1) + (wd & 1) + 2 * k : 4 * k + wd;
+          const int e = BITS == 8 ? 4 * wd + k : BITS == 4 ? 8 * (wd >> 1) + (wd & 1) + 2 * k : 4 * k + wd;
           acc |= d[L][e] << (8 * k);
         }
         w[wd] = acc;
       }
-      const int piece = BITS == 4 ? 6 * (part >> 1) + 2 * L + (part & 1) : 4 * L + part;
+      const int piece = BITS == 8 ? 3 * part + L : BITS == 4 ? 6 * (part >> 1) + 2 * L + (part & 1) : 4 * L + part;
       dst[piece * NG + g] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
@@ -354,7 +357,7 @@ __device__ __forceinline__ void xq_quantize_block16(const float (&v)[16], int g,
 #pragma unroll
   for (int e = 0; e < 16; ++e) sx += v[e];
   sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-  if (BITS == 4) {
+  if (BITS != 2) {
     if (active && (part & 1) == 0) cs[2 * g + (part >> 1)] = make_float2(csc, sx);
   } else {
     sx += __shfl_xor_sync(0xffffffffu, sx, 2);
@@ -389,6 +392,36 @@ __device__ __forceinline__ float group_dot(const uint4 q0, const uint4 q1, const
   }
   const int A = a0 * 256 + a1;  // |A| < 2^24: exact in fp32
   return fmaf((float)A, 256.0f, (float)a2);
+}
+
+// dp4a with unsigned bytes in a (codes up to 255) and signed bytes in b (digits).
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// group_dot for 8-bit codes: four chunks q[0..3] (64 bytes, one code per byte).  The
+// limb sums reach 2^21, so they are combined in 64-bit integers and rounded once.
+__device__ __forceinline__ float group_dot8(const uint4 (&q)[4], const uint32_t (&L)[48]) {
+  int a0 = 0, a1 = 0, a2 = 0;
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    const uint32_t w4[4] = {q[ch].x, q[ch].y, q[ch].z, q[ch].w};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      a0 = dp4a_us(w4[wi], L[ch * 12 + wi], a0);
+      a1 = dp4a_us(w4[wi], L[ch * 12 + 4 + wi], a1);
+      a2 = dp4a_us(w4[wi], L[ch * 12 + 8 + wi], a2);
+    }
+  }
+  const long long A = (long long)a0 * 65536 + (long long)a1 * 256 + a2;
+  return (float)A;
+}
+
+__device__ __forceinline__ void load_group_codes8(const uint8_t* row, int g, uint4 (&q)[4]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) q[c] = *reinterpret_cast<const uint4*>(row + g * 64 + 16 * c);
 }
 
 // Loads group g's 48 digit words from a vector of NG groups (interleaved pieces).
@@ -544,7 +577,7 @@ __device__ __forceinline__ void load_group_codes(const uint8_t* row, int g, uint
 // Chunk scalars of group g: {power-of-two scale of the digits, sum of x over the group}.
 template <int BITS>
 __device__ __forceinline__ float2 group_scalars(const float2* cs, int g) {
-  if (BITS == 4) {
+  if (BITS != 2) {
     const float2 a = cs[2 * g], b = cs[2 * g + 1];
     return make_float2(a.x, a.y + b.y);
   }
@@ -553,7 +586,7 @@ __device__ __forceinline__ float2 group_scalars(const float2* cs, int g) {
 
 template <int BITS>
 __device__ __forceinline__ float2 group_scalars_global(const float2* cs, int g) {
-  if (BITS == 4) {
+  if (BITS != 2) {
     const float2 a = __ldcg(cs + 2 * g), b = __ldcg(cs + 2 * g + 1);
     return make_float2(a.x, a.y + b.y);
   }
@@ -659,5 +692,33 @@ struct BankRef {
   long long off[9];
   int num_experts;
 };
+
+// Tensor copies global -> shared of one box (coordinates: the innermost is 0), completing
+// on the mbarrier `bar`, with an L2 cache policy.
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, int c1, int c2, uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap* m, int c1, int c2, int c3, uint32_t bar,
+                                       uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_5d(uint32_t dst, const CUtensorMap* m, int c1, int c2, int c3, int c4, uint32_t bar,
+                                       uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar), "l"(pol)
+      : "memory");
+}
 
 }  // namespace fmoe

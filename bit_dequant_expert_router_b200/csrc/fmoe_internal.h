@@ -277,7 +277,52 @@ struct GdnParams {
   int dk, dv;
   int early;                  // 1: read the state before the dependency wait
 };
+// Tensor-map encoding (cuTensorMapEncodeTiled through the runtime's driver entry point).
+// encode_map: one map over 8-byte elements, dims[0] elements per row, then the outer dims
+// with their byte strides (rank - 1 of them), and the box; false if it cannot be encoded.
+bool encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                const cuuint32_t* box);
+
 bool gdn_shape_supported(int dk);
+
+// Expert cache (k_cache.cu): host-resident records, HBM slots, tables in `state`.
+constexpr int kCacheMaxK = 32;
+struct CacheHeader {          // first 64 bytes of the state
+  unsigned int clock;         // lookups so far (a slot's last use is the lookup that used it)
+  int err;                    // kDevBadIndex after an index outside the bank (fetch entry point)
+  int n_copy;                 // records the current lookup copies
+  int pad0;
+  unsigned long long hits, misses, bytes;
+  unsigned long long pad1[3];
+};
+struct CacheParams {
+  const uint8_t* host;        // E records at host_stride (pinned host memory, mapped)
+  long long host_stride;
+  uint8_t* slots;             // C records at slot_stride (device)
+  long long slot_stride;
+  long long rec;              // bytes per copied record (multiple of 16)
+  int E, C;
+  uint8_t* state;             // header, copy list [2][kCacheMaxK], slots of the last lookup [kCacheMaxK],
+                              // slot_of [E], expert_of [C], last_use [C]
+};
+__host__ __device__ inline size_t cache_up16(size_t v) { return (v + 15) / 16 * 16; }
+__host__ __device__ inline int* cache_copy_expert(const CacheParams& c) {
+  return reinterpret_cast<int*>(c.state + sizeof(CacheHeader));
+}
+__host__ __device__ inline int* cache_copy_slot(const CacheParams& c) { return cache_copy_expert(c) + kCacheMaxK; }
+__host__ __device__ inline int* cache_slot_out(const CacheParams& c) { return cache_copy_slot(c) + kCacheMaxK; }
+__host__ __device__ inline int* cache_slot_of(const CacheParams& c) { return cache_slot_out(c) + kCacheMaxK; }
+__host__ __device__ inline int* cache_expert_of(const CacheParams& c) {
+  return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cache_slot_of(c)) + cache_up16((size_t)c.E * 4));
+}
+__host__ __device__ inline unsigned int* cache_last_use(const CacheParams& c) {
+  return reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(cache_expert_of(c)) + cache_up16((size_t)c.C * 4));
+}
+size_t cache_state_bytes(int E, int C);
+cudaError_t launch_cache_reset(const CacheParams& c, cudaStream_t s);
+// One lookup: the plan kernel (tables, copy list, slot_out [K]) then the copy kernel.
+cudaError_t launch_cache_lookup(const CacheParams& c, const int32_t* idx, int K, int32_t* slot_out, int* err, bool pdl,
+                                cudaStream_t s);
 cudaError_t launch_gdn_step(const GdnParams& p, bool pdl, cudaStream_t s);
 bool pdl_enabled();
 cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err,

@@ -54,14 +54,23 @@ struct GuCfg {
   static_assert(kRowPairs * kScaleBytes % 16 == 0 && kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
 };
 
+// The four scale arrays of a chunk (gate scales, gate biases, up scales, up biases) as
+// one tensor copy: a map over (row bytes / 8, {scale, bias}, {gate, up}, rows, experts)
+// lands a box as rows of [gate s | gate b | up s | up b].  sb[0]: routed bank, sb[1]: shared.
+struct GuMaps {
+  CUtensorMap sb[2];
+};
+
 // Persistent: CTA b owns units [b*U/G, (b+1)*U/G) (a unit = kRowPairs rows of
 // gate and up of one expert slot), cut into chunks of up to C::kChunkUnits units
-// of one slot, each staged with six bulk copies into a ring of nbuf chunk
-// buffers; warp w computes units w, w+8, .. of the chunk.  A lane always works
-// on the same groups of 64 columns, so it keeps their digits of x in registers
-// for the whole kernel.
+// of one slot, each staged into a ring of nbuf chunk buffers with three copies (gate
+// codes, up codes, and the four scale arrays as one tensor copy of a whole box of
+// C::kChunkRows rows) or, where the record layout has no such map, six bulk copies;
+// warp w computes units w, w+8, .. of the chunk.  A lane always works on the same
+// groups of 64 columns, so it keeps their digits of x in registers for the whole kernel.
 template <int BITS, int NG>
-__global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertParams p, int nbuf) {
+__global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertParams p, int nbuf, int use_maps,
+                                                                  const __grid_constant__ GuMaps maps) {
   using G = Geo<NG>;
   using C = GuCfg<BITS, NG>;
   constexpr int RP = C::kRowPairs, PASSES = C::kPasses;
@@ -104,14 +113,23 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
     const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_bar[c % nbuf]);
     const uint32_t cb = rows * RB, sb = rows * SB;
-    mbar_expect_tx(bar, 2 * cb + 4 * sb);
-    bulk_g2s(dst, rec + off[0] + (long long)r0 * RB, cb, bar, pol);
-    bulk_g2s(dst + CR * RB, rec + off[3] + (long long)r0 * RB, cb, bar, pol);
-    bulk_g2s(dst + 2 * CR * RB, rec + off[1] + (long long)r0 * SB, sb, bar, pol);
-    bulk_g2s(dst + 2 * CR * RB + CR * SB, rec + off[2] + (long long)r0 * SB, sb, bar, pol);
-    bulk_g2s(dst + 2 * CR * RB + 2 * CR * SB, rec + off[4] + (long long)r0 * SB, sb, bar, pol);
-    bulk_g2s(dst + 2 * CR * RB + 3 * CR * SB, rec + off[5] + (long long)r0 * SB, sb, bar, pol);
+    if (use_maps) {  // the scale box always moves C::kChunkRows rows (past the last row: zeros)
+      mbar_expect_tx(bar, 2 * cb + 4 * CR * SB);
+      bulk_g2s(dst, rec + off[0] + (long long)r0 * RB, cb, bar, pol);
+      bulk_g2s(dst + CR * RB, rec + off[3] + (long long)r0 * RB, cb, bar, pol);
+      tma_5d(dst + 2 * CR * RB, &maps.sb[routed ? 0 : 1], 0, 0, r0, routed ? s_idx[sl] : 0, bar, pol);
+    } else {
+      mbar_expect_tx(bar, 2 * cb + 4 * sb);
+      bulk_g2s(dst, rec + off[0] + (long long)r0 * RB, cb, bar, pol);
+      bulk_g2s(dst + CR * RB, rec + off[3] + (long long)r0 * RB, cb, bar, pol);
+      bulk_g2s(dst + 2 * CR * RB, rec + off[1] + (long long)r0 * SB, sb, bar, pol);
+      bulk_g2s(dst + 2 * CR * RB + CR * SB, rec + off[2] + (long long)r0 * SB, sb, bar, pol);
+      bulk_g2s(dst + 2 * CR * RB + 2 * CR * SB, rec + off[4] + (long long)r0 * SB, sb, bar, pol);
+      bulk_g2s(dst + 2 * CR * RB + 3 * CR * SB, rec + off[5] + (long long)r0 * SB, sb, bar, pol);
+    }
   };
+  // where a row's four scale arrays sit in a chunk buffer: row r, array a at (r * srow + a * sarr) bf16
+  const int srow = use_maps ? 2 * SB : SB / 2, sarr = use_maps ? SB / 2 : CR * SB / 2;
 
   // Shared-expert chunks need nothing from the router: request them first.
   if (tid == 0) {
@@ -220,11 +238,11 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
           uint4 q0, q1, v0, v1;
           load_group_codes<BITS>(buf + r * RB, g, q0, q1);
           load_group_codes<BITS>(buf + CR * RB + r * RB, g, v0, v1);
-          const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * CR * RB + r * SB);
-          const float gs = bf16_to_f32(sc[g]);
-          const float gb = bf16_to_f32(sc[CR * SB / 2 + g]);
-          const float us = bf16_to_f32(sc[CR * SB + g]);
-          const float ub = bf16_to_f32(sc[3 * CR * SB / 2 + g]);
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * CR * RB) + r * srow + g;
+          const float gs = bf16_to_f32(sc[0]);
+          const float gb = bf16_to_f32(sc[sarr]);
+          const float us = bf16_to_f32(sc[2 * sarr]);
+          const float ub = bf16_to_f32(sc[3 * sarr]);
           const float Sg = group_dot<BITS>(q0, q1, L[j]);
           const float Su = group_dot<BITS>(v0, v1, L[j]);
           accg[i] = fmaf(gs, cs[j].x * Sg, fmaf(gb, cs[j].y, accg[i]));
@@ -500,6 +518,30 @@ size_t round128(size_t v) { return (v + 127) / 128 * 128; }
 
 constexpr size_t kSmemBudget = 220 * 1024;
 
+// The gate/up scale maps of the routed and the shared bank, if the record layout allows
+// them: scale rows of a multiple of 16 bytes, and one distance from each scale array to
+// its bias array and from gate's arrays to up's.  The bank records are only read.
+bool encode_gu_scale_maps(GuMaps& m, const ExpertParams& p, int SB, int box_rows) {
+  if (SB % 16 != 0 || box_rows > 256 || SB / 8 > 256 || p.I > (1 << 24)) return false;
+  for (int bk = 0; bk < 2; ++bk) {
+    const BankRef& r = bk == 0 ? p.routed : p.shared;
+    if (bk == 1 && !p.has_shared) {
+      m.sb[1] = m.sb[0];
+      continue;
+    }
+    const long long* o = r.off;
+    const long long sb = o[2] - o[1], gu = o[4] - o[1];
+    if (sb <= 0 || gu <= 0 || o[5] - o[4] != sb || (sb & 15) || (gu & 15)) return false;
+    const long long ne = bk == 0 ? r.num_experts : 1;
+    if (ne < 1 || (bk == 0 && (r.stride <= 0 || (r.stride & 15)))) return false;
+    const cuuint64_t dims[5] = {(cuuint64_t)(SB / 8), 2, 2, (cuuint64_t)p.I, (cuuint64_t)ne};
+    const cuuint64_t st[4] = {(cuuint64_t)sb, (cuuint64_t)gu, (cuuint64_t)SB, (cuuint64_t)(bk == 0 ? r.stride : 16)};
+    const cuuint32_t box[5] = {(cuuint32_t)(SB / 8), 2, 2, (cuuint32_t)box_rows, 1};
+    if (!encode_map(&m.sb[bk], r.base + o[1], 5, dims, st, box)) return false;
+  }
+  return true;
+}
+
 template <int BITS, int NG>
 cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
   using C = GuCfg<BITS, NG>;
@@ -516,10 +558,12 @@ cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
   nbuf = nbuf > 8 ? 8 : nbuf;
   if (nbuf < 1) return cudaErrorInvalidValue;
   const size_t smem = C::kHead + (size_t)nbuf * C::kChunkBytes;
-  void (*k)(const ExpertParams, int) = gateup_kernel<BITS, NG>;
+  void (*k)(const ExpertParams, int, int, const GuMaps) = gateup_kernel<BITS, NG>;
   cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k, dim3(grid), dim3(kGuWarps * 32), smem, s, pdl, p, nbuf);
+  GuMaps maps;
+  const int use_maps = encode_gu_scale_maps(maps, p, C::kScaleBytes, C::kChunkRows) ? 1 : 0;
+  return launch_pdl(k, dim3(grid), dim3(kGuWarps * 32), smem, s, pdl, p, nbuf, use_maps, maps);
 }
 
 // Down-kernel staging: (chunk units, buffers, shared bytes) for NE slots, or false.

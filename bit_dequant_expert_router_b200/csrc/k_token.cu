@@ -218,32 +218,6 @@ struct TokMaps {
   CUtensorMap dn_codes[2];
 };
 
-__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, int c1, int c2, uint32_t bar, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
-      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(bar), "l"(pol)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap* m, int c1, int c2, int c3, uint32_t bar,
-                                       uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
-      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(pol)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_5d(uint32_t dst, const CUtensorMap* m, int c1, int c2, int c3, int c4, uint32_t bar,
-                                       uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
-      "l"(m), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar), "l"(pol)
-      : "memory");
-}
-
 // Block-wide top-K of logits [E] by the 256 consumer threads (E <= 1024), in two
 // stages: each warp's K largest keys of its logits e = tid + 256 i into cand,
 // then warp 0 the K largest candidates, the renormalised weights
@@ -855,32 +829,6 @@ __global__ void __launch_bounds__(kXThreads, 1) tok_expert_kernel(const TokExper
 
 size_t round128(size_t v) { return (v + 127) / 128 * 128; }
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return enc;
-}
-
-// One map over 8-byte elements: dims[0] elements per row, then the outer dims with
-// their byte strides; box: dims[0] x box_rows x the outer dims' full extents (last: 1).
-bool encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-                const cuuint32_t* box) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, rank, const_cast<void*>(base), dims, strides, box, es,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // The two-kernel path stages every array by tensor copies of whole boxes, which needs:
 // rows of at most 2048 bytes of codes, at least 16 bytes of scales, and a record
 // layout in which up's arrays sit at one distance from gate's, and each bias array at
@@ -956,6 +904,33 @@ cudaError_t expert_bits(const TokExpertParams& p, const TokMaps& m, int dppl, si
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return enc;
+}
+
+// One map over 8-byte elements: dims[0] elements per row, then the outer dims with
+// their byte strides; box: dims[0] x box_rows x the outer dims' full extents (last: 1).
+bool encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                const cuuint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, rank, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 
 // Shared memory of the expert kernel: the digits region (x, later the activations) and
 // one ring for the staged chunks.  A down range's NE chunks are in the ring together,

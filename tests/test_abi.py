@@ -149,3 +149,24 @@ def test_gdn_step_rejects_bad_arguments_before_any_launch():
     assert L.fmoe_gdn_step(S, q + 4, *good[2:], 64, 128, 128, 0, None) == 2
     assert L.fmoe_gdn_step(*good[:3], v + 2, *good[4:], 64, 128, 128, 0, None) == 2
     assert L.fmoe_gdn_step(*good[:6], o + 1, 64, 128, 128, 0, None) == 2
+
+
+def test_expert_cache_rejects_bad_arguments_before_any_launch():
+    L = fmoe.lib()
+    assert L.fmoe_expert_cache_state_size(0, 4) == 0
+    # header 64 B, three lists of 32 ints, slot_of [512], expert_of [64], last_use [64]
+    assert L.fmoe_expert_cache_state_size(512, 64) == 64 + 384 + 2048 + 256 + 256
+    C = fmoe.FmoeExpertCache
+    ok = dict(host_base=0x7000000000, host_stride=4096, slots=0x60000000, slot_stride=4096, record_bytes=4096,
+              num_experts=16, num_slots=4, state=0x61000000)
+    assert L.fmoe_expert_cache_reset(None, None) == 1
+    assert L.fmoe_expert_cache_reset(ctypes.byref(C(**dict(ok, state=None))), None) == 1
+    assert L.fmoe_expert_cache_reset(ctypes.byref(C(**dict(ok, num_slots=0))), None) == 1
+    assert L.fmoe_expert_cache_reset(ctypes.byref(C(**dict(ok, record_bytes=4008))), None) == 2
+    assert L.fmoe_expert_cache_reset(ctypes.byref(C(**dict(ok, slots=0x60000008))), None) == 2
+    assert L.fmoe_expert_cache_reset(ctypes.byref(C(**dict(ok, host_stride=2048))), None) == 1
+    # host_base that is not pinned, mapped host memory (here: no device at all)
+    assert L.fmoe_expert_cache_reset(ctypes.byref(C(**ok)), None) == 1
+    assert L.fmoe_expert_cache_fetch(ctypes.byref(C(**ok)), 0x62000000, 4, None, None) == 1
+    assert L.fmoe_moe_layer_cached(None, ctypes.byref(C(**ok)), 0x60000000, 1, 0x60000000, None, None, 0x50000000,
+                                   1 << 20, None) == 1
