@@ -33,7 +33,7 @@ EXPERT_TRAFFIC = {"qwen397-4bit": 30657536}
 # grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
 # (+ the shared expert): 1,051,820,288 B over 207.5 experts
 GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5069013}
-DTYPE_TOKEN = "i32 dp4a (u4/u2 codes x 24-bit fixed-point x) + f32"
+DTYPE_TOKEN = "i32 dp4a (u{bits} codes x 24-bit fixed-point x) + f32"
 DTYPE_BATCH = "i32 mma.sync (u4/u2 codes as u8 x 24-bit fixed-point x as three s8 limbs) + f32"
 BATCH_KERNELS = 8  # norm+digits, router GEMM, top-K, sort, gate/up, activation digits, down, combine
 # Per-token path: router, gate/up + SwiGLU, down + combine (three dependent launches);
@@ -47,6 +47,11 @@ WORKLOADS = {
                      "Qwen3.5-397B-A17B-shaped MoE layer, 4-bit group-64 experts, batch-1 decode"),
     "qwen397-2bit-zipf": (lambda: __import__("gen").qwen397_layer(2, zipf=1.1),
                           "Qwen3.5-397B-A17B-shaped MoE layer, 2-bit group-64 experts, Zipf(1.1) routing, batch-1 decode"),
+    "qwen397-8bit": (lambda: __import__("gen").qwen397_layer(8),
+                     "Qwen3.5-397B-A17B-shaped MoE layer, 8-bit group-64 experts, batch-1 decode"),
+    "qwen397-4bit-g128": (lambda: __import__("gen").LayerSpec(**{**__import__("gen").qwen397_layer(4).__dict__,
+                                                                 "group": 128}),
+                          "Qwen3.5-397B-A17B-shaped MoE layer, 4-bit group-128 experts, batch-1 decode"),
     "tiny-4bit": (lambda: __import__("gen").tiny_layer(4), "tiny MoE layer (H256, E8, I128, top-2), 4-bit"),
     "qwen397-4bit-batch64": (lambda: __import__("gen").qwen397_layer(4),
                              "Qwen3.5-397B-A17B-shaped MoE layer, 4-bit group-64 experts, batched decode of 64 "
@@ -551,7 +556,7 @@ def run_cached(args, world, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": max(args.warmup, 3, 4 * C // spec.top_k), "ms_per_step": ms / steps, "reps": len(times),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_TOKEN,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_TOKEN.format(bits=spec.bits),
             "data": "synthetic",
             "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
                        "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": 1, "cache_slots": C,
@@ -759,7 +764,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "reps": nreps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": DTYPE_BATCH if nbatch else DTYPE_TOKEN, "data": "synthetic",
+            "vs_baseline": None, "dtype": DTYPE_BATCH if nbatch else DTYPE_TOKEN.format(bits=spec.bits), "data": "synthetic",
             "config": {"workload": desc, "hidden": spec.hidden, "experts": spec.experts, "inter": spec.inter,
                        "top_k": spec.top_k, "bits": spec.bits, "group": spec.group, "batch": nb,
                        "active_experts_per_step": n_active,

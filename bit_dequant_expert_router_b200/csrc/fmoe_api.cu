@@ -116,8 +116,12 @@ fmoe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 fmoe_status check_bank(const fmoe_bank* b, const char* name) {
   if (!b) return fail(FMOE_ERR_INVALID_ARG, "%s bank is NULL", name);
   if (!b->base) return fail(FMOE_ERR_INVALID_ARG, "%s bank base is NULL", name);
-  if (b->bits != 2 && b->bits != 4) return fail(FMOE_ERR_UNSUPPORTED, "%s bank: bits %d (2 or 4)", name, b->bits);
-  if (b->group_size != kGroup) return fail(FMOE_ERR_UNSUPPORTED, "%s bank: group_size %d (64)", name, b->group_size);
+  if (b->bits != 2 && b->bits != 4 && b->bits != 8)
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: bits %d (2, 4 or 8)", name, b->bits);
+  if (b->group_size != kGroup && b->group_size != 2 * kGroup)
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: group_size %d (64 or 128)", name, b->group_size);
+  if (b->group_size == 2 * kGroup && (b->hidden < 1024 || b->inter < 1024))
+    return fail(FMOE_ERR_UNSUPPORTED, "%s bank: groups of 128 need hidden and inter of at least 1024", name);
   if (b->num_experts < 1) return fail(FMOE_ERR_INVALID_ARG, "%s bank: num_experts %d", name, b->num_experts);
   const int H = b->hidden, I = b->inter;
   if (H < 128 || I < 128 || H % 128 || I % 128)
@@ -214,8 +218,8 @@ const char* fmoe_status_string(fmoe_status s) {
 
 fmoe_status fmoe_bank_layout(int bits, int group_size, int hidden, int inter, int64_t* record_bytes, int64_t off[9]) {
   if (!record_bytes || !off) return fail(FMOE_ERR_INVALID_ARG, "NULL output");
-  if (bits != 2 && bits != 4) return fail(FMOE_ERR_UNSUPPORTED, "bits %d", bits);
-  if (group_size != kGroup) return fail(FMOE_ERR_UNSUPPORTED, "group_size %d", group_size);
+  if (bits != 2 && bits != 4 && bits != 8) return fail(FMOE_ERR_UNSUPPORTED, "bits %d", bits);
+  if (group_size != kGroup && group_size != 2 * kGroup) return fail(FMOE_ERR_UNSUPPORTED, "group_size %d", group_size);
   if (hidden <= 0 || inter <= 0 || hidden % group_size || inter % group_size)
     return fail(FMOE_ERR_INVALID_ARG, "hidden %d / inter %d", hidden, inter);
   const int64_t dims[3][2] = {{inter, hidden}, {inter, hidden}, {hidden, inter}};
@@ -345,7 +349,8 @@ fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, f
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + L.ctrl);
   const int bits = bank->bits;
-  if (!three_kernel_path() && token_path_supported(bits, bank->hidden, bank->inter, 1, 0, ref(*bank), ref(*bank))) {
+  if (!three_kernel_path() && bank->group_size == kGroup &&
+      token_path_supported(bits, bank->hidden, bank->inter, 1, 0, ref(*bank), ref(*bank))) {
     const bool pdl = pdl_enabled();
     cudaError_t e = launch_tok_xq(x, bank->hidden, bits, base + L.xq_limbs, reinterpret_cast<float2*>(base + L.xq_cs),
                                   &ctrl->tok_count, pdl, cs(stream));
@@ -374,6 +379,7 @@ fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, f
   ExpertParams p{};
   p.routed = ref(*bank);
   p.shared = ref(*bank);
+  p.gsh = bank->group_size == 2 * kGroup ? 1 : 0;
   p.route_idx = nullptr;
   p.route_w = nullptr;
   p.E = bank->num_experts;
@@ -403,8 +409,8 @@ static fmoe_status check_layer(const fmoe_layer* layer) {
   if (st != FMOE_OK) return st;
   if ((st = check_bank(&layer->shared, "shared")) != FMOE_OK) return st;
   const fmoe_bank &r = layer->routed, &s = layer->shared;
-  if (r.bits != s.bits || r.hidden != s.hidden || r.inter != s.inter)
-    return fail(FMOE_ERR_UNSUPPORTED, "routed and shared banks must share bits, hidden and inter");
+  if (r.bits != s.bits || r.hidden != s.hidden || r.inter != s.inter || r.group_size != s.group_size)
+    return fail(FMOE_ERR_UNSUPPORTED, "routed and shared banks must share bits, group size, hidden and inter");
   if (!layer->w_router || !layer->w_shared_gate) return fail(FMOE_ERR_INVALID_ARG, "w_router or w_shared_gate is NULL");
   if (!aligned16(layer->w_router) || !aligned16(layer->w_shared_gate))
     return fail(FMOE_ERR_ALIGNMENT, "w_router and w_shared_gate must be 16-byte aligned");
@@ -441,7 +447,7 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
 static fmoe_status layer_token(const fmoe_layer* layer, const float* h, float* out, int32_t* idx_out, float* w_out,
                                uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word = nullptr) {
   const fmoe_bank& r = layer->routed;
-  if (three_kernel_path() ||
+  if (three_kernel_path() || r.group_size != kGroup ||
       !token_path_supported(r.bits, r.hidden, r.inter, layer->top_k, 1, ref(r), ref(layer->shared)))
     return layer_token_3k(layer, h, out, idx_out, w_out, base, L, s, err_word);
   const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
@@ -548,6 +554,7 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
   ExpertParams p{};
   p.routed = ref(r);
   p.shared = ref(layer->shared);
+  p.gsh = r.group_size == 2 * kGroup ? 1 : 0;
   p.logits = rp.logits;
   p.idx_out = idx_out;
   p.w_out = w_out;
@@ -612,11 +619,12 @@ static fmoe_status run_fused(const fmoe_layer* layers, int nl, const float* h, i
                              float* w_out, uint8_t* base, const WsLayout& L, cudaStream_t s, int* err_word,
                              bool& taken) {
   taken = false;
-  if (!fused_enabled() || nl < 1 || nl > kFusedMaxLayers) return FMOE_OK;
+  if (!fused_enabled() || nl < 1 || nl > kFusedMaxLayers || layers[0].routed.group_size != kGroup) return FMOE_OK;
   const fmoe_bank& r0 = layers[0].routed;
   for (int l = 0; l < nl; ++l) {
     const fmoe_layer& y = layers[l];
     if (y.routed.bits != r0.bits || y.routed.hidden != r0.hidden || y.routed.inter != r0.inter ||
+        y.routed.group_size != r0.group_size ||
         y.routed.num_experts != r0.num_experts || y.top_k != layers[0].top_k || !same_offsets(y.routed, r0) ||
         !same_offsets(y.shared, r0))
       return FMOE_OK;
@@ -686,7 +694,8 @@ static fmoe_status run_grouped(const fmoe_layer* layer, const float* h, int T, f
   if (T < kGroupedMinT || (v && v[0] == '0')) return FMOE_OK;
   const fmoe_bank& r = layer->routed;
   const int H = r.hidden, E = r.num_experts, K = layer->top_k, I = r.inter, bits = r.bits;
-  if (!grouped_shapes_supported(bits, H, I, E, K, T) || !same_offsets(r, layer->shared)) return FMOE_OK;
+  if (r.group_size != kGroup || !grouped_shapes_supported(bits, H, I, E, K, T) || !same_offsets(r, layer->shared))
+    return FMOE_OK;
   const GLayout G = glayout(H, E, K, I, T);
   if (ws_bytes < G.total) return FMOE_OK;
   WsControl* ctrl = reinterpret_cast<WsControl*>(base + G.ctrl);
@@ -967,7 +976,8 @@ fmoe_status fmoe_moe_layer_cached(const fmoe_layer* layer, const fmoe_expert_cac
   if ((st = check_layer(&lc)) != FMOE_OK) return st;
   const int H = lc.routed.hidden, I = lc.routed.inter, K = lc.top_k, b = lc.routed.bits;
   if (K > cp.C) return fail(FMOE_ERR_INVALID_ARG, "top_k %d > num_slots %d", K, cp.C);
-  const int64_t qg = (int64_t)I * H * b / 8, sg = (int64_t)I * (H / 64) * 2, sd = (int64_t)H * (I / 64) * 2;
+  const int gs = lc.routed.group_size;
+  const int64_t qg = (int64_t)I * H * b / 8, sg = (int64_t)I * (H / gs) * 2, sd = (int64_t)H * (I / gs) * 2;
   const int64_t len[9] = {qg, sg, sg, qg, sg, sg, qg, sd, sd};
   for (int i = 0; i < 9; ++i)
     if (lc.routed.off[i] + len[i] > cp.rec)

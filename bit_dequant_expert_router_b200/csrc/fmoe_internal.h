@@ -62,6 +62,7 @@ struct ExpertParams {
   float* rt_w;                // [K+1], slot K = shared-gate sigma
   int E;
   int fixed_expert;
+  int gsh;                    // weight groups of 64 << gsh columns (0: 64, 1: 128); x digits stay per 64
   int K;                      // routed slots
   int has_shared;             // slot K is the shared expert
   int H, I;

@@ -1,7 +1,8 @@
 // k_expert.cu -- packed-code dequant GEMVs of the selected experts.
 //
 // gate/up + SwiGLU and down + combine, after "What is Flash-MoE" (a2a-mcp.org),
-// sections 2-3: 4-bit / 2-bit tiled dequant matvec, fused SwiGLU, and one
+// sections 2-3: 4-bit / 2-bit tiled dequant matvec (and 8-bit, which one page lists
+// among the formats the engine has tried), fused SwiGLU, and one
 // combine pass of the weighted experts, the sigmoid-gated shared expert and the
 // residual.  Weight = code * scale + bias per group of 64; the pages fold the
 // affine into fma(code, scale*x, bias*x) per element.  Here the fold is taken
@@ -34,15 +35,17 @@ constexpr int kGuWarps = 8;
 constexpr int kMaxChunkUnits = 20;  // units per staged chunk, at most (few, large copies: each costs issue time)
 constexpr size_t kGuSmemBudget = 220 * 1024;  // shared memory of the gate/up kernel
 
-template <int BITS, int NG>
+// GSH: log2 of the weight group size over 64 (0: groups of 64, 1: groups of 128; the
+// digits of x stay per 64 columns, and group g of 64 takes scale and bias g >> GSH).
+template <int BITS, int NG, int GSH = 0>
 struct GuCfg {
   using G = Geo<NG>;
-  static constexpr int kPasses = NG >= 32 ? (BITS == 4 ? 1 : 2) : 1;
+  static constexpr int kPasses = NG >= 32 && BITS == 2 ? 2 : 1;
   static constexpr int kRowPairs = G::kRowsPerPass * kPasses;  // rows of gate (and of up) per unit
   static constexpr int kRowBytes = NG * kGroup * BITS / 8;
-  static constexpr int kScaleBytes = NG * 2;
-  static constexpr int kChunks = NG * kGroup * BITS / 128;
-  static constexpr int kDigitBytes = NG * kGroupWords * 4 + kChunks * 8;  // x digits + chunk scalars
+  static constexpr int kScaleBytes = (NG >> GSH) * 2;
+  static constexpr int kChunks = NG * Fmt<BITS>::kCsPerGroup;             // {cscale, sum x} pairs of x
+  static constexpr int kDigitBytes = NG * kGroupWords * 4 + kChunks * 8;  // x digits + their scalars
   static constexpr int kHead = (kDigitBytes + 127) / 128 * 128;
   // units per chunk: kMaxChunkUnits, or fewer where two chunk buffers would not fit
   static constexpr int kUnitBytes = 2 * kRowPairs * (kRowBytes + 2 * kScaleBytes);
@@ -64,19 +67,19 @@ struct GuMaps {
 // Persistent: CTA b owns units [b*U/G, (b+1)*U/G) (a unit = kRowPairs rows of
 // gate and up of one expert slot), cut into chunks of up to C::kChunkUnits units
 // of one slot, each staged into a ring of nbuf chunk buffers with three copies (gate
-// codes, up codes, and the four scale arrays as one tensor copy of a whole box of
-// C::kChunkRows rows) or, where the record layout has no such map, six bulk copies;
+// codes, up codes, and the four scale arrays as one tensor copy of a whole box: as many
+// rows as the largest chunk of the launch) or, where the record layout has no such map,
+// six bulk copies;
 // warp w computes units w, w+8, .. of the chunk.  A lane always works on the same
 // groups of 64 columns, so it keeps their digits of x in registers for the whole kernel.
-template <int BITS, int NG>
+template <int BITS, int NG, int GSH>
 __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertParams p, int nbuf, int use_maps,
-                                                                  const __grid_constant__ GuMaps maps) {
+                                                                  int box_rows, const __grid_constant__ GuMaps maps) {
   using G = Geo<NG>;
-  using C = GuCfg<BITS, NG>;
+  using C = GuCfg<BITS, NG, GSH>;
   constexpr int RP = C::kRowPairs, PASSES = C::kPasses;
   constexpr int LPR = G::kLanesPerRow, RPP = G::kRowsPerPass, GPL = G::kGroupsPerLane;
   constexpr int RB = C::kRowBytes, SB = C::kScaleBytes, CR = C::kChunkRows, CHB = C::kChunkBytes;
-  constexpr int LW = Fmt<BITS>::kLimbWords;
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ __align__(8) uint64_t s_bar[8];
   __shared__ __align__(8) uint64_t s_bar_x;
@@ -113,8 +116,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
     const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_bar[c % nbuf]);
     const uint32_t cb = rows * RB, sb = rows * SB;
-    if (use_maps) {  // the scale box always moves C::kChunkRows rows (past the last row: zeros)
-      mbar_expect_tx(bar, 2 * cb + 4 * CR * SB);
+    if (use_maps) {  // the scale box always moves box_rows rows (past the last row: zeros)
+      mbar_expect_tx(bar, 2 * cb + 4 * box_rows * SB);
       bulk_g2s(dst, rec + off[0] + (long long)r0 * RB, cb, bar, pol);
       bulk_g2s(dst + CR * RB, rec + off[3] + (long long)r0 * RB, cb, bar, pol);
       tma_5d(dst + 2 * CR * RB, &maps.sb[routed ? 0 : 1], 0, 0, r0, routed ? s_idx[sl] : 0, bar, pol);
@@ -235,16 +238,25 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
 #pragma unroll
         for (int i = 0; i < PASSES; ++i) {
           const int r = k * RP + sub + RPP * i;  // row within the chunk
-          uint4 q0, q1, v0, v1;
-          load_group_codes<BITS>(buf + r * RB, g, q0, q1);
-          load_group_codes<BITS>(buf + CR * RB + r * RB, g, v0, v1);
-          const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * CR * RB) + r * srow + g;
+          float Sg, Su;
+          if constexpr (BITS == 8) {
+            uint4 q[4], v[4];
+            load_group_codes8(buf + r * RB, g, q);
+            load_group_codes8(buf + CR * RB + r * RB, g, v);
+            Sg = group_dot8(q, L[j]);
+            Su = group_dot8(v, L[j]);
+          } else {
+            uint4 q0, q1, v0, v1;
+            load_group_codes<BITS>(buf + r * RB, g, q0, q1);
+            load_group_codes<BITS>(buf + CR * RB + r * RB, g, v0, v1);
+            Sg = group_dot<BITS>(q0, q1, L[j]);
+            Su = group_dot<BITS>(v0, v1, L[j]);
+          }
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(buf + 2 * CR * RB) + r * srow + (g >> GSH);
           const float gs = bf16_to_f32(sc[0]);
           const float gb = bf16_to_f32(sc[sarr]);
           const float us = bf16_to_f32(sc[2 * sarr]);
           const float ub = bf16_to_f32(sc[3 * sarr]);
-          const float Sg = group_dot<BITS>(q0, q1, L[j]);
-          const float Su = group_dot<BITS>(v0, v1, L[j]);
           accg[i] = fmaf(gs, cs[j].x * Sg, fmaf(gb, cs[j].y, accg[i]));
           accu[i] = fmaf(us, cs[j].x * Su, fmaf(ub, cs[j].y, accu[i]));
         }
@@ -308,9 +320,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     __threadfence();
     const int g = g0 + t, slot = g * kGroup / I, gg = (g * kGroup % I) / kGroup;
     const float2 v = __ldcg(reinterpret_cast<const float2*>(p.act + (size_t)g * kGroup) + lane);
-    const int ncd = I * BITS / 128;
-    xq_quantize_group<BITS>(v.x, v.y, gg, I / kGroup, p.act_limbs + (size_t)slot * ncd * LW * 4,
-                            p.act_cs + (size_t)slot * ncd);
+    xq_quantize_group<BITS>(v.x, v.y, gg, I / kGroup, p.act_limbs + (size_t)slot * I * 3,
+                            p.act_cs + (size_t)slot * (I / kGroup) * Fmt<BITS>::kCsPerGroup);
     if (lane == 0) p.grp_cnt[g] = 0u;
   }
 }
@@ -319,13 +330,13 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
 
 constexpr int kDnWarps = 8;
 
-template <int BITS, int NG>
+template <int BITS, int NG, int GSH = 0>
 struct DnCfg {
   static constexpr int kRowBytes = NG * kGroup * BITS / 8;
-  static constexpr int kScaleBytes = NG * 2;
+  static constexpr int kScaleBytes = (NG >> GSH) * 2;
   // output rows per unit: 2, or more when a row's scales are too short for a 16-byte copy
   static constexpr int kRows = kScaleBytes >= 8 ? 2 : 16 / kScaleBytes;
-  static constexpr int kChunks = NG * kGroup * BITS / 128;
+  static constexpr int kChunks = NG * Fmt<BITS>::kCsPerGroup;  // {cscale, sum a} pairs of a slot's activations
   static_assert(kRows * kScaleBytes % 16 == 0 && kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
 };
 
@@ -337,9 +348,9 @@ struct DnCfg {
 // CTA's rows by then, so the copies come mostly from L2.  Lane l owns the (slot, group) pairs
 // q = l, l+32, .. (PPL of them) of every row and keeps their digits in
 // registers; the warp sums a row's pairs by shuffles.
-template <int BITS, int NG, int PPL>
+template <int BITS, int NG, int PPL, int GSH>
 __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertParams p, int chunk_units, int nbuf) {
-  using C = DnCfg<BITS, NG>;
+  using C = DnCfg<BITS, NG, GSH>;
   constexpr int RD = C::kRows;
   constexpr int RB = C::kRowBytes, SB = C::kScaleBytes;
   constexpr int NCH = C::kChunks;
@@ -480,12 +491,20 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
 #pragma unroll
         for (int r = 0; r < RD; ++r) {
           const int row = k * RD + r;  // row within the chunk
-          uint4 q0, q1;
-          load_group_codes<BITS>(sb + row * RB, qg[m], q0, q1);
-          const float sc = bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + crows * RB + row * SB)[qg[m]]);
+          float S;
+          if constexpr (BITS == 8) {
+            uint4 q[4];
+            load_group_codes8(sb + row * RB, qg[m], q);
+            S = group_dot8(q, L[m]);
+          } else {
+            uint4 q0, q1;
+            load_group_codes<BITS>(sb + row * RB, qg[m], q0, q1);
+            S = group_dot<BITS>(q0, q1, L[m]);
+          }
+          const float sc =
+              bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + crows * RB + row * SB)[qg[m] >> GSH]);
           const float bi =
-              bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + crows * RB + crows * SB + row * SB)[qg[m]]);
-          const float S = group_dot<BITS>(q0, q1, L[m]);
+              bf16_to_f32(reinterpret_cast<const uint16_t*>(sb + crows * RB + crows * SB + row * SB)[qg[m] >> GSH]);
           acc[r] = fmaf(wq[m], fmaf(sc, cs[m].x * S, bi * cs[m].y), acc[r]);
         }
       }
@@ -542,9 +561,9 @@ bool encode_gu_scale_maps(GuMaps& m, const ExpertParams& p, int SB, int box_rows
   return true;
 }
 
-template <int BITS, int NG>
+template <int BITS, int NG, int GSH>
 cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
-  using C = GuCfg<BITS, NG>;
+  using C = GuCfg<BITS, NG, GSH>;
   const int NE = p.K + p.has_shared;
   const int units = NE * (p.I / C::kRowPairs);
   int grid = num_sms();
@@ -558,18 +577,20 @@ cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
   nbuf = nbuf > 8 ? 8 : nbuf;
   if (nbuf < 1) return cudaErrorInvalidValue;
   const size_t smem = C::kHead + (size_t)nbuf * C::kChunkBytes;
-  void (*k)(const ExpertParams, int, int, const GuMaps) = gateup_kernel<BITS, NG>;
+  void (*k)(const ExpertParams, int, int, int, const GuMaps) = gateup_kernel<BITS, NG, GSH>;
   cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
   GuMaps maps;
-  const int use_maps = encode_gu_scale_maps(maps, p, C::kScaleBytes, C::kChunkRows) ? 1 : 0;
-  return launch_pdl(k, dim3(grid), dim3(kGuWarps * 32), smem, s, pdl, p, nbuf, use_maps, maps);
+  // a chunk never holds more units than a CTA's range: the scale box need not either
+  const int box_rows = C::kRowPairs * (per_cta < C::kChunkUnits ? per_cta : C::kChunkUnits);
+  const int use_maps = encode_gu_scale_maps(maps, p, C::kScaleBytes, box_rows) ? 1 : 0;
+  return launch_pdl(k, dim3(grid), dim3(kGuWarps * 32), smem, s, pdl, p, nbuf, use_maps, box_rows, maps);
 }
 
 // Down-kernel staging: (chunk units, buffers, shared bytes) for NE slots, or false.
-template <int BITS, int NG>
+template <int BITS, int NG, int GSH = 0>
 bool down_plan(int H, int NE, int& chunk_units, int& nbuf, size_t& smem) {
-  using C = DnCfg<BITS, NG>;
+  using C = DnCfg<BITS, NG, GSH>;
   const int units = H / C::kRows;
   int grid = num_sms();
   grid = grid > units ? units : grid;
@@ -589,21 +610,21 @@ bool down_plan(int H, int NE, int& chunk_units, int& nbuf, size_t& smem) {
   return true;
 }
 
-template <int BITS, int NG>
+template <int BITS, int NG, int GSH>
 cudaError_t down_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
-  using C = DnCfg<BITS, NG>;
+  using C = DnCfg<BITS, NG, GSH>;
   const int NE = p.K + p.has_shared;
   int cu = 0, nbuf = 0;
   size_t smem = 0;
   const int ppl = (NE * NG + 31) / 32;
-  if (!down_plan<BITS, NG>(p.H, NE, cu, nbuf, smem) || ppl > 4) return cudaErrorInvalidValue;
+  if (!down_plan<BITS, NG, GSH>(p.H, NE, cu, nbuf, smem) || ppl > 4) return cudaErrorInvalidValue;
   const int units = p.H / C::kRows;
   int grid = num_sms();
   grid = grid > units ? units : grid;
-  void (*k)(const ExpertParams, int, int) = ppl == 1 ? down_kernel<BITS, NG, 1>
-                                          : ppl == 2 ? down_kernel<BITS, NG, 2>
-                                          : ppl == 3 ? down_kernel<BITS, NG, 3>
-                                                     : down_kernel<BITS, NG, 4>;
+  void (*k)(const ExpertParams, int, int) = ppl == 1 ? down_kernel<BITS, NG, 1, GSH>
+                                          : ppl == 2 ? down_kernel<BITS, NG, 2, GSH>
+                                          : ppl == 3 ? down_kernel<BITS, NG, 3, GSH>
+                                                     : down_kernel<BITS, NG, 4, GSH>;
   cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(grid), dim3(kDnWarps * 32), smem, s, pdl, p, cu, nbuf);
@@ -611,28 +632,46 @@ cudaError_t down_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
 
 template <int BITS>
 cudaError_t gateup_bits(const ExpertParams& p, bool pdl, cudaStream_t s) {
+  if (p.gsh == 1) {  // groups of 128: rows of at least 16 groups of 64
+    switch (p.H / kGroup) {
+      case 16: return gateup_dispatch<BITS, 16, 1>(p, pdl, s);
+      case 32: return gateup_dispatch<BITS, 32, 1>(p, pdl, s);
+      case 64: return gateup_dispatch<BITS, 64, 1>(p, pdl, s);
+      case 128: return gateup_dispatch<BITS, 128, 1>(p, pdl, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (p.H / kGroup) {
-    case 2: return gateup_dispatch<BITS, 2>(p, pdl, s);
-    case 4: return gateup_dispatch<BITS, 4>(p, pdl, s);
-    case 8: return gateup_dispatch<BITS, 8>(p, pdl, s);
-    case 16: return gateup_dispatch<BITS, 16>(p, pdl, s);
-    case 32: return gateup_dispatch<BITS, 32>(p, pdl, s);
-    case 64: return gateup_dispatch<BITS, 64>(p, pdl, s);
-    case 128: return gateup_dispatch<BITS, 128>(p, pdl, s);
+    case 2: return gateup_dispatch<BITS, 2, 0>(p, pdl, s);
+    case 4: return gateup_dispatch<BITS, 4, 0>(p, pdl, s);
+    case 8: return gateup_dispatch<BITS, 8, 0>(p, pdl, s);
+    case 16: return gateup_dispatch<BITS, 16, 0>(p, pdl, s);
+    case 32: return gateup_dispatch<BITS, 32, 0>(p, pdl, s);
+    case 64: return gateup_dispatch<BITS, 64, 0>(p, pdl, s);
+    case 128: return gateup_dispatch<BITS, 128, 0>(p, pdl, s);
   }
   return cudaErrorInvalidValue;
 }
 
 template <int BITS>
 cudaError_t down_bits(const ExpertParams& p, bool pdl, cudaStream_t s) {
+  if (p.gsh == 1) {
+    switch (p.I / kGroup) {
+      case 16: return down_dispatch<BITS, 16, 1>(p, pdl, s);
+      case 32: return down_dispatch<BITS, 32, 1>(p, pdl, s);
+      case 64: return down_dispatch<BITS, 64, 1>(p, pdl, s);
+      case 128: return down_dispatch<BITS, 128, 1>(p, pdl, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (p.I / kGroup) {
-    case 2: return down_dispatch<BITS, 2>(p, pdl, s);
-    case 4: return down_dispatch<BITS, 4>(p, pdl, s);
-    case 8: return down_dispatch<BITS, 8>(p, pdl, s);
-    case 16: return down_dispatch<BITS, 16>(p, pdl, s);
-    case 32: return down_dispatch<BITS, 32>(p, pdl, s);
-    case 64: return down_dispatch<BITS, 64>(p, pdl, s);
-    case 128: return down_dispatch<BITS, 128>(p, pdl, s);
+    case 2: return down_dispatch<BITS, 2, 0>(p, pdl, s);
+    case 4: return down_dispatch<BITS, 4, 0>(p, pdl, s);
+    case 8: return down_dispatch<BITS, 8, 0>(p, pdl, s);
+    case 16: return down_dispatch<BITS, 16, 0>(p, pdl, s);
+    case 32: return down_dispatch<BITS, 32, 0>(p, pdl, s);
+    case 64: return down_dispatch<BITS, 64, 0>(p, pdl, s);
+    case 128: return down_dispatch<BITS, 128, 0>(p, pdl, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -730,7 +769,9 @@ bool fits_u(int ngu, int ngd, int ne) {
 
 bool expert_shapes_supported(int bits, int H, int I, int ne) {
   if (H % kGroup || I % kGroup) return false;
-  return bits == 4 ? fits_u<4>(H / kGroup, I / kGroup, ne) : fits_u<2>(H / kGroup, I / kGroup, ne);
+  return bits == 8   ? fits_u<8>(H / kGroup, I / kGroup, ne)
+         : bits == 4 ? fits_u<4>(H / kGroup, I / kGroup, ne)
+                     : fits_u<2>(H / kGroup, I / kGroup, ne);
 }
 
 cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err,
@@ -740,11 +781,11 @@ cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsig
 }
 
 cudaError_t launch_gateup(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {
-  return bits == 4 ? gateup_bits<4>(p, pdl, s) : gateup_bits<2>(p, pdl, s);
+  return bits == 8 ? gateup_bits<8>(p, pdl, s) : bits == 4 ? gateup_bits<4>(p, pdl, s) : gateup_bits<2>(p, pdl, s);
 }
 
 cudaError_t launch_down(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {
-  return bits == 4 ? down_bits<4>(p, pdl, s) : down_bits<2>(p, pdl, s);
+  return bits == 8 ? down_bits<8>(p, pdl, s) : bits == 4 ? down_bits<4>(p, pdl, s) : down_bits<2>(p, pdl, s);
 }
 
 }  // namespace fmoe

@@ -738,6 +738,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_kernel(const __grid_constant__ F
 FusedPlan plan_fused(int bits, int H, int I, int E, int K) {
   FusedPlan pl{};
   pl.ok = false;
+  if (bits != 2 && bits != 4) return pl;  // this path has no 8-bit form
   if (H % kGroup || I % kGroup || K < 1 || K > 32 || E < K || E > kFW * 64) return pl;
   const int NGH = H / kGroup, NGI = I / kGroup, NE = K + 1;
   if (NGH > 128 || NGI > 128) return pl;

@@ -1239,6 +1239,7 @@ cudaError_t down_bits_g(const GroupedParams& p, bool pdl, cudaStream_t s) {
 }  // namespace
 
 bool grouped_shapes_supported(int bits, int H, int I, int E, int K, int T) {
+  if (bits != 2 && bits != 4) return false;  // this path has no 8-bit form (token by token instead)
   if (H < 512 || I < 512) return false;  // scale rows of at least 16 bytes (one tensor-copy line)
   if (T * K > kMaxTK || ((size_t)T * K + 2 * (size_t)E) * 4 > 200 * 1024) return false;
   const TcConfig gu = gu_config(bits, H), dn = dn_config(bits, I);

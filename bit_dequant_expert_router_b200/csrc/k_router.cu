@@ -250,7 +250,9 @@ cudaError_t launch_rmsnorm(const float* h, const float* gamma, float eps, int T,
 cudaError_t launch_xq(const float* x, int H, int bits, uint8_t* limbs, float2* cs, cudaStream_t s) {
   const int groups = H / kGroup;
   const int grid = (groups + 7) / 8;
-  if (bits == 4)
+  if (bits == 8)
+    xq_kernel<8><<<grid, 256, 0, s>>>(x, H, limbs, cs);
+  else if (bits == 4)
     xq_kernel<4><<<grid, 256, 0, s>>>(x, H, limbs, cs);
   else
     xq_kernel<2><<<grid, 256, 0, s>>>(x, H, limbs, cs);
@@ -267,7 +269,10 @@ cudaError_t launch_router(RouterParams p, int xq_bits, bool pdl, cudaStream_t s)
   p.rows_per_cta = (R + nb - 1) / nb;
   const size_t smem = (size_t)p.rows_per_cta * p.H * 2 + (size_t)p.H * 4;
   cudaError_t e;
-  void (*k)(RouterParams) = xq_bits == 4 ? router_kernel<4> : (xq_bits == 2 ? router_kernel<2> : router_kernel<0>);
+  void (*k)(RouterParams) = xq_bits == 8   ? router_kernel<8>
+                            : xq_bits == 4 ? router_kernel<4>
+                            : xq_bits == 2 ? router_kernel<2>
+                                           : router_kernel<0>;
   if ((e = set_smem((const void*)k, smem)) != cudaSuccess) return e;
   return launch_pdl(k, dim3(nb, p.T), dim3(kRouterThreads), smem, s, pdl, p);
 }

@@ -996,6 +996,7 @@ TokPlan plan_token(int bits, int H, int I, int K, int has_shared) {
 }
 
 bool token_path_supported(int bits, int H, int I, int K, int has_shared, const BankRef& routed, const BankRef& shared) {
+  if (bits != 2 && bits != 4) return false;  // this path has no 8-bit form
   return plan_token(bits, H, I, K, has_shared).ok && tok_layout_ok(routed, bits, H, I) &&
          tok_layout_ok(shared, bits, H, I);
 }

@@ -22,7 +22,7 @@ __global__ void packed_bank_kernel(uint64_t seed, uint64_t layer, uint64_t exper
     const int e = (int)(t / ((long long)gpr * rows));
     const uint64_t key = fg_key(seed, fg_stream_id(layer, expert_id0 + (uint64_t)e, (uint64_t)kind));
     float w[256];
-    uint32_t words[16];
+    uint32_t words[32];
     for (int i = 0; i < wpg; ++i) words[i] = 0u;
     fg_draw_group(key, std, cols, r, g, gs, w);
     uint16_t sb, bb;
@@ -59,7 +59,7 @@ extern "C" {
 int fg_cuda_packed_bank(uint64_t seed, uint64_t layer, uint64_t expert_id0, int ne, int kind, float std, int bits,
                         int gs, int rows, int cols, void* base, long long stride, long long off_qw, long long off_s,
                         long long off_b, cudaStream_t stream) {
-  if (gs > 256 || gs * bits / 32 > 16 || cols % gs != 0 || (gs * bits) % 32 != 0) return (int)cudaErrorInvalidValue;
+  if (gs > 256 || gs * bits / 32 > 32 || cols % gs != 0 || (gs * bits) % 32 != 0) return (int)cudaErrorInvalidValue;
   const long long total = (long long)ne * rows * (cols / gs);
   packed_bank_kernel<<<grid_for(total), 256, 0, stream>>>(seed, layer, expert_id0, ne, kind, std, bits, gs, rows, cols,
                                                           (unsigned char*)base, stride, off_qw, off_s, off_b);

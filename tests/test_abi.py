@@ -38,14 +38,16 @@ def test_version_and_status_strings():
     assert L.fmoe_status_string(6) == b"FMOE_ERR_DEVICE_TIMEOUT"
 
 
-@pytest.mark.parametrize("bits,H,I", [(4, 4096, 1024), (2, 4096, 1024), (4, 256, 128), (2, 256, 128)])
-def test_bank_layout_matches_generator_layout(bits, H, I):
-    assert fmoe.bank_layout(bits, H, I) == gen.record_layout(bits, H, I)
+@pytest.mark.parametrize("bits,H,I,group", [(4, 4096, 1024, 64), (2, 4096, 1024, 64), (4, 256, 128, 64),
+                                             (2, 256, 128, 64), (8, 4096, 1024, 64), (4, 4096, 1024, 128),
+                                             (8, 1024, 2048, 128)])
+def test_bank_layout_matches_generator_layout(bits, H, I, group):
+    assert fmoe.bank_layout(bits, H, I, group) == gen.record_layout(bits, H, I, group)
 
 
-def _fake_bank(bits=4, H=4096, I=1024, E=512, base=0x10000000, stride=None, off=None):
-    nb, o = gen.record_layout(bits, H, I)
-    b = _abi.FmoeBank(bits, 64, H, I, E, 0, base, nb if stride is None else stride,
+def _fake_bank(bits=4, H=4096, I=1024, E=512, base=0x10000000, stride=None, off=None, group=64):
+    nb, o = gen.record_layout(bits, H, I, group)
+    b = _abi.FmoeBank(bits, group, H, I, E, 0, base, nb if stride is None else stride,
                       (ctypes.c_int64 * 9)(*(o if off is None else off)))
     return b
 
@@ -84,6 +86,14 @@ def test_layer_validation_errors_are_reported_before_any_launch():
     assert _call_layer(_fake_layer(), T=0) == 0            # empty batch: nothing enqueued
     # (top_k + 1) * inter*bits/128 must fit one 512-thread CTA
     assert _call_layer(_fake_layer(top_k=16)) == 3
+    # code widths 2, 4, 8 and groups of 64 or 128 pass the format checks (the misaligned
+    # base is then what fails); other widths and group sizes do not
+    assert _call_layer(_fake_layer(bits=8, base=0x10000008)) == 2
+    assert _call_layer(_fake_layer(group=128, base=0x10000008)) == 2
+    assert _call_layer(_fake_layer(bits=8, group=128, base=0x10000008)) == 2
+    assert _call_layer(_fake_layer(group=96)) == 3
+    assert _call_layer(_fake_layer(group=128, H=512, I=512)) == 3   # groups of 128 from hidden 1024 up
+    assert _call_layer(_fake_layer(bits=6)) == 3
 
 
 def test_workspace_size_query_is_positive_and_monotone():

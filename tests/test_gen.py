@@ -58,10 +58,14 @@ def test_zipf_bias_is_a_permuted_zipf_distribution():
 
 
 def test_record_layout_offsets_are_aligned_and_ordered():
-    for bits in (2, 4):
+    for bits in (2, 4, 8):
         for H, I in ((256, 128), (4096, 1024)):
             n, off = gen.record_layout(bits, H, I)
             assert all(o % 16 == 0 for o in off) and off == sorted(off) and n % 16 == 0
+    # groups of 128: the scale and bias arrays are half as long
+    n64, _ = gen.record_layout(4, 4096, 1024)
+    n128, _ = gen.record_layout(4, 4096, 1024, group=128)
+    assert n64 - n128 == 3 * 2 * 1024 * (4096 // 128) * 2
     assert gen.algorithmic_bytes_per_token(gen.qwen397_layer(4)) == 39583744
     assert gen.algorithmic_bytes_per_token(gen.qwen397_layer(2)) == 23855104
     assert gen.algorithmic_bytes_per_token(gen.tiny_layer()) == 169984

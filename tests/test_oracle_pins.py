@@ -55,6 +55,8 @@ def test_code_fields_lsb_first():
     # Word 0x76543210: field j holds j (4-bit); 0xE4 = 0b11100100 holds 0,1,2,3 (2-bit).
     assert [oracle.code([0x76543210], 4, c) for c in range(8)] == list(range(8))
     assert [oracle.code([0xE4E4E4E4], 2, c) for c in range(16)] == [0, 1, 2, 3] * 4
+    # 8-bit: one code per byte, byte 0 first; 0xFF is 255 (codes are unsigned)
+    assert [oracle.code([0xFF80_0100], 8, c) for c in range(4)] == [0, 1, 128, 255]
 
 
 def test_record_sizes_match_pages():
@@ -65,21 +67,23 @@ def test_record_sizes_match_pages():
     assert b2 == rs["two_bit_bytes"] and round(b2 / 1e6, 1) == rs["two_bit_mb_approx"]
 
 
-def _random_packed(rng, bits, rows, cols):
+def _random_packed(rng, bits, rows, cols, group=64):
     codes = rng.integers(0, 1 << bits, size=(rows, cols))
     # distinct, bf16-exact scales and biases per (row, group)
-    s = (rng.integers(1, 64, size=(rows, cols // 64)) / 256.0).astype(np.float32)
-    b = (rng.integers(-64, 64, size=(rows, cols // 64)) / 128.0).astype(np.float32)
-    dense = codes * np.repeat(s.astype(np.float64), 64, axis=1) + np.repeat(b.astype(np.float64), 64, axis=1)
+    s = (rng.integers(1, 64, size=(rows, cols // group)) / 256.0).astype(np.float32)
+    b = (rng.integers(-64, 64, size=(rows, cols // group)) / 128.0).astype(np.float32)
+    dense = codes * np.repeat(s.astype(np.float64), group, axis=1) + np.repeat(b.astype(np.float64), group, axis=1)
     return codes, np_pack(codes, bits), f32_to_bf16_exact(s), f32_to_bf16_exact(b), dense
 
 
-@pytest.mark.parametrize("bits,rows,cols", [(4, 3, 192), (2, 5, 128), (4, 7, 64), (2, 2, 320)])
-def test_onegrid_roundtrip_and_dense_bruteforce(bits, rows, cols):
-    rng = np.random.default_rng(bits * 1000 + rows)
-    codes, qw, s, b, dense = _random_packed(rng, bits, rows, cols)
+@pytest.mark.parametrize("bits,rows,cols,group", [(4, 3, 192, 64), (2, 5, 128, 64), (4, 7, 64, 64), (2, 2, 320, 64),
+                                                  (8, 3, 128, 64), (8, 2, 192, 64), (4, 3, 256, 128),
+                                                  (2, 2, 384, 128), (8, 3, 256, 128)])
+def test_onegrid_roundtrip_and_dense_bruteforce(bits, rows, cols, group):
+    rng = np.random.default_rng(bits * 1000 + rows + group)
+    codes, qw, s, b, dense = _random_packed(rng, bits, rows, cols, group)
     assert np.array_equal(np_unpack(qw, bits, cols), codes)
-    m = oracle.matrix(qw, s, b, bits, rows, cols)
+    m = oracle.matrix(qw, s, b, bits, rows, cols, group=group)
     got = np.array([[oracle.weight(m, r, c) for c in range(cols)] for r in range(rows)])
     assert np.array_equal(got, dense)  # on-grid weights are exact in fp64
     x = rng.standard_normal(cols)
@@ -204,7 +208,7 @@ def test_layer_combine_closed_form():
     assert np.allclose(r["out"][0], exp, rtol=1e-13, atol=1e-13)
 
 
-@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("bits", [4, 2, 8])
 def test_all_experts_identical_equals_dense_ffn(bits):
     # K = E with byte-identical experts: sum_k w_k y = y (weights sum to 1), so out = h + FFN(x) + sigma FFN_s(x),
     # checked against a dense numpy FFN built by whole-array unpacking.

@@ -56,7 +56,7 @@ def _run_layer(fmoe, dl, h_np, top_k=None, use_gamma=True, T_per_call=None):
     return out.cpu().numpy().astype(np.float64), idx.cpu().numpy(), w.cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("bits", [4, 2, 8])
 @pytest.mark.parametrize("random_gamma", [False, True])
 def test_tiny_layer_matches_oracle(fmoe, bits, random_gamma):
     spec = gen.LayerSpec(**{**gen.tiny_layer(bits).__dict__, "random_gamma": random_gamma})
@@ -116,7 +116,7 @@ def test_results_are_deterministic(fmoe):
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("bits", [4, 2, 8])
 def test_expert_ffn_matches_oracle(fmoe, bits):
     spec = gen.tiny_layer(bits)
     hl = gen.host_layer(spec, seed=4)
@@ -289,3 +289,65 @@ def test_two_kernel_path_full_size(fmoe, big, two_kernels):
     hl, L = full_size_oracle_layer(spec, h, idx)
     exact, _ = _compare_layer(hl, h, out, idx, w, L=L)
     assert exact >= 14, exact
+
+
+def test_eight_bit_small_layer_batch_runs_token_by_token(fmoe):
+    """8-bit codes (one of the formats the gillilab page lists): a 16-token batch of the
+    hidden-512 layer, which the grouped path does not take at 8 bits, against the oracle."""
+    spec = gen.LayerSpec(**{**gen.small_layer(8).__dict__, "random_gamma": True})
+    hl = gen.host_layer(spec, seed=81)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(8100, 16, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    exact, _ = _compare_layer(hl, h, out, idx, w)
+    assert exact >= 15
+
+
+def test_eight_bit_full_size_layer(fmoe):
+    """The Qwen3.5-397B-A17B-shaped layer with 8-bit codes: 16 fresh tokens against the oracle."""
+    spec = gen.qwen397_layer(8)
+    dl = gen.device_layer(spec, seed=0, layer=0)
+    T = 16
+    h = gen.host_tokens(8200, T, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    hl, L = full_size_oracle_layer(spec, h, idx)
+    nbytes = gen.record_bytes(spec)
+    e = int(idx[0, 0])
+    assert np.array_equal(dl.bank[e * nbytes:(e + 1) * nbytes].cpu().numpy(), hl.routed[e])
+    exact, _ = _compare_layer(hl, h, out, idx, w, L=L)
+    assert exact >= 14
+    del dl
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("bits", [4, 2, 8])
+def test_group_128_layer_matches_oracle(fmoe, bits):
+    """Weights grouped by 128 columns (the gillilab page gives groups of 128 or 64): hidden
+    and intermediate 1024, 8 experts, top-2, 16 tokens against the oracle."""
+    spec = gen.LayerSpec(hidden=1024, experts=8, inter=1024, top_k=2, bits=bits, group=128,
+                         router_std=1.0 / 32.0, random_gamma=True)
+    hl = gen.host_layer(spec, seed=128 + bits)
+    dl = gen.upload_layer(hl)
+    h = gen.host_tokens(12800, 16, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    exact, _ = _compare_layer(hl, h, out, idx, w)
+    assert exact >= 15
+    lay = gen.binding_layer(dl)
+    L = oracle_layer(hl)
+    x = np.random.default_rng(bits).standard_normal(spec.hidden).astype(np.float32)
+    y = fmoe.expert_ffn(lay.routed, 3, torch.from_numpy(x).cuda()).cpu().numpy()
+    assert max_rel_err(y, oracle.expert_ffn(L.routed, 3, x)) <= TOL
+
+
+def test_group_128_full_size_layer(fmoe):
+    """The Qwen3.5-397B-A17B-shaped 4-bit layer with groups of 128: 16 fresh tokens."""
+    spec = gen.LayerSpec(**{**gen.qwen397_layer(4).__dict__, "group": 128})
+    dl = gen.device_layer(spec, seed=0, layer=0)
+    T = 16
+    h = gen.host_tokens(12900, T, spec.hidden)
+    out, idx, w = _run_layer(fmoe, dl, h)
+    hl, L = full_size_oracle_layer(spec, h, idx)
+    exact, _ = _compare_layer(hl, h, out, idx, w, L=L)
+    assert exact >= 14
+    del dl
+    torch.cuda.empty_cache()
