@@ -543,13 +543,13 @@ static fmoe_status layer_token_3k(const fmoe_layer* layer, const float* h, float
     rp.route_w = reinterpret_cast<float*>(base + L.route_w);
     rp.idx_out = idx_out;
     rp.w_out = w_out;
+    rp.cache = *cache;
     given_idx = cache_slot_out(*cache);
     given_w = rp.route_w;
   }
   e = launch_router(rp, bits, pdl, s);
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
-  if (cache && (e = launch_cache_lookup(*cache, rp.route_idx, K, cache_slot_out(*cache), rp.err, pdl, s)) != cudaSuccess)
-    return cuda_fail(e, "cache lookup launch");
+  if (cache && (e = launch_cache_copy(*cache, pdl, s)) != cudaSuccess) return cuda_fail(e, "cache copy launch");
   if (trace && (e = trace_record(g_trace[1], s)) != cudaSuccess) return cuda_fail(e, "trace event");
   ExpertParams p{};
   p.routed = ref(r);

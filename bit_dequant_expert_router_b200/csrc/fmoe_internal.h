@@ -9,6 +9,98 @@
 
 namespace fmoe {
 
+// Expert cache (k_cache.cu): host-resident records, HBM slots, tables in `state`.
+constexpr int kCacheMaxK = 32;
+struct CacheHeader {          // first 64 bytes of the state
+  unsigned int clock;         // lookups so far (a slot's last use is the lookup that used it)
+  int err;                    // kDevBadIndex after an index outside the bank (fetch entry point)
+  int n_copy;                 // records the current lookup copies
+  int pad0;
+  unsigned long long hits, misses, bytes;
+  unsigned long long pad1[3];
+};
+struct CacheParams {
+  const uint8_t* host;        // E records at host_stride (pinned host memory, mapped)
+  long long host_stride;
+  uint8_t* slots;             // C records at slot_stride (device)
+  long long slot_stride;
+  long long rec;              // bytes per copied record (multiple of 16)
+  int E, C;
+  uint8_t* state;             // header, copy list [2][kCacheMaxK], slots of the last lookup [kCacheMaxK],
+                              // slot_of [E], expert_of [C], last_use [C]
+};
+__host__ __device__ inline size_t cache_up16(size_t v) { return (v + 15) / 16 * 16; }
+__host__ __device__ inline int* cache_copy_expert(const CacheParams& c) {
+  return reinterpret_cast<int*>(c.state + sizeof(CacheHeader));
+}
+__host__ __device__ inline int* cache_copy_slot(const CacheParams& c) { return cache_copy_expert(c) + kCacheMaxK; }
+__host__ __device__ inline int* cache_slot_out(const CacheParams& c) { return cache_copy_slot(c) + kCacheMaxK; }
+__host__ __device__ inline int* cache_slot_of(const CacheParams& c) { return cache_slot_out(c) + kCacheMaxK; }
+__host__ __device__ inline int* cache_expert_of(const CacheParams& c) {
+  return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cache_slot_of(c)) + cache_up16((size_t)c.E * 4));
+}
+__host__ __device__ inline unsigned int* cache_last_use(const CacheParams& c) {
+  return reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(cache_expert_of(c)) + cache_up16((size_t)c.C * 4));
+}
+
+// One lookup of K experts by one warp (every lane calls it; expert k is lane k's `mine`).
+// Marks them used, picks a victim slot for each missing one (least recently used among the
+// slots this lookup has not used; empty slots first, lowest index among equals), updates
+// the tables, writes the copy list and slot_out[k] (if not NULL).  An id outside [0, E)
+// is replaced by 0 and recorded in *err.  Lane 0 writes the tables; __syncwarp orders them.
+__device__ inline void cache_lookup_warp(const CacheParams& c, int mine, int K, int32_t* slot_out, int* err) {
+  const int lane = threadIdx.x & 31;
+  CacheHeader* hd = reinterpret_cast<CacheHeader*>(c.state);
+  int* slot_of = cache_slot_of(c);
+  int* expert_of = cache_expert_of(c);
+  unsigned int* last_use = cache_last_use(c);
+  const unsigned int now = hd->clock + 1u;
+  int n = 0;
+  unsigned long long hits = 0, misses = 0;
+  for (int k = 0; k < K; ++k) {  // uniform over the warp
+    int e = __shfl_sync(0xffffffffu, mine, k);
+    if (e < 0 || e >= c.E) {
+      if (lane == 0) atomicExch(err, 7);  // kDevBadIndex
+      e = 0;
+    }
+    int s = __ldcg(slot_of + e);
+    if (s < 0) {
+      unsigned long long best = ~0ull;
+      for (int q = lane; q < c.C; q += 32) {
+        const unsigned int t = __ldcg(last_use + q);
+        if (t != now) best = min(best, ((unsigned long long)t << 32) | (unsigned int)q);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+      s = (int)(best & 0xffffffffull);  // exists: at most K - 1 < C slots carry `now` so far
+      if (lane == 0) {
+        const int old = expert_of[s];
+        if (old >= 0) slot_of[old] = -1;
+        expert_of[s] = e;
+        slot_of[e] = s;
+        cache_copy_expert(c)[n] = e;
+        cache_copy_slot(c)[n] = s;
+      }
+      ++n;
+      ++misses;
+    } else {
+      ++hits;
+    }
+    if (lane == 0) {
+      last_use[s] = now;
+      if (slot_out) slot_out[k] = s;
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    hd->clock = now;
+    hd->n_copy = n;
+    hd->hits += hits;
+    hd->misses += misses;
+    hd->bytes += misses * (unsigned long long)c.rec;
+  }
+}
+
 // Router GEMV: logits[t][0..E) = Wr x_t (+ bias), logits[t][E] = wsg . x_t; one grid row per token.
 struct RouterParams {
   const float* h;             // [T][H] input (normalised in-kernel when norm != 0)
@@ -35,6 +127,8 @@ struct RouterParams {
   unsigned int* clear;        // or NULL: nclear counters that CTA 0 zeroes once the predecessor is
   int nclear;                 // complete (the gate/up kernel's group counters, so that a call never
                               // depends on the previous one having finished cleanly)
+  CacheParams cache;           // cache.state != NULL: the selecting CTA also runs the expert-cache
+                              // lookup of the selected experts (slots to cache_slot_out(cache))
   int* err;
 };
 
@@ -286,44 +380,13 @@ bool encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* di
 
 bool gdn_shape_supported(int dk);
 
-// Expert cache (k_cache.cu): host-resident records, HBM slots, tables in `state`.
-constexpr int kCacheMaxK = 32;
-struct CacheHeader {          // first 64 bytes of the state
-  unsigned int clock;         // lookups so far (a slot's last use is the lookup that used it)
-  int err;                    // kDevBadIndex after an index outside the bank (fetch entry point)
-  int n_copy;                 // records the current lookup copies
-  int pad0;
-  unsigned long long hits, misses, bytes;
-  unsigned long long pad1[3];
-};
-struct CacheParams {
-  const uint8_t* host;        // E records at host_stride (pinned host memory, mapped)
-  long long host_stride;
-  uint8_t* slots;             // C records at slot_stride (device)
-  long long slot_stride;
-  long long rec;              // bytes per copied record (multiple of 16)
-  int E, C;
-  uint8_t* state;             // header, copy list [2][kCacheMaxK], slots of the last lookup [kCacheMaxK],
-                              // slot_of [E], expert_of [C], last_use [C]
-};
-__host__ __device__ inline size_t cache_up16(size_t v) { return (v + 15) / 16 * 16; }
-__host__ __device__ inline int* cache_copy_expert(const CacheParams& c) {
-  return reinterpret_cast<int*>(c.state + sizeof(CacheHeader));
-}
-__host__ __device__ inline int* cache_copy_slot(const CacheParams& c) { return cache_copy_expert(c) + kCacheMaxK; }
-__host__ __device__ inline int* cache_slot_out(const CacheParams& c) { return cache_copy_slot(c) + kCacheMaxK; }
-__host__ __device__ inline int* cache_slot_of(const CacheParams& c) { return cache_slot_out(c) + kCacheMaxK; }
-__host__ __device__ inline int* cache_expert_of(const CacheParams& c) {
-  return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(cache_slot_of(c)) + cache_up16((size_t)c.E * 4));
-}
-__host__ __device__ inline unsigned int* cache_last_use(const CacheParams& c) {
-  return reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(cache_expert_of(c)) + cache_up16((size_t)c.C * 4));
-}
 size_t cache_state_bytes(int E, int C);
 cudaError_t launch_cache_reset(const CacheParams& c, cudaStream_t s);
 // One lookup: the plan kernel (tables, copy list, slot_out [K]) then the copy kernel.
 cudaError_t launch_cache_lookup(const CacheParams& c, const int32_t* idx, int K, int32_t* slot_out, int* err, bool pdl,
                                 cudaStream_t s);
+// The copy kernel alone (after a lookup made elsewhere, e.g. by the router's selecting CTA).
+cudaError_t launch_cache_copy(const CacheParams& c, bool pdl, cudaStream_t s);
 cudaError_t launch_gdn_step(const GdnParams& p, bool pdl, cudaStream_t s);
 bool pdl_enabled();
 cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsigned long long limit_ns, int* err,

@@ -4,10 +4,11 @@
 // (jeongsk), key technique 1: only the K selected experts of a layer are read from the
 // slow store, after routing.  Here the store is pinned host memory read by the GPU over
 // the host link, and the cache is managed on the GPU:
-//   cache_plan_kernel  (one warp) marks the selected experts used, picks a victim slot for
-//                      each missing one (least recently used among slots this lookup has
-//                      not used; empty slots first), updates the tables and writes the
-//                      copy list and the slot of every selected expert;
+//   cache_plan_kernel  (one warp; cache_lookup_warp) marks the selected experts used, picks
+//                      a victim slot for each missing one (least recently used among slots
+//                      this lookup has not used; empty slots first), updates the tables and
+//                      writes the copy list and the slot of every selected expert (inside a
+//                      layer call the router's selecting warp does this lookup itself);
 //   cache_copy_kernel  (every SM) copies the listed records, host -> slot, with 16-byte
 //                      loads from host memory (four in flight per thread) and stores to HBM.
 // Both run under dependent launch after the router, and the expert kernels after them.
@@ -48,56 +49,8 @@ __global__ void __launch_bounds__(32) cache_plan_kernel(const CacheParams c, con
   pdl_wait();  // the routing is complete
   pdl_trigger();
   const int lane = threadIdx.x;
-  CacheHeader* hd = reinterpret_cast<CacheHeader*>(c.state);
-  int* slot_of = cache_slot_of(c);
-  int* expert_of = cache_expert_of(c);
-  unsigned int* last_use = cache_last_use(c);
-  const unsigned int now = hd->clock + 1u;
-  int n = 0;
-  unsigned long long hits = 0, misses = 0;
-  for (int k = 0; k < K; ++k) {  // uniform over the warp
-    int e = __ldcg(idx + k);
-    if (e < 0 || e >= c.E) {
-      if (lane == 0) atomicExch(err, kDevBadIndex);
-      e = 0;
-    }
-    int s = __ldcg(slot_of + e);
-    if (s < 0) {
-      // victim: the smallest (last use, slot) among slots not used by this lookup
-      unsigned long long best = ~0ull;
-      for (int q = lane; q < c.C; q += 32) {
-        const unsigned int t = __ldcg(last_use + q);
-        if (t != now) best = min(best, ((unsigned long long)t << 32) | (unsigned int)q);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
-      s = (int)(best & 0xffffffffull);  // exists: at most K - 1 < C slots carry `now` so far
-      if (lane == 0) {
-        const int old = expert_of[s];
-        if (old >= 0) slot_of[old] = -1;
-        expert_of[s] = e;
-        slot_of[e] = s;
-        cache_copy_expert(c)[n] = e;
-        cache_copy_slot(c)[n] = s;
-      }
-      ++n;
-      ++misses;
-    } else {
-      ++hits;
-    }
-    if (lane == 0) {
-      last_use[s] = now;
-      if (slot_out) slot_out[k] = s;
-    }
-    __syncwarp();  // lane 0's table writes are seen by every lane in the next lookup
-  }
-  if (lane == 0) {
-    hd->clock = now;
-    hd->n_copy = n;
-    hd->hits += hits;
-    hd->misses += misses;
-    hd->bytes += misses * (unsigned long long)c.rec;
-  }
+  const int mine = lane < K ? __ldcg(idx + lane) : 0;
+  cache_lookup_warp(c, mine, K, slot_out, err);
 }
 
 // Copies the plan's records: CTA b takes the same contiguous share of every record.
@@ -142,6 +95,10 @@ cudaError_t launch_cache_lookup(const CacheParams& c, const int32_t* idx, int K,
                                 cudaStream_t s) {
   cudaError_t e = launch_pdl(cache_plan_kernel, dim3(1), dim3(32), 0, s, pdl, c, idx, K, slot_out, err);
   if (e != cudaSuccess) return e;
+  return launch_cache_copy(c, pdl, s);
+}
+
+cudaError_t launch_cache_copy(const CacheParams& c, bool pdl, cudaStream_t s) {
   return launch_pdl(cache_copy_kernel, dim3(4 * num_sms()), dim3(kCopyThreads), 0, s, pdl, c);
 }
 

@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const RouterPara
     p.route_w[(size_t)t * (K + 1) + K] = sig;
     p.tickets[t] = 0u;
   }
+  if (p.cache.state != nullptr) cache_lookup_warp(p.cache, ik, K, cache_slot_out(p.cache), p.err);
 }
 
 // One warp per token: top-K, renormalised weights and (optionally) full softmax.
