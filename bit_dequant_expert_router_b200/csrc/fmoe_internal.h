@@ -157,6 +157,7 @@ struct ExpertParams {
   int E;
   int fixed_expert;
   int gsh;                    // weight groups of 64 << gsh columns (0: 64, 1: 128); x digits stay per 64
+  int gu_sw;                  // gate/up split: a shared-expert unit weighs gu_sw eighths of a routed one
   int K;                      // routed slots
   int has_shared;             // slot K is the shared expert
   int H, I;

@@ -22,6 +22,7 @@
 // rows; the routed down rows once the routing is published) are issued before
 // griddepcontrol.wait, so they overlap the previous kernel under programmatic
 // dependent launch.
+#include <cstdlib>
 #include <mutex>
 
 #include "fmoe_internal.h"
@@ -56,6 +57,17 @@ struct GuCfg {
   static constexpr int kChunkBytes = (2 * kChunkRows * (kRowBytes + 2 * kScaleBytes) + 127) / 128 * 128;
   static_assert(kRowPairs * kScaleBytes % 16 == 0 && kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
 };
+
+// CTA b's units [u0, u1) under a weighted split of the unit line: a routed unit weighs 8,
+// a shared-expert unit sw (1..8).  The shared expert's rows are requested before the
+// dependency wait, so with sw < 8 its CTAs take more of them and the routed CTAs less.
+// sw = 8 is the even split.  The shared slot's units come last.
+__host__ __device__ inline void gu_range(int b, int G, int K, int ups, int has_shared, int sw, int& u0, int& u1) {
+  const long long R8 = 8LL * K * ups, Wt = R8 + (has_shared ? (long long)ups * sw : 0);
+  const long long w0 = (long long)b * Wt / G, w1 = (long long)(b + 1) * Wt / G;
+  u0 = w0 <= R8 ? (int)(w0 / 8) : K * ups + (int)((w0 - R8) / sw);
+  u1 = w1 <= R8 ? (int)(w1 / 8) : K * ups + (int)((w1 - R8) / sw);
+}
 
 // The four scale arrays of a chunk (gate scales, gate biases, up scales, up biases) as
 // one tensor copy: a map over (row bytes / 8, {scale, bias}, {gate, up}, rows, experts)
@@ -92,8 +104,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int I = p.I, NE = p.K + p.has_shared;
   const int ups = I / RP, U = NE * ups;
-  const int u0 = (int)((long long)blockIdx.x * U / gridDim.x);
-  const int u1 = (int)((long long)(blockIdx.x + 1) * U / gridDim.x);
+  int u0, u1;
+  gu_range(blockIdx.x, gridDim.x, p.K, ups, p.has_shared, p.gu_sw, u0, u1);
   const uint32_t* xs = reinterpret_cast<const uint32_t*>(sm);
   const float2* xcs = reinterpret_cast<const float2*>(sm + NG * kGroupWords * 4);
 
@@ -568,9 +580,14 @@ cudaError_t gateup_dispatch(const ExpertParams& p, bool pdl, cudaStream_t s) {
   const int units = NE * (p.I / C::kRowPairs);
   int grid = num_sms();
   grid = grid > units ? units : grid;
+  int per_cta = 0;  // the largest CTA range of the weighted split
+  for (int b = 0; b < grid; ++b) {
+    int a0, a1;
+    gu_range(b, grid, p.K, p.I / C::kRowPairs, p.has_shared, p.gu_sw, a0, a1);
+    per_cta = a1 - a0 > per_cta ? a1 - a0 : per_cta;
+  }
   // each CTA counts at most one block of threads' worth of activation groups
-  if ((long long)(units + grid - 1) / grid * C::kRowPairs / kGroup + 2 > kGuWarps * 32 - 32) return cudaErrorInvalidValue;
-  const int per_cta = (units + grid - 1) / grid;
+  if ((long long)per_cta * C::kRowPairs / kGroup + 2 > kGuWarps * 32 - 32) return cudaErrorInvalidValue;
   int nbuf = (int)((kGuSmemBudget - C::kHead) / C::kChunkBytes);
   const int need = (per_cta + C::kChunkUnits - 1) / C::kChunkUnits + 1;  // +1: a chunk may stop at a slot boundary
   nbuf = nbuf > need ? need : nbuf;
@@ -780,8 +797,22 @@ cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsig
   return cudaGetLastError();
 }
 
+// Weight of a shared-expert unit in the gate/up split, in eighths of a routed unit
+// (FMOE_GU_SHARED_WEIGHT, 1..8; 8, the even split, unless set).
+static int gu_shared_weight() {
+  static int w = -1;
+  if (w < 0) {
+    const char* v = getenv("FMOE_GU_SHARED_WEIGHT");
+    const int x = v ? atoi(v) : 8;
+    w = x >= 1 && x <= 8 ? x : 8;
+  }
+  return w;
+}
+
 cudaError_t launch_gateup(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {
-  return bits == 8 ? gateup_bits<8>(p, pdl, s) : bits == 4 ? gateup_bits<4>(p, pdl, s) : gateup_bits<2>(p, pdl, s);
+  ExpertParams q = p;
+  q.gu_sw = gu_shared_weight();
+  return bits == 8 ? gateup_bits<8>(q, pdl, s) : bits == 4 ? gateup_bits<4>(q, pdl, s) : gateup_bits<2>(q, pdl, s);
 }
 
 cudaError_t launch_down(const ExpertParams& p, int bits, bool pdl, cudaStream_t s) {
