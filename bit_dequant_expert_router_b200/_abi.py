@@ -15,7 +15,7 @@ SO_PATH = os.path.join(_HERE, "libfmoe.so")
 
 FMOE_OK = 0
 STATUS_NAMES = {0: "FMOE_OK", 1: "FMOE_ERR_INVALID_ARG", 2: "FMOE_ERR_ALIGNMENT", 3: "FMOE_ERR_UNSUPPORTED",
-                4: "FMOE_ERR_WORKSPACE", 5: "FMOE_ERR_CUDA", 6: "FMOE_ERR_DEVICE_TIMEOUT"}
+                4: "FMOE_ERR_WORKSPACE", 5: "FMOE_ERR_CUDA", 6: "FMOE_ERR_DEVICE_TIMEOUT", 7: "FMOE_ERR_DEVICE_BOUNDS"}
 
 
 class FmoeError(RuntimeError):
@@ -73,17 +73,20 @@ SIGNATURES = [
     ("fmoe_last_error", ctypes.c_char_p, []),
     ("fmoe_status_string", ctypes.c_char_p, [_i]),
     ("fmoe_version", _i, []),
+    ("fmoe_debug_bounds", _i, []),
 ]
 
 
 def lib():
-    """Loads libfmoe.so (built in-tree by build.py); raises if it is missing."""
+    """Loads libfmoe.so (built in-tree by build.py; FMOE_SO may name its debug build,
+    libfmoe_debug.so, instead); raises if it is missing."""
     global _lib
     if _lib is None:
-        if not os.path.exists(SO_PATH):
-            raise RuntimeError(f"{SO_PATH} is missing: build it with `python -m bit_dequant_expert_router_b200.build` "
+        so = os.environ.get("FMOE_SO") or SO_PATH
+        if not os.path.exists(so):
+            raise RuntimeError(f"{so} is missing: build it with `python -m bit_dequant_expert_router_b200.build` "
                                "(there is no fallback implementation)")
-        L = ctypes.CDLL(SO_PATH)
+        L = ctypes.CDLL(so)
         for name, res, args in SIGNATURES:
             fn = getattr(L, name)
             fn.restype = res

@@ -6,6 +6,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SO = os.path.join(HERE, "libfmoe.so")
+# the debug build: the same sources with FMOE_DEBUG_BOUNDS (device-side bounds checks)
+DEBUG_SO = os.path.join(HERE, "libfmoe_debug.so")
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
               "-Xptxas", "-warn-spills"]
 
@@ -19,12 +21,15 @@ def _deps():
         glob.glob(os.path.join(ROOT, "include", "*.h"))
 
 
-def build(force=False, verbose=False, extra_flags=()):
-    if not force and os.path.exists(SO):
-        t = os.path.getmtime(SO)
+def build(force=False, verbose=False, extra_flags=(), debug_bounds=False):
+    so = DEBUG_SO if debug_bounds else SO
+    if debug_bounds:
+        extra_flags = (*extra_flags, "-DFMOE_DEBUG_BOUNDS")
+    if not force and os.path.exists(so):
+        t = os.path.getmtime(so)
         if all(os.path.getmtime(d) <= t for d in _deps()):
-            return SO
-    objdir = os.path.join(HERE, "_build")
+            return so
+    objdir = os.path.join(HERE, "_build_debug" if debug_bounds else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in sources():
@@ -35,12 +40,13 @@ def build(force=False, verbose=False, extra_flags=()):
             print(" ".join(cmd))
         subprocess.check_call(cmd)
         objs.append(obj)
-    cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", SO]
+    cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", so]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)
-    return SO
+    return so
 
 
 if __name__ == "__main__":
-    build(force=True, verbose=True)
+    import sys
+    build(force=True, verbose=True, debug_bounds="--debug-bounds" in sys.argv)

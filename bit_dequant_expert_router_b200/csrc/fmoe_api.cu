@@ -201,6 +201,14 @@ extern "C" {
 
 int fmoe_version(void) { return 100; }
 
+int fmoe_debug_bounds(void) {
+#ifdef FMOE_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 const char* fmoe_last_error(void) { return g_msg; }
 
 const char* fmoe_status_string(fmoe_status s) {
@@ -212,6 +220,7 @@ const char* fmoe_status_string(fmoe_status s) {
     case FMOE_ERR_WORKSPACE: return "FMOE_ERR_WORKSPACE";
     case FMOE_ERR_CUDA: return "FMOE_ERR_CUDA";
     case FMOE_ERR_DEVICE_TIMEOUT: return "FMOE_ERR_DEVICE_TIMEOUT";
+    case FMOE_ERR_DEVICE_BOUNDS: return "FMOE_ERR_DEVICE_BOUNDS";
   }
   return "unknown fmoe_status";
 }
@@ -955,6 +964,7 @@ fmoe_status fmoe_expert_cache_stats(const fmoe_expert_cache* cache, int64_t* hit
     if ((e = cudaMemcpy(&reinterpret_cast<CacheHeader*>(cp.state)->err, &zero, sizeof(int), cudaMemcpyHostToDevice)) !=
         cudaSuccess)
       return cuda_fail(e, "cudaMemcpy");
+    if (hd.err == kDevBounds) return fail(FMOE_ERR_DEVICE_BOUNDS, "a device-side bounds check failed");
     return fail(FMOE_ERR_INVALID_ARG, "a lookup met an expert index outside the bank");
   }
   return FMOE_OK;
@@ -1086,6 +1096,7 @@ fmoe_status fmoe_workspace_check(void* ws, fmoe_stream_t stream) {
   if ((e = cudaMemcpy(&ctrl->err, &zero, sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e, "cudaMemcpy");
   if (err == kDevBadIndex) return fail(FMOE_ERR_INVALID_ARG, "a kernel met an expert index outside the bank");
+  if (err == kDevBounds) return fail(FMOE_ERR_DEVICE_BOUNDS, "a device-side bounds check failed");
   return fail(FMOE_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (code %d)", err);
 }
 

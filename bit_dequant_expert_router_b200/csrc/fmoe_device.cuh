@@ -13,6 +13,18 @@ constexpr int kGroup = 64;        // codes per scale/bias group
 constexpr int kChunkBytes = 16;   // one 128-bit load of codes
 constexpr int kDevTimeout = 6;    // workspace error word: a bounded wait gave up (FMOE_ERR_DEVICE_TIMEOUT)
 constexpr int kDevBadIndex = 7;   // workspace error word: an expert index outside the bank
+constexpr int kDevBounds = 8;     // workspace error word: a bounds check of a debug build failed
+
+// Device-side bounds checks of the debug build (compiled with FMOE_DEBUG_BOUNDS): where
+// an index, a row range or a copy would leave its buffer, FMOE_IN_BOUNDS records
+// kDevBounds in the error word and yields false, and the caller skips the access (a
+// skipped copy then also ends its barrier wait by the time limit).  In the normal build
+// it is the constant true and costs nothing.
+#ifdef FMOE_DEBUG_BOUNDS
+#define FMOE_IN_BOUNDS(cond, err) ((cond) ? true : (atomicExch((err), kDevBounds), false))
+#else
+#define FMOE_IN_BOUNDS(cond, err) true
+#endif
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bound on any device-side wait (2 s)
 
 // Control words at the start of every workspace.

@@ -58,12 +58,16 @@ __global__ void __launch_bounds__(kCopyThreads) cache_copy_kernel(const CachePar
   pdl_wait();  // the plan is complete
   pdl_trigger();
   const CacheHeader* hd = reinterpret_cast<const CacheHeader*>(c.state);
-  const int n = hd->n_copy;
+  const int n = min(hd->n_copy, kCacheMaxK);
   const long long r16 = c.rec / 16;
   const long long per = (r16 + gridDim.x - 1) / gridDim.x;
   const long long b0 = (long long)blockIdx.x * per;
   const long long b1 = b0 + per < r16 ? b0 + per : r16;
   for (int j = 0; j < n; ++j) {
+    if (!FMOE_IN_BOUNDS(n <= kCacheMaxK && cache_copy_expert(c)[j] >= 0 && cache_copy_expert(c)[j] < c.E &&
+                            cache_copy_slot(c)[j] >= 0 && cache_copy_slot(c)[j] < c.C,
+                        &reinterpret_cast<CacheHeader*>(c.state)->err))
+      continue;
     const uint4* src = reinterpret_cast<const uint4*>(c.host + (long long)cache_copy_expert(c)[j] * c.host_stride);
     uint4* dst = reinterpret_cast<uint4*>(c.slots + (long long)cache_copy_slot(c)[j] * c.slot_stride);
     for (long long i = b0 + threadIdx.x; i < b1; i += kCopyThreads * kCopyUnroll) {

@@ -128,6 +128,11 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
     const uint32_t dst = smem_addr(buf), bar = smem_addr(&s_bar[c % nbuf]);
     const uint32_t cb = rows * RB, sb = rows * SB;
+    // the rows stay inside the matrix and the chunk buffer; the record inside its bank
+    if (!FMOE_IN_BOUNDS(r0 >= 0 && rows > 0 && rows <= CR && r0 + rows <= p.I && c >= 0 &&
+                            (!routed || (s_idx[sl] >= 0 && s_idx[sl] < p.routed.num_experts)),
+                        p.err))
+      return;
     if (use_maps) {  // the scale box always moves box_rows rows (past the last row: zeros)
       mbar_expect_tx(bar, 2 * cb + 4 * box_rows * SB);
       bulk_g2s(dst, rec + off[0] + (long long)r0 * RB, cb, bar, pol);
@@ -285,7 +290,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
 #pragma unroll
         for (int i = 0; i < PASSES; ++i) {
           const float g = accg[i], uu = accu[i];
-          p.act[(size_t)sl * I + rbase + k * RP + sub + RPP * i] = g / (1.0f + expf(-g)) * uu;
+          const int row = rbase + k * RP + sub + RPP * i;
+          if (FMOE_IN_BOUNDS(row < I && sl < NE, p.err)) p.act[(size_t)sl * I + row] = g / (1.0f + expf(-g)) * uu;
         }
       }
     }
@@ -405,6 +411,8 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
     const uint64_t pol_r = l2_policy_evict_first(), pol_s = l2_policy_evict_last();
     if (expect) mbar_expect_tx(bar, (uint32_t)NE * rows * (RB + 2 * SB));
     for (int s = s0; s < s1; ++s) {
+      // the chunk's rows stay inside the matrix and the slot's part of the buffer
+      if (!FMOE_IN_BOUNDS(j0 + rows <= p.H && rows <= (uint32_t)crows && s < NE, p.err)) continue;
       const uint64_t pol = s < p.K ? pol_r : pol_s;
       const uint32_t d = smem_addr(buf + (size_t)s * slot_bytes);
       bulk_g2s(d, s_src[s][0] + j0 * RB, rows * RB, bar, pol);
@@ -526,7 +534,7 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1) down_kernel(const ExpertPara
       for (int r = 0; r < RD; ++r)
         if (lane == r) {
           const int row = (cu + k) * RD + r;
-          p.out[row] = (p.resid ? p.resid[row] : 0.0f) + acc[r];
+          if (FMOE_IN_BOUNDS(row < p.H, p.err)) p.out[row] = (p.resid ? p.resid[row] : 0.0f) + acc[r];
         }
     }
     __syncthreads();  // every warp is done with this chunk buffer

@@ -57,7 +57,8 @@ typedef enum {
   FMOE_ERR_UNSUPPORTED = 3,   /* a shape or width these kernels do not handle */
   FMOE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the size query returns */
   FMOE_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
-  FMOE_ERR_DEVICE_TIMEOUT = 6 /* a kernel's bounded wait ran out (reported by fmoe_workspace_check) */
+  FMOE_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out (reported by fmoe_workspace_check) */
+  FMOE_ERR_DEVICE_BOUNDS = 7   /* a device-side bounds check failed (debug build only; fmoe_workspace_check) */
 } fmoe_status;
 
 /* A bank of expert records in device memory.
@@ -250,6 +251,11 @@ const char* fmoe_status_string(fmoe_status status);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int fmoe_version(void);
+
+/* 1 if this library is the debug build, whose kernels check their indices, row ranges
+ * and copies against their buffers and report a failure as FMOE_ERR_DEVICE_BOUNDS
+ * (libfmoe_debug.so, built beside libfmoe.so); 0 otherwise. */
+int fmoe_debug_bounds(void);
 
 #ifdef __cplusplus
 }
