@@ -29,7 +29,7 @@ METRIC = "MoE-layer decode tokens/s and effective weight GB/s (fraction of HBM p
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the per-token
 # gate/up kernel, from one ncu capture of the current build per workload; absent where none was taken.
-EXPERT_TRAFFIC = {"qwen397-4bit": 30744192}
+EXPERT_TRAFFIC = {"qwen397-4bit": 23728640}
 # grouped gate/up: DRAM bytes (read + write) per launch of one ncu capture, per active expert
 # (+ the shared expert): 1,051,820,288 B over 207.5 experts
 GROUPED_GATEUP_TRAFFIC_PER_EXPERT = {"qwen397-4bit-batch64": 5069013}

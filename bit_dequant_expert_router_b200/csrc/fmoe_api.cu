@@ -173,14 +173,17 @@ int num_sms() {
   return cache[dev];
 }
 
-// L2 prefetch of the routed experts' down matrices from the gate/up kernel; FMOE_PREFETCH=0 turns it off.
+// L2 prefetch of the routed experts' down matrices from the gate/up kernel: 1 as soon as
+// the routing is known, 2 once a CTA's last chunk of gate/up rows has landed (so that it
+// does not share DRAM with the gate/up stream), 0 not at all (FMOE_PREFETCH; default 0:
+// measured fastest, the down kernel requests its rows itself before its dependency wait).
 int prefetch_down() {
-  static int on = -1;
-  if (on < 0) {
+  static int mode = -1;
+  if (mode < 0) {
     const char* v = getenv("FMOE_PREFETCH");
-    on = (v && v[0] == '0') ? 0 : 1;
+    mode = (v && v[0] == '1') ? 1 : (v && v[0] == '2') ? 2 : 0;
   }
-  return on;
+  return mode;
 }
 
 // Dependent launch between the block's kernels; FMOE_PDL=0 in the environment turns it off.

@@ -169,7 +169,8 @@ struct ExpertParams {
   unsigned int* grp_cnt;      // [K+has_shared][I/64] rows finished per group of 64 (zero between calls)
   const float* resid;         // down: residual [H] or NULL
   float* out;                 // down: [H]
-  int prefetch_down;          // gate/up asks L2 for the routed experts' down matrices
+  int prefetch_down;          // gate/up asks L2 for the routed experts' down matrices: 1 after the
+                              // routing, 2 after the CTA's last chunk has landed, 0 never
   unsigned int* route_ready;  // or NULL.  Gate/up CTA 0 sets it (release) after writing rt_idx / rt_w;
                               // the down kernel, seeing it set (acquire), reads the routing and requests
                               // the routed rows before its dependency wait; the next router clears it

@@ -196,6 +196,21 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
       st_release_gpu(p.route_ready, 1u);
     }
   }
+  // Warm L2 with this CTA's slice of each routed expert's down matrix (lane 0 of the
+  // last warp; CTAs whose range starts in a routed slot).
+  auto prefetch_down_rows = [&]() {
+    if (u0 / ups >= p.K) return;
+    const long long len[3] = {(long long)p.H * (I * BITS / 8), (long long)p.H * (I / (kGroup << GSH)) * 2,
+                              (long long)p.H * (I / (kGroup << GSH)) * 2};
+    for (int k = 0; k < p.K; ++k) {
+      const uint8_t* rec = p.routed.base + (long long)s_idx[k] * p.routed.stride;
+      for (int m = 0; m < 3; ++m) {
+        const long long a0 = (len[m] * blockIdx.x / gridDim.x) & ~15LL;
+        const long long a1 = (len[m] * (blockIdx.x + 1) / gridDim.x) & ~15LL;
+        if (a1 > a0) prefetch_l2(rec + p.routed.off[6 + m] + a0, (uint32_t)(a1 - a0));
+      }
+    }
+  };
   if (lane == 0) {
     // x digits by warp 0; the first routed chunks one per warp (lane 0), so that
     // their copies go out from several warps at once; the L2 warm-up by warp 7
@@ -211,19 +226,7 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
       if (cu / ups < p.K && c % kGuWarps == warp) issue(c, cu, ce);
       cu = ce;
     }
-    if (warp == kGuWarps - 1 && p.prefetch_down && u0 / ups < p.K) {
-      // Warm L2 with this CTA's slice of each routed expert's down matrix.
-      const long long len[3] = {(long long)p.H * (I * BITS / 8), (long long)p.H * (I / kGroup) * 2,
-                                (long long)p.H * (I / kGroup) * 2};
-      for (int k = 0; k < p.K; ++k) {
-        const uint8_t* rec = p.routed.base + (long long)s_idx[k] * p.routed.stride;
-        for (int m = 0; m < 3; ++m) {
-          const long long a0 = (len[m] * blockIdx.x / gridDim.x) & ~15LL;
-          const long long a1 = (len[m] * (blockIdx.x + 1) / gridDim.x) & ~15LL;
-          if (a1 > a0) prefetch_l2(rec + p.routed.off[6 + m] + a0, (uint32_t)(a1 - a0));
-        }
-      }
-    }
+    if (warp == kGuWarps - 1 && p.prefetch_down == 1) prefetch_down_rows();
   }
   __syncwarp();
 
@@ -244,6 +247,9 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
     const int ce = chunk_end(cu);
     const int sl = cu / ups, rbase = (cu % ups) * RP;
     if (!mbar_wait_bounded(smem_addr(&s_bar[c % nbuf]), (uint32_t)((c / nbuf) & 1), p.err)) ok = false;
+    // the late down prefetch: once the CTA's last chunk is in, its DRAM traffic no longer
+    // competes with this CTA's gate/up stream
+    if (ok && ce == u1 && p.prefetch_down == 2 && warp == kGuWarps - 1 && lane == 0) prefetch_down_rows();
     const uint8_t* buf = sm + C::kHead + (size_t)(c % nbuf) * CHB;
     for (int k = warp; ok && k < ce - cu; k += kGuWarps) {
       float accg[PASSES], accu[PASSES];
