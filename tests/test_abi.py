@@ -180,3 +180,20 @@ def test_expert_cache_rejects_bad_arguments_before_any_launch():
     assert L.fmoe_expert_cache_fetch(ctypes.byref(C(**ok)), 0x62000000, 4, None, None) == 1
     assert L.fmoe_moe_layer_cached(None, ctypes.byref(C(**ok)), 0x60000000, 1, 0x60000000, None, None, 0x50000000,
                                    1 << 20, None) == 1
+
+
+def test_debug_build_exports_the_same_entry_points():
+    """libfmoe_debug.so (the bounds-checking build) carries every declared entry point and
+    says it is the debug build; libfmoe.so says it is not."""
+    import os
+    dbg = os.path.join(os.path.dirname(_abi.SO_PATH), "libfmoe_debug.so")
+    if not os.path.exists(dbg):
+        pytest.skip("libfmoe_debug.so not built")
+    L = ctypes.CDLL(dbg)
+    for name in _declared():
+        assert hasattr(L, name), name
+    L.fmoe_debug_bounds.restype = ctypes.c_int
+    assert L.fmoe_debug_bounds() == 1
+    assert fmoe.lib().fmoe_debug_bounds() == 0
+    L.fmoe_status_string.restype = ctypes.c_char_p
+    assert L.fmoe_status_string(7) == b"FMOE_ERR_DEVICE_BOUNDS"
