@@ -25,12 +25,17 @@
  *     the last non-OK status of the calling host thread.
  *   - Layouts are row-major.  bf16 values are passed as uint16_t bit patterns.
  *
- * Packed matrix [out][in] with b-bit codes (b = 2 or 4) and group size 64:
+ * Packed matrix [out][in] with b-bit codes (b = 2 or 4; 8 as a further format) and
+ * group size G (64; 128 as a further format, for hidden and inter >= 1024), after
+ * "Running MoE models on Apple Silicon with flash-moe" (gillilab), which lists INT2/3/4/8
+ * and groups of 64 or 128:
  *   qw    uint32[out][in*b/32]  code of column c at word c/(32/b), bits
  *                               [b*(c%(32/b)), +b) counted from the LSB;
- *   scale bf16[out][in/64], bias bf16[out][in/64]: group g of row r covers
- *                               columns [64g, 64g+63];
- *   weight (r, c) = code(r, c) * scale[r][c/64] + bias[r][c/64].
+ *   scale bf16[out][in/G], bias bf16[out][in/G]: group g of row r covers
+ *                               columns [G*g, G*g + G-1];
+ *   weight (r, c) = code(r, c) * scale[r][c/G] + bias[r][c/G].
+ * Only the per-token kernels take 8-bit codes and groups of 128; the grouped, fused and
+ * two-kernel paths run 2/4-bit codes in groups of 64 and leave other formats to them.
  * Expert record: gate [I][H] | up [I][H] | down [H][I], each {qw, scale, bias},
  * every sub-array 16-byte aligned; at I = 1024, H = 4096 a record is
  * 7,077,888 bytes at 4-bit (the pages' "6.75 MB per expert") and 3,932,160
@@ -62,7 +67,7 @@ typedef enum {
 } fmoe_status;
 
 /* A bank of expert records in device memory.
- * bits: 2 or 4.  group_size: 64 (the only supported value).
+ * bits: 2, 4 or 8.  group_size: 64 or 128 (128 needs hidden and inter >= 1024).
  * hidden (H), inter (I): model width and expert intermediate width.
  * reserved: set to 0 (it spells out the padding before `base`, so that the layout is
  * the same under every compiler).
