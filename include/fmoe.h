@@ -135,7 +135,7 @@ size_t fmoe_router_topk_workspace_size(int T, int E);
  * bank: the expert bank; expert: record index in [0, num_experts).
  * x: fp32 [H]; y: fp32 [H].  ws: fmoe_expert_ffn_workspace_size(bank) bytes,
  * 256-byte aligned, zeroed once (fmoe_workspace_init).
- * Requirements: bits 2 or 4, group 64, H and I each 64 times a power of two,
+ * Requirements: bits 2, 4 or 8, group 64 or 128 (see fmoe_bank), H and I each 64 times a power of two,
  * 128 <= H, I <= 8192. */
 fmoe_status fmoe_expert_ffn(const fmoe_bank* bank, int expert, const float* x, float* y, void* ws, size_t ws_bytes,
                             fmoe_stream_t stream);
