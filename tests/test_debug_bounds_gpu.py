@@ -57,9 +57,8 @@ def test_debug_build_reports_no_failed_check_and_matches_the_normal_build(tmp_pa
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import numpy as np
-    dbg = os.path.join(ROOT, "bit_dequant_expert_router_b200", "libfmoe_debug.so")
-    if not os.path.exists(dbg):
-        pytest.fail("libfmoe_debug.so is missing: build it with __graft_entry__.build()")
+    import bit_dequant_expert_router_b200.build as pkg_build
+    dbg = pkg_build.build(debug_bounds=True)  # in-tree; rebuilt only if missing or stale
     (tmp_path / "d").mkdir()
     (tmp_path / "n").mkdir()
     _run(tmp_path / "d", dbg)
