@@ -197,3 +197,15 @@ def test_debug_build_exports_the_same_entry_points():
     assert fmoe.lib().fmoe_debug_bounds() == 0
     L.fmoe_status_string.restype = ctypes.c_char_p
     assert L.fmoe_status_string(7) == b"FMOE_ERR_DEVICE_BOUNDS"
+
+
+def test_binding_refuses_host_tensors_for_the_new_entry_points():
+    """The binding only marshals device tensors: host tensors are refused before the library
+    is called (no CPU fallback)."""
+    t = __import__("torch")
+    S = t.zeros((2, 4, 128))
+    q = t.zeros((2, 128))
+    with pytest.raises(ValueError):
+        fmoe.gdn_step(S, q, q, t.zeros((2, 4)), t.zeros(2), t.zeros(2), o=t.zeros((2, 4)))
+    with pytest.raises(ValueError):
+        fmoe.ExpertCache(t.zeros(1024, dtype=t.uint8), 4, 256, 256, 2)   # not pinned

@@ -69,3 +69,21 @@ def test_record_layout_offsets_are_aligned_and_ordered():
     assert gen.algorithmic_bytes_per_token(gen.qwen397_layer(4)) == 39583744
     assert gen.algorithmic_bytes_per_token(gen.qwen397_layer(2)) == 23855104
     assert gen.algorithmic_bytes_per_token(gen.tiny_layer()) == 169984
+
+
+def test_gdn_inputs_follow_the_recipe():
+    """Gated DeltaNet inputs: unit keys, queries of norm dk^-1/2, gates in their ranges on a
+    2^-24 grid, a seeded state with the stated spread; fresh draws per token and layer."""
+    spec = gen.GdnSpec(heads=16, dk=128, dv=64)
+    t0 = gen.host_gdn_token(spec, 2, 0)
+    assert np.allclose(np.linalg.norm(t0["k"].astype(np.float64), axis=1), 1.0, atol=1e-6)
+    assert np.allclose(np.linalg.norm(t0["q"].astype(np.float64), axis=1), 128 ** -0.5, atol=1e-6)
+    assert np.all((t0["alpha"] >= 0.8) & (t0["alpha"] < 1.0)) and np.all((t0["beta"] >= 0) & (t0["beta"] < 1))
+    assert np.all(t0["beta"] * 2.0 ** 24 == np.round(t0["beta"] * 2.0 ** 24))
+    assert t0["v"].shape == (16, 64) and t0["q"].shape == (16, 128)
+    t1 = gen.host_gdn_token(spec, 2, 1)
+    u = gen.host_gdn_token(spec, 3, 0)
+    assert not np.array_equal(t0["k"], t1["k"]) and not np.array_equal(t0["k"], u["k"])
+    assert np.array_equal(t0["k"], gen.host_gdn_token(spec, 2, 0)["k"])
+    S = gen.host_gdn_state(spec, layer=2)
+    assert S.shape == (16, 64, 128) and abs(float(S.std()) - 0.1) < 0.005
