@@ -1,7 +1,7 @@
 """The oracle's pins catch plausible mistakes (no GPU needed).
 
 Each case plants one slip in a copy of the oracle's C source: a wrong code
-order, a dropped or mis-signed term, a wrong group index, a transposed operand,
+order, an 8-bit code read as signed, a group size fixed at 64, a dropped or mis-signed term, a wrong group index, a transposed operand,
 a missing normalisation, a reversed tie-break, swapped SwiGLU operands, a
 missing residual or shared term; in the Gated DeltaNet step a skipped decay, a
 recall from the undecayed state, a wrong delta sign or a missing delta term, a
@@ -34,6 +34,9 @@ MUTATIONS = [
     ("group index of the first group only",
      "const int g = c / m->group;",
      "const int g = 0 * (c / m->group);"),
+    ("group size fixed at 64",
+     "const int g = c / m->group;",
+     "const int g = c / 64;"),
     ("group index by column modulo",
      "const int g = c / m->group;",
      "const int g = c % gpr;"),
@@ -96,6 +99,9 @@ MUTATIONS = [
     ("shared expert dropped",
      "for (int i = 0; i < H; ++i) ot[i] += sigma * y[i];",
      "for (int i = 0; i < H; ++i) ot[i] += 0.0 * sigma * y[i];"),
+    ("8-bit code read as signed",
+     "return (w >> (bits * (c % per_word))) & ((1u << bits) - 1u);",
+     "return bits == 8 ? (unsigned)(int)(signed char)((w >> (bits * (c % per_word))) & 0xFFu) : (w >> (bits * (c % per_word))) & ((1u << bits) - 1u);"),
     ("gdn decay skipped",
      "for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= a;",
      "for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= 1.0;"),
