@@ -1,14 +1,15 @@
 """The oracle's pins catch plausible mistakes (no GPU needed).
 
 Each case plants one slip in a copy of the oracle's C source: a wrong code
-order, an 8-bit code read as signed, a group size fixed at 64, a dropped or mis-signed term, a wrong group index, a transposed operand,
-a missing normalisation, a reversed tie-break, swapped SwiGLU operands, a
-missing residual or shared term; in the Gated DeltaNet step a skipped decay, a
-recall from the undecayed state, a wrong delta sign or a missing delta term, a
-dropped write strength, a transposed rank-1 update, a read-out with the wrong
-vector.  The copy is compiled with the oracle's own flags into a temporary directory, the pin suite (test_oracle_pins.py) runs
-against it in a child process, and at least one pin must fail.  The real
-oracle is never touched.
+order, an 8-bit code read as signed, a group size fixed at 64, a dropped or
+mis-signed term, a wrong group index, a transposed operand, a missing
+normalisation, a reversed tie-break, swapped SwiGLU operands, a missing residual
+or shared term; in the Gated DeltaNet step a skipped decay, a recall from the
+undecayed state, a wrong delta sign or a missing delta term, a dropped write
+strength, a transposed rank-1 update, a read-out with the wrong vector.  The copy
+is compiled with the oracle's own flags into a temporary directory, the pin suite
+(test_oracle_pins.py) runs against it in a child process, and at least one pin
+must fail.  The real oracle is never touched.
 """
 import os
 import subprocess
