@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int I = p.I, NE = p.K + p.has_shared;
-  const int ups = I / RP, U = NE * ups;
+  const int ups = I / RP;
   int u0, u1;
   gu_range(blockIdx.x, gridDim.x, p.K, ups, p.has_shared, p.gu_sw, u0, u1);
   const uint32_t* xs = reinterpret_cast<const uint32_t*>(sm);
