@@ -1,12 +1,15 @@
 """The oracle's pins catch plausible mistakes (no GPU needed).
 
 Each case plants one slip in a copy of the oracle's C source: a wrong code
-order, an 8-bit code read as signed, a group size fixed at 64, a dropped or
-mis-signed term, a wrong group index, a transposed operand, a missing
-normalisation, a reversed tie-break, swapped SwiGLU operands, a missing residual
-or shared term; in the Gated DeltaNet step a skipped decay, a recall from the
-undecayed state, a wrong delta sign or a missing delta term, a dropped write
-strength, a transposed rank-1 update, a read-out with the wrong vector.  The copy
+order, mask or codes-per-word count, an 8-bit code read as signed, a group size
+fixed at 64, a dropped or mis-signed term, a wrong group or row index of a scale
+or bias, a transposed operand or router, a missing normalisation or a mean over
+H - 1, a reversed tie-break, swapped SwiGLU operands or a sigmoid in place of
+SiLU, renormalisation over the wrong probabilities, a missing residual or shared
+term; in the Gated DeltaNet step a skipped decay or one applied after the
+update, a recall from the undecayed state, a wrong delta sign or a missing delta
+term, a dropped or misplaced write strength, a transposed rank-1 update, a
+read-out with the wrong vector or before the update.  The copy
 is compiled with the oracle's own flags into a temporary directory, the pin suite
 (test_oracle_pins.py) runs against it in a child process, and at least one pin
 must fail.  The real oracle is never touched.
@@ -100,6 +103,30 @@ MUTATIONS = [
     ("shared expert dropped",
      "for (int i = 0; i < H; ++i) ot[i] += sigma * y[i];",
      "for (int i = 0; i < H; ++i) ot[i] += 0.0 * sigma * y[i];"),
+    ("rmsnorm mean over H - 1",
+     "const double denom = sqrt(ss / (double)H + eps);",
+     "const double denom = sqrt(ss / (double)(H - 1) + eps);"),
+    ("scale of the next row",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]) + or_bf16(m->bias[(int64_t)r * gpr + g]);",
+     "return (double)q * or_bf16(m->scale[(int64_t)((r + 1) % m->rows) * gpr + g]) + or_bf16(m->bias[(int64_t)r * gpr + g]);"),
+    ("bias of the next group",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]) + or_bf16(m->bias[(int64_t)r * gpr + g]);",
+     "return (double)q * or_bf16(m->scale[(int64_t)r * gpr + g]) + or_bf16(m->bias[(int64_t)r * gpr + (g + 1) % gpr]);"),
+    ("code mask fixed at four bits",
+     "return (w >> (bits * (c % per_word))) & ((1u << bits) - 1u);",
+     "return (w >> (bits * (c % per_word))) & 0xFu;"),
+    ("codes per word fixed at eight",
+     "const int per_word = 32 / bits;",
+     "const int per_word = 8 + 0 * bits;"),
+    ("router transposed",
+     "for (int i = 0; i < H; ++i) acc += or_bf16(wr[(int64_t)e * H + i]) * x[i];",
+     "for (int i = 0; i < H; ++i) acc += or_bf16(wr[((int64_t)i * E + e) % ((int64_t)E * H)]) * x[i];"),
+    ("sigmoid in place of silu",
+     "g[r] = g[r] / (1.0 + exp(-g[r])) * u[r];",
+     "g[r] = 1.0 / (1.0 + exp(-g[r])) * u[r];"),
+    ("renormalised over the first K probabilities",
+     "for (int k = 0; k < K; ++k) psum += p[idx[k]];",
+     "for (int k = 0; k < K; ++k) psum += p[k];"),
     ("8-bit code read as signed",
      "return (w >> (bits * (c % per_word))) & ((1u << bits) - 1u);",
      "return bits == 8 ? (unsigned)(int)(signed char)((w >> (bits * (c % per_word))) & 0xFFu) : (w >> (bits * (c % per_word))) & ((1u << bits) - 1u);"),
@@ -121,6 +148,15 @@ MUTATIONS = [
     ("gdn outer product transposed",
      "Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];",
      "Sh[(int64_t)i * dk + j] += b * (vh[j % dv] - u[j % dv]) * kh[i % dk];"),
+    ("gdn write strength on the value only",
+     "Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];",
+     "Sh[(int64_t)i * dk + j] += (b * vh[i] - u[i]) * kh[j];"),
+    ("gdn read-out before the rank-1 update",
+     "    for (int i = 0; i < dv; ++i)\n      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];\n    for (int i = 0; i < dv; ++i) {\n      double acc = 0.0;\n      for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * qh[j];\n      o[(int64_t)h * dv + i] = acc;\n    }\n",
+     "    for (int i = 0; i < dv; ++i) {\n      double acc = 0.0;\n      for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * qh[j];\n      o[(int64_t)h * dv + i] = acc;\n    }\n    for (int i = 0; i < dv; ++i)\n      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];\n"),
+    ("gdn decay after the rank-1 update",
+     "    for (int i = 0; i < dv; ++i)\n      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= a;\n    for (int i = 0; i < dv; ++i) {\n      double acc = 0.0;\n      for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * kh[j];\n      u[i] = acc;\n    }\n    for (int i = 0; i < dv; ++i)\n      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];\n",
+     "    for (int i = 0; i < dv; ++i) {\n      double acc = 0.0;\n      for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * kh[j];\n      u[i] = acc;\n    }\n    for (int i = 0; i < dv; ++i)\n      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] += b * (vh[i] - u[i]) * kh[j];\n    for (int i = 0; i < dv; ++i)\n      for (int j = 0; j < dk; ++j) Sh[(int64_t)i * dk + j] *= a;\n"),
     ("gdn read-out with the key",
      "for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * qh[j];",
      "for (int j = 0; j < dk; ++j) acc += Sh[(int64_t)i * dk + j] * kh[j];"),
