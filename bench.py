@@ -221,15 +221,16 @@ def dist_setup(args):
     return world, rank, local
 
 
-def cpu_oracle_rate(spec, budget_s, t0=1_000_000):
-    """Times the CPU oracle (all host cores) on a bounded sample of the workload: tokens/s.
+def cpu_oracle_rate(spec, budget_s, t0=1_000_000, threads=None):
+    """Times the CPU oracle (all host cores, or `threads` of them) on a bounded sample of
+    the workload: tokens/s.
 
     Drawing the inputs (router, shared expert, the experts a token selects) is
     not timed; the oracle's whole forward pass (norm, router, softmax, top-K,
     K+1 expert FFNs, combine) is."""
     import gen
     import oracle
-    cores = len(os.sched_getaffinity(0))
+    cores = threads or len(os.sched_getaffinity(0))
     oracle.set_threads(cores)
     base = gen.host_layer(spec, 0, 0, experts=[])
     nbytes, off = gen.record_layout(spec.bits, spec.hidden, spec.inter, spec.group)
@@ -252,6 +253,13 @@ def cpu_oracle_rate(spec, budget_s, t0=1_000_000):
     return n / spent, cores, n, spent
 
 
+def single_thread_sample(rate_fn, *a, budget_s=2.0, unit="tokens/s"):
+    """The same oracle on one host thread, a short sample of its own (about `budget_s`
+    seconds): the per-core rate beside the all-core one."""
+    rate, _, n, spent = rate_fn(*a, budget_s, threads=1)
+    return {"value": rate, "unit": unit, "cores": 1, "sample": f"{n} steps ({spent:.1f} s of oracle time)"}
+
+
 def run_reference(args, spec, desc, world, rank):
     if rank != 0:
         return
@@ -262,7 +270,8 @@ def run_reference(args, spec, desc, world, rank):
             "config": {"workload": desc},
             "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{n} tokens of the workload ({spent:.1f} s of oracle time; the requested "
-                                       f"{args.steps} steps would not fit a few minutes)"},
+                                       f"{args.steps} steps would not fit a few minutes)",
+                             "single_thread": single_thread_sample(cpu_oracle_rate, spec)},
             "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -274,12 +283,12 @@ def gdn_bytes_per_step(spec):
     return 4 * (2 * n * dv * dk + n * (2 * dk + dv + 2) + n * dv)
 
 
-def cpu_oracle_gdn_rate(spec, layers, budget_s):
-    """Times the CPU oracle's gated-delta-rule step (all host cores) on a bounded sample of
-    layer-steps; drawing the inputs is not timed."""
+def cpu_oracle_gdn_rate(spec, layers, budget_s, threads=None):
+    """Times the CPU oracle's gated-delta-rule step (all host cores, or `threads` of them) on
+    a bounded sample of layer-steps; drawing the inputs is not timed."""
     import gen
     import oracle
-    cores = len(os.sched_getaffinity(0))
+    cores = threads or len(os.sched_getaffinity(0))
     oracle.set_threads(cores)
     states = {}
     n, spent = 0, 0.0
@@ -309,7 +318,9 @@ def run_gdn(args, world, rank, local):
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": desc},
                 "cpu_baseline": {"value": rate, "unit": "layer-steps/s", "cores": cores, "kind": "oracle",
-                                 "sample": f"{n} layer-steps ({spent:.1f} s of oracle time)"},
+                                 "sample": f"{n} layer-steps ({spent:.1f} s of oracle time)",
+                                 "single_thread": single_thread_sample(cpu_oracle_gdn_rate, spec, nlayers,
+                                                                       unit="layer-steps/s")},
                 "e2e": {"value": rate, "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -441,7 +452,8 @@ def run_gdn(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, n, spent = cpu_oracle_gdn_rate(spec, nlayers, args.cpu_seconds)
         cpu = {"value": rate, "unit": "layer-steps/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} layer-steps of this workload ({spent:.1f} s of oracle time)"}
+               "sample": f"{n} layer-steps of this workload ({spent:.1f} s of oracle time)",
+               "single_thread": single_thread_sample(cpu_oracle_gdn_rate, spec, nlayers, unit="layer-steps/s")}
     if rank == 0:
         line = {
             "metric": GDN_METRIC, "value": value, "unit": "layer-steps/s", "n_gpus": world, "steps": steps,
@@ -621,7 +633,8 @@ def run_cached(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, n, spent = cpu_oracle_rate(spec, args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} tokens of this workload, layer copy 0 ({spent:.1f} s of oracle time)"}
+               "sample": f"{n} tokens of this workload, layer copy 0 ({spent:.1f} s of oracle time)",
+               "single_thread": single_thread_sample(cpu_oracle_rate, spec)}
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
@@ -841,7 +854,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, n, spent = cpu_oracle_rate(spec, args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} tokens of this workload, layer copy 0 ({spent:.1f} s of oracle time)"}
+               "sample": f"{n} tokens of this workload, layer copy 0 ({spent:.1f} s of oracle time)",
+               "single_thread": single_thread_sample(cpu_oracle_rate, spec)}
 
     if rank == 0:
         line = {

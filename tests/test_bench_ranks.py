@@ -84,6 +84,8 @@ def test_reference_arm_prints_the_contract_line(workload):
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    one = line["cpu_baseline"]["single_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == line["unit"]
 
 
 def test_reference_arm_prints_only_on_rank_zero():
