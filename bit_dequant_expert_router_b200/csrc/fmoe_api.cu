@@ -441,10 +441,16 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T) {
   if (!layer) return 0;
   const int H = layer->routed.hidden, E = layer->routed.num_experts, K = layer->top_k, I = layer->routed.inter;
   size_t need = layout(H, E, K, I, 1).total;
-  if (T >= kGroupedMinT && K >= 1 && E >= 1 && H > 0 && I > 0) {
-    const size_t g = glayout(H, E, K, I, T).total;
-    need = g > need ? g : need;
-  }
+  // The grouped layout is not monotone in T (the router's split of H shrinks as token
+  // tiles are added), so take its largest size over every batch of at most T tokens:
+  // a workspace sized for T then takes the grouped path for any smaller batch too.
+  // Once the split is down to 1 it stays there, and the size only grows with t.
+  if (K >= 1 && E >= 1 && H > 0 && I > 0)
+    for (int t = kGroupedMinT; t <= T; ++t) {
+      const size_t g = glayout(H, E, K, I, t).total;
+      need = g > need ? g : need;
+      if (t < T && grouped_router_split(H, E, t) == 1) t = T - 1;
+    }
   return need;
 }
 

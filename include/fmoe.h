@@ -150,9 +150,11 @@ size_t fmoe_expert_ffn_workspace_size(const fmoe_bank* bank);
  * topk_idx (int32 [T][K]) and topk_w (fp32 [T][K]) receive the routing, or NULL.
  * ws: fmoe_moe_layer_workspace_size(layer, T) bytes, 256-byte aligned, zeroed
  * once before first use (fmoe_workspace_init); calls on one workspace must be
- * ordered on one stream.  T >= 8 tokens run expert-grouped (each active
- * expert's rows read once for its token group) when the workspace holds the
- * T-token size, hidden and inter are >= 512 and FMOE_GROUPED is not "0";
+ * ordered on one stream.  The size for T serves every call of at most T tokens.
+ * T >= 8 tokens run expert-grouped (each active expert's rows read once for
+ * its token group) when the workspace holds the grouped layout of T tokens
+ * (one of fmoe_moe_layer_workspace_size(layer, T') bytes, T' >= T, does),
+ * hidden and inter are >= 512 and FMOE_GROUPED is not "0";
  * otherwise token by token, for which the T = 1 size suffices (a smaller
  * workspace gives FMOE_ERR_WORKSPACE).  Requirements: those of fmoe_expert_ffn for both
  * banks (same bits, hidden, inter), 1 <= K <= min(E, 32), E <= 4096,
@@ -192,8 +194,8 @@ size_t fmoe_moe_layer_workspace_size(const fmoe_layer* layer, int T);
  * on the same device whose kernels may overlap (different streams without an
  * ordering between them, or different host threads) race on it and give wrong
  * results.  Order all calls on a device on one stream.
- * A layer whose scratch (fmoe_moe_layer_workspace_size(layer, T)) exceeds
- * FMOE_STATIC_SCRATCH_BYTES is rejected with FMOE_ERR_WORKSPACE before
+ * A layer whose per-token scratch (fmoe_moe_layer_workspace_size(layer, 1))
+ * exceeds FMOE_STATIC_SCRATCH_BYTES is rejected with FMOE_ERR_WORKSPACE before
  * anything is enqueued.  Every shape the other requirements admit needs at
  * most 435,968 bytes (the Qwen3.5-397B-A17B layer 214,016), so today that
  * check only guards against shapes later versions may admit. */

@@ -105,6 +105,29 @@ def test_workspace_size_query_is_positive_and_monotone():
     assert L.fmoe_router_topk_workspace_size(64, 512) > L.fmoe_router_topk_workspace_size(1, 512)
 
 
+def test_workspace_sizes_at_the_qwen_shapes():
+    """The per-token workspace covers every T below the grouped threshold (8 tokens); from
+    there the grouped layout is added.  The figures are the ones the design notes state.
+    The query never shrinks as T grows, although the grouped layout alone does (its router
+    split shrinks once a batch needs a second tile of 64 tokens): a workspace sized for T
+    holds the grouped layout of every smaller batch."""
+    L = fmoe.lib()
+    for kw in ({}, {"bits": 2}, {"H": 1024, "I": 512, "E": 8}, {"E": 64, "top_k": 8}):
+        lay = _fake_layer(**kw)
+        size = lambda T: L.fmoe_moe_layer_workspace_size(ctypes.byref(lay), T)
+        sizes = [size(T) for T in range(1, 600)]
+        assert all(b >= a for a, b in zip(sizes, sizes[1:])), kw
+    lay = _fake_layer()
+    size = lambda T: L.fmoe_moe_layer_workspace_size(ctypes.byref(lay), T)
+    assert [size(T) for T in (1, 2, 7)] == [214016] * 3
+    assert size(8) == 1686272 and size(64) == 11982848
+    assert size(65) == size(64)          # the T = 65 layout alone needs 11,101,440 bytes
+    assert size(1 << 20) > size(600)     # large T: no stall in the query, the size keeps growing
+    # FMOE_STATIC_SCRATCH_BYTES holds the per-token layout but not the grouped one at these
+    # shapes, so the static entry point runs batches of 8 or more token by token here
+    assert size(1) <= 524288 < size(8)
+
+
 def test_other_entry_points_validate():
     L = fmoe.lib()
     assert L.fmoe_rmsnorm(0x1000, None, 1e-6, 0, 4096, 0x1000, None) == 0
