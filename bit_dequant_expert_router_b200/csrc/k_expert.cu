@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1) gateup_kernel(const ExpertPa
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int I = p.I, NE = p.K + p.has_shared;
+  const int I = p.I;
+  [[maybe_unused]] const int NE = p.K + p.has_shared;  // read only by the debug build's bounds checks
   const int ups = I / RP;
   int u0, u1;
   gu_range(blockIdx.x, gridDim.x, p.K, ups, p.has_shared, p.gu_sw, u0, u1);
