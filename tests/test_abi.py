@@ -128,6 +128,37 @@ def test_workspace_sizes_at_the_qwen_shapes():
     assert size(1) <= 524288 < size(8)
 
 
+def test_last_error_is_per_host_thread():
+    """fmoe_last_error reports the last failure of the calling thread: two threads that fail
+    with different messages at the same time each read back their own."""
+    import threading
+    L = fmoe.lib()
+    bad = {"rmsnorm": lambda: L.fmoe_rmsnorm(None, None, 1e-6, 1, 4096, 0x1000, None),
+           "layer": lambda: L.fmoe_moe_layer(None, 0x1000, 1, 0x1000, None, None, 0x1000, 1 << 20, None)}
+    seen = {}
+    for name, call in bad.items():
+        assert call() == 1
+        seen[name] = L.fmoe_last_error()
+    assert seen["rmsnorm"] != seen["layer"]
+    start = threading.Barrier(2)
+    wrong = []
+
+    def worker(name):
+        start.wait()
+        for _ in range(2000):
+            bad[name]()
+            if L.fmoe_last_error() != seen[name]:
+                wrong.append(name)
+                return
+
+    ts = [threading.Thread(target=worker, args=(n,)) for n in bad]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert not wrong
+
+
 def test_other_entry_points_validate():
     L = fmoe.lib()
     assert L.fmoe_rmsnorm(0x1000, None, 1e-6, 0, 4096, 0x1000, None) == 0
