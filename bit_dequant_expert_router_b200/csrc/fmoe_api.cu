@@ -1,6 +1,7 @@
 // fmoe_api.cu -- the C ABI of libfmoe.so: argument validation, workspace
 // layout and kernel dispatch.  Every entry point validates on the host before
 // enqueuing anything and reports through fmoe_status (never aborts).
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -162,15 +163,15 @@ cudaError_t trace_record(cudaEvent_t ev, cudaStream_t s) {
 }  // namespace
 
 int num_sms() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64] = {};  // per device; calls may come from several host threads
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 // L2 prefetch of the routed experts' down matrices from the gate/up kernel: 1 as soon as
@@ -178,22 +179,20 @@ int num_sms() {
 // does not share DRAM with the gate/up stream), 0 not at all (FMOE_PREFETCH; default 0:
 // measured fastest, the down kernel requests its rows itself before its dependency wait).
 int prefetch_down() {
-  static int mode = -1;
-  if (mode < 0) {
+  static const int mode = [] {  // read once (thread-safe static initialisation)
     const char* v = getenv("FMOE_PREFETCH");
-    mode = (v && v[0] == '1') ? 1 : (v && v[0] == '2') ? 2 : 0;
-  }
+    return (v && v[0] == '1') ? 1 : (v && v[0] == '2') ? 2 : 0;
+  }();
   return mode;
 }
 
 // Dependent launch between the block's kernels; FMOE_PDL=0 in the environment turns it off.
 bool pdl_enabled() {
-  static int on = -1;
-  if (on < 0) {
+  static const bool on = [] {
     const char* v = getenv("FMOE_PDL");
-    on = (v && v[0] == '0') ? 0 : 1;
-  }
-  return on == 1;
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 }  // namespace fmoe

@@ -815,12 +815,11 @@ cudaError_t launch_wait_flag(const unsigned int* flag, unsigned int value, unsig
 // Weight of a shared-expert unit in the gate/up split, in eighths of a routed unit
 // (FMOE_GU_SHARED_WEIGHT, 1..8; 8, the even split, unless set).
 static int gu_shared_weight() {
-  static int w = -1;
-  if (w < 0) {
+  static const int w = [] {  // read once (thread-safe static initialisation)
     const char* v = getenv("FMOE_GU_SHARED_WEIGHT");
     const int x = v ? atoi(v) : 8;
-    w = x >= 1 && x <= 8 ? x : 8;
-  }
+    return x >= 1 && x <= 8 ? x : 8;
+  }();
   return w;
 }
 

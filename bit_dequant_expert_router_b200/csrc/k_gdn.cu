@@ -125,11 +125,10 @@ cudaError_t launch_nc(const GdnParams& p, bool pdl, cudaStream_t s) {
 // (2.31 us per 64-head step against 2.60 with two and 4.09 with four): every state row of
 // the step is requested at once, and no warp works through two rows in turn.
 int rows_per_warp() {
-  static int r = -1;
-  if (r < 0) {
+  static const int r = [] {  // read once (thread-safe static initialisation)
     const char* e = getenv("FMOE_GDN_RPW");
-    r = (e && (e[0] == '1' || e[0] == '2' || e[0] == '4')) ? e[0] - '0' : 1;
-  }
+    return (e && (e[0] == '1' || e[0] == '2' || e[0] == '4')) ? e[0] - '0' : 1;
+  }();
   return r;
 }
 
