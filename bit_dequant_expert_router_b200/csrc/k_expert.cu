@@ -710,9 +710,6 @@ cudaError_t down_bits(const ExpertParams& p, bool pdl, cudaStream_t s) {
 
 }  // namespace
 
-// Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
-// again only if a larger size is asked for, so that launches captured into a
-// CUDA graph make no attribute call.
 // Asks for the largest shared-memory carveout for a kernel, once per (kernel, device):
 // kernels that sit on an SM together under dependent launch must run with the same
 // carveout, else the later one waits for the SM to drain before it can start there.
@@ -735,6 +732,9 @@ cudaError_t set_carveout_max(const void* kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
+// again only if a larger size is asked for, so that launches captured into a
+// CUDA graph make no attribute call.
 cudaError_t set_smem(const void* kernel, size_t bytes) {
   struct Entry {
     const void* fn;
