@@ -373,3 +373,23 @@ def test_gdn_heads_are_independent():
     for h in range(3):
         Sh, oh = oracle.gdn_step(S[h:h + 1], q[h:h + 1], k[h:h + 1], v[h:h + 1], alpha[h:h + 1], beta[h:h + 1])
         assert np.array_equal(Sh[0], S2[h]) and np.array_equal(oh[0], o[h])
+
+
+def test_results_do_not_depend_on_the_thread_count():
+    """Threads split only independent output rows and heads, so one thread and many give
+    the same bits (the bench times the oracle on all host cores, the tests on few)."""
+    before = oracle.lib().or_get_threads()
+    try:
+        hl = gen.host_layer(gen.tiny_layer(4), seed=3)
+        L = oracle_layer(hl)
+        h = gen.host_tokens(77, 3, hl.spec.hidden)
+        S, q, k, v, alpha, beta = _gdn_case(9, n=8, dk=16, dv=16)
+        runs = []
+        for n in (1, 4):
+            oracle.set_threads(n)
+            r = L.forward(h)
+            runs.append((r["out"], r["idx"], r["w"], *oracle.gdn_step(S, q, k, v, alpha, beta)))
+        for a, b in zip(*runs):
+            assert np.array_equal(a, b)
+    finally:
+        oracle.set_threads(before)
